@@ -1,0 +1,65 @@
+"""fp64 CPU oracle of the nanochat GPT forward pass + token cross-entropy.
+
+TEST INFRASTRUCTURE ONLY.  This package is the plain, slow, obviously correct
+statement of what the CUDA library computes.  Only the test-suite, the package's
+``smoke()`` check and the CPU-baseline leg of the bench may import it; the
+product path (the CUDA library and its Python binding) never does, and the
+oracle imports nothing from the product path.  It shares no code, table or
+constant generator with the CUDA side; both receive their inputs from the
+separate ``workloads`` module, which holds no arithmetic of the method.
+
+Sources (page title, section):
+
+* "从文本到聊天模型" (onehacker.top) -- §4.1 input/target shift, §5.1 model
+  configuration, §5.2 token embedding, §5.3 pre-norm residual block, §5.4
+  separate Q/K/V projections and their (B,T,H,D) / (B,T,Hkv,D) shapes, §5.5 causal
+  attention, §5.6 RoPE, §5.7 ReLU^2 MLP, §5.8 untied LM head and cross-entropy
+  with ``ignore_index=-1``.
+* "Nanochat与nanoGPT对比：关键升级" (lzwjava.github.io) -- §1 architecture table
+  and its notes: RoPE without learned positions, parameter-free RMSNorm, ReLU^2,
+  split c_q/c_k/c_v/c_proj, GQA, QK-norm applied after RoPE, no biases, untied
+  embedding, no dropout, tanh logit soft-cap at +-15, SSSL sliding window (three
+  quarter-context layers then one full layer, the last layer always full), the
+  final normalisation before the logit projection (Backout note).
+* "约100美元训出对话模型，nanochat源码全链路拆解" (ikfou.com) -- the example
+  config (sequence_len 2048, vocab 32768, SSSL) and fp32 weights cast to bf16 at
+  matmul time; nanochat README mirror (dev.wehub.plus), "精度 / dtype".
+
+Readings where the pages are silent (each is a config field or a single
+function here, and the CUDA library takes the same reading independently):
+
+* RMSNorm eps = 1e-6; QK-norm is per head over the head dimension D.
+* RoPE: theta_i = base^(-2i/D), base 10000, positions 0..T-1 in each row, pairs
+  (u_i, u_{i+D/2}) rotated by +t*theta_i.
+* softmax scale 1/sqrt(D), applied after QK-norm.
+* window predicate: key j is visible from query i iff j <= i and i - j < W
+  (exactly W keys including the query itself).
+* layer l uses pattern[l % len(pattern)], and the last layer is forced full.
+* GQA: query head h reads kv head h // (H / Hkv).
+* no norm after the embedding; one parameter-free RMSNorm before lm_head.
+* soft-cap 15*tanh(z/15) is applied before the loss and the returned logits are
+  the capped ones; loss = mean natural-log NLL over targets != -1 (NaN if none).
+
+Parity pins live in ``tests/test_oracle_pins.py``.  Every function below is
+pinned there by closed forms, invariants, brute force or an independent library
+routine.  The composition of the full forward at random weights is pinned only
+structurally (zero-projection closed form, causality, row independence): no page
+prints logits or losses for any input, so the absolute values of a random-weight
+forward are "parity unpinned" beyond those structural pins.
+"""
+from .model import (  # noqa: F401
+    OracleConfig,
+    derive_config,
+    layer_windows,
+    window_visible,
+    rms_norm,
+    rope_tables,
+    rope,
+    rope_qknorm,
+    attention,
+    relu2_mlp,
+    softcap,
+    cross_entropy,
+    embed,
+    forward,
+)

@@ -1,0 +1,247 @@
+"""fp64 oracle of the nanochat GPT block-stack forward + cross-entropy.
+
+TEST INFRASTRUCTURE ONLY -- see the package docstring for who may import this
+module, the sources and the readings taken where the pages are silent.
+
+Everything is numpy float64.  fp32 inputs (weights) are upcast exactly.  The
+matrix products use numpy's matmul as a library primitive; nothing is blocked,
+fused or reordered beyond the definitions written here.
+"""
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass, field
+
+import numpy as np
+
+F64 = np.float64
+
+
+@dataclass(frozen=True)
+class OracleConfig:
+    n_layer: int
+    d_model: int
+    n_head: int
+    n_kv_head: int
+    head_dim: int
+    seq_len: int
+    vocab: int
+    window_pattern: str = "SSSL"
+    short_window: int = 0  # 0 -> seq_len // 4
+    softcap: float = 15.0
+    norm_eps: float = 1e-6
+    rope_base: float = 10000.0
+
+    @property
+    def short(self) -> int:
+        return self.short_window if self.short_window > 0 else self.seq_len // 4
+
+
+def derive_config(depth: int, aspect_ratio: int = 64, head_dim: int = 128,
+                  n_kv_head: int = 0, seq_len: int = 2048, vocab: int = 32768,
+                  **kw) -> OracleConfig:
+    """Depth-derived sizes.
+
+    "从文本到聊天模型" §5.1: model_dim = depth * aspect_ratio and
+    num_heads = model_dim // head_dim (d24: 1536 wide, 12 heads).
+    n_kv_head = 0 means "as many kv heads as query heads" (plain MHA).
+    """
+    d_model = depth * aspect_ratio
+    n_head = d_model // head_dim
+    return OracleConfig(n_layer=depth, d_model=d_model, n_head=n_head,
+                        n_kv_head=n_kv_head if n_kv_head > 0 else n_head,
+                        head_dim=head_dim, seq_len=seq_len, vocab=vocab, **kw)
+
+
+def layer_windows(cfg: OracleConfig) -> list:
+    """Attention window (number of visible keys) of every layer.
+
+    "Nanochat与nanoGPT对比：关键升级" §1, sliding-window note: in the SSSL
+    pattern three layers use a short window of a quarter of the context and one
+    layer the full context, cycling over the layers; the last layer is always
+    full.  'S' -> short window, 'L' -> seq_len.
+    """
+    pat = cfg.window_pattern
+    out = []
+    for l in range(cfg.n_layer):
+        ch = pat[l % len(pat)]
+        if l == cfg.n_layer - 1:
+            ch = "L"
+        out.append(cfg.seq_len if ch == "L" else cfg.short)
+    return out
+
+
+def window_visible(i: int, j: int, W: int) -> bool:
+    """Key j is visible from query i: causal ("从文本到聊天模型" §5.5) and inside
+    a window of W keys that ends at the query itself."""
+    return j <= i and (i - j) < W
+
+
+def rms_norm(u: np.ndarray, eps: float) -> np.ndarray:
+    """Parameter-free RMSNorm over the last axis ("Nanochat与nanoGPT对比" §1:
+    RMSNorm without learnable parameters): u / sqrt(mean(u^2) + eps)."""
+    u = np.asarray(u, dtype=F64)
+    ms = np.mean(u * u, axis=-1, keepdims=True)
+    return u / np.sqrt(ms + eps)
+
+
+def rope_tables(T: int, D: int, base: float):
+    """cos/sin of t * theta_i, theta_i = base^(-2i/D), shapes [T, D/2] (fp64)."""
+    half = D // 2
+    i = np.arange(half, dtype=F64)
+    theta = base ** (-2.0 * i / D)
+    t = np.arange(T, dtype=F64)
+    ang = t[:, None] * theta[None, :]
+    return np.cos(ang), np.sin(ang)
+
+
+def rope(u: np.ndarray, cos: np.ndarray, sin: np.ndarray, pos0: int = 0) -> np.ndarray:
+    """Rotary position embedding ("从文本到聊天模型" §5.6; "Nanochat与nanoGPT对比"
+    §1: rotation in complex space, no learned position table).
+
+    u: [..., T, heads, D] with the sequence axis third from the end.  Pair
+    (u_i, u_{i+D/2}) at position t is rotated by the angle t * theta_i.
+    """
+    u = np.asarray(u, dtype=F64)
+    T, D = u.shape[-3], u.shape[-1]
+    half = D // 2
+    c = cos[pos0:pos0 + T][:, None, :]  # [T, 1, D/2]
+    s = sin[pos0:pos0 + T][:, None, :]
+    a, b = u[..., :half], u[..., half:]
+    return np.concatenate([a * c - b * s, a * s + b * c], axis=-1)
+
+
+def rope_qknorm(q: np.ndarray, k: np.ndarray, cfg: OracleConfig):
+    """RoPE, then per-head RMSNorm of q and k ("Nanochat与nanoGPT对比" §1: q and
+    k are normalised after RoPE)."""
+    T, D = q.shape[-3], q.shape[-1]
+    cos, sin = rope_tables(T, D, cfg.rope_base)
+    return (rms_norm(rope(q, cos, sin), cfg.norm_eps),
+            rms_norm(rope(k, cos, sin), cfg.norm_eps))
+
+
+def attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, W: int,
+              query_positions=None) -> np.ndarray:
+    """Causal sliding-window attention with GQA.
+
+    q [B,T,H,D], k and v [B,T,Hkv,D] ("从文本到聊天模型" §5.4).  Query head h
+    reads kv head h // (H/Hkv) (several query heads share one kv head).  For query
+    i: s_j = q_i . k_j / sqrt(D) over the visible keys j, o_i = sum_j softmax(s)_j v_j.
+    ``query_positions`` (optional) restricts the output to those rows; the
+    result then has shape [B, len(query_positions), H, D].
+    """
+    q = np.asarray(q, dtype=F64)
+    k = np.asarray(k, dtype=F64)
+    v = np.asarray(v, dtype=F64)
+    B, T, H, D = q.shape
+    Hkv = k.shape[2]
+    assert H % Hkv == 0
+    group = H // Hkv
+    rows = np.arange(T) if query_positions is None else np.asarray(query_positions)
+    out = np.zeros((B, len(rows), H, D), dtype=F64)
+    scale = 1.0 / math.sqrt(D)
+    jj = np.arange(T)
+    for r, i in enumerate(rows):
+        vis = (jj <= i) & ((i - jj) < W)
+        idx = jj[vis]
+        for h in range(H):
+            g = h // group
+            s = (k[:, idx, g, :] @ q[:, i, h, :, None])[..., 0] * scale  # [B, n]
+            s = s - s.max(axis=1, keepdims=True)
+            p = np.exp(s)
+            p = p / p.sum(axis=1, keepdims=True)
+            out[:, r, h, :] = (p[:, None, :] @ v[:, idx, g, :])[:, 0, :]
+    return out
+
+
+def relu2_mlp(a: np.ndarray, w_fc: np.ndarray, w_proj: np.ndarray) -> np.ndarray:
+    """"从文本到聊天模型" §5.7: c_fc (C -> 4C), relu(x)^2, c_proj (4C -> C)."""
+    h = np.asarray(a, dtype=F64) @ np.asarray(w_fc, dtype=F64).T
+    h = np.maximum(h, 0.0) ** 2
+    return h @ np.asarray(w_proj, dtype=F64).T
+
+
+def softcap(z: np.ndarray, cap: float) -> np.ndarray:
+    """"Nanochat与nanoGPT对比" §1: tanh logit soft-cap at +-cap."""
+    return cap * np.tanh(np.asarray(z, dtype=F64) / cap)
+
+
+def cross_entropy(logits: np.ndarray, targets: np.ndarray):
+    """Token-level cross-entropy with ignore_index = -1 ("从文本到聊天模型" §5.8).
+
+    logits [..., V], targets [...] int.  Returns (per-token NLL with 0 at ignored
+    positions, mean NLL over the non-ignored positions; NaN if there are none).
+    """
+    l = np.asarray(logits, dtype=F64)
+    y = np.asarray(targets).astype(np.int64)
+    m = l.max(axis=-1, keepdims=True)
+    lse = (m + np.log(np.exp(l - m).sum(axis=-1, keepdims=True)))[..., 0]
+    valid = y != -1
+    ysafe = np.where(valid, y, 0)
+    picked = np.take_along_axis(l, ysafe[..., None], axis=-1)[..., 0]
+    nll = np.where(valid, lse - picked, 0.0)
+    n = int(valid.sum())
+    loss = float(nll.sum() / n) if n > 0 else float("nan")
+    return nll, loss
+
+
+def embed(wte: np.ndarray, idx: np.ndarray) -> np.ndarray:
+    """"从文本到聊天模型" §5.2: x = wte(idx), (B,T) -> (B,T,C)."""
+    return np.asarray(wte, dtype=F64)[np.asarray(idx)]
+
+
+def _w(a):
+    return np.asarray(a, dtype=F64)
+
+
+def forward(cfg: OracleConfig, weights: dict, idx: np.ndarray, targets=None,
+            want_logits: bool = True):
+    """The whole forward for the rows of ``idx`` ([B, T] int).
+
+    Steps in the order of "从文本到聊天模型" §5 (embedding, blocks of
+    ``x = x + attn(norm(x)); x = x + mlp(norm(x))``, LM head, cross-entropy) with
+    the block internals of "Nanochat与nanoGPT对比" §1 (split c_q/c_k/c_v,
+    RoPE then QK-norm, SSSL windows, GQA, ReLU^2, final norm, soft-cap).
+
+    Returns a dict with ``logits`` ([B,T,V] capped, fp64, if ``want_logits``),
+    ``token_loss`` ([B,T]) and ``loss`` (scalar) when targets are given.
+    Rows are processed one at a time to bound memory.
+    """
+    idx = np.asarray(idx)
+    B, T = idx.shape
+    C, H, Hkv, D = cfg.d_model, cfg.n_head, cfg.n_kv_head, cfg.head_dim
+    eps = cfg.norm_eps
+    windows = layer_windows(cfg)
+    cos, sin = rope_tables(T, D, cfg.rope_base)
+    logits_out = [] if want_logits else None
+    nll_rows = []
+    for b in range(B):
+        x = embed(weights["wte"], idx[b:b + 1])  # [1,T,C]
+        for l, lw in enumerate(weights["layers"]):
+            a = rms_norm(x, eps)
+            q = (a @ _w(lw["c_q"]).T).reshape(1, T, H, D)
+            k = (a @ _w(lw["c_k"]).T).reshape(1, T, Hkv, D)
+            v = (a @ _w(lw["c_v"]).T).reshape(1, T, Hkv, D)
+            q = rms_norm(rope(q, cos, sin), eps)
+            k = rms_norm(rope(k, cos, sin), eps)
+            o = attention(q, k, v, windows[l])
+            x = x + o.reshape(1, T, H * D) @ _w(lw["attn_proj"]).T
+            a = rms_norm(x, eps)
+            x = x + relu2_mlp(a, lw["c_fc"], lw["mlp_proj"])
+        a = rms_norm(x, eps)
+        logits = softcap(a @ _w(weights["lm_head"]).T, cfg.softcap)  # [1,T,V]
+        if want_logits:
+            logits_out.append(logits[0])
+        if targets is not None:
+            nll, _ = cross_entropy(logits[0], np.asarray(targets)[b])
+            nll_rows.append(nll)
+    res = {}
+    if want_logits:
+        res["logits"] = np.stack(logits_out)
+    if targets is not None:
+        tl = np.stack(nll_rows)
+        y = np.asarray(targets)
+        n = int((y != -1).sum())
+        res["token_loss"] = tl
+        res["loss"] = float(tl.sum() / n) if n > 0 else float("nan")
+    return res
