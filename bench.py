@@ -1,0 +1,399 @@
+#!/usr/bin/env python3
+"""Throughput of the forward + loss of the nanochat GPT block stack on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config d20] [--impl ours|reference]
+
+One step = one whole forward + loss (fp32 -> bf16 weight cast, embedding, all
+blocks, lm_head, soft-capped cross-entropy) over one [B, T] batch of synthetic
+tokens, on each rank.  With N > 1 (torchrun, one process per GPU) each rank
+runs its own batch shard (weak scaling, weights replicated) and the global mean
+loss is formed by one all-reduce of (loss sum, token count) per step.
+
+Prints one JSON line (rank 0).  ``value`` is device-timed tokens/s over all
+ranks (CUDA events, max over ranks) with inputs resident in HBM; ``e2e`` is the
+same metric through the public API with the tokens copied from pinned host
+memory and the loss read back every step; ``roofline`` is the dominant kernel
+(the tcgen05 projection GEMM) timed per launch with CUDA events on the forward's
+stream inside the timed region; ``cpu_baseline`` is the fp64 oracle on a bounded
+sample, timed on the host cores.  ``--impl reference`` times that oracle alone.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from workloads import SHAPES, TOKEN_SEED, make_tokens, make_weights  # noqa: E402
+
+METRIC = "forward+loss tokens/sec at d20 (1×B200); % of bf16 dense tensor peak"
+UNIT = "tokens/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+GEMM_KINDS = ("gemm_qkv", "gemm_attn_proj", "gemm_fc", "gemm_mlp_proj", "gemm_lm_head")
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_work(s, kind):
+    """Algorithmic FLOPs (GEMM/attention) or bytes (bandwidth-bound kernels) of one
+    launch of `kind` in the forward of workload `s` (per-layer kinds: one layer)."""
+    M = s.batch * s.seq_len
+    C, H, Hkv, D, V = s.d_model, s.n_head, s.n_kv_head, s.head_dim, s.vocab
+    if kind == "gemm_qkv":
+        return 2.0 * M * C * (H + 2 * Hkv) * D
+    if kind == "gemm_attn_proj":
+        return 2.0 * M * H * D * C
+    if kind in ("gemm_fc", "gemm_mlp_proj"):
+        return 8.0 * M * C * C
+    if kind == "gemm_lm_head":
+        return 2.0 * M * C * V
+    if kind == "rmsnorm":  # fp32 read + bf16 write
+        return M * C * 6.0
+    if kind == "rope_qknorm":  # bf16 read + write of q and k, table read
+        return M * (H + Hkv) * D * 4.0
+    if kind == "embedding":
+        return M * C * 8.0 + M * 4.0
+    if kind == "cast":
+        L = s.n_layer
+        n = L * (C * (H + 2 * Hkv) * D + C * H * D + 8 * C * C) + V * C
+        return n * 6.0
+    return 0.0
+
+
+class ClockSampler:
+    """nvidia-smi clocks/throttle reasons sampled every 200 ms while running."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu_index = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu_index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        rows = []
+        try:
+            with open(self.path) as f:
+                for line in f:
+                    parts = [p.strip() for p in line.split(",")]
+                    if len(parts) >= 9:
+                        rows.append(parts)
+        except OSError:
+            pass
+        finally:
+            try:
+                os.unlink(self.path)
+            except OSError:
+                pass
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return len(os.sched_getaffinity(0))
+
+
+def oracle_sample(s, prefix, seed=TOKEN_SEED, weights=None):
+    """Runs the fp64 oracle on batch row 0, first `prefix` positions; returns
+    (tokens processed, seconds)."""
+    import oracle
+    w = make_weights(s) if weights is None else weights
+    x, y = make_tokens(s, seed=seed)
+    cfg = oracle.OracleConfig(s.n_layer, s.d_model, s.n_head, s.n_kv_head, s.head_dim, s.seq_len,
+                              s.vocab, short_window=s.short_window)
+    t0 = time.perf_counter()
+    oracle.forward(cfg, w, x[:1, :prefix], y[:1, :prefix], want_logits=False)
+    return prefix, time.perf_counter() - t0
+
+
+def run_reference(args, s):
+    """The oracle arm: rank 0 times the fp64 CPU oracle; other ranks exit."""
+    if int(os.environ.get("RANK", "0")) != 0:
+        return
+    prefix = args.ref_prefix
+    w = make_weights(s)
+    for _ in range(args.warmup):
+        oracle_sample(s, prefix, weights=w)
+    times = [oracle_sample(s, prefix, weights=w)[1] for _ in range(args.steps)]
+    sec = sum(times) / len(times)
+    value = prefix / sec
+    sample = f"{s.name} batch row 0, first {prefix} positions, forward+loss per step"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": s.name, "global_batch": 1, "seq_len": prefix, "parallelism": "none"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args, s):
+    import torch
+    import torch.distributed as dist
+
+    import decoder_only_transformer_nc_b200 as nc
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", device_id=dev, timeout=timedelta(seconds=120))
+
+    cfg = nc.make_config(s.n_layer, s.d_model, s.n_head, s.n_kv_head, s.head_dim, s.seq_len, s.vocab,
+                         s.short_window)
+    weights = make_weights(s)
+    model = nc.Model.from_numpy(cfg, weights, device=dev)
+    B, T = s.batch, s.seq_len
+    x, y = make_tokens(s, seed=TOKEN_SEED + rank)
+    tx, ty = torch.from_numpy(x).to(dev), torch.from_numpy(y).to(dev)
+    ws = torch.empty(nc.workspace_bytes(cfg, B, T), dtype=torch.uint8, device=dev)
+    out = {"loss": torch.empty((), dtype=torch.float32, device=dev)}
+    red = torch.zeros(2, dtype=torch.float64, device=dev)
+    n_valid = float((y != -1).sum())
+
+    def step(trace=None, toks=tx, tgts=ty):
+        nc.forward(model, toks, tgts, workspace=ws, out=out, trace=trace)
+        if world > 1:
+            red[0] = out["loss"].double() * n_valid
+            red[1] = n_valid
+            dist.all_reduce(red)
+
+    def barrier():
+        if world > 1:
+            dist.barrier(device_ids=[local])
+
+    # warm-up (untimed)
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    status = nc.get_status(ws)
+    if status != 0:
+        raise SystemExit(f"device status after warm-up: {nc.STATUS_NAMES.get(status, status)}")
+
+    probe = nc.LaunchTrace(4)
+    try:
+        nc.forward(model, tx, ty, workspace=ws, out=out, trace=probe)
+    except nc.NcError:
+        pass
+    n_launch = probe.struct.count
+    probe.close()
+    torch.cuda.synchronize()
+    traces = [nc.LaunchTrace(n_launch) for _ in range(args.steps)]
+
+    stream = torch.cuda.current_stream()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clocks:
+        t0.record(stream)
+        for k in range(args.steps):
+            step(traces[k])
+        t1.record(stream)
+        torch.cuda.synchronize()
+    barrier()
+    ms = t0.elapsed_time(t1) / args.steps
+    status = nc.get_status(ws)
+    clk = clocks.summary()
+
+    # per-kind launch times from the events of the timed region
+    per_kind = {}
+    for tr in traces:
+        for kind, kms in tr.launches():
+            d = per_kind.setdefault(kind, [0.0, 0])
+            d[0] += kms
+            d[1] += 1
+    for tr in traces:
+        tr.close()
+
+    # ---- e2e through the public API: pinned host inputs in, loss out, every step
+    hx = torch.from_numpy(x).pin_memory()
+    hy = torch.from_numpy(y).pin_memory()
+    dx, dy = torch.empty_like(tx), torch.empty_like(ty)
+    hloss = torch.empty((), dtype=torch.float32).pin_memory()
+    for _ in range(2):
+        dx.copy_(hx, non_blocking=True)
+        dy.copy_(hy, non_blocking=True)
+        step(toks=dx, tgts=dy)
+        hloss.copy_(out["loss"], non_blocking=True)
+    barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        dx.copy_(hx, non_blocking=True)
+        dy.copy_(hy, non_blocking=True)
+        step(toks=dx, tgts=dy)
+        hloss.copy_(out["loss"], non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = e0.elapsed_time(e1) / args.steps
+
+    # max over ranks
+    if world > 1:
+        tt = torch.tensor([ms, e2e_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms, e2e_ms = float(tt[0]), float(tt[1])
+
+    tokens_all = world * B * T
+    value = tokens_all / (ms / 1e3)
+    e2e_value = tokens_all / (e2e_ms / 1e3)
+    flops = nc.forward_flops(cfg, B, T)
+    peaks, peak_src = load_peaks()
+
+    gemm_ms = sum(per_kind[k][0] for k in GEMM_KINDS if k in per_kind)
+    gemm_launches = sum(per_kind[k][1] for k in GEMM_KINDS if k in per_kind)
+    gemm_flops = sum(kernel_work(s, k) * per_kind[k][1] for k in GEMM_KINDS if k in per_kind)
+    achieved = gemm_flops / (gemm_ms / 1e3) / 1e12 if gemm_ms > 0 else 0.0
+    peak = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+    total_traced = sum(v[0] for v in per_kind.values())
+    attn_flops_step = flops - sum(kernel_work(s, g) * per_kind[g][1] / args.steps
+                                  for g in GEMM_KINDS if g in per_kind)
+    kernels = {}
+    for k, (kms, n) in sorted(per_kind.items(), key=lambda kv: -kv[1][0]):
+        ent = {"launches": n, "ms_total": round(kms, 3), "share": round(kms / total_traced, 4)}
+        if k.startswith("gemm"):
+            ent["tflops"] = round(kernel_work(s, k) * n / (kms / 1e3) / 1e12, 1)
+        elif k == "attention":
+            ent["tflops"] = round(attn_flops_step * args.steps / (kms / 1e3) / 1e12, 1)
+        elif kernel_work(s, k) > 0:
+            ent["gbs"] = round(kernel_work(s, k) * n / (kms / 1e3) / 1e9, 1)
+        kernels[k] = ent
+
+    result = None
+    if rank == 0:
+        tflops = flops * world / (ms / 1e3) / 1e12
+        burst = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+        result = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": s.name, "global_batch": world * B, "seq_len": T,
+                       "parallelism": f"dp{world}" if world > 1 else "none",
+                       "layers": s.n_layer, "d_model": s.d_model,
+                       "l2": "inputs larger than L2 (fp32 weights %.2f GB, residual stream %.2f GB per step)"
+                             % (4 * sum(a.size for a in _flat(weights)) / 1e9, 4 * B * T * s.d_model / 1e9)},
+            "tflops": round(tflops, 1),
+            "pct_of_bf16_peak": {"measured_burst": round(100 * tflops / world / burst, 2),
+                                 "measured_sustained": round(100 * tflops / world / peak, 2),
+                                 "datasheet_dense_2250": round(100 * tflops / world / 2250.0, 2),
+                                 "source": peak_src},
+            "roofline": {"kernel": "gemm_kernel (tcgen05 projection GEMMs: qkv, attn c_proj, c_fc, mlp c_proj, lm_head)",
+                         "bound": "tensor", "achieved": round(achieved, 1),
+                         "peak": peak, "peak_kind": f"bf16_tflops_sustained ({peak_src})",
+                         "unit": "TFLOP/s", "frac": round(achieved / peak, 4), "traffic": None,
+                         "launches": gemm_launches, "avg_launch_ms": round(gemm_ms / max(1, gemm_launches), 4)},
+            "kernels": kernels,
+            "gpu_launches": n_launch * args.steps,
+            "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": int(x.nbytes + y.nbytes),
+                    "d2h_bytes_per_step": 4},
+            "clocks": clk,
+            "device_status": nc.STATUS_NAMES.get(status, status),
+        }
+    if world > 1:
+        dist.barrier(device_ids=[local])
+        dist.destroy_process_group()
+    if rank == 0:
+        if world == 1 and not args.no_cpu_baseline:
+            del model, ws
+            torch.cuda.empty_cache()
+            n_tok, sec = oracle_sample(s, args.cpu_prefix, weights=weights)
+            result["cpu_baseline"] = {
+                "value": n_tok / sec, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+                "sample": f"{s.name} batch row 0, first {args.cpu_prefix} positions, fp64 forward+loss "
+                          f"({sec:.1f} s)"}
+        print(json.dumps(result), flush=True)
+
+
+def _flat(w):
+    yield w["wte"]
+    yield w["lm_head"]
+    for lw in w["layers"]:
+        yield from lw.values()
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", default="d20", choices=sorted(SHAPES))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-prefix", type=int, default=1024,
+                    help="positions of batch row 0 in the oracle CPU-baseline sample")
+    ap.add_argument("--ref-prefix", type=int, default=256,
+                    help="positions of batch row 0 per step of the reference (oracle) arm")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    s = SHAPES[args.config]
+    if args.impl == "reference":
+        run_reference(args, s)
+    else:
+        run_ours(args, s)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,346 @@
+"""B200-native forward pass + loss of the nanochat GPT block stack.
+
+Thin ctypes binding of ``libnc.so`` (the C ABI declared in ``include/nc.h``).
+This module only marshals arguments: every step of the forward runs in the
+library's CUDA kernels.  PyTorch provides device memory and streams.  There is
+no CPU fallback: if the library is missing or the device is not sm_100 every
+call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+__all__ = [
+    "NcError", "NcConfig", "lib", "init_config", "make_config", "check_config", "layer_window",
+    "workspace_bytes", "forward_flops", "Model", "forward", "LaunchTrace", "KERNEL_KINDS", "get_status", "cast_bf16", "embedding",
+    "rmsnorm", "rope_table", "rope_qknorm", "attention", "linear", "softcap_ce", "loss_mean",
+    "EPI_STORE_BF16", "EPI_RELU2_BF16", "EPI_RESID_F32", "EPI_STORE_F32", "EPI_SOFTCAP_F32",
+]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libnc.so")
+
+EPI_STORE_BF16, EPI_RELU2_BF16, EPI_RESID_F32, EPI_STORE_F32, EPI_SOFTCAP_F32 = range(5)
+DEV_TOKEN_RANGE, DEV_TARGET_RANGE, DEV_TIMEOUT = 0x1, 0x2, 0x4
+
+STATUS_NAMES = {0: "NC_OK", 1: "NC_ERR_INVALID_ARG", 2: "NC_ERR_CONFIG", 3: "NC_ERR_SHAPE",
+                4: "NC_ERR_ALIGNMENT", 5: "NC_ERR_WORKSPACE", 6: "NC_ERR_TOKEN_RANGE",
+                7: "NC_ERR_TIMEOUT", 8: "NC_ERR_UNSUPPORTED_DEVICE", 9: "NC_ERR_CUDA"}
+
+
+class NcError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where}: {STATUS_NAMES.get(code, code)}")
+
+
+class NcConfig(ctypes.Structure):
+    _fields_ = [("n_layer", ctypes.c_int32), ("d_model", ctypes.c_int32), ("n_head", ctypes.c_int32),
+                ("n_kv_head", ctypes.c_int32), ("head_dim", ctypes.c_int32), ("vocab", ctypes.c_int32),
+                ("seq_len", ctypes.c_int32), ("short_window", ctypes.c_int32),
+                ("window_pattern", ctypes.c_char * 8), ("softcap", ctypes.c_float),
+                ("norm_eps", ctypes.c_float), ("rope_base", ctypes.c_float)]
+
+    def __repr__(self):
+        return ("NcConfig(n_layer=%d, d_model=%d, n_head=%d, n_kv_head=%d, head_dim=%d, vocab=%d, "
+                "seq_len=%d, short_window=%d, pattern=%r)" % (
+                    self.n_layer, self.d_model, self.n_head, self.n_kv_head, self.head_dim,
+                    self.vocab, self.seq_len, self.short_window, self.window_pattern.decode()))
+
+
+_FPP = ctypes.POINTER(ctypes.c_void_p)
+
+
+class NcWeights(ctypes.Structure):
+    _fields_ = [("wte", ctypes.c_void_p), ("c_q", _FPP), ("c_k", _FPP), ("c_v", _FPP),
+                ("attn_proj", _FPP), ("c_fc", _FPP), ("mlp_proj", _FPP), ("lm_head", ctypes.c_void_p)]
+
+
+class NcTrace(ctypes.Structure):
+    _fields_ = [("events", ctypes.POINTER(ctypes.c_void_p)), ("capacity", ctypes.c_int32),
+                ("count", ctypes.c_int32), ("kinds", ctypes.POINTER(ctypes.c_int32))]
+
+
+KERNEL_KINDS = ("rope_table", "cast", "embedding", "rmsnorm", "gemm_qkv", "rope_qknorm", "attention",
+                "gemm_attn_proj", "gemm_fc", "gemm_mlp_proj", "gemm_lm_head", "ce_finalize", "loss_mean")
+
+_lib = None
+
+
+def lib():
+    """The loaded CUDA library (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(
+                f"{LIB_PATH} is missing: build it with `python -m decoder_only_transformer_nc_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, i32, i64, f32, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t
+        cfgp = ctypes.POINTER(NcConfig)
+        sigs = {
+            "nc_init_config": (i32, [cfgp, i32, i32, i32, i32, i32, i32]),
+            "nc_check_config": (i32, [cfgp]),
+            "nc_layer_window": (i32, [cfgp, i32]),
+            "nc_workspace_bytes": (sz, [cfgp, i32, i32]),
+            "nc_forward_flops": (ctypes.c_double, [cfgp, i32, i32]),
+            "nc_status_string": (ctypes.c_char_p, [i32]),
+            "nc_version": (i32, []),
+            "nc_forward": (i32, [cfgp, ctypes.POINTER(NcWeights), vp, vp, i32, i32, vp, vp, vp, vp, sz, vp]),
+            "nc_forward_traced": (i32, [cfgp, ctypes.POINTER(NcWeights), vp, vp, i32, i32, vp, vp, vp, vp,
+                                        sz, vp, ctypes.POINTER(NcTrace)]),
+            "nc_event_create": (i32, [ctypes.POINTER(ctypes.c_void_p)]),
+            "nc_event_destroy": (i32, [vp]),
+            "nc_event_elapsed_ms": (i32, [vp, vp, ctypes.POINTER(ctypes.c_float)]),
+            "nc_get_status": (i32, [vp, vp]),
+            "nc_cast_bf16": (i32, [vp, vp, i64, vp]),
+            "nc_embedding": (i32, [vp, vp, vp, i32, i32, i32, vp, vp]),
+            "nc_rmsnorm": (i32, [vp, vp, i32, i32, f32, vp]),
+            "nc_rope_table": (i32, [vp, i32, i32, f32, vp]),
+            "nc_rope_qknorm": (i32, [vp, vp, vp, i32, i32, i32, i32, i32, i64, i64, f32, vp]),
+            "nc_attention": (i32, [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, vp]),
+            "nc_attention_strided": (i32, [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i64, i64, vp]),
+            "nc_linear": (i32, [vp, vp, vp, i32, i32, i32, i64, i32, f32, vp, vp]),
+            "nc_softcap_ce": (i32, [vp, vp, vp, vp, i32, i32, f32, vp, vp]),
+            "nc_loss_mean": (i32, [vp, vp, i32, i32, vp, vp]),
+            "nc_selftest_bounded_wait": (i32, [vp, ctypes.c_uint32, vp]),
+        }
+        for name, (res, args) in sigs.items():
+            fn = getattr(L, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = L
+    return _lib
+
+
+def _check(code: int, where: str):
+    if code != 0:
+        raise NcError(code, where)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    import torch
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+# ---------------------------------------------------------------- configuration
+
+def init_config(depth: int, aspect_ratio: int = 64, head_dim: int = 128, n_kv_head: int = 0,
+                seq_len: int = 2048, vocab: int = 32768) -> NcConfig:
+    c = NcConfig()
+    _check(lib().nc_init_config(ctypes.byref(c), depth, aspect_ratio, head_dim, n_kv_head, seq_len,
+                                vocab), "nc_init_config")
+    return c
+
+
+def make_config(n_layer, d_model, n_head, n_kv_head, head_dim, seq_len, vocab, short_window=0,
+                window_pattern="SSSL", softcap=15.0, norm_eps=1e-6, rope_base=10000.0) -> NcConfig:
+    c = NcConfig(n_layer, d_model, n_head, n_kv_head, head_dim, vocab, seq_len,
+                 short_window if short_window > 0 else seq_len // 4, window_pattern.encode(),
+                 softcap, norm_eps, rope_base)
+    _check(lib().nc_check_config(ctypes.byref(c)), "nc_check_config")
+    return c
+
+
+def check_config(c: NcConfig) -> int:
+    return lib().nc_check_config(ctypes.byref(c))
+
+
+def layer_window(c: NcConfig, layer: int) -> int:
+    return lib().nc_layer_window(ctypes.byref(c), layer)
+
+
+def workspace_bytes(c: NcConfig, B: int, T: int) -> int:
+    return lib().nc_workspace_bytes(ctypes.byref(c), B, T)
+
+
+def forward_flops(c: NcConfig, B: int, T: int) -> float:
+    return lib().nc_forward_flops(ctypes.byref(c), B, T)
+
+
+# ---------------------------------------------------------------- model
+
+@dataclass
+class Model:
+    """fp32 weights resident on the device plus the nc_weights view of them."""
+
+    cfg: NcConfig
+    tensors: dict
+    weights: NcWeights
+    _keep: list
+
+    @classmethod
+    def from_tensors(cls, cfg: NcConfig, t: dict) -> "Model":
+        """t: {"wte", "lm_head", "layers": [{c_q, c_k, c_v, attn_proj, c_fc, mlp_proj}]}
+        with contiguous float32 CUDA tensors in [out, in] layout."""
+        L = cfg.n_layer
+        arrs = {}
+        for name in ("c_q", "c_k", "c_v", "attn_proj", "c_fc", "mlp_proj"):
+            a = (ctypes.c_void_p * L)(*[t["layers"][l][name].data_ptr() for l in range(L)])
+            arrs[name] = a
+        w = NcWeights(t["wte"].data_ptr(), *[ctypes.cast(arrs[n], _FPP) for n in
+                                             ("c_q", "c_k", "c_v", "attn_proj", "c_fc", "mlp_proj")],
+                      t["lm_head"].data_ptr())
+        return cls(cfg, t, w, list(arrs.values()))
+
+    @classmethod
+    def from_numpy(cls, cfg: NcConfig, w: dict, device="cuda") -> "Model":
+        import torch
+        dev = lambda a: torch.from_numpy(a).to(device).contiguous()
+        t = {"wte": dev(w["wte"]), "lm_head": dev(w["lm_head"]),
+             "layers": [{k: dev(v) for k, v in lw.items()} for lw in w["layers"]]}
+        return cls.from_tensors(cfg, t)
+
+
+def forward(model: Model, tokens, targets=None, want_logits=False, want_token_loss=False,
+            workspace=None, stream=None, out=None, trace: "LaunchTrace | None" = None):
+    """Runs nc_forward.  tokens/targets: int32 CUDA tensors [B, T].
+
+    Returns a dict of CUDA tensors: ``loss`` (scalar, if targets), ``token_loss``
+    ([B,T], if asked), ``logits`` ([B,T,V] fp32 soft-capped, if asked) and the
+    ``workspace`` used (its first word is the device status of the call).
+    ``out`` may hold preallocated tensors under the same keys.
+    """
+    import torch
+    cfg = model.cfg
+    B, T = tokens.shape
+    out = {} if out is None else out
+    dev = tokens.device
+    need = workspace_bytes(cfg, B, T)
+    if need == 0:
+        raise NcError(3, "nc_workspace_bytes")
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    res = {"workspace": workspace}
+    logits = tl = loss = None
+    if want_logits:
+        logits = out.get("logits")
+        if logits is None:
+            logits = torch.empty((B, T, cfg.vocab), dtype=torch.float32, device=dev)
+        res["logits"] = logits
+    if targets is not None:
+        loss = out.get("loss")
+        if loss is None:
+            loss = torch.empty((), dtype=torch.float32, device=dev)
+        res["loss"] = loss
+        if want_token_loss:
+            tl = out.get("token_loss")
+            if tl is None:
+                tl = torch.empty((B, T), dtype=torch.float32, device=dev)
+            res["token_loss"] = tl
+    _check(lib().nc_forward_traced(ctypes.byref(cfg), ctypes.byref(model.weights), _ptr(tokens),
+                                   _ptr(targets), B, T, _ptr(logits), _ptr(tl), _ptr(loss),
+                                   _ptr(workspace), workspace.numel(), _stream(stream),
+                                   None if trace is None else ctypes.byref(trace.struct)),
+           "nc_forward")
+    return res
+
+
+class LaunchTrace:
+    """Per-launch CUDA events for one traced forward (see nc_forward_traced)."""
+
+    def __init__(self, capacity: int):
+        L = lib()
+        self.capacity = capacity
+        self._ev = (ctypes.c_void_p * (2 * capacity))()
+        for i in range(2 * capacity):
+            h = ctypes.c_void_p()
+            _check(L.nc_event_create(ctypes.byref(h)), "nc_event_create")
+            self._ev[i] = h
+        self._kinds = (ctypes.c_int32 * capacity)()
+        self.struct = NcTrace(ctypes.cast(self._ev, ctypes.POINTER(ctypes.c_void_p)), capacity, 0,
+                              ctypes.cast(self._kinds, ctypes.POINTER(ctypes.c_int32)))
+
+    def launches(self):
+        """[(kind name, milliseconds)] of the last traced forward (waits for it)."""
+        L = lib()
+        out = []
+        ms = ctypes.c_float()
+        for i in range(self.struct.count):
+            _check(L.nc_event_elapsed_ms(self._ev[2 * i], self._ev[2 * i + 1], ctypes.byref(ms)),
+                   "nc_event_elapsed_ms")
+            out.append((KERNEL_KINDS[self._kinds[i]], ms.value))
+        return out
+
+    def close(self):
+        if self._ev is not None:
+            for i in range(2 * self.capacity):
+                lib().nc_event_destroy(self._ev[i])
+            self._ev = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def get_status(status_tensor, stream=None) -> int:
+    """Synchronises the stream and returns the nc_status of a device status word."""
+    return lib().nc_get_status(_ptr(status_tensor), _stream(stream))
+
+
+# ---------------------------------------------------------------- single steps
+
+def cast_bf16(src, dst, stream=None):
+    _check(lib().nc_cast_bf16(_ptr(src), _ptr(dst), src.numel(), _stream(stream)), "nc_cast_bf16")
+
+
+def embedding(tokens, wte, x, status=None, stream=None):
+    M = tokens.numel()
+    V, C = wte.shape
+    _check(lib().nc_embedding(_ptr(tokens), _ptr(wte), _ptr(x), M, C, V, _ptr(status), _stream(stream)),
+           "nc_embedding")
+
+
+def rmsnorm(x, out, eps=1e-6, stream=None):
+    C = x.shape[-1]
+    _check(lib().nc_rmsnorm(_ptr(x), _ptr(out), x.numel() // C, C, eps, _stream(stream)), "nc_rmsnorm")
+
+
+def rope_table(table, T, D, base=10000.0, stream=None):
+    _check(lib().nc_rope_table(_ptr(table), T, D, base, _stream(stream)), "nc_rope_table")
+
+
+def rope_qknorm(q, k, table, B, T, H, Hkv, D, q_row_stride=None, k_row_stride=None, eps=1e-6,
+                stream=None):
+    qs = H * D if q_row_stride is None else q_row_stride
+    ks = Hkv * D if k_row_stride is None else k_row_stride
+    _check(lib().nc_rope_qknorm(_ptr(q), _ptr(k), _ptr(table), B, T, H, Hkv, D, qs, ks, eps,
+                                _stream(stream)), "nc_rope_qknorm")
+
+
+def attention(q, k, v, out, window, stream=None):
+    B, T, H, D = q.shape
+    Hkv = k.shape[2]
+    _check(lib().nc_attention(_ptr(q), _ptr(k), _ptr(v), _ptr(out), B, T, H, Hkv, D, window,
+                              _stream(stream)), "nc_attention")
+
+
+def linear(a, w, out, epilogue, cap=15.0, status=None, stream=None):
+    M, K = a.shape
+    N = w.shape[0]
+    _check(lib().nc_linear(_ptr(a), _ptr(w), _ptr(out), M, N, K, out.stride(0), epilogue, cap,
+                           _ptr(status), _stream(stream)), "nc_linear")
+
+
+def softcap_ce(z, targets, token_loss, capped_out=None, cap=15.0, status=None, stream=None):
+    M, V = z.shape
+    _check(lib().nc_softcap_ce(_ptr(z), _ptr(targets), _ptr(capped_out), _ptr(token_loss), M, V, cap,
+                               _ptr(status), _stream(stream)), "nc_softcap_ce")
+
+
+def selftest_bounded_wait(status, limit_us=20000, stream=None):
+    _check(lib().nc_selftest_bounded_wait(_ptr(status), limit_us, _stream(stream)),
+           "nc_selftest_bounded_wait")
+
+
+def loss_mean(token_loss, targets, V, loss, stream=None):
+    _check(lib().nc_loss_mean(_ptr(token_loss), _ptr(targets), token_loss.numel(), V, _ptr(loss),
+                              _stream(stream)), "nc_loss_mean")

@@ -1,0 +1,526 @@
+// Public C ABI (include/nc.h): argument checks, workspace layout and the
+// launch sequence of the forward pass.
+//
+// Forward ("从文本到聊天模型" §5; block internals from "Nanochat与nanoGPT对比：
+// 关键升级" §1), all on the caller's stream:
+//   RoPE table; fp32 -> bf16 weight cast (Wq|Wk|Wv packed as one [(H+2Hkv)D, C]
+//   matrix per layer); embedding gather;
+//   per layer: RMSNorm -> QKV GEMM -> RoPE+QK-norm -> attention (layer window)
+//              -> c_proj GEMM with residual add -> RMSNorm -> c_fc GEMM with
+//              ReLU^2 -> c_proj GEMM with residual add;
+//   final RMSNorm -> lm_head GEMM whose epilogue applies the soft-cap and
+//   reduces each 256-column tile to sum(exp(l - cap)) (+ the target logit)
+//   -> per-row combine to NLL -> fixed-order mean.
+// The residual stream stays fp32; matmul operands are bf16 with fp32
+// accumulation.
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "nc_internal.h"
+
+namespace nc {
+
+namespace {
+struct DevInfo {
+  int sms = 0;
+  bool sm100 = false;
+  bool init = false;
+};
+DevInfo g_dev[64];
+std::mutex g_dev_mu;
+
+const DevInfo* dev_info() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  DevInfo& d = g_dev[dev];
+  if (!d.init) {
+    cudaDeviceProp p;
+    if (cudaGetDeviceProperties(&p, dev) != cudaSuccess) return nullptr;
+    d.sms = p.multiProcessorCount;
+    d.sm100 = (p.major == 10 && p.minor == 0);
+    d.init = true;
+  }
+  return &d;
+}
+}  // namespace
+
+int device_sm_count() {
+  const DevInfo* d = dev_info();
+  return d ? d->sms : 148;
+}
+bool device_is_sm100() {
+  const DevInfo* d = dev_info();
+  return d && d->sm100;
+}
+
+}  // namespace nc
+
+using namespace nc;
+
+namespace {
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+bool config_ok(const nc_config* c) {
+  if (!c) return false;
+  if (c->n_layer < 1 || c->d_model < 64 || c->n_head < 1 || c->n_kv_head < 1) return false;
+  if (c->n_head % c->n_kv_head != 0) return false;
+  if (c->head_dim != 64 && c->head_dim != 128) return false;
+  if (c->vocab < 64 || c->vocab % 64 != 0) return false;
+  if (c->seq_len < 1 || c->short_window < 1) return false;
+  if (c->d_model % 64 != 0) return false;
+  if ((int64_t)c->n_head * c->head_dim % 64 != 0) return false;
+  if (!(c->softcap > 0.0f) || !(c->norm_eps >= 0.0f) || !(c->rope_base > 1.0f)) return false;
+  const size_t plen = strnlen(c->window_pattern, sizeof(c->window_pattern));
+  if (plen == 0 || plen >= sizeof(c->window_pattern)) return false;
+  for (size_t i = 0; i < plen; ++i)
+    if (c->window_pattern[i] != 'S' && c->window_pattern[i] != 'L') return false;
+  return true;
+}
+
+// Workspace layout of nc_forward.  Offsets are 256-byte aligned.
+struct WsLayout {
+  size_t status, rope, wqkv, wo, wfc, wmp, wlm, x, a, qkv, o, h, part, tgt, tl, total;
+  size_t wqkv_elems, wo_elems, wfc_elems, wmp_elems;  // per layer
+};
+
+WsLayout ws_layout(const nc_config* c, int B, int T) {
+  WsLayout L;
+  const size_t M = (size_t)B * T;
+  const size_t C = c->d_model, D = c->head_dim, H = c->n_head, Hkv = c->n_kv_head, V = c->vocab;
+  const size_t nqkv = (H + 2 * Hkv) * D;
+  L.wqkv_elems = nqkv * C;
+  L.wo_elems = C * H * D;
+  L.wfc_elems = 4 * C * C;
+  L.wmp_elems = C * 4 * C;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    size_t o = off;
+    off = align_up(off + bytes, 256);
+    return o;
+  };
+  L.status = take(256);
+  L.rope = take((size_t)T * D * sizeof(float));
+  L.wqkv = take(c->n_layer * L.wqkv_elems * 2);
+  L.wo = take(c->n_layer * L.wo_elems * 2);
+  L.wfc = take(c->n_layer * L.wfc_elems * 2);
+  L.wmp = take(c->n_layer * L.wmp_elems * 2);
+  L.wlm = take(V * C * 2);
+  L.x = take(M * C * 4);
+  L.a = take(M * C * 2);
+  L.qkv = take(M * nqkv * 2);
+  L.o = take(M * H * D * 2);
+  L.h = take(M * 4 * C * 2);
+  L.part = take(M * (size_t)gemm_num_n_tiles((int)V) * 4);
+  L.tgt = take(M * 4);
+  L.tl = take(M * 4);
+  L.total = off;
+  return L;
+}
+
+inline cudaStream_t S(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+// Brackets each launch of the forward with a caller-provided pair of events.
+struct Tracer {
+  nc_trace* t;
+  cudaStream_t st;
+  int n = 0;
+  bool dry;  // count launches only
+  bool begin(int kind) {
+    if (!t) return true;
+    if (!dry && n < t->capacity) {
+      if (t->kinds) t->kinds[n] = kind;
+      return cudaEventRecord(static_cast<cudaEvent_t>(t->events[2 * n]), st) == cudaSuccess;
+    }
+    return true;
+  }
+  bool end() {
+    if (!t) return true;
+    bool ok = true;
+    if (!dry && n < t->capacity)
+      ok = cudaEventRecord(static_cast<cudaEvent_t>(t->events[2 * n + 1]), st) == cudaSuccess;
+    ++n;
+    return ok;
+  }
+};
+
+// Number of kernel launches of one forward.
+int forward_launch_count(const nc_config* c, bool targets, bool loss, bool logits) {
+  int n = 3 + c->n_layer * 8 + 1;  // rope table, cast, embedding; layers; final norm
+  if (targets) n += 2 + (loss ? 1 : 0);
+  else if (logits) n += 1;
+  return n;
+}
+
+nc_status device_ok() {
+  return device_is_sm100() ? NC_OK : NC_ERR_UNSUPPORTED_DEVICE;
+}
+
+}  // namespace
+
+extern "C" {
+
+int nc_version(void) { return 100; }
+
+const char* nc_status_string(nc_status s) {
+  switch (s) {
+    case NC_OK: return "ok";
+    case NC_ERR_INVALID_ARG: return "invalid argument";
+    case NC_ERR_CONFIG: return "invalid configuration";
+    case NC_ERR_SHAPE: return "unsupported shape";
+    case NC_ERR_ALIGNMENT: return "pointer not 16-byte aligned";
+    case NC_ERR_WORKSPACE: return "workspace too small";
+    case NC_ERR_TOKEN_RANGE: return "token or target id out of range";
+    case NC_ERR_TIMEOUT: return "bounded device wait ran out";
+    case NC_ERR_UNSUPPORTED_DEVICE: return "device is not sm_100";
+    case NC_ERR_CUDA: return "CUDA runtime error";
+  }
+  return "unknown status";
+}
+
+nc_status nc_init_config(nc_config* out, int depth, int aspect_ratio, int head_dim, int n_kv_head,
+                         int seq_len, int vocab) {
+  if (!out || depth < 1 || aspect_ratio < 1 || head_dim < 1 || n_kv_head < 0 || seq_len < 4 ||
+      vocab < 1)
+    return NC_ERR_INVALID_ARG;
+  nc_config c;
+  memset(&c, 0, sizeof(c));
+  c.n_layer = depth;
+  c.d_model = depth * aspect_ratio;
+  c.head_dim = head_dim;
+  c.n_head = c.d_model / head_dim;
+  c.n_kv_head = n_kv_head > 0 ? n_kv_head : c.n_head;
+  c.vocab = vocab;
+  c.seq_len = seq_len;
+  c.short_window = seq_len / 4;
+  strcpy(c.window_pattern, "SSSL");
+  c.softcap = 15.0f;
+  c.norm_eps = 1e-6f;
+  c.rope_base = 10000.0f;
+  *out = c;
+  return config_ok(&c) ? NC_OK : NC_ERR_CONFIG;
+}
+
+nc_status nc_check_config(const nc_config* cfg) {
+  if (!cfg) return NC_ERR_INVALID_ARG;
+  return config_ok(cfg) ? NC_OK : NC_ERR_CONFIG;
+}
+
+int nc_layer_window(const nc_config* cfg, int layer) {
+  if (!config_ok(cfg) || layer < 0 || layer >= cfg->n_layer) return -1;
+  const size_t plen = strlen(cfg->window_pattern);
+  char kind = cfg->window_pattern[layer % plen];
+  if (layer == cfg->n_layer - 1) kind = 'L';
+  return kind == 'L' ? cfg->seq_len : cfg->short_window;
+}
+
+size_t nc_workspace_bytes(const nc_config* cfg, int B, int T) {
+  if (!config_ok(cfg) || B < 1 || T < 1 || T > cfg->seq_len) return 0;
+  return ws_layout(cfg, B, T).total;
+}
+
+double nc_forward_flops(const nc_config* cfg, int B, int T) {
+  if (!config_ok(cfg) || B < 1 || T < 1) return 0.0;
+  const double M = (double)B * T, C = cfg->d_model, D = cfg->head_dim, H = cfg->n_head,
+               Hkv = cfg->n_kv_head, V = cfg->vocab;
+  const double per_layer_proj = 2.0 * M * C * (H + 2 * Hkv) * D + 2.0 * M * H * D * C + 16.0 * M * C * C;
+  double f = cfg->n_layer * per_layer_proj + 2.0 * M * C * V;
+  for (int l = 0; l < cfg->n_layer; ++l) {
+    const int W = nc_layer_window(cfg, l);
+    double keys = 0.0;  // sum over query positions of visible keys
+    for (int i = 0; i < T; ++i) keys += (double)(i + 1 < W ? i + 1 : W);
+    f += 4.0 * D * H * B * keys;  // QK^T and PV, 2 flops per multiply-add each
+  }
+  return f;
+}
+
+nc_status nc_get_status(const void* dev_status, void* stream) {
+  if (!dev_status) return NC_ERR_INVALID_ARG;
+  uint32_t st = 0;
+  if (cudaStreamSynchronize(S(stream)) != cudaSuccess) return NC_ERR_CUDA;
+  if (cudaMemcpy(&st, dev_status, sizeof(st), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return NC_ERR_CUDA;
+  if (st & NC_DEV_TIMEOUT) return NC_ERR_TIMEOUT;
+  if (st & (NC_DEV_TOKEN_RANGE | NC_DEV_TARGET_RANGE)) return NC_ERR_TOKEN_RANGE;
+  return NC_OK;
+}
+
+nc_status nc_cast_bf16(const float* src, uint16_t* dst, int64_t n, void* stream) {
+  if (!src || !dst || n < 0 || n % 8 != 0) return NC_ERR_INVALID_ARG;
+  if (!aligned16(src) || !aligned16(dst)) return NC_ERR_ALIGNMENT;
+  if (nc_status s = device_ok()) return s;
+  CastSeg seg{src, dst, n};
+  return cast_launch(&seg, 1, S(stream));
+}
+
+nc_status nc_embedding(const int32_t* tokens, const float* wte, float* x, int M, int C, int V,
+                       uint32_t* dev_status, void* stream) {
+  if (!tokens || !wte || !x || M < 0 || C < 4 || C % 4 != 0 || V < 1) return NC_ERR_INVALID_ARG;
+  if (!aligned16(wte) || !aligned16(x)) return NC_ERR_ALIGNMENT;
+  if (nc_status s = device_ok()) return s;
+  return embedding_launch(tokens, wte, x, M, C, V, dev_status, S(stream));
+}
+
+nc_status nc_rmsnorm(const float* x, uint16_t* out, int M, int C, float eps, void* stream) {
+  if (!x || !out || M < 0 || C < 8 || C % 8 != 0 || !(eps >= 0.0f)) return NC_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(out)) return NC_ERR_ALIGNMENT;
+  if (nc_status s = device_ok()) return s;
+  return rmsnorm_launch(x, out, M, C, eps, S(stream));
+}
+
+nc_status nc_rope_table(float* table, int T, int D, float base, void* stream) {
+  if (!table || T < 1 || D < 2 || D % 2 != 0 || !(base > 1.0f)) return NC_ERR_INVALID_ARG;
+  if (nc_status s = device_ok()) return s;
+  return rope_table_launch(table, T, D, base, S(stream));
+}
+
+nc_status nc_rope_qknorm(uint16_t* q, uint16_t* k, const float* table, int B, int T, int H, int Hkv,
+                         int D, int64_t q_row_stride, int64_t k_row_stride, float eps,
+                         void* stream) {
+  if (!q || !k || !table || B < 0 || T < 1 || H < 1 || Hkv < 1) return NC_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return NC_ERR_SHAPE;
+  if (q_row_stride < (int64_t)H * D || k_row_stride < (int64_t)Hkv * D || q_row_stride % 8 ||
+      k_row_stride % 8)
+    return NC_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(table)) return NC_ERR_ALIGNMENT;
+  if (nc_status s = device_ok()) return s;
+  return rope_qknorm_launch(q, k, table, B, T, H, Hkv, D, q_row_stride, k_row_stride, eps,
+                            S(stream));
+}
+
+nc_status nc_attention_strided(const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                               uint16_t* out, int B, int T, int H, int Hkv, int D, int window,
+                               int64_t q_row_stride, int64_t kv_row_stride, void* stream) {
+  if (!q || !k || !v || !out || B < 0 || T < 0 || H < 1 || Hkv < 1 || H % Hkv != 0)
+    return NC_ERR_INVALID_ARG;
+  if (D != 128) return NC_ERR_SHAPE;
+  if (q_row_stride < (int64_t)H * D || kv_row_stride < (int64_t)Hkv * D || q_row_stride % 8 ||
+      kv_row_stride % 8)
+    return NC_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return NC_ERR_ALIGNMENT;
+  if (nc_status s = device_ok()) return s;
+  return attention_launch(q, k, v, out, B, T, H, Hkv, D, window, q_row_stride, kv_row_stride,
+                          S(stream));
+}
+
+nc_status nc_attention(const uint16_t* q, const uint16_t* k, const uint16_t* v, uint16_t* out, int B,
+                       int T, int H, int Hkv, int D, int window, void* stream) {
+  return nc_attention_strided(q, k, v, out, B, T, H, Hkv, D, window, (int64_t)H * D,
+                              (int64_t)Hkv * D, stream);
+}
+
+nc_status nc_linear(const uint16_t* a, const uint16_t* w, void* out, int M, int N, int K,
+                    int64_t ldo, nc_epilogue epilogue, float cap, uint32_t* dev_status,
+                    void* stream) {
+  if (!a || !w || !out || M < 0 || N < 32 || K < 8) return NC_ERR_INVALID_ARG;
+  if ((int)epilogue < 0 || (int)epilogue > (int)NC_EPI_SOFTCAP_F32) return NC_ERR_INVALID_ARG;
+  if (N % 32 != 0 || K % 8 != 0 || ldo < N || ldo % 8 != 0) return NC_ERR_SHAPE;
+  if (epilogue == NC_EPI_SOFTCAP_F32 && !(cap > 0.0f)) return NC_ERR_INVALID_ARG;
+  if (!aligned16(a) || !aligned16(w) || !aligned16(out)) return NC_ERR_ALIGNMENT;
+  if (nc_status s = device_ok()) return s;
+  if (M == 0) return NC_OK;
+  EpiParams ep{};
+  ep.out = out;
+  ep.ldo = ldo;
+  ep.cap = cap;
+  return gemm_launch(a, K, w, K, M, N, K, (int)epilogue, ep, dev_status, S(stream));
+}
+
+nc_status nc_softcap_ce(const float* z, const int32_t* targets, float* capped_out,
+                        float* token_loss, int M, int V, float cap, uint32_t* dev_status,
+                        void* stream) {
+  if (!z || !targets || !token_loss || M < 0 || V < 4 || V % 4 != 0 || !(cap > 0.0f))
+    return NC_ERR_INVALID_ARG;
+  if (!aligned16(z) || (capped_out && !aligned16(capped_out))) return NC_ERR_ALIGNMENT;
+  if (nc_status s = device_ok()) return s;
+  return softcap_ce_launch(z, targets, capped_out, token_loss, M, V, cap, dev_status, S(stream));
+}
+
+nc_status nc_loss_mean(const float* token_loss, const int32_t* targets, int M, int V, float* loss,
+                       void* stream) {
+  if (!token_loss || !targets || !loss || M < 0 || V < 1) return NC_ERR_INVALID_ARG;
+  if (nc_status s = device_ok()) return s;
+  return loss_mean_launch(token_loss, targets, M, V, loss, S(stream));
+}
+
+nc_status nc_forward_traced(const nc_config* cfg, const nc_weights* w, const int32_t* tokens,
+                            const int32_t* targets, int B, int T, float* logits,
+                            float* token_loss, float* loss, void* workspace, size_t ws_bytes,
+                            void* stream, nc_trace* trace) {
+  if (!cfg || !w || !tokens || !workspace) return NC_ERR_INVALID_ARG;
+  if (!config_ok(cfg)) return NC_ERR_CONFIG;
+  if (B < 1 || T < 1 || T > cfg->seq_len) return NC_ERR_SHAPE;
+  if ((token_loss || loss) && !targets) return NC_ERR_INVALID_ARG;
+  if (!w->wte || !w->lm_head || !w->c_q || !w->c_k || !w->c_v || !w->attn_proj || !w->c_fc ||
+      !w->mlp_proj)
+    return NC_ERR_INVALID_ARG;
+  if ((int64_t)B * T > (int64_t)1 << 30) return NC_ERR_SHAPE;
+  const WsLayout L = ws_layout(cfg, B, T);
+  if (ws_bytes < L.total) return NC_ERR_WORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return NC_ERR_ALIGNMENT;
+  if (!aligned16(w->wte) || !aligned16(w->lm_head) || (logits && !aligned16(logits)))
+    return NC_ERR_ALIGNMENT;
+  for (int l = 0; l < cfg->n_layer; ++l) {
+    const float* ps[6] = {w->c_q[l], w->c_k[l], w->c_v[l], w->attn_proj[l], w->c_fc[l], w->mlp_proj[l]};
+    for (const float* p : ps) {
+      if (!p) return NC_ERR_INVALID_ARG;
+      if (!aligned16(p)) return NC_ERR_ALIGNMENT;
+    }
+  }
+  if (trace) {
+    const int need = forward_launch_count(cfg, targets != nullptr, loss != nullptr, logits != nullptr);
+    trace->count = need;
+    if (!trace->events || trace->capacity < need) return NC_ERR_INVALID_ARG;
+    for (int i = 0; i < 2 * need; ++i)
+      if (!trace->events[i]) return NC_ERR_INVALID_ARG;
+  }
+  if (nc_status s = device_ok()) return s;
+
+  cudaStream_t st = S(stream);
+  Tracer tr{trace, st, 0, false};
+#define NC_RUN(kind, call)                          \
+  do {                                              \
+    if (!tr.begin(kind)) return NC_ERR_CUDA;        \
+    nc_status s_ = (call);                          \
+    if (s_ != NC_OK) return s_;                     \
+    if (!tr.end()) return NC_ERR_CUDA;              \
+  } while (0)
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  uint32_t* status = reinterpret_cast<uint32_t*>(ws + L.status);
+  float* rope = reinterpret_cast<float*>(ws + L.rope);
+  uint16_t* wqkv = reinterpret_cast<uint16_t*>(ws + L.wqkv);
+  uint16_t* wo = reinterpret_cast<uint16_t*>(ws + L.wo);
+  uint16_t* wfc = reinterpret_cast<uint16_t*>(ws + L.wfc);
+  uint16_t* wmp = reinterpret_cast<uint16_t*>(ws + L.wmp);
+  uint16_t* wlm = reinterpret_cast<uint16_t*>(ws + L.wlm);
+  float* x = reinterpret_cast<float*>(ws + L.x);
+  uint16_t* a = reinterpret_cast<uint16_t*>(ws + L.a);
+  uint16_t* qkv = reinterpret_cast<uint16_t*>(ws + L.qkv);
+  uint16_t* o = reinterpret_cast<uint16_t*>(ws + L.o);
+  uint16_t* h = reinterpret_cast<uint16_t*>(ws + L.h);
+  float* part = reinterpret_cast<float*>(ws + L.part);
+  float* tgt = reinterpret_cast<float*>(ws + L.tgt);
+  float* tl = token_loss ? token_loss : reinterpret_cast<float*>(ws + L.tl);
+
+  const int M = B * T;
+  const int C = cfg->d_model, D = cfg->head_dim, H = cfg->n_head, Hkv = cfg->n_kv_head,
+            V = cfg->vocab;
+  const int NQKV = (H + 2 * Hkv) * D;
+
+  if (cudaMemsetAsync(status, 0, 256, st) != cudaSuccess) return NC_ERR_CUDA;
+  NC_RUN(NC_K_ROPE_TABLE, rope_table_launch(rope, T, D, cfg->rope_base, st));
+
+  // fp32 -> bf16 weight cast; c_q|c_k|c_v rows packed into one matrix per layer.
+  {
+    std::vector<CastSeg> segs;
+    segs.reserve(cfg->n_layer * 6 + 1);
+    const size_t nq = (size_t)H * D * C, nk = (size_t)Hkv * D * C;
+    for (int l = 0; l < cfg->n_layer; ++l) {
+      uint16_t* dq = wqkv + l * L.wqkv_elems;
+      segs.push_back({w->c_q[l], dq, (int64_t)nq});
+      segs.push_back({w->c_k[l], dq + nq, (int64_t)nk});
+      segs.push_back({w->c_v[l], dq + nq + nk, (int64_t)nk});
+      segs.push_back({w->attn_proj[l], wo + l * L.wo_elems, (int64_t)L.wo_elems});
+      segs.push_back({w->c_fc[l], wfc + l * L.wfc_elems, (int64_t)L.wfc_elems});
+      segs.push_back({w->mlp_proj[l], wmp + l * L.wmp_elems, (int64_t)L.wmp_elems});
+    }
+    segs.push_back({w->lm_head, wlm, (int64_t)V * C});
+    NC_RUN(NC_K_CAST, cast_launch(segs.data(), (int)segs.size(), st));
+  }
+
+  NC_RUN(NC_K_EMBEDDING, embedding_launch(tokens, w->wte, x, M, C, V, status, st));
+
+  for (int l = 0; l < cfg->n_layer; ++l) {
+    const int W = nc_layer_window(cfg, l);
+    EpiParams ep{};
+    NC_RUN(NC_K_RMSNORM, rmsnorm_launch(x, a, M, C, cfg->norm_eps, st));
+    ep.out = qkv;
+    ep.ldo = NQKV;
+    NC_RUN(NC_K_GEMM_QKV,
+           gemm_launch(a, C, wqkv + l * L.wqkv_elems, C, M, NQKV, C, EPI_STORE_BF16, ep, status, st));
+    NC_RUN(NC_K_ROPE_QKNORM, rope_qknorm_launch(qkv, qkv + H * D, rope, B, T, H, Hkv, D, NQKV, NQKV,
+                                                cfg->norm_eps, st));
+    NC_RUN(NC_K_ATTENTION, attention_launch(qkv, qkv + H * D, qkv + (H + Hkv) * D, o, B, T, H, Hkv,
+                                            D, W, NQKV, NQKV, st));
+    ep.out = x;
+    ep.ldo = C;
+    NC_RUN(NC_K_GEMM_ATTN_PROJ, gemm_launch(o, H * D, wo + l * L.wo_elems, H * D, M, C, H * D,
+                                            EPI_RESID_F32, ep, status, st));
+    NC_RUN(NC_K_RMSNORM, rmsnorm_launch(x, a, M, C, cfg->norm_eps, st));
+    ep.out = h;
+    ep.ldo = 4 * C;
+    NC_RUN(NC_K_GEMM_FC,
+           gemm_launch(a, C, wfc + l * L.wfc_elems, C, M, 4 * C, C, EPI_RELU2_BF16, ep, status, st));
+    ep.out = x;
+    ep.ldo = C;
+    NC_RUN(NC_K_GEMM_MLP_PROJ, gemm_launch(h, 4 * C, wmp + l * L.wmp_elems, 4 * C, M, C, 4 * C,
+                                           EPI_RESID_F32, ep, status, st));
+  }
+
+  NC_RUN(NC_K_RMSNORM, rmsnorm_launch(x, a, M, C, cfg->norm_eps, st));
+  if (targets) {
+    EpiParams ep{};
+    ep.out = logits;
+    ep.ldo = V;
+    ep.cap = cfg->softcap;
+    ep.store_logits = logits != nullptr;
+    ep.ce_partial = part;
+    ep.ce_target = tgt;
+    ep.targets = targets;
+    NC_RUN(NC_K_GEMM_LM_HEAD, gemm_launch(a, C, wlm, C, M, V, C, EPI_CE_PARTIAL, ep, status, st));
+    NC_RUN(NC_K_CE_FINALIZE, ce_finalize_launch(part, gemm_num_n_tiles(V), tgt, targets, tl, M, V,
+                                                cfg->softcap, status, st));
+    if (loss) NC_RUN(NC_K_LOSS_MEAN, loss_mean_launch(tl, targets, M, V, loss, st));
+  } else if (logits) {
+    EpiParams ep{};
+    ep.out = logits;
+    ep.ldo = V;
+    ep.cap = cfg->softcap;
+    NC_RUN(NC_K_GEMM_LM_HEAD, gemm_launch(a, C, wlm, C, M, V, C, EPI_SOFTCAP_F32, ep, status, st));
+  }
+#undef NC_RUN
+  return NC_OK;
+}
+
+nc_status nc_forward(const nc_config* cfg, const nc_weights* w, const int32_t* tokens,
+                     const int32_t* targets, int B, int T, float* logits, float* token_loss,
+                     float* loss, void* workspace, size_t ws_bytes, void* stream) {
+  return nc_forward_traced(cfg, w, tokens, targets, B, T, logits, token_loss, loss, workspace,
+                           ws_bytes, stream, nullptr);
+}
+
+nc_status nc_selftest_bounded_wait(uint32_t* dev_status, uint32_t limit_us, void* stream) {
+  if (!dev_status || limit_us < 1 || limit_us > 2000000u) return NC_ERR_INVALID_ARG;
+  if (nc_status s = device_ok()) return s;
+  return selftest_wait_launch(dev_status, (uint64_t)limit_us * 1000ull, S(stream));
+}
+
+nc_status nc_event_create(void** event) {
+  if (!event) return NC_ERR_INVALID_ARG;
+  cudaEvent_t e;
+  if (cudaEventCreate(&e) != cudaSuccess) return NC_ERR_CUDA;
+  *event = e;
+  return NC_OK;
+}
+
+nc_status nc_event_destroy(void* event) {
+  if (!event) return NC_ERR_INVALID_ARG;
+  return cudaEventDestroy(static_cast<cudaEvent_t>(event)) == cudaSuccess ? NC_OK : NC_ERR_CUDA;
+}
+
+nc_status nc_event_elapsed_ms(void* start, void* end, float* ms) {
+  if (!start || !end || !ms) return NC_ERR_INVALID_ARG;
+  if (cudaEventSynchronize(static_cast<cudaEvent_t>(end)) != cudaSuccess) return NC_ERR_CUDA;
+  return cudaEventElapsedTime(ms, static_cast<cudaEvent_t>(start), static_cast<cudaEvent_t>(end)) ==
+                 cudaSuccess
+             ? NC_OK
+             : NC_ERR_CUDA;
+}
+
+}  // extern "C"

@@ -1,0 +1,77 @@
+// Declarations shared by the translation units of the library (not part of
+// the public ABI, which is include/nc.h).
+#pragma once
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "nc.h"
+
+namespace nc {
+
+// Default bound of every in-kernel wait: two seconds of wall time.
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
+
+// Epilogue selectors of the GEMM (the first five equal nc_epilogue).
+enum : int {
+  EPI_STORE_BF16 = NC_EPI_STORE_BF16,
+  EPI_RELU2_BF16 = NC_EPI_RELU2_BF16,
+  EPI_RESID_F32 = NC_EPI_RESID_F32,
+  EPI_STORE_F32 = NC_EPI_STORE_F32,
+  EPI_SOFTCAP_F32 = NC_EPI_SOFTCAP_F32,
+  EPI_CE_PARTIAL = 5,  // soft-cap, per-tile sum of exp(l - cap), target logit
+};
+
+struct EpiParams {
+  void* out;                // bf16 or fp32 output (or logits for EPI_CE_PARTIAL)
+  int64_t ldo;              // output row stride in elements
+  float cap;                // soft-cap
+  int store_logits;         // EPI_CE_PARTIAL: also write capped logits to out
+  float* ce_partial;        // EPI_CE_PARTIAL: [M, gemm_num_n_tiles(N)]
+  float* ce_target;         // EPI_CE_PARTIAL: [M], l[m, y_m] (written by one tile)
+  const int32_t* targets;   // EPI_CE_PARTIAL: [M]
+};
+
+// ---- device / argument helpers (nc_api.cu)
+int device_sm_count();
+bool device_is_sm100();
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// ---- GEMM (nc_gemm.cu)
+int gemm_num_n_tiles(int N);
+nc_status gemm_launch(const uint16_t* a, int64_t lda, const uint16_t* w, int64_t ldw, int M, int N,
+                      int K, int epi, const EpiParams& ep, uint32_t* dev_status,
+                      cudaStream_t stream, uint64_t limit_ns = kWaitLimitNs);
+
+nc_status selftest_wait_launch(uint32_t* dev_status, uint64_t limit_ns, cudaStream_t stream);
+
+// ---- attention (nc_attention.cu)
+nc_status attention_launch(const uint16_t* q, const uint16_t* k, const uint16_t* v, uint16_t* out,
+                           int B, int T, int H, int Hkv, int D, int window, int64_t q_stride,
+                           int64_t kv_stride, cudaStream_t stream);
+
+// ---- elementwise / row kernels (nc_rowops.cu)
+struct CastSeg {
+  const float* src;
+  uint16_t* dst;
+  int64_t n;  // multiple of 8
+};
+nc_status cast_launch(const CastSeg* segs, int nseg, cudaStream_t stream);
+nc_status embedding_launch(const int32_t* tokens, const float* wte, float* x, int M, int C, int V,
+                           uint32_t* dev_status, cudaStream_t stream);
+nc_status rmsnorm_launch(const float* x, uint16_t* out, int M, int C, float eps,
+                         cudaStream_t stream);
+nc_status rope_table_launch(float* table, int T, int D, float base, cudaStream_t stream);
+nc_status rope_qknorm_launch(uint16_t* q, uint16_t* k, const float* table, int B, int T, int H,
+                             int Hkv, int D, int64_t q_stride, int64_t k_stride, float eps,
+                             cudaStream_t stream);
+nc_status softcap_ce_launch(const float* z, const int32_t* targets, float* capped_out,
+                            float* token_loss, int M, int V, float cap, uint32_t* dev_status,
+                            cudaStream_t stream);
+nc_status ce_finalize_launch(const float* partial, int n_tiles, const float* target_logit,
+                             const int32_t* targets, float* token_loss, int M, int V, float cap,
+                             uint32_t* dev_status, cudaStream_t stream);
+nc_status loss_mean_launch(const float* token_loss, const int32_t* targets, int M, int V,
+                           float* loss, cudaStream_t stream);
+
+}  // namespace nc

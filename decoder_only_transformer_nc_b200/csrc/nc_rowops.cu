@@ -1,0 +1,409 @@
+// Bandwidth-bound steps of the forward: weight cast, embedding gather,
+// parameter-free RMSNorm, RoPE table, fused RoPE + QK-norm, fused soft-cap +
+// log-softmax + NLL, and the loss reductions.  Each kernel reads and writes
+// every byte once with 8- or 16-byte coalesced accesses; reductions are warp
+// shuffles in a fixed order, so results are run-to-run deterministic.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+
+#include "nc_internal.h"
+
+namespace nc {
+namespace {
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+__device__ __forceinline__ float2 unpack_bf16x2(uint32_t u) {
+  __nv_bfloat162 h = *reinterpret_cast<__nv_bfloat162*>(&u);
+  return __bfloat1622float2(h);
+}
+
+// ---------------------------------------------------------------- weight cast
+
+constexpr int kMaxCastSegs = 48;
+struct CastBatch {
+  const float* src[kMaxCastSegs];
+  uint16_t* dst[kMaxCastSegs];
+  int64_t gstart[kMaxCastSegs + 1];  // prefix sums in groups of 8 elements
+  int nseg;
+};
+
+__global__ void __launch_bounds__(256) cast_kernel(const __grid_constant__ CastBatch cb) {
+  const int64_t total = cb.gstart[cb.nseg];
+  for (int64_t g = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; g < total;
+       g += (int64_t)gridDim.x * blockDim.x) {
+    int lo = 0, hi = cb.nseg - 1;  // last segment with gstart <= g
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (cb.gstart[mid] <= g) lo = mid; else hi = mid - 1;
+    }
+    const int64_t off = (g - cb.gstart[lo]) * 8;
+    const float4* s = reinterpret_cast<const float4*>(cb.src[lo] + off);
+    const float4 a = __ldcs(s);
+    const float4 b = __ldcs(s + 1);
+    uint4 o;
+    o.x = pack_bf16x2(a.x, a.y);
+    o.y = pack_bf16x2(a.z, a.w);
+    o.z = pack_bf16x2(b.x, b.y);
+    o.w = pack_bf16x2(b.z, b.w);
+    *reinterpret_cast<uint4*>(cb.dst[lo] + off) = o;
+  }
+}
+
+// ---------------------------------------------------------------- embedding
+
+__global__ void __launch_bounds__(256) embedding_kernel(const int32_t* __restrict__ tokens,
+                                                        const float* __restrict__ wte,
+                                                        float* __restrict__ x, int M, int C, int V,
+                                                        uint32_t* dev_status) {
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (warp >= M) return;
+  int tok = tokens[warp];
+  if (tok < 0 || tok >= V) {
+    if (lane == 0 && dev_status) atomicOr(dev_status, NC_DEV_TOKEN_RANGE);
+    tok = 0;
+  }
+  const float4* src = reinterpret_cast<const float4*>(wte + (int64_t)tok * C);
+  float4* dst = reinterpret_cast<float4*>(x + (int64_t)warp * C);
+  for (int i = lane; i < C / 4; i += 32) dst[i] = src[i];
+}
+
+// ---------------------------------------------------------------- RMSNorm
+
+// One warp per row; the row is held in registers (C <= 32 * 4 * NV).
+template <int NV>
+__global__ void __launch_bounds__(256) rmsnorm_kernel(const float* __restrict__ x,
+                                                      uint16_t* __restrict__ out, int M, int C,
+                                                      float eps) {
+  const int row = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (row >= M) return;
+  const float4* xr = reinterpret_cast<const float4*>(x + (int64_t)row * C);
+  const int n4 = C >> 2;
+  float4 v[NV];
+  float ss = 0.0f;
+#pragma unroll
+  for (int j = 0; j < NV; ++j) {
+    const int i = j * 32 + lane;
+    v[j] = i < n4 ? xr[i] : make_float4(0.f, 0.f, 0.f, 0.f);
+    ss += v[j].x * v[j].x + v[j].y * v[j].y + v[j].z * v[j].z + v[j].w * v[j].w;
+  }
+  ss = warp_sum(ss);
+  const float r = rsqrtf(ss / (float)C + eps);
+  uint2* o = reinterpret_cast<uint2*>(out + (int64_t)row * C);
+#pragma unroll
+  for (int j = 0; j < NV; ++j) {
+    const int i = j * 32 + lane;
+    if (i < n4) o[i] = make_uint2(pack_bf16x2(v[j].x * r, v[j].y * r), pack_bf16x2(v[j].z * r, v[j].w * r));
+  }
+}
+
+// Two-pass variant for wide rows.
+__global__ void __launch_bounds__(256) rmsnorm_wide_kernel(const float* __restrict__ x,
+                                                           uint16_t* __restrict__ out, int M, int C,
+                                                           float eps) {
+  const int row = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (row >= M) return;
+  const float4* xr = reinterpret_cast<const float4*>(x + (int64_t)row * C);
+  const int n4 = C >> 2;
+  float ss = 0.0f;
+  for (int i = lane; i < n4; i += 32) {
+    const float4 a = xr[i];
+    ss += a.x * a.x + a.y * a.y + a.z * a.z + a.w * a.w;
+  }
+  ss = warp_sum(ss);
+  const float r = rsqrtf(ss / (float)C + eps);
+  uint2* o = reinterpret_cast<uint2*>(out + (int64_t)row * C);
+  for (int i = lane; i < n4; i += 32) {
+    const float4 a = xr[i];
+    o[i] = make_uint2(pack_bf16x2(a.x * r, a.y * r), pack_bf16x2(a.z * r, a.w * r));
+  }
+}
+
+// ---------------------------------------------------------------- RoPE
+
+__global__ void rope_table_kernel(float* __restrict__ table, int T, int D, double base) {
+  const int half = D / 2;
+  const int idx = blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= T * half) return;
+  const int t = idx / half;
+  const int i = idx - t * half;
+  const double theta = pow(base, -2.0 * (double)i / (double)D);
+  const double ang = (double)t * theta;
+  table[idx] = (float)cos(ang);
+  table[(int64_t)T * half + idx] = (float)sin(ang);
+}
+
+// One group of D/4 lanes per (token, head).  Lane l of the group holds the
+// bf16 pairs at dims (2l, 2l+1) and (D/2+2l, D/2+2l+1), i.e. both members of
+// the RoPE pairs 2l and 2l+1, so the rotation needs no shuffles; the per-head
+// sum of squares is a shuffle reduction inside the group.
+template <int D>
+__global__ void __launch_bounds__(256) rope_qknorm_kernel(uint16_t* __restrict__ q,
+                                                          uint16_t* __restrict__ k,
+                                                          const float* __restrict__ table, int M,
+                                                          int T, int H, int Hkv, int64_t q_stride,
+                                                          int64_t k_stride, float eps) {
+  constexpr int LPH = D / 4;  // lanes per head
+  constexpr int HALF = D / 2;
+  const int64_t gid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const int64_t unit = gid / LPH;  // (token, head) index
+  const int l = (int)(gid % LPH);
+  const int heads = H + Hkv;
+  const bool active = unit < (int64_t)M * heads;
+  const int64_t m = active ? unit / heads : 0;
+  const int j = active ? (int)(unit - m * heads) : 0;
+  const int t = (int)(m % T);
+  uint16_t* p = j < H ? q + m * q_stride + (int64_t)j * D : k + m * k_stride + (int64_t)(j - H) * D;
+  float ra0 = 0.f, ra1 = 0.f, rb0 = 0.f, rb1 = 0.f;
+  if (active) {
+    const float2 a = unpack_bf16x2(*reinterpret_cast<const uint32_t*>(p + 2 * l));
+    const float2 b = unpack_bf16x2(*reinterpret_cast<const uint32_t*>(p + HALF + 2 * l));
+    const float2 c = *reinterpret_cast<const float2*>(table + (int64_t)t * HALF + 2 * l);
+    const float2 s = *reinterpret_cast<const float2*>(table + (int64_t)T * HALF + (int64_t)t * HALF + 2 * l);
+    ra0 = a.x * c.x - b.x * s.x;
+    rb0 = a.x * s.x + b.x * c.x;
+    ra1 = a.y * c.y - b.y * s.y;
+    rb1 = a.y * s.y + b.y * c.y;
+  }
+  float ss = ra0 * ra0 + ra1 * ra1 + rb0 * rb0 + rb1 * rb1;
+#pragma unroll
+  for (int o = LPH / 2; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+  if (active) {
+    const float r = rsqrtf(ss / (float)D + eps);
+    *reinterpret_cast<uint32_t*>(p + 2 * l) = pack_bf16x2(ra0 * r, ra1 * r);
+    *reinterpret_cast<uint32_t*>(p + HALF + 2 * l) = pack_bf16x2(rb0 * r, rb1 * r);
+  }
+}
+
+// ---------------------------------------------------------------- cross-entropy
+
+// Block-wide sum in a fixed order (warp shuffles, then warp 0 over the partials).
+__device__ __forceinline__ float block_sum(float v, float* red) {
+  v = warp_sum(v);
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (lane == 0) red[w] = v;
+  __syncthreads();
+  if (w == 0) {
+    float t = lane < (int)(blockDim.x >> 5) ? red[lane] : 0.0f;
+    t = warp_sum(t);
+    if (lane == 0) red[32] = t;
+  }
+  __syncthreads();
+  const float r = red[32];
+  __syncthreads();
+  return r;
+}
+
+// One CTA per row.  Soft-capped logits lie in (-cap, cap), so
+// logsumexp(l) = cap + log(sum exp(l - cap)) needs no running maximum.
+__global__ void __launch_bounds__(256) softcap_ce_kernel(const float* __restrict__ z,
+                                                         const int32_t* __restrict__ targets,
+                                                         float* capped_out,
+                                                         float* __restrict__ token_loss, int V,
+                                                         float cap, uint32_t* dev_status) {
+  __shared__ float red[33];
+  const int64_t row = blockIdx.x;
+  const float4* zr = reinterpret_cast<const float4*>(z + row * V);
+  float4* cr = capped_out ? reinterpret_cast<float4*>(capped_out + row * V) : nullptr;
+  const float inv = 1.0f / cap;
+  float s = 0.0f;
+  for (int i = threadIdx.x; i < V / 4; i += blockDim.x) {
+    float4 a = __ldcs(zr + i);
+    a.x = cap * tanhf(a.x * inv);
+    a.y = cap * tanhf(a.y * inv);
+    a.z = cap * tanhf(a.z * inv);
+    a.w = cap * tanhf(a.w * inv);
+    s += __expf(a.x - cap) + __expf(a.y - cap) + __expf(a.z - cap) + __expf(a.w - cap);
+    if (cr) cr[i] = a;
+  }
+  s = block_sum(s, red);
+  if (threadIdx.x == 0) {
+    const int y = targets[row];
+    float nll = 0.0f;
+    if (y >= 0 && y < V) {
+      const float ly = cap * tanhf(z[row * V + y] * inv);
+      nll = cap + logf(s) - ly;
+    } else if (y != -1 && dev_status) {
+      atomicOr(dev_status, NC_DEV_TARGET_RANGE);
+    }
+    token_loss[row] = nll;
+  }
+}
+
+// Combines the per-tile partial sums written by the lm_head GEMM epilogue:
+// one warp per row, fixed summation order.
+__global__ void __launch_bounds__(256) ce_finalize_kernel(const float* __restrict__ partial,
+                                                          int n_tiles,
+                                                          const float* __restrict__ target_logit,
+                                                          const int32_t* __restrict__ targets,
+                                                          float* __restrict__ token_loss, int M,
+                                                          int V, float cap, uint32_t* dev_status) {
+  const int row = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (row >= M) return;
+  const float* pr = partial + (int64_t)row * n_tiles;
+  float s = 0.0f;
+  for (int i = lane; i < n_tiles; i += 32) s += pr[i];
+  s = warp_sum(s);
+  if (lane == 0) {
+    const int y = targets[row];
+    float nll = 0.0f;
+    if (y >= 0 && y < V) {
+      nll = cap + logf(s) - target_logit[row];
+    } else if (y != -1 && dev_status) {
+      atomicOr(dev_status, NC_DEV_TARGET_RANGE);
+    }
+    token_loss[row] = nll;
+  }
+}
+
+// Single CTA, fixed-order reduction in fp64: mean over valid targets.
+__global__ void __launch_bounds__(1024) loss_mean_kernel(const float* __restrict__ token_loss,
+                                                         const int32_t* __restrict__ targets, int M,
+                                                         int V, float* loss) {
+  __shared__ double rs[32];
+  __shared__ int rc[32];
+  double s = 0.0;
+  int c = 0;
+  for (int i = threadIdx.x; i < M; i += blockDim.x) {
+    const int y = targets[i];
+    if (y >= 0 && y < V) {
+      s += (double)token_loss[i];
+      ++c;
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    s += __shfl_xor_sync(0xffffffffu, s, o);
+    c += __shfl_xor_sync(0xffffffffu, c, o);
+  }
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (lane == 0) {
+    rs[w] = s;
+    rc[w] = c;
+  }
+  __syncthreads();
+  if (w == 0) {
+    const int nw = blockDim.x >> 5;
+    s = lane < nw ? rs[lane] : 0.0;
+    c = lane < nw ? rc[lane] : 0;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      s += __shfl_xor_sync(0xffffffffu, s, o);
+      c += __shfl_xor_sync(0xffffffffu, c, o);
+    }
+    if (lane == 0) loss[0] = c > 0 ? (float)(s / (double)c) : __int_as_float(0x7fc00000);
+  }
+}
+
+inline nc_status last_error() { return cudaGetLastError() == cudaSuccess ? NC_OK : NC_ERR_CUDA; }
+
+}  // namespace
+
+nc_status cast_launch(const CastSeg* segs, int nseg, cudaStream_t stream) {
+  for (int base = 0; base < nseg; base += kMaxCastSegs) {
+    CastBatch cb;
+    cb.nseg = nseg - base < kMaxCastSegs ? nseg - base : kMaxCastSegs;
+    cb.gstart[0] = 0;
+    for (int i = 0; i < cb.nseg; ++i) {
+      cb.src[i] = segs[base + i].src;
+      cb.dst[i] = segs[base + i].dst;
+      cb.gstart[i + 1] = cb.gstart[i] + segs[base + i].n / 8;
+    }
+    const int64_t groups = cb.gstart[cb.nseg];
+    if (groups == 0) continue;
+    const int64_t want = (groups + 255) / 256;
+    const int grid = (int)(want < 148 * 16 ? want : 148 * 16);
+    cast_kernel<<<grid, 256, 0, stream>>>(cb);
+    if (cudaGetLastError() != cudaSuccess) return NC_ERR_CUDA;
+  }
+  return NC_OK;
+}
+
+nc_status embedding_launch(const int32_t* tokens, const float* wte, float* x, int M, int C, int V,
+                           uint32_t* dev_status, cudaStream_t stream) {
+  if (M == 0) return NC_OK;
+  const int grid = (M + 7) / 8;
+  embedding_kernel<<<grid, 256, 0, stream>>>(tokens, wte, x, M, C, V, dev_status);
+  return last_error();
+}
+
+nc_status rmsnorm_launch(const float* x, uint16_t* out, int M, int C, float eps,
+                         cudaStream_t stream) {
+  if (M == 0) return NC_OK;
+  const int grid = (M + 7) / 8;
+  if (C <= 32 * 4 * 4)
+    rmsnorm_kernel<4><<<grid, 256, 0, stream>>>(x, out, M, C, eps);
+  else if (C <= 32 * 4 * 8)
+    rmsnorm_kernel<8><<<grid, 256, 0, stream>>>(x, out, M, C, eps);
+  else if (C <= 32 * 4 * 16)
+    rmsnorm_kernel<16><<<grid, 256, 0, stream>>>(x, out, M, C, eps);
+  else
+    rmsnorm_wide_kernel<<<grid, 256, 0, stream>>>(x, out, M, C, eps);
+  return last_error();
+}
+
+nc_status rope_table_launch(float* table, int T, int D, float base, cudaStream_t stream) {
+  const int n = T * (D / 2);
+  if (n == 0) return NC_OK;
+  rope_table_kernel<<<(n + 255) / 256, 256, 0, stream>>>(table, T, D, (double)base);
+  return last_error();
+}
+
+nc_status rope_qknorm_launch(uint16_t* q, uint16_t* k, const float* table, int B, int T, int H,
+                             int Hkv, int D, int64_t q_stride, int64_t k_stride, float eps,
+                             cudaStream_t stream) {
+  const int64_t M = (int64_t)B * T;
+  const int64_t threads = M * (H + Hkv) * (D / 4);
+  if (threads == 0) return NC_OK;
+  const int64_t grid = (threads + 255) / 256;
+  if (D == 128)
+    rope_qknorm_kernel<128><<<(unsigned)grid, 256, 0, stream>>>(q, k, table, (int)M, T, H, Hkv,
+                                                                q_stride, k_stride, eps);
+  else if (D == 64)
+    rope_qknorm_kernel<64><<<(unsigned)grid, 256, 0, stream>>>(q, k, table, (int)M, T, H, Hkv,
+                                                               q_stride, k_stride, eps);
+  else
+    return NC_ERR_SHAPE;
+  return last_error();
+}
+
+nc_status softcap_ce_launch(const float* z, const int32_t* targets, float* capped_out,
+                            float* token_loss, int M, int V, float cap, uint32_t* dev_status,
+                            cudaStream_t stream) {
+  if (M == 0) return NC_OK;
+  softcap_ce_kernel<<<M, 256, 0, stream>>>(z, targets, capped_out, token_loss, V, cap, dev_status);
+  return last_error();
+}
+
+nc_status ce_finalize_launch(const float* partial, int n_tiles, const float* target_logit,
+                             const int32_t* targets, float* token_loss, int M, int V, float cap,
+                             uint32_t* dev_status, cudaStream_t stream) {
+  if (M == 0) return NC_OK;
+  ce_finalize_kernel<<<(M + 7) / 8, 256, 0, stream>>>(partial, n_tiles, target_logit, targets,
+                                                      token_loss, M, V, cap, dev_status);
+  return last_error();
+}
+
+nc_status loss_mean_launch(const float* token_loss, const int32_t* targets, int M, int V,
+                           float* loss, cudaStream_t stream) {
+  loss_mean_kernel<<<1, 1024, 0, stream>>>(token_loss, targets, M, V, loss);
+  return last_error();
+}
+
+}  // namespace nc

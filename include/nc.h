@@ -1,0 +1,280 @@
+/*
+ * nc.h -- C ABI of the B200 (sm_100a) forward pass + loss of the nanochat GPT
+ * block stack.
+ *
+ * What is computed (page title, section):
+ *   "从文本到聊天模型" (onehacker.top) §5: token embedding (§5.2), blocks
+ *   x = x + attn(norm(x)); x = x + mlp(norm(x)) (§5.3), separate c_q/c_k/c_v
+ *   projections with Q (B,T,H,D) and K/V (B,T,Hkv,D) (§5.4), causal attention
+ *   (§5.5), RoPE (§5.6), ReLU^2 MLP C -> 4C -> C (§5.7), LM head and token
+ *   cross-entropy with ignore_index = -1 (§5.8);
+ *   "Nanochat与nanoGPT对比：关键升级" (lzwjava.github.io) §1: parameter-free
+ *   RMSNorm, QK-norm after RoPE, GQA, no biases, untied lm_head, tanh logit
+ *   soft-cap at +-15, SSSL sliding window (last layer full), final norm before
+ *   the logit projection;
+ *   nanochat README mirror (dev.wehub.plus), "精度 / dtype": weights are kept
+ *   in fp32 and cast to bf16 at matmul time.
+ *
+ * Conventions for every entry point:
+ *   - All tensor pointers are DEVICE pointers of the current CUDA device unless
+ *     a parameter says "host".  The caller owns every buffer; the library
+ *     allocates no device memory and frees nothing.
+ *   - bf16 tensors are passed as uint16_t* holding bfloat16 bit patterns.
+ *   - Matrices are row-major.  Weights use the [out_features, in_features]
+ *     layout of a bias-free linear layer, so y = x W^T.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Work is
+ *     enqueued asynchronously; results are valid once the stream has synchronised.
+ *   - Arguments are checked on the host before anything is enqueued; a failed
+ *     check returns an error code and enqueues nothing.  Nothing aborts, traps
+ *     or prints.
+ *   - Device-detected conditions (a token id outside [0, V), a target outside
+ *     {-1} U [0, V), a bounded wait inside a kernel that ran out) are OR-ed into
+ *     a caller-provided 32-bit device status word as NC_DEV_* bits; kernels
+ *     clamp indices so that no out-of-bounds access happens.  Pass NULL to
+ *     ignore them.  nc_get_status() turns a status word into an nc_status.
+ *   - Pointers must be 16-byte aligned (NC_ERR_ALIGNMENT otherwise).
+ *   - Every entry point requires an sm_100 device (NC_ERR_UNSUPPORTED_DEVICE).
+ */
+#ifndef NC_H_
+#define NC_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  NC_OK = 0,
+  NC_ERR_INVALID_ARG = 1,        /* NULL pointer, negative size, bad enum */
+  NC_ERR_CONFIG = 2,             /* inconsistent nc_config                   */
+  NC_ERR_SHAPE = 3,              /* sizes the kernels do not support         */
+  NC_ERR_ALIGNMENT = 4,          /* a pointer is not 16-byte aligned         */
+  NC_ERR_WORKSPACE = 5,          /* workspace smaller than nc_workspace_bytes */
+  NC_ERR_TOKEN_RANGE = 6,        /* device: token or target id out of range  */
+  NC_ERR_TIMEOUT = 7,            /* device: a bounded wait in a kernel ran out */
+  NC_ERR_UNSUPPORTED_DEVICE = 8, /* current device is not sm_100             */
+  NC_ERR_CUDA = 9                /* a CUDA runtime call failed               */
+} nc_status;
+
+/* Bits of the device status word. */
+#define NC_DEV_TOKEN_RANGE 0x1u  /* a token id was outside [0, V): row 0 used  */
+#define NC_DEV_TARGET_RANGE 0x2u /* a target was outside {-1} U [0, V): ignored */
+#define NC_DEV_TIMEOUT 0x4u      /* a pipeline wait gave up; outputs invalid   */
+
+/* Model configuration.  "从文本到聊天模型" §5.1: d_model = depth * aspect_ratio,
+ * n_head = d_model / head_dim.  window_pattern: one char per layer, cycled;
+ * 'S' = short window (short_window keys), 'L' = full context; the last layer is
+ * always 'L' ("Nanochat与nanoGPT对比" §1, sliding-window note). */
+typedef struct {
+  int32_t n_layer;
+  int32_t d_model;
+  int32_t n_head;
+  int32_t n_kv_head;         /* n_head % n_kv_head == 0 (GQA groups)          */
+  int32_t head_dim;          /* 64 or 128                                     */
+  int32_t vocab;             /* multiple of 64                                */
+  int32_t seq_len;           /* maximum T                                     */
+  int32_t short_window;      /* keys visible in 'S' layers (seq_len / 4)      */
+  char window_pattern[8];    /* NUL-terminated, e.g. "SSSL"                   */
+  float softcap;             /* logits = softcap * tanh(z / softcap), 15      */
+  float norm_eps;            /* RMSNorm epsilon, 1e-6                         */
+  float rope_base;           /* RoPE base, 10000                              */
+} nc_config;
+
+/* fp32 master weights (device pointers; the per-layer members are HOST arrays
+ * of n_layer device pointers).  Read only. */
+typedef struct {
+  const float* wte;                  /* [V, C]                                */
+  const float* const* c_q;           /* n_layer x [H*D, C]                    */
+  const float* const* c_k;           /* n_layer x [Hkv*D, C]                  */
+  const float* const* c_v;           /* n_layer x [Hkv*D, C]                  */
+  const float* const* attn_proj;     /* n_layer x [C, H*D]                    */
+  const float* const* c_fc;          /* n_layer x [4C, C]                     */
+  const float* const* mlp_proj;      /* n_layer x [C, 4C]                     */
+  const float* lm_head;              /* [V, C]                                */
+} nc_weights;
+
+/* ---------------------------------------------------------------- host-only */
+
+/* Fills *out from the depth knob ("从文本到聊天模型" §5.1): d_model =
+ * depth*aspect_ratio, n_head = d_model/head_dim, n_kv_head = n_kv_head or
+ * n_head when 0, pattern "SSSL", short_window = seq_len/4, softcap 15,
+ * norm_eps 1e-6, rope_base 10000.  Host only; touches no device. */
+nc_status nc_init_config(nc_config* out, int depth, int aspect_ratio, int head_dim,
+                         int n_kv_head, int seq_len, int vocab);
+
+/* Checks a configuration (NC_OK or NC_ERR_CONFIG).  Host only. */
+nc_status nc_check_config(const nc_config* cfg);
+
+/* Number of keys layer `layer` lets each query see (short_window or seq_len),
+ * or -1 for a bad argument.  Host only. */
+int nc_layer_window(const nc_config* cfg, int layer);
+
+/* Bytes of workspace nc_forward needs for a [B, T] batch (0 on bad input).
+ * Host only. */
+size_t nc_workspace_bytes(const nc_config* cfg, int B, int T);
+
+/* Algorithmic FLOPs of one forward over [B, T] tokens: 2 per multiply-add of
+ * every projection and of attention counted only over visible keys.  Host only. */
+double nc_forward_flops(const nc_config* cfg, int B, int T);
+
+/* Human-readable name of a status code (static string). */
+const char* nc_status_string(nc_status s);
+
+/* Library ABI version (major*100 + minor). */
+int nc_version(void);
+
+/* ---------------------------------------------------------------- forward */
+
+/* Whole forward + loss.
+ *   tokens   [B, T] int32 (device), ids in [0, V).
+ *   targets  [B, T] int32 (device) or NULL; -1 = ignored position.
+ *   logits   [B, T, V] fp32 (device) or NULL: soft-capped logits.
+ *   token_loss [B, T] fp32 (device) or NULL: NLL per position, 0 where ignored.
+ *   loss     1 fp32 (device) or NULL: mean NLL over non-ignored targets (NaN if
+ *            none).  token_loss/loss need targets.
+ *   workspace/ws_bytes: device scratch of at least nc_workspace_bytes(cfg,B,T)
+ *            bytes, 256-byte aligned.  Its first 4 bytes are the device status
+ *            word of this call (cleared at the start of the call).
+ * T <= seq_len.  Asynchronous on `stream`; poll errors with nc_get_status. */
+nc_status nc_forward(const nc_config* cfg, const nc_weights* w, const int32_t* tokens,
+                     const int32_t* targets, int B, int T, float* logits, float* token_loss,
+                     float* loss, void* workspace, size_t ws_bytes, void* stream);
+
+/* Kinds of kernel launch reported by nc_forward_traced. */
+typedef enum {
+  NC_K_ROPE_TABLE = 0,
+  NC_K_CAST = 1,
+  NC_K_EMBEDDING = 2,
+  NC_K_RMSNORM = 3,
+  NC_K_GEMM_QKV = 4,
+  NC_K_ROPE_QKNORM = 5,
+  NC_K_ATTENTION = 6,
+  NC_K_GEMM_ATTN_PROJ = 7,
+  NC_K_GEMM_FC = 8,
+  NC_K_GEMM_MLP_PROJ = 9,
+  NC_K_GEMM_LM_HEAD = 10,
+  NC_K_CE_FINALIZE = 11,
+  NC_K_LOSS_MEAN = 12,
+  NC_K_COUNT = 13
+} nc_kernel_kind;
+
+/* Per-launch timing hook.  `events` holds 2*capacity cudaEvent_t handles
+ * created by nc_event_create; launch i is bracketed by events[2i] and
+ * events[2i+1] recorded on the forward's stream, and kinds[i] names it.
+ * On return `count` holds the number of launches (NC_ERR_INVALID_ARG, with
+ * nothing enqueued, if capacity is too small: count then says how many are
+ * needed). */
+typedef struct {
+  void* const* events;
+  int32_t capacity;
+  int32_t count;
+  int32_t* kinds; /* host array of capacity entries */
+} nc_trace;
+
+/* nc_forward with a timing hook (trace may be NULL). */
+nc_status nc_forward_traced(const nc_config* cfg, const nc_weights* w, const int32_t* tokens,
+                            const int32_t* targets, int B, int T, float* logits,
+                            float* token_loss, float* loss, void* workspace, size_t ws_bytes,
+                            void* stream, nc_trace* trace);
+
+/* Timing events (thin wrappers of the CUDA runtime; no device memory). */
+nc_status nc_event_create(void** event);
+nc_status nc_event_destroy(void* event);
+/* Milliseconds between two recorded events (waits for `end`). */
+nc_status nc_event_elapsed_ms(void* start, void* end, float* ms);
+
+/* Synchronises `stream` and returns the status recorded in the device status
+ * word at `dev_status` (e.g. the workspace of nc_forward): NC_OK,
+ * NC_ERR_TOKEN_RANGE, NC_ERR_TIMEOUT, or NC_ERR_CUDA for a sticky CUDA error. */
+nc_status nc_get_status(const void* dev_status, void* stream);
+
+/* ---------------------------------------------------------------- single steps */
+
+/* fp32 -> bf16 (round to nearest even) of n elements; n % 8 == 0. */
+nc_status nc_cast_bf16(const float* src, uint16_t* dst, int64_t n, void* stream);
+
+/* x[m, :] = wte[tokens[m], :] for m < M ("从文本到聊天模型" §5.2).
+ * x [M, C] fp32; wte [V, C] fp32.  Bad ids set NC_DEV_TOKEN_RANGE and read row 0. */
+nc_status nc_embedding(const int32_t* tokens, const float* wte, float* x, int M, int C, int V,
+                       uint32_t* dev_status, void* stream);
+
+/* out[m, :] = bf16( x[m, :] / sqrt(mean(x[m, :]^2) + eps) ), parameter-free
+ * RMSNorm ("Nanochat与nanoGPT对比" §1).  x [M, C] fp32, out [M, C] bf16;
+ * C % 8 == 0. */
+nc_status nc_rmsnorm(const float* x, uint16_t* out, int M, int C, float eps, void* stream);
+
+/* RoPE angle table: table[0][t][i] = cos(t * base^(-2i/D)),
+ * table[1][t][i] = sin(...), fp32, t < T, i < D/2 (angles in fp64). */
+nc_status nc_rope_table(float* table, int T, int D, float base, void* stream);
+
+/* In place: q <- rmsnorm(rope(q)), k <- rmsnorm(rope(k)) per head over D
+ * ("从文本到聊天模型" §5.6; "Nanochat与nanoGPT对比" §1: QK-norm after RoPE).
+ * q [B, T, H, D] bf16 with q_row_stride elements between consecutive tokens
+ * (H*D when contiguous); k [B, T, Hkv, D] with k_row_stride.  Pair
+ * (u_i, u_{i+D/2}) of the token at position t is rotated by t * theta_i,
+ * table from nc_rope_table.  D in {64, 128}. */
+nc_status nc_rope_qknorm(uint16_t* q, uint16_t* k, const float* table, int B, int T, int H,
+                         int Hkv, int D, int64_t q_row_stride, int64_t k_row_stride, float eps,
+                         void* stream);
+
+/* Causal sliding-window attention with GQA ("从文本到聊天模型" §5.4-5.5):
+ * out[b,i,h,:] = sum_j softmax_j(q[b,i,h,:].k[b,j,g,:] / sqrt(D)) v[b,j,g,:],
+ * g = h / (H/Hkv), over keys j <= i with i - j < window (window <= 0 or
+ * >= T: full causal).  q/out [B,T,H,D], k/v [B,T,Hkv,D], contiguous bf16.
+ * D == 128. */
+nc_status nc_attention(const uint16_t* q, const uint16_t* k, const uint16_t* v, uint16_t* out,
+                       int B, int T, int H, int Hkv, int D, int window, void* stream);
+
+/* Same with explicit token strides (elements between consecutive tokens) for
+ * q, k, v (e.g. the three column blocks of one fused [M, (H+2Hkv)D] buffer);
+ * out is contiguous [B, T, H, D]. */
+nc_status nc_attention_strided(const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                               uint16_t* out, int B, int T, int H, int Hkv, int D, int window,
+                               int64_t q_row_stride, int64_t kv_row_stride, void* stream);
+
+/* Epilogues of nc_linear. */
+typedef enum {
+  NC_EPI_STORE_BF16 = 0,   /* out bf16 [M, ldo]: acc                             */
+  NC_EPI_RELU2_BF16 = 1,   /* out bf16: relu(acc)^2 ("从文本到聊天模型" §5.7)    */
+  NC_EPI_RESID_F32 = 2,    /* out fp32: out += acc (residual add, §5.3)          */
+  NC_EPI_STORE_F32 = 3,    /* out fp32: acc                                      */
+  NC_EPI_SOFTCAP_F32 = 4   /* out fp32: cap * tanh(acc / cap)                    */
+} nc_epilogue;
+
+/* out = epilogue(a @ w^T): a [M, K] bf16 row-major, w [N, K] bf16 row-major,
+ * out row stride ldo elements (>= N).  tcgen05 tensor cores, fp32 accumulation
+ * in tensor memory.  K % 8 == 0, N % 32 == 0.  dev_status gets NC_DEV_TIMEOUT
+ * if a pipeline wait ran out. */
+nc_status nc_linear(const uint16_t* a, const uint16_t* w, void* out, int M, int N, int K,
+                    int64_t ldo, nc_epilogue epilogue, float cap, uint32_t* dev_status,
+                    void* stream);
+
+/* Fused soft-cap + log-softmax + NLL over the vocabulary ("Nanochat与nanoGPT对比"
+ * §1 soft-cap; "从文本到聊天模型" §5.8 cross-entropy, ignore_index -1):
+ *   l = cap * tanh(z / cap);  token_loss[m] = logsumexp(l[m, :]) - l[m, y_m]
+ *   (0 where y_m == -1).  z [M, V] raw fp32 logits; capped_out [M, V] fp32 or
+ *   NULL (may equal z); token_loss [M] fp32.  Bad targets set
+ *   NC_DEV_TARGET_RANGE and count as ignored. */
+nc_status nc_softcap_ce(const float* z, const int32_t* targets, float* capped_out,
+                        float* token_loss, int M, int V, float cap, uint32_t* dev_status,
+                        void* stream);
+
+/* loss[0] = sum(token_loss[m] over targets[m] != -1 and in range) / count,
+ * NaN if the count is 0; fixed-order (run-to-run deterministic) reduction. */
+nc_status nc_loss_mean(const float* token_loss, const int32_t* targets, int M, int V,
+                       float* loss, void* stream);
+
+/* Self-test of the failure path of in-kernel waits: one CTA waits on an
+ * mbarrier that nothing arrives on, through the same bounded wait the GEMM
+ * pipeline uses, for at most limit_us microseconds, then sets NC_DEV_TIMEOUT in
+ * *dev_status and exits normally (the context stays usable).  Expect
+ * nc_get_status(dev_status) == NC_ERR_TIMEOUT afterwards.  limit_us in
+ * [1, 2000000]. */
+nc_status nc_selftest_bounded_wait(uint32_t* dev_status, uint32_t limit_us, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* NC_H_ */

@@ -138,19 +138,20 @@ def attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, W: int,
     assert H % Hkv == 0
     group = H // Hkv
     rows = np.arange(T) if query_positions is None else np.asarray(query_positions)
-    out = np.zeros((B, len(rows), H, D), dtype=F64)
     scale = 1.0 / math.sqrt(D)
-    jj = np.arange(T)
-    for r, i in enumerate(rows):
-        vis = (jj <= i) & ((i - jj) < W)
-        idx = jj[vis]
+    i = rows[:, None]
+    j = np.arange(T)[None, :]
+    visible = (j <= i) & ((i - j) < W)  # [R, T]
+    out = np.zeros((B, len(rows), H, D), dtype=F64)
+    for b in range(B):
         for h in range(H):
             g = h // group
-            s = (k[:, idx, g, :] @ q[:, i, h, :, None])[..., 0] * scale  # [B, n]
+            s = (q[b, rows, h, :] @ k[b, :, g, :].T) * scale  # [R, T]
+            s = np.where(visible, s, -np.inf)
             s = s - s.max(axis=1, keepdims=True)
             p = np.exp(s)
             p = p / p.sum(axis=1, keepdims=True)
-            out[:, r, h, :] = (p[:, None, :] @ v[:, idx, g, :])[:, 0, :]
+            out[b, :, h, :] = p @ v[b, :, g, :]
     return out
 
 
@@ -205,7 +206,6 @@ def forward(cfg: OracleConfig, weights: dict, idx: np.ndarray, targets=None,
 
     Returns a dict with ``logits`` ([B,T,V] capped, fp64, if ``want_logits``),
     ``token_loss`` ([B,T]) and ``loss`` (scalar) when targets are given.
-    Rows are processed one at a time to bound memory.
     """
     idx = np.asarray(idx)
     B, T = idx.shape
@@ -213,35 +213,25 @@ def forward(cfg: OracleConfig, weights: dict, idx: np.ndarray, targets=None,
     eps = cfg.norm_eps
     windows = layer_windows(cfg)
     cos, sin = rope_tables(T, D, cfg.rope_base)
-    logits_out = [] if want_logits else None
-    nll_rows = []
-    for b in range(B):
-        x = embed(weights["wte"], idx[b:b + 1])  # [1,T,C]
-        for l, lw in enumerate(weights["layers"]):
-            a = rms_norm(x, eps)
-            q = (a @ _w(lw["c_q"]).T).reshape(1, T, H, D)
-            k = (a @ _w(lw["c_k"]).T).reshape(1, T, Hkv, D)
-            v = (a @ _w(lw["c_v"]).T).reshape(1, T, Hkv, D)
-            q = rms_norm(rope(q, cos, sin), eps)
-            k = rms_norm(rope(k, cos, sin), eps)
-            o = attention(q, k, v, windows[l])
-            x = x + o.reshape(1, T, H * D) @ _w(lw["attn_proj"]).T
-            a = rms_norm(x, eps)
-            x = x + relu2_mlp(a, lw["c_fc"], lw["mlp_proj"])
+    x = embed(weights["wte"], idx)  # [B,T,C]
+    for l, lw in enumerate(weights["layers"]):
         a = rms_norm(x, eps)
-        logits = softcap(a @ _w(weights["lm_head"]).T, cfg.softcap)  # [1,T,V]
-        if want_logits:
-            logits_out.append(logits[0])
-        if targets is not None:
-            nll, _ = cross_entropy(logits[0], np.asarray(targets)[b])
-            nll_rows.append(nll)
+        q = (a @ _w(lw["c_q"]).T).reshape(B, T, H, D)
+        k = (a @ _w(lw["c_k"]).T).reshape(B, T, Hkv, D)
+        v = (a @ _w(lw["c_v"]).T).reshape(B, T, Hkv, D)
+        q = rms_norm(rope(q, cos, sin), eps)
+        k = rms_norm(rope(k, cos, sin), eps)
+        o = attention(q, k, v, windows[l])
+        x = x + o.reshape(B, T, H * D) @ _w(lw["attn_proj"]).T
+        a = rms_norm(x, eps)
+        x = x + relu2_mlp(a, lw["c_fc"], lw["mlp_proj"])
+    a = rms_norm(x, eps)
+    logits = softcap(a @ _w(weights["lm_head"]).T, cfg.softcap)  # [B,T,V]
     res = {}
     if want_logits:
-        res["logits"] = np.stack(logits_out)
+        res["logits"] = logits
     if targets is not None:
-        tl = np.stack(nll_rows)
-        y = np.asarray(targets)
-        n = int((y != -1).sum())
-        res["token_loss"] = tl
-        res["loss"] = float(tl.sum() / n) if n > 0 else float("nan")
+        nll, loss = cross_entropy(logits, np.asarray(targets))
+        res["token_loss"] = nll
+        res["loss"] = loss
     return res

@@ -1,0 +1,157 @@
+"""CPU-only checks of the C ABI: the library loads, exports every entry point the
+header declares, derives configurations as the pages do, and rejects bad
+arguments on the host before touching a device."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import oracle
+from workloads import SHAPES
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+GOLDEN = os.path.join(ROOT, "tests", "golden")
+
+
+def _declared_symbols():
+    with open(os.path.join(ROOT, "include", "nc.h")) as f:
+        text = f.read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(nc_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_symbols_exported(nclib):
+    names = _declared_symbols()
+    assert len(names) >= 20
+    L = nclib.lib()
+    for n in names:
+        assert hasattr(L, n), f"{n} declared in include/nc.h but not exported"
+    assert L.nc_version() >= 100
+
+
+def test_init_config_matches_pages_and_oracle(nclib):
+    rows = [l.split() for l in open(os.path.join(GOLDEN, "config_examples.txt"))
+            if l.strip() and not l.startswith("#") and l.startswith("derive")]
+    for _, depth, aspect, hd, model_dim, heads in rows:
+        c = nclib.init_config(int(depth), int(aspect), int(hd))
+        assert (c.d_model, c.n_head, c.n_kv_head, c.head_dim) == (int(model_dim), int(heads), int(heads), int(hd))
+        assert c.short_window == 512 and c.window_pattern == b"SSSL" and c.softcap == 15.0
+
+
+@pytest.mark.parametrize("name", list(SHAPES))
+def test_layer_windows_agree_with_oracle(nclib, name):
+    s = SHAPES[name]
+    c = nclib.make_config(s.n_layer, s.d_model, s.n_head, s.n_kv_head, s.head_dim, s.seq_len, s.vocab,
+                          s.short_window)
+    oc = oracle.OracleConfig(s.n_layer, s.d_model, s.n_head, s.n_kv_head, s.head_dim, s.seq_len, s.vocab,
+                             short_window=s.short_window)
+    assert [nclib.layer_window(c, l) for l in range(s.n_layer)] == oracle.layer_windows(oc)
+    assert nclib.layer_window(c, s.n_layer) == -1
+
+
+def test_forward_flops_counts(nclib):
+    # published totals of the FLOP model (attention counted inside the window only)
+    want = {"d12": 3.965, "d20": 61.011, "d26": 63.611, "d26_gqa": 83.650}
+    for name, tf in want.items():
+        s = SHAPES[name]
+        c = nclib.make_config(s.n_layer, s.d_model, s.n_head, s.n_kv_head, s.head_dim, s.seq_len,
+                              s.vocab, s.short_window)
+        assert abs(nclib.forward_flops(c, s.batch, s.seq_len) / 1e12 - tf) < 5e-4
+    # brute-force count of visible (query, key) pairs on a tiny case
+    c = nclib.make_config(2, 128, 2, 1, 64, 16, 512, 5)
+    T, B = 16, 3
+    pairs = 0
+    for W in (5, 16):
+        pairs += sum(oracle.window_visible(i, j, W) for i in range(T) for j in range(T))
+    M, C, D, H, Hkv, V = B * T, 128, 64, 2, 1, 512
+    proj = 2 * (2 * M * C * (H + 2 * Hkv) * D + 2 * M * H * D * C + 16 * M * C * C) + 2 * M * C * V
+    assert nclib.forward_flops(c, B, T) == pytest.approx(proj + 4 * D * H * B * pairs, rel=1e-12)
+
+
+def test_workspace_bytes(nclib):
+    c = nclib.init_config(20)
+    ws = nclib.workspace_bytes(c, 32, 2048)
+    assert 2.5e9 < ws < 3.5e9
+    assert nclib.workspace_bytes(c, 32, 4096) == 0  # T > seq_len
+    assert nclib.workspace_bytes(c, 0, 2048) == 0
+
+
+def test_bad_configs_rejected(nclib):
+    L = nclib.lib()
+    c = nclib.NcConfig()
+    assert L.nc_init_config(None, 20, 64, 128, 0, 2048, 32768) == 1
+    assert L.nc_init_config(ctypes.byref(c), 20, 64, 128, 3, 2048, 32768) == 2  # 10 % 3 != 0
+    assert L.nc_init_config(ctypes.byref(c), 20, 64, 96, 0, 2048, 32768) == 2  # head_dim
+    assert L.nc_init_config(ctypes.byref(c), 20, 64, 128, 0, 2048, 1000) == 2  # vocab % 64
+    good = nclib.init_config(2, 64, 64, 0, 256, 512)
+    bad = nclib.NcConfig.from_buffer_copy(good)
+    bad.window_pattern = b"SSXL"
+    assert nclib.check_config(bad) == 2
+    assert nclib.check_config(good) == 0
+
+
+class _FakeWeights:
+    """nc_weights whose device pointers are aligned integers never dereferenced."""
+
+    def __init__(self, nclib, n_layer, base=1 << 40, misalign=False):
+        mk = lambda: (ctypes.c_void_p * n_layer)(*[base + 4096 * i for i in range(n_layer)])
+        self.arrs = [mk() for _ in range(6)]
+        if misalign:
+            self.arrs[4][0] = base + 8
+        FPP = ctypes.POINTER(ctypes.c_void_p)
+        self.w = nclib.NcWeights(base, *[ctypes.cast(a, FPP) for a in self.arrs], base + 64)
+
+
+def _fwd(nclib, cfg, fw, B, T, tokens=1 << 41, targets=1 << 41, ws=1 << 42, ws_bytes=None, loss=None):
+    L = nclib.lib()
+    if ws_bytes is None:
+        ws_bytes = max(nclib.workspace_bytes(cfg, B, T), 1)
+    return L.nc_forward(ctypes.byref(cfg), ctypes.byref(fw.w), tokens, targets, B, T, None, None, loss,
+                        ws, ws_bytes, None)
+
+
+def test_forward_host_validation(nclib):
+    cfg = nclib.init_config(2, 64, 64, 0, 256, 512)
+    fw = _FakeWeights(nclib, 2)
+    assert _fwd(nclib, cfg, fw, 2, 512) == 3                      # T > seq_len
+    assert _fwd(nclib, cfg, fw, 0, 16) == 3                       # B < 1
+    assert _fwd(nclib, cfg, fw, 2, 16, tokens=None) == 1          # NULL tokens
+    assert _fwd(nclib, cfg, fw, 2, 16, targets=None, loss=1 << 43) == 1  # loss without targets
+    assert _fwd(nclib, cfg, fw, 2, 16, ws_bytes=1024) == 5        # workspace too small
+    assert _fwd(nclib, cfg, fw, 2, 16, ws=(1 << 42) + 16) == 4    # workspace not 256-aligned
+    assert _fwd(nclib, cfg, _FakeWeights(nclib, 2, misalign=True), 2, 16) == 4
+    bad = nclib.NcConfig.from_buffer_copy(cfg)
+    bad.n_kv_head = 3
+    assert _fwd(nclib, bad, fw, 2, 16) == 2
+
+
+def test_no_device_fails_loudly(nclib):
+    """With valid arguments and no sm_100 device every compute entry point refuses."""
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present; the device check passes there")
+    cfg = nclib.init_config(2, 64, 64, 0, 256, 512)
+    fw = _FakeWeights(nclib, 2)
+    assert _fwd(nclib, cfg, fw, 2, 16) == 8
+    L = nclib.lib()
+    assert L.nc_rmsnorm(1 << 40, 1 << 41, 8, 128, 1e-6, None) == 8
+    assert L.nc_attention(1 << 40, 1 << 40, 1 << 40, 1 << 41, 1, 16, 2, 2, 128, 0, None) == 8
+    assert L.nc_linear(1 << 40, 1 << 40, 1 << 41, 128, 256, 64, 256, 0, 15.0, None, None) == 8
+    assert L.nc_selftest_bounded_wait(1 << 40, 100, None) == 8
+
+
+def test_single_step_argument_checks(nclib):
+    L = nclib.lib()
+    assert L.nc_linear(1 << 40, 1 << 40, 1 << 41, 128, 250, 64, 256, 0, 15.0, None, None) == 3  # N % 32
+    assert L.nc_linear(1 << 40, 1 << 40, 1 << 41, 128, 256, 60, 256, 0, 15.0, None, None) == 3  # K % 8
+    assert L.nc_linear((1 << 40) + 2, 1 << 40, 1 << 41, 128, 256, 64, 256, 0, 15.0, None, None) == 4
+    assert L.nc_linear(1 << 40, 1 << 40, 1 << 41, 128, 256, 64, 256, 9, 15.0, None, None) == 1
+    assert L.nc_attention(1 << 40, 1 << 40, 1 << 40, 1 << 41, 1, 16, 4, 3, 128, 0, None) == 1  # H % Hkv
+    assert L.nc_attention(1 << 40, 1 << 40, 1 << 40, 1 << 41, 1, 16, 4, 4, 64, 0, None) == 3
+    assert L.nc_rope_qknorm(1 << 40, 1 << 40, 1 << 40, 1, 16, 2, 2, 96, 192, 192, 1e-6, None) == 3
+    assert L.nc_cast_bf16(1 << 40, 1 << 41, 12, None) == 1
+    assert L.nc_softcap_ce(1 << 40, 1 << 40, None, 1 << 41, 4, 512, -1.0, None, None) == 1
+    assert L.nc_selftest_bounded_wait(None, 100, None) == 1
+    assert L.nc_status_string(7) == b"bounded device wait ran out"
