@@ -36,6 +36,9 @@ function here, and the CUDA library takes the same reading independently):
   (exactly W keys including the query itself).
 * layer l uses pattern[l % len(pattern)], and the last layer is forced full.
 * GQA: query head h reads kv head h // (H / Hkv).
+* weights enter every matrix product as their bf16 (round-to-nearest-even)
+  values -- the pages fix that cast -- and the products and everything else are
+  fp64; the embedding table is read as given (fp32, no cast).
 * no norm after the embedding; one parameter-free RMSNorm before lm_head.
 * soft-cap 15*tanh(z/15) is applied before the loss and the returned logits are
   the capped ones; loss = mean natural-log NLL over targets != -1 (NaN if none).
@@ -58,6 +61,8 @@ from .model import (  # noqa: F401
     rope_qknorm,
     attention,
     relu2_mlp,
+    to_bf16,
+    linear,
     softcap,
     cross_entropy,
     embed,

@@ -157,9 +157,9 @@ def attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, W: int,
 
 def relu2_mlp(a: np.ndarray, w_fc: np.ndarray, w_proj: np.ndarray) -> np.ndarray:
     """"从文本到聊天模型" §5.7: c_fc (C -> 4C), relu(x)^2, c_proj (4C -> C)."""
-    h = np.asarray(a, dtype=F64) @ np.asarray(w_fc, dtype=F64).T
+    h = linear(a, w_fc)
     h = np.maximum(h, 0.0) ** 2
-    return h @ np.asarray(w_proj, dtype=F64).T
+    return linear(h, w_proj)
 
 
 def softcap(z: np.ndarray, cap: float) -> np.ndarray:
@@ -186,13 +186,34 @@ def cross_entropy(logits: np.ndarray, targets: np.ndarray):
     return nll, loss
 
 
+def to_bf16(w: np.ndarray) -> np.ndarray:
+    """Round to the nearest bfloat16 value, ties to even, returned as float64.
+
+    The method keeps its weights in fp32 and converts them to the compute dtype
+    (bf16) when they enter a matrix product (nanochat README mirror, "精度 /
+    dtype"; "约100美元训出对话模型" on the custom Linear layer).  bfloat16 keeps
+    the top 16 bits of the fp32 pattern; the dropped low half is rounded half to
+    even on the kept least-significant bit.  NaN stays NaN.
+    """
+    a = np.ascontiguousarray(w, dtype=np.float32)
+    bits = a.view(np.uint32).astype(np.uint64)
+    keep_lsb = (bits >> np.uint64(16)) & np.uint64(1)
+    rounded = (bits + np.uint64(0x7FFF) + keep_lsb) >> np.uint64(16)
+    out = (rounded << np.uint64(16)).astype(np.uint32).view(np.float32)
+    out = np.where(np.isnan(a), a, out)
+    return out.astype(F64)
+
+
+def linear(x: np.ndarray, w: np.ndarray) -> np.ndarray:
+    """Bias-free linear layer y = x W^T with W in [out, in] layout ("Nanochat与
+    nanoGPT对比" §1: no biases).  The fp32 weight is cast to bf16 first (see
+    ``to_bf16``); the product itself is exact fp64."""
+    return np.asarray(x, dtype=F64) @ to_bf16(w).T
+
+
 def embed(wte: np.ndarray, idx: np.ndarray) -> np.ndarray:
     """"从文本到聊天模型" §5.2: x = wte(idx), (B,T) -> (B,T,C)."""
     return np.asarray(wte, dtype=F64)[np.asarray(idx)]
-
-
-def _w(a):
-    return np.asarray(a, dtype=F64)
 
 
 def forward(cfg: OracleConfig, weights: dict, idx: np.ndarray, targets=None,
@@ -216,17 +237,17 @@ def forward(cfg: OracleConfig, weights: dict, idx: np.ndarray, targets=None,
     x = embed(weights["wte"], idx)  # [B,T,C]
     for l, lw in enumerate(weights["layers"]):
         a = rms_norm(x, eps)
-        q = (a @ _w(lw["c_q"]).T).reshape(B, T, H, D)
-        k = (a @ _w(lw["c_k"]).T).reshape(B, T, Hkv, D)
-        v = (a @ _w(lw["c_v"]).T).reshape(B, T, Hkv, D)
+        q = linear(a, lw["c_q"]).reshape(B, T, H, D)
+        k = linear(a, lw["c_k"]).reshape(B, T, Hkv, D)
+        v = linear(a, lw["c_v"]).reshape(B, T, Hkv, D)
         q = rms_norm(rope(q, cos, sin), eps)
         k = rms_norm(rope(k, cos, sin), eps)
         o = attention(q, k, v, windows[l])
-        x = x + o.reshape(B, T, H * D) @ _w(lw["attn_proj"]).T
+        x = x + linear(o.reshape(B, T, H * D), lw["attn_proj"])
         a = rms_norm(x, eps)
         x = x + relu2_mlp(a, lw["c_fc"], lw["mlp_proj"])
     a = rms_norm(x, eps)
-    logits = softcap(a @ _w(weights["lm_head"]).T, cfg.softcap)  # [B,T,V]
+    logits = softcap(linear(a, weights["lm_head"]), cfg.softcap)  # [B,T,V]
     res = {}
     if want_logits:
         res["logits"] = logits

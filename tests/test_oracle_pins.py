@@ -22,6 +22,11 @@ from workloads import SHAPES, make_tokens, make_weights, round_to_bf16
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
 
 
+def bf16_weights_torch(a):
+    """fp32 weights as their bf16 values, through torch's own conversion."""
+    return torch.from_numpy(np.asarray(a, dtype=np.float32)).to(torch.bfloat16).to(torch.float64)
+
+
 def _golden_lines(name):
     with open(os.path.join(GOLDEN, name)) as f:
         return [l.split() for l in f if l.strip() and not l.startswith("#")]
@@ -235,6 +240,37 @@ def test_attention_special_cases():
     np.testing.assert_allclose(oracle.attention(q, k, v, 5, rows), oracle.attention(q, k, v, 5)[:, rows], atol=0)
 
 
+# ---------------------------------------------------------------- bf16 weight cast
+
+def test_to_bf16_hand_values():
+    # bf16 keeps 8 significant bits: the spacing just above 1 is 2^-7.
+    cases = [(1.0, 1.0), (1.0 + 2.0 ** -9, 1.0), (1.0 + 3 * 2.0 ** -9, 1.0 + 2.0 ** -7),
+             (1.0 + 2.0 ** -8, 1.0),                         # tie -> even significand (1.0)
+             (1.0 + 3 * 2.0 ** -8, 1.0 + 2.0 ** -6),          # tie -> even (1 + 2^-6)
+             (-2.0 - 2.0 ** -7, -2.0), (0.0, 0.0), (3.0e38, 226 * 2.0 ** 120)]  # spacing 2^120 there
+    got = oracle.to_bf16(np.array([c[0] for c in cases], dtype=np.float32))
+    np.testing.assert_array_equal(got, np.array([c[1] for c in cases], dtype=np.float32).astype(np.float64))
+    assert np.isnan(oracle.to_bf16(np.array([np.nan], dtype=np.float32)))[0]
+
+
+def test_to_bf16_matches_torch_conversion():
+    rng = np.random.default_rng(13)
+    a = (rng.standard_normal(200_000) * 10.0 ** rng.uniform(-20, 20, 200_000)).astype(np.float32)
+    bits = rng.integers(0, 2 ** 32, 20_000, dtype=np.uint64).astype(np.uint32)
+    b = bits.view(np.float32)
+    b = b[np.isfinite(b)]
+    for x in (a, b):
+        np.testing.assert_array_equal(oracle.to_bf16(x), bf16_weights_torch(x).numpy())
+
+
+def test_linear_uses_cast_weights():
+    # a weight that bf16 cannot hold changes the product: 1 + 2^-9 acts as 1
+    x = np.array([[2.0, -1.0]])
+    w = np.array([[1.0 + 2.0 ** -9, 0.5]], dtype=np.float32)
+    np.testing.assert_array_equal(oracle.linear(x, w), [[2.0 - 0.5]])
+    assert oracle.linear(np.eye(3), np.full((4, 3), 0.1, dtype=np.float32)).dtype == np.float64
+
+
 # ---------------------------------------------------------------- MLP / soft-cap / CE
 
 def test_relu2_mlp_hand_values():
@@ -308,7 +344,7 @@ def test_forward_zero_projections_closed_form():
     res = oracle.forward(c, w, idx, y)
     a = w["wte"][idx]
     a = a / np.sqrt(np.mean(a * a, -1, keepdims=True) + c.norm_eps)
-    want = 15.0 * np.tanh((a @ w["lm_head"].T) / 15.0)
+    want = 15.0 * np.tanh((a @ bf16_weights_torch(w["lm_head"]).numpy().T) / 15.0)
     np.testing.assert_allclose(res["logits"], want, rtol=1e-12, atol=1e-12)
     want_nll = F.cross_entropy(torch.from_numpy(want).reshape(-1, c.vocab), torch.from_numpy(y).reshape(-1),
                                reduction="none").numpy().reshape(2, -1)
@@ -350,9 +386,9 @@ def test_forward_qk_norm_makes_attention_scale_free():
     rng = np.random.default_rng(8)
     idx = rng.integers(0, c.vocab, (1, c.seq_len))
     base = oracle.forward(c, w, idx)["logits"]
-    for lw in w["layers"]:
-        lw["c_q"] *= 37.0
-        lw["c_k"] *= 0.05
+    for lw in w["layers"]:  # powers of two commute with the bf16 weight cast
+        lw["c_q"] *= 32.0
+        lw["c_k"] *= 0.0625
     np.testing.assert_allclose(oracle.forward(c, w, idx)["logits"], base, rtol=1e-7, atol=1e-8)
 
 
@@ -368,7 +404,7 @@ def test_forward_matches_independent_torch_composition():
     y = rng.integers(-1, c.vocab, (2, c.seq_len))
     res = oracle.forward(c, w, idx, y)
 
-    T = lambda a: torch.from_numpy(np.asarray(a, dtype=np.float64))
+    T = bf16_weights_torch  # every weight enters its product as its bf16 value
     B, S = idx.shape
     H, Hkv, D, C = c.n_head, c.n_kv_head, c.head_dim, c.d_model
     theta = c.rope_base ** (-torch.arange(D // 2, dtype=torch.float64) * 2 / D)
@@ -380,7 +416,7 @@ def test_forward_matches_independent_torch_composition():
         return torch.cat([z.real, z.imag], -1)
 
     nrm = lambda u: F.rms_norm(u, (u.shape[-1],), eps=c.norm_eps)
-    x = F.embedding(torch.from_numpy(idx), T(w["wte"]))
+    x = F.embedding(torch.from_numpy(idx), torch.from_numpy(np.asarray(w["wte"], dtype=np.float64)))
     windows = [7, 7, 21]  # S S L (last layer forced full)
     for l, lw in enumerate(w["layers"]):
         a = nrm(x)
