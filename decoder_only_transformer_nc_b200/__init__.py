@@ -15,14 +15,16 @@ from dataclasses import dataclass
 __all__ = [
     "NcError", "NcConfig", "lib", "init_config", "make_config", "check_config", "layer_window",
     "workspace_bytes", "forward_flops", "Model", "forward", "LaunchTrace", "KERNEL_KINDS", "get_status", "cast_bf16", "embedding",
-    "rmsnorm", "rope_table", "rope_qknorm", "attention", "linear", "softcap_ce", "loss_mean",
-    "EPI_STORE_BF16", "EPI_RELU2_BF16", "EPI_RESID_F32", "EPI_STORE_F32", "EPI_SOFTCAP_F32",
+    "rmsnorm", "rope_table", "rope_qknorm", "attention", "linear", "qkv_rope", "softcap_ce",
+    "loss_mean", "cast_weights", "selftest_bounded_wait", "BF16", "F16",
+    "EPI_STORE_16", "EPI_RELU2_16", "EPI_RESID_F32", "EPI_STORE_F32", "EPI_SOFTCAP_F32",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libnc.so")
 
-EPI_STORE_BF16, EPI_RELU2_BF16, EPI_RESID_F32, EPI_STORE_F32, EPI_SOFTCAP_F32 = range(5)
+EPI_STORE_16, EPI_RELU2_16, EPI_RESID_F32, EPI_STORE_F32, EPI_SOFTCAP_F32 = range(5)
+BF16, F16 = 0, 1  # nc_dtype
 DEV_TOKEN_RANGE, DEV_TARGET_RANGE, DEV_TIMEOUT = 0x1, 0x2, 0x4
 
 STATUS_NAMES = {0: "NC_OK", 1: "NC_ERR_INVALID_ARG", 2: "NC_ERR_CONFIG", 3: "NC_ERR_SHAPE",
@@ -41,7 +43,7 @@ class NcConfig(ctypes.Structure):
                 ("n_kv_head", ctypes.c_int32), ("head_dim", ctypes.c_int32), ("vocab", ctypes.c_int32),
                 ("seq_len", ctypes.c_int32), ("short_window", ctypes.c_int32),
                 ("window_pattern", ctypes.c_char * 8), ("softcap", ctypes.c_float),
-                ("norm_eps", ctypes.c_float), ("rope_base", ctypes.c_float)]
+                ("norm_eps", ctypes.c_float), ("rope_base", ctypes.c_float), ("act_dtype", ctypes.c_int32)]
 
     def __repr__(self):
         return ("NcConfig(n_layer=%d, d_model=%d, n_head=%d, n_kv_head=%d, head_dim=%d, vocab=%d, "
@@ -94,14 +96,15 @@ def lib():
             "nc_event_destroy": (i32, [vp]),
             "nc_event_elapsed_ms": (i32, [vp, vp, ctypes.POINTER(ctypes.c_float)]),
             "nc_get_status": (i32, [vp, vp]),
-            "nc_cast_bf16": (i32, [vp, vp, i64, vp]),
+            "nc_cast_weights": (i32, [vp, vp, i64, i32, vp]),
             "nc_embedding": (i32, [vp, vp, vp, i32, i32, i32, vp, vp]),
-            "nc_rmsnorm": (i32, [vp, vp, i32, i32, f32, vp]),
+            "nc_rmsnorm": (i32, [vp, vp, i32, i32, f32, i32, vp]),
             "nc_rope_table": (i32, [vp, i32, i32, f32, vp]),
-            "nc_rope_qknorm": (i32, [vp, vp, vp, i32, i32, i32, i32, i32, i64, i64, f32, vp]),
-            "nc_attention": (i32, [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, vp]),
-            "nc_attention_strided": (i32, [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i64, i64, vp]),
-            "nc_linear": (i32, [vp, vp, vp, i32, i32, i32, i64, i32, f32, vp, vp]),
+            "nc_rope_qknorm": (i32, [vp, vp, vp, i32, i32, i32, i32, i32, i64, i64, f32, i32, vp]),
+            "nc_attention": (i32, [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, vp]),
+            "nc_attention_strided": (i32, [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i64, i64, i32, vp]),
+            "nc_linear": (i32, [vp, vp, vp, i32, i32, i32, i64, i32, f32, i32, vp, vp]),
+            "nc_qkv_rope": (i32, [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, f32, i32, vp, vp]),
             "nc_softcap_ce": (i32, [vp, vp, vp, vp, i32, i32, f32, vp, vp]),
             "nc_loss_mean": (i32, [vp, vp, i32, i32, vp, vp]),
             "nc_selftest_bounded_wait": (i32, [vp, ctypes.c_uint32, vp]),
@@ -140,10 +143,11 @@ def init_config(depth: int, aspect_ratio: int = 64, head_dim: int = 128, n_kv_he
 
 
 def make_config(n_layer, d_model, n_head, n_kv_head, head_dim, seq_len, vocab, short_window=0,
-                window_pattern="SSSL", softcap=15.0, norm_eps=1e-6, rope_base=10000.0) -> NcConfig:
+                window_pattern="SSSL", softcap=15.0, norm_eps=1e-6, rope_base=10000.0,
+                act_dtype=F16) -> NcConfig:
     c = NcConfig(n_layer, d_model, n_head, n_kv_head, head_dim, vocab, seq_len,
                  short_window if short_window > 0 else seq_len // 4, window_pattern.encode(),
-                 softcap, norm_eps, rope_base)
+                 softcap, norm_eps, rope_base, act_dtype)
     _check(lib().nc_check_config(ctypes.byref(c)), "nc_check_config")
     return c
 
@@ -288,8 +292,20 @@ def get_status(status_tensor, stream=None) -> int:
 
 # ---------------------------------------------------------------- single steps
 
-def cast_bf16(src, dst, stream=None):
-    _check(lib().nc_cast_bf16(_ptr(src), _ptr(dst), src.numel(), _stream(stream)), "nc_cast_bf16")
+def _dt(t):
+    """nc_dtype of a 16-bit torch tensor."""
+    import torch
+    if t.dtype == torch.float16:
+        return F16
+    if t.dtype == torch.bfloat16:
+        return BF16
+    raise TypeError(f"expected a float16 or bfloat16 tensor, got {t.dtype}")
+
+
+def cast_weights(src, dst, stream=None):
+    """fp32 -> bf16-rounded weights in dst's format (bfloat16, or float16 holding the bf16 values)."""
+    _check(lib().nc_cast_weights(_ptr(src), _ptr(dst), src.numel(), _dt(dst), _stream(stream)),
+           "nc_cast_weights")
 
 
 def embedding(tokens, wte, x, status=None, stream=None):
@@ -301,7 +317,8 @@ def embedding(tokens, wte, x, status=None, stream=None):
 
 def rmsnorm(x, out, eps=1e-6, stream=None):
     C = x.shape[-1]
-    _check(lib().nc_rmsnorm(_ptr(x), _ptr(out), x.numel() // C, C, eps, _stream(stream)), "nc_rmsnorm")
+    _check(lib().nc_rmsnorm(_ptr(x), _ptr(out), x.numel() // C, C, eps, _dt(out), _stream(stream)),
+           "nc_rmsnorm")
 
 
 def rope_table(table, T, D, base=10000.0, stream=None):
@@ -312,22 +329,28 @@ def rope_qknorm(q, k, table, B, T, H, Hkv, D, q_row_stride=None, k_row_stride=No
                 stream=None):
     qs = H * D if q_row_stride is None else q_row_stride
     ks = Hkv * D if k_row_stride is None else k_row_stride
-    _check(lib().nc_rope_qknorm(_ptr(q), _ptr(k), _ptr(table), B, T, H, Hkv, D, qs, ks, eps,
+    _check(lib().nc_rope_qknorm(_ptr(q), _ptr(k), _ptr(table), B, T, H, Hkv, D, qs, ks, eps, _dt(q),
                                 _stream(stream)), "nc_rope_qknorm")
 
 
 def attention(q, k, v, out, window, stream=None):
     B, T, H, D = q.shape
     Hkv = k.shape[2]
-    _check(lib().nc_attention(_ptr(q), _ptr(k), _ptr(v), _ptr(out), B, T, H, Hkv, D, window,
+    _check(lib().nc_attention(_ptr(q), _ptr(k), _ptr(v), _ptr(out), B, T, H, Hkv, D, window, _dt(q),
                               _stream(stream)), "nc_attention")
 
 
 def linear(a, w, out, epilogue, cap=15.0, status=None, stream=None):
     M, K = a.shape
     N = w.shape[0]
-    _check(lib().nc_linear(_ptr(a), _ptr(w), _ptr(out), M, N, K, out.stride(0), epilogue, cap,
+    _check(lib().nc_linear(_ptr(a), _ptr(w), _ptr(out), M, N, K, out.stride(0), epilogue, cap, _dt(a),
                            _ptr(status), _stream(stream)), "nc_linear")
+
+
+def qkv_rope(a, w, out, table, T, H, Hkv, D, eps=1e-6, status=None, stream=None):
+    M, C = a.shape
+    _check(lib().nc_qkv_rope(_ptr(a), _ptr(w), _ptr(out), _ptr(table), M, T, C, H, Hkv, D, eps, _dt(a),
+                             _ptr(status), _stream(stream)), "nc_qkv_rope")
 
 
 def softcap_ce(z, targets, token_loss, capped_out=None, cap=15.0, status=None, stream=None):

@@ -77,6 +77,7 @@ bool config_ok(const nc_config* c) {
   if (c->d_model % 64 != 0) return false;
   if ((int64_t)c->n_head * c->head_dim % 64 != 0) return false;
   if (!(c->softcap > 0.0f) || !(c->norm_eps >= 0.0f) || !(c->rope_base > 1.0f)) return false;
+  if (c->act_dtype != NC_F16 && c->act_dtype != NC_BF16) return false;
   const size_t plen = strnlen(c->window_pattern, sizeof(c->window_pattern));
   if (plen == 0 || plen >= sizeof(c->window_pattern)) return false;
   for (size_t i = 0; i < plen; ++i)
@@ -152,7 +153,7 @@ struct Tracer {
 
 // Number of kernel launches of one forward.
 int forward_launch_count(const nc_config* c, bool targets, bool loss, bool logits) {
-  int n = 3 + c->n_layer * 8 + 1;  // rope table, cast, embedding; layers; final norm
+  int n = 3 + c->n_layer * 7 + 1;  // rope table, cast, embedding; layers; final norm
   if (targets) n += 2 + (loss ? 1 : 0);
   else if (logits) n += 1;
   return n;
@@ -203,6 +204,7 @@ nc_status nc_init_config(nc_config* out, int depth, int aspect_ratio, int head_d
   c.softcap = 15.0f;
   c.norm_eps = 1e-6f;
   c.rope_base = 10000.0f;
+  c.act_dtype = NC_F16;
   *out = c;
   return config_ok(&c) ? NC_OK : NC_ERR_CONFIG;
 }
@@ -251,12 +253,15 @@ nc_status nc_get_status(const void* dev_status, void* stream) {
   return NC_OK;
 }
 
-nc_status nc_cast_bf16(const float* src, uint16_t* dst, int64_t n, void* stream) {
-  if (!src || !dst || n < 0 || n % 8 != 0) return NC_ERR_INVALID_ARG;
+inline bool dtype_ok(int d) { return d == NC_F16 || d == NC_BF16; }
+
+nc_status nc_cast_weights(const float* src, uint16_t* dst, int64_t n, nc_dtype container,
+                          void* stream) {
+  if (!src || !dst || n < 0 || n % 8 != 0 || !dtype_ok(container)) return NC_ERR_INVALID_ARG;
   if (!aligned16(src) || !aligned16(dst)) return NC_ERR_ALIGNMENT;
   if (nc_status s = device_ok()) return s;
   CastSeg seg{src, dst, n};
-  return cast_launch(&seg, 1, S(stream));
+  return cast_launch(&seg, 1, container == NC_F16, S(stream));
 }
 
 nc_status nc_embedding(const int32_t* tokens, const float* wte, float* x, int M, int C, int V,
@@ -267,11 +272,13 @@ nc_status nc_embedding(const int32_t* tokens, const float* wte, float* x, int M,
   return embedding_launch(tokens, wte, x, M, C, V, dev_status, S(stream));
 }
 
-nc_status nc_rmsnorm(const float* x, uint16_t* out, int M, int C, float eps, void* stream) {
-  if (!x || !out || M < 0 || C < 8 || C % 8 != 0 || !(eps >= 0.0f)) return NC_ERR_INVALID_ARG;
+nc_status nc_rmsnorm(const float* x, uint16_t* out, int M, int C, float eps, nc_dtype dtype,
+                     void* stream) {
+  if (!x || !out || M < 0 || C < 8 || C % 8 != 0 || !(eps >= 0.0f) || !dtype_ok(dtype))
+    return NC_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(out)) return NC_ERR_ALIGNMENT;
   if (nc_status s = device_ok()) return s;
-  return rmsnorm_launch(x, out, M, C, eps, S(stream));
+  return rmsnorm_launch(x, out, M, C, eps, dtype == NC_F16, S(stream));
 }
 
 nc_status nc_rope_table(float* table, int T, int D, float base, void* stream) {
@@ -282,8 +289,9 @@ nc_status nc_rope_table(float* table, int T, int D, float base, void* stream) {
 
 nc_status nc_rope_qknorm(uint16_t* q, uint16_t* k, const float* table, int B, int T, int H, int Hkv,
                          int D, int64_t q_row_stride, int64_t k_row_stride, float eps,
-                         void* stream) {
-  if (!q || !k || !table || B < 0 || T < 1 || H < 1 || Hkv < 1) return NC_ERR_INVALID_ARG;
+                         nc_dtype dtype, void* stream) {
+  if (!q || !k || !table || B < 0 || T < 1 || H < 1 || Hkv < 1 || !dtype_ok(dtype))
+    return NC_ERR_INVALID_ARG;
   if (D != 64 && D != 128) return NC_ERR_SHAPE;
   if (q_row_stride < (int64_t)H * D || k_row_stride < (int64_t)Hkv * D || q_row_stride % 8 ||
       k_row_stride % 8)
@@ -291,34 +299,36 @@ nc_status nc_rope_qknorm(uint16_t* q, uint16_t* k, const float* table, int B, in
   if (!aligned16(q) || !aligned16(k) || !aligned16(table)) return NC_ERR_ALIGNMENT;
   if (nc_status s = device_ok()) return s;
   return rope_qknorm_launch(q, k, table, B, T, H, Hkv, D, q_row_stride, k_row_stride, eps,
-                            S(stream));
+                            dtype == NC_F16, S(stream));
 }
 
 nc_status nc_attention_strided(const uint16_t* q, const uint16_t* k, const uint16_t* v,
                                uint16_t* out, int B, int T, int H, int Hkv, int D, int window,
-                               int64_t q_row_stride, int64_t kv_row_stride, void* stream) {
-  if (!q || !k || !v || !out || B < 0 || T < 0 || H < 1 || Hkv < 1 || H % Hkv != 0)
+                               int64_t q_row_stride, int64_t kv_row_stride, nc_dtype dtype,
+                               void* stream) {
+  if (!q || !k || !v || !out || B < 0 || T < 0 || H < 1 || Hkv < 1 || H % Hkv != 0 ||
+      !dtype_ok(dtype))
     return NC_ERR_INVALID_ARG;
-  if (D != 128) return NC_ERR_SHAPE;
+  if (D != 64 && D != 128) return NC_ERR_SHAPE;
   if (q_row_stride < (int64_t)H * D || kv_row_stride < (int64_t)Hkv * D || q_row_stride % 8 ||
       kv_row_stride % 8)
     return NC_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return NC_ERR_ALIGNMENT;
   if (nc_status s = device_ok()) return s;
   return attention_launch(q, k, v, out, B, T, H, Hkv, D, window, q_row_stride, kv_row_stride,
-                          S(stream));
+                          dtype == NC_F16, S(stream));
 }
 
 nc_status nc_attention(const uint16_t* q, const uint16_t* k, const uint16_t* v, uint16_t* out, int B,
-                       int T, int H, int Hkv, int D, int window, void* stream) {
+                       int T, int H, int Hkv, int D, int window, nc_dtype dtype, void* stream) {
   return nc_attention_strided(q, k, v, out, B, T, H, Hkv, D, window, (int64_t)H * D,
-                              (int64_t)Hkv * D, stream);
+                              (int64_t)Hkv * D, dtype, stream);
 }
 
 nc_status nc_linear(const uint16_t* a, const uint16_t* w, void* out, int M, int N, int K,
-                    int64_t ldo, nc_epilogue epilogue, float cap, uint32_t* dev_status,
-                    void* stream) {
-  if (!a || !w || !out || M < 0 || N < 32 || K < 8) return NC_ERR_INVALID_ARG;
+                    int64_t ldo, nc_epilogue epilogue, float cap, nc_dtype dtype,
+                    uint32_t* dev_status, void* stream) {
+  if (!a || !w || !out || M < 0 || N < 32 || K < 8 || !dtype_ok(dtype)) return NC_ERR_INVALID_ARG;
   if ((int)epilogue < 0 || (int)epilogue > (int)NC_EPI_SOFTCAP_F32) return NC_ERR_INVALID_ARG;
   if (N % 32 != 0 || K % 8 != 0 || ldo < N || ldo % 8 != 0) return NC_ERR_SHAPE;
   if (epilogue == NC_EPI_SOFTCAP_F32 && !(cap > 0.0f)) return NC_ERR_INVALID_ARG;
@@ -329,7 +339,31 @@ nc_status nc_linear(const uint16_t* a, const uint16_t* w, void* out, int M, int 
   ep.out = out;
   ep.ldo = ldo;
   ep.cap = cap;
-  return gemm_launch(a, K, w, K, M, N, K, (int)epilogue, ep, dev_status, S(stream));
+  return gemm_launch(a, K, w, K, M, N, K, (int)epilogue, dtype == NC_F16, ep, dev_status, S(stream));
+}
+
+nc_status nc_qkv_rope(const uint16_t* a, const uint16_t* w, uint16_t* out, const float* table,
+                      int M, int T, int C, int H, int Hkv, int D, float eps, nc_dtype dtype,
+                      uint32_t* dev_status, void* stream) {
+  if (!a || !w || !out || !table || M < 0 || T < 1 || C < 8 || H < 1 || Hkv < 1 ||
+      !(eps >= 0.0f) || !dtype_ok(dtype))
+    return NC_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return NC_ERR_SHAPE;
+  if (C % 8 != 0) return NC_ERR_SHAPE;
+  if (!aligned16(a) || !aligned16(w) || !aligned16(out) || !aligned16(table)) return NC_ERR_ALIGNMENT;
+  if (nc_status s = device_ok()) return s;
+  if (M == 0) return NC_OK;
+  const int N = (H + 2 * Hkv) * D;
+  EpiParams ep{};
+  ep.out = out;
+  ep.ldo = N;
+  ep.rope = table;
+  ep.T = T;
+  ep.H = H;
+  ep.Hkv = Hkv;
+  ep.D = D;
+  ep.eps = eps;
+  return gemm_launch(a, C, w, C, M, N, C, EPI_QKV_ROPE, dtype == NC_F16, ep, dev_status, S(stream));
 }
 
 nc_status nc_softcap_ce(const float* z, const int32_t* targets, float* capped_out,
@@ -412,6 +446,7 @@ nc_status nc_forward_traced(const nc_config* cfg, const nc_weights* w, const int
   const int C = cfg->d_model, D = cfg->head_dim, H = cfg->n_head, Hkv = cfg->n_kv_head,
             V = cfg->vocab;
   const int NQKV = (H + 2 * Hkv) * D;
+  const bool f16 = cfg->act_dtype == NC_F16;
 
   if (cudaMemsetAsync(status, 0, 256, st) != cudaSuccess) return NC_ERR_CUDA;
   NC_RUN(NC_K_ROPE_TABLE, rope_table_launch(rope, T, D, cfg->rope_base, st));
@@ -431,39 +466,44 @@ nc_status nc_forward_traced(const nc_config* cfg, const nc_weights* w, const int
       segs.push_back({w->mlp_proj[l], wmp + l * L.wmp_elems, (int64_t)L.wmp_elems});
     }
     segs.push_back({w->lm_head, wlm, (int64_t)V * C});
-    NC_RUN(NC_K_CAST, cast_launch(segs.data(), (int)segs.size(), st));
+    NC_RUN(NC_K_CAST, cast_launch(segs.data(), (int)segs.size(), f16, st));
   }
 
   NC_RUN(NC_K_EMBEDDING, embedding_launch(tokens, w->wte, x, M, C, V, status, st));
 
   for (int l = 0; l < cfg->n_layer; ++l) {
     const int W = nc_layer_window(cfg, l);
-    EpiParams ep{};
-    NC_RUN(NC_K_RMSNORM, rmsnorm_launch(x, a, M, C, cfg->norm_eps, st));
-    ep.out = qkv;
-    ep.ldo = NQKV;
+    NC_RUN(NC_K_RMSNORM, rmsnorm_launch(x, a, M, C, cfg->norm_eps, f16, st));
+    EpiParams eq{};  // QKV projection with RoPE + QK-norm in the epilogue
+    eq.out = qkv;
+    eq.ldo = NQKV;
+    eq.rope = rope;
+    eq.T = T;
+    eq.H = H;
+    eq.Hkv = Hkv;
+    eq.D = D;
+    eq.eps = cfg->norm_eps;
     NC_RUN(NC_K_GEMM_QKV,
-           gemm_launch(a, C, wqkv + l * L.wqkv_elems, C, M, NQKV, C, EPI_STORE_BF16, ep, status, st));
-    NC_RUN(NC_K_ROPE_QKNORM, rope_qknorm_launch(qkv, qkv + H * D, rope, B, T, H, Hkv, D, NQKV, NQKV,
-                                                cfg->norm_eps, st));
+           gemm_launch(a, C, wqkv + l * L.wqkv_elems, C, M, NQKV, C, EPI_QKV_ROPE, f16, eq, status, st));
     NC_RUN(NC_K_ATTENTION, attention_launch(qkv, qkv + H * D, qkv + (H + Hkv) * D, o, B, T, H, Hkv,
-                                            D, W, NQKV, NQKV, st));
+                                            D, W, NQKV, NQKV, f16, st));
+    EpiParams ep{};
     ep.out = x;
     ep.ldo = C;
     NC_RUN(NC_K_GEMM_ATTN_PROJ, gemm_launch(o, H * D, wo + l * L.wo_elems, H * D, M, C, H * D,
-                                            EPI_RESID_F32, ep, status, st));
-    NC_RUN(NC_K_RMSNORM, rmsnorm_launch(x, a, M, C, cfg->norm_eps, st));
+                                            EPI_RESID_F32, f16, ep, status, st));
+    NC_RUN(NC_K_RMSNORM, rmsnorm_launch(x, a, M, C, cfg->norm_eps, f16, st));
     ep.out = h;
     ep.ldo = 4 * C;
     NC_RUN(NC_K_GEMM_FC,
-           gemm_launch(a, C, wfc + l * L.wfc_elems, C, M, 4 * C, C, EPI_RELU2_BF16, ep, status, st));
+           gemm_launch(a, C, wfc + l * L.wfc_elems, C, M, 4 * C, C, EPI_RELU2_16, f16, ep, status, st));
     ep.out = x;
     ep.ldo = C;
     NC_RUN(NC_K_GEMM_MLP_PROJ, gemm_launch(h, 4 * C, wmp + l * L.wmp_elems, 4 * C, M, C, 4 * C,
-                                           EPI_RESID_F32, ep, status, st));
+                                           EPI_RESID_F32, f16, ep, status, st));
   }
 
-  NC_RUN(NC_K_RMSNORM, rmsnorm_launch(x, a, M, C, cfg->norm_eps, st));
+  NC_RUN(NC_K_RMSNORM, rmsnorm_launch(x, a, M, C, cfg->norm_eps, f16, st));
   if (targets) {
     EpiParams ep{};
     ep.out = logits;
@@ -473,7 +513,7 @@ nc_status nc_forward_traced(const nc_config* cfg, const nc_weights* w, const int
     ep.ce_partial = part;
     ep.ce_target = tgt;
     ep.targets = targets;
-    NC_RUN(NC_K_GEMM_LM_HEAD, gemm_launch(a, C, wlm, C, M, V, C, EPI_CE_PARTIAL, ep, status, st));
+    NC_RUN(NC_K_GEMM_LM_HEAD, gemm_launch(a, C, wlm, C, M, V, C, EPI_CE_PARTIAL, f16, ep, status, st));
     NC_RUN(NC_K_CE_FINALIZE, ce_finalize_launch(part, gemm_num_n_tiles(V), tgt, targets, tl, M, V,
                                                 cfg->softcap, status, st));
     if (loss) NC_RUN(NC_K_LOSS_MEAN, loss_mean_launch(tl, targets, M, V, loss, st));
@@ -482,7 +522,7 @@ nc_status nc_forward_traced(const nc_config* cfg, const nc_weights* w, const int
     ep.out = logits;
     ep.ldo = V;
     ep.cap = cfg->softcap;
-    NC_RUN(NC_K_GEMM_LM_HEAD, gemm_launch(a, C, wlm, C, M, V, C, EPI_SOFTCAP_F32, ep, status, st));
+    NC_RUN(NC_K_GEMM_LM_HEAD, gemm_launch(a, C, wlm, C, M, V, C, EPI_SOFTCAP_F32, f16, ep, status, st));
   }
 #undef NC_RUN
   return NC_OK;

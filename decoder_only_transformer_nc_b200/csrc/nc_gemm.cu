@@ -27,6 +27,7 @@
 #include <cstring>
 #include <mutex>
 
+#include "nc_half.cuh"
 #include "nc_internal.h"
 #include "nc_ptx.cuh"
 
@@ -45,7 +46,8 @@ constexpr int TMEM_COLS = 512;  // NUM_ACC * BN
 constexpr int NUM_THREADS = 192;
 constexpr int EPI_WARPS = 4;
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
-constexpr uint32_t IDESC = idesc_bf16_f32(BM, BN);
+constexpr uint32_t IDESC_BF16 = idesc_f32acc(BM, BN, false);
+constexpr uint32_t IDESC_F16 = idesc_f32acc(BM, BN, true);
 
 struct Smem {  // barrier block placed after the tile ring
   uint64_t full[STAGES];
@@ -58,63 +60,100 @@ struct Smem {  // barrier block placed after the tile ring
 };
 static_assert(sizeof(Smem) <= 256, "barrier block");
 
-template <int EPI>
-__device__ __forceinline__ void epilogue_chunk(const uint32_t (&r)[32], int row, int col0, int N,
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ float rcp_approx(float x) {
+  float y;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// Soft-cap l = cap * tanh(z / cap) written as cap - 2 cap / (1 + e^(2z/cap)),
+// plus p = exp(l - cap) = exp(-2 cap / (1 + e^(2z/cap))): three MUFU operations
+// per logit.  The limits are exact (z -> +inf: l = cap; z -> -inf: l = -cap).
+struct SoftCap {
+  float k_in;   // 2 log2(e) / cap
+  float two_cap;
+  float cap;
+  float k_out;  // -2 cap log2(e)
+  __device__ __forceinline__ explicit SoftCap(float c)
+      : k_in(2.0f * 1.4426950408889634f / c), two_cap(2.0f * c), cap(c),
+        k_out(-2.0f * c * 1.4426950408889634f) {}
+  __device__ __forceinline__ float apply(float z, float& p) const {
+    const float r = rcp_approx(1.0f + ex2_approx(z * k_in));
+    p = ex2_approx(k_out * r);
+    return fmaf(-two_cap, r, cap);
+  }
+  __device__ __forceinline__ float apply(float z) const {
+    const float r = rcp_approx(1.0f + ex2_approx(z * k_in));
+    return fmaf(-two_cap, r, cap);
+  }
+};
+
+template <bool F16, int NV>
+__device__ __forceinline__ void store16(uint16_t* o, const float* v) {
+#pragma unroll
+  for (int j = 0; j < NV / 8; ++j) {
+    uint4 pk;
+    pk.x = Half<F16>::pack2(v[8 * j + 0], v[8 * j + 1]);
+    pk.y = Half<F16>::pack2(v[8 * j + 2], v[8 * j + 3]);
+    pk.z = Half<F16>::pack2(v[8 * j + 4], v[8 * j + 5]);
+    pk.w = Half<F16>::pack2(v[8 * j + 6], v[8 * j + 7]);
+    reinterpret_cast<uint4*>(o)[j] = pk;
+  }
+}
+
+// Epilogue of one 32-column chunk held by this thread (one tile row).
+template <int EPI, bool F16>
+__device__ __forceinline__ void epilogue_chunk(const uint32_t (&r)[32], int row, int col0,
                                                const EpiParams& ep, float& ce_sum, float& ce_tl,
                                                int target) {
   float v[32];
 #pragma unroll
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
-  if constexpr (EPI == EPI_STORE_BF16 || EPI == EPI_RELU2_BF16) {
-    if constexpr (EPI == EPI_RELU2_BF16) {
+  if constexpr (EPI == EPI_STORE_16 || EPI == EPI_RELU2_16) {
+    if constexpr (EPI == EPI_RELU2_16) {
 #pragma unroll
       for (int i = 0; i < 32; ++i) {
         const float t = fmaxf(v[i], 0.0f);
         v[i] = t * t;
       }
     }
-    __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(ep.out) + (int64_t)row * ep.ldo + col0;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      uint4 pk;
-      __nv_bfloat162 h0 = __floats2bfloat162_rn(v[8 * j + 0], v[8 * j + 1]);
-      __nv_bfloat162 h1 = __floats2bfloat162_rn(v[8 * j + 2], v[8 * j + 3]);
-      __nv_bfloat162 h2 = __floats2bfloat162_rn(v[8 * j + 4], v[8 * j + 5]);
-      __nv_bfloat162 h3 = __floats2bfloat162_rn(v[8 * j + 6], v[8 * j + 7]);
-      pk.x = *reinterpret_cast<uint32_t*>(&h0);
-      pk.y = *reinterpret_cast<uint32_t*>(&h1);
-      pk.z = *reinterpret_cast<uint32_t*>(&h2);
-      pk.w = *reinterpret_cast<uint32_t*>(&h3);
-      reinterpret_cast<uint4*>(o)[j] = pk;
-    }
+    store16<F16, 32>(reinterpret_cast<uint16_t*>(ep.out) + (int64_t)row * ep.ldo + col0, v);
   } else if constexpr (EPI == EPI_RESID_F32) {
-    float* o = reinterpret_cast<float*>(ep.out) + (int64_t)row * ep.ldo + col0;
+    float4* o = reinterpret_cast<float4*>(reinterpret_cast<float*>(ep.out) + (int64_t)row * ep.ldo + col0);
+    float4 x[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) x[j] = o[j];
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
-      float4 x = reinterpret_cast<float4*>(o)[j];
-      x.x += v[4 * j + 0];
-      x.y += v[4 * j + 1];
-      x.z += v[4 * j + 2];
-      x.w += v[4 * j + 3];
-      reinterpret_cast<float4*>(o)[j] = x;
+      x[j].x += v[4 * j + 0];
+      x[j].y += v[4 * j + 1];
+      x[j].z += v[4 * j + 2];
+      x[j].w += v[4 * j + 3];
+      o[j] = x[j];
     }
   } else if constexpr (EPI == EPI_STORE_F32 || EPI == EPI_SOFTCAP_F32) {
     if constexpr (EPI == EPI_SOFTCAP_F32) {
+      const SoftCap sc(ep.cap);
 #pragma unroll
-      for (int i = 0; i < 32; ++i) v[i] = ep.cap * tanhf(v[i] / ep.cap);
+      for (int i = 0; i < 32; ++i) v[i] = sc.apply(v[i]);
     }
-    float* o = reinterpret_cast<float*>(ep.out) + (int64_t)row * ep.ldo + col0;
+    float4* o = reinterpret_cast<float4*>(reinterpret_cast<float*>(ep.out) + (int64_t)row * ep.ldo + col0);
 #pragma unroll
-    for (int j = 0; j < 8; ++j)
-      reinterpret_cast<float4*>(o)[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+    for (int j = 0; j < 8; ++j) o[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
   } else if constexpr (EPI == EPI_CE_PARTIAL) {
-    // Soft-capped logits l in (-cap, cap): exp(l - cap) never overflows, so the
-    // per-tile partial sums combine by plain addition.
+    // Soft-capped logits l lie in (-cap, cap): exp(l - cap) never overflows, so
+    // the per-tile partial sums combine by plain addition.
+    const SoftCap sc(ep.cap);
 #pragma unroll
     for (int i = 0; i < 32; ++i) {
-      const float l = ep.cap * tanhf(v[i] / ep.cap);
-      v[i] = l;
-      ce_sum += __expf(l - ep.cap);
+      float p;
+      v[i] = sc.apply(v[i], p);
+      ce_sum += p;
     }
     const int rel = target - col0;
     if (rel >= 0 && rel < 32) {
@@ -123,19 +162,85 @@ __device__ __forceinline__ void epilogue_chunk(const uint32_t (&r)[32], int row,
         if (i == rel) ce_tl = v[i];
     }
     if (ep.store_logits) {
-      float* o = reinterpret_cast<float*>(ep.out) + (int64_t)row * ep.ldo + col0;
+      float4* o = reinterpret_cast<float4*>(reinterpret_cast<float*>(ep.out) + (int64_t)row * ep.ldo + col0);
 #pragma unroll
-      for (int j = 0; j < 8; ++j)
-        reinterpret_cast<float4*>(o)[j] =
-            make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+      for (int j = 0; j < 8; ++j) o[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
     }
   }
 }
 
-template <int EPI>
+// QKV projection epilogue for one head of HD columns: q and k heads get RoPE
+// (pair (u_i, u_{i+HD/2}) rotated by t * theta_i) and RMSNorm over the head
+// ("Nanochat与nanoGPT对比" §1: QK-norm after RoPE); v heads are stored as is.
+// The rotation preserves the head's norm, so pass 1 takes the RMS straight from
+// the fp32 accumulator; pass 2 re-reads one (i, i + HD/2) chunk pair at a time,
+// rotates, scales and stores it.
+template <bool F16, int HD>
+__device__ __forceinline__ void epilogue_qkv_head(uint32_t taddr, int row, int col0, int M,
+                                                  const EpiParams& ep) {
+  const int head = col0 / HD;
+  uint16_t* out = reinterpret_cast<uint16_t*>(ep.out) + (int64_t)row * ep.ldo + col0;
+  if (head >= ep.H + ep.Hkv) {  // v head (warp-uniform)
+#pragma unroll 1
+    for (int c = 0; c < HD / 32; ++c) {
+      uint32_t r[32];
+      tmem_ld_32x32b_x32(taddr + c * 32, r);
+      tmem_wait_ld();
+      float v[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+      if (row < M) store16<F16, 32>(out + c * 32, v);
+    }
+    return;
+  }
+  float ss = 0.0f;
+#pragma unroll 1
+  for (int c = 0; c < HD / 32; ++c) {
+    uint32_t r[32];
+    tmem_ld_32x32b_x32(taddr + c * 32, r);
+    tmem_wait_ld();
+#pragma unroll
+    for (int i = 0; i < 32; ++i) ss = fmaf(__uint_as_float(r[i]), __uint_as_float(r[i]), ss);
+  }
+  const float rs = rsqrtf(ss * (1.0f / HD) + ep.eps);
+  const int t = (row < M ? row : 0) % ep.T;
+  const float* cs = ep.rope + (int64_t)t * (HD / 2);
+  const float* sn = ep.rope + ((int64_t)ep.T + t) * (HD / 2);
+#pragma unroll 1
+  for (int c = 0; c < HD / 64; ++c) {
+    uint32_t ra[32], rb[32];
+    tmem_ld_32x32b_x32(taddr + c * 32, ra);
+    tmem_ld_32x32b_x32(taddr + HD / 2 + c * 32, rb);
+    tmem_wait_ld();
+    float va[32], vb[32];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const float4 c4 = __ldg(reinterpret_cast<const float4*>(cs + c * 32) + j);
+      const float4 s4 = __ldg(reinterpret_cast<const float4*>(sn + c * 32) + j);
+      const float cc[4] = {c4.x, c4.y, c4.z, c4.w};
+      const float sv[4] = {s4.x, s4.y, s4.z, s4.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int i = 4 * j + e;
+        const float a = __uint_as_float(ra[i]), b = __uint_as_float(rb[i]);
+        va[i] = (a * cc[e] - b * sv[e]) * rs;
+        vb[i] = (a * sv[e] + b * cc[e]) * rs;
+      }
+    }
+    if (row < M) {
+      store16<F16, 32>(out + c * 32, va);
+      store16<F16, 32>(out + HD / 2 + c * 32, vb);
+    }
+  }
+}
+
+// EPI: epilogue; F16: operands (and 16-bit outputs) fp16 instead of bf16;
+// HD: head size of the EPI_QKV_ROPE epilogue (0 otherwise).
+template <int EPI, bool F16, int HD>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 int M, int N, int K, EpiParams ep, uint32_t* dev_status, uint64_t limit_ns) {
+  constexpr uint32_t IDESC = F16 ? IDESC_F16 : IDESC_BF16;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* tiles = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~static_cast<uintptr_t>(1023));
@@ -237,7 +342,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           for (int k = 0; k < BK / 16; ++k) {
             const uint64_t adesc = sw128_kmajor_desc(a_addr + k * 32);
             const uint64_t bdesc = sw128_kmajor_desc(b_addr + k * 32);
-            umma_bf16(d_tmem, adesc, bdesc, IDESC, (kb | k) != 0 ? 1u : 0u);
+            umma_f16(d_tmem, adesc, bdesc, IDESC, (kb | k) != 0 ? 1u : 0u);
           }
           umma_commit(smem_u32(&sm->empty[stage]));
           if (++stage == STAGES) {
@@ -278,14 +383,23 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       if constexpr (EPI == EPI_CE_PARTIAL) {
         if (row < M) target = ep.targets ? ep.targets[row] : -1;
       }
+      if constexpr (EPI == EPI_QKV_ROPE) {
 #pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c) {
-        const int col0 = n0 + c * 32;
-        if (col0 >= N) break;  // warp-uniform
-        uint32_t r[32];
-        tmem_ld_32x32b_x32(taddr + c * 32, r);
-        tmem_wait_ld();
-        if (row < M) epilogue_chunk<EPI>(r, row, col0, N, ep, ce_sum, ce_tl, target);
+        for (int hh = 0; hh < BN / HD; ++hh) {
+          const int col0 = n0 + hh * HD;
+          if (col0 >= N) break;  // warp-uniform
+          epilogue_qkv_head<F16, HD>(taddr + hh * HD, row, col0, M, ep);
+        }
+      } else {
+#pragma unroll 1
+        for (int c = 0; c < BN / 32; ++c) {
+          const int col0 = n0 + c * 32;
+          if (col0 >= N) break;  // warp-uniform
+          uint32_t r[32];
+          tmem_ld_32x32b_x32(taddr + c * 32, r);
+          tmem_wait_ld();
+          if (row < M) epilogue_chunk<EPI, F16>(r, row, col0, ep, ce_sum, ce_tl, target);
+        }
       }
       if constexpr (EPI == EPI_CE_PARTIAL) {
         if (row < M) {
@@ -329,22 +443,23 @@ static EncodeTiledFn get_encode_fn() {
   return fn;
 }
 
-// bf16 row-major [rows, cols] with row stride `ld` elements; box = 64 x box_rows.
+// 16-bit row-major [rows, cols] with row stride `ld` elements; box = 64 x box_rows.
 static bool make_map(CUtensorMap* map, const void* ptr, int64_t rows, int64_t cols, int64_t ld,
-                     int box_rows) {
+                     int box_rows, bool f16) {
   EncodeTiledFn enc = get_encode_fn();
   if (!enc) return false;
   cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
   cuuint64_t strides[1] = {(cuuint64_t)(ld * 2)};
   cuuint32_t box[2] = {(cuuint32_t)BK, (cuuint32_t)box_rows};
   cuuint32_t estr[2] = {1, 1};
-  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides,
-                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  CUresult r = enc(map, f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                   const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
 
-template <int EPI>
+template <int EPI, bool F16, int HD>
 static cudaError_t launch_t(const CUtensorMap& ma, const CUtensorMap& mb, int M, int N, int K,
                             const EpiParams& ep, uint32_t* dev_status, uint64_t limit_ns,
                             cudaStream_t stream) {
@@ -352,17 +467,34 @@ static cudaError_t launch_t(const CUtensorMap& ma, const CUtensorMap& mb, int M,
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 64 && !attr_done[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_kernel<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         SMEM_BYTES);
+    cudaError_t e = cudaFuncSetAttribute(gemm_kernel<EPI, F16, HD>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
     if (e != cudaSuccess) return e;
     attr_done[dev] = true;
   }
   const int tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
   const int sms = device_sm_count();
   const int grid = tiles < sms ? tiles : sms;
-  gemm_kernel<EPI><<<grid, NUM_THREADS, SMEM_BYTES, stream>>>(ma, mb, M, N, K, ep, dev_status,
-                                                              limit_ns);
+  gemm_kernel<EPI, F16, HD><<<grid, NUM_THREADS, SMEM_BYTES, stream>>>(ma, mb, M, N, K, ep,
+                                                                       dev_status, limit_ns);
   return cudaGetLastError();
+}
+
+template <bool F16>
+static cudaError_t dispatch(int epi, const CUtensorMap& ma, const CUtensorMap& mb, int M, int N, int K,
+                            const EpiParams& ep, uint32_t* st, uint64_t lim, cudaStream_t s) {
+  switch (epi) {
+    case EPI_STORE_16: return launch_t<EPI_STORE_16, F16, 0>(ma, mb, M, N, K, ep, st, lim, s);
+    case EPI_RELU2_16: return launch_t<EPI_RELU2_16, F16, 0>(ma, mb, M, N, K, ep, st, lim, s);
+    case EPI_RESID_F32: return launch_t<EPI_RESID_F32, F16, 0>(ma, mb, M, N, K, ep, st, lim, s);
+    case EPI_STORE_F32: return launch_t<EPI_STORE_F32, F16, 0>(ma, mb, M, N, K, ep, st, lim, s);
+    case EPI_SOFTCAP_F32: return launch_t<EPI_SOFTCAP_F32, F16, 0>(ma, mb, M, N, K, ep, st, lim, s);
+    case EPI_CE_PARTIAL: return launch_t<EPI_CE_PARTIAL, F16, 0>(ma, mb, M, N, K, ep, st, lim, s);
+    case EPI_QKV_ROPE:
+      return ep.D == 128 ? launch_t<EPI_QKV_ROPE, F16, 128>(ma, mb, M, N, K, ep, st, lim, s)
+                         : launch_t<EPI_QKV_ROPE, F16, 64>(ma, mb, M, N, K, ep, st, lim, s);
+    default: return cudaErrorInvalidValue;
+  }
 }
 
 // One thread waits for a phase that never completes; the bounded wait gives
@@ -393,22 +525,16 @@ nc_status selftest_wait_launch(uint32_t* dev_status, uint64_t limit_ns, cudaStre
 int gemm_num_n_tiles(int N) { return (N + gemm::BN - 1) / gemm::BN; }
 
 nc_status gemm_launch(const uint16_t* a, int64_t lda, const uint16_t* w, int64_t ldw, int M, int N,
-                      int K, int epi, const EpiParams& ep, uint32_t* dev_status,
+                      int K, int epi, bool f16, const EpiParams& ep, uint32_t* dev_status,
                       cudaStream_t stream, uint64_t limit_ns) {
   using namespace gemm;
+  if (epi < EPI_STORE_16 || epi > EPI_QKV_ROPE) return NC_ERR_INVALID_ARG;
+  if (epi == EPI_QKV_ROPE && (ep.D != 64 && ep.D != 128)) return NC_ERR_SHAPE;
   CUtensorMap ma, mb;
-  if (!make_map(&ma, a, M, K, lda, BM)) return NC_ERR_CUDA;
-  if (!make_map(&mb, w, N, K, ldw, BN)) return NC_ERR_CUDA;
-  cudaError_t e;
-  switch (epi) {
-    case EPI_STORE_BF16: e = launch_t<EPI_STORE_BF16>(ma, mb, M, N, K, ep, dev_status, limit_ns, stream); break;
-    case EPI_RELU2_BF16: e = launch_t<EPI_RELU2_BF16>(ma, mb, M, N, K, ep, dev_status, limit_ns, stream); break;
-    case EPI_RESID_F32: e = launch_t<EPI_RESID_F32>(ma, mb, M, N, K, ep, dev_status, limit_ns, stream); break;
-    case EPI_STORE_F32: e = launch_t<EPI_STORE_F32>(ma, mb, M, N, K, ep, dev_status, limit_ns, stream); break;
-    case EPI_SOFTCAP_F32: e = launch_t<EPI_SOFTCAP_F32>(ma, mb, M, N, K, ep, dev_status, limit_ns, stream); break;
-    case EPI_CE_PARTIAL: e = launch_t<EPI_CE_PARTIAL>(ma, mb, M, N, K, ep, dev_status, limit_ns, stream); break;
-    default: return NC_ERR_INVALID_ARG;
-  }
+  if (!make_map(&ma, a, M, K, lda, BM, f16)) return NC_ERR_CUDA;
+  if (!make_map(&mb, w, N, K, ldw, BN, f16)) return NC_ERR_CUDA;
+  const cudaError_t e = f16 ? dispatch<true>(epi, ma, mb, M, N, K, ep, dev_status, limit_ns, stream)
+                            : dispatch<false>(epi, ma, mb, M, N, K, ep, dev_status, limit_ns, stream);
   return e == cudaSuccess ? NC_OK : NC_ERR_CUDA;
 }
 

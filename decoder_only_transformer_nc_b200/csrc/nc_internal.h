@@ -14,22 +14,27 @@ constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
 // Epilogue selectors of the GEMM (the first five equal nc_epilogue).
 enum : int {
-  EPI_STORE_BF16 = NC_EPI_STORE_BF16,
-  EPI_RELU2_BF16 = NC_EPI_RELU2_BF16,
+  EPI_STORE_16 = NC_EPI_STORE_16,
+  EPI_RELU2_16 = NC_EPI_RELU2_16,
   EPI_RESID_F32 = NC_EPI_RESID_F32,
   EPI_STORE_F32 = NC_EPI_STORE_F32,
   EPI_SOFTCAP_F32 = NC_EPI_SOFTCAP_F32,
-  EPI_CE_PARTIAL = 5,  // soft-cap, per-tile sum of exp(l - cap), target logit
+  EPI_CE_PARTIAL = 5,   // soft-cap, per-tile sum of exp(l - cap), target logit
+  EPI_QKV_ROPE = 6,     // q/k heads: RoPE + per-head RMSNorm; v heads: plain store
 };
 
 struct EpiParams {
-  void* out;                // bf16 or fp32 output (or logits for EPI_CE_PARTIAL)
+  void* out;                // 16-bit or fp32 output (or logits for EPI_CE_PARTIAL)
   int64_t ldo;              // output row stride in elements
   float cap;                // soft-cap
   int store_logits;         // EPI_CE_PARTIAL: also write capped logits to out
   float* ce_partial;        // EPI_CE_PARTIAL: [M, gemm_num_n_tiles(N)]
   float* ce_target;         // EPI_CE_PARTIAL: [M], l[m, y_m] (written by one tile)
   const int32_t* targets;   // EPI_CE_PARTIAL: [M]
+  const float* rope;        // EPI_QKV_ROPE: [2][T][D/2] cos, sin
+  int T;                    // EPI_QKV_ROPE: positions per sequence (row m is at m % T)
+  int H, Hkv, D;            // EPI_QKV_ROPE: head counts and head size
+  float eps;                // EPI_QKV_ROPE: RMSNorm epsilon
 };
 
 // ---- device / argument helpers (nc_api.cu)
@@ -39,8 +44,10 @@ inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 
 // ---- GEMM (nc_gemm.cu)
 int gemm_num_n_tiles(int N);
+// a [M, K] (row stride lda) and w [N, K] (row stride ldw) are 16-bit in format
+// `f16` (true: fp16, false: bf16); 16-bit outputs use the same format.
 nc_status gemm_launch(const uint16_t* a, int64_t lda, const uint16_t* w, int64_t ldw, int M, int N,
-                      int K, int epi, const EpiParams& ep, uint32_t* dev_status,
+                      int K, int epi, bool f16, const EpiParams& ep, uint32_t* dev_status,
                       cudaStream_t stream, uint64_t limit_ns = kWaitLimitNs);
 
 nc_status selftest_wait_launch(uint32_t* dev_status, uint64_t limit_ns, cudaStream_t stream);
@@ -48,7 +55,7 @@ nc_status selftest_wait_launch(uint32_t* dev_status, uint64_t limit_ns, cudaStre
 // ---- attention (nc_attention.cu)
 nc_status attention_launch(const uint16_t* q, const uint16_t* k, const uint16_t* v, uint16_t* out,
                            int B, int T, int H, int Hkv, int D, int window, int64_t q_stride,
-                           int64_t kv_stride, cudaStream_t stream);
+                           int64_t kv_stride, bool f16, cudaStream_t stream);
 
 // ---- elementwise / row kernels (nc_rowops.cu)
 struct CastSeg {
@@ -56,14 +63,15 @@ struct CastSeg {
   uint16_t* dst;
   int64_t n;  // multiple of 8
 };
-nc_status cast_launch(const CastSeg* segs, int nseg, cudaStream_t stream);
+// fp32 -> bf16 (round to nearest even); with f16 the bf16 value is stored as fp16.
+nc_status cast_launch(const CastSeg* segs, int nseg, bool f16, cudaStream_t stream);
 nc_status embedding_launch(const int32_t* tokens, const float* wte, float* x, int M, int C, int V,
                            uint32_t* dev_status, cudaStream_t stream);
-nc_status rmsnorm_launch(const float* x, uint16_t* out, int M, int C, float eps,
+nc_status rmsnorm_launch(const float* x, uint16_t* out, int M, int C, float eps, bool f16,
                          cudaStream_t stream);
 nc_status rope_table_launch(float* table, int T, int D, float base, cudaStream_t stream);
 nc_status rope_qknorm_launch(uint16_t* q, uint16_t* k, const float* table, int B, int T, int H,
-                             int Hkv, int D, int64_t q_stride, int64_t k_stride, float eps,
+                             int Hkv, int D, int64_t q_stride, int64_t k_stride, float eps, bool f16,
                              cudaStream_t stream);
 nc_status softcap_ce_launch(const float* z, const int32_t* targets, float* capped_out,
                             float* token_loss, int M, int V, float cap, uint32_t* dev_status,

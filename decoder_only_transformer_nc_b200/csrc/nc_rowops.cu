@@ -9,6 +9,7 @@
 #include <cmath>
 #include <cstdint>
 
+#include "nc_half.cuh"
 #include "nc_internal.h"
 
 namespace nc {
@@ -18,16 +19,6 @@ __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
   return v;
-}
-
-__device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
-  __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
-  return *reinterpret_cast<uint32_t*>(&h);
-}
-
-__device__ __forceinline__ float2 unpack_bf16x2(uint32_t u) {
-  __nv_bfloat162 h = *reinterpret_cast<__nv_bfloat162*>(&u);
-  return __bfloat1622float2(h);
 }
 
 // ---------------------------------------------------------------- weight cast
@@ -40,6 +31,22 @@ struct CastBatch {
   int nseg;
 };
 
+// Each fp32 weight is rounded to bf16 (nearest even).  With F16 that bf16
+// value is then stored in an fp16 container: exact for |w| >= 2^-14 (every
+// bf16 value with 8 significant bits fits fp16's 11), nearest fp16 subnormal
+// below that (absolute change <= 2^-25).
+template <bool F16>
+__device__ __forceinline__ uint32_t cast_pair(float a, float b) {
+  if constexpr (F16) {
+    const float ra = __bfloat162float(__float2bfloat16_rn(a));
+    const float rb = __bfloat162float(__float2bfloat16_rn(b));
+    return Half<true>::pack2(ra, rb);
+  } else {
+    return Half<false>::pack2(a, b);
+  }
+}
+
+template <bool F16>
 __global__ void __launch_bounds__(256) cast_kernel(const __grid_constant__ CastBatch cb) {
   const int64_t total = cb.gstart[cb.nseg];
   for (int64_t g = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; g < total;
@@ -54,10 +61,10 @@ __global__ void __launch_bounds__(256) cast_kernel(const __grid_constant__ CastB
     const float4 a = __ldcs(s);
     const float4 b = __ldcs(s + 1);
     uint4 o;
-    o.x = pack_bf16x2(a.x, a.y);
-    o.y = pack_bf16x2(a.z, a.w);
-    o.z = pack_bf16x2(b.x, b.y);
-    o.w = pack_bf16x2(b.z, b.w);
+    o.x = cast_pair<F16>(a.x, a.y);
+    o.y = cast_pair<F16>(a.z, a.w);
+    o.z = cast_pair<F16>(b.x, b.y);
+    o.w = cast_pair<F16>(b.z, b.w);
     *reinterpret_cast<uint4*>(cb.dst[lo] + off) = o;
   }
 }
@@ -84,7 +91,7 @@ __global__ void __launch_bounds__(256) embedding_kernel(const int32_t* __restric
 // ---------------------------------------------------------------- RMSNorm
 
 // One warp per row; the row is held in registers (C <= 32 * 4 * NV).
-template <int NV>
+template <int NV, bool F16>
 __global__ void __launch_bounds__(256) rmsnorm_kernel(const float* __restrict__ x,
                                                       uint16_t* __restrict__ out, int M, int C,
                                                       float eps) {
@@ -107,11 +114,13 @@ __global__ void __launch_bounds__(256) rmsnorm_kernel(const float* __restrict__ 
 #pragma unroll
   for (int j = 0; j < NV; ++j) {
     const int i = j * 32 + lane;
-    if (i < n4) o[i] = make_uint2(pack_bf16x2(v[j].x * r, v[j].y * r), pack_bf16x2(v[j].z * r, v[j].w * r));
+    if (i < n4)
+      o[i] = make_uint2(Half<F16>::pack2(v[j].x * r, v[j].y * r), Half<F16>::pack2(v[j].z * r, v[j].w * r));
   }
 }
 
 // Two-pass variant for wide rows.
+template <bool F16>
 __global__ void __launch_bounds__(256) rmsnorm_wide_kernel(const float* __restrict__ x,
                                                            uint16_t* __restrict__ out, int M, int C,
                                                            float eps) {
@@ -130,7 +139,7 @@ __global__ void __launch_bounds__(256) rmsnorm_wide_kernel(const float* __restri
   uint2* o = reinterpret_cast<uint2*>(out + (int64_t)row * C);
   for (int i = lane; i < n4; i += 32) {
     const float4 a = xr[i];
-    o[i] = make_uint2(pack_bf16x2(a.x * r, a.y * r), pack_bf16x2(a.z * r, a.w * r));
+    o[i] = make_uint2(Half<F16>::pack2(a.x * r, a.y * r), Half<F16>::pack2(a.z * r, a.w * r));
   }
 }
 
@@ -152,7 +161,7 @@ __global__ void rope_table_kernel(float* __restrict__ table, int T, int D, doubl
 // bf16 pairs at dims (2l, 2l+1) and (D/2+2l, D/2+2l+1), i.e. both members of
 // the RoPE pairs 2l and 2l+1, so the rotation needs no shuffles; the per-head
 // sum of squares is a shuffle reduction inside the group.
-template <int D>
+template <int D, bool F16>
 __global__ void __launch_bounds__(256) rope_qknorm_kernel(uint16_t* __restrict__ q,
                                                           uint16_t* __restrict__ k,
                                                           const float* __restrict__ table, int M,
@@ -171,8 +180,8 @@ __global__ void __launch_bounds__(256) rope_qknorm_kernel(uint16_t* __restrict__
   uint16_t* p = j < H ? q + m * q_stride + (int64_t)j * D : k + m * k_stride + (int64_t)(j - H) * D;
   float ra0 = 0.f, ra1 = 0.f, rb0 = 0.f, rb1 = 0.f;
   if (active) {
-    const float2 a = unpack_bf16x2(*reinterpret_cast<const uint32_t*>(p + 2 * l));
-    const float2 b = unpack_bf16x2(*reinterpret_cast<const uint32_t*>(p + HALF + 2 * l));
+    const float2 a = Half<F16>::unpack2(*reinterpret_cast<const uint32_t*>(p + 2 * l));
+    const float2 b = Half<F16>::unpack2(*reinterpret_cast<const uint32_t*>(p + HALF + 2 * l));
     const float2 c = *reinterpret_cast<const float2*>(table + (int64_t)t * HALF + 2 * l);
     const float2 s = *reinterpret_cast<const float2*>(table + (int64_t)T * HALF + (int64_t)t * HALF + 2 * l);
     ra0 = a.x * c.x - b.x * s.x;
@@ -185,8 +194,8 @@ __global__ void __launch_bounds__(256) rope_qknorm_kernel(uint16_t* __restrict__
   for (int o = LPH / 2; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
   if (active) {
     const float r = rsqrtf(ss / (float)D + eps);
-    *reinterpret_cast<uint32_t*>(p + 2 * l) = pack_bf16x2(ra0 * r, ra1 * r);
-    *reinterpret_cast<uint32_t*>(p + HALF + 2 * l) = pack_bf16x2(rb0 * r, rb1 * r);
+    *reinterpret_cast<uint32_t*>(p + 2 * l) = Half<F16>::pack2(ra0 * r, ra1 * r);
+    *reinterpret_cast<uint32_t*>(p + HALF + 2 * l) = Half<F16>::pack2(rb0 * r, rb1 * r);
   }
 }
 
@@ -209,6 +218,25 @@ __device__ __forceinline__ float block_sum(float v, float* red) {
   return r;
 }
 
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ float rcp_approx(float x) {
+  float y;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// l = cap * tanh(z / cap) = cap - 2 cap r with r = 1 / (1 + e^(2z/cap)), and
+// exp(l - cap) = e^(-2 cap r): three MUFU operations per logit, exact limits.
+__device__ __forceinline__ float softcap_p(float z, float k_in, float cap, float k_out, float& p) {
+  const float r = rcp_approx(1.0f + ex2_approx(z * k_in));
+  p = ex2_approx(k_out * r);
+  return fmaf(-2.0f * cap, r, cap);
+}
+
 // One CTA per row.  Soft-capped logits lie in (-cap, cap), so
 // logsumexp(l) = cap + log(sum exp(l - cap)) needs no running maximum.
 __global__ void __launch_bounds__(256) softcap_ce_kernel(const float* __restrict__ z,
@@ -220,15 +248,17 @@ __global__ void __launch_bounds__(256) softcap_ce_kernel(const float* __restrict
   const int64_t row = blockIdx.x;
   const float4* zr = reinterpret_cast<const float4*>(z + row * V);
   float4* cr = capped_out ? reinterpret_cast<float4*>(capped_out + row * V) : nullptr;
-  const float inv = 1.0f / cap;
+  const float k_in = 2.0f * 1.4426950408889634f / cap;
+  const float k_out = -2.0f * cap * 1.4426950408889634f;
   float s = 0.0f;
   for (int i = threadIdx.x; i < V / 4; i += blockDim.x) {
     float4 a = __ldcs(zr + i);
-    a.x = cap * tanhf(a.x * inv);
-    a.y = cap * tanhf(a.y * inv);
-    a.z = cap * tanhf(a.z * inv);
-    a.w = cap * tanhf(a.w * inv);
-    s += __expf(a.x - cap) + __expf(a.y - cap) + __expf(a.z - cap) + __expf(a.w - cap);
+    float p0, p1, p2, p3;
+    a.x = softcap_p(a.x, k_in, cap, k_out, p0);
+    a.y = softcap_p(a.y, k_in, cap, k_out, p1);
+    a.z = softcap_p(a.z, k_in, cap, k_out, p2);
+    a.w = softcap_p(a.w, k_in, cap, k_out, p3);
+    s += (p0 + p1) + (p2 + p3);
     if (cr) cr[i] = a;
   }
   s = block_sum(s, red);
@@ -236,7 +266,8 @@ __global__ void __launch_bounds__(256) softcap_ce_kernel(const float* __restrict
     const int y = targets[row];
     float nll = 0.0f;
     if (y >= 0 && y < V) {
-      const float ly = cap * tanhf(z[row * V + y] * inv);
+      float unused;
+      const float ly = softcap_p(z[row * V + y], k_in, cap, k_out, unused);
       nll = cap + logf(s) - ly;
     } else if (y != -1 && dev_status) {
       atomicOr(dev_status, NC_DEV_TARGET_RANGE);
@@ -315,7 +346,7 @@ inline nc_status last_error() { return cudaGetLastError() == cudaSuccess ? NC_OK
 
 }  // namespace
 
-nc_status cast_launch(const CastSeg* segs, int nseg, cudaStream_t stream) {
+nc_status cast_launch(const CastSeg* segs, int nseg, bool f16, cudaStream_t stream) {
   for (int base = 0; base < nseg; base += kMaxCastSegs) {
     CastBatch cb;
     cb.nseg = nseg - base < kMaxCastSegs ? nseg - base : kMaxCastSegs;
@@ -329,7 +360,10 @@ nc_status cast_launch(const CastSeg* segs, int nseg, cudaStream_t stream) {
     if (groups == 0) continue;
     const int64_t want = (groups + 255) / 256;
     const int grid = (int)(want < 148 * 16 ? want : 148 * 16);
-    cast_kernel<<<grid, 256, 0, stream>>>(cb);
+    if (f16)
+      cast_kernel<true><<<grid, 256, 0, stream>>>(cb);
+    else
+      cast_kernel<false><<<grid, 256, 0, stream>>>(cb);
     if (cudaGetLastError() != cudaSuccess) return NC_ERR_CUDA;
   }
   return NC_OK;
@@ -343,18 +377,27 @@ nc_status embedding_launch(const int32_t* tokens, const float* wte, float* x, in
   return last_error();
 }
 
-nc_status rmsnorm_launch(const float* x, uint16_t* out, int M, int C, float eps,
-                         cudaStream_t stream) {
-  if (M == 0) return NC_OK;
+template <bool F16>
+static void rmsnorm_dispatch(const float* x, uint16_t* out, int M, int C, float eps,
+                             cudaStream_t stream) {
   const int grid = (M + 7) / 8;
   if (C <= 32 * 4 * 4)
-    rmsnorm_kernel<4><<<grid, 256, 0, stream>>>(x, out, M, C, eps);
+    rmsnorm_kernel<4, F16><<<grid, 256, 0, stream>>>(x, out, M, C, eps);
   else if (C <= 32 * 4 * 8)
-    rmsnorm_kernel<8><<<grid, 256, 0, stream>>>(x, out, M, C, eps);
+    rmsnorm_kernel<8, F16><<<grid, 256, 0, stream>>>(x, out, M, C, eps);
   else if (C <= 32 * 4 * 16)
-    rmsnorm_kernel<16><<<grid, 256, 0, stream>>>(x, out, M, C, eps);
+    rmsnorm_kernel<16, F16><<<grid, 256, 0, stream>>>(x, out, M, C, eps);
   else
-    rmsnorm_wide_kernel<<<grid, 256, 0, stream>>>(x, out, M, C, eps);
+    rmsnorm_wide_kernel<F16><<<grid, 256, 0, stream>>>(x, out, M, C, eps);
+}
+
+nc_status rmsnorm_launch(const float* x, uint16_t* out, int M, int C, float eps, bool f16,
+                         cudaStream_t stream) {
+  if (M == 0) return NC_OK;
+  if (f16)
+    rmsnorm_dispatch<true>(x, out, M, C, eps, stream);
+  else
+    rmsnorm_dispatch<false>(x, out, M, C, eps, stream);
   return last_error();
 }
 
@@ -366,18 +409,20 @@ nc_status rope_table_launch(float* table, int T, int D, float base, cudaStream_t
 }
 
 nc_status rope_qknorm_launch(uint16_t* q, uint16_t* k, const float* table, int B, int T, int H,
-                             int Hkv, int D, int64_t q_stride, int64_t k_stride, float eps,
+                             int Hkv, int D, int64_t q_stride, int64_t k_stride, float eps, bool f16,
                              cudaStream_t stream) {
   const int64_t M = (int64_t)B * T;
   const int64_t threads = M * (H + Hkv) * (D / 4);
   if (threads == 0) return NC_OK;
-  const int64_t grid = (threads + 255) / 256;
-  if (D == 128)
-    rope_qknorm_kernel<128><<<(unsigned)grid, 256, 0, stream>>>(q, k, table, (int)M, T, H, Hkv,
-                                                                q_stride, k_stride, eps);
+  const unsigned grid = (unsigned)((threads + 255) / 256);
+  if (D == 128 && f16)
+    rope_qknorm_kernel<128, true><<<grid, 256, 0, stream>>>(q, k, table, (int)M, T, H, Hkv, q_stride, k_stride, eps);
+  else if (D == 128)
+    rope_qknorm_kernel<128, false><<<grid, 256, 0, stream>>>(q, k, table, (int)M, T, H, Hkv, q_stride, k_stride, eps);
+  else if (D == 64 && f16)
+    rope_qknorm_kernel<64, true><<<grid, 256, 0, stream>>>(q, k, table, (int)M, T, H, Hkv, q_stride, k_stride, eps);
   else if (D == 64)
-    rope_qknorm_kernel<64><<<(unsigned)grid, 256, 0, stream>>>(q, k, table, (int)M, T, H, Hkv,
-                                                               q_stride, k_stride, eps);
+    rope_qknorm_kernel<64, false><<<grid, 256, 0, stream>>>(q, k, table, (int)M, T, H, Hkv, q_stride, k_stride, eps);
   else
     return NC_ERR_SHAPE;
   return last_error();

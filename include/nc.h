@@ -19,7 +19,8 @@
  *   - All tensor pointers are DEVICE pointers of the current CUDA device unless
  *     a parameter says "host".  The caller owns every buffer; the library
  *     allocates no device memory and frees nothing.
- *   - bf16 tensors are passed as uint16_t* holding bfloat16 bit patterns.
+ *   - 16-bit tensors are uint16_t* holding bfloat16 or IEEE fp16 bit patterns, as
+ *     the call's nc_dtype argument says.
  *   - Matrices are row-major.  Weights use the [out_features, in_features]
  *     layout of a bias-free linear layer, so y = x W^T.
  *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Work is
@@ -58,6 +59,12 @@ typedef enum {
   NC_ERR_CUDA = 9                /* a CUDA runtime call failed               */
 } nc_status;
 
+/* 16-bit storage formats. */
+typedef enum {
+  NC_BF16 = 0, /* bfloat16: 8 significant bits, fp32 range                     */
+  NC_F16 = 1   /* IEEE binary16: 11 significant bits, |x| <= 65504 (saturating) */
+} nc_dtype;
+
 /* Bits of the device status word. */
 #define NC_DEV_TOKEN_RANGE 0x1u  /* a token id was outside [0, V): row 0 used  */
 #define NC_DEV_TARGET_RANGE 0x2u /* a target was outside {-1} U [0, V): ignored */
@@ -80,6 +87,12 @@ typedef struct {
   float softcap;             /* logits = softcap * tanh(z / softcap), 15      */
   float norm_eps;            /* RMSNorm epsilon, 1e-6                         */
   float rope_base;           /* RoPE base, 10000                              */
+  int32_t act_dtype;         /* nc_dtype of activations and matmul operands:
+                                NC_F16 (default) or NC_BF16.  Weights always
+                                enter the matmuls as their bf16 (round to
+                                nearest even) values; with NC_F16 those values
+                                are held in fp16 (exact for |w| >= 2^-14) so
+                                both tensor-core operands share one format. */
 } nc_config;
 
 /* fp32 master weights (device pointers; the per-layer members are HOST arrays
@@ -100,7 +113,8 @@ typedef struct {
 /* Fills *out from the depth knob ("从文本到聊天模型" §5.1): d_model =
  * depth*aspect_ratio, n_head = d_model/head_dim, n_kv_head = n_kv_head or
  * n_head when 0, pattern "SSSL", short_window = seq_len/4, softcap 15,
- * norm_eps 1e-6, rope_base 10000.  Host only; touches no device. */
+ * norm_eps 1e-6, rope_base 10000, act_dtype NC_F16.  Host only; touches no
+ * device. */
 nc_status nc_init_config(nc_config* out, int depth, int aspect_ratio, int head_dim,
                          int n_kv_head, int seq_len, int vocab);
 
@@ -192,18 +206,23 @@ nc_status nc_get_status(const void* dev_status, void* stream);
 
 /* ---------------------------------------------------------------- single steps */
 
-/* fp32 -> bf16 (round to nearest even) of n elements; n % 8 == 0. */
-nc_status nc_cast_bf16(const float* src, uint16_t* dst, int64_t n, void* stream);
+/* Weight cast ("约100美元训出对话模型": fp32 weights converted to bf16 for the
+ * matmul): each of n fp32 values is rounded to bf16 (nearest, ties to even).
+ * container NC_BF16 stores the bf16 bits; NC_F16 stores that bf16 value as fp16
+ * (exact for |w| >= 2^-14, nearest fp16 subnormal below).  n % 8 == 0. */
+nc_status nc_cast_weights(const float* src, uint16_t* dst, int64_t n, nc_dtype container,
+                          void* stream);
 
 /* x[m, :] = wte[tokens[m], :] for m < M ("从文本到聊天模型" §5.2).
  * x [M, C] fp32; wte [V, C] fp32.  Bad ids set NC_DEV_TOKEN_RANGE and read row 0. */
 nc_status nc_embedding(const int32_t* tokens, const float* wte, float* x, int M, int C, int V,
                        uint32_t* dev_status, void* stream);
 
-/* out[m, :] = bf16( x[m, :] / sqrt(mean(x[m, :]^2) + eps) ), parameter-free
- * RMSNorm ("Nanochat与nanoGPT对比" §1).  x [M, C] fp32, out [M, C] bf16;
+/* out[m, :] = x[m, :] / sqrt(mean(x[m, :]^2) + eps), parameter-free RMSNorm
+ * ("Nanochat与nanoGPT对比" §1).  x [M, C] fp32, out [M, C] 16-bit (dtype);
  * C % 8 == 0. */
-nc_status nc_rmsnorm(const float* x, uint16_t* out, int M, int C, float eps, void* stream);
+nc_status nc_rmsnorm(const float* x, uint16_t* out, int M, int C, float eps, nc_dtype dtype,
+                     void* stream);
 
 /* RoPE angle table: table[0][t][i] = cos(t * base^(-2i/D)),
  * table[1][t][i] = sin(...), fp32, t < T, i < D/2 (angles in fp64). */
@@ -211,45 +230,59 @@ nc_status nc_rope_table(float* table, int T, int D, float base, void* stream);
 
 /* In place: q <- rmsnorm(rope(q)), k <- rmsnorm(rope(k)) per head over D
  * ("从文本到聊天模型" §5.6; "Nanochat与nanoGPT对比" §1: QK-norm after RoPE).
- * q [B, T, H, D] bf16 with q_row_stride elements between consecutive tokens
- * (H*D when contiguous); k [B, T, Hkv, D] with k_row_stride.  Pair
- * (u_i, u_{i+D/2}) of the token at position t is rotated by t * theta_i,
- * table from nc_rope_table.  D in {64, 128}. */
+ * q [B, T, H, D] 16-bit (dtype) with q_row_stride elements between
+ * consecutive tokens (H*D when contiguous); k [B, T, Hkv, D] with
+ * k_row_stride.  Pair (u_i, u_{i+D/2}) of the token at position t is rotated by
+ * t * theta_i, table from nc_rope_table.  D in {64, 128}. */
 nc_status nc_rope_qknorm(uint16_t* q, uint16_t* k, const float* table, int B, int T, int H,
                          int Hkv, int D, int64_t q_row_stride, int64_t k_row_stride, float eps,
-                         void* stream);
+                         nc_dtype dtype, void* stream);
 
 /* Causal sliding-window attention with GQA ("从文本到聊天模型" §5.4-5.5):
  * out[b,i,h,:] = sum_j softmax_j(q[b,i,h,:].k[b,j,g,:] / sqrt(D)) v[b,j,g,:],
  * g = h / (H/Hkv), over keys j <= i with i - j < window (window <= 0 or
- * >= T: full causal).  q/out [B,T,H,D], k/v [B,T,Hkv,D], contiguous bf16.
- * D == 128. */
+ * >= T: full causal).  q/out [B,T,H,D], k/v [B,T,Hkv,D], contiguous 16-bit
+ * (dtype; the probabilities enter P.V in the same format).  D in {64, 128}. */
 nc_status nc_attention(const uint16_t* q, const uint16_t* k, const uint16_t* v, uint16_t* out,
-                       int B, int T, int H, int Hkv, int D, int window, void* stream);
+                       int B, int T, int H, int Hkv, int D, int window, nc_dtype dtype,
+                       void* stream);
 
 /* Same with explicit token strides (elements between consecutive tokens) for
  * q, k, v (e.g. the three column blocks of one fused [M, (H+2Hkv)D] buffer);
  * out is contiguous [B, T, H, D]. */
 nc_status nc_attention_strided(const uint16_t* q, const uint16_t* k, const uint16_t* v,
                                uint16_t* out, int B, int T, int H, int Hkv, int D, int window,
-                               int64_t q_row_stride, int64_t kv_row_stride, void* stream);
+                               int64_t q_row_stride, int64_t kv_row_stride, nc_dtype dtype,
+                               void* stream);
 
 /* Epilogues of nc_linear. */
 typedef enum {
-  NC_EPI_STORE_BF16 = 0,   /* out bf16 [M, ldo]: acc                             */
-  NC_EPI_RELU2_BF16 = 1,   /* out bf16: relu(acc)^2 ("从文本到聊天模型" §5.7)    */
+  NC_EPI_STORE_16 = 0,     /* out 16-bit (dtype) [M, ldo]: acc                   */
+  NC_EPI_RELU2_16 = 1,     /* out 16-bit: relu(acc)^2 ("从文本到聊天模型" §5.7)  */
   NC_EPI_RESID_F32 = 2,    /* out fp32: out += acc (residual add, §5.3)          */
   NC_EPI_STORE_F32 = 3,    /* out fp32: acc                                      */
   NC_EPI_SOFTCAP_F32 = 4   /* out fp32: cap * tanh(acc / cap)                    */
 } nc_epilogue;
 
-/* out = epilogue(a @ w^T): a [M, K] bf16 row-major, w [N, K] bf16 row-major,
- * out row stride ldo elements (>= N).  tcgen05 tensor cores, fp32 accumulation
- * in tensor memory.  K % 8 == 0, N % 32 == 0.  dev_status gets NC_DEV_TIMEOUT
- * if a pipeline wait ran out. */
+/* out = epilogue(a @ w^T): a [M, K] and w [N, K] row-major 16-bit, both in
+ * format dtype; 16-bit outputs use the same format.  out row stride ldo
+ * elements (>= N).  tcgen05 tensor cores, fp32 accumulation in tensor memory.
+ * K % 8 == 0, N % 32 == 0.  dev_status gets NC_DEV_TIMEOUT if a pipeline wait
+ * ran out. */
 nc_status nc_linear(const uint16_t* a, const uint16_t* w, void* out, int M, int N, int K,
-                    int64_t ldo, nc_epilogue epilogue, float cap, uint32_t* dev_status,
-                    void* stream);
+                    int64_t ldo, nc_epilogue epilogue, float cap, nc_dtype dtype,
+                    uint32_t* dev_status, void* stream);
+
+/* Fused Q/K/V projection ("从文本到聊天模型" §5.4) + RoPE + QK-norm
+ * ("Nanochat与nanoGPT对比" §1) in one GEMM: qkv = a @ w^T with w the
+ * [(H+2Hkv)*D, C] stack of c_q, c_k, c_v; in each token row the first H heads
+ * (q) and the next Hkv heads (k) are rotated (pair (u_i, u_{i+D/2}) of row m by
+ * (m % T) * theta_i, table from nc_rope_table) and RMS-normalised over D; the
+ * last Hkv heads (v) are stored as computed.  a [M, C], w, out [M, (H+2Hkv)*D]
+ * 16-bit in format dtype.  D in {64, 128}, C % 8 == 0. */
+nc_status nc_qkv_rope(const uint16_t* a, const uint16_t* w, uint16_t* out, const float* table,
+                      int M, int T, int C, int H, int Hkv, int D, float eps, nc_dtype dtype,
+                      uint32_t* dev_status, void* stream);
 
 /* Fused soft-cap + log-softmax + NLL over the vocabulary ("Nanochat与nanoGPT对比"
  * §1 soft-cap; "从文本到聊天模型" §5.8 cross-entropy, ignore_index -1):

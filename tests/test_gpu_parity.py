@@ -5,10 +5,11 @@ step consumes bf16, both sides get the same bf16-rounded values.  Tolerances:
 
 * whole forward (the published bar): max-abs logit error <= 3e-2 and relative
   loss error <= 5e-3; attention output max-abs <= 2e-2;
-* single steps, derived from the arithmetic: a bf16 output carries at most half
-  an ulp of rounding (2^-9 relative) on top of fp32 arithmetic, so it must sit
-  within 2^-8 * |x| (+ a small absolute term for fp32 table/accumulation error);
-  fp32 outputs of fp32 arithmetic within 1e-5 relative.
+* single steps, derived from the arithmetic: a 16-bit output carries at most
+  half an ulp of rounding (2^-9 relative for bf16, 2^-12 for fp16) on top of
+  fp32 arithmetic, so it must sit within twice that (2^-8, 2^-11) times |x|, plus
+  a small absolute term for fp32 table/accumulation error; fp32 outputs of fp32
+  arithmetic within 1e-5 relative.  Every single-step test runs in both formats.
 """
 import math
 
@@ -23,10 +24,23 @@ pytestmark = pytest.mark.gpu
 
 DEV = "cuda"
 BF16_REL = 2.0 ** -8
+REL = {"bf16": 2.0 ** -8, "f16": 2.0 ** -11}
+TDT = {"bf16": torch.bfloat16, "f16": torch.float16}
+DTYPES = ["f16", "bf16"]
 
 
 def bf16_dev(a):
     return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(DEV).to(torch.bfloat16)
+
+
+def round16(a, dt):
+    """float32 values rounded to the 16-bit format (nearest even), as float32."""
+    a = np.ascontiguousarray(a, dtype=np.float32)
+    return round_to_bf16(a) if dt == "bf16" else a.astype(np.float16).astype(np.float32)
+
+
+def dev16(a, dt):
+    return torch.from_numpy(round16(a, dt)).to(DEV).to(TDT[dt])
 
 
 def host(t):
@@ -37,25 +51,36 @@ def status_word():
     return torch.zeros(64, dtype=torch.int32, device=DEV)
 
 
-def assert_close_bf16(got, want, atol, what):
-    err = np.abs(got - want) - (BF16_REL * np.abs(want) + atol)
+def assert_close_bf16(got, want, atol, what, rel=BF16_REL):
+    err = np.abs(got - want) - (rel * np.abs(want) + atol)
     worst = float(err.max()) if err.size else -1.0
-    assert worst <= 0.0, f"{what}: exceeds bf16 bound by {worst:.3e} (max abs err {np.abs(got - want).max():.3e})"
+    assert worst <= 0.0, f"{what}: exceeds the 16-bit bound by {worst:.3e} (max abs err {np.abs(got - want).max():.3e})"
 
 
 # ---------------------------------------------------------------- single steps
 
-def test_cast_bf16_bit_exact(gpu):
+def test_cast_weights_bit_exact(gpu):
     rng = np.random.default_rng(1)
     a = (rng.standard_normal(100_000) * 10.0 ** rng.uniform(-30, 30, 100_000)).astype(np.float32)
     a[:8] = [0.0, -0.0, 1.0, -1.5, 3.0e38, -3.0e38, 1e-40, 65504.0]
     src = torch.from_numpy(a).to(DEV)
     dst = torch.empty(a.size, dtype=torch.bfloat16, device=DEV)
-    gpu.cast_bf16(src, dst)
+    gpu.cast_weights(src, dst)
     torch.cuda.synchronize()
     want = torch.from_numpy(a).to(torch.bfloat16)
     assert torch.equal(dst.cpu().view(torch.int16), want.view(torch.int16))
-    np.testing.assert_array_equal(dst.float().cpu().numpy(), round_to_bf16(a))
+    np.testing.assert_array_equal(dst.float().cpu().numpy(), oracle.to_bf16(a).astype(np.float32))
+    # fp16 container: the bf16 value, held exactly where fp16 can (|w| >= 2^-14)
+    w = (rng.standard_normal(100_000) * 0.02).astype(np.float32)
+    w[:4] = [1e-6, -3e-5, 7e-5, 0.0]
+    d16 = torch.empty(w.size, dtype=torch.float16, device=DEV)
+    gpu.cast_weights(torch.from_numpy(w).to(DEV), d16)
+    torch.cuda.synchronize()
+    want = oracle.to_bf16(w)
+    got = d16.cpu().numpy().astype(np.float64)
+    normal = np.abs(want) >= 2.0 ** -14
+    np.testing.assert_array_equal(got[normal], want[normal])
+    assert np.abs(got[~normal] - want[~normal]).max() <= 2.0 ** -25
 
 
 def test_embedding_exact_and_token_range(gpu):
@@ -75,15 +100,16 @@ def test_embedding_exact_and_token_range(gpu):
     np.testing.assert_array_equal(x[5].cpu().numpy(), wte[0])
 
 
+@pytest.mark.parametrize("dt", DTYPES)
 @pytest.mark.parametrize("C", [128, 768, 1280, 1664, 2048, 4096])
-def test_rmsnorm_parity(gpu, C):
+def test_rmsnorm_parity(gpu, C, dt):
     rng = np.random.default_rng(C)
     M = 1001
     x = (rng.standard_normal((M, C)) * rng.uniform(0.01, 30, (M, 1))).astype(np.float32)
-    out = torch.empty((M, C), dtype=torch.bfloat16, device=DEV)
+    out = torch.empty((M, C), dtype=TDT[dt], device=DEV)
     gpu.rmsnorm(torch.from_numpy(x).to(DEV), out, eps=1e-6)
     torch.cuda.synchronize()
-    assert_close_bf16(host(out), oracle.rms_norm(x, 1e-6), 1e-6, f"rmsnorm C={C}")
+    assert_close_bf16(host(out), oracle.rms_norm(x, 1e-6), 1e-6, f"rmsnorm C={C}", rel=2 * REL[dt])
 
 
 @pytest.mark.parametrize("T,D", [(300, 64), (2048, 128), (8192, 128)])
@@ -96,45 +122,48 @@ def test_rope_table(gpu, T, D):
     np.testing.assert_allclose(tab[1].cpu().numpy(), sin, atol=6e-8, rtol=0)
 
 
+@pytest.mark.parametrize("dt", DTYPES)
 @pytest.mark.parametrize("D,H,Hkv,fused", [(64, 4, 2, False), (128, 4, 4, False), (128, 6, 2, True),
                                            (128, 10, 10, True)])
-def test_rope_qknorm_parity(gpu, D, H, Hkv, fused):
+def test_rope_qknorm_parity(gpu, D, H, Hkv, fused, dt):
     rng = np.random.default_rng(D + H + Hkv)
     B, T = 2, 301
-    q = round_to_bf16((rng.standard_normal((B, T, H, D)) * 3).astype(np.float32))
-    k = round_to_bf16((rng.standard_normal((B, T, Hkv, D)) * 0.2).astype(np.float32))
+    q = round16((rng.standard_normal((B, T, H, D)) * 3).astype(np.float32), dt)
+    k = round16((rng.standard_normal((B, T, Hkv, D)) * 0.2).astype(np.float32), dt)
     cfg = oracle.OracleConfig(1, 64, H, Hkv, D, T, 512)
     wq, wk = oracle.rope_qknorm(q, k, cfg)
     tab = torch.empty((2, T, D // 2), dtype=torch.float32, device=DEV)
     gpu.rope_table(tab, T, D, 10000.0)
     if fused:  # q and k as column blocks of one [B*T, (H+2Hkv)*D] buffer
         n = (H + 2 * Hkv) * D
-        buf = torch.zeros((B * T, n), dtype=torch.bfloat16, device=DEV)
-        buf[:, :H * D] = bf16_dev(q.reshape(B * T, H * D))
-        buf[:, H * D:(H + Hkv) * D] = bf16_dev(k.reshape(B * T, Hkv * D))
+        buf = torch.zeros((B * T, n), dtype=TDT[dt], device=DEV)
+        buf[:, :H * D] = dev16(q.reshape(B * T, H * D), dt)
+        buf[:, H * D:(H + Hkv) * D] = dev16(k.reshape(B * T, Hkv * D), dt)
         qv, kv = buf[:, :H * D], buf[:, H * D:(H + Hkv) * D]
         gpu.rope_qknorm(buf, buf[:, H * D:], tab, B, T, H, Hkv, D, q_row_stride=n, k_row_stride=n)
         torch.cuda.synchronize()
         gq, gk = host(qv).reshape(B, T, H, D), host(kv).reshape(B, T, Hkv, D)
         assert torch.all(buf[:, (H + Hkv) * D:] == 0)  # v block untouched
     else:
-        tq, tk = bf16_dev(q), bf16_dev(k)
+        tq, tk = dev16(q, dt), dev16(k, dt)
         gpu.rope_qknorm(tq, tk, tab, B, T, H, Hkv, D)
         torch.cuda.synchronize()
         gq, gk = host(tq), host(tk)
-    assert_close_bf16(gq, wq, 1e-4, "rope_qknorm q")
-    assert_close_bf16(gk, wk, 1e-4, "rope_qknorm k")
+    assert_close_bf16(gq, wq, 1e-4, "rope_qknorm q", rel=2 * REL[dt])
+    assert_close_bf16(gk, wk, 1e-4, "rope_qknorm k", rel=2 * REL[dt])
 
 
-@pytest.mark.parametrize("T,H,Hkv,W", [(1, 2, 2, 0), (17, 4, 4, 5), (128, 4, 2, 64), (300, 4, 1, 0),
-                                       (300, 4, 4, 1), (1000, 4, 2, 200), (1000, 2, 2, 1000),
-                                       (777, 8, 2, 256)])
-def test_attention_parity(gpu, T, H, Hkv, W):
-    B, D = 2, 128
+@pytest.mark.parametrize("T,H,Hkv,W,D", [(1, 2, 2, 0, 128), (17, 4, 4, 5, 128), (128, 4, 2, 64, 128),
+                                         (300, 4, 1, 0, 128), (300, 4, 4, 1, 128), (1000, 4, 2, 200, 128),
+                                         (1000, 2, 2, 1000, 128), (777, 8, 2, 256, 128), (256, 2, 2, 64, 64),
+                                         (300, 4, 2, 0, 64), (129, 2, 1, 7, 64)])
+@pytest.mark.parametrize("dt", DTYPES)
+def test_attention_parity(gpu, T, H, Hkv, W, D, dt):
+    B = 2
     q, k, v = make_qkv(B, T, H, Hkv, D, seed=T * 7 + W)
-    q, k, v = round_to_bf16(q), round_to_bf16(k), round_to_bf16(v)
-    out = torch.empty((B, T, H, D), dtype=torch.bfloat16, device=DEV)
-    gpu.attention(bf16_dev(q), bf16_dev(k), bf16_dev(v), out, W)
+    q, k, v = round16(q, dt), round16(k, dt), round16(v, dt)
+    out = torch.empty((B, T, H, D), dtype=TDT[dt], device=DEV)
+    gpu.attention(dev16(q, dt), dev16(k, dt), dev16(v, dt), out, W)
     torch.cuda.synchronize()
     want = oracle.attention(q, k, v, W if W > 0 else T)
     err = np.abs(host(out) - want).max()
@@ -144,19 +173,20 @@ def test_attention_parity(gpu, T, H, Hkv, W):
 @pytest.mark.parametrize("T", [2048, 4096, 8192])
 @pytest.mark.parametrize("Hkv", [16, 4])
 @pytest.mark.parametrize("full", [False, True])
-def test_attention_sweep_parity(gpu, T, Hkv, full):
+@pytest.mark.parametrize("dt", DTYPES)
+def test_attention_sweep_parity(gpu, T, Hkv, full, dt):
     """The attention-only workload: B=4, H=16, D=128, N(0,1) bf16 q/k/v, RoPE +
     QK-norm first (GPU kernel vs fp64 oracle from the same bf16 values), window
     T/4 or full; oracle evaluated on sampled query rows."""
     B, H, D = 4, 16, 128
     W = T if full else T // 4
     q, k, v = make_qkv(B, T, H, Hkv, D)
-    q, k, v = round_to_bf16(q), round_to_bf16(k), round_to_bf16(v)
-    tq, tk, tv = bf16_dev(q), bf16_dev(k), bf16_dev(v)
+    q, k, v = round16(q, dt), round16(k, dt), round16(v, dt)
+    tq, tk, tv = dev16(q, dt), dev16(k, dt), dev16(v, dt)
     tab = torch.empty((2, T, D // 2), dtype=torch.float32, device=DEV)
     gpu.rope_table(tab, T, D, 10000.0)
     gpu.rope_qknorm(tq, tk, tab, B, T, H, Hkv, D)
-    out = torch.empty((B, T, H, D), dtype=torch.bfloat16, device=DEV)
+    out = torch.empty((B, T, H, D), dtype=TDT[dt], device=DEV)
     gpu.attention(tq, tk, tv, out, W)
     torch.cuda.synchronize()
     cfg = oracle.OracleConfig(1, 64, H, Hkv, D, T, 512)
@@ -175,31 +205,59 @@ GEMM_SHAPES = [(128, 256, 64), (1, 256, 128), (300, 352, 200), (1000, 800, 520),
 
 
 @pytest.mark.parametrize("M,N,K", GEMM_SHAPES)
-@pytest.mark.parametrize("epi", ["store_bf16", "relu2_bf16", "resid_f32", "store_f32", "softcap_f32"])
-def test_linear_parity(gpu, M, N, K, epi):
+@pytest.mark.parametrize("epi", ["store_16", "relu2_16", "resid_f32", "store_f32", "softcap_f32"])
+@pytest.mark.parametrize("dt", DTYPES)
+def test_linear_parity(gpu, M, N, K, epi, dt):
     rng = np.random.default_rng(M * 31 + N * 7 + K)
-    a = round_to_bf16(rng.standard_normal((M, K)).astype(np.float32))
-    w = round_to_bf16((rng.standard_normal((N, K)) / math.sqrt(K) * 3).astype(np.float32))
+    a = round16(rng.standard_normal((M, K)).astype(np.float32), dt)
+    w = round16((rng.standard_normal((N, K)) / math.sqrt(K) * 3).astype(np.float32), dt)
     acc = a.astype(np.float64) @ w.astype(np.float64).T
     st = status_word()
-    if epi in ("store_bf16", "relu2_bf16"):
-        out = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device=DEV)
-        code = gpu.EPI_STORE_BF16 if epi == "store_bf16" else gpu.EPI_RELU2_BF16
-        gpu.linear(bf16_dev(a), bf16_dev(w), out, code, status=st)
-        want = acc if epi == "store_bf16" else oracle.relu2_mlp(a, w, np.eye(N))
+    if epi in ("store_16", "relu2_16"):
+        out = torch.full((M, N), float("nan"), dtype=TDT[dt], device=DEV)
+        code = gpu.EPI_STORE_16 if epi == "store_16" else gpu.EPI_RELU2_16
+        gpu.linear(dev16(a, dt), dev16(w, dt), out, code, status=st)
+        want = acc if epi == "store_16" else np.maximum(acc, 0.0) ** 2
         assert gpu.get_status(st) == 0
-        assert_close_bf16(host(out), want, 1e-5 * math.sqrt(K), f"linear {epi}")
+        assert_close_bf16(host(out), want, 1e-5 * math.sqrt(K), f"linear {epi}", rel=2 * REL[dt])
     else:
         x0 = rng.standard_normal((M, N)).astype(np.float32)
         out = torch.from_numpy(x0).to(DEV) if epi == "resid_f32" else \
             torch.full((M, N), float("nan"), dtype=torch.float32, device=DEV)
         code = {"resid_f32": gpu.EPI_RESID_F32, "store_f32": gpu.EPI_STORE_F32,
                 "softcap_f32": gpu.EPI_SOFTCAP_F32}[epi]
-        gpu.linear(bf16_dev(a), bf16_dev(w), out, code, cap=15.0, status=st)
+        gpu.linear(dev16(a, dt), dev16(w, dt), out, code, cap=15.0, status=st)
         want = {"resid_f32": x0 + acc, "store_f32": acc, "softcap_f32": oracle.softcap(acc, 15.0)}[epi]
         assert gpu.get_status(st) == 0
         got = out.cpu().numpy().astype(np.float64)
         np.testing.assert_allclose(got, want, rtol=1e-5, atol=2e-6 * math.sqrt(K), err_msg=f"linear {epi}")
+
+
+@pytest.mark.parametrize("dt", DTYPES)
+@pytest.mark.parametrize("M,C,H,Hkv,D,T", [(2 * 300, 256, 2, 1, 64, 300), (1024, 768, 6, 6, 128, 512),
+                                          (384, 512, 4, 2, 128, 128), (4096, 1280, 10, 10, 128, 2048)])
+def test_qkv_rope_parity(gpu, M, C, H, Hkv, D, T, dt):
+    """Fused QKV projection + RoPE + QK-norm against the oracle's projection, RoPE
+    and per-head RMSNorm (positions restart every T rows)."""
+    rng = np.random.default_rng(M + C + D)
+    N = (H + 2 * Hkv) * D
+    a = round16(rng.standard_normal((M, C)).astype(np.float32), dt)
+    w = round16((rng.standard_normal((N, C)) * 0.02).astype(np.float32), dt)
+    tab = torch.empty((2, T, D // 2), dtype=torch.float32, device=DEV)
+    gpu.rope_table(tab, T, D, 10000.0)
+    out = torch.full((M, N), float("nan"), dtype=TDT[dt], device=DEV)
+    st = status_word()
+    gpu.qkv_rope(dev16(a, dt), dev16(w, dt), out, tab, T, H, Hkv, D, eps=1e-6, status=st)
+    assert gpu.get_status(st) == 0
+    acc = a.astype(np.float64) @ w.astype(np.float64).T
+    B = M // T
+    q = acc[:, :H * D].reshape(B, T, H, D)
+    k = acc[:, H * D:(H + Hkv) * D].reshape(B, T, Hkv, D)
+    wq, wk = oracle.rope_qknorm(q, k, oracle.OracleConfig(1, C, H, Hkv, D, T, 512))
+    got = host(out)
+    assert_close_bf16(got[:, :H * D], wq.reshape(M, H * D), 2e-4, "qkv_rope q", rel=2 * REL[dt])
+    assert_close_bf16(got[:, H * D:(H + Hkv) * D], wk.reshape(M, Hkv * D), 2e-4, "qkv_rope k", rel=2 * REL[dt])
+    assert_close_bf16(got[:, (H + Hkv) * D:], acc[:, (H + Hkv) * D:], 2e-4, "qkv_rope v", rel=2 * REL[dt])
 
 
 def test_linear_row_stride(gpu):
@@ -303,6 +361,21 @@ def test_forward_tiny_full_batch(gpu):
     res2 = gpu.forward(model, tx, None, want_logits=True)
     torch.cuda.synchronize()
     assert torch.equal(res2["logits"], res["logits"])
+
+
+def test_forward_tiny_bf16_activations(gpu):
+    """The all-bf16 activation mode (act_dtype NC_BF16) on the tiny workload."""
+    s = SHAPES["tiny"]
+    w = make_weights(s)
+    cfg = gpu.make_config(s.n_layer, s.d_model, s.n_head, s.n_kv_head, s.head_dim, s.seq_len, s.vocab,
+                          s.short_window, act_dtype=gpu.BF16)
+    model = gpu.Model.from_numpy(cfg, w)
+    x, y = make_tokens(s)
+    res = gpu.forward(model, torch.from_numpy(x).to(DEV), torch.from_numpy(y).to(DEV), want_logits=True)
+    assert gpu.get_status(res["workspace"]) == 0
+    want = oracle.forward(_oracle_cfg(s), w, x, y)
+    assert np.abs(res["logits"].cpu().numpy() - want["logits"]).max() <= 3e-2
+    assert abs(res["loss"].item() - want["loss"]) <= 5e-3 * abs(want["loss"])
 
 
 @pytest.mark.parametrize("B,T", [(1, 1), (3, 100), (1, 256), (2, 65)])

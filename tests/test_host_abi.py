@@ -136,22 +136,30 @@ def test_no_device_fails_loudly(nclib):
     fw = _FakeWeights(nclib, 2)
     assert _fwd(nclib, cfg, fw, 2, 16) == 8
     L = nclib.lib()
-    assert L.nc_rmsnorm(1 << 40, 1 << 41, 8, 128, 1e-6, None) == 8
-    assert L.nc_attention(1 << 40, 1 << 40, 1 << 40, 1 << 41, 1, 16, 2, 2, 128, 0, None) == 8
-    assert L.nc_linear(1 << 40, 1 << 40, 1 << 41, 128, 256, 64, 256, 0, 15.0, None, None) == 8
+    assert L.nc_rmsnorm(1 << 40, 1 << 41, 8, 128, 1e-6, 1, None) == 8
+    assert L.nc_attention(1 << 40, 1 << 40, 1 << 40, 1 << 41, 1, 16, 2, 2, 128, 0, 1, None) == 8
+    assert L.nc_linear(1 << 40, 1 << 40, 1 << 41, 128, 256, 64, 256, 0, 15.0, 1, None, None) == 8
     assert L.nc_selftest_bounded_wait(1 << 40, 100, None) == 8
 
 
 def test_single_step_argument_checks(nclib):
     L = nclib.lib()
-    assert L.nc_linear(1 << 40, 1 << 40, 1 << 41, 128, 250, 64, 256, 0, 15.0, None, None) == 3  # N % 32
-    assert L.nc_linear(1 << 40, 1 << 40, 1 << 41, 128, 256, 60, 256, 0, 15.0, None, None) == 3  # K % 8
-    assert L.nc_linear((1 << 40) + 2, 1 << 40, 1 << 41, 128, 256, 64, 256, 0, 15.0, None, None) == 4
-    assert L.nc_linear(1 << 40, 1 << 40, 1 << 41, 128, 256, 64, 256, 9, 15.0, None, None) == 1
-    assert L.nc_attention(1 << 40, 1 << 40, 1 << 40, 1 << 41, 1, 16, 4, 3, 128, 0, None) == 1  # H % Hkv
-    assert L.nc_attention(1 << 40, 1 << 40, 1 << 40, 1 << 41, 1, 16, 4, 4, 64, 0, None) == 3
-    assert L.nc_rope_qknorm(1 << 40, 1 << 40, 1 << 40, 1, 16, 2, 2, 96, 192, 192, 1e-6, None) == 3
-    assert L.nc_cast_bf16(1 << 40, 1 << 41, 12, None) == 1
-    assert L.nc_softcap_ce(1 << 40, 1 << 40, None, 1 << 41, 4, 512, -1.0, None, None) == 1
+    A, B_ = 1 << 40, 1 << 41
+    assert L.nc_linear(A, A, B_, 128, 250, 64, 256, 0, 15.0, 1, None, None) == 3  # N % 32
+    assert L.nc_linear(A, A, B_, 128, 256, 60, 256, 0, 15.0, 1, None, None) == 3  # K % 8
+    assert L.nc_linear(A + 2, A, B_, 128, 256, 64, 256, 0, 15.0, 1, None, None) == 4
+    assert L.nc_linear(A, A, B_, 128, 256, 64, 256, 9, 15.0, 1, None, None) == 1  # epilogue
+    assert L.nc_linear(A, A, B_, 128, 256, 64, 256, 0, 15.0, 7, None, None) == 1  # dtype
+    assert L.nc_attention(A, A, A, B_, 1, 16, 4, 3, 128, 0, 1, None) == 1  # H % Hkv
+    assert L.nc_attention(A, A, A, B_, 1, 16, 4, 4, 96, 0, 1, None) == 3
+    assert L.nc_rope_qknorm(A, A, A, 1, 16, 2, 2, 96, 192, 192, 1e-6, 1, None) == 3
+    assert L.nc_qkv_rope(A, A, B_, A, 128, 16, 128, 2, 2, 96, 1e-6, 1, None, None) == 3
+    assert L.nc_cast_weights(A, B_, 12, 1, None) == 1
+    assert L.nc_cast_weights(A, B_, 16, 5, None) == 1
+    assert L.nc_softcap_ce(A, A, None, B_, 4, 512, -1.0, None, None) == 1
     assert L.nc_selftest_bounded_wait(None, 100, None) == 1
     assert L.nc_status_string(7) == b"bounded device wait ran out"
+    c = nclib.init_config(2, 64, 64, 0, 256, 512)
+    assert c.act_dtype == nclib.F16
+    c.act_dtype = 3
+    assert nclib.check_config(c) == 2
