@@ -299,6 +299,33 @@ nc_status nc_softcap_ce(const float* z, const int32_t* targets, float* capped_ou
 nc_status nc_loss_mean(const float* token_loss, const int32_t* targets, int M, int V,
                        float* loss, void* stream);
 
+/* Loss head without any scratch allocation.  The pages have no counterpart
+ * to this entry point; it exists for callers that cannot provide scratch
+ * memory: code embedded in a host application whose memory manager owns the
+ * whole device budget, and code on a latency-critical path where cudaMalloc's
+ * implicit device-wide synchronisation is not acceptable.
+ *
+ * Computes what the last step of nc_forward computes, from the final-norm
+ * activations: l = cap * tanh((a @ w_lm^T) / cap), token_loss[m] =
+ * logsumexp(l[m, :]) - l[m, y_m] (0 where y_m == -1), loss = mean over valid
+ * targets.  a [M, C] and w_lm [V, C] are 16-bit in format dtype (w_lm holding
+ * the bf16-rounded weights, e.g. from nc_cast_weights); targets [M] int32;
+ * token_loss [M] fp32 (required); loss 1 fp32 or NULL.
+ *
+ * Instead of a workspace it uses one fixed device array of this library
+ * (about 4.2 MB, held on every GPU that loads the library until the process
+ * exits), so it allocates nothing and calls no allocating routine.  Limits:
+ * M <= 8192 rows and V <= 32768 (NC_ERR_SHAPE beyond them).  The first call
+ * on a device looks up the array's device address (cudaGetSymbolAddress, with
+ * that device current); make that first call before any stream capture.  All
+ * calls share the array and it keeps the previous call's contents (nothing in
+ * it needs clearing), so calls whose work overlaps on the GPU race with each
+ * other: order them on one stream. */
+nc_status nc_lm_head_loss_static(const uint16_t* a, const uint16_t* w_lm, const int32_t* targets,
+                                 int M, int C, int V, float cap, nc_dtype dtype,
+                                 float* token_loss, float* loss, uint32_t* dev_status,
+                                 void* stream);
+
 /* Self-test of the failure path of in-kernel waits: one CTA waits on an
  * mbarrier that nothing arrives on, through the same bounded wait the GEMM
  * pipeline uses, for at most limit_us microseconds, then sets NC_DEV_TIMEOUT in
