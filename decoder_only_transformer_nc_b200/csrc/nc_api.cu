@@ -118,7 +118,7 @@ WsLayout ws_layout(const nc_config* c, int B, int T) {
   L.qkv = take(M * nqkv * 2);
   L.o = take(M * H * D * 2);
   L.h = take(M * 4 * C * 2);
-  L.part = take(M * (size_t)gemm_num_n_tiles((int)V) * 4);
+  L.part = take(M * (size_t)gemm_ce_partials_per_row((int)V) * 4);
   L.tgt = take(M * 4);
   L.tl = take(M * 4);
   L.total = off;
@@ -514,7 +514,7 @@ nc_status nc_forward_traced(const nc_config* cfg, const nc_weights* w, const int
     ep.ce_target = tgt;
     ep.targets = targets;
     NC_RUN(NC_K_GEMM_LM_HEAD, gemm_launch(a, C, wlm, C, M, V, C, EPI_CE_PARTIAL, f16, ep, status, st));
-    NC_RUN(NC_K_CE_FINALIZE, ce_finalize_launch(part, gemm_num_n_tiles(V), tgt, targets, tl, M, V,
+    NC_RUN(NC_K_CE_FINALIZE, ce_finalize_launch(part, gemm_ce_partials_per_row(V), tgt, targets, tl, M, V,
                                                 cfg->softcap, status, st));
     if (loss) NC_RUN(NC_K_LOSS_MEAN, loss_mean_launch(tl, targets, M, V, loss, st));
   } else if (logits) {

@@ -12,9 +12,11 @@
 //   warp 1      allocates 512 TMEM columns; one thread issues
 //               tcgen05.mma.cta_group::1.kind::f16 (M=128, N=256, K=16) into one of
 //               two 256-column fp32 accumulators and commits stage releases;
-//   warps 2..5  epilogue: tcgen05.ld of the accumulator (each warp owns the 32
-//               TMEM lanes = tile rows its warp index selects), fused epilogue
-//               op, direct global stores; then hand the accumulator back.
+//   warps 2..9  epilogue: tcgen05.ld of the accumulator (a warp may only read
+//               the 32 TMEM lanes = tile rows its warp index mod 4 selects, so
+//               two warps share each lane quarter and split the 256 columns),
+//               fused epilogue op, direct global stores; then hand the
+//               accumulator back.
 // Tiles are visited with the N index fastest so consecutive CTAs share one A
 // row-block and the weight matrix stays resident in L2.
 // Every mbarrier wait is bounded; on timeout the CTA records NC_DEV_TIMEOUT,
@@ -43,8 +45,9 @@ constexpr int B_BYTES = BN * BK * 2;
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int NUM_ACC = 2;
 constexpr int TMEM_COLS = 512;  // NUM_ACC * BN
-constexpr int NUM_THREADS = 192;
-constexpr int EPI_WARPS = 4;
+constexpr int EPI_WARPS = 8;  // two per TMEM lane quarter, each owning half the columns
+constexpr int NUM_THREADS = 64 + 32 * EPI_WARPS;
+constexpr int EPI_COLS = BN / 2;  // columns per epilogue warp
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
 constexpr uint32_t IDESC_BF16 = idesc_f32acc(BM, BN, false);
 constexpr uint32_t IDESC_F16 = idesc_f32acc(BM, BN, true);
@@ -366,6 +369,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   } else {
     // ---------------- epilogue warps
     const uint32_t quarter = warp & 3u;
+    const int half = (int)(warp - 2) / 4;  // which half of the tile's columns
     const int row_in_tile = quarter * 32 + lane;
     int acc = 0;
     uint32_t acc_phase = 0;
@@ -373,11 +377,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const int m_blk = tile / num_n;
       const int n_blk = tile % num_n;
       const int m0 = m_blk * BM;
-      const int n0 = n_blk * BN;
+      const int n0 = n_blk * BN + half * EPI_COLS;  // this warp's first column
+      const int row = m0 + row_in_tile;
+      if constexpr (EPI == EPI_RESID_F32) {
+        // Pull this thread's residual row segment towards L2 while the MMAs run.
+        if (row < M && n0 < N) {
+          const char* p = reinterpret_cast<const char*>(reinterpret_cast<const float*>(ep.out) +
+                                                        (int64_t)row * ep.ldo + n0);
+#pragma unroll
+          for (int l = 0; l < EPI_COLS * 4 / 128; ++l)
+            asm volatile("prefetch.global.L2 [%0];" ::"l"(p + 128 * l));
+        }
+      }
       if (!mbar_wait(smem_u32(&sm->tmem_full[acc]), acc_phase, ctl)) break;
       tc_fence_after();
-      const int row = m0 + row_in_tile;
-      const uint32_t taddr = tmem_base + ((quarter * 32u) << 16) + acc * BN;
+      const uint32_t taddr = tmem_base + ((quarter * 32u) << 16) + acc * BN + half * EPI_COLS;
       float ce_sum = 0.0f, ce_tl = 0.0f;
       int target = -1;
       if constexpr (EPI == EPI_CE_PARTIAL) {
@@ -385,14 +399,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
       if constexpr (EPI == EPI_QKV_ROPE) {
 #pragma unroll 1
-        for (int hh = 0; hh < BN / HD; ++hh) {
+        for (int hh = 0; hh < EPI_COLS / HD; ++hh) {
           const int col0 = n0 + hh * HD;
           if (col0 >= N) break;  // warp-uniform
           epilogue_qkv_head<F16, HD>(taddr + hh * HD, row, col0, M, ep);
         }
       } else {
 #pragma unroll 1
-        for (int c = 0; c < BN / 32; ++c) {
+        for (int c = 0; c < EPI_COLS / 32; ++c) {
           const int col0 = n0 + c * 32;
           if (col0 >= N) break;  // warp-uniform
           uint32_t r[32];
@@ -403,8 +417,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
       if constexpr (EPI == EPI_CE_PARTIAL) {
         if (row < M) {
-          ep.ce_partial[(int64_t)row * num_n + n_blk] = ce_sum;
-          if (target >= n0 && target < n0 + BN && target < N) ep.ce_target[row] = ce_tl;
+          ep.ce_partial[(int64_t)row * (2 * num_n) + 2 * n_blk + half] = ce_sum;
+          if (target >= n0 && target < n0 + EPI_COLS && target < N) ep.ce_target[row] = ce_tl;
         }
       }
       tc_fence_before();
@@ -522,7 +536,7 @@ nc_status selftest_wait_launch(uint32_t* dev_status, uint64_t limit_ns, cudaStre
   return cudaGetLastError() == cudaSuccess ? NC_OK : NC_ERR_CUDA;
 }
 
-int gemm_num_n_tiles(int N) { return (N + gemm::BN - 1) / gemm::BN; }
+int gemm_ce_partials_per_row(int N) { return 2 * ((N + gemm::BN - 1) / gemm::BN); }
 
 nc_status gemm_launch(const uint16_t* a, int64_t lda, const uint16_t* w, int64_t ldw, int M, int N,
                       int K, int epi, bool f16, const EpiParams& ep, uint32_t* dev_status,

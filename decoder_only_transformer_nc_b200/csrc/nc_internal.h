@@ -28,7 +28,7 @@ struct EpiParams {
   int64_t ldo;              // output row stride in elements
   float cap;                // soft-cap
   int store_logits;         // EPI_CE_PARTIAL: also write capped logits to out
-  float* ce_partial;        // EPI_CE_PARTIAL: [M, gemm_num_n_tiles(N)]
+  float* ce_partial;        // EPI_CE_PARTIAL: [M, gemm_ce_partials_per_row(N)]
   float* ce_target;         // EPI_CE_PARTIAL: [M], l[m, y_m] (written by one tile)
   const int32_t* targets;   // EPI_CE_PARTIAL: [M]
   const float* rope;        // EPI_QKV_ROPE: [2][T][D/2] cos, sin
@@ -43,7 +43,8 @@ bool device_is_sm100();
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 // ---- GEMM (nc_gemm.cu)
-int gemm_num_n_tiles(int N);
+// Number of soft-cap/CE partial sums the EPI_CE_PARTIAL epilogue writes per row.
+int gemm_ce_partials_per_row(int N);
 // a [M, K] (row stride lda) and w [N, K] (row stride ldw) are 16-bit in format
 // `f16` (true: fp16, false: bf16); 16-bit outputs use the same format.
 nc_status gemm_launch(const uint16_t* a, int64_t lda, const uint16_t* w, int64_t ldw, int M, int N,

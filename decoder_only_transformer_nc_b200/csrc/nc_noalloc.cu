@@ -24,12 +24,13 @@
 namespace nc {
 namespace {
 
-constexpr int kMaxRows = 8192;      // M limit
-constexpr int kMaxVocabTiles = 128;  // V limit: 128 tiles of 256 columns = 32768
-constexpr size_t kPartialFloats = (size_t)kMaxRows * kMaxVocabTiles;
-constexpr size_t kStaticBytes = (kPartialFloats + kMaxRows) * sizeof(float);  // 4.2 MB
+constexpr int kMaxRows = 8192;  // M limit
+constexpr int kMaxVocab = 32768;
+constexpr int kMaxPartials = 256;  // partial sums per row at V = 32768
+constexpr size_t kPartialFloats = (size_t)kMaxRows * kMaxPartials;
+constexpr size_t kStaticBytes = (kPartialFloats + kMaxRows) * sizeof(float);  // 8.4 MB
 
-// partials [kMaxRows][kMaxVocabTiles] followed by target logits [kMaxRows].
+// partials [kMaxRows][kMaxPartials] followed by target logits [kMaxRows].
 static __device__ __align__(256) float g_loss_scratch[kPartialFloats + kMaxRows];
 
 std::mutex g_mu;
@@ -60,15 +61,16 @@ extern "C" nc_status nc_lm_head_loss_static(const uint16_t* a, const uint16_t* w
   if (!a || !w_lm || !targets || !token_loss || M < 1 || C < 8 || V < 64 || !(cap > 0.0f) ||
       (dtype != NC_F16 && dtype != NC_BF16))
     return NC_ERR_INVALID_ARG;
-  if (M > kMaxRows || gemm_num_n_tiles(V) > kMaxVocabTiles || C % 8 != 0 || V % 64 != 0)
+  if (M > kMaxRows || V > kMaxVocab || gemm_ce_partials_per_row(V) > kMaxPartials || C % 8 != 0 ||
+      V % 64 != 0)
     return NC_ERR_SHAPE;
   if (!aligned16(a) || !aligned16(w_lm)) return NC_ERR_ALIGNMENT;
   if (!device_is_sm100()) return NC_ERR_UNSUPPORTED_DEVICE;
   float* scratch = scratch_address();
   if (!scratch) return NC_ERR_CUDA;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  const int n_tiles = gemm_num_n_tiles(V);
-  // Every (row, tile) partial is rewritten by the GEMM and the target logit of
+  const int n_tiles = gemm_ce_partials_per_row(V);
+  // Every (row, partial) slot is rewritten by the GEMM and the target logit of
   // every row with a valid target is rewritten too (rows without one are never
   // read), so nothing has to be cleared between calls.
   float* partial = scratch;

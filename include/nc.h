@@ -313,7 +313,7 @@ nc_status nc_loss_mean(const float* token_loss, const int32_t* targets, int M, i
  * token_loss [M] fp32 (required); loss 1 fp32 or NULL.
  *
  * Instead of a workspace it uses one fixed device array of this library
- * (about 4.2 MB, held on every GPU that loads the library until the process
+ * (about 8.4 MB, held on every GPU that loads the library until the process
  * exits), so it allocates nothing and calls no allocating routine.  Limits:
  * M <= 8192 rows and V <= 32768 (NC_ERR_SHAPE beyond them).  The first call
  * on a device looks up the array's device address (cudaGetSymbolAddress, with
