@@ -23,7 +23,7 @@ __device__ __forceinline__ float warp_sum(float v) {
 
 // ---------------------------------------------------------------- weight cast
 
-constexpr int kMaxCastSegs = 48;
+constexpr int kMaxCastSegs = 160;  // 3.9 KB of kernel parameters: one launch up to 26 layers
 struct CastBatch {
   const float* src[kMaxCastSegs];
   uint16_t* dst[kMaxCastSegs];
