@@ -316,7 +316,7 @@ nc_status nc_attention_strided(const uint16_t* q, const uint16_t* k, const uint1
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return NC_ERR_ALIGNMENT;
   if (nc_status s = device_ok()) return s;
   return attention_launch(q, k, v, out, B, T, H, Hkv, D, window, q_row_stride, kv_row_stride,
-                          dtype == NC_F16, S(stream));
+                          dtype == NC_F16, nullptr, S(stream));
 }
 
 nc_status nc_attention(const uint16_t* q, const uint16_t* k, const uint16_t* v, uint16_t* out, int B,
@@ -486,7 +486,7 @@ nc_status nc_forward_traced(const nc_config* cfg, const nc_weights* w, const int
     NC_RUN(NC_K_GEMM_QKV,
            gemm_launch(a, C, wqkv + l * L.wqkv_elems, C, M, NQKV, C, EPI_QKV_ROPE, f16, eq, status, st));
     NC_RUN(NC_K_ATTENTION, attention_launch(qkv, qkv + H * D, qkv + (H + Hkv) * D, o, B, T, H, Hkv,
-                                            D, W, NQKV, NQKV, f16, st));
+                                            D, W, NQKV, NQKV, f16, status, st));
     EpiParams ep{};
     ep.out = x;
     ep.ldo = C;

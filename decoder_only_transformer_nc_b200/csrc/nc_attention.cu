@@ -1,317 +1,455 @@
-// Causal sliding-window attention with GQA ("从文本到聊天模型" §5.4-5.5;
-// window pattern and GQA from "Nanochat与nanoGPT对比：关键升级" §1).
+// Causal sliding-window attention with GQA on the 5th-generation tensor cores
+// ("从文本到聊天模型" §5.4-5.5; window pattern and GQA from "Nanochat与nanoGPT对比：
+// 关键升级" §1).
 //
 //   o[b,i,h,:] = sum_{j visible} softmax_j(q[b,i,h,:].k[b,j,g,:] / sqrt(D)) v[b,j,g,:]
 //   visible: j <= i and i - j < W;  g = h / (H / Hkv)
 //
-// One CTA per (128-query block, head, batch row); 8 warps x 16 query rows.
-// K/V tiles of 64 keys are double-buffered in shared memory with cp.async
-// (XOR-swizzled 16-byte chunks, conflict-free ldmatrix).  Only the key tiles
-// that intersect [q0 - W + 1, q0 + 127] are visited, so short-window layers
-// cost O(T * W) instead of O(T^2); the mask is evaluated only on tiles that
-// straddle the causal diagonal or the window edge.  Online softmax in fp32
-// registers (exp2 with the 1/sqrt(D) * log2(e) scale folded in); P is reused
-// from the score registers as the bf16 A operand of P.V.
+// Persistent kernel, one CTA per SM, work items (128-query block, head, batch
+// row) handed out round-robin, longest rows first.  Warp roles:
+//   warp 0     TMA: the item's Q tile, then K/V tiles of 128 keys into a
+//              2-stage ring (4-D tensor maps over [B, T, heads, D]: tokens past
+//              T read as zeros, so tiles never leak into the next sequence);
+//   warp 1     owns 512 TMEM columns; one thread issues S = Q K^T (M=128,
+//              N=128 keys) into one of two S buffers, then O += P V (A = P from
+//              shared memory, B = V read MN-major) into the O accumulator;
+//   warps 2-5  one query row per thread: read the S row from TMEM, mask the
+//              window/causal edge only on tiles that straddle it, online
+//              softmax in fp32 with exp2, write P (16-bit) to a swizzled
+//              shared-memory tile for the next MMA; O is rescaled in TMEM
+//              only when the running row maximum grows by more than 2^8 in the
+//              exponent (P stays <= 256, exact in fp16); finally O / l -> out.
+// Only key tiles intersecting [q0 - W + 1, q0 + 127] are visited.
+// Every wait is bounded; on timeout the CTA records NC_DEV_TIMEOUT, drains
+// its copies and MMAs, frees its tensor memory and exits.
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <cstdint>
 
 #include "nc_half.cuh"
 #include "nc_internal.h"
+#include "nc_ptx.cuh"
 
 namespace nc {
 namespace attn {
 
-constexpr int BQ = 128;
-constexpr int BKV = 64;
-constexpr int NWARPS = 8;
-constexpr int NTHREADS = NWARPS * 32;
+constexpr int BQ = 128;   // query rows per work item
+constexpr int BKV = 128;  // keys per tile
+constexpr int NUM_THREADS = 192;
+constexpr int ATOM = 128 * 128;  // bytes of one [128 rows][64 x 16-bit] swizzle tile
+constexpr float kRescaleLog2 = 8.0f;
 
 template <int D>
 struct Geo {
-  static constexpr int ROW_BYTES = D * 2;
-  static constexpr int CHUNKS = D / 8;  // 16-byte chunks per row
-  static constexpr int Q_BYTES = BQ * ROW_BYTES;
-  static constexpr int KV_BYTES = BKV * ROW_BYTES;
-  static constexpr int SMEM_BYTES = Q_BYTES + 4 * KV_BYTES;  // Q + 2x K + 2x V
+  static constexpr int KA = D / 64;                  // 64-wide swizzle atoms along D
+  static constexpr int Q_BYTES = KA * ATOM;
+  static constexpr int KV_STAGE = 2 * KA * ATOM;     // K then V
+  static constexpr int P_BYTES = (BKV / 64) * ATOM;  // [128 rows][128 keys]
+  static constexpr int OFF_KV = Q_BYTES;
+  static constexpr int OFF_P = OFF_KV + 2 * KV_STAGE;
+  static constexpr int OFF_BAR = OFF_P + 2 * P_BYTES;
+  static constexpr int SMEM_BYTES = OFF_BAR + 256 + 1024;  // barriers + alignment slack
 };
 
-// Byte offset of 16-byte chunk `chunk` of row `row`: the chunk index is XOR-ed
-// with the row's low 3 bits so the 8 rows of one ldmatrix hit 8 distinct banks.
-template <int D>
-__device__ __forceinline__ uint32_t swz(int row, int chunk) {
-  return (uint32_t)(row * Geo<D>::ROW_BYTES + ((chunk ^ (row & 7)) << 4));
+struct Bars {
+  uint64_t q_full, q_empty;
+  uint64_t kv_full[2], kv_empty[2];
+  uint64_t s_full[2], s_free[2];
+  uint64_t p_full[2], p_free[2];
+  uint64_t o_free;
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+static_assert(sizeof(Bars) <= 256, "barrier block");
+
+__device__ __forceinline__ float ex2f(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
 }
 
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool valid) {
-  const int n = valid ? 16 : 0;  // 0 source bytes -> zero fill
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(n)
-               : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
+struct Item {
+  int b, h, q0, kt0, n_tiles;
+};
 
-__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
-                                        uint32_t& r3) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
-               : "r"(addr));
-}
-__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
-                                          uint32_t& r3) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
-               : "r"(addr));
-}
-
-template <bool F16>
-__device__ __forceinline__ void mma16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0,
-                                         uint32_t b1) {
-  if constexpr (F16) {
-    asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-        "{%0,%1,%2,%3};"
-        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-  } else {
-    asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-        "{%0,%1,%2,%3};"
-        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-  }
-}
-
-// Copies `rows` token rows (D bf16 each) starting at token r0 into a swizzled
-// tile; rows at or beyond T are zero-filled.
-template <int D>
-__device__ __forceinline__ void load_tile(uint32_t s_base, const uint16_t* g, int64_t stride, int r0,
-                                          int rows, int T) {
-  constexpr int CH = Geo<D>::CHUNKS;
-  const int chunks = rows * CH;
-  for (int c = threadIdx.x; c < chunks; c += NTHREADS) {
-    const int r = c / CH;
-    const int ch = c % CH;
-    const int tok = r0 + r;
-    const bool valid = tok < T;
-    const uint16_t* src = g + (int64_t)(valid ? tok : 0) * stride + ch * 8;
-    cp_async16(s_base + swz<D>(r, ch), src, valid);
-  }
-}
-
-// F16: q, k, v, P and the output in fp16 (else bf16).
-template <int D, bool F16>
-__global__ void __launch_bounds__(NTHREADS, 1)
-    attn_fwd_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__ k,
-                    const uint16_t* __restrict__ v, uint16_t* __restrict__ out, int T, int H,
-                    int Hkv, int W, int64_t q_stride, int64_t kv_stride, float scale_log2) {
-  extern __shared__ __align__(128) uint8_t smem[];
-  const uint32_t s_q = (uint32_t)__cvta_generic_to_shared(smem);
-  constexpr int KV_BYTES = Geo<D>::KV_BYTES;
-  constexpr int KSTEPS = D / 16;  // k-steps of Q.K^T
-  constexpr int NT = D / 8;       // 8-wide output column tiles
-  const uint32_t s_k0 = s_q + Geo<D>::Q_BYTES;
-  const uint32_t s_v0 = s_k0 + 2 * KV_BYTES;
-
+__device__ __forceinline__ Item item_of(int idx, int B, int H, int T, int W) {
   const int n_qb = (T + BQ - 1) / BQ;
-  const int qb = n_qb - 1 - (int)blockIdx.x;  // longest rows first
-  const int h = blockIdx.y;
-  const int b = blockIdx.z;
-  const int g = h / (H / Hkv);
-  const int q0 = qb * BQ;
-  const int warp = threadIdx.x >> 5;
-  const int lane = threadIdx.x & 31;
-  const int qw0 = q0 + warp * 16;
+  Item it;
+  it.b = idx % B;
+  idx /= B;
+  it.h = idx % H;
+  const int qb = n_qb - 1 - idx / H;  // longest rows first
+  it.q0 = qb * BQ;
+  const int lo = max(0, it.q0 - W + 1);
+  const int hi = min(T, it.q0 + BQ) - 1;
+  it.kt0 = lo / BKV;
+  it.n_tiles = hi / BKV - it.kt0 + 1;
+  return it;
+}
 
-  const uint16_t* qg = q + (int64_t)b * T * q_stride + (int64_t)h * D;
-  const uint16_t* kg = k + (int64_t)b * T * kv_stride + (int64_t)g * D;
-  const uint16_t* vg = v + (int64_t)b * T * kv_stride + (int64_t)g * D;
+template <int D, bool F16>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                   const __grid_constant__ CUtensorMap tmV, uint16_t* __restrict__ out, int B,
+                   int T, int H, int Hkv, int W, float scale_log2, uint32_t* dev_status,
+                   uint64_t limit_ns) {
+  using G = Geo<D>;
+  constexpr uint32_t IDESC_S = idesc_f32acc(BQ, BKV, F16);
+  constexpr uint32_t IDESC_PV = idesc_f32acc_bmn(BQ, D, F16);
+  constexpr uint32_t TMEM_COLS = 512;
+  constexpr uint32_t O_COL = 2 * BKV;
 
-  const int lo = max(0, q0 - W + 1);
-  const int hi = min(T, q0 + BQ) - 1;
-  const int kt0 = lo / BKV;
-  const int kt1 = hi / BKV;
-  const int n_tiles = kt1 - kt0 + 1;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                           ~static_cast<uintptr_t>(1023));
+  Bars* bar = reinterpret_cast<Bars*>(sm + G::OFF_BAR);
+  const uint32_t s_q = smem_u32(sm);
+  const uint32_t s_kv = s_q + G::OFF_KV;
+  const uint32_t s_p = s_q + G::OFF_P;
 
-  load_tile<D>(s_q, qg + (int64_t)q0 * q_stride, q_stride, 0, BQ, T - q0);
-  load_tile<D>(s_k0, kg, kv_stride, kt0 * BKV, BKV, T);
-  load_tile<D>(s_v0, vg, kv_stride, kt0 * BKV, BKV, T);
-  cp_async_commit();
+  const uint32_t warp = warp_id_sync();
+  const uint32_t lane = lane_id();
+  const int n_qb = (T + BQ - 1) / BQ;
+  const int n_items = B * H * n_qb;
+  const int group = H / Hkv;
 
-  uint32_t qa[KSTEPS][4];
-  float o[NT][4];
-#pragma unroll
-  for (int i = 0; i < NT; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.0f;
-  float m_run[2] = {-INFINITY, -INFINITY};
-  float l_run[2] = {0.0f, 0.0f};
-
-  const int gq = lane >> 2;  // row within the 8-row group
-  const int tq = lane & 3;   // column pair within the 8-column n-tile
-
-  for (int it = 0; it < n_tiles; ++it) {
-    const int buf = it & 1;
-    if (it + 1 < n_tiles) {
-      const int nb = buf ^ 1;
-      load_tile<D>(s_k0 + nb * KV_BYTES, kg, kv_stride, (kt0 + it + 1) * BKV, BKV, T);
-      load_tile<D>(s_v0 + nb * KV_BYTES, vg, kv_stride, (kt0 + it + 1) * BKV, BKV, T);
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bar->q_full), 1);
+    mbar_init(smem_u32(&bar->q_empty), 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(smem_u32(&bar->kv_full[i]), 1);
+      mbar_init(smem_u32(&bar->kv_empty[i]), 1);
+      mbar_init(smem_u32(&bar->s_full[i]), 1);
+      mbar_init(smem_u32(&bar->s_free[i]), 4);
+      mbar_init(smem_u32(&bar->p_full[i]), 4);
+      mbar_init(smem_u32(&bar->p_free[i]), 1);
     }
-    cp_async_commit();
-    cp_async_wait<1>();
-    __syncthreads();
+    mbar_init(smem_u32(&bar->o_free), 4);
+    mbar_init(smem_u32(&bar->drain), 1);
+    bar->abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tmQ);
+    prefetch_tmap(&tmK);
+    prefetch_tmap(&tmV);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(&bar->tmem_base), TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bar->tmem_base;
+  const WaitCtl ctl{&bar->abort_flag, dev_status, limit_ns};
 
-    if (it == 0) {
-#pragma unroll
-      for (int kk = 0; kk < KSTEPS; ++kk) {
-        const int r = warp * 16 + (lane & 15);
-        const int ch = 2 * kk + (lane >> 4);
-        ldsm_x4(s_q + swz<D>(r, ch), qa[kk][0], qa[kk][1], qa[kk][2], qa[kk][3]);
-      }
-    }
-
-    const int k0 = (kt0 + it) * BKV;
-    // Warp-uniform: does any (row, key) pair of this warp fall inside the window?
-    const bool skip = (k0 > qw0 + 15) || (qw0 - (k0 + BKV - 1) >= W);
-    if (!skip) {
-      const uint32_t s_k = s_k0 + buf * KV_BYTES;
-      const uint32_t s_v = s_v0 + buf * KV_BYTES;
-      float s[8][4];
-#pragma unroll
-      for (int n = 0; n < 8; ++n) s[n][0] = s[n][1] = s[n][2] = s[n][3] = 0.0f;
-#pragma unroll
-      for (int kk = 0; kk < KSTEPS; ++kk) {
-#pragma unroll
-        for (int jj = 0; jj < 4; ++jj) {
-          const int key = 16 * jj + (lane & 7) + ((lane >> 4) << 3);
-          const int ch = 2 * kk + ((lane >> 3) & 1);
-          uint32_t b0, b1, b2, b3;
-          ldsm_x4(s_k + swz<D>(key, ch), b0, b1, b2, b3);
-          mma16816<F16>(s[2 * jj], qa[kk], b0, b1);
-          mma16816<F16>(s[2 * jj + 1], qa[kk], b2, b3);
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------- TMA producer
+      uint32_t outstanding = 0, out_phase = 0;  // bits 0,1: kv stages; bit 2: Q
+      int g = 0;
+      bool ok = true;
+      for (int idx = blockIdx.x, n = 0; idx < n_items && ok; idx += gridDim.x, ++n) {
+        const Item it = item_of(idx, B, H, T, W);
+        const int gh = it.h / group;
+        if (!mbar_wait(smem_u32(&bar->q_empty), (n & 1) ^ 1, ctl)) break;
+        mbar_arrive_expect_tx(smem_u32(&bar->q_full), G::Q_BYTES);
+        for (int a = 0; a < G::KA; ++a)
+          tma_load_4d(s_q + a * ATOM, &tmQ, a * 64, it.h, it.q0, it.b, smem_u32(&bar->q_full));
+        outstanding |= 4u;
+        out_phase = (out_phase & ~4u) | ((uint32_t)(n & 1) << 2);
+        for (int j = 0; j < it.n_tiles; ++j, ++g) {
+          const int st = g & 1;
+          const uint32_t use = (uint32_t)(g >> 1);
+          if (!mbar_wait(smem_u32(&bar->kv_empty[st]), (use & 1) ^ 1, ctl)) {
+            ok = false;
+            break;
+          }
+          const uint32_t fb = smem_u32(&bar->kv_full[st]);
+          mbar_arrive_expect_tx(fb, G::KV_STAGE);
+          const int k0 = (it.kt0 + j) * BKV;
+          const uint32_t kbase = s_kv + st * G::KV_STAGE;
+          for (int a = 0; a < G::KA; ++a) {
+            tma_load_4d(kbase + a * ATOM, &tmK, a * 64, gh, k0, it.b, fb);
+            tma_load_4d(kbase + (G::KA + a) * ATOM, &tmV, a * 64, gh, k0, it.b, fb);
+          }
+          outstanding |= 1u << st;
+          out_phase = (out_phase & ~(1u << st)) | ((use & 1) << st);
         }
       }
-      const bool need_mask = !((k0 + BKV - 1 <= qw0) && (qw0 + 15 - k0 < W) && (k0 + BKV <= T));
-      if (need_mask) {
+      if (!ok || bar->abort_flag) {
+        int zero = 0;
+        const WaitCtl dctl{&zero, nullptr, limit_ns};
+        for (int st = 0; st < 2; ++st)
+          if (outstanding & (1u << st))
+            mbar_wait(smem_u32(&bar->kv_full[st]), (out_phase >> st) & 1u, dctl);
+        if (outstanding & 4u) mbar_wait(smem_u32(&bar->q_full), (out_phase >> 2) & 1u, dctl);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ---------------- MMA issuer
+      int g = 0;
+      bool ok = true;
+      for (int idx = blockIdx.x, n = 0; idx < n_items && ok; idx += gridDim.x, ++n) {
+        const Item it = item_of(idx, B, H, T, W);
+        if (!mbar_wait(smem_u32(&bar->q_full), n & 1, ctl)) break;
+        tc_fence_after();
+        for (int j = 0; j <= it.n_tiles && ok; ++j) {
+          if (j < it.n_tiles) {
+            const int gj = g + j;
+            const int sb = gj & 1;
+            const uint32_t use = (uint32_t)(gj >> 1);
+            if (!mbar_wait(smem_u32(&bar->kv_full[sb]), use & 1, ctl) ||
+                !mbar_wait(smem_u32(&bar->s_free[sb]), (use & 1) ^ 1, ctl)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t kbase = s_kv + sb * G::KV_STAGE;
 #pragma unroll
-        for (int n = 0; n < 8; ++n) {
+            for (int k = 0; k < D / 16; ++k) {
+              const uint32_t off = (k >> 2) * ATOM + (k & 3) * 32;
+              umma_f16(tmem + sb * BKV, sw128_kmajor_desc(s_q + off), sw128_kmajor_desc(kbase + off),
+                       IDESC_S, k > 0 ? 1u : 0u);
+            }
+            umma_commit(smem_u32(&bar->s_full[sb]));
+            if (j == it.n_tiles - 1) umma_commit(smem_u32(&bar->q_empty));
+          }
+          if (j > 0) {
+            const int gp = g + j - 1;
+            const int pb = gp & 1;
+            const uint32_t use = (uint32_t)(gp >> 1);
+            if (!mbar_wait(smem_u32(&bar->p_full[pb]), use & 1, ctl)) {
+              ok = false;
+              break;
+            }
+            if (j == 1 && !mbar_wait(smem_u32(&bar->o_free), (n & 1) ^ 1, ctl)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t pbase = s_p + pb * G::P_BYTES;
+            const uint32_t vbase = s_kv + pb * G::KV_STAGE + G::KA * ATOM;
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int i = qw0 + gq + ((e >> 1) << 3);
-            const int j = k0 + 8 * n + 2 * tq + (e & 1);
-            const bool vis = (j <= i) && (i - j < W) && (j < T);
-            if (!vis) s[n][e] = -INFINITY;
+            for (int k = 0; k < BKV / 16; ++k) {
+              const uint64_t adesc = sw128_kmajor_desc(pbase + (k >> 2) * ATOM + (k & 3) * 32);
+              const uint64_t bdesc = sw128_desc(vbase + k * 2048, ATOM, 1024);
+              umma_f16(tmem + O_COL, adesc, bdesc, IDESC_PV, (j > 1 || k > 0) ? 1u : 0u);
+            }
+            umma_commit(smem_u32(&bar->p_free[pb]));
+            umma_commit(smem_u32(&bar->kv_empty[pb]));
+          }
+        }
+        g += it.n_tiles;
+      }
+      umma_commit(smem_u32(&bar->drain));
+      int zero = 0;
+      const WaitCtl dctl{&zero, nullptr, limit_ns};
+      mbar_wait(smem_u32(&bar->drain), 0, dctl);
+    }
+  } else {
+    // ---------------- softmax / correction / epilogue (one query row per thread)
+    const uint32_t quarter = warp & 3u;
+    const int r = (int)(quarter * 32 + lane);
+    const uint32_t lane_off = (quarter * 32u) << 16;
+    const float thresh = kRescaleLog2 / scale_log2;  // in raw score units
+    int g = 0;
+    bool ok = true;
+    for (int idx = blockIdx.x, n = 0; idx < n_items && ok; idx += gridDim.x, ++n) {
+      const Item it = item_of(idx, B, H, T, W);
+      const int i = it.q0 + r;  // this thread's query position
+      float m_used = -INFINITY, l = 0.0f;
+      for (int j = 0; j < it.n_tiles; ++j) {
+        const int gj = g + j;
+        const int sb = gj & 1;
+        const uint32_t use = (uint32_t)(gj >> 1);
+        if (__any_sync(0xffffffffu, !mbar_wait(smem_u32(&bar->s_full[sb]), use & 1, ctl))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        float s[BKV];
+#pragma unroll
+        for (int c = 0; c < BKV / 32; ++c) {
+          uint32_t rr[32];
+          tmem_ld_32x32b_x32(tmem + lane_off + sb * BKV + c * 32, rr);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) s[c * 32 + e] = __uint_as_float(rr[e]);
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&bar->s_free[sb]));
+
+        const int k0 = (it.kt0 + j) * BKV;
+        const bool full_tile = (k0 + BKV - 1 <= it.q0) && (it.q0 + BQ - 1 - k0 < W) && (k0 + BKV <= T);
+        if (!full_tile) {
+#pragma unroll
+          for (int c = 0; c < BKV; ++c) {
+            const int key = k0 + c;
+            if (!(key <= i && i - key < W && key < T)) s[c] = -INFINITY;
+          }
+        }
+        float mx = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < BKV; ++c) mx = fmaxf(mx, s[c]);
+        const float m_new = fmaxf(m_used, mx);
+        bool need = false;
+        if (m_used == -INFINITY) {
+          m_used = m_new;  // O and l are still zero for this row
+        } else if (m_new > m_used + thresh) {
+          need = true;
+        }
+        if (__any_sync(0xffffffffu, need)) {
+          // Rescale this warp's O rows; the previous P.V must have landed.
+          const int gp = gj - 1;
+          const bool landed = mbar_wait(smem_u32(&bar->p_free[gp & 1]), (uint32_t)(gp >> 1) & 1, ctl);
+          if (__any_sync(0xffffffffu, !landed)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const float alpha = need ? ex2f((m_used - m_new) * scale_log2) : 1.0f;
+#pragma unroll 1
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t rr[32];
+            tmem_ld_32x32b_x32(tmem + lane_off + O_COL + c * 32, rr);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) rr[e] = __float_as_uint(__uint_as_float(rr[e]) * alpha);
+            tmem_st_32x32b_x32(tmem + lane_off + O_COL + c * 32, rr);
+          }
+          tmem_wait_st();
+          if (need) {
+            l *= alpha;
+            m_used = m_new;
+          }
+        }
+        const float ms = (m_used == -INFINITY) ? 0.0f : m_used * scale_log2;
+        // P buffer sb is free once the P.V two tiles back has completed.
+        if (__any_sync(0xffffffffu, !mbar_wait(smem_u32(&bar->p_free[sb]), (use & 1) ^ 1, ctl))) {
+          ok = false;
+          break;
+        }
+        uint8_t* prow = sm + G::OFF_P + sb * G::P_BYTES + r * 128;
+        float lsum = 0.0f;
+#pragma unroll
+        for (int c = 0; c < BKV / 8; ++c) {
+          float p[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            p[e] = ex2f(fmaf(s[c * 8 + e], scale_log2, -ms));
+            lsum += p[e];
+          }
+          uint4 pk;
+          pk.x = Half<F16>::pack2(p[0], p[1]);
+          pk.y = Half<F16>::pack2(p[2], p[3]);
+          pk.z = Half<F16>::pack2(p[4], p[5]);
+          pk.w = Half<F16>::pack2(p[6], p[7]);
+          const int atom = c >> 3, cc = c & 7;
+          *reinterpret_cast<uint4*>(prow + atom * ATOM + ((cc ^ (r & 7)) << 4)) = pk;
+        }
+        l += lsum;
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&bar->p_full[sb]));
+      }
+      if (!ok) break;
+      // epilogue: wait for the last P.V, then out = O / l
+      const int gl = g + it.n_tiles - 1;
+      if (__any_sync(0xffffffffu, !mbar_wait(smem_u32(&bar->p_free[gl & 1]), (uint32_t)(gl >> 1) & 1, ctl))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const float inv = l > 0.0f ? 1.0f / l : 0.0f;
+      uint16_t* orow = out + (((int64_t)it.b * T + i) * H + it.h) * D;
+#pragma unroll 1
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t rr[32];
+        tmem_ld_32x32b_x32(tmem + lane_off + O_COL + c * 32, rr);
+        tmem_wait_ld();
+        if (i < T) {
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            uint4 pk;
+            pk.x = Half<F16>::pack2(__uint_as_float(rr[8 * q + 0]) * inv, __uint_as_float(rr[8 * q + 1]) * inv);
+            pk.y = Half<F16>::pack2(__uint_as_float(rr[8 * q + 2]) * inv, __uint_as_float(rr[8 * q + 3]) * inv);
+            pk.z = Half<F16>::pack2(__uint_as_float(rr[8 * q + 4]) * inv, __uint_as_float(rr[8 * q + 5]) * inv);
+            pk.w = Half<F16>::pack2(__uint_as_float(rr[8 * q + 6]) * inv, __uint_as_float(rr[8 * q + 7]) * inv);
+            reinterpret_cast<uint4*>(orow + c * 32)[q] = pk;
           }
         }
       }
-      // online softmax, rows gq (e = 0,1) and gq + 8 (e = 2,3)
-#pragma unroll
-      for (int r = 0; r < 2; ++r) {
-        float mx = -INFINITY;
-#pragma unroll
-        for (int n = 0; n < 8; ++n) mx = fmaxf(mx, fmaxf(s[n][2 * r], s[n][2 * r + 1]));
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-        const float m_new = fmaxf(m_run[r], mx);
-        const float ms = (m_new == -INFINITY) ? 0.0f : m_new * scale_log2;
-        const float alpha = exp2f(m_run[r] * scale_log2 - ms);
-        float rs = 0.0f;
-#pragma unroll
-        for (int n = 0; n < 8; ++n) {
-          const float p0 = exp2f(s[n][2 * r] * scale_log2 - ms);
-          const float p1 = exp2f(s[n][2 * r + 1] * scale_log2 - ms);
-          s[n][2 * r] = p0;
-          s[n][2 * r + 1] = p1;
-          rs += p0 + p1;
-        }
-        l_run[r] = l_run[r] * alpha + rs;
-        m_run[r] = m_new;
-#pragma unroll
-        for (int dn = 0; dn < NT; ++dn) {
-          o[dn][2 * r] *= alpha;
-          o[dn][2 * r + 1] *= alpha;
-        }
-      }
-      // O += P V
-#pragma unroll
-      for (int kk = 0; kk < 4; ++kk) {
-        uint32_t pa[4];
-        pa[0] = Half<F16>::pack2(s[2 * kk][0], s[2 * kk][1]);
-        pa[1] = Half<F16>::pack2(s[2 * kk][2], s[2 * kk][3]);
-        pa[2] = Half<F16>::pack2(s[2 * kk + 1][0], s[2 * kk + 1][1]);
-        pa[3] = Half<F16>::pack2(s[2 * kk + 1][2], s[2 * kk + 1][3]);
-#pragma unroll
-        for (int dn = 0; dn < NT / 2; ++dn) {
-          const int key = 16 * kk + (lane & 7) + (((lane >> 3) & 1) << 3);
-          const int ch = 2 * dn + (lane >> 4);
-          uint32_t b0, b1, b2, b3;
-          ldsm_x4_t(s_v + swz<D>(key, ch), b0, b1, b2, b3);
-          mma16816<F16>(o[2 * dn], pa, b0, b1);
-          mma16816<F16>(o[2 * dn + 1], pa, b2, b3);
-        }
-      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&bar->o_free));
+      g += it.n_tiles;
     }
-    __syncthreads();
   }
 
-  // normalise and store
-#pragma unroll
-  for (int r = 0; r < 2; ++r) {
-    float l = l_run[r];
-    l += __shfl_xor_sync(0xffffffffu, l, 1);
-    l += __shfl_xor_sync(0xffffffffu, l, 2);
-    const float inv = l > 0.0f ? 1.0f / l : 0.0f;
-    const int i = qw0 + gq + 8 * r;
-    if (i < T) {
-      uint16_t* orow = out + ((int64_t)b * T + i) * ((int64_t)H * D) + (int64_t)h * D;
-#pragma unroll
-      for (int dn = 0; dn < NT; ++dn) {
-        *reinterpret_cast<uint32_t*>(orow + 8 * dn + 2 * tq) =
-            Half<F16>::pack2(o[dn][2 * r] * inv, o[dn][2 * r + 1] * inv);
-      }
-    }
-  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, TMEM_COLS);
 }
 
-}  // namespace attn
+// 4-D map over a [B, T, heads, D] 16-bit tensor with `row_stride` elements
+// between consecutive tokens; box = 64 dims x 1 head x 128 tokens x 1 row.
+static bool make_map4(CUtensorMap* map, const void* base, int B, int T, int heads, int D,
+                      int64_t row_stride, bool f16) {
+  const uint64_t dims[4] = {(uint64_t)D, (uint64_t)heads, (uint64_t)T, (uint64_t)B};
+  const uint64_t strides[3] = {(uint64_t)D * 2, (uint64_t)row_stride * 2,
+                               (uint64_t)T * (uint64_t)row_stride * 2};
+  const uint32_t box[4] = {64, 1, (uint32_t)BKV, 1};
+  return encode_tensor_map(map, f16, 4, base, dims, strides, box);
+}
 
 template <int D, bool F16>
-static cudaError_t attn_launch_t(const uint16_t* q, const uint16_t* k, const uint16_t* v,
-                                 uint16_t* out, int B, int T, int H, int Hkv, int W,
-                                 int64_t q_stride, int64_t kv_stride, cudaStream_t stream) {
-  using namespace attn;
+static nc_status launch_t(const uint16_t* q, const uint16_t* k, const uint16_t* v, uint16_t* out,
+                          int B, int T, int H, int Hkv, int W, int64_t q_stride, int64_t kv_stride,
+                          uint32_t* dev_status, cudaStream_t stream) {
+  using G = Geo<D>;
   static bool attr_done[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 64 && !attr_done[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel<D, F16>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         Geo<D>::SMEM_BYTES);
-    if (e != cudaSuccess) return e;
+    if (cudaFuncSetAttribute(attn_tc_kernel<D, F16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             G::SMEM_BYTES) != cudaSuccess)
+      return NC_ERR_CUDA;
     attr_done[dev] = true;
   }
+  CUtensorMap mq, mk, mv;
+  if (!make_map4(&mq, q, B, T, H, D, q_stride, F16) || !make_map4(&mk, k, B, T, Hkv, D, kv_stride, F16) ||
+      !make_map4(&mv, v, B, T, Hkv, D, kv_stride, F16))
+    return NC_ERR_CUDA;
+  const int items = B * H * ((T + BQ - 1) / BQ);
+  const int sms = device_sm_count();
+  const int grid = items < sms ? items : sms;
   const float scale_log2 = 1.4426950408889634f / sqrtf((float)D);
-  dim3 grid((T + BQ - 1) / BQ, H, B);
-  attn_fwd_kernel<D, F16><<<grid, NTHREADS, Geo<D>::SMEM_BYTES, stream>>>(
-      q, k, v, out, T, H, Hkv, W, q_stride, kv_stride, scale_log2);
-  return cudaGetLastError();
+  attn_tc_kernel<D, F16><<<grid, NUM_THREADS, G::SMEM_BYTES, stream>>>(
+      mq, mk, mv, out, B, T, H, Hkv, W, scale_log2, dev_status, kWaitLimitNs);
+  return cudaGetLastError() == cudaSuccess ? NC_OK : NC_ERR_CUDA;
 }
+
+}  // namespace attn
 
 nc_status attention_launch(const uint16_t* q, const uint16_t* k, const uint16_t* v, uint16_t* out,
                            int B, int T, int H, int Hkv, int D, int window, int64_t q_stride,
-                           int64_t kv_stride, bool f16, cudaStream_t stream) {
+                           int64_t kv_stride, bool f16, uint32_t* dev_status, cudaStream_t stream) {
   if (D != 64 && D != 128) return NC_ERR_SHAPE;
   if (B == 0 || T == 0) return NC_OK;
   const int W = (window <= 0 || window > T) ? T : window;
-  cudaError_t e;
   if (D == 128)
-    e = f16 ? attn_launch_t<128, true>(q, k, v, out, B, T, H, Hkv, W, q_stride, kv_stride, stream)
-            : attn_launch_t<128, false>(q, k, v, out, B, T, H, Hkv, W, q_stride, kv_stride, stream);
-  else
-    e = f16 ? attn_launch_t<64, true>(q, k, v, out, B, T, H, Hkv, W, q_stride, kv_stride, stream)
-            : attn_launch_t<64, false>(q, k, v, out, B, T, H, Hkv, W, q_stride, kv_stride, stream);
-  return e == cudaSuccess ? NC_OK : NC_ERR_CUDA;
+    return f16 ? attn::launch_t<128, true>(q, k, v, out, B, T, H, Hkv, W, q_stride, kv_stride, dev_status, stream)
+               : attn::launch_t<128, false>(q, k, v, out, B, T, H, Hkv, W, q_stride, kv_stride, dev_status, stream);
+  return f16 ? attn::launch_t<64, true>(q, k, v, out, B, T, H, Hkv, W, q_stride, kv_stride, dev_status, stream)
+             : attn::launch_t<64, false>(q, k, v, out, B, T, H, Hkv, W, q_stride, kv_stride, dev_status, stream);
 }
 
 }  // namespace nc

@@ -1,6 +1,7 @@
 // Declarations shared by the translation units of the library (not part of
 // the public ABI, which is include/nc.h).
 #pragma once
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <cstdint>
@@ -53,10 +54,15 @@ nc_status gemm_launch(const uint16_t* a, int64_t lda, const uint16_t* w, int64_t
 
 nc_status selftest_wait_launch(uint32_t* dev_status, uint64_t limit_ns, cudaStream_t stream);
 
+// TMA tensor map of a 16-bit tensor (fp16 if f16, else bf16) with 128-byte
+// swizzling: dims innermost first, strides in bytes for dims 1..rank-1.
+bool encode_tensor_map(CUtensorMap* map, bool f16, int rank, const void* base, const uint64_t* dims,
+                       const uint64_t* strides, const uint32_t* box);
+
 // ---- attention (nc_attention.cu)
 nc_status attention_launch(const uint16_t* q, const uint16_t* k, const uint16_t* v, uint16_t* out,
                            int B, int T, int H, int Hkv, int D, int window, int64_t q_stride,
-                           int64_t kv_stride, bool f16, cudaStream_t stream);
+                           int64_t kv_stride, bool f16, uint32_t* dev_status, cudaStream_t stream);
 
 // ---- elementwise / row kernels (nc_rowops.cu)
 struct CastSeg {
