@@ -190,6 +190,7 @@ def run_ours(args, s):
     import torch.distributed as dist
 
     import decoder_only_transformer_nc_b200 as nc
+    from decoder_only_transformer_nc_b200 import dp
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -207,7 +208,7 @@ def run_ours(args, s):
     weights = make_weights(s)
     model = nc.Model.from_numpy(cfg, weights, device=dev)
     B, T = s.batch, s.seq_len
-    x, y = make_tokens(s, seed=TOKEN_SEED + rank)
+    x, y = make_tokens(s, seed=dp.shard_seed(TOKEN_SEED, rank))
     tx, ty = torch.from_numpy(x).to(dev), torch.from_numpy(y).to(dev)
     ws = torch.empty(nc.workspace_bytes(cfg, B, T), dtype=torch.uint8, device=dev)
     out = {"loss": torch.empty((), dtype=torch.float32, device=dev)}
@@ -217,9 +218,7 @@ def run_ours(args, s):
     def step(trace=None, toks=tx, tgts=ty):
         nc.forward(model, toks, tgts, workspace=ws, out=out, trace=trace)
         if world > 1:
-            red[0] = out["loss"].double() * n_valid
-            red[1] = n_valid
-            dist.all_reduce(red)
+            dp.reduce_loss_into(red, out["loss"], n_valid)
 
     def barrier():
         if world > 1:
