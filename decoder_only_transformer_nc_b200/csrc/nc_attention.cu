@@ -6,10 +6,13 @@
 //   visible: j <= i and i - j < W;  g = h / (H / Hkv)
 //
 // Persistent kernel, one CTA per SM, work items (128-query block, head, batch
-// row) handed out round-robin, longest rows first.  Warp roles:
-//   warp 0     TMA: the item's Q tile, then K/V tiles of 128 keys into a
-//              2-stage ring (4-D tensor maps over [B, T, heads, D]: tokens past
-//              T read as zeros, so tiles never leak into the next sequence);
+// row) handed out round-robin.  Warp roles:
+//   warp 0     TMA: the item's Q tile, then K and V tiles of 128 keys into two
+//              2-slot rings (4-D tensor maps over [B, T, heads, D]: tokens past
+//              T read as zeros, so tiles never leak into the next sequence).
+//              A K slot is released as soon as its S = Q K^T has completed and a
+//              V slot after its P V, so the next K tile loads while the softmax
+//              of the current one runs;
 //   warp 1     owns 512 TMEM columns; one thread issues S = Q K^T (M=128,
 //              N=128 keys) into one of two S buffers, then O += P V (A = P from
 //              shared memory, B = V read MN-major) into the O accumulator;
@@ -54,7 +57,8 @@ struct Geo {
 
 struct Bars {
   uint64_t q_full, q_empty;
-  uint64_t kv_full[2], kv_empty[2];
+  uint64_t k_full[2], k_empty[2];
+  uint64_t v_full[2], v_empty[2];
   uint64_t s_full[2], s_free[2];
   uint64_t p_full[2], p_free[2];
   uint64_t o_free;
@@ -74,13 +78,17 @@ struct Item {
   int b, h, q0, kt0, n_tiles;
 };
 
+// Items are numbered with the query block fastest (last block first), then the
+// head, then the batch row: the CTAs running at the same time cover all query
+// blocks of a few heads, so each head's K/V is fetched from HBM about once and
+// then served from L2.
 __device__ __forceinline__ Item item_of(int idx, int B, int H, int T, int W) {
   const int n_qb = (T + BQ - 1) / BQ;
   Item it;
-  it.b = idx % B;
-  idx /= B;
+  const int qb = n_qb - 1 - idx % n_qb;
+  idx /= n_qb;
   it.h = idx % H;
-  const int qb = n_qb - 1 - idx / H;  // longest rows first
+  it.b = idx / H;
   it.q0 = qb * BQ;
   const int lo = max(0, it.q0 - W + 1);
   const int hi = min(T, it.q0 + BQ) - 1;
@@ -119,8 +127,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     mbar_init(smem_u32(&bar->q_full), 1);
     mbar_init(smem_u32(&bar->q_empty), 1);
     for (int i = 0; i < 2; ++i) {
-      mbar_init(smem_u32(&bar->kv_full[i]), 1);
-      mbar_init(smem_u32(&bar->kv_empty[i]), 1);
+      mbar_init(smem_u32(&bar->k_full[i]), 1);
+      mbar_init(smem_u32(&bar->k_empty[i]), 1);
+      mbar_init(smem_u32(&bar->v_full[i]), 1);
+      mbar_init(smem_u32(&bar->v_empty[i]), 1);
       mbar_init(smem_u32(&bar->s_full[i]), 1);
       mbar_init(smem_u32(&bar->s_free[i]), 4);
       mbar_init(smem_u32(&bar->p_full[i]), 4);
@@ -149,7 +159,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   if (warp == 0) {
     if (lane == 0) {
       // ---------------- TMA producer
-      uint32_t outstanding = 0, out_phase = 0;  // bits 0,1: kv stages; bit 2: Q
+      uint32_t outstanding = 0, out_phase = 0;  // bits 0,1: K slots; bit 2: Q; bits 3,4: V slots
       int g = 0;
       bool ok = true;
       for (int idx = blockIdx.x, n = 0; idx < n_items && ok; idx += gridDim.x, ++n) {
@@ -161,31 +171,50 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           tma_load_4d(s_q + a * ATOM, &tmQ, a * 64, it.h, it.q0, it.b, smem_u32(&bar->q_full));
         outstanding |= 4u;
         out_phase = (out_phase & ~4u) | ((uint32_t)(n & 1) << 2);
-        for (int j = 0; j < it.n_tiles; ++j, ++g) {
-          const int st = g & 1;
-          const uint32_t use = (uint32_t)(g >> 1);
-          if (!mbar_wait(smem_u32(&bar->kv_empty[st]), (use & 1) ^ 1, ctl)) {
-            ok = false;
-            break;
+        // V runs one tile behind K (K0, K1, V0, K2, V1, ...): a K load waits only
+        // for the S two tiles back, never for a P V.
+        for (int j = 0; j <= it.n_tiles; ++j) {
+          if (j < it.n_tiles) {
+            const int gk = g + j;
+            const int st = gk & 1;
+            const uint32_t use = (uint32_t)(gk >> 1);
+            if (!mbar_wait(smem_u32(&bar->k_empty[st]), (use & 1) ^ 1, ctl)) {
+              ok = false;
+              break;
+            }
+            mbar_arrive_expect_tx(smem_u32(&bar->k_full[st]), G::KA * ATOM);
+            for (int a = 0; a < G::KA; ++a)
+              tma_load_4d(s_kv + st * G::KV_STAGE + a * ATOM, &tmK, a * 64, gh, (it.kt0 + j) * BKV, it.b,
+                          smem_u32(&bar->k_full[st]));
+            outstanding |= 1u << st;
+            out_phase = (out_phase & ~(1u << st)) | ((use & 1) << st);
           }
-          const uint32_t fb = smem_u32(&bar->kv_full[st]);
-          mbar_arrive_expect_tx(fb, G::KV_STAGE);
-          const int k0 = (it.kt0 + j) * BKV;
-          const uint32_t kbase = s_kv + st * G::KV_STAGE;
-          for (int a = 0; a < G::KA; ++a) {
-            tma_load_4d(kbase + a * ATOM, &tmK, a * 64, gh, k0, it.b, fb);
-            tma_load_4d(kbase + (G::KA + a) * ATOM, &tmV, a * 64, gh, k0, it.b, fb);
+          if (j > 0) {
+            const int gv = g + j - 1;
+            const int st = gv & 1;
+            const uint32_t use = (uint32_t)(gv >> 1);
+            if (!mbar_wait(smem_u32(&bar->v_empty[st]), (use & 1) ^ 1, ctl)) {
+              ok = false;
+              break;
+            }
+            mbar_arrive_expect_tx(smem_u32(&bar->v_full[st]), G::KA * ATOM);
+            for (int a = 0; a < G::KA; ++a)
+              tma_load_4d(s_kv + st * G::KV_STAGE + (G::KA + a) * ATOM, &tmV, a * 64, gh,
+                          (it.kt0 + j - 1) * BKV, it.b, smem_u32(&bar->v_full[st]));
+            outstanding |= 8u << st;
+            out_phase = (out_phase & ~(8u << st)) | ((use & 1) << (3 + st));
           }
-          outstanding |= 1u << st;
-          out_phase = (out_phase & ~(1u << st)) | ((use & 1) << st);
         }
+        g += it.n_tiles;
       }
       if (!ok || bar->abort_flag) {
         int zero = 0;
         const WaitCtl dctl{&zero, nullptr, limit_ns};
-        for (int st = 0; st < 2; ++st)
-          if (outstanding & (1u << st))
-            mbar_wait(smem_u32(&bar->kv_full[st]), (out_phase >> st) & 1u, dctl);
+        for (int st = 0; st < 2; ++st) {
+          if (outstanding & (1u << st)) mbar_wait(smem_u32(&bar->k_full[st]), (out_phase >> st) & 1u, dctl);
+          if (outstanding & (8u << st))
+            mbar_wait(smem_u32(&bar->v_full[st]), (out_phase >> (3 + st)) & 1u, dctl);
+        }
         if (outstanding & 4u) mbar_wait(smem_u32(&bar->q_full), (out_phase >> 2) & 1u, dctl);
       }
     }
@@ -203,7 +232,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             const int gj = g + j;
             const int sb = gj & 1;
             const uint32_t use = (uint32_t)(gj >> 1);
-            if (!mbar_wait(smem_u32(&bar->kv_full[sb]), use & 1, ctl) ||
+            if (!mbar_wait(smem_u32(&bar->k_full[sb]), use & 1, ctl) ||
                 !mbar_wait(smem_u32(&bar->s_free[sb]), (use & 1) ^ 1, ctl)) {
               ok = false;
               break;
@@ -217,13 +246,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                        IDESC_S, k > 0 ? 1u : 0u);
             }
             umma_commit(smem_u32(&bar->s_full[sb]));
+            umma_commit(smem_u32(&bar->k_empty[sb]));
             if (j == it.n_tiles - 1) umma_commit(smem_u32(&bar->q_empty));
           }
           if (j > 0) {
             const int gp = g + j - 1;
             const int pb = gp & 1;
             const uint32_t use = (uint32_t)(gp >> 1);
-            if (!mbar_wait(smem_u32(&bar->p_full[pb]), use & 1, ctl)) {
+            if (!mbar_wait(smem_u32(&bar->p_full[pb]), use & 1, ctl) ||
+                !mbar_wait(smem_u32(&bar->v_full[pb]), use & 1, ctl)) {
               ok = false;
               break;
             }
@@ -241,7 +272,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               umma_f16(tmem + O_COL, adesc, bdesc, IDESC_PV, (j > 1 || k > 0) ? 1u : 0u);
             }
             umma_commit(smem_u32(&bar->p_free[pb]));
-            umma_commit(smem_u32(&bar->kv_empty[pb]));
+            umma_commit(smem_u32(&bar->v_empty[pb]));
           }
         }
         g += it.n_tiles;
@@ -273,13 +304,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
         tc_fence_after();
         float s[BKV];
+        {
+          uint32_t rr[BKV / 32][32];
 #pragma unroll
-        for (int c = 0; c < BKV / 32; ++c) {
-          uint32_t rr[32];
-          tmem_ld_32x32b_x32(tmem + lane_off + sb * BKV + c * 32, rr);
-          tmem_wait_ld();
+          for (int c = 0; c < BKV / 32; ++c) tmem_ld_32x32b_x32(tmem + lane_off + sb * BKV + c * 32, rr[c]);
+          tmem_wait_ld();  // one wait for all four loads
 #pragma unroll
-          for (int e = 0; e < 32; ++e) s[c * 32 + e] = __uint_as_float(rr[e]);
+          for (int c = 0; c < BKV / 32; ++c)
+#pragma unroll
+            for (int e = 0; e < 32; ++e) s[c * 32 + e] = __uint_as_float(rr[c][e]);
         }
         tc_fence_before();
         __syncwarp();
@@ -294,9 +327,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             if (!(key <= i && i - key < W && key < T)) s[c] = -INFINITY;
           }
         }
-        float mx = -INFINITY;
+        // row maximum with 8 independent chains (max is exact in any order)
+        float mx8[8];
 #pragma unroll
-        for (int c = 0; c < BKV; ++c) mx = fmaxf(mx, s[c]);
+        for (int e = 0; e < 8; ++e) mx8[e] = s[e];
+#pragma unroll
+        for (int c = 8; c < BKV; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], s[c]);
+        const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                               fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
         const float m_new = fmaxf(m_used, mx);
         bool need = false;
         if (m_used == -INFINITY) {
@@ -336,14 +374,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           break;
         }
         uint8_t* prow = sm + G::OFF_P + sb * G::P_BYTES + r * 128;
-        float lsum = 0.0f;
+        float ls8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};  // 8 independent sums
 #pragma unroll
         for (int c = 0; c < BKV / 8; ++c) {
           float p[8];
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
             p[e] = ex2f(fmaf(s[c * 8 + e], scale_log2, -ms));
-            lsum += p[e];
+            ls8[e] += p[e];
           }
           uint4 pk;
           pk.x = Half<F16>::pack2(p[0], p[1]);
@@ -353,7 +391,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           const int atom = c >> 3, cc = c & 7;
           *reinterpret_cast<uint4*>(prow + atom * ATOM + ((cc ^ (r & 7)) << 4)) = pk;
         }
-        l += lsum;
+        l += ((ls8[0] + ls8[1]) + (ls8[2] + ls8[3])) + ((ls8[4] + ls8[5]) + (ls8[6] + ls8[7]));
         fence_proxy_async_smem();
         tc_fence_before();
         __syncwarp();

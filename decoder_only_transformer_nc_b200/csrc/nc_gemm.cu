@@ -48,11 +48,13 @@ constexpr int TMEM_COLS = 512;  // NUM_ACC * BN
 constexpr int EPI_WARPS = 8;  // two per TMEM lane quarter, each owning half the columns
 constexpr int NUM_THREADS = 64 + 32 * EPI_WARPS;
 constexpr int EPI_COLS = BN / 2;  // columns per epilogue warp
-constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
+constexpr int STG_BYTES = 32 * 128;  // per epilogue warp: 32 rows x 128 B staging tile
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + EPI_WARPS * STG_BYTES + 1024 /*align*/ +
+                           256 /*barriers*/;
 constexpr uint32_t IDESC_BF16 = idesc_f32acc(BM, BN, false);
 constexpr uint32_t IDESC_F16 = idesc_f32acc(BM, BN, true);
 
-struct Smem {  // barrier block placed after the tile ring
+struct Smem {  // barrier block placed after the tile ring and the staging tiles
   uint64_t full[STAGES];
   uint64_t empty[STAGES];
   uint64_t tmem_full[NUM_ACC];
@@ -96,79 +98,122 @@ struct SoftCap {
   }
 };
 
-template <bool F16, int NV>
-__device__ __forceinline__ void store16(uint16_t* o, const float* v) {
+// Row r (0..31) of a warp's staging tile: 128 bytes written as eight 16-byte
+// chunks at the positions the TMA 128-byte swizzle expects (chunk j of row r
+// lives at chunk j ^ (r % 8)); a warp's 32 stores of one chunk hit 8 distinct
+// 16-byte bank groups, the minimum of 4 wavefronts for 512 bytes.
+__device__ __forceinline__ void stage_row(uint8_t* stg, int r, const uint32_t (&w)[32]) {
 #pragma unroll
-  for (int j = 0; j < NV / 8; ++j) {
-    uint4 pk;
-    pk.x = Half<F16>::pack2(v[8 * j + 0], v[8 * j + 1]);
-    pk.y = Half<F16>::pack2(v[8 * j + 2], v[8 * j + 3]);
-    pk.z = Half<F16>::pack2(v[8 * j + 4], v[8 * j + 5]);
-    pk.w = Half<F16>::pack2(v[8 * j + 6], v[8 * j + 7]);
-    reinterpret_cast<uint4*>(o)[j] = pk;
-  }
+  for (int j = 0; j < 8; ++j)
+    *reinterpret_cast<uint4*>(stg + r * 128 + ((j ^ (r & 7)) << 4)) =
+        make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
 }
 
-// Epilogue of one 32-column chunk held by this thread (one tile row).
-template <int EPI, bool F16>
-__device__ __forceinline__ void epilogue_chunk(const uint32_t (&r)[32], int row, int col0,
-                                               const EpiParams& ep, float& ce_sum, float& ce_tl,
-                                               int target) {
+// Half of row r: 64 bytes into chunks [c0, c0 + 4) of the swizzled row.
+__device__ __forceinline__ void stage_half_row(uint8_t* stg, int r, int c0, const uint32_t (&w)[16]) {
+#pragma unroll
+  for (int j = 0; j < 4; ++j)
+    *reinterpret_cast<uint4*>(stg + r * 128 + (((c0 + j) ^ (r & 7)) << 4)) =
+        make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
+}
+
+// Hand the warp's staging tile to TMA: store (or add into the fp32 destination)
+// the 32-row box whose top-left element is (row0, col0).  Lane 0 waits until
+// TMA has read the tile before anyone reuses the buffer.
+template <bool REDUCE>
+__device__ __forceinline__ void flush_stage(const CUtensorMap* map, uint8_t* stg, int col0, int row0,
+                                            uint32_t lane) {
+  fence_proxy_async_smem();
+  __syncwarp();
+  if (lane == 0) {
+    if constexpr (REDUCE)
+      tma_reduce_add_2d(map, smem_u32(stg), col0, row0);
+    else
+      tma_store_2d(map, smem_u32(stg), col0, row0);
+    bulk_commit();
+    bulk_wait_read0();
+  }
+  __syncwarp();
+}
+
+// Epilogue of one 32-column chunk for the CE path (partial sums; logits are
+// written directly when asked for).
+__device__ __forceinline__ void epilogue_ce_chunk(const uint32_t (&r)[32], int row, int col0,
+                                                  const EpiParams& ep, float& ce_sum, float& ce_tl,
+                                                  int target) {
+  // Soft-capped logits l lie in (-cap, cap): exp(l - cap) never overflows, so
+  // the per-tile partial sums combine by plain addition.
+  const SoftCap sc(ep.cap);
   float v[32];
 #pragma unroll
-  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
-  if constexpr (EPI == EPI_STORE_16 || EPI == EPI_RELU2_16) {
-    if constexpr (EPI == EPI_RELU2_16) {
+  for (int i = 0; i < 32; ++i) {
+    float p;
+    v[i] = sc.apply(__uint_as_float(r[i]), p);
+    ce_sum += p;
+  }
+  const int rel = target - col0;
+  if (rel >= 0 && rel < 32) {
 #pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        const float t = fmaxf(v[i], 0.0f);
-        v[i] = t * t;
-      }
-    }
-    store16<F16, 32>(reinterpret_cast<uint16_t*>(ep.out) + (int64_t)row * ep.ldo + col0, v);
-  } else if constexpr (EPI == EPI_RESID_F32) {
-    float4* o = reinterpret_cast<float4*>(reinterpret_cast<float*>(ep.out) + (int64_t)row * ep.ldo + col0);
-    float4 x[8];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) x[j] = o[j];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      x[j].x += v[4 * j + 0];
-      x[j].y += v[4 * j + 1];
-      x[j].z += v[4 * j + 2];
-      x[j].w += v[4 * j + 3];
-      o[j] = x[j];
-    }
-  } else if constexpr (EPI == EPI_STORE_F32 || EPI == EPI_SOFTCAP_F32) {
-    if constexpr (EPI == EPI_SOFTCAP_F32) {
-      const SoftCap sc(ep.cap);
-#pragma unroll
-      for (int i = 0; i < 32; ++i) v[i] = sc.apply(v[i]);
-    }
+    for (int i = 0; i < 32; ++i)
+      if (i == rel) ce_tl = v[i];
+  }
+  if (ep.store_logits) {
     float4* o = reinterpret_cast<float4*>(reinterpret_cast<float*>(ep.out) + (int64_t)row * ep.ldo + col0);
 #pragma unroll
     for (int j = 0; j < 8; ++j) o[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
-  } else if constexpr (EPI == EPI_CE_PARTIAL) {
-    // Soft-capped logits l lie in (-cap, cap): exp(l - cap) never overflows, so
-    // the per-tile partial sums combine by plain addition.
-    const SoftCap sc(ep.cap);
+  }
+}
+
+// fp32 epilogues (residual add, plain store, soft-cap): 32-column chunks.
+template <int EPI>
+__device__ __forceinline__ void epilogue_f32_half(uint32_t taddr, const CUtensorMap* tmC, uint8_t* stg,
+                                                  int n0, int row0, int N, const EpiParams& ep,
+                                                  uint32_t lane) {
+#pragma unroll 1
+  for (int c = 0; c < EPI_COLS / 32; ++c) {
+    const int col0 = n0 + c * 32;
+    if (col0 >= N) break;  // warp-uniform
+    uint32_t r[32];
+    tmem_ld_32x32b_x32(taddr + c * 32, r);
+    tmem_wait_ld();
+    if constexpr (EPI == EPI_SOFTCAP_F32) {
+      const SoftCap sc(ep.cap);
 #pragma unroll
-    for (int i = 0; i < 32; ++i) {
-      float p;
-      v[i] = sc.apply(v[i], p);
-      ce_sum += p;
+      for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(sc.apply(__uint_as_float(r[i])));
     }
-    const int rel = target - col0;
-    if (rel >= 0 && rel < 32) {
+    stage_row(stg, (int)lane, r);
+    flush_stage<EPI == EPI_RESID_F32>(tmC, stg, col0, row0, lane);
+  }
+}
+
+// 16-bit epilogues (plain store, relu^2): 64-column chunks (128 B per row).
+template <int EPI, bool F16>
+__device__ __forceinline__ void epilogue_16_half(uint32_t taddr, const CUtensorMap* tmC, uint8_t* stg,
+                                                 int n0, int row0, int N, uint32_t lane) {
+#pragma unroll 1
+  for (int c = 0; c < EPI_COLS / 64; ++c) {
+    const int col0 = n0 + c * 64;
+    if (col0 >= N) break;  // warp-uniform
+    uint32_t r[2][32];
+    tmem_ld_32x32b_x32(taddr + c * 64, r[0]);
+    tmem_ld_32x32b_x32(taddr + c * 64 + 32, r[1]);
+    tmem_wait_ld();
+    uint32_t w[32];
 #pragma unroll
-      for (int i = 0; i < 32; ++i)
-        if (i == rel) ce_tl = v[i];
-    }
-    if (ep.store_logits) {
-      float4* o = reinterpret_cast<float4*>(reinterpret_cast<float*>(ep.out) + (int64_t)row * ep.ldo + col0);
+    for (int h = 0; h < 2; ++h)
 #pragma unroll
-      for (int j = 0; j < 8; ++j) o[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
-    }
+      for (int i = 0; i < 16; ++i) {
+        float a = __uint_as_float(r[h][2 * i]), b = __uint_as_float(r[h][2 * i + 1]);
+        if constexpr (EPI == EPI_RELU2_16) {
+          a = fmaxf(a, 0.0f);
+          b = fmaxf(b, 0.0f);
+          a *= a;
+          b *= b;
+        }
+        w[16 * h + i] = Half<F16>::pack2(a, b);
+      }
+    stage_row(stg, (int)lane, w);
+    flush_stage<false>(tmC, stg, col0, row0, lane);
   }
 }
 
@@ -176,24 +221,17 @@ __device__ __forceinline__ void epilogue_chunk(const uint32_t (&r)[32], int row,
 // (pair (u_i, u_{i+HD/2}) rotated by t * theta_i) and RMSNorm over the head
 // ("Nanochat与nanoGPT对比" §1: QK-norm after RoPE); v heads are stored as is.
 // The rotation preserves the head's norm, so pass 1 takes the RMS straight from
-// the fp32 accumulator; pass 2 re-reads one (i, i + HD/2) chunk pair at a time,
-// rotates, scales and stores it.
+// the fp32 accumulator.  Pass 2 rotates 32-pair groups; the first halves of the
+// pairs fill the staging tile (columns [0, HD/2) of the head) while the second
+// halves wait in registers, then take its place for columns [HD/2, HD).
 template <bool F16, int HD>
-__device__ __forceinline__ void epilogue_qkv_head(uint32_t taddr, int row, int col0, int M,
-                                                  const EpiParams& ep) {
+__device__ __forceinline__ void epilogue_qkv_head(uint32_t taddr, const CUtensorMap* tmC, uint8_t* stg,
+                                                  int row, int col0, int row0, int M,
+                                                  const EpiParams& ep, uint32_t lane) {
+  constexpr int G = HD / 64;  // 32-pair groups per head (1 or 2)
   const int head = col0 / HD;
-  uint16_t* out = reinterpret_cast<uint16_t*>(ep.out) + (int64_t)row * ep.ldo + col0;
-  if (head >= ep.H + ep.Hkv) {  // v head (warp-uniform)
-#pragma unroll 1
-    for (int c = 0; c < HD / 32; ++c) {
-      uint32_t r[32];
-      tmem_ld_32x32b_x32(taddr + c * 32, r);
-      tmem_wait_ld();
-      float v[32];
-#pragma unroll
-      for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
-      if (row < M) store16<F16, 32>(out + c * 32, v);
-    }
+  if (head >= ep.H + ep.Hkv) {  // v head (warp-uniform): plain 16-bit store
+    epilogue_16_half<EPI_STORE_16, F16>(taddr, tmC, stg, col0, row0, col0 + HD, lane);
     return;
   }
   float ss = 0.0f;
@@ -209,45 +247,53 @@ __device__ __forceinline__ void epilogue_qkv_head(uint32_t taddr, int row, int c
   const int t = (row < M ? row : 0) % ep.T;
   const float* cs = ep.rope + (int64_t)t * (HD / 2);
   const float* sn = ep.rope + ((int64_t)ep.T + t) * (HD / 2);
+  // Pass 2 runs twice: first the rotated first halves u'_i (columns [0, HD/2)),
+  // then -- re-reading TMEM -- the second halves u'_{i+HD/2}, so no half has to
+  // be held in registers across a TMA store.
 #pragma unroll 1
-  for (int c = 0; c < HD / 64; ++c) {
-    uint32_t ra[32], rb[32];
-    tmem_ld_32x32b_x32(taddr + c * 32, ra);
-    tmem_ld_32x32b_x32(taddr + HD / 2 + c * 32, rb);
-    tmem_wait_ld();
-    float va[32], vb[32];
+  for (int part = 0; part < 2; ++part) {
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const float4 c4 = __ldg(reinterpret_cast<const float4*>(cs + c * 32) + j);
-      const float4 s4 = __ldg(reinterpret_cast<const float4*>(sn + c * 32) + j);
-      const float cc[4] = {c4.x, c4.y, c4.z, c4.w};
-      const float sv[4] = {s4.x, s4.y, s4.z, s4.w};
+    for (int g = 0; g < G; ++g) {
+      uint32_t ra[32], rb[32];
+      tmem_ld_32x32b_x32(taddr + g * 32, ra);
+      tmem_ld_32x32b_x32(taddr + HD / 2 + g * 32, rb);
+      tmem_wait_ld();
+      uint32_t w[16];
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int i = 4 * j + e;
-        const float a = __uint_as_float(ra[i]), b = __uint_as_float(rb[i]);
-        va[i] = (a * cc[e] - b * sv[e]) * rs;
-        vb[i] = (a * sv[e] + b * cc[e]) * rs;
+      for (int j = 0; j < 8; ++j) {
+        const float4 c4 = __ldg(reinterpret_cast<const float4*>(cs + g * 32) + j);
+        const float4 s4 = __ldg(reinterpret_cast<const float4*>(sn + g * 32) + j);
+        const float cc[4] = {c4.x, c4.y, c4.z, c4.w};
+        const float sv[4] = {s4.x, s4.y, s4.z, s4.w};
+        float v[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float a = __uint_as_float(ra[4 * j + e]), b = __uint_as_float(rb[4 * j + e]);
+          v[e] = (part == 0 ? (a * cc[e] - b * sv[e]) : (a * sv[e] + b * cc[e])) * rs;
+        }
+        w[2 * j] = Half<F16>::pack2(v[0], v[1]);
+        w[2 * j + 1] = Half<F16>::pack2(v[2], v[3]);
       }
+      // HD = 128: each part is one 64-column chunk (groups at chunks 0-3, 4-7);
+      // HD = 64: one chunk holds both parts (first halves 0-3, second 4-7).
+      stage_half_row(stg, (int)lane, HD == 128 ? 4 * g : 4 * part, w);
     }
-    if (row < M) {
-      store16<F16, 32>(out + c * 32, va);
-      store16<F16, 32>(out + HD / 2 + c * 32, vb);
-    }
+    if constexpr (HD == 128) flush_stage<false>(tmC, stg, col0 + 64 * part, row0, lane);
   }
+  if constexpr (HD == 64) flush_stage<false>(tmC, stg, col0, row0, lane);
 }
 
-// EPI: epilogue; F16: operands (and 16-bit outputs) fp16 instead of bf16;
-// HD: head size of the EPI_QKV_ROPE epilogue (0 otherwise).
 template <int EPI, bool F16, int HD>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                int M, int N, int K, EpiParams ep, uint32_t* dev_status, uint64_t limit_ns) {
+                const __grid_constant__ CUtensorMap tmC, int M, int N, int K, EpiParams ep,
+                uint32_t* dev_status, uint64_t limit_ns) {
   constexpr uint32_t IDESC = F16 ? IDESC_F16 : IDESC_BF16;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* tiles = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~static_cast<uintptr_t>(1023));
-  Smem* sm = reinterpret_cast<Smem*>(tiles + STAGES * STAGE_BYTES);
+  uint8_t* staging = tiles + STAGES * STAGE_BYTES;  // EPI_WARPS x STG_BYTES
+  Smem* sm = reinterpret_cast<Smem*>(staging + EPI_WARPS * STG_BYTES);
 
   const uint32_t warp = warp_id_sync();
   const uint32_t lane = lane_id();
@@ -371,6 +417,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const uint32_t quarter = warp & 3u;
     const int half = (int)(warp - 2) / 4;  // which half of the tile's columns
     const int row_in_tile = quarter * 32 + lane;
+    uint8_t* stg = staging + (warp - 2) * STG_BYTES;  // this warp's staging tile
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
@@ -379,32 +426,23 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const int m0 = m_blk * BM;
       const int n0 = n_blk * BN + half * EPI_COLS;  // this warp's first column
       const int row = m0 + row_in_tile;
-      if constexpr (EPI == EPI_RESID_F32) {
-        // Pull this thread's residual row segment towards L2 while the MMAs run.
-        if (row < M && n0 < N) {
-          const char* p = reinterpret_cast<const char*>(reinterpret_cast<const float*>(ep.out) +
-                                                        (int64_t)row * ep.ldo + n0);
-#pragma unroll
-          for (int l = 0; l < EPI_COLS * 4 / 128; ++l)
-            asm volatile("prefetch.global.L2 [%0];" ::"l"(p + 128 * l));
-        }
-      }
       if (!mbar_wait(smem_u32(&sm->tmem_full[acc]), acc_phase, ctl)) break;
       tc_fence_after();
       const uint32_t taddr = tmem_base + ((quarter * 32u) << 16) + acc * BN + half * EPI_COLS;
+      const int row0 = m0 + (int)quarter * 32;  // first tile row of this warp
       float ce_sum = 0.0f, ce_tl = 0.0f;
       int target = -1;
-      if constexpr (EPI == EPI_CE_PARTIAL) {
-        if (row < M) target = ep.targets ? ep.targets[row] : -1;
-      }
       if constexpr (EPI == EPI_QKV_ROPE) {
 #pragma unroll 1
         for (int hh = 0; hh < EPI_COLS / HD; ++hh) {
           const int col0 = n0 + hh * HD;
           if (col0 >= N) break;  // warp-uniform
-          epilogue_qkv_head<F16, HD>(taddr + hh * HD, row, col0, M, ep);
+          epilogue_qkv_head<F16, HD>(taddr + hh * HD, &tmC, stg, row, col0, row0, M, ep, lane);
         }
-      } else {
+      } else if constexpr (EPI == EPI_STORE_16 || EPI == EPI_RELU2_16) {
+        epilogue_16_half<EPI, F16>(taddr, &tmC, stg, n0, row0, N, lane);
+      } else if constexpr (EPI == EPI_CE_PARTIAL) {
+        if (row < M) target = ep.targets ? ep.targets[row] : -1;
 #pragma unroll 1
         for (int c = 0; c < EPI_COLS / 32; ++c) {
           const int col0 = n0 + c * 32;
@@ -412,8 +450,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           uint32_t r[32];
           tmem_ld_32x32b_x32(taddr + c * 32, r);
           tmem_wait_ld();
-          if (row < M) epilogue_chunk<EPI, F16>(r, row, col0, ep, ce_sum, ce_tl, target);
+          if (row < M) epilogue_ce_chunk(r, row, col0, ep, ce_sum, ce_tl, target);
         }
+      } else {
+        epilogue_f32_half<EPI>(taddr, &tmC, stg, n0, row0, N, ep, lane);
       }
       if constexpr (EPI == EPI_CE_PARTIAL) {
         if (row < M) {
@@ -429,6 +469,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         acc_phase ^= 1u;
       }
     }
+    if (lane == 0) bulk_wait0();  // every TMA store / reduce of this warp has landed
+    __syncwarp();
   }
 
   tc_fence_before();
@@ -467,8 +509,8 @@ static bool make_map(CUtensorMap* map, const void* ptr, int64_t rows, int64_t co
 }
 
 template <int EPI, bool F16, int HD>
-static cudaError_t launch_t(const CUtensorMap& ma, const CUtensorMap& mb, int M, int N, int K,
-                            const EpiParams& ep, uint32_t* dev_status, uint64_t limit_ns,
+static cudaError_t launch_t(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& mc, int M,
+                            int N, int K, const EpiParams& ep, uint32_t* dev_status, uint64_t limit_ns,
                             cudaStream_t stream) {
   static bool attr_done[64] = {};
   int dev = 0;
@@ -482,24 +524,25 @@ static cudaError_t launch_t(const CUtensorMap& ma, const CUtensorMap& mb, int M,
   const int tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
   const int sms = device_sm_count();
   const int grid = tiles < sms ? tiles : sms;
-  gemm_kernel<EPI, F16, HD><<<grid, NUM_THREADS, SMEM_BYTES, stream>>>(ma, mb, M, N, K, ep,
+  gemm_kernel<EPI, F16, HD><<<grid, NUM_THREADS, SMEM_BYTES, stream>>>(ma, mb, mc, M, N, K, ep,
                                                                        dev_status, limit_ns);
   return cudaGetLastError();
 }
 
 template <bool F16>
-static cudaError_t dispatch(int epi, const CUtensorMap& ma, const CUtensorMap& mb, int M, int N, int K,
-                            const EpiParams& ep, uint32_t* st, uint64_t lim, cudaStream_t s) {
+static cudaError_t dispatch(int epi, const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& mc,
+                            int M, int N, int K, const EpiParams& ep, uint32_t* st, uint64_t lim,
+                            cudaStream_t s) {
   switch (epi) {
-    case EPI_STORE_16: return launch_t<EPI_STORE_16, F16, 0>(ma, mb, M, N, K, ep, st, lim, s);
-    case EPI_RELU2_16: return launch_t<EPI_RELU2_16, F16, 0>(ma, mb, M, N, K, ep, st, lim, s);
-    case EPI_RESID_F32: return launch_t<EPI_RESID_F32, F16, 0>(ma, mb, M, N, K, ep, st, lim, s);
-    case EPI_STORE_F32: return launch_t<EPI_STORE_F32, F16, 0>(ma, mb, M, N, K, ep, st, lim, s);
-    case EPI_SOFTCAP_F32: return launch_t<EPI_SOFTCAP_F32, F16, 0>(ma, mb, M, N, K, ep, st, lim, s);
-    case EPI_CE_PARTIAL: return launch_t<EPI_CE_PARTIAL, F16, 0>(ma, mb, M, N, K, ep, st, lim, s);
+    case EPI_STORE_16: return launch_t<EPI_STORE_16, F16, 0>(ma, mb, mc, M, N, K, ep, st, lim, s);
+    case EPI_RELU2_16: return launch_t<EPI_RELU2_16, F16, 0>(ma, mb, mc, M, N, K, ep, st, lim, s);
+    case EPI_RESID_F32: return launch_t<EPI_RESID_F32, F16, 0>(ma, mb, mc, M, N, K, ep, st, lim, s);
+    case EPI_STORE_F32: return launch_t<EPI_STORE_F32, F16, 0>(ma, mb, mc, M, N, K, ep, st, lim, s);
+    case EPI_SOFTCAP_F32: return launch_t<EPI_SOFTCAP_F32, F16, 0>(ma, mb, mc, M, N, K, ep, st, lim, s);
+    case EPI_CE_PARTIAL: return launch_t<EPI_CE_PARTIAL, F16, 0>(ma, mb, mc, M, N, K, ep, st, lim, s);
     case EPI_QKV_ROPE:
-      return ep.D == 128 ? launch_t<EPI_QKV_ROPE, F16, 128>(ma, mb, M, N, K, ep, st, lim, s)
-                         : launch_t<EPI_QKV_ROPE, F16, 64>(ma, mb, M, N, K, ep, st, lim, s);
+      return ep.D == 128 ? launch_t<EPI_QKV_ROPE, F16, 128>(ma, mb, mc, M, N, K, ep, st, lim, s)
+                         : launch_t<EPI_QKV_ROPE, F16, 64>(ma, mb, mc, M, N, K, ep, st, lim, s);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -524,8 +567,22 @@ __global__ void selftest_wait_kernel(uint32_t* dev_status, uint64_t limit_ns) {
 
 }  // namespace gemm
 
+static bool encode_any(CUtensorMap* map, CUtensorMapDataType dt, int rank, const void* base,
+                       const uint64_t* dims, const uint64_t* strides, const uint32_t* box);
+
 bool encode_tensor_map(CUtensorMap* map, bool f16, int rank, const void* base, const uint64_t* dims,
                        const uint64_t* strides, const uint32_t* box) {
+  return encode_any(map, f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank,
+                    base, dims, strides, box);
+}
+
+bool encode_tensor_map_f32(CUtensorMap* map, int rank, const void* base, const uint64_t* dims,
+                           const uint64_t* strides, const uint32_t* box) {
+  return encode_any(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, rank, base, dims, strides, box);
+}
+
+static bool encode_any(CUtensorMap* map, CUtensorMapDataType dt, int rank, const void* base,
+                       const uint64_t* dims, const uint64_t* strides, const uint32_t* box) {
   gemm::EncodeTiledFn enc = gemm::get_encode_fn();
   if (!enc || rank < 1 || rank > 5) return false;
   cuuint64_t d[5], st[4];
@@ -536,8 +593,7 @@ bool encode_tensor_map(CUtensorMap* map, bool f16, int rank, const void* base, c
     es[i] = 1;
   }
   for (int i = 0; i + 1 < rank; ++i) st[i] = strides[i];
-  const CUresult r = enc(map, f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
-                         (cuuint32_t)rank, const_cast<void*>(base), d, st, bx, es,
+  const CUresult r = enc(map, dt, (cuuint32_t)rank, const_cast<void*>(base), d, st, bx, es,
                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
@@ -556,11 +612,23 @@ nc_status gemm_launch(const uint16_t* a, int64_t lda, const uint16_t* w, int64_t
   using namespace gemm;
   if (epi < EPI_STORE_16 || epi > EPI_QKV_ROPE) return NC_ERR_INVALID_ARG;
   if (epi == EPI_QKV_ROPE && (ep.D != 64 && ep.D != 128)) return NC_ERR_SHAPE;
-  CUtensorMap ma, mb;
+  CUtensorMap ma, mb, mc;
   if (!make_map(&ma, a, M, K, lda, BM, f16)) return NC_ERR_CUDA;
   if (!make_map(&mb, w, N, K, ldw, BN, f16)) return NC_ERR_CUDA;
-  const cudaError_t e = f16 ? dispatch<true>(epi, ma, mb, M, N, K, ep, dev_status, limit_ns, stream)
-                            : dispatch<false>(epi, ma, mb, M, N, K, ep, dev_status, limit_ns, stream);
+  // Output tile map for the TMA stores of the epilogue: 32 rows x 128 bytes
+  // (64 16-bit or 32 fp32 columns), the box one epilogue warp stages.
+  memset(&mc, 0, sizeof(mc));
+  if (epi != EPI_CE_PARTIAL) {
+    const uint64_t dims[2] = {(uint64_t)N, (uint64_t)M};
+    const bool out16 = (epi == EPI_STORE_16 || epi == EPI_RELU2_16 || epi == EPI_QKV_ROPE);
+    const uint64_t strides[1] = {(uint64_t)ep.ldo * (out16 ? 2 : 4)};
+    const uint32_t box[2] = {out16 ? 64u : 32u, 32u};
+    const bool ok = out16 ? encode_tensor_map(&mc, f16, 2, ep.out, dims, strides, box)
+                          : encode_tensor_map_f32(&mc, 2, ep.out, dims, strides, box);
+    if (!ok) return NC_ERR_CUDA;
+  }
+  const cudaError_t e = f16 ? dispatch<true>(epi, ma, mb, mc, M, N, K, ep, dev_status, limit_ns, stream)
+                            : dispatch<false>(epi, ma, mb, mc, M, N, K, ep, dev_status, limit_ns, stream);
   return e == cudaSuccess ? NC_OK : NC_ERR_CUDA;
 }
 

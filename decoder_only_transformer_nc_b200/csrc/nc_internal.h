@@ -54,10 +54,13 @@ nc_status gemm_launch(const uint16_t* a, int64_t lda, const uint16_t* w, int64_t
 
 nc_status selftest_wait_launch(uint32_t* dev_status, uint64_t limit_ns, cudaStream_t stream);
 
-// TMA tensor map of a 16-bit tensor (fp16 if f16, else bf16) with 128-byte
-// swizzling: dims innermost first, strides in bytes for dims 1..rank-1.
+// TMA tensor map with 128-byte swizzling: dims innermost first, strides in
+// bytes for dims 1..rank-1.  Element type: fp16 if f16, else bf16; the _f32
+// variant maps fp32 data.
 bool encode_tensor_map(CUtensorMap* map, bool f16, int rank, const void* base, const uint64_t* dims,
                        const uint64_t* strides, const uint32_t* box);
+bool encode_tensor_map_f32(CUtensorMap* map, int rank, const void* base, const uint64_t* dims,
+                           const uint64_t* strides, const uint32_t* box);
 
 // ---- attention (nc_attention.cu)
 nc_status attention_launch(const uint16_t* q, const uint16_t* k, const uint16_t* v, uint16_t* out,
