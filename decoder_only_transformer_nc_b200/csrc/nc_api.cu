@@ -249,6 +249,7 @@ nc_status nc_get_status(const void* dev_status, void* stream) {
   if (cudaMemcpy(&st, dev_status, sizeof(st), cudaMemcpyDeviceToHost) != cudaSuccess)
     return NC_ERR_CUDA;
   if (st & NC_DEV_TIMEOUT) return NC_ERR_TIMEOUT;
+  if (st & NC_DEV_SMEM_ALIGN) return NC_ERR_CUDA;
   if (st & (NC_DEV_TOKEN_RANGE | NC_DEV_TARGET_RANGE)) return NC_ERR_TOKEN_RANGE;
   return NC_OK;
 }

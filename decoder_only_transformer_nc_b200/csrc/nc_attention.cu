@@ -16,12 +16,16 @@
 //   warp 1     owns 512 TMEM columns; one thread issues S = Q K^T (M=128,
 //              N=128 keys) into one of two S buffers, then O += P V (A = P from
 //              shared memory, B = V read MN-major) into the O accumulator;
-//   warps 2-5  one query row per thread: read the S row from TMEM, mask the
-//              window/causal edge only on tiles that straddle it, online
+//   warps 2-9  softmax: each TMEM lane quarter (32 query rows, one per thread)
+//              is served by two warps that own 64 of the tile's 128 keys; they
+//              swap partial row maxima (and, at the end, row sums) through
+//              shared memory.  Mask the window/causal edge only on tiles that
+//              straddle it (one visible-column interval per row), online
 //              softmax in fp32 with exp2, write P (16-bit) to a swizzled
-//              shared-memory tile for the next MMA; O is rescaled in TMEM
-//              only when the running row maximum grows by more than 2^8 in the
-//              exponent (P stays <= 256, exact in fp16); finally O / l -> out.
+//              shared-memory tile for the next MMA; O is rescaled in TMEM only
+//              when the running row maximum grows by more than 2^8 in the
+//              exponent (P stays <= 256, exact in fp16); finally O / l, staged
+//              in the freed P tile and written by a TMA store.
 // Only key tiles intersecting [q0 - W + 1, q0 + 127] are visited.
 // Every wait is bounded; on timeout the CTA records NC_DEV_TIMEOUT, drains
 // its copies and MMAs, frees its tensor memory and exits.
@@ -29,6 +33,7 @@
 #include <cuda_runtime.h>
 
 #include <cstdint>
+#include <cstring>
 
 #include "nc_half.cuh"
 #include "nc_internal.h"
@@ -39,7 +44,8 @@ namespace attn {
 
 constexpr int BQ = 128;   // query rows per work item
 constexpr int BKV = 128;  // keys per tile
-constexpr int NUM_THREADS = 192;
+constexpr int SM_WARPS = 8;  // softmax warps: two per TMEM lane quarter, 64 keys each
+constexpr int NUM_THREADS = 64 + 32 * SM_WARPS;
 constexpr int ATOM = 128 * 128;  // bytes of one [128 rows][64 x 16-bit] swizzle tile
 constexpr float kRescaleLog2 = 8.0f;
 
@@ -52,7 +58,8 @@ struct Geo {
   static constexpr int OFF_KV = Q_BYTES;
   static constexpr int OFF_P = OFF_KV + 2 * KV_STAGE;
   static constexpr int OFF_BAR = OFF_P + 2 * P_BYTES;
-  static constexpr int SMEM_BYTES = OFF_BAR + 256 + 1024;  // barriers + alignment slack
+  static constexpr int OFF_X = OFF_BAR + 256;       // row-statistics exchange [2 slots][2 halves][128]
+  static constexpr int SMEM_BYTES = OFF_X + 2 * 2 * 128 * 4;
 };
 
 struct Bars {
@@ -62,6 +69,7 @@ struct Bars {
   uint64_t s_full[2], s_free[2];
   uint64_t p_full[2], p_free[2];
   uint64_t o_free;
+  uint64_t xbar[4];  // per lane quarter: both column halves posted their row statistics
   uint64_t drain;
   uint32_t tmem_base;
   int abort_flag;
@@ -100,7 +108,8 @@ __device__ __forceinline__ Item item_of(int idx, int B, int H, int T, int W) {
 template <int D, bool F16>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                   const __grid_constant__ CUtensorMap tmV, uint16_t* __restrict__ out, int B,
+                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+                   uint16_t* __restrict__ out, int B,
                    int T, int H, int Hkv, int W, float scale_log2, uint32_t* dev_status,
                    uint64_t limit_ns) {
   using G = Geo<D>;
@@ -109,9 +118,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   constexpr uint32_t TMEM_COLS = 512;
   constexpr uint32_t O_COL = 2 * BKV;
 
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                           ~static_cast<uintptr_t>(1023));
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  // The swizzled tiles need a 1024-byte aligned base; the dynamic window starts
+  // aligned in practice.  If it ever does not, fail cleanly instead of faulting.
+  if ((smem_u32(smem_raw) & 1023u) != 0) {
+    if (threadIdx.x == 0 && dev_status) atomicOr(dev_status, NC_DEV_SMEM_ALIGN);
+    return;
+  }
+  uint8_t* sm = smem_raw;
+  float* xval = reinterpret_cast<float*>(sm + G::OFF_X);
   Bars* bar = reinterpret_cast<Bars*>(sm + G::OFF_BAR);
   const uint32_t s_q = smem_u32(sm);
   const uint32_t s_kv = s_q + G::OFF_KV;
@@ -132,11 +147,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_init(smem_u32(&bar->v_full[i]), 1);
       mbar_init(smem_u32(&bar->v_empty[i]), 1);
       mbar_init(smem_u32(&bar->s_full[i]), 1);
-      mbar_init(smem_u32(&bar->s_free[i]), 4);
-      mbar_init(smem_u32(&bar->p_full[i]), 4);
+      mbar_init(smem_u32(&bar->s_free[i]), SM_WARPS);
+      mbar_init(smem_u32(&bar->p_full[i]), SM_WARPS);
       mbar_init(smem_u32(&bar->p_free[i]), 1);
     }
-    mbar_init(smem_u32(&bar->o_free), 4);
+    mbar_init(smem_u32(&bar->o_free), SM_WARPS);
+    for (int i = 0; i < 4; ++i) mbar_init(smem_u32(&bar->xbar[i]), 2);
     mbar_init(smem_u32(&bar->drain), 1);
     bar->abort_flag = 0;
     fence_mbar_init();
@@ -283,11 +299,29 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_wait(smem_u32(&bar->drain), 0, dctl);
     }
   } else {
-    // ---------------- softmax / correction / epilogue (one query row per thread)
+    // ---------------- softmax / correction / epilogue
     const uint32_t quarter = warp & 3u;
+    const int half = (int)(warp - 2) / 4;  // which 64 keys of each tile (and D/2 of O)
     const int r = (int)(quarter * 32 + lane);
     const uint32_t lane_off = (quarter * 32u) << 16;
     const float thresh = kRescaleLog2 / scale_log2;  // in raw score units
+    constexpr int KC = BKV / 2;                       // keys per warp and tile
+    constexpr int DC = D / 2;                         // O columns per warp
+    uint32_t xphase = 0;  // exchanges done by this warp (same count in its partner)
+    // Post v for this row, wait for the partner half, return the partner's value.
+    auto exchange = [&](float v, bool& ok_) -> float {
+      const int slot = xphase & 1;
+      xval[(slot * 2 + half) * 128 + r] = v;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&bar->xbar[quarter]));
+      const bool got = mbar_wait(smem_u32(&bar->xbar[quarter]), xphase & 1u, ctl);
+      ++xphase;
+      if (__any_sync(0xffffffffu, !got)) {
+        ok_ = false;
+        return 0.0f;
+      }
+      return xval[(slot * 2 + (half ^ 1)) * 128 + r];
+    };
     int g = 0;
     bool ok = true;
     for (int idx = blockIdx.x, n = 0; idx < n_items && ok; idx += gridDim.x, ++n) {
@@ -303,14 +337,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           break;
         }
         tc_fence_after();
-        float s[BKV];
+        float s[KC];
         {
-          uint32_t rr[BKV / 32][32];
+          uint32_t rr[KC / 32][32];
 #pragma unroll
-          for (int c = 0; c < BKV / 32; ++c) tmem_ld_32x32b_x32(tmem + lane_off + sb * BKV + c * 32, rr[c]);
-          tmem_wait_ld();  // one wait for all four loads
+          for (int c = 0; c < KC / 32; ++c)
+            tmem_ld_32x32b_x32(tmem + lane_off + sb * BKV + half * KC + c * 32, rr[c]);
+          tmem_wait_ld();
 #pragma unroll
-          for (int c = 0; c < BKV / 32; ++c)
+          for (int c = 0; c < KC / 32; ++c)
 #pragma unroll
             for (int e = 0; e < 32; ++e) s[c * 32 + e] = __uint_as_float(rr[c][e]);
         }
@@ -318,23 +353,24 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(&bar->s_free[sb]));
 
-        const int k0 = (it.kt0 + j) * BKV;
-        const bool full_tile = (k0 + BKV - 1 <= it.q0) && (it.q0 + BQ - 1 - k0 < W) && (k0 + BKV <= T);
-        if (!full_tile) {
+        const int k0 = (it.kt0 + j) * BKV + half * KC;  // first key of this warp's columns
+        const bool full = (k0 + KC - 1 <= it.q0) && (it.q0 + BQ - 1 - k0 < W);
+        if (!full) {
+          // visible columns of this row: lo <= c <= hi  (j <= i and i - j < W)
+          const int lo = i - W + 1 - k0;
+          const int hi = i - k0;
 #pragma unroll
-          for (int c = 0; c < BKV; ++c) {
-            const int key = k0 + c;
-            if (!(key <= i && i - key < W && key < T)) s[c] = -INFINITY;
-          }
+          for (int c = 0; c < KC; ++c) s[c] = (c >= lo && c <= hi) ? s[c] : -INFINITY;
         }
-        // row maximum with 8 independent chains (max is exact in any order)
         float mx8[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) mx8[e] = s[e];
 #pragma unroll
-        for (int c = 8; c < BKV; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], s[c]);
-        const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                               fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+        for (int c = 8; c < KC; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], s[c]);
+        float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                         fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+        mx = fmaxf(mx, exchange(mx, ok));  // both halves now hold the row maximum
+        if (!ok) break;
         const float m_new = fmaxf(m_used, mx);
         bool need = false;
         if (m_used == -INFINITY) {
@@ -343,7 +379,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           need = true;
         }
         if (__any_sync(0xffffffffu, need)) {
-          // Rescale this warp's O rows; the previous P.V must have landed.
+          // Rescale this warp's half of the O row; the previous P V must have landed.
           const int gp = gj - 1;
           const bool landed = mbar_wait(smem_u32(&bar->p_free[gp & 1]), (uint32_t)(gp >> 1) & 1, ctl);
           if (__any_sync(0xffffffffu, !landed)) {
@@ -353,13 +389,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           tc_fence_after();
           const float alpha = need ? ex2f((m_used - m_new) * scale_log2) : 1.0f;
 #pragma unroll 1
-          for (int c = 0; c < D / 32; ++c) {
+          for (int c = 0; c < DC / 32; ++c) {
             uint32_t rr[32];
-            tmem_ld_32x32b_x32(tmem + lane_off + O_COL + c * 32, rr);
+            tmem_ld_32x32b_x32(tmem + lane_off + O_COL + half * DC + c * 32, rr);
             tmem_wait_ld();
 #pragma unroll
             for (int e = 0; e < 32; ++e) rr[e] = __float_as_uint(__uint_as_float(rr[e]) * alpha);
-            tmem_st_32x32b_x32(tmem + lane_off + O_COL + c * 32, rr);
+            tmem_st_32x32b_x32(tmem + lane_off + O_COL + half * DC + c * 32, rr);
           }
           tmem_wait_st();
           if (need) {
@@ -368,15 +404,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
         }
         const float ms = (m_used == -INFINITY) ? 0.0f : m_used * scale_log2;
-        // P buffer sb is free once the P.V two tiles back has completed.
+        // P buffer sb is free once the P V two tiles back has completed.
         if (__any_sync(0xffffffffu, !mbar_wait(smem_u32(&bar->p_free[sb]), (use & 1) ^ 1, ctl))) {
           ok = false;
           break;
         }
-        uint8_t* prow = sm + G::OFF_P + sb * G::P_BYTES + r * 128;
+        uint8_t* prow = sm + G::OFF_P + sb * G::P_BYTES + half * ATOM + r * 128;
         float ls8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};  // 8 independent sums
 #pragma unroll
-        for (int c = 0; c < BKV / 8; ++c) {
+        for (int c = 0; c < KC / 8; ++c) {
           float p[8];
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
@@ -388,8 +424,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           pk.y = Half<F16>::pack2(p[2], p[3]);
           pk.z = Half<F16>::pack2(p[4], p[5]);
           pk.w = Half<F16>::pack2(p[6], p[7]);
-          const int atom = c >> 3, cc = c & 7;
-          *reinterpret_cast<uint4*>(prow + atom * ATOM + ((cc ^ (r & 7)) << 4)) = pk;
+          *reinterpret_cast<uint4*>(prow + ((c ^ (r & 7)) << 4)) = pk;
         }
         l += ((ls8[0] + ls8[1]) + (ls8[2] + ls8[3])) + ((ls8[4] + ls8[5]) + (ls8[6] + ls8[7]));
         fence_proxy_async_smem();
@@ -398,7 +433,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (lane == 0) mbar_arrive(smem_u32(&bar->p_full[sb]));
       }
       if (!ok) break;
-      // epilogue: wait for the last P.V, then out = O / l
+      // epilogue: full row sum, wait for the last P V, then out = O / l
+      l += exchange(l, ok);
+      if (!ok) break;
       const int gl = g + it.n_tiles - 1;
       if (__any_sync(0xffffffffu, !mbar_wait(smem_u32(&bar->p_free[gl & 1]), (uint32_t)(gl >> 1) & 1, ctl))) {
         ok = false;
@@ -406,21 +443,46 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
       tc_fence_after();
       const float inv = l > 0.0f ? 1.0f / l : 0.0f;
-      uint16_t* orow = out + (((int64_t)it.b * T + i) * H + it.h) * D;
-#pragma unroll 1
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t rr[32];
-        tmem_ld_32x32b_x32(tmem + lane_off + O_COL + c * 32, rr);
-        tmem_wait_ld();
-        if (i < T) {
+      uint32_t rr[DC / 32][32];
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
+      for (int c = 0; c < DC / 32; ++c) tmem_ld_32x32b_x32(tmem + lane_off + O_COL + half * DC + c * 32, rr[c]);
+      tmem_wait_ld();
+      if constexpr (D == 128) {
+        // Stage this warp's 32 rows x 64 columns in the last tile's P buffer
+        // (its P V has completed; only this warp writes these rows of this
+        // half) and let TMA write them to out.
+        uint8_t* srow = sm + G::OFF_P + (gl & 1) * G::P_BYTES + half * ATOM + r * 128;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          uint4 pk;
+          const int c = q >> 2, e0 = (q & 3) * 8;
+          pk.x = Half<F16>::pack2(__uint_as_float(rr[c][e0 + 0]) * inv, __uint_as_float(rr[c][e0 + 1]) * inv);
+          pk.y = Half<F16>::pack2(__uint_as_float(rr[c][e0 + 2]) * inv, __uint_as_float(rr[c][e0 + 3]) * inv);
+          pk.z = Half<F16>::pack2(__uint_as_float(rr[c][e0 + 4]) * inv, __uint_as_float(rr[c][e0 + 5]) * inv);
+          pk.w = Half<F16>::pack2(__uint_as_float(rr[c][e0 + 6]) * inv, __uint_as_float(rr[c][e0 + 7]) * inv);
+          *reinterpret_cast<uint4*>(srow + ((q ^ (r & 7)) << 4)) = pk;
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_4d(&tmO, smem_u32(sm + G::OFF_P + (gl & 1) * G::P_BYTES + half * ATOM + quarter * 32 * 128),
+                       half * DC, it.h, it.q0 + (int)quarter * 32, it.b);
+          bulk_commit();
+          bulk_wait_read0();
+        }
+        __syncwarp();
+      } else {
+        if (i < T) {
+          uint16_t* orow = out + (((int64_t)it.b * T + i) * H + it.h) * D + half * DC;
+#pragma unroll
+          for (int q = 0; q < DC / 8; ++q) {
             uint4 pk;
-            pk.x = Half<F16>::pack2(__uint_as_float(rr[8 * q + 0]) * inv, __uint_as_float(rr[8 * q + 1]) * inv);
-            pk.y = Half<F16>::pack2(__uint_as_float(rr[8 * q + 2]) * inv, __uint_as_float(rr[8 * q + 3]) * inv);
-            pk.z = Half<F16>::pack2(__uint_as_float(rr[8 * q + 4]) * inv, __uint_as_float(rr[8 * q + 5]) * inv);
-            pk.w = Half<F16>::pack2(__uint_as_float(rr[8 * q + 6]) * inv, __uint_as_float(rr[8 * q + 7]) * inv);
-            reinterpret_cast<uint4*>(orow + c * 32)[q] = pk;
+            const int c = q >> 2, e0 = (q & 3) * 8;
+            pk.x = Half<F16>::pack2(__uint_as_float(rr[c][e0 + 0]) * inv, __uint_as_float(rr[c][e0 + 1]) * inv);
+            pk.y = Half<F16>::pack2(__uint_as_float(rr[c][e0 + 2]) * inv, __uint_as_float(rr[c][e0 + 3]) * inv);
+            pk.z = Half<F16>::pack2(__uint_as_float(rr[c][e0 + 4]) * inv, __uint_as_float(rr[c][e0 + 5]) * inv);
+            pk.w = Half<F16>::pack2(__uint_as_float(rr[c][e0 + 6]) * inv, __uint_as_float(rr[c][e0 + 7]) * inv);
+            reinterpret_cast<uint4*>(orow)[q] = pk;
           }
         }
       }
@@ -429,6 +491,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       if (lane == 0) mbar_arrive(smem_u32(&bar->o_free));
       g += it.n_tiles;
     }
+    if (lane == 0) bulk_wait0();
+    __syncwarp();
   }
 
   tc_fence_before();
@@ -462,16 +526,23 @@ static nc_status launch_t(const uint16_t* q, const uint16_t* k, const uint16_t* 
       return NC_ERR_CUDA;
     attr_done[dev] = true;
   }
-  CUtensorMap mq, mk, mv;
+  CUtensorMap mq, mk, mv, mo;
   if (!make_map4(&mq, q, B, T, H, D, q_stride, F16) || !make_map4(&mk, k, B, T, Hkv, D, kv_stride, F16) ||
       !make_map4(&mv, v, B, T, Hkv, D, kv_stride, F16))
     return NC_ERR_CUDA;
+  memset(&mo, 0, sizeof(mo));
+  if (D == 128) {  // out [B, T, H, D]: boxes of 64 dims x 32 tokens (one softmax warp's rows)
+    const uint64_t dims[4] = {(uint64_t)D, (uint64_t)H, (uint64_t)T, (uint64_t)B};
+    const uint64_t strides[3] = {(uint64_t)D * 2, (uint64_t)H * D * 2, (uint64_t)T * H * D * 2};
+    const uint32_t box[4] = {64, 1, 32, 1};
+    if (!encode_tensor_map(&mo, F16, 4, out, dims, strides, box)) return NC_ERR_CUDA;
+  }
   const int items = B * H * ((T + BQ - 1) / BQ);
   const int sms = device_sm_count();
   const int grid = items < sms ? items : sms;
   const float scale_log2 = 1.4426950408889634f / sqrtf((float)D);
   attn_tc_kernel<D, F16><<<grid, NUM_THREADS, G::SMEM_BYTES, stream>>>(
-      mq, mk, mv, out, B, T, H, Hkv, W, scale_log2, dev_status, kWaitLimitNs);
+      mq, mk, mv, mo, out, B, T, H, Hkv, W, scale_log2, dev_status, kWaitLimitNs);
   return cudaGetLastError() == cudaSuccess ? NC_OK : NC_ERR_CUDA;
 }
 

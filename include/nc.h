@@ -69,6 +69,8 @@ typedef enum {
 #define NC_DEV_TOKEN_RANGE 0x1u  /* a token id was outside [0, V): row 0 used  */
 #define NC_DEV_TARGET_RANGE 0x2u /* a target was outside {-1} U [0, V): ignored */
 #define NC_DEV_TIMEOUT 0x4u      /* a pipeline wait gave up; outputs invalid   */
+#define NC_DEV_SMEM_ALIGN 0x8u   /* a kernel's shared-memory window was not 1024-byte
+                                    aligned; it did nothing (reported as NC_ERR_CUDA) */
 
 /* Model configuration.  "从文本到聊天模型" §5.1: d_model = depth * aspect_ratio,
  * n_head = d_model / head_dim.  window_pattern: one char per layer, cycled;
