@@ -4,7 +4,10 @@
 // Forward ("从文本到聊天模型" §5; block internals from "Nanochat与nanoGPT对比：
 // 关键升级" §1), all on the caller's stream:
 //   RoPE table; fp32 -> bf16 weight cast (Wq|Wk|Wv packed as one [(H+2Hkv)D, C]
-//   matrix per layer); embedding gather;
+//   matrix per layer, the rows of every q and k head reordered so that the
+//   RoPE partners u_j and u_{j+D/2} are neighbours; q and k therefore leave the
+//   QKV GEMM with the same pair-interleaved head layout, which leaves q.k and
+//   hence attention unchanged); embedding gather;
 //   per layer: RMSNorm -> QKV GEMM -> RoPE+QK-norm -> attention (layer window)
 //              -> c_proj GEMM with residual add -> RMSNorm -> c_fc GEMM with
 //              ReLU^2 -> c_proj GEMM with residual add;
@@ -459,15 +462,15 @@ nc_status nc_forward_traced(const nc_config* cfg, const nc_weights* w, const int
     const size_t nq = (size_t)H * D * C, nk = (size_t)Hkv * D * C;
     for (int l = 0; l < cfg->n_layer; ++l) {
       uint16_t* dq = wqkv + l * L.wqkv_elems;
-      segs.push_back({w->c_q[l], dq, (int64_t)nq});
-      segs.push_back({w->c_k[l], dq + nq, (int64_t)nk});
+      segs.push_back({w->c_q[l], dq, (int64_t)nq, true});  // RoPE pairs made adjacent
+      segs.push_back({w->c_k[l], dq + nq, (int64_t)nk, true});
       segs.push_back({w->c_v[l], dq + nq + nk, (int64_t)nk});
       segs.push_back({w->attn_proj[l], wo + l * L.wo_elems, (int64_t)L.wo_elems});
       segs.push_back({w->c_fc[l], wfc + l * L.wfc_elems, (int64_t)L.wfc_elems});
       segs.push_back({w->mlp_proj[l], wmp + l * L.wmp_elems, (int64_t)L.wmp_elems});
     }
     segs.push_back({w->lm_head, wlm, (int64_t)V * C});
-    NC_RUN(NC_K_CAST, cast_launch(segs.data(), (int)segs.size(), f16, st));
+    NC_RUN(NC_K_CAST, cast_launch(segs.data(), (int)segs.size(), f16, st, C, D));
   }
 
   NC_RUN(NC_K_EMBEDDING, embedding_launch(tokens, w->wte, x, M, C, V, status, st));
@@ -484,8 +487,8 @@ nc_status nc_forward_traced(const nc_config* cfg, const nc_weights* w, const int
     eq.Hkv = Hkv;
     eq.D = D;
     eq.eps = cfg->norm_eps;
-    NC_RUN(NC_K_GEMM_QKV,
-           gemm_launch(a, C, wqkv + l * L.wqkv_elems, C, M, NQKV, C, EPI_QKV_ROPE, f16, eq, status, st));
+    NC_RUN(NC_K_GEMM_QKV, gemm_launch(a, C, wqkv + l * L.wqkv_elems, C, M, NQKV, C, EPI_QKV_ROPE_IL, f16,
+                                      eq, status, st));
     NC_RUN(NC_K_ATTENTION, attention_launch(qkv, qkv + H * D, qkv + (H + Hkv) * D, o, B, T, H, Hkv,
                                             D, W, NQKV, NQKV, f16, status, st));
     EpiParams ep{};

@@ -121,7 +121,7 @@ __device__ __forceinline__ void stage_half_row(uint8_t* stg, int r, int c0, cons
 // the 32-row box whose top-left element is (row0, col0).  Lane 0 waits until
 // TMA has read the tile before anyone reuses the buffer.
 template <bool REDUCE>
-__device__ __forceinline__ void flush_stage(const CUtensorMap* map, uint8_t* stg, int col0, int row0,
+__device__ __forceinline__ void flush_issue(const CUtensorMap* map, uint8_t* stg, int col0, int row0,
                                             uint32_t lane) {
   fence_proxy_async_smem();
   __syncwarp();
@@ -131,9 +131,20 @@ __device__ __forceinline__ void flush_stage(const CUtensorMap* map, uint8_t* stg
     else
       tma_store_2d(map, smem_u32(stg), col0, row0);
     bulk_commit();
-    bulk_wait_read0();
   }
+}
+
+// The staging tile may be rewritten once TMA has read it.
+__device__ __forceinline__ void flush_wait(uint32_t lane) {
+  if (lane == 0) bulk_wait_read0();
   __syncwarp();
+}
+
+template <bool REDUCE>
+__device__ __forceinline__ void flush_stage(const CUtensorMap* map, uint8_t* stg, int col0, int row0,
+                                            uint32_t lane) {
+  flush_issue<REDUCE>(map, stg, col0, row0, lane);
+  flush_wait(lane);
 }
 
 // Epilogue of one 32-column chunk for the CE path (partial sums; logits are
@@ -164,40 +175,52 @@ __device__ __forceinline__ void epilogue_ce_chunk(const uint32_t (&r)[32], int r
   }
 }
 
-// fp32 epilogues (residual add, plain store, soft-cap): 32-column chunks.
+// fp32 epilogues (residual add, plain store, soft-cap): 32-column chunks.  The
+// TMEM load of chunk c+1 overlaps the TMA read of chunk c.
 template <int EPI>
 __device__ __forceinline__ void epilogue_f32_half(uint32_t taddr, const CUtensorMap* tmC, uint8_t* stg,
                                                   int n0, int row0, int N, const EpiParams& ep,
                                                   uint32_t lane) {
+  uint32_t r[32];
+  if (n0 < N) {
+    tmem_ld_32x32b_x32(taddr, r);
+    tmem_wait_ld();
+  }
 #pragma unroll 1
   for (int c = 0; c < EPI_COLS / 32; ++c) {
     const int col0 = n0 + c * 32;
     if (col0 >= N) break;  // warp-uniform
-    uint32_t r[32];
-    tmem_ld_32x32b_x32(taddr + c * 32, r);
-    tmem_wait_ld();
     if constexpr (EPI == EPI_SOFTCAP_F32) {
       const SoftCap sc(ep.cap);
 #pragma unroll
       for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(sc.apply(__uint_as_float(r[i])));
     }
+    if (c > 0) flush_wait(lane);  // previous chunk read out of the staging tile
     stage_row(stg, (int)lane, r);
-    flush_stage<EPI == EPI_RESID_F32>(tmC, stg, col0, row0, lane);
+    flush_issue<EPI == EPI_RESID_F32>(tmC, stg, col0, row0, lane);
+    if (c + 1 < EPI_COLS / 32 && col0 + 32 < N) {
+      tmem_ld_32x32b_x32(taddr + (c + 1) * 32, r);
+      tmem_wait_ld();
+    }
   }
+  flush_wait(lane);
 }
 
 // 16-bit epilogues (plain store, relu^2): 64-column chunks (128 B per row).
+// The TMEM loads of chunk c+1 overlap the TMA read of chunk c.
 template <int EPI, bool F16>
 __device__ __forceinline__ void epilogue_16_half(uint32_t taddr, const CUtensorMap* tmC, uint8_t* stg,
                                                  int n0, int row0, int N, uint32_t lane) {
+  uint32_t r[2][32];
+  if (n0 < N) {
+    tmem_ld_32x32b_x32(taddr, r[0]);
+    tmem_ld_32x32b_x32(taddr + 32, r[1]);
+    tmem_wait_ld();
+  }
 #pragma unroll 1
   for (int c = 0; c < EPI_COLS / 64; ++c) {
     const int col0 = n0 + c * 64;
     if (col0 >= N) break;  // warp-uniform
-    uint32_t r[2][32];
-    tmem_ld_32x32b_x32(taddr + c * 64, r[0]);
-    tmem_ld_32x32b_x32(taddr + c * 64 + 32, r[1]);
-    tmem_wait_ld();
     uint32_t w[32];
 #pragma unroll
     for (int h = 0; h < 2; ++h)
@@ -212,9 +235,16 @@ __device__ __forceinline__ void epilogue_16_half(uint32_t taddr, const CUtensorM
         }
         w[16 * h + i] = Half<F16>::pack2(a, b);
       }
+    if (c + 1 < EPI_COLS / 64 && col0 + 64 < N) {
+      tmem_ld_32x32b_x32(taddr + (c + 1) * 64, r[0]);
+      tmem_ld_32x32b_x32(taddr + (c + 1) * 64 + 32, r[1]);
+    }
+    if (c > 0) flush_wait(lane);
     stage_row(stg, (int)lane, w);
-    flush_stage<false>(tmC, stg, col0, row0, lane);
+    flush_issue<false>(tmC, stg, col0, row0, lane);
+    tmem_wait_ld();
   }
+  flush_wait(lane);
 }
 
 // QKV projection epilogue for one head of HD columns: q and k heads get RoPE
@@ -235,13 +265,19 @@ __device__ __forceinline__ void epilogue_qkv_head(uint32_t taddr, const CUtensor
     return;
   }
   float ss = 0.0f;
-#pragma unroll 1
-  for (int c = 0; c < HD / 32; ++c) {
-    uint32_t r[32];
-    tmem_ld_32x32b_x32(taddr + c * 32, r);
-    tmem_wait_ld();
 #pragma unroll
-    for (int i = 0; i < 32; ++i) ss = fmaf(__uint_as_float(r[i]), __uint_as_float(r[i]), ss);
+  for (int c = 0; c < HD / 64; ++c) {  // two 32-column loads per wait
+    uint32_t r0[32], r1[32];
+    tmem_ld_32x32b_x32(taddr + c * 64, r0);
+    tmem_ld_32x32b_x32(taddr + c * 64 + 32, r1);
+    tmem_wait_ld();
+    float s4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      s4[i & 3] = fmaf(__uint_as_float(r0[i]), __uint_as_float(r0[i]), s4[i & 3]);
+      s4[i & 3] = fmaf(__uint_as_float(r1[i]), __uint_as_float(r1[i]), s4[i & 3]);
+    }
+    ss += (s4[0] + s4[1]) + (s4[2] + s4[3]);
   }
   const float rs = rsqrtf(ss * (1.0f / HD) + ep.eps);
   const int t = (row < M ? row : 0) % ep.T;
@@ -283,6 +319,71 @@ __device__ __forceinline__ void epilogue_qkv_head(uint32_t taddr, const CUtensor
   if constexpr (HD == 64) flush_stage<false>(tmC, stg, col0, row0, lane);
 }
 
+// The same for a projection whose q and k rows were pair-interleaved by the
+// weight cast: inside each q/k head, column 2p holds u_p and column 2p+1 holds
+// u_{p+HD/2}, so every 64-column chunk carries 32 whole RoPE pairs and is
+// rotated, normalised and stored on its own (output in the same interleaved
+// order, for q and k alike -- attention scores are unchanged by a common
+// permutation of the head dimension).
+template <bool F16, int HD>
+__device__ __forceinline__ void epilogue_qkv_head_il(uint32_t taddr, const CUtensorMap* tmC,
+                                                     uint8_t* stg, int row, int col0, int row0, int M,
+                                                     const EpiParams& ep, uint32_t lane) {
+  const int head = col0 / HD;
+  if (head >= ep.H + ep.Hkv) {  // v head (warp-uniform): plain 16-bit store
+    epilogue_16_half<EPI_STORE_16, F16>(taddr, tmC, stg, col0, row0, col0 + HD, lane);
+    return;
+  }
+  float ss = 0.0f;
+#pragma unroll
+  for (int c = 0; c < HD / 64; ++c) {
+    uint32_t r0[32], r1[32];
+    tmem_ld_32x32b_x32(taddr + c * 64, r0);
+    tmem_ld_32x32b_x32(taddr + c * 64 + 32, r1);
+    tmem_wait_ld();
+    float s4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      s4[i & 3] = fmaf(__uint_as_float(r0[i]), __uint_as_float(r0[i]), s4[i & 3]);
+      s4[i & 3] = fmaf(__uint_as_float(r1[i]), __uint_as_float(r1[i]), s4[i & 3]);
+    }
+    ss += (s4[0] + s4[1]) + (s4[2] + s4[3]);
+  }
+  const float rs = rsqrtf(ss * (1.0f / HD) + ep.eps);
+  const int t = (row < M ? row : 0) % ep.T;
+  const float* cs = ep.rope + (int64_t)t * (HD / 2);
+  const float* sn = ep.rope + ((int64_t)ep.T + t) * (HD / 2);
+#pragma unroll 1
+  for (int c = 0; c < HD / 64; ++c) {  // pairs 32c .. 32c+31
+    uint32_t r0[32], r1[32];
+    tmem_ld_32x32b_x32(taddr + c * 64, r0);
+    tmem_ld_32x32b_x32(taddr + c * 64 + 32, r1);
+    tmem_wait_ld();
+    uint32_t w[32];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const float4 c4 = __ldg(reinterpret_cast<const float4*>(cs + c * 32) + j);
+      const float4 s4 = __ldg(reinterpret_cast<const float4*>(sn + c * 32) + j);
+      const float cc[4] = {c4.x, c4.y, c4.z, c4.w};
+      const float sv[4] = {s4.x, s4.y, s4.z, s4.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int pp = 4 * j + e;  // pair within the chunk
+        const uint32_t* src = pp < 16 ? r0 : r1;
+        const int kk = pp & 15;
+        const float a = __uint_as_float(src[2 * kk]), b = __uint_as_float(src[2 * kk + 1]);
+        w[pp] = Half<F16>::pack2((a * cc[e] - b * sv[e]) * rs, (a * sv[e] + b * cc[e]) * rs);
+      }
+    }
+    if (c > 0) flush_wait(lane);
+    stage_row(stg, (int)lane, w);
+    flush_issue<false>(tmC, stg, col0 + 64 * c, row0, lane);
+  }
+  flush_wait(lane);
+}
+
+// EPI: epilogue selector; F16: operands (and 16-bit outputs) fp16 instead of
+// bf16; HD: head size of the QKV epilogues (0 otherwise).
 template <int EPI, bool F16, int HD>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
@@ -426,18 +527,35 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const int m0 = m_blk * BM;
       const int n0 = n_blk * BN + half * EPI_COLS;  // this warp's first column
       const int row = m0 + row_in_tile;
+      if constexpr (EPI == EPI_QKV_ROPE || EPI == EPI_QKV_ROPE_IL) {
+        // This row's cos/sin lines are known before the accumulator is ready:
+        // pull them into L1 while the MMAs run (q and k heads only).
+        if (row < M && n0 < N && n0 / HD < ep.H + ep.Hkv) {
+          const int t = row % ep.T;
+          const char* cl = reinterpret_cast<const char*>(ep.rope + (int64_t)t * (HD / 2));
+          const char* sl = reinterpret_cast<const char*>(ep.rope + ((int64_t)ep.T + t) * (HD / 2));
+#pragma unroll
+          for (int l = 0; l < HD * 2 / 128; ++l) {
+            asm volatile("prefetch.global.L1 [%0];" ::"l"(cl + 128 * l));
+            asm volatile("prefetch.global.L1 [%0];" ::"l"(sl + 128 * l));
+          }
+        }
+      }
       if (!mbar_wait(smem_u32(&sm->tmem_full[acc]), acc_phase, ctl)) break;
       tc_fence_after();
       const uint32_t taddr = tmem_base + ((quarter * 32u) << 16) + acc * BN + half * EPI_COLS;
       const int row0 = m0 + (int)quarter * 32;  // first tile row of this warp
       float ce_sum = 0.0f, ce_tl = 0.0f;
       int target = -1;
-      if constexpr (EPI == EPI_QKV_ROPE) {
+      if constexpr (EPI == EPI_QKV_ROPE || EPI == EPI_QKV_ROPE_IL) {
 #pragma unroll 1
         for (int hh = 0; hh < EPI_COLS / HD; ++hh) {
           const int col0 = n0 + hh * HD;
           if (col0 >= N) break;  // warp-uniform
-          epilogue_qkv_head<F16, HD>(taddr + hh * HD, &tmC, stg, row, col0, row0, M, ep, lane);
+          if constexpr (EPI == EPI_QKV_ROPE)
+            epilogue_qkv_head<F16, HD>(taddr + hh * HD, &tmC, stg, row, col0, row0, M, ep, lane);
+          else
+            epilogue_qkv_head_il<F16, HD>(taddr + hh * HD, &tmC, stg, row, col0, row0, M, ep, lane);
         }
       } else if constexpr (EPI == EPI_STORE_16 || EPI == EPI_RELU2_16) {
         epilogue_16_half<EPI, F16>(taddr, &tmC, stg, n0, row0, N, lane);
@@ -543,6 +661,9 @@ static cudaError_t dispatch(int epi, const CUtensorMap& ma, const CUtensorMap& m
     case EPI_QKV_ROPE:
       return ep.D == 128 ? launch_t<EPI_QKV_ROPE, F16, 128>(ma, mb, mc, M, N, K, ep, st, lim, s)
                          : launch_t<EPI_QKV_ROPE, F16, 64>(ma, mb, mc, M, N, K, ep, st, lim, s);
+    case EPI_QKV_ROPE_IL:
+      return ep.D == 128 ? launch_t<EPI_QKV_ROPE_IL, F16, 128>(ma, mb, mc, M, N, K, ep, st, lim, s)
+                         : launch_t<EPI_QKV_ROPE_IL, F16, 64>(ma, mb, mc, M, N, K, ep, st, lim, s);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -610,8 +731,8 @@ nc_status gemm_launch(const uint16_t* a, int64_t lda, const uint16_t* w, int64_t
                       int K, int epi, bool f16, const EpiParams& ep, uint32_t* dev_status,
                       cudaStream_t stream, uint64_t limit_ns) {
   using namespace gemm;
-  if (epi < EPI_STORE_16 || epi > EPI_QKV_ROPE) return NC_ERR_INVALID_ARG;
-  if (epi == EPI_QKV_ROPE && (ep.D != 64 && ep.D != 128)) return NC_ERR_SHAPE;
+  if (epi < EPI_STORE_16 || epi > EPI_QKV_ROPE_IL) return NC_ERR_INVALID_ARG;
+  if ((epi == EPI_QKV_ROPE || epi == EPI_QKV_ROPE_IL) && (ep.D != 64 && ep.D != 128)) return NC_ERR_SHAPE;
   CUtensorMap ma, mb, mc;
   if (!make_map(&ma, a, M, K, lda, BM, f16)) return NC_ERR_CUDA;
   if (!make_map(&mb, w, N, K, ldw, BN, f16)) return NC_ERR_CUDA;
@@ -620,7 +741,8 @@ nc_status gemm_launch(const uint16_t* a, int64_t lda, const uint16_t* w, int64_t
   memset(&mc, 0, sizeof(mc));
   if (epi != EPI_CE_PARTIAL) {
     const uint64_t dims[2] = {(uint64_t)N, (uint64_t)M};
-    const bool out16 = (epi == EPI_STORE_16 || epi == EPI_RELU2_16 || epi == EPI_QKV_ROPE);
+    const bool out16 = (epi == EPI_STORE_16 || epi == EPI_RELU2_16 || epi == EPI_QKV_ROPE ||
+                        epi == EPI_QKV_ROPE_IL);
     const uint64_t strides[1] = {(uint64_t)ep.ldo * (out16 ? 2 : 4)};
     const uint32_t box[2] = {out16 ? 64u : 32u, 32u};
     const bool ok = out16 ? encode_tensor_map(&mc, f16, 2, ep.out, dims, strides, box)

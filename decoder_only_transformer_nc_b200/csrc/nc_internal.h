@@ -22,6 +22,7 @@ enum : int {
   EPI_SOFTCAP_F32 = NC_EPI_SOFTCAP_F32,
   EPI_CE_PARTIAL = 5,   // soft-cap, per-tile sum of exp(l - cap), target logit
   EPI_QKV_ROPE = 6,     // q/k heads: RoPE + per-head RMSNorm; v heads: plain store
+  EPI_QKV_ROPE_IL = 7,  // as EPI_QKV_ROPE with q/k head dims pair-interleaved (see nc_forward)
 };
 
 struct EpiParams {
@@ -71,10 +72,16 @@ nc_status attention_launch(const uint16_t* q, const uint16_t* k, const uint16_t*
 struct CastSeg {
   const float* src;
   uint16_t* dst;
-  int64_t n;  // multiple of 8
+  int64_t n;          // multiple of 8
+  bool pair_rows = false;  // rows reordered within each block of perm_d rows (see below)
 };
 // fp32 -> bf16 (round to nearest even); with f16 the bf16 value is stored as fp16.
-nc_status cast_launch(const CastSeg* segs, int nseg, bool f16, cudaStream_t stream);
+// Segments flagged pair_rows are [rows, perm_cols] matrices whose rows are
+// reordered inside every block of perm_d rows so that the RoPE partners j and
+// j + perm_d/2 become neighbours: destination row 2j <- source row j,
+// destination row 2j+1 <- source row j + perm_d/2.
+nc_status cast_launch(const CastSeg* segs, int nseg, bool f16, cudaStream_t stream, int perm_cols = 0,
+                      int perm_d = 0);
 nc_status embedding_launch(const int32_t* tokens, const float* wte, float* x, int M, int C, int V,
                            uint32_t* dev_status, cudaStream_t stream);
 nc_status rmsnorm_launch(const float* x, uint16_t* out, int M, int C, float eps, bool f16,

@@ -23,12 +23,14 @@ __device__ __forceinline__ float warp_sum(float v) {
 
 // ---------------------------------------------------------------- weight cast
 
-constexpr int kMaxCastSegs = 160;  // 3.9 KB of kernel parameters: one launch up to 26 layers
+constexpr int kMaxCastSegs = 160;  // 4.0 KB of kernel parameters: one launch up to 26 layers
 struct CastBatch {
   const float* src[kMaxCastSegs];
   uint16_t* dst[kMaxCastSegs];
   int64_t gstart[kMaxCastSegs + 1];  // prefix sums in groups of 8 elements
+  uint8_t pair_rows[kMaxCastSegs];   // segment rows pair-interleaved within perm_d-row blocks
   int nseg;
+  int perm_cols, perm_d;
 };
 
 // Each fp32 weight is rounded to bf16 (nearest even).  With F16 that bf16
@@ -56,8 +58,15 @@ __global__ void __launch_bounds__(256) cast_kernel(const __grid_constant__ CastB
       const int mid = (lo + hi + 1) >> 1;
       if (cb.gstart[mid] <= g) lo = mid; else hi = mid - 1;
     }
-    const int64_t off = (g - cb.gstart[lo]) * 8;
-    const float4* s = reinterpret_cast<const float4*>(cb.src[lo] + off);
+    const int64_t off = (g - cb.gstart[lo]) * 8;  // destination element offset
+    int64_t soff = off;
+    if (cb.pair_rows[lo]) {  // destination row 2j(+1) of a block reads source row j (+ d/2)
+      const int64_t row = off / cb.perm_cols, col = off - row * cb.perm_cols;
+      const int64_t blk = row / cb.perm_d, jj = row - blk * cb.perm_d;
+      const int64_t srow = blk * cb.perm_d + (jj >> 1) + (jj & 1) * (cb.perm_d / 2);
+      soff = srow * cb.perm_cols + col;
+    }
+    const float4* s = reinterpret_cast<const float4*>(cb.src[lo] + soff);
     const float4 a = __ldcs(s);
     const float4 b = __ldcs(s + 1);
     uint4 o;
@@ -346,15 +355,20 @@ inline nc_status last_error() { return cudaGetLastError() == cudaSuccess ? NC_OK
 
 }  // namespace
 
-nc_status cast_launch(const CastSeg* segs, int nseg, bool f16, cudaStream_t stream) {
+nc_status cast_launch(const CastSeg* segs, int nseg, bool f16, cudaStream_t stream, int perm_cols,
+                      int perm_d) {
   for (int base = 0; base < nseg; base += kMaxCastSegs) {
     CastBatch cb;
     cb.nseg = nseg - base < kMaxCastSegs ? nseg - base : kMaxCastSegs;
+    cb.perm_cols = perm_cols;
+    cb.perm_d = perm_d;
     cb.gstart[0] = 0;
     for (int i = 0; i < cb.nseg; ++i) {
       cb.src[i] = segs[base + i].src;
       cb.dst[i] = segs[base + i].dst;
       cb.gstart[i + 1] = cb.gstart[i] + segs[base + i].n / 8;
+      cb.pair_rows[i] = segs[base + i].pair_rows ? 1 : 0;
+      if (cb.pair_rows[i] && (perm_cols <= 0 || perm_cols % 8 || perm_d < 2 || perm_d % 2)) return NC_ERR_INVALID_ARG;
     }
     const int64_t groups = cb.gstart[cb.nseg];
     if (groups == 0) continue;
