@@ -20,6 +20,7 @@ sample, timed on the host cores.  ``--impl reference`` times that oracle alone.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import json
 import os
 import statistics
@@ -386,10 +387,16 @@ def main():
     ap.add_argument("--ref-prefix", type=int, default=256,
                     help="positions of batch row 0 per step of the reference (oracle) arm")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--batch", type=int, default=None,
+                    help="per-rank batch rows instead of the workload's (small profiler captures)")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
     s = SHAPES[args.config]
+    if args.batch is not None:
+        if args.batch < 1:
+            raise SystemExit("--batch must be >= 1")
+        s = dataclasses.replace(s, batch=args.batch)
     if args.impl == "reference":
         run_reference(args, s)
     else:

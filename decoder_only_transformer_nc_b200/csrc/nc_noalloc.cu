@@ -32,6 +32,7 @@ constexpr size_t kStaticBytes = (kPartialFloats + kMaxRows) * sizeof(float);  //
 
 // partials [kMaxRows][kMaxPartials] followed by target logits [kMaxRows].
 static __device__ __align__(256) float g_loss_scratch[kPartialFloats + kMaxRows];
+static_assert(sizeof(g_loss_scratch) == kStaticBytes, "scratch size");
 
 std::mutex g_mu;
 float* g_scratch_ptr[64] = {};
