@@ -5,8 +5,10 @@
 //   o[b,i,h,:] = sum_{j visible} softmax_j(q[b,i,h,:].k[b,j,g,:] / sqrt(D)) v[b,j,g,:]
 //   visible: j <= i and i - j < W;  g = h / (H / Hkv)
 //
-// Persistent kernel, one CTA per SM, work items (128-query block, head, batch
-// row) handed out round-robin.  Warp roles:
+// Work items are (128-query block, head, batch row).  The grid holds one CTA
+// per item, but a running CTA cancels the launch of a CTA that has not started
+// and takes its item (cluster launch control), so in effect one CTA per SM
+// runs and items go to whichever SM frees up first.  Warp roles:
 //   warp 0     TMA: the item's Q tile, then K and V tiles of 128 keys into two
 //              2-slot rings (4-D tensor maps over [B, T, heads, D]: tokens past
 //              T read as zeros, so tiles never leak into the next sequence).
@@ -15,7 +17,8 @@
 //              of the current one runs;
 //   warp 1     owns 512 TMEM columns; one thread issues S = Q K^T (M=128,
 //              N=128 keys) into one of two S buffers, then O += P V (A = P from
-//              shared memory, B = V read MN-major) into the O accumulator;
+//              shared memory, B = V read MN-major) into one of two O
+//              accumulators (item n uses accumulator n & 1);
 //   warps 2-9  softmax: each TMEM lane quarter (32 query rows, one per thread)
 //              is served by two warps that own 64 of the tile's 128 keys; they
 //              swap partial row maxima (and, at the end, row sums) through
@@ -24,8 +27,10 @@
 //              softmax in fp32 with exp2, write P (16-bit) to a swizzled
 //              shared-memory tile for the next MMA; O is rescaled in TMEM only
 //              when the running row maximum grows by more than 2^8 in the
-//              exponent (P stays <= 256, exact in fp16); finally O / l, staged
-//              in the freed P tile and written by a TMA store.
+//              exponent (P stays <= 256, exact in fp16).  The output O / l of
+//              an item is written after the first tile of the next item has
+//              gone to the MMA warp, so neither the last P V nor the store
+//              stalls the softmax: staged in the freed P tile, TMA-stored.
 // Only key tiles intersecting [q0 - W + 1, q0 + 127] are visited.
 // Every wait is bounded; on timeout the CTA records NC_DEV_TIMEOUT, drains
 // its copies and MMAs, frees its tensor memory and exits.
@@ -58,23 +63,58 @@ struct Geo {
   static constexpr int OFF_KV = Q_BYTES;
   static constexpr int OFF_P = OFF_KV + 2 * KV_STAGE;
   static constexpr int OFF_BAR = OFF_P + 2 * P_BYTES;
-  static constexpr int OFF_X = OFF_BAR + 256;       // row-statistics exchange [2 slots][2 halves][128]
+  static constexpr int OFF_X = OFF_BAR + 512;       // row-statistics exchange [2 slots][2 halves][128]
   static constexpr int SMEM_BYTES = OFF_X + 2 * 2 * 128 * 4;
 };
 
 struct Bars {
+  uint32_t next_item[2][4];  // work-request answers (16 B each, 16-byte aligned)
+  uint64_t next_full[2];     // answer n & 1 has landed
+  uint64_t next_empty[2];    // every role has read answer n & 1
   uint64_t q_full, q_empty;
   uint64_t k_full[2], k_empty[2];
   uint64_t v_full[2], v_empty[2];
   uint64_t s_full[2], s_free[2];
   uint64_t p_full[2], p_free[2];
-  uint64_t o_free;
+  uint64_t o_free[2];  // O accumulator n & 1 has been read out for item n
   uint64_t xbar[4];  // per lane quarter: both column halves posted their row statistics
   uint64_t drain;
   uint32_t tmem_base;
   int abort_flag;
 };
-static_assert(sizeof(Bars) <= 256, "barrier block");
+static_assert(sizeof(Bars) <= 512, "barrier block");
+constexpr int kNextReaders = 2 + SM_WARPS;  // TMA thread, MMA thread, softmax warps
+
+// Dynamic work distribution.  The grid has one CTA per work item.  While a
+// CTA works on an item it asks the hardware scheduler to cancel the launch of
+// a CTA that has not started yet (cluster launch control) and, if that
+// succeeds, takes over that CTA's item next.  Items are thus handed out in
+// launch order to whichever SM frees up first, while each SM keeps its
+// barriers, tensor memory and pipelines across items.  One request is in
+// flight at a time and none is issued after one has failed.
+__device__ __forceinline__ void next_item_request(uint32_t answer, uint32_t bar) {
+  asm volatile("clusterlaunchcontrol.try_cancel.async.shared::cta.mbarrier::complete_tx::bytes.b128 [%0], [%1];"
+               ::"r"(answer), "r"(bar)
+               : "memory");
+}
+
+// Item index carried by an answer, or -1 when no launch was cancelled.
+__device__ __forceinline__ int next_item_decode(uint32_t answer, int n_items) {
+  uint32_t got = 0, x = 0, y = 0, z = 0;
+  asm volatile(
+      "{\n\t"
+      ".reg .pred p;\n\t"
+      ".reg .b128 r;\n\t"
+      "ld.shared.b128 r, [%4];\n\t"
+      "clusterlaunchcontrol.query_cancel.is_canceled.pred.b128 p, r;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t"
+      "@p clusterlaunchcontrol.query_cancel.get_first_ctaid.v4.b32.b128 {%1, %2, %3, _}, r;\n\t"
+      "}"
+      : "+r"(got), "+r"(x), "+r"(y), "+r"(z)
+      : "r"(answer)
+      : "memory");
+  return (got && (int)x < n_items) ? (int)x : -1;
+}
 
 __device__ __forceinline__ float ex2f(float x) {
   float y;
@@ -87,9 +127,10 @@ struct Item {
 };
 
 // Items are numbered with the query block fastest (last block first), then the
-// head, then the batch row: the CTAs running at the same time cover all query
-// blocks of a few heads, so each head's K/V is fetched from HBM about once and
-// then served from L2.
+// head, then the batch row.  They are handed out in about that order, so the
+// CTAs running at the same time cover all query blocks of a few heads (each
+// head's K/V is fetched from HBM about once and then served from L2), and
+// within a head the longest items go first, which keeps the tail short.
 __device__ __forceinline__ Item item_of(int idx, int B, int H, int T, int W) {
   const int n_qb = (T + BQ - 1) / BQ;
   Item it;
@@ -139,6 +180,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const int group = H / Hkv;
 
   if (threadIdx.x == 0) {
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(smem_u32(&bar->next_full[i]), 1);
+      mbar_init(smem_u32(&bar->next_empty[i]), kNextReaders);
+    }
     mbar_init(smem_u32(&bar->q_full), 1);
     mbar_init(smem_u32(&bar->q_empty), 1);
     for (int i = 0; i < 2; ++i) {
@@ -151,7 +196,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_init(smem_u32(&bar->p_full[i]), SM_WARPS);
       mbar_init(smem_u32(&bar->p_free[i]), 1);
     }
-    mbar_init(smem_u32(&bar->o_free), SM_WARPS);
+    mbar_init(smem_u32(&bar->o_free[0]), SM_WARPS);
+    mbar_init(smem_u32(&bar->o_free[1]), SM_WARPS);
     for (int i = 0; i < 4; ++i) mbar_init(smem_u32(&bar->xbar[i]), 2);
     mbar_init(smem_u32(&bar->drain), 1);
     bar->abort_flag = 0;
@@ -178,9 +224,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       uint32_t outstanding = 0, out_phase = 0;  // bits 0,1: K slots; bit 2: Q; bits 3,4: V slots
       int g = 0;
       bool ok = true;
-      for (int idx = blockIdx.x, n = 0; idx < n_items && ok; idx += gridDim.x, ++n) {
+      bool asked = false;  // a work request is in flight (answer slot ask_slot, phase ask_phase)
+      int ask_slot = 0;
+      uint32_t ask_phase = 0;
+      int idx = blockIdx.x;
+      for (int n = 0; idx >= 0 && ok; ++n) {
         const Item it = item_of(idx, B, H, T, W);
         const int gh = it.h / group;
+        const int ns = n & 1;
+        // Ask for the next item now; the answer is read once this item is loaded.
+        if (!mbar_wait(smem_u32(&bar->next_empty[ns]), ((uint32_t)(n >> 1) & 1) ^ 1, ctl)) break;
+        mbar_arrive_expect_tx(smem_u32(&bar->next_full[ns]), 16);
+        next_item_request(smem_u32(&bar->next_item[ns][0]), smem_u32(&bar->next_full[ns]));
+        asked = true;
+        ask_slot = ns;
+        ask_phase = (uint32_t)(n >> 1) & 1;
         if (!mbar_wait(smem_u32(&bar->q_empty), (n & 1) ^ 1, ctl)) break;
         mbar_arrive_expect_tx(smem_u32(&bar->q_full), G::Q_BYTES);
         for (int a = 0; a < G::KA; ++a)
@@ -222,10 +280,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
         }
         g += it.n_tiles;
+        if (!ok) break;
+        if (!mbar_wait(smem_u32(&bar->next_full[ns]), (uint32_t)(n >> 1) & 1, ctl)) break;
+        asked = false;
+        idx = next_item_decode(smem_u32(&bar->next_item[ns][0]), n_items);
+        fence_proxy_async_smem();
+        mbar_arrive(smem_u32(&bar->next_empty[ns]));
       }
       if (!ok || bar->abort_flag) {
         int zero = 0;
         const WaitCtl dctl{&zero, nullptr, limit_ns};
+        if (asked) mbar_wait(smem_u32(&bar->next_full[ask_slot]), ask_phase, dctl);
         for (int st = 0; st < 2; ++st) {
           if (outstanding & (1u << st)) mbar_wait(smem_u32(&bar->k_full[st]), (out_phase >> st) & 1u, dctl);
           if (outstanding & (8u << st))
@@ -239,7 +304,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       // ---------------- MMA issuer
       int g = 0;
       bool ok = true;
-      for (int idx = blockIdx.x, n = 0; idx < n_items && ok; idx += gridDim.x, ++n) {
+      int idx = blockIdx.x;
+      for (int n = 0; idx >= 0 && ok; ++n) {
         const Item it = item_of(idx, B, H, T, W);
         if (!mbar_wait(smem_u32(&bar->q_full), n & 1, ctl)) break;
         tc_fence_after();
@@ -274,7 +340,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               ok = false;
               break;
             }
-            if (j == 1 && !mbar_wait(smem_u32(&bar->o_free), (n & 1) ^ 1, ctl)) {
+            if (j == 1 && !mbar_wait(smem_u32(&bar->o_free[n & 1]), ((uint32_t)(n >> 1) & 1) ^ 1, ctl)) {
               ok = false;
               break;
             }
@@ -285,13 +351,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             for (int k = 0; k < BKV / 16; ++k) {
               const uint64_t adesc = sw128_kmajor_desc(pbase + (k >> 2) * ATOM + (k & 3) * 32);
               const uint64_t bdesc = sw128_desc(vbase + k * 2048, ATOM, 1024);
-              umma_f16(tmem + O_COL, adesc, bdesc, IDESC_PV, (j > 1 || k > 0) ? 1u : 0u);
+              umma_f16(tmem + O_COL + (n & 1) * D, adesc, bdesc, IDESC_PV, (j > 1 || k > 0) ? 1u : 0u);
             }
             umma_commit(smem_u32(&bar->p_free[pb]));
             umma_commit(smem_u32(&bar->v_empty[pb]));
           }
         }
         g += it.n_tiles;
+        if (!ok) break;
+        const int ns = n & 1;
+        if (!mbar_wait(smem_u32(&bar->next_full[ns]), (uint32_t)(n >> 1) & 1, ctl)) break;
+        idx = next_item_decode(smem_u32(&bar->next_item[ns][0]), n_items);
+        fence_proxy_async_smem();
+        mbar_arrive(smem_u32(&bar->next_empty[ns]));
       }
       umma_commit(smem_u32(&bar->drain));
       int zero = 0;
@@ -322,11 +394,84 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
       return xval[(slot * 2 + (half ^ 1)) * 128 + r];
     };
+    // The output of item n is written while item n + 1 runs: once the first
+    // tile of n + 1 has been handed to the MMA warp, the last P V of n has had
+    // a tile's worth of softmax time to land in O buffer n & 1, and the TMA
+    // store stages in the P buffer of n's last tile, which the next tile of
+    // n + 1 does not use.
+    struct Pending {
+      int b, h, q0, gl, ob;
+      float l;
+    };
+    Pending pend{};
+    bool has_pend = false;
+    uint32_t store_busy = 0;  // P buffers a TMA store of this warp may still be reading
+    auto finish = [&](const Pending& pd, bool& ok_) {
+      const float lsum = pd.l + exchange(pd.l, ok_);  // full row sum
+      if (!ok_) return;
+      if (__any_sync(0xffffffffu,
+                     !mbar_wait(smem_u32(&bar->p_free[pd.gl & 1]), (uint32_t)(pd.gl >> 1) & 1, ctl))) {
+        ok_ = false;
+        return;
+      }
+      tc_fence_after();
+      const float inv = lsum > 0.0f ? 1.0f / lsum : 0.0f;
+      const uint32_t ocol = O_COL + pd.ob * D + half * DC;
+      uint32_t rr[DC / 32][32];
+#pragma unroll
+      for (int c = 0; c < DC / 32; ++c) tmem_ld_32x32b_x32(tmem + lane_off + ocol + c * 32, rr[c]);
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&bar->o_free[pd.ob]));
+      if constexpr (D == 128) {
+        // Stage this warp's 32 rows x 64 columns in the P buffer of the item's
+        // last tile (only this warp writes these rows of this half) and let
+        // TMA write them to out.
+        uint8_t* sbase = sm + G::OFF_P + (pd.gl & 1) * G::P_BYTES + half * ATOM;
+        uint8_t* srow = sbase + r * 128;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          uint4 pk;
+          const int c = q >> 2, e0 = (q & 3) * 8;
+          pk.x = Half<F16>::pack2(__uint_as_float(rr[c][e0 + 0]) * inv, __uint_as_float(rr[c][e0 + 1]) * inv);
+          pk.y = Half<F16>::pack2(__uint_as_float(rr[c][e0 + 2]) * inv, __uint_as_float(rr[c][e0 + 3]) * inv);
+          pk.z = Half<F16>::pack2(__uint_as_float(rr[c][e0 + 4]) * inv, __uint_as_float(rr[c][e0 + 5]) * inv);
+          pk.w = Half<F16>::pack2(__uint_as_float(rr[c][e0 + 6]) * inv, __uint_as_float(rr[c][e0 + 7]) * inv);
+          *reinterpret_cast<uint4*>(srow + ((q ^ (r & 7)) << 4)) = pk;
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_4d(&tmO, smem_u32(sbase + quarter * 32 * 128), half * DC, pd.h, pd.q0 + (int)quarter * 32,
+                       pd.b);
+          bulk_commit();
+        }
+        store_busy |= 1u << (pd.gl & 1);
+      } else {
+        const int i = pd.q0 + r;
+        if (i < T) {
+          uint16_t* orow = out + (((int64_t)pd.b * T + i) * H + pd.h) * D + half * DC;
+#pragma unroll
+          for (int q = 0; q < DC / 8; ++q) {
+            uint4 pk;
+            const int c = q >> 2, e0 = (q & 3) * 8;
+            pk.x = Half<F16>::pack2(__uint_as_float(rr[c][e0 + 0]) * inv, __uint_as_float(rr[c][e0 + 1]) * inv);
+            pk.y = Half<F16>::pack2(__uint_as_float(rr[c][e0 + 2]) * inv, __uint_as_float(rr[c][e0 + 3]) * inv);
+            pk.z = Half<F16>::pack2(__uint_as_float(rr[c][e0 + 4]) * inv, __uint_as_float(rr[c][e0 + 5]) * inv);
+            pk.w = Half<F16>::pack2(__uint_as_float(rr[c][e0 + 6]) * inv, __uint_as_float(rr[c][e0 + 7]) * inv);
+            reinterpret_cast<uint4*>(orow)[q] = pk;
+          }
+        }
+      }
+    };
     int g = 0;
     bool ok = true;
-    for (int idx = blockIdx.x, n = 0; idx < n_items && ok; idx += gridDim.x, ++n) {
+    int idx = blockIdx.x;
+    for (int n = 0; idx >= 0 && ok; ++n) {
       const Item it = item_of(idx, B, H, T, W);
       const int i = it.q0 + r;  // this thread's query position
+      const uint32_t ocol = O_COL + (n & 1) * D + half * DC;
       float m_used = -INFINITY, l = 0.0f;
       for (int j = 0; j < it.n_tiles; ++j) {
         const int gj = g + j;
@@ -391,11 +536,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll 1
           for (int c = 0; c < DC / 32; ++c) {
             uint32_t rr[32];
-            tmem_ld_32x32b_x32(tmem + lane_off + O_COL + half * DC + c * 32, rr);
+            tmem_ld_32x32b_x32(tmem + lane_off + ocol + c * 32, rr);
             tmem_wait_ld();
 #pragma unroll
             for (int e = 0; e < 32; ++e) rr[e] = __float_as_uint(__uint_as_float(rr[e]) * alpha);
-            tmem_st_32x32b_x32(tmem + lane_off + O_COL + half * DC + c * 32, rr);
+            tmem_st_32x32b_x32(tmem + lane_off + ocol + c * 32, rr);
           }
           tmem_wait_st();
           if (need) {
@@ -408,6 +553,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (__any_sync(0xffffffffu, !mbar_wait(smem_u32(&bar->p_free[sb]), (use & 1) ^ 1, ctl))) {
           ok = false;
           break;
+        }
+        if (store_busy & (1u << sb)) {  // an output store still reads this buffer
+          if (lane == 0) bulk_wait_read0();
+          __syncwarp();
+          store_busy = 0;
         }
         uint8_t* prow = sm + G::OFF_P + sb * G::P_BYTES + half * ATOM + r * 128;
         float ls8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};  // 8 independent sums
@@ -431,66 +581,27 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(&bar->p_full[sb]));
+        if (j == 0 && has_pend) {
+          has_pend = false;
+          finish(pend, ok);
+          if (!ok) break;
+        }
       }
       if (!ok) break;
-      // epilogue: full row sum, wait for the last P V, then out = O / l
-      l += exchange(l, ok);
-      if (!ok) break;
-      const int gl = g + it.n_tiles - 1;
-      if (__any_sync(0xffffffffu, !mbar_wait(smem_u32(&bar->p_free[gl & 1]), (uint32_t)(gl >> 1) & 1, ctl))) {
+      pend = Pending{it.b, it.h, it.q0, g + it.n_tiles - 1, n & 1, l};
+      has_pend = true;
+      g += it.n_tiles;
+      const int ns = n & 1;
+      if (__any_sync(0xffffffffu, !mbar_wait(smem_u32(&bar->next_full[ns]), (uint32_t)(n >> 1) & 1, ctl))) {
         ok = false;
         break;
       }
-      tc_fence_after();
-      const float inv = l > 0.0f ? 1.0f / l : 0.0f;
-      uint32_t rr[DC / 32][32];
-#pragma unroll
-      for (int c = 0; c < DC / 32; ++c) tmem_ld_32x32b_x32(tmem + lane_off + O_COL + half * DC + c * 32, rr[c]);
-      tmem_wait_ld();
-      if constexpr (D == 128) {
-        // Stage this warp's 32 rows x 64 columns in the last tile's P buffer
-        // (its P V has completed; only this warp writes these rows of this
-        // half) and let TMA write them to out.
-        uint8_t* srow = sm + G::OFF_P + (gl & 1) * G::P_BYTES + half * ATOM + r * 128;
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          uint4 pk;
-          const int c = q >> 2, e0 = (q & 3) * 8;
-          pk.x = Half<F16>::pack2(__uint_as_float(rr[c][e0 + 0]) * inv, __uint_as_float(rr[c][e0 + 1]) * inv);
-          pk.y = Half<F16>::pack2(__uint_as_float(rr[c][e0 + 2]) * inv, __uint_as_float(rr[c][e0 + 3]) * inv);
-          pk.z = Half<F16>::pack2(__uint_as_float(rr[c][e0 + 4]) * inv, __uint_as_float(rr[c][e0 + 5]) * inv);
-          pk.w = Half<F16>::pack2(__uint_as_float(rr[c][e0 + 6]) * inv, __uint_as_float(rr[c][e0 + 7]) * inv);
-          *reinterpret_cast<uint4*>(srow + ((q ^ (r & 7)) << 4)) = pk;
-        }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) {
-          tma_store_4d(&tmO, smem_u32(sm + G::OFF_P + (gl & 1) * G::P_BYTES + half * ATOM + quarter * 32 * 128),
-                       half * DC, it.h, it.q0 + (int)quarter * 32, it.b);
-          bulk_commit();
-          bulk_wait_read0();
-        }
-        __syncwarp();
-      } else {
-        if (i < T) {
-          uint16_t* orow = out + (((int64_t)it.b * T + i) * H + it.h) * D + half * DC;
-#pragma unroll
-          for (int q = 0; q < DC / 8; ++q) {
-            uint4 pk;
-            const int c = q >> 2, e0 = (q & 3) * 8;
-            pk.x = Half<F16>::pack2(__uint_as_float(rr[c][e0 + 0]) * inv, __uint_as_float(rr[c][e0 + 1]) * inv);
-            pk.y = Half<F16>::pack2(__uint_as_float(rr[c][e0 + 2]) * inv, __uint_as_float(rr[c][e0 + 3]) * inv);
-            pk.z = Half<F16>::pack2(__uint_as_float(rr[c][e0 + 4]) * inv, __uint_as_float(rr[c][e0 + 5]) * inv);
-            pk.w = Half<F16>::pack2(__uint_as_float(rr[c][e0 + 6]) * inv, __uint_as_float(rr[c][e0 + 7]) * inv);
-            reinterpret_cast<uint4*>(orow)[q] = pk;
-          }
-        }
-      }
-      tc_fence_before();
+      idx = next_item_decode(smem_u32(&bar->next_item[ns][0]), n_items);
+      fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&bar->o_free));
-      g += it.n_tiles;
+      if (lane == 0) mbar_arrive(smem_u32(&bar->next_empty[ns]));
     }
+    if (ok && has_pend) finish(pend, ok);
     if (lane == 0) bulk_wait0();
     __syncwarp();
   }
@@ -537,9 +648,9 @@ static nc_status launch_t(const uint16_t* q, const uint16_t* k, const uint16_t* 
     const uint32_t box[4] = {64, 1, 32, 1};
     if (!encode_tensor_map(&mo, F16, 4, out, dims, strides, box)) return NC_ERR_CUDA;
   }
-  const int items = B * H * ((T + BQ - 1) / BQ);
-  const int sms = device_sm_count();
-  const int grid = items < sms ? items : sms;
+  // One CTA per work item; running CTAs take over the items of CTAs that have
+  // not started (see next_item_request), so about one CTA per SM ever runs.
+  const int grid = B * H * ((T + BQ - 1) / BQ);
   const float scale_log2 = 1.4426950408889634f / sqrtf((float)D);
   attn_tc_kernel<D, F16><<<grid, NUM_THREADS, G::SMEM_BYTES, stream>>>(
       mq, mk, mv, mo, out, B, T, H, Hkv, W, scale_log2, dev_status, kWaitLimitNs);
