@@ -43,6 +43,12 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 DTYPE_NOTE = ("f16 tensor-core operands (weights rounded fp32->bf16 as the method casts them, "
               "held exactly in f16; activations f16), fp32 accumulation, fp32 residual/softmax/loss")
 GEMM_KINDS = ("gemm_qkv", "gemm_attn_proj", "gemm_fc", "gemm_mlp_proj", "gemm_lm_head")
+ROOFLINE_KIND = "gemm_fc"  # the kind with the largest share of the step
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one c_fc launch of
+# the d20 workload at B=32, T=2048, from a one-pass ncu capture of this kernel:
+# 181.33 MB read (A + W once) + 618.75 MB written (the rest of the 671 MB output
+# is still in L2 when the kernel ends).  Valid for that workload and kernel only.
+FC_TRAFFIC = {("d20", 32, 2048): 181.33e6 + 618.75e6}
 
 
 def load_peaks():
@@ -304,6 +310,8 @@ def run_ours(args, s):
     flops = nc.forward_flops(cfg, B, T)
     peaks, peak_src = load_peaks()
 
+    rk_ms, rk_n = per_kind.get(ROOFLINE_KIND, [0.0, 0])
+    rk_achieved = kernel_work(s, ROOFLINE_KIND) * rk_n / (rk_ms / 1e3) / 1e12 if rk_ms > 0 else 0.0
     gemm_ms = sum(per_kind[k][0] for k in GEMM_KINDS if k in per_kind)
     gemm_launches = sum(per_kind[k][1] for k in GEMM_KINDS if k in per_kind)
     gemm_flops = sum(kernel_work(s, k) * per_kind[k][1] for k in GEMM_KINDS if k in per_kind)
@@ -341,11 +349,18 @@ def run_ours(args, s):
                                  "measured_sustained": round(100 * tflops / world / peak, 2),
                                  "datasheet_dense_2250": round(100 * tflops / world / 2250.0, 2),
                                  "source": peak_src},
-            "roofline": {"kernel": "gemm_kernel (tcgen05 projection GEMMs: qkv, attn c_proj, c_fc, mlp c_proj, lm_head)",
-                         "bound": "tensor", "achieved": round(achieved, 1),
-                         "peak": peak, "peak_kind": f"bf16_tflops_sustained ({peak_src})",
-                         "unit": "TFLOP/s", "frac": round(achieved / peak, 4), "traffic": None,
-                         "launches": gemm_launches, "avg_launch_ms": round(gemm_ms / max(1, gemm_launches), 4)},
+            "roofline": {"kernel": "gemm_kernel<EPI_RELU2_16> (c_fc + ReLU^2: M=B*T, N=4C, K=C)",
+                         "bound": "tensor", "achieved": round(rk_achieved, 1),
+                         "peak": peak,
+                         "peak_kind": f"bf16_tflops_sustained ({peak_src}); f16 operands, same nominal rate",
+                         "unit": "TFLOP/s", "frac": round(rk_achieved / peak, 4),
+                         "traffic": FC_TRAFFIC.get((s.name, B, T)),
+                         "algorithmic_bytes": 2 * (B * T * s.d_model + 4 * s.d_model * s.d_model
+                                                   + 4 * B * T * s.d_model),
+                         "launches": rk_n, "avg_launch_ms": round(rk_ms / max(1, rk_n), 4)},
+            "gemm_family": {"kernel": "gemm_kernel, all projections (qkv, attn c_proj, c_fc, mlp c_proj, lm_head)",
+                            "achieved": round(achieved, 1), "frac": round(achieved / peak, 4),
+                            "launches": gemm_launches},
             "kernels": kernels,
             "gpu_launches": n_launch * args.steps,
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": int(x.nbytes + y.nbytes),
