@@ -43,6 +43,23 @@ function here, and the CUDA library takes the same reading independently):
 * soft-cap 15*tanh(z/15) is applied before the loss and the returned logits are
   the capped ones; loss = mean natural-log NLL over targets != -1 (NaN if none).
 
+Further terms of the full nanochat forward ("Nanochat与nanoGPT对比" §1 table and
+notes), each optional (``forward(..., extras=...)``), with these readings of the
+one-line descriptions there:
+
+* smear: gate is a bias-free linear map C -> 1 applied to the current token's
+  embedding (its weight enters as bf16 like every linear layer);
+  x_t = e_t + sigmoid(gate(e_t)) e_{t-1}, position 0 of each row unchanged;
+* residual lambdas + x0: before block l, x = resid_lambdas[l] x +
+  x0_lambdas[l] x0, x0 being the (smeared) embedding output;
+* value embeddings: a table [V, Hkv*D] per layer on every other layer counted
+  back from the last (which always has one); v = v + gate * table[idx] with one
+  plain learnable gate per kv head, added to v after its projection;
+* backout: x_mid is the stream after the first L // 2 blocks (before block
+  L // 2 mixes in x0); before the final norm x = x - lambda * x_mid.
+
+Those pins live in ``tests/test_oracle_extras.py``.
+
 Parity pins live in ``tests/test_oracle_pins.py``.  Every function below is
 pinned there by closed forms, invariants, brute force or an independent library
 routine.  The composition of the full forward at random weights is pinned only
@@ -67,4 +84,7 @@ from .model import (  # noqa: F401
     cross_entropy,
     embed,
     forward,
+    smear,
+    value_embed_layers,
+    backout_layer,
 )

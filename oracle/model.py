@@ -216,8 +216,39 @@ def embed(wte: np.ndarray, idx: np.ndarray) -> np.ndarray:
     return np.asarray(wte, dtype=F64)[np.asarray(idx)]
 
 
+def value_embed_layers(n_layer: int) -> list:
+    """Layers that carry a value embedding: every other layer, counted back from
+    the last one, which always has one ("Nanochat与nanoGPT对比" §1, value
+    residual note)."""
+    return [(n_layer - 1 - l) % 2 == 0 for l in range(n_layer)]
+
+
+def backout_layer(n_layer: int) -> int:
+    """The block whose input is cached for backout: the middle of the stack,
+    i.e. the residual stream after the first n_layer // 2 blocks (reading of the
+    backout note in "Nanochat与nanoGPT对比" §1, which only says "a middle
+    layer")."""
+    return n_layer // 2
+
+
+def smear(x: np.ndarray, gate_w: np.ndarray) -> np.ndarray:
+    """"Nanochat与nanoGPT对比" §1, smear note: mix the previous token's embedding
+    into the current one through a learnable gate, x_t + sigmoid(gate(x_t)) x_{t-1}.
+
+    gate is a bias-free linear map C -> 1 (its fp32 weight enters as bf16, like
+    every linear layer, see ``linear``); the first position of each row has no
+    previous token and is left unchanged.  x: [B, T, C].
+    """
+    x = np.asarray(x, dtype=F64)
+    z = linear(x, np.asarray(gate_w).reshape(1, -1))[..., 0]  # [B, T]
+    g = 1.0 / (1.0 + np.exp(-z))
+    prev = np.zeros_like(x)
+    prev[:, 1:] = x[:, :-1]
+    return x + g[..., None] * prev
+
+
 def forward(cfg: OracleConfig, weights: dict, idx: np.ndarray, targets=None,
-            want_logits: bool = True):
+            want_logits: bool = True, extras: dict = None):
     """The whole forward for the rows of ``idx`` ([B, T] int).
 
     Steps in the order of "从文本到聊天模型" §5 (embedding, blocks of
@@ -225,9 +256,24 @@ def forward(cfg: OracleConfig, weights: dict, idx: np.ndarray, targets=None,
     the block internals of "Nanochat与nanoGPT对比" §1 (split c_q/c_k/c_v,
     RoPE then QK-norm, SSSL windows, GQA, ReLU^2, final norm, soft-cap).
 
+    ``extras`` (optional) adds the further terms of the full nanochat forward
+    listed in "Nanochat与nanoGPT对比" §1; each key switches one on:
+
+    * ``smear_gate`` [C]: x = smear(wte[idx]) (see ``smear``);
+    * ``resid_lambdas`` / ``x0_lambdas`` [L]: before block l the stream becomes
+      resid_lambdas[l] * x + x0_lambdas[l] * x0, x0 being the (smeared)
+      embedding output;
+    * ``value_embeds`` (list of L entries, [V, Hkv*D] or None) and ``ve_gates``
+      (list of L entries, [Hkv] or None): on the layers of
+      ``value_embed_layers``, v = v + gate * ve with ve = value_embeds[l][idx]
+      and one gate per kv head;
+    * ``backout_lambda`` (scalar): x_mid = the stream after the first
+      ``backout_layer`` blocks; before the final norm x = x - lambda * x_mid.
+
     Returns a dict with ``logits`` ([B,T,V] capped, fp64, if ``want_logits``),
     ``token_loss`` ([B,T]) and ``loss`` (scalar) when targets are given.
     """
+    ex = extras or {}
     idx = np.asarray(idx)
     B, T = idx.shape
     C, H, Hkv, D = cfg.d_model, cfg.n_head, cfg.n_kv_head, cfg.head_dim
@@ -235,17 +281,31 @@ def forward(cfg: OracleConfig, weights: dict, idx: np.ndarray, targets=None,
     windows = layer_windows(cfg)
     cos, sin = rope_tables(T, D, cfg.rope_base)
     x = embed(weights["wte"], idx)  # [B,T,C]
+    if "smear_gate" in ex:
+        x = smear(x, ex["smear_gate"])
+    x0 = x
+    L = len(weights["layers"])
+    x_mid = None
     for l, lw in enumerate(weights["layers"]):
+        if "backout_lambda" in ex and l == backout_layer(L):
+            x_mid = x
+        if "resid_lambdas" in ex:
+            x = F64(ex["resid_lambdas"][l]) * x + F64(ex["x0_lambdas"][l]) * x0
         a = rms_norm(x, eps)
         q = linear(a, lw["c_q"]).reshape(B, T, H, D)
         k = linear(a, lw["c_k"]).reshape(B, T, Hkv, D)
         v = linear(a, lw["c_v"]).reshape(B, T, Hkv, D)
+        if "value_embeds" in ex and value_embed_layers(L)[l]:
+            ve = embed(ex["value_embeds"][l], idx).reshape(B, T, Hkv, D)
+            v = v + np.asarray(ex["ve_gates"][l], dtype=F64)[None, None, :, None] * ve
         q = rms_norm(rope(q, cos, sin), eps)
         k = rms_norm(rope(k, cos, sin), eps)
         o = attention(q, k, v, windows[l])
         x = x + linear(o.reshape(B, T, H * D), lw["attn_proj"])
         a = rms_norm(x, eps)
         x = x + relu2_mlp(a, lw["c_fc"], lw["mlp_proj"])
+    if x_mid is not None:
+        x = x - F64(ex["backout_lambda"]) * x_mid
     a = rms_norm(x, eps)
     logits = softcap(linear(a, weights["lm_head"]), cfg.softcap)  # [B,T,V]
     res = {}

@@ -13,7 +13,14 @@ Recipe (all draws are numpy ``Generator(PCG64(seed))``):
 * tokens, seed 5678, a ``[B, T+1]`` int32 array uniform in ``[0, V)``; the model
   reads ``[:, :-1]`` and is scored against ``[:, 1:]`` (the one-token shift of the
   pretraining dataloader);
-* attention-sweep q/k/v, seed 91011, float32 ``standard_normal``.
+* attention-sweep q/k/v, seed 91011, float32 ``standard_normal``;
+* the further weights of the full nanochat forward (``make_extras``), seed 4321,
+  in the order smear gate [C] (``standard_normal``), resid lambdas [L]
+  (``1 + 0.1 * standard_normal``), x0 lambdas [L] (``0.1 * standard_normal``),
+  backout lambda (``0.5 + 0.1 * standard_normal``); then, from the sub-stream
+  ``PCG64([4321, l + 1])`` of layer l, a value embedding table [V, Hkv*D]
+  (``0.5 * standard_normal``) and per-kv-head gates [Hkv] (``standard_normal``).  Tables are drawn for every layer; which layers
+  use one is the model's rule, not the generator's.
 
 The shapes are those of the five benchmark configurations of the nanochat
 GPT forward: a tiny 2-layer model, d12, d20, d26 and a d26-depth GQA variant.
@@ -27,6 +34,7 @@ import numpy as np
 WEIGHT_SEED = 1234
 TOKEN_SEED = 5678
 ATTN_SEED = 91011
+EXTRAS_SEED = 4321
 INIT_STD = 0.02
 
 
@@ -101,6 +109,39 @@ def make_weights(s: ModelShape, seed: int = WEIGHT_SEED) -> dict:
     for _ in range(s.n_layer):
         out["layers"].append({n: draw(n) for n in LAYER_WEIGHT_NAMES})
     out["lm_head"] = draw("lm_head")
+    return out
+
+
+def make_extras(s: ModelShape, seed: int = EXTRAS_SEED, layers=None) -> dict:
+    """Seeded weights of the full nanochat forward's further terms (float32).
+
+    ``layers`` (optional iterable of layer indices) limits which layers get a
+    value-embedding table and gates drawn (the others are None); the draws of
+    the drawn layers do not depend on that choice.
+    """
+    rng = np.random.Generator(np.random.PCG64(seed))
+    L, C, V = s.n_layer, s.d_model, s.vocab
+    kvw = s.n_kv_head * s.head_dim
+    out = {
+        "smear_gate": rng.standard_normal(C, dtype=np.float32),
+        "resid_lambdas": (1.0 + 0.1 * rng.standard_normal(L)).astype(np.float32),
+        "x0_lambdas": (0.1 * rng.standard_normal(L)).astype(np.float32),
+        "backout_lambda": np.float32(0.5 + 0.1 * rng.standard_normal()),
+        "value_embeds": [],
+        "ve_gates": [],
+    }
+    keep = set(range(L)) if layers is None else set(layers)
+    for l in range(L):
+        # one sub-stream per layer, so skipping a layer leaves the others intact
+        sub = np.random.Generator(np.random.PCG64([seed, l + 1]))
+        if l in keep:
+            t = sub.standard_normal((V, kvw), dtype=np.float32)
+            t *= np.float32(0.5)
+            out["value_embeds"].append(t)
+            out["ve_gates"].append(sub.standard_normal(s.n_kv_head, dtype=np.float32))
+        else:
+            out["value_embeds"].append(None)
+            out["ve_gates"].append(None)
     return out
 
 
