@@ -12,6 +12,8 @@ import ctypes
 import os
 from dataclasses import dataclass
 
+import numpy as np
+
 __all__ = [
     "NcError", "NcConfig", "lib", "init_config", "make_config", "check_config", "layer_window",
     "workspace_bytes", "forward_flops", "Model", "forward", "LaunchTrace", "KERNEL_KINDS", "get_status", "cast_bf16", "embedding",
@@ -43,7 +45,8 @@ class NcConfig(ctypes.Structure):
                 ("n_kv_head", ctypes.c_int32), ("head_dim", ctypes.c_int32), ("vocab", ctypes.c_int32),
                 ("seq_len", ctypes.c_int32), ("short_window", ctypes.c_int32),
                 ("window_pattern", ctypes.c_char * 8), ("softcap", ctypes.c_float),
-                ("norm_eps", ctypes.c_float), ("rope_base", ctypes.c_float), ("act_dtype", ctypes.c_int32)]
+                ("norm_eps", ctypes.c_float), ("rope_base", ctypes.c_float), ("act_dtype", ctypes.c_int32),
+                ("extras", ctypes.c_uint32)]
 
     def __repr__(self):
         return ("NcConfig(n_layer=%d, d_model=%d, n_head=%d, n_kv_head=%d, head_dim=%d, vocab=%d, "
@@ -57,7 +60,15 @@ _FPP = ctypes.POINTER(ctypes.c_void_p)
 
 class NcWeights(ctypes.Structure):
     _fields_ = [("wte", ctypes.c_void_p), ("c_q", _FPP), ("c_k", _FPP), ("c_v", _FPP),
-                ("attn_proj", _FPP), ("c_fc", _FPP), ("mlp_proj", _FPP), ("lm_head", ctypes.c_void_p)]
+                ("attn_proj", _FPP), ("c_fc", _FPP), ("mlp_proj", _FPP), ("lm_head", ctypes.c_void_p),
+                ("smear_gate", ctypes.c_void_p), ("value_embeds", _FPP), ("ve_gates", _FPP),
+                ("resid_lambdas", ctypes.c_void_p), ("x0_lambdas", ctypes.c_void_p),
+                ("backout_lambda", ctypes.c_void_p)]
+
+
+# Further terms of the full nanochat forward (bits of NcConfig.extras).
+EXTRA_SMEAR, EXTRA_VALUE_EMBED, EXTRA_RESID_LAMBDAS, EXTRA_BACKOUT = 1, 2, 4, 8
+EXTRA_ALL = 15
 
 
 class NcTrace(ctypes.Structure):
@@ -85,6 +96,7 @@ def lib():
             "nc_init_config": (i32, [cfgp, i32, i32, i32, i32, i32, i32]),
             "nc_check_config": (i32, [cfgp]),
             "nc_layer_window": (i32, [cfgp, i32]),
+            "nc_layer_value_embed": (i32, [cfgp, i32]),
             "nc_workspace_bytes": (sz, [cfgp, i32, i32]),
             "nc_forward_flops": (ctypes.c_double, [cfgp, i32, i32]),
             "nc_status_string": (ctypes.c_char_p, [i32]),
@@ -144,10 +156,10 @@ def init_config(depth: int, aspect_ratio: int = 64, head_dim: int = 128, n_kv_he
 
 def make_config(n_layer, d_model, n_head, n_kv_head, head_dim, seq_len, vocab, short_window=0,
                 window_pattern="SSSL", softcap=15.0, norm_eps=1e-6, rope_base=10000.0,
-                act_dtype=F16) -> NcConfig:
+                act_dtype=F16, extras=0) -> NcConfig:
     c = NcConfig(n_layer, d_model, n_head, n_kv_head, head_dim, vocab, seq_len,
                  short_window if short_window > 0 else seq_len // 4, window_pattern.encode(),
-                 softcap, norm_eps, rope_base, act_dtype)
+                 softcap, norm_eps, rope_base, act_dtype, extras)
     _check(lib().nc_check_config(ctypes.byref(c)), "nc_check_config")
     return c
 
@@ -158,6 +170,10 @@ def check_config(c: NcConfig) -> int:
 
 def layer_window(c: NcConfig, layer: int) -> int:
     return lib().nc_layer_window(ctypes.byref(c), layer)
+
+
+def layer_value_embed(c: NcConfig, layer: int) -> int:
+    return lib().nc_layer_value_embed(ctypes.byref(c), layer)
 
 
 def workspace_bytes(c: NcConfig, B: int, T: int) -> int:
@@ -182,23 +198,51 @@ class Model:
     @classmethod
     def from_tensors(cls, cfg: NcConfig, t: dict) -> "Model":
         """t: {"wte", "lm_head", "layers": [{c_q, c_k, c_v, attn_proj, c_fc, mlp_proj}]}
-        with contiguous float32 CUDA tensors in [out, in] layout."""
+        with contiguous float32 CUDA tensors in [out, in] layout, and optionally
+        t["extras"] = {"smear_gate", "resid_lambdas", "x0_lambdas",
+        "backout_lambda", "value_embeds": [L], "ve_gates": [L]} (list entries may
+        be None) for the terms enabled in cfg.extras."""
         L = cfg.n_layer
         arrs = {}
         for name in ("c_q", "c_k", "c_v", "attn_proj", "c_fc", "mlp_proj"):
             a = (ctypes.c_void_p * L)(*[t["layers"][l][name].data_ptr() for l in range(L)])
             arrs[name] = a
+        ex = t.get("extras") or {}
+        p = lambda x: None if x is None else x.data_ptr()
+        for name in ("value_embeds", "ve_gates"):
+            lst = ex.get(name)
+            arrs[name] = None if lst is None else (ctypes.c_void_p * L)(*[p(v) for v in lst])
+        fpp = lambda a: None if a is None else ctypes.cast(a, _FPP)
         w = NcWeights(t["wte"].data_ptr(), *[ctypes.cast(arrs[n], _FPP) for n in
                                              ("c_q", "c_k", "c_v", "attn_proj", "c_fc", "mlp_proj")],
-                      t["lm_head"].data_ptr())
-        return cls(cfg, t, w, list(arrs.values()))
+                      t["lm_head"].data_ptr(), p(ex.get("smear_gate")), fpp(arrs["value_embeds"]),
+                      fpp(arrs["ve_gates"]), p(ex.get("resid_lambdas")), p(ex.get("x0_lambdas")),
+                      p(ex.get("backout_lambda")))
+        return cls(cfg, t, w, [a for a in arrs.values() if a is not None])
 
     @classmethod
-    def from_numpy(cls, cfg: NcConfig, w: dict, device="cuda") -> "Model":
+    def from_numpy(cls, cfg: NcConfig, w: dict, device="cuda", extras: dict | None = None) -> "Model":
+        """As from_tensors, from float32 numpy arrays.  ``extras`` holds the further
+        weights (numpy, the layout of ``from_tensors``); only the tables of layers
+        that use a value embedding are copied to the device."""
         import torch
-        dev = lambda a: torch.from_numpy(a).to(device).contiguous()
+        dev = lambda a: torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(device).contiguous()
         t = {"wte": dev(w["wte"]), "lm_head": dev(w["lm_head"]),
              "layers": [{k: dev(v) for k, v in lw.items()} for lw in w["layers"]]}
+        if extras:
+            e = {}
+            for k in ("smear_gate", "resid_lambdas", "x0_lambdas"):
+                if extras.get(k) is not None:
+                    e[k] = dev(extras[k])
+            if extras.get("backout_lambda") is not None:
+                e["backout_lambda"] = dev(np.asarray(extras["backout_lambda"], dtype=np.float32).reshape(1))
+            if extras.get("value_embeds") is not None:
+                use = [layer_value_embed(cfg, l) == 1 for l in range(cfg.n_layer)]
+                e["value_embeds"] = [dev(v) if u and v is not None else None
+                                     for u, v in zip(use, extras["value_embeds"])]
+                e["ve_gates"] = [dev(g) if u and g is not None else None
+                                 for u, g in zip(use, extras["ve_gates"])]
+            t["extras"] = e
         return cls.from_tensors(cfg, t)
 
 

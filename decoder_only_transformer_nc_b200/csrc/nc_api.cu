@@ -81,6 +81,7 @@ bool config_ok(const nc_config* c) {
   if ((int64_t)c->n_head * c->head_dim % 64 != 0) return false;
   if (!(c->softcap > 0.0f) || !(c->norm_eps >= 0.0f) || !(c->rope_base > 1.0f)) return false;
   if (c->act_dtype != NC_F16 && c->act_dtype != NC_BF16) return false;
+  if ((c->extras & ~NC_EXTRA_ALL) != 0) return false;
   const size_t plen = strnlen(c->window_pattern, sizeof(c->window_pattern));
   if (plen == 0 || plen >= sizeof(c->window_pattern)) return false;
   for (size_t i = 0; i < plen; ++i)
@@ -90,7 +91,7 @@ bool config_ok(const nc_config* c) {
 
 // Workspace layout of nc_forward.  Offsets are 256-byte aligned.
 struct WsLayout {
-  size_t status, rope, wqkv, wo, wfc, wmp, wlm, x, a, qkv, o, h, part, tgt, tl, total;
+  size_t status, rope, wqkv, wo, wfc, wmp, wlm, x, a, qkv, o, h, part, tgt, tl, x0, xmid, total;
   size_t wqkv_elems, wo_elems, wfc_elems, wmp_elems;  // per layer
 };
 
@@ -124,6 +125,8 @@ WsLayout ws_layout(const nc_config* c, int B, int T) {
   L.part = take(M * (size_t)gemm_ce_partials_per_row((int)V) * 4);
   L.tgt = take(M * 4);
   L.tl = take(M * 4);
+  L.x0 = (c->extras & NC_EXTRA_RESID_LAMBDAS) ? take(M * C * 4) : 0;
+  L.xmid = (c->extras & NC_EXTRA_BACKOUT) ? take(M * C * 4) : 0;
   L.total = off;
   return L;
 }
@@ -170,7 +173,7 @@ nc_status device_ok() {
 
 extern "C" {
 
-int nc_version(void) { return 100; }
+int nc_version(void) { return 101; }
 
 const char* nc_status_string(nc_status s) {
   switch (s) {
@@ -223,6 +226,11 @@ int nc_layer_window(const nc_config* cfg, int layer) {
   char kind = cfg->window_pattern[layer % plen];
   if (layer == cfg->n_layer - 1) kind = 'L';
   return kind == 'L' ? cfg->seq_len : cfg->short_window;
+}
+
+int nc_layer_value_embed(const nc_config* cfg, int layer) {
+  if (!config_ok(cfg) || layer < 0 || layer >= cfg->n_layer) return -1;
+  return (cfg->n_layer - 1 - layer) % 2 == 0 ? 1 : 0;
 }
 
 size_t nc_workspace_bytes(const nc_config* cfg, int B, int T) {
@@ -411,6 +419,21 @@ nc_status nc_forward_traced(const nc_config* cfg, const nc_weights* w, const int
       if (!aligned16(p)) return NC_ERR_ALIGNMENT;
     }
   }
+  const uint32_t ex = cfg->extras;
+  if (ex & NC_EXTRA_SMEAR) {
+    if (!w->smear_gate) return NC_ERR_INVALID_ARG;
+    if (!aligned16(w->smear_gate)) return NC_ERR_ALIGNMENT;
+  }
+  if (ex & NC_EXTRA_VALUE_EMBED) {
+    if (!w->value_embeds || !w->ve_gates) return NC_ERR_INVALID_ARG;
+    for (int l = 0; l < cfg->n_layer; ++l) {
+      if (nc_layer_value_embed(cfg, l) != 1) continue;
+      if (!w->value_embeds[l] || !w->ve_gates[l]) return NC_ERR_INVALID_ARG;
+      if (!aligned16(w->value_embeds[l])) return NC_ERR_ALIGNMENT;
+    }
+  }
+  if ((ex & NC_EXTRA_RESID_LAMBDAS) && (!w->resid_lambdas || !w->x0_lambdas)) return NC_ERR_INVALID_ARG;
+  if ((ex & NC_EXTRA_BACKOUT) && !w->backout_lambda) return NC_ERR_INVALID_ARG;
   if (trace) {
     const int need = forward_launch_count(cfg, targets != nullptr, loss != nullptr, logits != nullptr);
     trace->count = need;
@@ -445,6 +468,9 @@ nc_status nc_forward_traced(const nc_config* cfg, const nc_weights* w, const int
   float* part = reinterpret_cast<float*>(ws + L.part);
   float* tgt = reinterpret_cast<float*>(ws + L.tgt);
   float* tl = token_loss ? token_loss : reinterpret_cast<float*>(ws + L.tl);
+  float* x0 = (ex & NC_EXTRA_RESID_LAMBDAS) ? reinterpret_cast<float*>(ws + L.x0) : nullptr;
+  float* xmid = (ex & NC_EXTRA_BACKOUT) ? reinterpret_cast<float*>(ws + L.xmid) : nullptr;
+  const int mid = cfg->n_layer / 2;  // backout: the stream after the first n_layer / 2 blocks
 
   const int M = B * T;
   const int C = cfg->d_model, D = cfg->head_dim, H = cfg->n_head, Hkv = cfg->n_kv_head,
@@ -473,11 +499,21 @@ nc_status nc_forward_traced(const nc_config* cfg, const nc_weights* w, const int
     NC_RUN(NC_K_CAST, cast_launch(segs.data(), (int)segs.size(), f16, st, C, D));
   }
 
-  NC_RUN(NC_K_EMBEDDING, embedding_launch(tokens, w->wte, x, M, C, V, status, st));
+  if (ex & (NC_EXTRA_SMEAR | NC_EXTRA_RESID_LAMBDAS))
+    NC_RUN(NC_K_EMBEDDING, embedding_extra_launch(tokens, w->wte, (ex & NC_EXTRA_SMEAR) ? w->smear_gate : nullptr,
+                                                  x, x0, M, C, V, T, status, st));
+  else
+    NC_RUN(NC_K_EMBEDDING, embedding_launch(tokens, w->wte, x, M, C, V, status, st));
 
   for (int l = 0; l < cfg->n_layer; ++l) {
     const int W = nc_layer_window(cfg, l);
-    NC_RUN(NC_K_RMSNORM, rmsnorm_launch(x, a, M, C, cfg->norm_eps, f16, st));
+    float* keep = (xmid && l == mid) ? xmid : nullptr;
+    if (x0 || keep)  // x_mid = the stream entering block `mid`; then x = a_l x + b_l x0
+      NC_RUN(NC_K_RMSNORM, rmsnorm_mix_launch(x, x0, x0 ? w->resid_lambdas + l : nullptr,
+                                              x0 ? w->x0_lambdas + l : nullptr, keep, nullptr, nullptr,
+                                              x0 != nullptr, a, M, C, cfg->norm_eps, f16, st));
+    else
+      NC_RUN(NC_K_RMSNORM, rmsnorm_launch(x, a, M, C, cfg->norm_eps, f16, st));
     EpiParams eq{};  // QKV projection with RoPE + QK-norm in the epilogue
     eq.out = qkv;
     eq.ldo = NQKV;
@@ -487,6 +523,12 @@ nc_status nc_forward_traced(const nc_config* cfg, const nc_weights* w, const int
     eq.Hkv = Hkv;
     eq.D = D;
     eq.eps = cfg->norm_eps;
+    if ((ex & NC_EXTRA_VALUE_EMBED) && nc_layer_value_embed(cfg, l) == 1) {
+      eq.tokens = tokens;
+      eq.ve = w->value_embeds[l];
+      eq.ve_gate = w->ve_gates[l];
+      eq.V = V;
+    }
     NC_RUN(NC_K_GEMM_QKV, gemm_launch(a, C, wqkv + l * L.wqkv_elems, C, M, NQKV, C, EPI_QKV_ROPE_IL, f16,
                                       eq, status, st));
     NC_RUN(NC_K_ATTENTION, attention_launch(qkv, qkv + H * D, qkv + (H + Hkv) * D, o, B, T, H, Hkv,
@@ -507,7 +549,11 @@ nc_status nc_forward_traced(const nc_config* cfg, const nc_weights* w, const int
                                            EPI_RESID_F32, f16, ep, status, st));
   }
 
-  NC_RUN(NC_K_RMSNORM, rmsnorm_launch(x, a, M, C, cfg->norm_eps, f16, st));
+  if (xmid)  // backout: x - lambda * x_mid, then the final norm
+    NC_RUN(NC_K_RMSNORM, rmsnorm_mix_launch(x, nullptr, nullptr, nullptr, nullptr, xmid, w->backout_lambda, false,
+                                            a, M, C, cfg->norm_eps, f16, st));
+  else
+    NC_RUN(NC_K_RMSNORM, rmsnorm_launch(x, a, M, C, cfg->norm_eps, f16, st));
   if (targets) {
     EpiParams ep{};
     ep.out = logits;

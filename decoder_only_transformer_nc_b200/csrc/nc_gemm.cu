@@ -325,13 +325,52 @@ __device__ __forceinline__ void epilogue_qkv_head(uint32_t taddr, const CUtensor
 // rotated, normalised and stored on its own (output in the same interleaved
 // order, for q and k alike -- attention scores are unchanged by a common
 // permutation of the head dimension).
+// v head of the QKV projection with a value embedding (full nanochat forward,
+// "Nanochat与nanoGPT对比" §1, value-residual note): v + gate[g] * table[token]
+// for kv head g, the table row read in fp32 and added to the fp32 accumulator.
+template <bool F16, int HD>
+__device__ __forceinline__ void epilogue_v_embed(uint32_t taddr, const CUtensorMap* tmC, uint8_t* stg,
+                                                 int row, int col0, int row0, int M, const EpiParams& ep,
+                                                 uint32_t lane) {
+  const int g = col0 / HD - ep.H - ep.Hkv;  // kv head
+  int tok = row < M ? ep.tokens[row] : 0;
+  if (tok < 0 || tok >= ep.V) tok = 0;  // flagged by the embedding kernel
+  const float4* ve = reinterpret_cast<const float4*>(ep.ve + (int64_t)tok * ep.Hkv * HD + (int64_t)g * HD);
+  const float gate = ep.ve_gate[g];
+#pragma unroll 1
+  for (int c = 0; c < HD / 64; ++c) {
+    uint32_t r0[32], r1[32];
+    tmem_ld_32x32b_x32(taddr + c * 64, r0);
+    tmem_ld_32x32b_x32(taddr + c * 64 + 32, r1);
+    tmem_wait_ld();
+    uint32_t w[32];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {  // columns 4j .. 4j+3 of this 64-column chunk
+      const float4 e = __ldg(ve + c * 16 + j);
+      const uint32_t* src = j < 8 ? r0 : r1;
+      const int k = (j & 7) * 4;
+      w[2 * j] = Half<F16>::pack2(fmaf(gate, e.x, __uint_as_float(src[k])),
+                                  fmaf(gate, e.y, __uint_as_float(src[k + 1])));
+      w[2 * j + 1] = Half<F16>::pack2(fmaf(gate, e.z, __uint_as_float(src[k + 2])),
+                                      fmaf(gate, e.w, __uint_as_float(src[k + 3])));
+    }
+    if (c > 0) flush_wait(lane);
+    stage_row(stg, (int)lane, w);
+    flush_issue<false>(tmC, stg, col0 + 64 * c, row0, lane);
+  }
+  flush_wait(lane);
+}
+
 template <bool F16, int HD>
 __device__ __forceinline__ void epilogue_qkv_head_il(uint32_t taddr, const CUtensorMap* tmC,
                                                      uint8_t* stg, int row, int col0, int row0, int M,
                                                      const EpiParams& ep, uint32_t lane) {
   const int head = col0 / HD;
-  if (head >= ep.H + ep.Hkv) {  // v head (warp-uniform): plain 16-bit store
-    epilogue_16_half<EPI_STORE_16, F16>(taddr, tmC, stg, col0, row0, col0 + HD, lane);
+  if (head >= ep.H + ep.Hkv) {  // v head (warp-uniform)
+    if (ep.ve)
+      epilogue_v_embed<F16, HD>(taddr, tmC, stg, row, col0, row0, M, ep, lane);
+    else  // plain 16-bit store
+      epilogue_16_half<EPI_STORE_16, F16>(taddr, tmC, stg, col0, row0, col0 + HD, lane);
     return;
   }
   float ss = 0.0f;

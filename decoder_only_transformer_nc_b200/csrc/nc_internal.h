@@ -37,6 +37,10 @@ struct EpiParams {
   int T;                    // EPI_QKV_ROPE: positions per sequence (row m is at m % T)
   int H, Hkv, D;            // EPI_QKV_ROPE: head counts and head size
   float eps;                // EPI_QKV_ROPE: RMSNorm epsilon
+  const int32_t* tokens;    // EPI_QKV_ROPE_IL with value embedding: [M] token ids
+  const float* ve;          //   [V, Hkv*D] table of this layer (NULL: none)
+  const float* ve_gate;     //   [Hkv] gates
+  int V;                    //   vocabulary size (ids outside [0, V) read row 0)
 };
 
 // ---- device / argument helpers (nc_api.cu)
@@ -84,6 +88,17 @@ nc_status cast_launch(const CastSeg* segs, int nseg, bool f16, cudaStream_t stre
                       int perm_d = 0);
 nc_status embedding_launch(const int32_t* tokens, const float* wte, float* x, int M, int C, int V,
                            uint32_t* dev_status, cudaStream_t stream);
+// Embedding with the smear term (gate may be NULL: plain lookup) and an optional
+// copy of the result into x0.  T: positions per row (row m is at m % T).
+nc_status embedding_extra_launch(const int32_t* tokens, const float* wte, const float* smear_gate,
+                                 float* x, float* x0, int M, int C, int V, int T, uint32_t* dev_status,
+                                 cudaStream_t stream);
+// RMSNorm of u, where per row u = x, then (x_keep: x_keep = u), then (x0: u =
+// lam_r[0] u + lam_0[0] x0), then (x_sub: u = u - lam_sub[0] x_sub); with
+// write_back the row of x becomes u.  Scalars are read from device memory.
+nc_status rmsnorm_mix_launch(float* x, const float* x0, const float* lam_r, const float* lam_0,
+                             float* x_keep, const float* x_sub, const float* lam_sub, bool write_back,
+                             uint16_t* out, int M, int C, float eps, bool f16, cudaStream_t stream);
 nc_status rmsnorm_launch(const float* x, uint16_t* out, int M, int C, float eps, bool f16,
                          cudaStream_t stream);
 nc_status rope_table_launch(float* table, int T, int D, float base, cudaStream_t stream);

@@ -97,6 +97,67 @@ __global__ void __launch_bounds__(256) embedding_kernel(const int32_t* __restric
   for (int i = lane; i < C / 4; i += 32) dst[i] = src[i];
 }
 
+// Embedding with the smear term of the full nanochat forward ("Nanochat与nanoGPT
+// 对比" §1, smear note): x_t = e_t + sigmoid(gate . e_t) e_{t-1} with e = wte[idx],
+// gate's fp32 weights taken at their bf16 values, position 0 of a row
+// unchanged.  One warp per token; the gate dot product is a warp reduction in
+// fp32.  x0 (optional) receives a copy of the result.
+template <bool SMEAR>
+__global__ void __launch_bounds__(256) embedding_extra_kernel(const int32_t* __restrict__ tokens,
+                                                              const float* __restrict__ wte,
+                                                              const float* __restrict__ gate,
+                                                              float* __restrict__ x, float* __restrict__ x0,
+                                                              int M, int C, int V, int T,
+                                                              uint32_t* dev_status) {
+  const int m = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (m >= M) return;
+  int tok = tokens[m];
+  if (tok < 0 || tok >= V) {
+    if (lane == 0 && dev_status) atomicOr(dev_status, NC_DEV_TOKEN_RANGE);
+    tok = 0;
+  }
+  const float4* e = reinterpret_cast<const float4*>(wte + (int64_t)tok * C);
+  float4* dst = reinterpret_cast<float4*>(x + (int64_t)m * C);
+  float4* dst0 = x0 ? reinterpret_cast<float4*>(x0 + (int64_t)m * C) : nullptr;
+  const int n4 = C / 4;
+  if constexpr (SMEAR) {
+    const bool has_prev = (m % T) != 0;
+    int ptok = has_prev ? tokens[m - 1] : 0;
+    if (ptok < 0 || ptok >= V) ptok = 0;  // flagged by that token's own warp
+    const float4* ep = reinterpret_cast<const float4*>(wte + (int64_t)ptok * C);
+    const float4* g4 = reinterpret_cast<const float4*>(gate);
+    float dot = 0.0f;
+    for (int i = lane; i < n4; i += 32) {
+      const float4 a = e[i], g = g4[i];
+      dot = fmaf(a.x, __bfloat162float(__float2bfloat16_rn(g.x)), dot);
+      dot = fmaf(a.y, __bfloat162float(__float2bfloat16_rn(g.y)), dot);
+      dot = fmaf(a.z, __bfloat162float(__float2bfloat16_rn(g.z)), dot);
+      dot = fmaf(a.w, __bfloat162float(__float2bfloat16_rn(g.w)), dot);
+    }
+    dot = warp_sum(dot);
+    const float sg = has_prev ? 1.0f / (1.0f + expf(-dot)) : 0.0f;
+    for (int i = lane; i < n4; i += 32) {
+      float4 a = e[i];
+      if (has_prev) {
+        const float4 b = ep[i];
+        a.x = fmaf(sg, b.x, a.x);
+        a.y = fmaf(sg, b.y, a.y);
+        a.z = fmaf(sg, b.z, a.z);
+        a.w = fmaf(sg, b.w, a.w);
+      }
+      dst[i] = a;
+      if (dst0) dst0[i] = a;
+    }
+  } else {
+    for (int i = lane; i < n4; i += 32) {
+      const float4 a = e[i];
+      dst[i] = a;
+      if (dst0) dst0[i] = a;
+    }
+  }
+}
+
 // ---------------------------------------------------------------- RMSNorm
 
 // One warp per row; the row is held in registers (C <= 32 * 4 * NV).
@@ -149,6 +210,93 @@ __global__ void __launch_bounds__(256) rmsnorm_wide_kernel(const float* __restri
   for (int i = lane; i < n4; i += 32) {
     const float4 a = xr[i];
     o[i] = make_uint2(Half<F16>::pack2(a.x * r, a.y * r), Half<F16>::pack2(a.z * r, a.w * r));
+  }
+}
+
+// RMSNorm fused with the residual-stream terms of the full nanochat forward
+// ("Nanochat与nanoGPT对比" §1: per-layer resid_lambdas + x0, backout).  Per row:
+// u = x; x_keep = u (optional); u = lam_r u + lam_0 x0 (optional); u = u -
+// lam_sub x_sub (optional); x = u (write_back); out = u / sqrt(mean(u^2) + eps).
+// One warp per row; the row is held in registers (C <= 32 * 4 * NV), or streamed
+// twice when NV == 0.
+template <int NV, bool F16>
+__global__ void __launch_bounds__(256) rmsnorm_mix_kernel(float* __restrict__ x,
+                                                          const float* __restrict__ x0,
+                                                          const float* __restrict__ lam_r,
+                                                          const float* __restrict__ lam_0,
+                                                          float* __restrict__ x_keep,
+                                                          const float* __restrict__ x_sub,
+                                                          const float* __restrict__ lam_sub, int write_back,
+                                                          uint16_t* __restrict__ out, int M, int C,
+                                                          float eps) {
+  const int row = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (row >= M) return;
+  const int64_t base = (int64_t)row * C;
+  const int n4 = C >> 2;
+  const float lr = x0 ? *lam_r : 1.0f, l0 = x0 ? *lam_0 : 0.0f;
+  const float ls = x_sub ? *lam_sub : 0.0f;
+  float4* xr = reinterpret_cast<float4*>(x + base);
+  auto mix = [&](int i) -> float4 {
+    float4 u = xr[i];
+    if (x_keep) reinterpret_cast<float4*>(x_keep + base)[i] = u;
+    if (x0) {
+      const float4 b = reinterpret_cast<const float4*>(x0 + base)[i];
+      u = make_float4(fmaf(lr, u.x, l0 * b.x), fmaf(lr, u.y, l0 * b.y), fmaf(lr, u.z, l0 * b.z),
+                      fmaf(lr, u.w, l0 * b.w));
+    }
+    if (x_sub) {
+      const float4 b = reinterpret_cast<const float4*>(x_sub + base)[i];
+      u = make_float4(fmaf(-ls, b.x, u.x), fmaf(-ls, b.y, u.y), fmaf(-ls, b.z, u.z), fmaf(-ls, b.w, u.w));
+    }
+    if (write_back) xr[i] = u;
+    return u;
+  };
+  uint2* o = reinterpret_cast<uint2*>(out + base);
+  if constexpr (NV > 0) {
+    float4 v[NV];
+    float ss = 0.0f;
+#pragma unroll
+    for (int j = 0; j < NV; ++j) {
+      const int i = j * 32 + lane;
+      v[j] = i < n4 ? mix(i) : make_float4(0.f, 0.f, 0.f, 0.f);
+      ss += v[j].x * v[j].x + v[j].y * v[j].y + v[j].z * v[j].z + v[j].w * v[j].w;
+    }
+    ss = warp_sum(ss);
+    const float r = rsqrtf(ss / (float)C + eps);
+#pragma unroll
+    for (int j = 0; j < NV; ++j) {
+      const int i = j * 32 + lane;
+      if (i < n4)
+        o[i] = make_uint2(Half<F16>::pack2(v[j].x * r, v[j].y * r), Half<F16>::pack2(v[j].z * r, v[j].w * r));
+    }
+  } else {
+    // Wide rows: pass 1 forms u (written back, or kept nowhere) and its sum of
+    // squares; pass 2 re-reads u from x when written back, else forms it again
+    // (x_keep only in pass 1).
+    float ss = 0.0f;
+    for (int i = lane; i < n4; i += 32) {
+      const float4 u = mix(i);
+      ss += u.x * u.x + u.y * u.y + u.z * u.z + u.w * u.w;
+    }
+    ss = warp_sum(ss);
+    const float r = rsqrtf(ss / (float)C + eps);
+    __syncwarp();
+    for (int i = lane; i < n4; i += 32) {
+      float4 u = xr[i];
+      if (!write_back) {
+        if (x0) {
+          const float4 b = reinterpret_cast<const float4*>(x0 + base)[i];
+          u = make_float4(fmaf(lr, u.x, l0 * b.x), fmaf(lr, u.y, l0 * b.y), fmaf(lr, u.z, l0 * b.z),
+                          fmaf(lr, u.w, l0 * b.w));
+        }
+        if (x_sub) {
+          const float4 b = reinterpret_cast<const float4*>(x_sub + base)[i];
+          u = make_float4(fmaf(-ls, b.x, u.x), fmaf(-ls, b.y, u.y), fmaf(-ls, b.z, u.z), fmaf(-ls, b.w, u.w));
+        }
+      }
+      o[i] = make_uint2(Half<F16>::pack2(u.x * r, u.y * r), Half<F16>::pack2(u.z * r, u.w * r));
+    }
   }
 }
 
@@ -388,6 +536,46 @@ nc_status embedding_launch(const int32_t* tokens, const float* wte, float* x, in
   if (M == 0) return NC_OK;
   const int grid = (M + 7) / 8;
   embedding_kernel<<<grid, 256, 0, stream>>>(tokens, wte, x, M, C, V, dev_status);
+  return last_error();
+}
+
+nc_status embedding_extra_launch(const int32_t* tokens, const float* wte, const float* smear_gate,
+                                 float* x, float* x0, int M, int C, int V, int T, uint32_t* dev_status,
+                                 cudaStream_t stream) {
+  if (M == 0) return NC_OK;
+  const int grid = (M + 7) / 8;
+  if (smear_gate)
+    embedding_extra_kernel<true><<<grid, 256, 0, stream>>>(tokens, wte, smear_gate, x, x0, M, C, V, T, dev_status);
+  else
+    embedding_extra_kernel<false><<<grid, 256, 0, stream>>>(tokens, wte, nullptr, x, x0, M, C, V, T, dev_status);
+  return last_error();
+}
+
+template <bool F16>
+static void rmsnorm_mix_dispatch(float* x, const float* x0, const float* lr, const float* l0, float* keep,
+                                 const float* sub, const float* ls, int wb, uint16_t* out, int M, int C,
+                                 float eps, cudaStream_t stream) {
+  const int grid = (M + 7) / 8;
+  if (C <= 32 * 4 * 4)
+    rmsnorm_mix_kernel<4, F16><<<grid, 256, 0, stream>>>(x, x0, lr, l0, keep, sub, ls, wb, out, M, C, eps);
+  else if (C <= 32 * 4 * 8)
+    rmsnorm_mix_kernel<8, F16><<<grid, 256, 0, stream>>>(x, x0, lr, l0, keep, sub, ls, wb, out, M, C, eps);
+  else if (C <= 32 * 4 * 16)
+    rmsnorm_mix_kernel<16, F16><<<grid, 256, 0, stream>>>(x, x0, lr, l0, keep, sub, ls, wb, out, M, C, eps);
+  else
+    rmsnorm_mix_kernel<0, F16><<<grid, 256, 0, stream>>>(x, x0, lr, l0, keep, sub, ls, wb, out, M, C, eps);
+}
+
+nc_status rmsnorm_mix_launch(float* x, const float* x0, const float* lam_r, const float* lam_0,
+                             float* x_keep, const float* x_sub, const float* lam_sub, bool write_back,
+                             uint16_t* out, int M, int C, float eps, bool f16, cudaStream_t stream) {
+  if (M == 0) return NC_OK;
+  if (f16)
+    rmsnorm_mix_dispatch<true>(x, x0, lam_r, lam_0, x_keep, x_sub, lam_sub, write_back ? 1 : 0, out, M, C, eps,
+                               stream);
+  else
+    rmsnorm_mix_dispatch<false>(x, x0, lam_r, lam_0, x_keep, x_sub, lam_sub, write_back ? 1 : 0, out, M, C,
+                                eps, stream);
   return last_error();
 }
 

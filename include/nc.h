@@ -72,6 +72,24 @@ typedef enum {
 #define NC_DEV_SMEM_ALIGN 0x8u   /* a kernel's shared-memory window was not 1024-byte
                                     aligned; it did nothing (reported as NC_ERR_CUDA) */
 
+/* Further terms of the full nanochat forward ("Nanochat与nanoGPT对比" §1,
+ * architecture table and notes); bits of nc_config.extras.  Each reads its
+ * weights from nc_weights.  The pages give one line per term; the readings
+ * taken are stated here. */
+#define NC_EXTRA_SMEAR 0x1u         /* after the embedding lookup:
+                                       x_t = e_t + sigmoid(gate . e_t) e_{t-1}, position 0 of each
+                                       row unchanged; gate is a bias-free linear map C -> 1 whose
+                                       fp32 weight enters as bf16 like every linear weight       */
+#define NC_EXTRA_VALUE_EMBED 0x2u   /* on every other layer counted back from the last (which
+                                       always has one): v += gate[g] * table[token][g*D .. g*D+D)
+                                       for kv head g, added to the v projection                   */
+#define NC_EXTRA_RESID_LAMBDAS 0x4u /* before block l: x = resid_lambdas[l] x + x0_lambdas[l] x0,
+                                       x0 the (smeared) embedding output                          */
+#define NC_EXTRA_BACKOUT 0x8u       /* before the final norm: x -= backout_lambda * x_mid, x_mid
+                                       the stream after the first n_layer / 2 blocks (before block
+                                       n_layer / 2 mixes in x0)                                   */
+#define NC_EXTRA_ALL 0xFu
+
 /* Model configuration.  "从文本到聊天模型" §5.1: d_model = depth * aspect_ratio,
  * n_head = d_model / head_dim.  window_pattern: one char per layer, cycled;
  * 'S' = short window (short_window keys), 'L' = full context; the last layer is
@@ -95,6 +113,7 @@ typedef struct {
                                 nearest even) values; with NC_F16 those values
                                 are held in fp16 (exact for |w| >= 2^-14) so
                                 both tensor-core operands share one format. */
+  uint32_t extras;           /* NC_EXTRA_* bits (0: the plain block stack)    */
 } nc_config;
 
 /* fp32 master weights (device pointers; the per-layer members are HOST arrays
@@ -108,6 +127,15 @@ typedef struct {
   const float* const* c_fc;          /* n_layer x [4C, C]                     */
   const float* const* mlp_proj;      /* n_layer x [C, 4C]                     */
   const float* lm_head;              /* [V, C]                                */
+  /* Read only for the terms enabled in nc_config.extras (may be NULL otherwise). */
+  const float* smear_gate;           /* [C]                NC_EXTRA_SMEAR      */
+  const float* const* value_embeds;  /* n_layer x [V, Hkv*D] fp32, and        */
+  const float* const* ve_gates;      /* n_layer x [Hkv]: NC_EXTRA_VALUE_EMBED;
+                                        entries of layers without a value
+                                        embedding are not read (may be NULL)   */
+  const float* resid_lambdas;        /* [n_layer]          NC_EXTRA_RESID_LAMBDAS */
+  const float* x0_lambdas;           /* [n_layer]          NC_EXTRA_RESID_LAMBDAS */
+  const float* backout_lambda;       /* [1]                NC_EXTRA_BACKOUT    */
 } nc_weights;
 
 /* ---------------------------------------------------------------- host-only */
@@ -115,7 +143,7 @@ typedef struct {
 /* Fills *out from the depth knob ("从文本到聊天模型" §5.1): d_model =
  * depth*aspect_ratio, n_head = d_model/head_dim, n_kv_head = n_kv_head or
  * n_head when 0, pattern "SSSL", short_window = seq_len/4, softcap 15,
- * norm_eps 1e-6, rope_base 10000, act_dtype NC_F16.  Host only; touches no
+ * norm_eps 1e-6, rope_base 10000, act_dtype NC_F16, extras 0.  Host only; touches no
  * device. */
 nc_status nc_init_config(nc_config* out, int depth, int aspect_ratio, int head_dim,
                          int n_kv_head, int seq_len, int vocab);
@@ -127,8 +155,14 @@ nc_status nc_check_config(const nc_config* cfg);
  * or -1 for a bad argument.  Host only. */
 int nc_layer_window(const nc_config* cfg, int layer);
 
-/* Bytes of workspace nc_forward needs for a [B, T] batch (0 on bad input).
- * Host only. */
+/* 1 if layer `layer` carries a value embedding under NC_EXTRA_VALUE_EMBED
+ * (every other layer counted back from the last), 0 if not, -1 for a bad
+ * argument.  Host only. */
+int nc_layer_value_embed(const nc_config* cfg, int layer);
+
+/* Bytes of workspace nc_forward needs for a [B, T] batch (0 on bad input); the
+ * extras NC_EXTRA_RESID_LAMBDAS and NC_EXTRA_BACKOUT each add one fp32 [B*T, C]
+ * stream.  Host only. */
 size_t nc_workspace_bytes(const nc_config* cfg, int B, int T);
 
 /* Algorithmic FLOPs of one forward over [B, T] tokens: 2 per multiply-add of

@@ -163,3 +163,45 @@ def test_single_step_argument_checks(nclib):
     assert c.act_dtype == nclib.F16
     c.act_dtype = 3
     assert nclib.check_config(c) == 2
+
+
+def test_extras_host_rules(nclib):
+    """Full-nanochat terms: layer rule, config bits, workspace growth and host checks."""
+    c4 = nclib.init_config(4, 64, 64, 0, 256, 512)
+    c5 = nclib.init_config(5, 64, 64, 0, 256, 512)
+    # every other layer counted back from the last (which always has one)
+    assert [nclib.layer_value_embed(c4, l) for l in range(4)] == [0, 1, 0, 1]
+    assert [nclib.layer_value_embed(c5, l) for l in range(5)] == [1, 0, 1, 0, 1]
+    assert [bool(nclib.layer_value_embed(c5, l)) for l in range(5)] == oracle.value_embed_layers(5)
+    assert nclib.layer_value_embed(c4, 4) == -1 and nclib.layer_value_embed(c4, -1) == -1
+    bad = nclib.NcConfig.from_buffer_copy(c4)
+    bad.extras = 16
+    assert nclib.check_config(bad) == 2
+    # x0 (resid lambdas) and x_mid (backout) streams are fp32 [B*T, C] each
+    base = nclib.workspace_bytes(c4, 2, 256)
+    stream = 2 * 256 * c4.d_model * 4
+    for bits, n in ((nclib.EXTRA_SMEAR, 0), (nclib.EXTRA_VALUE_EMBED, 0), (nclib.EXTRA_RESID_LAMBDAS, 1),
+                    (nclib.EXTRA_BACKOUT, 1), (nclib.EXTRA_ALL, 2)):
+        cx = nclib.NcConfig.from_buffer_copy(c4)
+        cx.extras = bits
+        assert nclib.workspace_bytes(cx, 2, 256) == base + n * stream
+    # enabled terms need their weights (checked before any device work)
+    cfg = nclib.init_config(2, 64, 64, 0, 256, 512)
+    fw = _FakeWeights(nclib, 2)
+    for bits in (nclib.EXTRA_SMEAR, nclib.EXTRA_VALUE_EMBED, nclib.EXTRA_RESID_LAMBDAS, nclib.EXTRA_BACKOUT):
+        cx = nclib.NcConfig.from_buffer_copy(cfg)
+        cx.extras = bits
+        assert _fwd(nclib, cx, fw, 2, 16) == 1
+    # a value-embedding table is required only on the layers that use one
+    cx = nclib.NcConfig.from_buffer_copy(cfg)
+    cx.extras = nclib.EXTRA_VALUE_EMBED
+    FPP = ctypes.POINTER(ctypes.c_void_p)
+    tabs = (ctypes.c_void_p * 2)(None, 1 << 44)
+    gates = (ctypes.c_void_p * 2)(None, (1 << 44) + 4096)
+    fw.w.value_embeds, fw.w.ve_gates = ctypes.cast(tabs, FPP), ctypes.cast(gates, FPP)
+    import torch
+    want = 0 if torch.cuda.is_available() else 8  # passes the host checks
+    if want == 8:
+        assert _fwd(nclib, cx, fw, 2, 16) == 8
+    tabs[1] = (1 << 44) + 8  # misaligned table
+    assert _fwd(nclib, cx, fw, 2, 16) == 4
