@@ -35,7 +35,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
-from workloads import SHAPES, TOKEN_SEED, make_tokens, make_weights  # noqa: E402
+from workloads import SHAPES, TOKEN_SEED, make_extras, make_tokens, make_weights  # noqa: E402
 
 METRIC = "forward+loss tokens/sec at d20 (1×B200); % of bf16 dense tensor peak"
 UNIT = "tokens/s"
@@ -155,17 +155,28 @@ def blas_threads():
     return len(os.sched_getaffinity(0))
 
 
-def oracle_sample(s, prefix, seed=TOKEN_SEED, weights=None):
-    """Runs the fp64 oracle on batch row 0, first `prefix` positions; returns
-    (tokens processed, seconds)."""
+def oracle_sample(s, prefix, seed=TOKEN_SEED, weights=None, extras=None):
+    """Runs the fp64 oracle on batch row 0, first `prefix` positions (with the
+    full-nanochat terms when `extras` is given); returns (tokens processed,
+    seconds)."""
     import oracle
     w = make_weights(s) if weights is None else weights
     x, y = make_tokens(s, seed=seed)
     cfg = oracle.OracleConfig(s.n_layer, s.d_model, s.n_head, s.n_kv_head, s.head_dim, s.seq_len,
                               s.vocab, short_window=s.short_window)
     t0 = time.perf_counter()
-    oracle.forward(cfg, w, x[:1, :prefix], y[:1, :prefix], want_logits=False)
+    oracle.forward(cfg, w, x[:1, :prefix], y[:1, :prefix], want_logits=False, extras=extras)
     return prefix, time.perf_counter() - t0
+
+
+def _extras_for(s, nc=None):
+    """Seeded weights of the full-nanochat terms, value-embedding tables only for
+    the layers the library uses them on (nc given) or for every layer."""
+    if nc is None:
+        return make_extras(s)
+    cfg = nc.make_config(s.n_layer, s.d_model, s.n_head, s.n_kv_head, s.head_dim, s.seq_len, s.vocab,
+                         s.short_window)
+    return make_extras(s, layers=[l for l in range(s.n_layer) if nc.layer_value_embed(cfg, l) == 1])
 
 
 def run_reference(args, s):
@@ -174,9 +185,10 @@ def run_reference(args, s):
         return
     prefix = args.ref_prefix
     w = make_weights(s)
+    ex = _extras_for(s) if args.extras == "all" else None
     for _ in range(args.warmup):
-        oracle_sample(s, prefix, weights=w)
-    times = [oracle_sample(s, prefix, weights=w)[1] for _ in range(args.steps)]
+        oracle_sample(s, prefix, weights=w, extras=ex)
+    times = [oracle_sample(s, prefix, weights=w, extras=ex)[1] for _ in range(args.steps)]
     sec = sum(times) / len(times)
     value = prefix / sec
     sample = f"{s.name} batch row 0, first {prefix} positions, forward+loss per step"
@@ -184,7 +196,8 @@ def run_reference(args, s):
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": s.name, "global_batch": 1, "seq_len": prefix, "parallelism": "none"},
+        "config": {"workload": s.name + ("+extras" if ex else ""), "global_batch": 1, "seq_len": prefix,
+                   "parallelism": "none"},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -210,10 +223,12 @@ def run_ours(args, s):
         from datetime import timedelta
         dist.init_process_group("nccl", device_id=dev, timeout=timedelta(seconds=120))
 
+    bits = nc.EXTRA_ALL if args.extras == "all" else 0
     cfg = nc.make_config(s.n_layer, s.d_model, s.n_head, s.n_kv_head, s.head_dim, s.seq_len, s.vocab,
-                         s.short_window)
+                         s.short_window, extras=bits)
     weights = make_weights(s)
-    model = nc.Model.from_numpy(cfg, weights, device=dev)
+    extras = _extras_for(s, nc) if bits else None
+    model = nc.Model.from_numpy(cfg, weights, device=dev, extras=extras)
     B, T = s.batch, s.seq_len
     x, y = make_tokens(s, seed=dp.shard_seed(TOKEN_SEED, rank))
     tx, ty = torch.from_numpy(x).to(dev), torch.from_numpy(y).to(dev)
@@ -339,7 +354,7 @@ def run_ours(args, s):
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": DTYPE_NOTE, "data": "synthetic",
-            "config": {"workload": s.name, "global_batch": world * B, "seq_len": T,
+            "config": {"workload": s.name + ("+extras" if bits else ""), "global_batch": world * B, "seq_len": T,
                        "parallelism": f"dp{world}" if world > 1 else "none",
                        "layers": s.n_layer, "d_model": s.d_model,
                        "l2": "inputs larger than L2 (fp32 weights %.2f GB, residual stream %.2f GB per step)"
@@ -375,7 +390,7 @@ def run_ours(args, s):
         if world == 1 and not args.no_cpu_baseline:
             del model, ws
             torch.cuda.empty_cache()
-            n_tok, sec = oracle_sample(s, args.cpu_prefix, weights=weights)
+            n_tok, sec = oracle_sample(s, args.cpu_prefix, weights=weights, extras=extras)
             result["cpu_baseline"] = {
                 "value": n_tok / sec, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
                 "sample": f"{s.name} batch row 0, first {args.cpu_prefix} positions, fp64 forward+loss "
@@ -402,6 +417,9 @@ def main():
     ap.add_argument("--ref-prefix", type=int, default=256,
                     help="positions of batch row 0 per step of the reference (oracle) arm")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--extras", default="none", choices=["none", "all"],
+                    help="all: also run the full nanochat terms (smear, value embeddings, "
+                         "residual lambdas + x0, backout)")
     ap.add_argument("--batch", type=int, default=None,
                     help="per-rank batch rows instead of the workload's (small profiler captures)")
     args = ap.parse_args()

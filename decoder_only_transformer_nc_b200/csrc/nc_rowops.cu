@@ -254,12 +254,53 @@ __global__ void __launch_bounds__(256) rmsnorm_mix_kernel(float* __restrict__ x,
   };
   uint2* o = reinterpret_cast<uint2*>(out + base);
   if constexpr (NV > 0) {
-    float4 v[NV];
+    // All loads of the row are issued before any arithmetic, so each lane keeps
+    // up to 2 NV 16-byte reads in flight.
+    float4 v[NV], b[NV];
+#pragma unroll
+    for (int j = 0; j < NV; ++j) {
+      const int i = j * 32 + lane;
+      v[j] = i < n4 ? xr[i] : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    const float* other = x0 ? x0 : x_sub;
+    if (other) {
+#pragma unroll
+      for (int j = 0; j < NV; ++j) {
+        const int i = j * 32 + lane;
+        b[j] = i < n4 ? reinterpret_cast<const float4*>(other + base)[i] : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+    }
+    if (x_keep) {
+#pragma unroll
+      for (int j = 0; j < NV; ++j) {
+        const int i = j * 32 + lane;
+        if (i < n4) reinterpret_cast<float4*>(x_keep + base)[i] = v[j];
+      }
+    }
+    if (x0) {
+#pragma unroll
+      for (int j = 0; j < NV; ++j)
+        v[j] = make_float4(fmaf(lr, v[j].x, l0 * b[j].x), fmaf(lr, v[j].y, l0 * b[j].y),
+                           fmaf(lr, v[j].z, l0 * b[j].z), fmaf(lr, v[j].w, l0 * b[j].w));
+    }
+    if (x_sub) {
+      if (x0) {  // both terms: x_sub is read now (not in the forward, which never combines them)
+#pragma unroll
+        for (int j = 0; j < NV; ++j) {
+          const int i = j * 32 + lane;
+          b[j] = i < n4 ? reinterpret_cast<const float4*>(x_sub + base)[i] : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < NV; ++j)
+        v[j] = make_float4(fmaf(-ls, b[j].x, v[j].x), fmaf(-ls, b[j].y, v[j].y), fmaf(-ls, b[j].z, v[j].z),
+                           fmaf(-ls, b[j].w, v[j].w));
+    }
     float ss = 0.0f;
 #pragma unroll
     for (int j = 0; j < NV; ++j) {
       const int i = j * 32 + lane;
-      v[j] = i < n4 ? mix(i) : make_float4(0.f, 0.f, 0.f, 0.f);
+      if (write_back && i < n4) xr[i] = v[j];
       ss += v[j].x * v[j].x + v[j].y * v[j].y + v[j].z * v[j].z + v[j].w * v[j].w;
     }
     ss = warp_sum(ss);

@@ -148,3 +148,21 @@ def test_forward_extras_full_size_sampled_rows(gpu, name):
     assert err <= 3e-2, f"{name}+all logits max-abs {err:.3e}"
     rel_rows = np.abs(got_tl - want["token_loss"]) / np.abs(want["token_loss"])
     assert rel_rows.max() <= 5e-3, f"{name}+all per-token loss rel {rel_rows.max():.3e}"
+
+
+def test_forward_extras_wide_rows(gpu):
+    """d_model 2560 > 2048: the two-pass path of the fused norm kernels."""
+    from workloads import ModelShape
+    s = ModelShape("wide", n_layer=2, d_model=2560, n_head=20, n_kv_head=4, head_dim=128, vocab=512,
+                   seq_len=64, batch=2, short_window=16)
+    w = make_weights(s)
+    ex = make_extras(s)
+    bits = gpu.EXTRA_ALL
+    cfg = gpu.make_config(s.n_layer, s.d_model, s.n_head, s.n_kv_head, s.head_dim, s.seq_len, s.vocab,
+                          s.short_window, extras=bits)
+    model = gpu.Model.from_numpy(cfg, w, extras=ex)
+    x, y = make_tokens(s)
+    r = gpu.forward(model, torch.from_numpy(x).to(DEV), torch.from_numpy(y).to(DEV), want_logits=True)
+    assert gpu.get_status(r["workspace"]) == 0
+    want = oracle.forward(_oracle_cfg(s), w, x, y, extras=_oracle_extras(ex, bits, gpu))
+    _check({"logits": r["logits"].cpu().numpy(), "loss": r["loss"].item()}, want, "wide+all")
