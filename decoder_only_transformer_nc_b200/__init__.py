@@ -120,6 +120,10 @@ def lib():
             "nc_softcap_ce": (i32, [vp, vp, vp, vp, i32, i32, f32, vp, vp]),
             "nc_loss_mean": (i32, [vp, vp, i32, i32, vp, vp]),
             "nc_selftest_bounded_wait": (i32, [vp, ctypes.c_uint32, vp]),
+            "nc_session_bytes": (sz, [cfgp, i32, i32]),
+            "nc_prefill_workspace_bytes": (sz, [cfgp, i32, i32]),
+            "nc_prefill": (i32, [cfgp, ctypes.POINTER(NcWeights), vp, i32, i32, vp, vp, sz, i32, vp, sz, vp]),
+            "nc_decode_step": (i32, [cfgp, ctypes.POINTER(NcWeights), vp, i32, i32, vp, vp, sz, i32, vp]),
         }
         for name, (res, args) in sigs.items():
             fn = getattr(L, name)
@@ -288,6 +292,50 @@ def forward(model: Model, tokens, targets=None, want_logits=False, want_token_lo
                                    None if trace is None else ctypes.byref(trace.struct)),
            "nc_forward")
     return res
+
+
+class Session:
+    """KV-cache inference state on the device (see nc_prefill / nc_decode_step):
+    the weights cast once, the RoPE table and every layer's cache for B rows of
+    up to T_max positions."""
+
+    def __init__(self, model: Model, B: int, T_max: int, device="cuda"):
+        import torch
+        n = lib().nc_session_bytes(ctypes.byref(model.cfg), B, T_max)
+        if n == 0:
+            raise NcError(3, "nc_session_bytes")
+        self.model, self.B, self.T_max = model, B, T_max
+        self.buffer = torch.empty(n, dtype=torch.uint8, device=device)
+        self.pos = 0
+
+    def prefill(self, tokens, want_logits=False, stream=None):
+        """Runs the prompt tokens [B, T]; returns the logits [B, T, V] if asked."""
+        import torch
+        cfg = self.model.cfg
+        B, T = tokens.shape
+        ws = torch.empty(max(1, lib().nc_prefill_workspace_bytes(ctypes.byref(cfg), B, T)), dtype=torch.uint8,
+                         device=tokens.device)
+        logits = torch.empty((B, T, cfg.vocab), dtype=torch.float32, device=tokens.device) if want_logits else None
+        _check(lib().nc_prefill(ctypes.byref(cfg), ctypes.byref(self.model.weights), _ptr(tokens), B, T,
+                                _ptr(logits), _ptr(self.buffer), self.buffer.numel(), self.T_max, _ptr(ws),
+                                ws.numel(), _stream(stream)), "nc_prefill")
+        self.pos = T
+        return logits
+
+    def decode(self, tokens, logits=None, stream=None):
+        """One position for every row: tokens [B] int32; returns logits [B, V]."""
+        import torch
+        cfg = self.model.cfg
+        if logits is None:
+            logits = torch.empty((self.B, cfg.vocab), dtype=torch.float32, device=tokens.device)
+        _check(lib().nc_decode_step(ctypes.byref(cfg), ctypes.byref(self.model.weights), _ptr(tokens), self.B,
+                                    self.pos, _ptr(logits), _ptr(self.buffer), self.buffer.numel(), self.T_max,
+                                    _stream(stream)), "nc_decode_step")
+        self.pos += 1
+        return logits
+
+    def status(self):
+        return get_status(self.buffer)
 
 
 class LaunchTrace:

@@ -95,7 +95,7 @@ struct WsLayout {
   size_t wqkv_elems, wo_elems, wfc_elems, wmp_elems;  // per layer
 };
 
-WsLayout ws_layout(const nc_config* c, int B, int T) {
+WsLayout ws_layout(const nc_config* c, int B, int T, bool own_weights = true) {
   WsLayout L;
   const size_t M = (size_t)B * T;
   const size_t C = c->d_model, D = c->head_dim, H = c->n_head, Hkv = c->n_kv_head, V = c->vocab;
@@ -111,12 +111,16 @@ WsLayout ws_layout(const nc_config* c, int B, int T) {
     return o;
   };
   L.status = take(256);
-  L.rope = take((size_t)T * D * sizeof(float));
-  L.wqkv = take(c->n_layer * L.wqkv_elems * 2);
-  L.wo = take(c->n_layer * L.wo_elems * 2);
-  L.wfc = take(c->n_layer * L.wfc_elems * 2);
-  L.wmp = take(c->n_layer * L.wmp_elems * 2);
-  L.wlm = take(V * C * 2);
+  if (own_weights) {  // else the 16-bit weights and the RoPE table live in a session
+    L.rope = take((size_t)T * D * sizeof(float));
+    L.wqkv = take(c->n_layer * L.wqkv_elems * 2);
+    L.wo = take(c->n_layer * L.wo_elems * 2);
+    L.wfc = take(c->n_layer * L.wfc_elems * 2);
+    L.wmp = take(c->n_layer * L.wmp_elems * 2);
+    L.wlm = take(V * C * 2);
+  } else {
+    L.rope = L.wqkv = L.wo = L.wfc = L.wmp = L.wlm = 0;
+  }
   L.x = take(M * C * 4);
   L.a = take(M * C * 2);
   L.qkv = take(M * nqkv * 2);
@@ -130,6 +134,53 @@ WsLayout ws_layout(const nc_config* c, int B, int T) {
   L.total = off;
   return L;
 }
+
+// KV-cache session: the 16-bit weights and the RoPE table (cast and built once
+// by nc_prefill), the cache of every layer, and the scratch of one decode step
+// (B rows).  Offsets are 256-byte aligned.
+struct SessionLayout {
+  size_t status, rope, wqkv, wo, wfc, wmp, wlm, cache, x, a, qkv, o, h, part, total;
+  size_t wqkv_elems, wo_elems, wfc_elems, wmp_elems, cache_layer_elems;
+};
+
+SessionLayout session_layout(const nc_config* c, int B, int T_max) {
+  SessionLayout L;
+  const size_t C = c->d_model, D = c->head_dim, H = c->n_head, Hkv = c->n_kv_head, V = c->vocab;
+  const size_t nqkv = (H + 2 * Hkv) * D, Bs = (size_t)B;
+  L.wqkv_elems = nqkv * C;
+  L.wo_elems = C * H * D;
+  L.wfc_elems = 4 * C * C;
+  L.wmp_elems = C * 4 * C;
+  L.cache_layer_elems = Bs * T_max * 2 * Hkv * D;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    size_t o = off;
+    off = align_up(off + bytes, 256);
+    return o;
+  };
+  L.status = take(256);
+  L.rope = take((size_t)T_max * D * sizeof(float));
+  L.wqkv = take(c->n_layer * L.wqkv_elems * 2);
+  L.wo = take(c->n_layer * L.wo_elems * 2);
+  L.wfc = take(c->n_layer * L.wfc_elems * 2);
+  L.wmp = take(c->n_layer * L.wmp_elems * 2);
+  L.wlm = take(V * C * 2);
+  L.cache = take(c->n_layer * L.cache_layer_elems * 2);
+  L.x = take(Bs * C * 4);
+  L.a = take(Bs * C * 2);
+  L.qkv = take(Bs * nqkv * 2);
+  L.o = take(Bs * H * D * 2);
+  L.h = take(Bs * 4 * C * 2);
+  L.part = take(Bs * H * (size_t)decode_attention_max_splits() * (2 + D) * 4);
+  L.total = off;
+  return L;
+}
+
+// Where nc_prefill puts what a later decode step reads.
+struct SessionRef {
+  uint8_t* base;
+  int T_max;
+};
 
 inline cudaStream_t S(void* s) { return reinterpret_cast<cudaStream_t>(s); }
 
@@ -395,10 +446,48 @@ nc_status nc_loss_mean(const float* token_loss, const int32_t* targets, int M, i
   return loss_mean_launch(token_loss, targets, M, V, loss, S(stream));
 }
 
-nc_status nc_forward_traced(const nc_config* cfg, const nc_weights* w, const int32_t* tokens,
-                            const int32_t* targets, int B, int T, float* logits,
-                            float* token_loss, float* loss, void* workspace, size_t ws_bytes,
-                            void* stream, nc_trace* trace) {
+// The one weight-cast launch: every fp32 matmul weight -> its bf16 value (held
+// in fp16 when f16); c_q, c_k, c_v of a layer packed into one matrix, with the
+// rows of c_q and c_k reordered so each RoPE pair is adjacent.
+static nc_status launch_weight_cast(const nc_config* cfg, const nc_weights* w, uint16_t* wqkv, uint16_t* wo,
+                                    uint16_t* wfc, uint16_t* wmp, uint16_t* wlm, size_t e_qkv, size_t e_wo,
+                                    size_t e_fc, size_t e_mp, bool f16, cudaStream_t st) {
+  const int C = cfg->d_model, D = cfg->head_dim, H = cfg->n_head, Hkv = cfg->n_kv_head, V = cfg->vocab;
+  std::vector<CastSeg> segs;
+  segs.reserve(cfg->n_layer * 6 + 1);
+  const size_t nq = (size_t)H * D * C, nk = (size_t)Hkv * D * C;
+  for (int l = 0; l < cfg->n_layer; ++l) {
+    uint16_t* dq = wqkv + l * e_qkv;
+    segs.push_back({w->c_q[l], dq, (int64_t)nq, true});  // RoPE pairs made adjacent
+    segs.push_back({w->c_k[l], dq + nq, (int64_t)nk, true});
+    segs.push_back({w->c_v[l], dq + nq + nk, (int64_t)nk});
+    segs.push_back({w->attn_proj[l], wo + l * e_wo, (int64_t)e_wo});
+    segs.push_back({w->c_fc[l], wfc + l * e_fc, (int64_t)e_fc});
+    segs.push_back({w->mlp_proj[l], wmp + l * e_mp, (int64_t)e_mp});
+  }
+  segs.push_back({w->lm_head, wlm, (int64_t)V * C});
+  return cast_launch(segs.data(), (int)segs.size(), f16, st, C, D);
+}
+
+// Checks the fp32 weight pointers of the plain block stack.
+static nc_status check_weights(const nc_config* cfg, const nc_weights* w) {
+  if (!w->wte || !w->lm_head || !w->c_q || !w->c_k || !w->c_v || !w->attn_proj || !w->c_fc || !w->mlp_proj)
+    return NC_ERR_INVALID_ARG;
+  if (!aligned16(w->wte) || !aligned16(w->lm_head)) return NC_ERR_ALIGNMENT;
+  for (int l = 0; l < cfg->n_layer; ++l) {
+    const float* ps[6] = {w->c_q[l], w->c_k[l], w->c_v[l], w->attn_proj[l], w->c_fc[l], w->mlp_proj[l]};
+    for (const float* p : ps) {
+      if (!p) return NC_ERR_INVALID_ARG;
+      if (!aligned16(p)) return NC_ERR_ALIGNMENT;
+    }
+  }
+  return NC_OK;
+}
+
+static nc_status forward_impl(const nc_config* cfg, const nc_weights* w, const int32_t* tokens,
+                              const int32_t* targets, int B, int T, float* logits, float* token_loss,
+                              float* loss, void* workspace, size_t ws_bytes, void* stream, nc_trace* trace,
+                              const SessionRef* sess) {
   if (!cfg || !w || !tokens || !workspace) return NC_ERR_INVALID_ARG;
   if (!config_ok(cfg)) return NC_ERR_CONFIG;
   if (B < 1 || T < 1 || T > cfg->seq_len) return NC_ERR_SHAPE;
@@ -407,7 +496,7 @@ nc_status nc_forward_traced(const nc_config* cfg, const nc_weights* w, const int
       !w->mlp_proj)
     return NC_ERR_INVALID_ARG;
   if ((int64_t)B * T > (int64_t)1 << 30) return NC_ERR_SHAPE;
-  const WsLayout L = ws_layout(cfg, B, T);
+  const WsLayout L = ws_layout(cfg, B, T, sess == nullptr);
   if (ws_bytes < L.total) return NC_ERR_WORKSPACE;
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return NC_ERR_ALIGNMENT;
   if (!aligned16(w->wte) || !aligned16(w->lm_head) || (logits && !aligned16(logits)))
@@ -453,13 +542,31 @@ nc_status nc_forward_traced(const nc_config* cfg, const nc_weights* w, const int
     if (!tr.end()) return NC_ERR_CUDA;              \
   } while (0)
   uint8_t* ws = static_cast<uint8_t*>(workspace);
-  uint32_t* status = reinterpret_cast<uint32_t*>(ws + L.status);
-  float* rope = reinterpret_cast<float*>(ws + L.rope);
-  uint16_t* wqkv = reinterpret_cast<uint16_t*>(ws + L.wqkv);
-  uint16_t* wo = reinterpret_cast<uint16_t*>(ws + L.wo);
-  uint16_t* wfc = reinterpret_cast<uint16_t*>(ws + L.wfc);
-  uint16_t* wmp = reinterpret_cast<uint16_t*>(ws + L.wmp);
-  uint16_t* wlm = reinterpret_cast<uint16_t*>(ws + L.wlm);
+  // 16-bit weights and RoPE table: in the workspace, or in the session (prefill)
+  SessionLayout SL{};
+  uint8_t* wbase = ws;
+  size_t o_st = L.status, o_rope = L.rope, o_wqkv = L.wqkv, o_wo = L.wo, o_wfc = L.wfc, o_wmp = L.wmp,
+         o_wlm = L.wlm;
+  int T_rope = T;
+  if (sess) {
+    SL = session_layout(cfg, B, sess->T_max);
+    wbase = sess->base;
+    o_st = SL.status;
+    o_rope = SL.rope;
+    o_wqkv = SL.wqkv;
+    o_wo = SL.wo;
+    o_wfc = SL.wfc;
+    o_wmp = SL.wmp;
+    o_wlm = SL.wlm;
+    T_rope = sess->T_max;
+  }
+  uint32_t* status = reinterpret_cast<uint32_t*>(wbase + o_st);
+  float* rope = reinterpret_cast<float*>(wbase + o_rope);
+  uint16_t* wqkv = reinterpret_cast<uint16_t*>(wbase + o_wqkv);
+  uint16_t* wo = reinterpret_cast<uint16_t*>(wbase + o_wo);
+  uint16_t* wfc = reinterpret_cast<uint16_t*>(wbase + o_wfc);
+  uint16_t* wmp = reinterpret_cast<uint16_t*>(wbase + o_wmp);
+  uint16_t* wlm = reinterpret_cast<uint16_t*>(wbase + o_wlm);
   float* x = reinterpret_cast<float*>(ws + L.x);
   uint16_t* a = reinterpret_cast<uint16_t*>(ws + L.a);
   uint16_t* qkv = reinterpret_cast<uint16_t*>(ws + L.qkv);
@@ -479,25 +586,11 @@ nc_status nc_forward_traced(const nc_config* cfg, const nc_weights* w, const int
   const bool f16 = cfg->act_dtype == NC_F16;
 
   if (cudaMemsetAsync(status, 0, 256, st) != cudaSuccess) return NC_ERR_CUDA;
-  NC_RUN(NC_K_ROPE_TABLE, rope_table_launch(rope, T, D, cfg->rope_base, st));
+  NC_RUN(NC_K_ROPE_TABLE, rope_table_launch(rope, T_rope, D, cfg->rope_base, st));
 
   // fp32 -> bf16 weight cast; c_q|c_k|c_v rows packed into one matrix per layer.
-  {
-    std::vector<CastSeg> segs;
-    segs.reserve(cfg->n_layer * 6 + 1);
-    const size_t nq = (size_t)H * D * C, nk = (size_t)Hkv * D * C;
-    for (int l = 0; l < cfg->n_layer; ++l) {
-      uint16_t* dq = wqkv + l * L.wqkv_elems;
-      segs.push_back({w->c_q[l], dq, (int64_t)nq, true});  // RoPE pairs made adjacent
-      segs.push_back({w->c_k[l], dq + nq, (int64_t)nk, true});
-      segs.push_back({w->c_v[l], dq + nq + nk, (int64_t)nk});
-      segs.push_back({w->attn_proj[l], wo + l * L.wo_elems, (int64_t)L.wo_elems});
-      segs.push_back({w->c_fc[l], wfc + l * L.wfc_elems, (int64_t)L.wfc_elems});
-      segs.push_back({w->mlp_proj[l], wmp + l * L.wmp_elems, (int64_t)L.wmp_elems});
-    }
-    segs.push_back({w->lm_head, wlm, (int64_t)V * C});
-    NC_RUN(NC_K_CAST, cast_launch(segs.data(), (int)segs.size(), f16, st, C, D));
-  }
+  NC_RUN(NC_K_CAST, launch_weight_cast(cfg, w, wqkv, wo, wfc, wmp, wlm, L.wqkv_elems, L.wo_elems, L.wfc_elems,
+                                       L.wmp_elems, f16, st));
 
   if (ex & (NC_EXTRA_SMEAR | NC_EXTRA_RESID_LAMBDAS))
     NC_RUN(NC_K_EMBEDDING, embedding_extra_launch(tokens, w->wte, (ex & NC_EXTRA_SMEAR) ? w->smear_gate : nullptr,
@@ -523,6 +616,7 @@ nc_status nc_forward_traced(const nc_config* cfg, const nc_weights* w, const int
     eq.Hkv = Hkv;
     eq.D = D;
     eq.eps = cfg->norm_eps;
+    eq.rope_T = T_rope;
     if ((ex & NC_EXTRA_VALUE_EMBED) && nc_layer_value_embed(cfg, l) == 1) {
       eq.tokens = tokens;
       eq.ve = w->value_embeds[l];
@@ -531,6 +625,11 @@ nc_status nc_forward_traced(const nc_config* cfg, const nc_weights* w, const int
     }
     NC_RUN(NC_K_GEMM_QKV, gemm_launch(a, C, wqkv + l * L.wqkv_elems, C, M, NQKV, C, EPI_QKV_ROPE_IL, f16,
                                       eq, status, st));
+    if (sess) {  // keep this layer's k and v for decoding
+      uint16_t* cache = reinterpret_cast<uint16_t*>(sess->base + SL.cache) + l * SL.cache_layer_elems;
+      nc_status s_ = kv_append_launch(qkv, NQKV, H * D, 2 * Hkv * D, cache, M, T, sess->T_max, 0, st);
+      if (s_ != NC_OK) return s_;
+    }
     NC_RUN(NC_K_ATTENTION, attention_launch(qkv, qkv + H * D, qkv + (H + Hkv) * D, o, B, T, H, Hkv,
                                             D, W, NQKV, NQKV, f16, status, st));
     EpiParams ep{};
@@ -578,11 +677,138 @@ nc_status nc_forward_traced(const nc_config* cfg, const nc_weights* w, const int
   return NC_OK;
 }
 
+nc_status nc_forward_traced(const nc_config* cfg, const nc_weights* w, const int32_t* tokens,
+                            const int32_t* targets, int B, int T, float* logits,
+                            float* token_loss, float* loss, void* workspace, size_t ws_bytes,
+                            void* stream, nc_trace* trace) {
+  return forward_impl(cfg, w, tokens, targets, B, T, logits, token_loss, loss, workspace, ws_bytes, stream,
+                      trace, nullptr);
+}
+
 nc_status nc_forward(const nc_config* cfg, const nc_weights* w, const int32_t* tokens,
                      const int32_t* targets, int B, int T, float* logits, float* token_loss,
                      float* loss, void* workspace, size_t ws_bytes, void* stream) {
   return nc_forward_traced(cfg, w, tokens, targets, B, T, logits, token_loss, loss, workspace,
                            ws_bytes, stream, nullptr);
+}
+
+size_t nc_session_bytes(const nc_config* cfg, int B, int T_max) {
+  if (!config_ok(cfg) || B < 1 || T_max < 1 || T_max > cfg->seq_len) return 0;
+  return session_layout(cfg, B, T_max).total;
+}
+
+size_t nc_prefill_workspace_bytes(const nc_config* cfg, int B, int T) {
+  if (!config_ok(cfg) || B < 1 || T < 1 || T > cfg->seq_len) return 0;
+  return ws_layout(cfg, B, T, false).total;
+}
+
+nc_status nc_prefill(const nc_config* cfg, const nc_weights* w, const int32_t* tokens, int B, int T,
+                     float* logits, void* session, size_t session_bytes, int T_max, void* workspace,
+                     size_t ws_bytes, void* stream) {
+  if (!cfg || !w || !session) return NC_ERR_INVALID_ARG;
+  if (!config_ok(cfg) || cfg->extras != 0) return NC_ERR_CONFIG;
+  if (T_max < 1 || T_max > cfg->seq_len || T < 0 || T > T_max || B < 1) return NC_ERR_SHAPE;
+  const SessionLayout SL = session_layout(cfg, B, T_max);
+  if (session_bytes < SL.total) return NC_ERR_WORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(session) & 255u) != 0) return NC_ERR_ALIGNMENT;
+  if (T == 0) {  // no prompt: only the weight cast and the RoPE table
+    if (nc_status s = check_weights(cfg, w)) return s;
+    if (nc_status s = device_ok()) return s;
+    uint8_t* base = static_cast<uint8_t*>(session);
+    cudaStream_t st = S(stream);
+    if (cudaMemsetAsync(base + SL.status, 0, 256, st) != cudaSuccess) return NC_ERR_CUDA;
+    if (nc_status s = rope_table_launch(reinterpret_cast<float*>(base + SL.rope), T_max, cfg->head_dim,
+                                        cfg->rope_base, st))
+      return s;
+    return launch_weight_cast(cfg, w, reinterpret_cast<uint16_t*>(base + SL.wqkv),
+                              reinterpret_cast<uint16_t*>(base + SL.wo), reinterpret_cast<uint16_t*>(base + SL.wfc),
+                              reinterpret_cast<uint16_t*>(base + SL.wmp), reinterpret_cast<uint16_t*>(base + SL.wlm),
+                              SL.wqkv_elems, SL.wo_elems, SL.wfc_elems, SL.wmp_elems, cfg->act_dtype == NC_F16, st);
+  }
+  const SessionRef sess{static_cast<uint8_t*>(session), T_max};
+  return forward_impl(cfg, w, tokens, nullptr, B, T, logits, nullptr, nullptr, workspace, ws_bytes, stream,
+                      nullptr, &sess);
+}
+
+nc_status nc_decode_step(const nc_config* cfg, const nc_weights* w, const int32_t* tokens, int B, int pos,
+                         float* logits, void* session, size_t session_bytes, int T_max, void* stream) {
+  if (!cfg || !w || !w->wte || !tokens || !logits || !session) return NC_ERR_INVALID_ARG;
+  if (!config_ok(cfg) || cfg->extras != 0) return NC_ERR_CONFIG;
+  if (T_max < 1 || T_max > cfg->seq_len || B < 1 || pos < 0 || pos >= T_max) return NC_ERR_SHAPE;
+  const SessionLayout SL = session_layout(cfg, B, T_max);
+  if (session_bytes < SL.total) return NC_ERR_WORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(session) & 255u) != 0) return NC_ERR_ALIGNMENT;
+  if (!aligned16(w->wte) || !aligned16(logits)) return NC_ERR_ALIGNMENT;
+  if (cfg->n_head / cfg->n_kv_head > 8 || (cfg->n_head / cfg->n_kv_head) & (cfg->n_head / cfg->n_kv_head - 1))
+    return NC_ERR_SHAPE;  // decode attention groups of 1, 2, 4 or 8 query heads
+  if (nc_status s = device_ok()) return s;
+
+  cudaStream_t st = S(stream);
+  uint8_t* base = static_cast<uint8_t*>(session);
+  uint32_t* status = reinterpret_cast<uint32_t*>(base + SL.status);
+  const float* rope = reinterpret_cast<const float*>(base + SL.rope);
+  const uint16_t* wqkv = reinterpret_cast<const uint16_t*>(base + SL.wqkv);
+  const uint16_t* wo = reinterpret_cast<const uint16_t*>(base + SL.wo);
+  const uint16_t* wfc = reinterpret_cast<const uint16_t*>(base + SL.wfc);
+  const uint16_t* wmp = reinterpret_cast<const uint16_t*>(base + SL.wmp);
+  const uint16_t* wlm = reinterpret_cast<const uint16_t*>(base + SL.wlm);
+  uint16_t* cache = reinterpret_cast<uint16_t*>(base + SL.cache);
+  float* x = reinterpret_cast<float*>(base + SL.x);
+  uint16_t* a = reinterpret_cast<uint16_t*>(base + SL.a);
+  uint16_t* qkv = reinterpret_cast<uint16_t*>(base + SL.qkv);
+  uint16_t* o = reinterpret_cast<uint16_t*>(base + SL.o);
+  uint16_t* h = reinterpret_cast<uint16_t*>(base + SL.h);
+  float* part = reinterpret_cast<float*>(base + SL.part);
+  const int C = cfg->d_model, D = cfg->head_dim, H = cfg->n_head, Hkv = cfg->n_kv_head, V = cfg->vocab;
+  const int NQKV = (H + 2 * Hkv) * D;
+  const bool f16 = cfg->act_dtype == NC_F16;
+  const float eps = cfg->norm_eps;
+  nc_status s;
+#define NC_TRY(call)    \
+  do {                  \
+    s = (call);         \
+    if (s != NC_OK) return s; \
+  } while (0)
+  if (cudaMemsetAsync(status, 0, 256, st) != cudaSuccess) return NC_ERR_CUDA;
+  NC_TRY(embedding_launch(tokens, w->wte, x, B, C, V, status, st));
+  for (int l = 0; l < cfg->n_layer; ++l) {
+    NC_TRY(rmsnorm_launch(x, a, B, C, eps, f16, st));
+    EpiParams eq{};  // one row per sequence, at position pos
+    eq.out = qkv;
+    eq.ldo = NQKV;
+    eq.rope = rope;
+    eq.T = 1;
+    eq.pos0 = pos;
+    eq.rope_T = T_max;
+    eq.H = H;
+    eq.Hkv = Hkv;
+    eq.D = D;
+    eq.eps = eps;
+    NC_TRY(gemm_launch(a, C, wqkv + l * SL.wqkv_elems, C, B, NQKV, C, EPI_QKV_ROPE_IL, f16, eq, status, st));
+    uint16_t* cl = cache + l * SL.cache_layer_elems;
+    NC_TRY(kv_append_launch(qkv, NQKV, H * D, 2 * Hkv * D, cl, B, 1, T_max, pos, st));
+    NC_TRY(decode_attention_launch(qkv, NQKV, cl, part, o, B, H, Hkv, D, T_max, pos, nc_layer_window(cfg, l),
+                                   f16, st));
+    EpiParams ep{};
+    ep.out = x;
+    ep.ldo = C;
+    NC_TRY(gemm_launch(o, H * D, wo + l * SL.wo_elems, H * D, B, C, H * D, EPI_RESID_F32, f16, ep, status, st));
+    NC_TRY(rmsnorm_launch(x, a, B, C, eps, f16, st));
+    ep.out = h;
+    ep.ldo = 4 * C;
+    NC_TRY(gemm_launch(a, C, wfc + l * SL.wfc_elems, C, B, 4 * C, C, EPI_RELU2_16, f16, ep, status, st));
+    ep.out = x;
+    ep.ldo = C;
+    NC_TRY(gemm_launch(h, 4 * C, wmp + l * SL.wmp_elems, 4 * C, B, C, 4 * C, EPI_RESID_F32, f16, ep, status, st));
+  }
+  NC_TRY(rmsnorm_launch(x, a, B, C, eps, f16, st));
+  EpiParams ep{};
+  ep.out = logits;
+  ep.ldo = V;
+  ep.cap = cfg->softcap;
+  NC_TRY(gemm_launch(a, C, wlm, C, B, V, C, EPI_SOFTCAP_F32, f16, ep, status, st));
+#undef NC_TRY
+  return NC_OK;
 }
 
 nc_status nc_selftest_bounded_wait(uint32_t* dev_status, uint32_t limit_us, void* stream) {

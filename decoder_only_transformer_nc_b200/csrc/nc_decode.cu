@@ -1,0 +1,258 @@
+// KV-cache inference: cache append and the attention of one new position per
+// row over the cached keys ("从文本到聊天模型" §10.1-10.4: the prompt's keys and
+// values are kept per layer, and each further token attends over them instead
+// of recomputing the whole prefix).
+//
+// Cache of one layer: [B][T_max][2][Hkv][D] 16-bit -- for each row and position
+// the k heads (after RoPE and QK-norm, in the pair-interleaved order the
+// forward's QKV epilogue produces) followed by the v heads.  q uses the same
+// order, so q . k is unchanged.
+//
+// Decode attention is bound by reading the cached K/V.  Grid (split, kv head,
+// row): each CTA takes a contiguous chunk of the visible keys [lo, pos] for all
+// query heads of one kv group (GQA: the group's heads share every K/V row the
+// CTA reads), four warps stride over the chunk, and every lane holds D/32
+// dimensions, so a warp reads whole 256-byte K and V rows.  Softmax is the
+// exact online form in fp32 (log2 domain).  Each CTA leaves (m, l, o) per head;
+// a second kernel merges the splits.
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "nc_half.cuh"
+#include "nc_internal.h"
+
+namespace nc {
+namespace {
+
+constexpr int kMaxSplits = 32;
+constexpr int kWarps = 4;
+
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ float warp_allsum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+__global__ void __launch_bounds__(256) kv_append_kernel(const uint4* __restrict__ qkv, int64_t ldq16,
+                                                        int col16, int width16, uint4* __restrict__ cache,
+                                                        int M, int T, int T_max, int pos0) {
+  const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= (int64_t)M * width16) return;
+  const int m = (int)(idx / width16);
+  const int c = (int)(idx - (int64_t)m * width16);
+  const int b = m / T, t = pos0 + m % T;
+  cache[((int64_t)b * T_max + t) * width16 + c] = qkv[(int64_t)m * ldq16 + col16 + c];
+}
+
+// DW: dimensions per lane (D / 32); G: query heads per kv head.
+template <int DW, int G, bool F16>
+__global__ void __launch_bounds__(kWarps * 32) decode_attn_kernel(const uint16_t* __restrict__ q, int64_t ldq,
+                                                                  const uint16_t* __restrict__ cache,
+                                                                  float* __restrict__ partial, int H, int Hkv,
+                                                                  int T_max, int lo, int hi, int chunk,
+                                                                  float scale_log2) {
+  constexpr int D = DW * 32;
+  const int s = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int k_begin = lo + s * chunk;
+  const int k_end = min(k_begin + chunk, hi + 1);
+
+  float qv[G][DW];
+#pragma unroll
+  for (int i = 0; i < G; ++i) {
+    const uint16_t* qp = q + (int64_t)b * ldq + (int64_t)(g * G + i) * D + lane * DW;
+#pragma unroll
+    for (int d = 0; d < DW; d += 2) {
+      const float2 f = Half<F16>::unpack2(*reinterpret_cast<const uint32_t*>(qp + d));
+      qv[i][d] = f.x;
+      qv[i][d + 1] = f.y;
+    }
+  }
+  float m[G], l[G], o[G][DW];
+#pragma unroll
+  for (int i = 0; i < G; ++i) {
+    m[i] = -INFINITY;
+    l[i] = 0.0f;
+#pragma unroll
+    for (int d = 0; d < DW; ++d) o[i][d] = 0.0f;
+  }
+  const int64_t row_stride = 2 * (int64_t)Hkv * D;  // one cached position
+  const uint16_t* kbase = cache + (int64_t)b * T_max * row_stride + (int64_t)g * D + lane * DW;
+  const uint16_t* vbase = kbase + (int64_t)Hkv * D;
+  for (int j0 = k_begin + warp; j0 < k_end; j0 += 2 * kWarps) {
+    // two keys per step, both rows' loads issued before either is used
+    const int j1 = j0 + kWarps;
+    const bool has1 = j1 < k_end;
+    float kf[2][DW], vf[2][DW];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int j = u == 0 ? j0 : (has1 ? j1 : j0);
+#pragma unroll
+      for (int d = 0; d < DW; d += 2) {
+        const float2 kk = Half<F16>::unpack2(*reinterpret_cast<const uint32_t*>(kbase + j * row_stride + d));
+        const float2 vv = Half<F16>::unpack2(*reinterpret_cast<const uint32_t*>(vbase + j * row_stride + d));
+        kf[u][d] = kk.x;
+        kf[u][d + 1] = kk.y;
+        vf[u][d] = vv.x;
+        vf[u][d + 1] = vv.y;
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      if (u == 1 && !has1) break;  // warp-uniform
+#pragma unroll
+      for (int i = 0; i < G; ++i) {
+        float dot = 0.0f;
+#pragma unroll
+        for (int d = 0; d < DW; ++d) dot = fmaf(qv[i][d], kf[u][d], dot);
+        const float sc = warp_allsum(dot) * scale_log2;
+        const float mn = fmaxf(m[i], sc);
+        const float a = ex2(m[i] - mn);  // 0 on the first key (m = -inf)
+        const float p = ex2(sc - mn);
+        l[i] = fmaf(l[i], a, p);
+#pragma unroll
+        for (int d = 0; d < DW; ++d) o[i][d] = fmaf(o[i][d], a, p * vf[u][d]);
+        m[i] = mn;
+      }
+    }
+  }
+  // merge the four warps, then write this split's (m, l, o) per head
+  __shared__ float sm_ml[kWarps][G][2];
+  __shared__ float sm_o[kWarps][G][D];
+#pragma unroll
+  for (int i = 0; i < G; ++i) {
+    if (lane == 0) {
+      sm_ml[warp][i][0] = m[i];
+      sm_ml[warp][i][1] = l[i];
+    }
+#pragma unroll
+    for (int d = 0; d < DW; ++d) sm_o[warp][i][lane * DW + d] = o[i][d];
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < G * D; e += kWarps * 32) {
+    const int i = e / D, d = e - i * D;
+    float mm = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) mm = fmaxf(mm, sm_ml[w][i][0]);
+    float ll = 0.0f, oo = 0.0f;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) {
+      const float mw = sm_ml[w][i][0];
+      const float f = mw == -INFINITY ? 0.0f : ex2(mw - mm);
+      ll = fmaf(sm_ml[w][i][1], f, ll);
+      oo = fmaf(sm_o[w][i][d], f, oo);
+    }
+    float* dst = partial + (((int64_t)b * H + g * G + i) * kMaxSplits + s) * (2 + D);
+    if (d == 0) {
+      dst[0] = mm;
+      dst[1] = ll;
+    }
+    dst[2 + d] = oo;
+  }
+}
+
+// One block per (row, head); thread d merges dimension d over the splits.
+template <bool F16>
+__global__ void decode_combine_kernel(const float* __restrict__ partial, uint16_t* __restrict__ out, int H, int D,
+                                      int splits) {
+  const int bh = blockIdx.x;
+  const int d = threadIdx.x;
+  const float* p = partial + (int64_t)bh * kMaxSplits * (2 + D);
+  float mm = -INFINITY;
+  for (int s = 0; s < splits; ++s) mm = fmaxf(mm, p[s * (2 + D)]);
+  float ll = 0.0f, oo = 0.0f;
+  for (int s = 0; s < splits; ++s) {
+    const float* q = p + s * (2 + D);
+    const float f = q[0] == -INFINITY ? 0.0f : ex2(q[0] - mm);
+    ll = fmaf(q[1], f, ll);
+    oo = fmaf(q[2 + d], f, oo);
+  }
+  const float v = ll > 0.0f ? oo / ll : 0.0f;
+  const float v1 = __shfl_down_sync(0xffffffffu, v, 1);  // blockDim = D, a multiple of 32
+  if ((d & 1) == 0) *reinterpret_cast<uint32_t*>(out + (int64_t)bh * D + d) = Half<F16>::pack2(v, v1);
+}
+
+template <int DW, bool F16>
+nc_status decode_dispatch(const uint16_t* q, int64_t ldq, const uint16_t* cache, float* partial, int B, int H,
+                          int Hkv, int T_max, int lo, int hi, int splits, int chunk, float scale_log2,
+                          cudaStream_t stream) {
+  const dim3 grid(splits, Hkv, B);
+  switch (H / Hkv) {
+    case 1:
+      decode_attn_kernel<DW, 1, F16><<<grid, kWarps * 32, 0, stream>>>(q, ldq, cache, partial, H, Hkv, T_max, lo,
+                                                                       hi, chunk, scale_log2);
+      break;
+    case 2:
+      decode_attn_kernel<DW, 2, F16><<<grid, kWarps * 32, 0, stream>>>(q, ldq, cache, partial, H, Hkv, T_max, lo,
+                                                                       hi, chunk, scale_log2);
+      break;
+    case 4:
+      decode_attn_kernel<DW, 4, F16><<<grid, kWarps * 32, 0, stream>>>(q, ldq, cache, partial, H, Hkv, T_max, lo,
+                                                                       hi, chunk, scale_log2);
+      break;
+    case 8:
+      decode_attn_kernel<DW, 8, F16><<<grid, kWarps * 32, 0, stream>>>(q, ldq, cache, partial, H, Hkv, T_max, lo,
+                                                                       hi, chunk, scale_log2);
+      break;
+    default:
+      return NC_ERR_SHAPE;
+  }
+  return cudaGetLastError() == cudaSuccess ? NC_OK : NC_ERR_CUDA;
+}
+
+}  // namespace
+
+int decode_attention_max_splits() { return kMaxSplits; }
+
+nc_status kv_append_launch(const uint16_t* qkv, int64_t ldq, int col0, int width, uint16_t* cache, int M, int T,
+                           int T_max, int pos0, cudaStream_t stream) {
+  if (M == 0) return NC_OK;
+  if (ldq % 8 || col0 % 8 || width % 8) return NC_ERR_SHAPE;
+  const int64_t n = (int64_t)M * (width / 8);
+  kv_append_kernel<<<(unsigned)((n + 255) / 256), 256, 0, stream>>>(
+      reinterpret_cast<const uint4*>(qkv), ldq / 8, col0 / 8, width / 8, reinterpret_cast<uint4*>(cache), M, T,
+      T_max, pos0);
+  return cudaGetLastError() == cudaSuccess ? NC_OK : NC_ERR_CUDA;
+}
+
+nc_status decode_attention_launch(const uint16_t* q, int64_t ldq, const uint16_t* cache, float* partial,
+                                  uint16_t* out, int B, int H, int Hkv, int D, int T_max, int pos, int W, bool f16,
+                                  cudaStream_t stream) {
+  if (B == 0) return NC_OK;
+  if ((D != 64 && D != 128) || H % Hkv != 0) return NC_ERR_SHAPE;
+  const int lo = pos - W + 1 > 0 ? pos - W + 1 : 0;
+  const int n_keys = pos - lo + 1;
+  // enough CTAs to keep every SM streaming K/V: about 8 per SM
+  int splits = (8 * device_sm_count() + B * Hkv - 1) / (B * Hkv);
+  splits = splits < 1 ? 1 : (splits > kMaxSplits ? kMaxSplits : splits);
+  int chunk = (n_keys + splits - 1) / splits;
+  chunk = chunk < 16 ? 16 : chunk;
+  splits = (n_keys + chunk - 1) / chunk;
+  const float scale_log2 = 1.4426950408889634f / sqrtf((float)D);
+  nc_status s;
+  if (D == 128)
+    s = f16 ? decode_dispatch<4, true>(q, ldq, cache, partial, B, H, Hkv, T_max, lo, pos, splits, chunk, scale_log2,
+                                       stream)
+            : decode_dispatch<4, false>(q, ldq, cache, partial, B, H, Hkv, T_max, lo, pos, splits, chunk,
+                                        scale_log2, stream);
+  else
+    s = f16 ? decode_dispatch<2, true>(q, ldq, cache, partial, B, H, Hkv, T_max, lo, pos, splits, chunk, scale_log2,
+                                       stream)
+            : decode_dispatch<2, false>(q, ldq, cache, partial, B, H, Hkv, T_max, lo, pos, splits, chunk,
+                                        scale_log2, stream);
+  if (s != NC_OK) return s;
+  if (f16)
+    decode_combine_kernel<true><<<B * H, D, 0, stream>>>(partial, out, H, D, splits);
+  else
+    decode_combine_kernel<false><<<B * H, D, 0, stream>>>(partial, out, H, D, splits);
+  return cudaGetLastError() == cudaSuccess ? NC_OK : NC_ERR_CUDA;
+}
+
+}  // namespace nc

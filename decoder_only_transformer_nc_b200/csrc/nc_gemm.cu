@@ -280,9 +280,9 @@ __device__ __forceinline__ void epilogue_qkv_head(uint32_t taddr, const CUtensor
     ss += (s4[0] + s4[1]) + (s4[2] + s4[3]);
   }
   const float rs = rsqrtf(ss * (1.0f / HD) + ep.eps);
-  const int t = (row < M ? row : 0) % ep.T;
+  const int t = ep.pos0 + (row < M ? row : 0) % ep.T;
   const float* cs = ep.rope + (int64_t)t * (HD / 2);
-  const float* sn = ep.rope + ((int64_t)ep.T + t) * (HD / 2);
+  const float* sn = ep.rope + ((int64_t)(ep.rope_T > 0 ? ep.rope_T : ep.T) + t) * (HD / 2);
   // Pass 2 runs twice: first the rotated first halves u'_i (columns [0, HD/2)),
   // then -- re-reading TMEM -- the second halves u'_{i+HD/2}, so no half has to
   // be held in registers across a TMA store.
@@ -389,9 +389,9 @@ __device__ __forceinline__ void epilogue_qkv_head_il(uint32_t taddr, const CUten
     ss += (s4[0] + s4[1]) + (s4[2] + s4[3]);
   }
   const float rs = rsqrtf(ss * (1.0f / HD) + ep.eps);
-  const int t = (row < M ? row : 0) % ep.T;
+  const int t = ep.pos0 + (row < M ? row : 0) % ep.T;
   const float* cs = ep.rope + (int64_t)t * (HD / 2);
-  const float* sn = ep.rope + ((int64_t)ep.T + t) * (HD / 2);
+  const float* sn = ep.rope + ((int64_t)(ep.rope_T > 0 ? ep.rope_T : ep.T) + t) * (HD / 2);
 #pragma unroll 1
   for (int c = 0; c < HD / 64; ++c) {  // pairs 32c .. 32c+31
     uint32_t r0[32], r1[32];
@@ -570,9 +570,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         // This row's cos/sin lines are known before the accumulator is ready:
         // pull them into L1 while the MMAs run (q and k heads only).
         if (row < M && n0 < N && n0 / HD < ep.H + ep.Hkv) {
-          const int t = row % ep.T;
+          const int t = ep.pos0 + row % ep.T;
+          const int rt = ep.rope_T > 0 ? ep.rope_T : ep.T;
           const char* cl = reinterpret_cast<const char*>(ep.rope + (int64_t)t * (HD / 2));
-          const char* sl = reinterpret_cast<const char*>(ep.rope + ((int64_t)ep.T + t) * (HD / 2));
+          const char* sl = reinterpret_cast<const char*>(ep.rope + ((int64_t)rt + t) * (HD / 2));
 #pragma unroll
           for (int l = 0; l < HD * 2 / 128; ++l) {
             asm volatile("prefetch.global.L1 [%0];" ::"l"(cl + 128 * l));

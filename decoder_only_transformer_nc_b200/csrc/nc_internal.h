@@ -34,7 +34,9 @@ struct EpiParams {
   float* ce_target;         // EPI_CE_PARTIAL: [M], l[m, y_m] (written by one tile)
   const int32_t* targets;   // EPI_CE_PARTIAL: [M]
   const float* rope;        // EPI_QKV_ROPE: [2][T][D/2] cos, sin
-  int T;                    // EPI_QKV_ROPE: positions per sequence (row m is at m % T)
+  int T;                    // EPI_QKV_ROPE: positions per sequence (row m is at pos0 + m % T)
+  int pos0;                 // EPI_QKV_ROPE: position of the first row of each sequence
+  int rope_T;               // EPI_QKV_ROPE: positions in the rope table (0: T)
   int H, Hkv, D;            // EPI_QKV_ROPE: head counts and head size
   float eps;                // EPI_QKV_ROPE: RMSNorm epsilon
   const int32_t* tokens;    // EPI_QKV_ROPE_IL with value embedding: [M] token ids
@@ -99,6 +101,20 @@ nc_status embedding_extra_launch(const int32_t* tokens, const float* wte, const 
 nc_status rmsnorm_mix_launch(float* x, const float* x0, const float* lam_r, const float* lam_0,
                              float* x_keep, const float* x_sub, const float* lam_sub, bool write_back,
                              uint16_t* out, int M, int C, float eps, bool f16, cudaStream_t stream);
+// ---- KV-cache decode (nc_decode.cu)
+// Copies the k|v columns [col0, col0 + width) of the M rows of qkv (row stride
+// ldq) into a layer's cache [B][T_max][width]: row m goes to (m / T, pos0 + m % T).
+nc_status kv_append_launch(const uint16_t* qkv, int64_t ldq, int col0, int width, uint16_t* cache, int M, int T,
+                           int T_max, int pos0, cudaStream_t stream);
+// Attention of one query position `pos` per row over the cached keys [lo, pos],
+// lo = max(0, pos - W + 1): q [B, H*D] (row stride ldq), cache [B][T_max][2][Hkv][D]
+// -> out [B, H*D] (16-bit).  `partial` holds splits x (2 + D) fp32 per (b, h).
+nc_status decode_attention_launch(const uint16_t* q, int64_t ldq, const uint16_t* cache, float* partial,
+                                  uint16_t* out, int B, int H, int Hkv, int D, int T_max, int pos, int W,
+                                  bool f16, cudaStream_t stream);
+// Upper bound of the per-(b, h) splits decode_attention_launch uses.
+int decode_attention_max_splits();
+
 nc_status rmsnorm_launch(const float* x, uint16_t* out, int M, int C, float eps, bool f16,
                          cudaStream_t stream);
 nc_status rope_table_launch(float* table, int T, int D, float base, cudaStream_t stream);

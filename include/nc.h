@@ -192,6 +192,52 @@ nc_status nc_forward(const nc_config* cfg, const nc_weights* w, const int32_t* t
                      const int32_t* targets, int B, int T, float* logits, float* token_loss,
                      float* loss, void* workspace, size_t ws_bytes, void* stream);
 
+/* ---------------------------------------------------------------- KV-cache inference */
+
+/* "从文本到聊天模型" §10.1-10.4: the prompt runs once (prefill) and its keys
+ * and values are kept per layer; each further token then runs the stack on one
+ * position per row (decode) and attends over the kept keys instead of the
+ * whole prefix.  The state between calls is one caller-owned device buffer,
+ * the session:
+ *   the 16-bit weights (cast once by nc_prefill from the fp32 weights),
+ *   the RoPE table for T_max positions,
+ *   the cache of every layer, [B][T_max][2][Hkv][D] 16-bit -- per row and
+ *     position the k heads after RoPE and QK-norm (in the library's internal
+ *     head-dimension order) then the v heads,
+ *   the scratch of one decode step, and the device status word (first 4
+ *     bytes, cleared by every call).
+ * The KV-cache path covers the plain block stack: cfg->extras must be 0
+ * (NC_ERR_CONFIG otherwise).  Decode attention needs n_head / n_kv_head in
+ * {1, 2, 4, 8} (NC_ERR_SHAPE otherwise).  T_max <= cfg->seq_len. */
+
+/* Session bytes for B rows of up to T_max positions (0 on bad input).  Host only. */
+size_t nc_session_bytes(const nc_config* cfg, int B, int T_max);
+
+/* Scratch bytes nc_prefill needs for a [B, T] prompt (the forward's workspace
+ * without the weight copy, which lives in the session).  Host only. */
+size_t nc_prefill_workspace_bytes(const nc_config* cfg, int B, int T);
+
+/* Runs the forward over tokens [B, T] (device int32), casts the weights into
+ * the session and stores positions [0, T) of every layer's cache.  logits
+ * [B, T, V] fp32 (device) or NULL: the soft-capped logits of every position.
+ * session: nc_session_bytes(cfg, B, T_max) bytes, 256-byte aligned;
+ * workspace: nc_prefill_workspace_bytes(cfg, B, T) bytes, 256-byte aligned.
+ * Asynchronous on `stream`. */
+nc_status nc_prefill(const nc_config* cfg, const nc_weights* w, const int32_t* tokens, int B, int T,
+                     float* logits, void* session, size_t session_bytes, int T_max, void* workspace,
+                     size_t ws_bytes, void* stream);
+
+/* One decode step: tokens [B] (device int32) are the tokens at position `pos`
+ * of every row (0 <= pos < T_max); the session must hold positions [0, pos) of
+ * the same rows (nc_prefill of T = pos tokens, then one step per further
+ * position) and the weights cast from the same `w`, whose fp32 wte this step
+ * reads.  Stores position pos of every layer's cache and writes logits [B, V]
+ * fp32 (device, 16-byte aligned): the soft-capped logits at position pos,
+ * equal to those of nc_forward over the whole prefix.  Asynchronous on
+ * `stream`. */
+nc_status nc_decode_step(const nc_config* cfg, const nc_weights* w, const int32_t* tokens, int B, int pos,
+                         float* logits, void* session, size_t session_bytes, int T_max, void* stream);
+
 /* Kinds of kernel launch reported by nc_forward_traced. */
 typedef enum {
   NC_K_ROPE_TABLE = 0,

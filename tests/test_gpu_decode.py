@@ -1,0 +1,95 @@
+"""KV-cache inference (nc_prefill / nc_decode_step) against the oracle.
+
+"从文本到聊天模型" §10.1-10.4: a decode step for position t attends over the
+cached keys of positions [0, t] and must give the logits the whole forward
+gives at position t -- the oracle's forward over the prefix is the reference.
+Bars as for the forward: logits max-abs <= 3e-2.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from workloads import SHAPES, make_tokens, make_weights
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+
+def _oracle_cfg(s):
+    return oracle.OracleConfig(s.n_layer, s.d_model, s.n_head, s.n_kv_head, s.head_dim, s.seq_len,
+                               s.vocab, short_window=s.short_window)
+
+
+def _model(nc, s):
+    w = make_weights(s)
+    cfg = nc.make_config(s.n_layer, s.d_model, s.n_head, s.n_kv_head, s.head_dim, s.seq_len, s.vocab,
+                         s.short_window)
+    return w, nc.Model.from_numpy(cfg, w)
+
+
+def _run(nc, model, x, T0, steps, T_max):
+    """Prefill x[:, :T0], then decode positions T0 .. T0+steps-1 feeding x's own
+    tokens.  Returns (prefill logits [B, T0, V], decode logits [steps, B, V])."""
+    B = x.shape[0]
+    sess = nc.Session(model, B, T_max)
+    tx = torch.from_numpy(x).to(DEV)
+    pre = sess.prefill(tx[:, :T0].contiguous(), want_logits=True)
+    outs = []
+    for k in range(steps):
+        outs.append(sess.decode(tx[:, T0 + k].contiguous()).clone())
+    torch.cuda.synchronize()
+    assert sess.status() == 0
+    return pre, torch.stack(outs)
+
+
+def test_decode_matches_forward_tiny(gpu):
+    s = SHAPES["tiny"]
+    w, model = _model(gpu, s)
+    x, _ = make_tokens(s, batch=2)
+    T0, steps = 100, 12  # positions past the 64-key short window
+    pre, dec = _run(gpu, model, x, T0, steps, s.seq_len)
+    # prefill is the forward: same logits as nc_forward over the prompt
+    fwd = gpu.forward(model, torch.from_numpy(x[:, :T0].copy()).to(DEV), None, want_logits=True)
+    torch.cuda.synchronize()
+    assert torch.equal(pre, fwd["logits"])
+    want = oracle.forward(_oracle_cfg(s), w, x[:, :T0 + steps])["logits"]
+    err = np.abs(dec.cpu().numpy() - np.transpose(want[:, T0:T0 + steps], (1, 0, 2))).max()
+    assert err <= 3e-2, f"tiny decode logits max-abs {err:.3e}"
+    err_pre = np.abs(pre.cpu().numpy() - want[:, :T0]).max()
+    assert err_pre <= 3e-2
+
+
+def test_decode_from_position_zero_and_short_prompt(gpu):
+    """pos 0 (nothing cached yet) and a one-token prompt."""
+    s = SHAPES["tiny"]
+    w, model = _model(gpu, s)
+    x, _ = make_tokens(s, seed=77, batch=3)
+    sess = gpu.Session(model, 3, 32)
+    tx = torch.from_numpy(x).to(DEV)
+    sess.prefill(torch.empty((3, 0), dtype=torch.int32, device=DEV))  # weights and RoPE table only
+    assert sess.pos == 0
+    outs = [sess.decode(tx[:, k].contiguous()).clone() for k in range(5)]
+    torch.cuda.synchronize()
+    want = oracle.forward(_oracle_cfg(s), w, x[:, :5])["logits"]
+    got = torch.stack(outs).cpu().numpy()
+    assert np.abs(got - np.transpose(want, (1, 0, 2))).max() <= 3e-2
+    pre, dec = _run(gpu, model, x, 1, 4, 32)
+    assert np.abs(dec.cpu().numpy() - np.transpose(want[:, 1:5], (1, 0, 2))).max() <= 3e-2
+
+
+@pytest.mark.parametrize("name,T0", [("d20", 1000), ("d26_gqa", 700)])
+def test_decode_full_size_model(gpu, name, T0):
+    """d20 (MHA) and d26-GQA (4 query heads per kv head), past the 512-key short
+    window, two rows; the oracle recomputes row 1."""
+    s = SHAPES[name]
+    w, model = _model(gpu, s)
+    x, _ = make_tokens(s, batch=2)
+    steps = 4
+    _, dec = _run(gpu, model, x, T0, steps, s.seq_len)
+    del model
+    torch.cuda.empty_cache()
+    want = oracle.forward(_oracle_cfg(s), w, x[1:2, :T0 + steps])["logits"][0, T0:]
+    err = np.abs(dec[:, 1].cpu().numpy() - want).max()
+    assert err <= 3e-2, f"{name} decode logits max-abs {err:.3e}"

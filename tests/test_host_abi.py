@@ -205,3 +205,31 @@ def test_extras_host_rules(nclib):
         assert _fwd(nclib, cx, fw, 2, 16) == 8
     tabs[1] = (1 << 44) + 8  # misaligned table
     assert _fwd(nclib, cx, fw, 2, 16) == 4
+
+
+def test_kv_cache_host_rules(nclib):
+    """Session sizing and the host-side refusals of nc_prefill / nc_decode_step."""
+    L = nclib.lib()
+    cfg = nclib.init_config(2, 64, 64, 0, 256, 512)
+    n = L.nc_session_bytes(ctypes.byref(cfg), 2, 256)
+    # at least the cache: layers x B x T_max x (k, v) x Hkv x D x 2 bytes
+    assert n >= 2 * 2 * 256 * 2 * cfg.n_kv_head * cfg.head_dim * 2
+    assert L.nc_session_bytes(ctypes.byref(cfg), 2, 257) == 0  # T_max > seq_len
+    assert L.nc_prefill_workspace_bytes(ctypes.byref(cfg), 2, 100) < nclib.workspace_bytes(cfg, 2, 100)
+    fw = _FakeWeights(nclib, 2)
+    sess, tok, out = 1 << 43, 1 << 41, 1 << 44
+    dec = lambda c, pos, nbytes=n, T_max=256: L.nc_decode_step(ctypes.byref(c), ctypes.byref(fw.w), tok, 2, pos,
+                                                               out, sess, nbytes, T_max, None)
+    assert dec(cfg, 256) == 3           # pos >= T_max
+    assert dec(cfg, -1) == 3
+    assert dec(cfg, 5, nbytes=n - 1) == 5  # session too small
+    cx = nclib.NcConfig.from_buffer_copy(cfg)
+    cx.extras = nclib.EXTRA_SMEAR
+    assert dec(cx, 5) == 2               # the KV-cache path is the plain stack
+    pre = lambda T, T_max=256: L.nc_prefill(ctypes.byref(cfg), ctypes.byref(fw.w), tok, 2, T, None, sess, n, T_max,
+                                             1 << 42, 1 << 30, None)
+    assert pre(300) == 3                 # T > T_max
+    import torch
+    if not torch.cuda.is_available():
+        assert dec(cfg, 5) == 8          # valid arguments, no sm_100 device
+        assert pre(100) == 8
