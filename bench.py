@@ -398,6 +398,120 @@ def run_ours(args, s):
         print(json.dumps(result), flush=True)
 
 
+def decode_bytes(s, B, pos):
+    """Algorithmic HBM bytes of one decode step at position `pos`: every 16-bit
+    projection weight once, the fp32 embedding rows, each layer's visible cached
+    K and V rows, and the new position's K and V written."""
+    C, H, Hkv, D, V, L = s.d_model, s.n_head, s.n_kv_head, s.head_dim, s.vocab, s.n_layer
+    weights = 2 * (L * (C * (H + 2 * Hkv) * D + H * D * C + 8 * C * C) + V * C)
+    kv_row = 2 * Hkv * D * 2
+    keys = 0
+    for l in range(L):
+        W = s.seq_len if (l % 4 == 3 or l == L - 1) else s.short_window
+        keys += min(pos + 1, W)
+    return weights + B * C * 4 + B * kv_row * keys + L * B * kv_row
+
+
+def run_decode(args, s):
+    """KV-cache decode throughput: prefill `--prompt` tokens (untimed), then time
+    `--steps` single-position steps for all B rows."""
+    import torch
+
+    import decoder_only_transformer_nc_b200 as nc
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import torch.distributed as dist
+        from datetime import timedelta
+        dist.init_process_group("nccl", device_id=dev, timeout=timedelta(seconds=120))
+    B, T0 = s.batch, args.prompt
+    K, Wm = args.steps, args.warmup
+    T_max = T0 + Wm + 2 * K + 4
+    if T_max > s.seq_len:
+        raise SystemExit(f"prompt + steps exceed seq_len {s.seq_len}")
+    cfg = nc.make_config(s.n_layer, s.d_model, s.n_head, s.n_kv_head, s.head_dim, s.seq_len, s.vocab,
+                         s.short_window)
+    model = nc.Model.from_numpy(cfg, make_weights(s), device=dev)
+    from decoder_only_transformer_nc_b200 import dp
+    x, _ = make_tokens(s, seed=dp.shard_seed(TOKEN_SEED, rank), seq_len=T_max)
+    tx = torch.from_numpy(x).to(dev)
+    sess = nc.Session(model, B, T_max, device=dev)
+    sess.prefill(tx[:, :T0].contiguous())
+    logits = torch.empty((B, s.vocab), dtype=torch.float32, device=dev)
+    steps_tok = [tx[:, T0 + k].contiguous() for k in range(Wm + 2 * K)]
+    for k in range(Wm):
+        sess.decode(steps_tok[k], logits=logits)
+    torch.cuda.synchronize()
+    if sess.status() != 0:
+        raise SystemExit(f"device status after warm-up: {sess.status()}")
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier(device_ids=[local])
+
+    stream = torch.cuda.current_stream()
+    pos0 = sess.pos
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clocks:
+        t0.record(stream)
+        for k in range(K):
+            sess.decode(steps_tok[Wm + k], logits=logits)
+        t1.record(stream)
+        torch.cuda.synchronize()
+    barrier()
+    ms = t0.elapsed_time(t1) / K
+    # e2e: tokens from pinned host memory in, the step's logits out, every step
+    hx = torch.from_numpy(x).pin_memory()
+    hlog = torch.empty((B, s.vocab), dtype=torch.float32).pin_memory()
+    dtok = torch.empty(B, dtype=torch.int32, device=dev)
+    barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for k in range(K):
+        dtok.copy_(hx[:, sess.pos], non_blocking=True)
+        sess.decode(dtok, logits=logits)
+        hlog.copy_(logits, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = e0.elapsed_time(e1) / K
+    if world > 1:
+        tt = torch.tensor([ms, e2e_ms], dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
+        ms, e2e_ms = float(tt[0]), float(tt[1])
+    byts = sum(decode_bytes(s, B, pos0 + k) for k in range(K)) / K
+    peaks, peak_src = load_peaks()
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    achieved = byts / (ms / 1e3) / 1e9
+    if rank == 0:
+        print(json.dumps({
+            "metric": "decode tokens/sec (KV cache, one position per row per step)", "value": world * B / (ms / 1e3),
+            "unit": UNIT, "n_gpus": world, "steps": K, "warmup": Wm, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": DTYPE_NOTE, "data": "synthetic",
+            "config": {"workload": f"{s.name} decode", "global_batch": world * B, "prompt": T0,
+                       "positions": [pos0, pos0 + K - 1], "parallelism": f"dp{world}" if world > 1 else "none",
+                       "l2": "weights (0.87 GB 16-bit) and KV cache larger than L2"},
+            "roofline": {"kernel": "whole decode step (weights + cached K/V streamed once)", "bound": "hbm",
+                         "achieved": round(achieved, 1), "peak": hbm, "peak_kind": f"hbm_gbs ({peak_src})",
+                         "unit": "GB/s", "frac": round(achieved / hbm, 4), "traffic": None,
+                         "algorithmic_bytes": int(byts)},
+            "gpu_launches": (3 + 10 * s.n_layer) * K,  # embedding; 10 per layer; final norm, lm_head
+            "e2e": {"value": world * B / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": B * 4,
+                    "d2h_bytes_per_step": B * s.vocab * 4},
+            "clocks": clocks.summary(),
+        }), flush=True)
+    if world > 1:
+        torch.distributed.barrier(device_ids=[local])
+        torch.distributed.destroy_process_group()
+
+
 def _flat(w):
     yield w["wte"]
     yield w["lm_head"]
@@ -417,6 +531,9 @@ def main():
     ap.add_argument("--ref-prefix", type=int, default=256,
                     help="positions of batch row 0 per step of the reference (oracle) arm")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--mode", default="forward", choices=["forward", "decode"],
+                    help="decode: KV-cache decode steps after a prefill of --prompt tokens")
+    ap.add_argument("--prompt", type=int, default=1024, help="decode mode: prompt length")
     ap.add_argument("--extras", default="none", choices=["none", "all"],
                     help="all: also run the full nanochat terms (smear, value embeddings, "
                          "residual lambdas + x0, backout)")
@@ -432,6 +549,8 @@ def main():
         s = dataclasses.replace(s, batch=args.batch)
     if args.impl == "reference":
         run_reference(args, s)
+    elif args.mode == "decode":
+        run_decode(args, s)
     else:
         run_ours(args, s)
 

@@ -139,7 +139,7 @@ WsLayout ws_layout(const nc_config* c, int B, int T, bool own_weights = true) {
 // by nc_prefill), the cache of every layer, and the scratch of one decode step
 // (B rows).  Offsets are 256-byte aligned.
 struct SessionLayout {
-  size_t status, rope, wqkv, wo, wfc, wmp, wlm, cache, x, a, qkv, o, h, part, total;
+  size_t status, rope, wqkv, wo, wfc, wmp, wlm, cache, x, a, qkv, o, h, part, acc, total;
   size_t wqkv_elems, wo_elems, wfc_elems, wmp_elems, cache_layer_elems;
 };
 
@@ -172,6 +172,7 @@ SessionLayout session_layout(const nc_config* c, int B, int T_max) {
   L.o = take(Bs * H * D * 2);
   L.h = take(Bs * 4 * C * 2);
   L.part = take(Bs * H * (size_t)decode_attention_max_splits() * (2 + D) * 4);
+  L.acc = take(Bs * (nqkv > 4 * C ? nqkv : 4 * C) * 4);  // fp32 split-K sums of QKV, then c_fc
   L.total = off;
   return L;
 }
@@ -730,6 +731,14 @@ nc_status nc_prefill(const nc_config* cfg, const nc_weights* w, const int32_t* t
                       nullptr, &sess);
 }
 
+// K slices for a residual-add GEMM with few output tiles: about one tile per SM.
+static int resid_ksplit(int M, int N, int K) {
+  const int tiles = ((M + 127) / 128) * ((N + 255) / 256);
+  const int kb = (K + 63) / 64;
+  int s = (device_sm_count() + tiles - 1) / tiles;
+  return s < 1 ? 1 : (s > kb ? kb : s);
+}
+
 nc_status nc_decode_step(const nc_config* cfg, const nc_weights* w, const int32_t* tokens, int B, int pos,
                          float* logits, void* session, size_t session_bytes, int T_max, void* stream) {
   if (!cfg || !w || !w->wte || !tokens || !logits || !session) return NC_ERR_INVALID_ARG;
@@ -759,6 +768,7 @@ nc_status nc_decode_step(const nc_config* cfg, const nc_weights* w, const int32_
   uint16_t* o = reinterpret_cast<uint16_t*>(base + SL.o);
   uint16_t* h = reinterpret_cast<uint16_t*>(base + SL.h);
   float* part = reinterpret_cast<float*>(base + SL.part);
+  float* acc = reinterpret_cast<float*>(base + SL.acc);
   const int C = cfg->d_model, D = cfg->head_dim, H = cfg->n_head, Hkv = cfg->n_kv_head, V = cfg->vocab;
   const int NQKV = (H + 2 * Hkv) * D;
   const bool f16 = cfg->act_dtype == NC_F16;
@@ -771,34 +781,38 @@ nc_status nc_decode_step(const nc_config* cfg, const nc_weights* w, const int32_
   } while (0)
   if (cudaMemsetAsync(status, 0, 256, st) != cudaSuccess) return NC_ERR_CUDA;
   NC_TRY(embedding_launch(tokens, w->wte, x, B, C, V, status, st));
+  // Few rows (B): every projection splits K over about one tile per SM.  The
+  // residual adds land in x directly; QKV and c_fc sum into an fp32 scratch that
+  // a small kernel finishes (RoPE + QK-norm + cache write, or ReLU^2).
+  const int ks_qkv = resid_ksplit(B, NQKV, C), ks_fc = resid_ksplit(B, 4 * C, C);
   for (int l = 0; l < cfg->n_layer; ++l) {
     NC_TRY(rmsnorm_launch(x, a, B, C, eps, f16, st));
-    EpiParams eq{};  // one row per sequence, at position pos
-    eq.out = qkv;
-    eq.ldo = NQKV;
-    eq.rope = rope;
-    eq.T = 1;
-    eq.pos0 = pos;
-    eq.rope_T = T_max;
-    eq.H = H;
-    eq.Hkv = Hkv;
-    eq.D = D;
-    eq.eps = eps;
-    NC_TRY(gemm_launch(a, C, wqkv + l * SL.wqkv_elems, C, B, NQKV, C, EPI_QKV_ROPE_IL, f16, eq, status, st));
     uint16_t* cl = cache + l * SL.cache_layer_elems;
-    NC_TRY(kv_append_launch(qkv, NQKV, H * D, 2 * Hkv * D, cl, B, 1, T_max, pos, st));
+    EpiParams eq{};
+    eq.out = acc;
+    eq.ldo = NQKV;
+    eq.ksplit = ks_qkv;
+    if (cudaMemsetAsync(acc, 0, (size_t)B * NQKV * 4, st) != cudaSuccess) return NC_ERR_CUDA;
+    NC_TRY(gemm_launch(a, C, wqkv + l * SL.wqkv_elems, C, B, NQKV, C, EPI_RESID_F32, f16, eq, status, st));
+    NC_TRY(qkv_finish_launch(acc, qkv, cl, rope, T_max, pos, B, H, Hkv, D, T_max, eps, f16, st));
     NC_TRY(decode_attention_launch(qkv, NQKV, cl, part, o, B, H, Hkv, D, T_max, pos, nc_layer_window(cfg, l),
                                    f16, st));
+    // Few rows: the residual adds split K over about one tile per SM (the
+    // partial products land in x by TMA reduce-add, in no fixed order).
     EpiParams ep{};
     ep.out = x;
     ep.ldo = C;
+    ep.ksplit = resid_ksplit(B, C, H * D);
     NC_TRY(gemm_launch(o, H * D, wo + l * SL.wo_elems, H * D, B, C, H * D, EPI_RESID_F32, f16, ep, status, st));
     NC_TRY(rmsnorm_launch(x, a, B, C, eps, f16, st));
-    ep.out = h;
-    ep.ldo = 4 * C;
-    NC_TRY(gemm_launch(a, C, wfc + l * SL.wfc_elems, C, B, 4 * C, C, EPI_RELU2_16, f16, ep, status, st));
-    ep.out = x;
-    ep.ldo = C;
+    EpiParams ef{};
+    ef.out = acc;
+    ef.ldo = 4 * C;
+    ef.ksplit = ks_fc;
+    if (cudaMemsetAsync(acc, 0, (size_t)B * 4 * C * 4, st) != cudaSuccess) return NC_ERR_CUDA;
+    NC_TRY(gemm_launch(a, C, wfc + l * SL.wfc_elems, C, B, 4 * C, C, EPI_RESID_F32, f16, ef, status, st));
+    NC_TRY(relu2_finish_launch(acc, h, (int64_t)B * 4 * C, f16, st));
+    ep.ksplit = resid_ksplit(B, C, 4 * C);
     NC_TRY(gemm_launch(h, 4 * C, wmp + l * SL.wmp_elems, 4 * C, B, C, 4 * C, EPI_RESID_F32, f16, ep, status, st));
   }
   NC_TRY(rmsnorm_launch(x, a, B, C, eps, f16, st));

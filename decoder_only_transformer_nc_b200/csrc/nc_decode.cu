@@ -12,7 +12,7 @@
 // row): each CTA takes a contiguous chunk of the visible keys [lo, pos] for all
 // query heads of one kv group (GQA: the group's heads share every K/V row the
 // CTA reads), four warps stride over the chunk, and every lane holds D/32
-// dimensions, so a warp reads whole 256-byte K and V rows.  Softmax is the
+// dimensions, so a warp reads whole 256-byte K and V rows, four keys at a time.  Softmax is the
 // exact online form in fp32 (log2 domain).  Each CTA leaves (m, l, o) per head;
 // a second kernel merges the splits.
 #include <cuda_runtime.h>
@@ -27,6 +27,7 @@ namespace {
 
 constexpr int kMaxSplits = 32;
 constexpr int kWarps = 4;
+constexpr int kUnroll = 4;  // keys a warp has in flight
 
 __device__ __forceinline__ float ex2(float x) {
   float y;
@@ -86,14 +87,13 @@ __global__ void __launch_bounds__(kWarps * 32) decode_attn_kernel(const uint16_t
   const int64_t row_stride = 2 * (int64_t)Hkv * D;  // one cached position
   const uint16_t* kbase = cache + (int64_t)b * T_max * row_stride + (int64_t)g * D + lane * DW;
   const uint16_t* vbase = kbase + (int64_t)Hkv * D;
-  for (int j0 = k_begin + warp; j0 < k_end; j0 += 2 * kWarps) {
-    // two keys per step, both rows' loads issued before either is used
-    const int j1 = j0 + kWarps;
-    const bool has1 = j1 < k_end;
-    float kf[2][DW], vf[2][DW];
+  for (int j0 = k_begin + warp; j0 < k_end; j0 += kUnroll * kWarps) {
+    // kUnroll keys per step, every row's loads issued before any is used
+    float kf[kUnroll][DW], vf[kUnroll][DW];
 #pragma unroll
-    for (int u = 0; u < 2; ++u) {
-      const int j = u == 0 ? j0 : (has1 ? j1 : j0);
+    for (int u = 0; u < kUnroll; ++u) {
+      const int ju = j0 + u * kWarps;
+      const int j = ju < k_end ? ju : j0;  // past the end: reload a valid row, unused
 #pragma unroll
       for (int d = 0; d < DW; d += 2) {
         const float2 kk = Half<F16>::unpack2(*reinterpret_cast<const uint32_t*>(kbase + j * row_stride + d));
@@ -105,8 +105,8 @@ __global__ void __launch_bounds__(kWarps * 32) decode_attn_kernel(const uint16_t
       }
     }
 #pragma unroll
-    for (int u = 0; u < 2; ++u) {
-      if (u == 1 && !has1) break;  // warp-uniform
+    for (int u = 0; u < kUnroll; ++u) {
+      if (j0 + u * kWarps >= k_end) break;  // warp-uniform
 #pragma unroll
       for (int i = 0; i < G; ++i) {
         float dot = 0.0f;
@@ -179,6 +179,76 @@ __global__ void decode_combine_kernel(const float* __restrict__ partial, uint16_
   if ((d & 1) == 0) *reinterpret_cast<uint32_t*>(out + (int64_t)bh * D + d) = Half<F16>::pack2(v, v1);
 }
 
+// Finish of the split-K QKV projection of a decode step: acc [B, (H + 2 Hkv) D]
+// fp32 (q and k columns in the pair-interleaved order of the packed weights:
+// columns 2i, 2i+1 of a head are the RoPE pair (u_i, u_{i+D/2})).  q and k heads
+// are rotated by pos * theta_i and RMS-normalised over the head ("Nanochat与
+// nanoGPT对比" §1: QK-norm after RoPE); v heads are converted.  Every head goes
+// to qkv [B, (H + 2 Hkv) D] 16-bit; k and v heads also to the layer's cache at
+// position pos.  One warp per (row, head); lane l holds columns 4l .. 4l+3
+// (D = 128) or 2l, 2l+1 (D = 64).
+template <int DW, bool F16>
+__global__ void __launch_bounds__(256) qkv_finish_kernel(const float* __restrict__ acc, uint16_t* __restrict__ qkv,
+                                                         uint16_t* __restrict__ cache, const float* __restrict__ rope,
+                                                         int rope_T, int pos, int B, int H, int Hkv, int T_max,
+                                                         float eps) {
+  constexpr int D = DW * 32;
+  const int heads = H + 2 * Hkv;
+  const int wid = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (wid >= B * heads) return;
+  const int b = wid / heads, hd = wid - b * heads;
+  const float* src = acc + ((int64_t)b * heads + hd) * D + lane * DW;
+  float v[DW];
+#pragma unroll
+  for (int d = 0; d < DW; ++d) v[d] = src[d];
+  if (hd < H + Hkv) {  // q or k head: RoPE on the adjacent pairs, then the head's RMSNorm
+    const float* cs = rope + (int64_t)pos * (D / 2);
+    const float* sn = rope + ((int64_t)rope_T + pos) * (D / 2);
+    float ss = 0.0f;
+#pragma unroll
+    for (int p = 0; p < DW / 2; ++p) {
+      const int i = lane * (DW / 2) + p;  // pair index
+      const float c = cs[i], sv = sn[i];
+      const float a = v[2 * p], bb = v[2 * p + 1];
+      v[2 * p] = a * c - bb * sv;
+      v[2 * p + 1] = a * sv + bb * c;
+      ss = fmaf(v[2 * p], v[2 * p], ss);
+      ss = fmaf(v[2 * p + 1], v[2 * p + 1], ss);
+    }
+    const float r = rsqrtf(warp_allsum(ss) * (1.0f / D) + eps);
+#pragma unroll
+    for (int d = 0; d < DW; ++d) v[d] *= r;
+  }
+  uint32_t pk[DW / 2];
+#pragma unroll
+  for (int p = 0; p < DW / 2; ++p) pk[p] = Half<F16>::pack2(v[2 * p], v[2 * p + 1]);
+  uint16_t* dst = qkv + ((int64_t)b * heads + hd) * D + lane * DW;
+  uint16_t* cdst = hd >= H ? cache + ((int64_t)b * T_max + pos) * 2 * Hkv * D + (int64_t)(hd - H) * D + lane * DW
+                           : nullptr;
+  if constexpr (DW == 4) {
+    const uint2 w2 = make_uint2(pk[0], pk[1]);
+    *reinterpret_cast<uint2*>(dst) = w2;
+    if (cdst) *reinterpret_cast<uint2*>(cdst) = w2;
+  } else {
+    *reinterpret_cast<uint32_t*>(dst) = pk[0];
+    if (cdst) *reinterpret_cast<uint32_t*>(cdst) = pk[0];
+  }
+}
+
+// relu(acc)^2 -> 16-bit ("从文本到聊天模型" §5.7), for the split-K c_fc of a decode step.
+template <bool F16>
+__global__ void relu2_finish_kernel(const float4* __restrict__ acc, uint2* __restrict__ out, int64_t n4) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n4) return;
+  float4 a = acc[i];
+  a.x = fmaxf(a.x, 0.f);
+  a.y = fmaxf(a.y, 0.f);
+  a.z = fmaxf(a.z, 0.f);
+  a.w = fmaxf(a.w, 0.f);
+  out[i] = make_uint2(Half<F16>::pack2(a.x * a.x, a.y * a.y), Half<F16>::pack2(a.z * a.z, a.w * a.w));
+}
+
 template <int DW, bool F16>
 nc_status decode_dispatch(const uint16_t* q, int64_t ldq, const uint16_t* cache, float* partial, int B, int H,
                           int Hkv, int T_max, int lo, int hi, int splits, int chunk, float scale_log2,
@@ -211,6 +281,39 @@ nc_status decode_dispatch(const uint16_t* q, int64_t ldq, const uint16_t* cache,
 
 int decode_attention_max_splits() { return kMaxSplits; }
 
+nc_status qkv_finish_launch(const float* acc, uint16_t* qkv, uint16_t* cache, const float* rope, int rope_T,
+                            int pos, int B, int H, int Hkv, int D, int T_max, float eps, bool f16,
+                            cudaStream_t stream) {
+  const int warps = B * (H + 2 * Hkv);
+  if (warps == 0) return NC_OK;
+  const unsigned grid = (unsigned)((warps + 7) / 8);
+  if (D == 128)
+    f16 ? qkv_finish_kernel<4, true><<<grid, 256, 0, stream>>>(acc, qkv, cache, rope, rope_T, pos, B, H, Hkv, T_max, eps)
+        : qkv_finish_kernel<4, false><<<grid, 256, 0, stream>>>(acc, qkv, cache, rope, rope_T, pos, B, H, Hkv, T_max,
+                                                                eps);
+  else if (D == 64)
+    f16 ? qkv_finish_kernel<2, true><<<grid, 256, 0, stream>>>(acc, qkv, cache, rope, rope_T, pos, B, H, Hkv, T_max, eps)
+        : qkv_finish_kernel<2, false><<<grid, 256, 0, stream>>>(acc, qkv, cache, rope, rope_T, pos, B, H, Hkv, T_max,
+                                                                eps);
+  else
+    return NC_ERR_SHAPE;
+  return cudaGetLastError() == cudaSuccess ? NC_OK : NC_ERR_CUDA;
+}
+
+nc_status relu2_finish_launch(const float* acc, uint16_t* out, int64_t n, bool f16, cudaStream_t stream) {
+  if (n == 0) return NC_OK;
+  if (n % 4) return NC_ERR_SHAPE;
+  const int64_t n4 = n / 4;
+  const unsigned grid = (unsigned)((n4 + 255) / 256);
+  if (f16)
+    relu2_finish_kernel<true><<<grid, 256, 0, stream>>>(reinterpret_cast<const float4*>(acc),
+                                                        reinterpret_cast<uint2*>(out), n4);
+  else
+    relu2_finish_kernel<false><<<grid, 256, 0, stream>>>(reinterpret_cast<const float4*>(acc),
+                                                         reinterpret_cast<uint2*>(out), n4);
+  return cudaGetLastError() == cudaSuccess ? NC_OK : NC_ERR_CUDA;
+}
+
 nc_status kv_append_launch(const uint16_t* qkv, int64_t ldq, int col0, int width, uint16_t* cache, int M, int T,
                            int T_max, int pos0, cudaStream_t stream) {
   if (M == 0) return NC_OK;
@@ -229,8 +332,8 @@ nc_status decode_attention_launch(const uint16_t* q, int64_t ldq, const uint16_t
   if ((D != 64 && D != 128) || H % Hkv != 0) return NC_ERR_SHAPE;
   const int lo = pos - W + 1 > 0 ? pos - W + 1 : 0;
   const int n_keys = pos - lo + 1;
-  // enough CTAs to keep every SM streaming K/V: about 8 per SM
-  int splits = (8 * device_sm_count() + B * Hkv - 1) / (B * Hkv);
+  // enough CTAs to keep every SM streaming K/V: about 16 per SM
+  int splits = (16 * device_sm_count() + B * Hkv - 1) / (B * Hkv);
   splits = splits < 1 ? 1 : (splits > kMaxSplits ? kMaxSplits : splits);
   int chunk = (n_keys + splits - 1) / splits;
   chunk = chunk < 16 ? 16 : chunk;

@@ -439,7 +439,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const uint32_t lane = lane_id();
   const int num_m = (M + BM - 1) / BM;
   const int num_n = (N + BN - 1) / BN;
-  const int num_tiles = num_m * num_n;
+  // Split-K (residual-add epilogue only): tile t covers K slice t / (num_m * num_n).
+  const int ksplit = (EPI == EPI_RESID_F32 && ep.ksplit > 1) ? ep.ksplit : 1;
+  const int num_mn = num_m * num_n;
+  const int num_tiles = num_mn * ksplit;
   const int num_kb = (K + BK - 1) / BK;
 
   if (threadIdx.x == 0) {
@@ -478,9 +481,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       uint32_t out_phase = 0;    // bit s: phase of that load
       bool ok = true;
       for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-        const int m0 = (tile / num_n) * BM;
-        const int n0 = (tile % num_n) * BN;
-        for (int kb = 0; kb < num_kb; ++kb) {
+        const int mn = tile % num_mn, ks = tile / num_mn;
+        const int m0 = (mn / num_n) * BM;
+        const int n0 = (mn % num_n) * BN;
+        const int kb_end = (ks + 1) * num_kb / ksplit;
+        for (int kb = ks * num_kb / ksplit; kb < kb_end; ++kb) {
           if (!mbar_wait(smem_u32(&sm->empty[stage]), phase ^ 1u, ctl)) {
             ok = false;
             break;
@@ -519,7 +524,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (!mbar_wait(smem_u32(&sm->tmem_empty[acc]), acc_phase ^ 1u, ctl)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * BN;
-        for (int kb = 0; kb < num_kb; ++kb) {
+        const int ks = tile / num_mn;
+        const int kb_begin = ks * num_kb / ksplit, kb_end = (ks + 1) * num_kb / ksplit;
+        for (int kb = kb_begin; kb < kb_end; ++kb) {
           if (!mbar_wait(smem_u32(&sm->full[stage]), phase, ctl)) {
             ok = false;
             break;
@@ -531,7 +538,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           for (int k = 0; k < BK / 16; ++k) {
             const uint64_t adesc = sw128_kmajor_desc(a_addr + k * 32);
             const uint64_t bdesc = sw128_kmajor_desc(b_addr + k * 32);
-            umma_f16(d_tmem, adesc, bdesc, IDESC, (kb | k) != 0 ? 1u : 0u);
+            umma_f16(d_tmem, adesc, bdesc, IDESC, (kb != kb_begin || k != 0) ? 1u : 0u);
           }
           umma_commit(smem_u32(&sm->empty[stage]));
           if (++stage == STAGES) {
@@ -561,8 +568,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
-      const int m_blk = tile / num_n;
-      const int n_blk = tile % num_n;
+      const int m_blk = (tile % num_mn) / num_n;
+      const int n_blk = (tile % num_mn) % num_n;
       const int m0 = m_blk * BM;
       const int n0 = n_blk * BN + half * EPI_COLS;  // this warp's first column
       const int row = m0 + row_in_tile;
@@ -679,7 +686,7 @@ static cudaError_t launch_t(const CUtensorMap& ma, const CUtensorMap& mb, const 
     if (e != cudaSuccess) return e;
     attr_done[dev] = true;
   }
-  const int tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
+  const int tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN) * (EPI == EPI_RESID_F32 && ep.ksplit > 1 ? ep.ksplit : 1);
   const int sms = device_sm_count();
   const int grid = tiles < sms ? tiles : sms;
   gemm_kernel<EPI, F16, HD><<<grid, NUM_THREADS, SMEM_BYTES, stream>>>(ma, mb, mc, M, N, K, ep,
@@ -773,6 +780,7 @@ nc_status gemm_launch(const uint16_t* a, int64_t lda, const uint16_t* w, int64_t
   using namespace gemm;
   if (epi < EPI_STORE_16 || epi > EPI_QKV_ROPE_IL) return NC_ERR_INVALID_ARG;
   if ((epi == EPI_QKV_ROPE || epi == EPI_QKV_ROPE_IL) && (ep.D != 64 && ep.D != 128)) return NC_ERR_SHAPE;
+  if (ep.ksplit > 1 && (epi != EPI_RESID_F32 || ep.ksplit > (K + BK - 1) / BK)) return NC_ERR_INVALID_ARG;
   CUtensorMap ma, mb, mc;
   if (!make_map(&ma, a, M, K, lda, BM, f16)) return NC_ERR_CUDA;
   if (!make_map(&mb, w, N, K, ldw, BN, f16)) return NC_ERR_CUDA;

@@ -37,6 +37,9 @@ struct EpiParams {
   int T;                    // EPI_QKV_ROPE: positions per sequence (row m is at pos0 + m % T)
   int pos0;                 // EPI_QKV_ROPE: position of the first row of each sequence
   int rope_T;               // EPI_QKV_ROPE: positions in the rope table (0: T)
+  int ksplit;               // EPI_RESID_F32: K is split into this many slices, each tile of a
+                            //   slice adding its partial product into out (0 or 1: no split;
+                            //   the fp32 sums then depend on the order the slices land)
   int H, Hkv, D;            // EPI_QKV_ROPE: head counts and head size
   float eps;                // EPI_QKV_ROPE: RMSNorm epsilon
   const int32_t* tokens;    // EPI_QKV_ROPE_IL with value embedding: [M] token ids
@@ -114,6 +117,14 @@ nc_status decode_attention_launch(const uint16_t* q, int64_t ldq, const uint16_t
                                   bool f16, cudaStream_t stream);
 // Upper bound of the per-(b, h) splits decode_attention_launch uses.
 int decode_attention_max_splits();
+// From the fp32 split-K sum of a decode step's QKV projection: RoPE at `pos` and
+// QK-norm of q and k heads (pair-interleaved columns), 16-bit qkv, and k|v heads
+// into the layer's cache at `pos`.
+nc_status qkv_finish_launch(const float* acc, uint16_t* qkv, uint16_t* cache, const float* rope, int rope_T,
+                            int pos, int B, int H, int Hkv, int D, int T_max, float eps, bool f16,
+                            cudaStream_t stream);
+// out = relu(acc)^2 as 16-bit (n elements, n % 4 == 0).
+nc_status relu2_finish_launch(const float* acc, uint16_t* out, int64_t n, bool f16, cudaStream_t stream);
 
 nc_status rmsnorm_launch(const float* x, uint16_t* out, int M, int C, float eps, bool f16,
                          cudaStream_t stream);
