@@ -9,12 +9,13 @@
 // order, so q . k is unchanged.
 //
 // Decode attention is bound by reading the cached K/V.  Grid (split, kv head,
-// row): each CTA takes a contiguous chunk of the visible keys [lo, pos] for all
-// query heads of one kv group (GQA: the group's heads share every K/V row the
-// CTA reads), four warps stride over the chunk, and every lane holds D/32
-// dimensions, so a warp reads whole 256-byte K and V rows, four keys at a time.  Softmax is the
-// exact online form in fp32 (log2 domain).  Each CTA leaves (m, l, o) per head;
-// a second kernel merges the splits.
+// row): each CTA takes a chunk of 64 (or more) consecutive visible keys of
+// [lo, pos] for all query heads of one kv group (GQA: the group's heads share
+// every K/V row the CTA reads).  It copies the chunk's K and V head slices into
+// shared memory with 16-byte asynchronous copies, all in flight at once, then
+// four warps stride over the keys with every lane holding D/32 dimensions.
+// Softmax is the exact online form in fp32 (log2 domain).  Each CTA leaves
+// (m, l, o) per head; a second kernel merges the splits.
 #include <cuda_runtime.h>
 
 #include <cstdint>
@@ -27,7 +28,6 @@ namespace {
 
 constexpr int kMaxSplits = 32;
 constexpr int kWarps = 4;
-constexpr int kUnroll = 4;  // keys a warp has in flight
 
 __device__ __forceinline__ float ex2(float x) {
   float y;
@@ -52,7 +52,10 @@ __global__ void __launch_bounds__(256) kv_append_kernel(const uint4* __restrict_
   cache[((int64_t)b * T_max + t) * width16 + c] = qkv[(int64_t)m * ldq16 + col16 + c];
 }
 
-// DW: dimensions per lane (D / 32); G: query heads per kv head.
+// DW: dimensions per lane (D / 32); G: query heads per kv head.  The CTA first
+// copies the K and V head slices of its chunk of keys (kChunk rows of D 16-bit
+// values each) into shared memory with 16-byte asynchronous copies, all in
+// flight at once, then computes from there.
 template <int DW, int G, bool F16>
 __global__ void __launch_bounds__(kWarps * 32) decode_attn_kernel(const uint16_t* __restrict__ q, int64_t ldq,
                                                                   const uint16_t* __restrict__ cache,
@@ -63,7 +66,22 @@ __global__ void __launch_bounds__(kWarps * 32) decode_attn_kernel(const uint16_t
   const int s = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int k_begin = lo + s * chunk;
-  const int k_end = min(k_begin + chunk, hi + 1);
+  const int n = min(k_begin + chunk, hi + 1) - k_begin;  // keys of this CTA (<= kChunk)
+
+  extern __shared__ __align__(16) uint16_t kv_s[];  // [n][2][D]: k then v of each key
+  {
+    constexpr int PARTS = 2 * D / 8;  // 16-byte pieces per key (k and v)
+    const int64_t row_stride = 2 * (int64_t)Hkv * D;
+    const uint16_t* base = cache + ((int64_t)b * T_max + k_begin) * row_stride;
+    for (int e = threadIdx.x; e < n * PARTS; e += kWarps * 32) {
+      const int r = e / PARTS, part = e - r * PARTS;
+      const int kv = part / (D / 8), off = (part % (D / 8)) * 8;
+      const uint16_t* src = base + r * row_stride + (int64_t)(kv * Hkv + g) * D + off;
+      const uint32_t dst = (uint32_t)__cvta_generic_to_shared(kv_s + (r * 2 + kv) * D + off);
+      asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+  }
 
   float qv[G][DW];
 #pragma unroll
@@ -84,20 +102,23 @@ __global__ void __launch_bounds__(kWarps * 32) decode_attn_kernel(const uint16_t
 #pragma unroll
     for (int d = 0; d < DW; ++d) o[i][d] = 0.0f;
   }
-  const int64_t row_stride = 2 * (int64_t)Hkv * D;  // one cached position
-  const uint16_t* kbase = cache + (int64_t)b * T_max * row_stride + (int64_t)g * D + lane * DW;
-  const uint16_t* vbase = kbase + (int64_t)Hkv * D;
-  for (int j0 = k_begin + warp; j0 < k_end; j0 += kUnroll * kWarps) {
-    // kUnroll keys per step, every row's loads issued before any is used
-    float kf[kUnroll][DW], vf[kUnroll][DW];
+  asm volatile("cp.async.wait_group 0;" ::: "memory");
+  __syncthreads();
+
+  // Keys in groups of four per warp: four independent dot-product reductions,
+  // then one max / rescale for the group, so the online softmax's dependency
+  // chain is per group rather than per key.
+  constexpr int U = 4;
+  for (int r0 = warp * U; r0 < n; r0 += kWarps * U) {
+    float kf[U][DW], vf[U][DW];
 #pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
-      const int ju = j0 + u * kWarps;
-      const int j = ju < k_end ? ju : j0;  // past the end: reload a valid row, unused
+    for (int u = 0; u < U; ++u) {
+      const int r = r0 + u < n ? r0 + u : r0;  // past the end: a valid row, masked below
+      const uint16_t* kr = kv_s + (r * 2) * D + lane * DW;
 #pragma unroll
       for (int d = 0; d < DW; d += 2) {
-        const float2 kk = Half<F16>::unpack2(*reinterpret_cast<const uint32_t*>(kbase + j * row_stride + d));
-        const float2 vv = Half<F16>::unpack2(*reinterpret_cast<const uint32_t*>(vbase + j * row_stride + d));
+        const float2 kk = Half<F16>::unpack2(*reinterpret_cast<const uint32_t*>(kr + d));
+        const float2 vv = Half<F16>::unpack2(*reinterpret_cast<const uint32_t*>(kr + D + d));
         kf[u][d] = kk.x;
         kf[u][d + 1] = kk.y;
         vf[u][d] = vv.x;
@@ -105,49 +126,69 @@ __global__ void __launch_bounds__(kWarps * 32) decode_attn_kernel(const uint16_t
       }
     }
 #pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
-      if (j0 + u * kWarps >= k_end) break;  // warp-uniform
+    for (int i = 0; i < G; ++i) {
+      float sc[U];
 #pragma unroll
-      for (int i = 0; i < G; ++i) {
+      for (int u = 0; u < U; ++u) {
         float dot = 0.0f;
 #pragma unroll
         for (int d = 0; d < DW; ++d) dot = fmaf(qv[i][d], kf[u][d], dot);
-        const float sc = warp_allsum(dot) * scale_log2;
-        const float mn = fmaxf(m[i], sc);
-        const float a = ex2(m[i] - mn);  // 0 on the first key (m = -inf)
-        const float p = ex2(sc - mn);
-        l[i] = fmaf(l[i], a, p);
-#pragma unroll
-        for (int d = 0; d < DW; ++d) o[i][d] = fmaf(o[i][d], a, p * vf[u][d]);
-        m[i] = mn;
+        sc[u] = dot;
       }
+#pragma unroll
+      for (int o2 = 16; o2 > 0; o2 >>= 1)
+#pragma unroll
+        for (int u = 0; u < U; ++u) sc[u] += __shfl_xor_sync(0xffffffffu, sc[u], o2);
+      float mx = m[i];
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        sc[u] = r0 + u < n ? sc[u] * scale_log2 : -INFINITY;
+        mx = fmaxf(mx, sc[u]);
+      }
+      const float a = ex2(m[i] - mx);  // 0 on the first group (m = -inf)
+      float ps = 0.0f, pv[DW];
+#pragma unroll
+      for (int d = 0; d < DW; ++d) pv[d] = 0.0f;
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const float p = ex2(sc[u] - mx);  // 0 for the masked tail
+        ps += p;
+#pragma unroll
+        for (int d = 0; d < DW; ++d) pv[d] = fmaf(p, vf[u][d], pv[d]);
+      }
+      l[i] = fmaf(l[i], a, ps);
+#pragma unroll
+      for (int d = 0; d < DW; ++d) o[i][d] = fmaf(o[i][d], a, pv[d]);
+      m[i] = mx;
     }
   }
-  // merge the four warps, then write this split's (m, l, o) per head
-  __shared__ float sm_ml[kWarps][G][2];
-  __shared__ float sm_o[kWarps][G][D];
+  // merge the four warps (reusing the K/V staging area), then write this
+  // split's (m, l, o) per head
+  __syncthreads();
+  float* sm_ml = reinterpret_cast<float*>(kv_s);          // [kWarps][G][2]
+  float* sm_o = sm_ml + kWarps * G * 2;                    // [kWarps][G][D]
 #pragma unroll
   for (int i = 0; i < G; ++i) {
     if (lane == 0) {
-      sm_ml[warp][i][0] = m[i];
-      sm_ml[warp][i][1] = l[i];
+      sm_ml[(warp * G + i) * 2] = m[i];
+      sm_ml[(warp * G + i) * 2 + 1] = l[i];
     }
 #pragma unroll
-    for (int d = 0; d < DW; ++d) sm_o[warp][i][lane * DW + d] = o[i][d];
+    for (int d = 0; d < DW; ++d) sm_o[(warp * G + i) * D + lane * DW + d] = o[i][d];
   }
   __syncthreads();
   for (int e = threadIdx.x; e < G * D; e += kWarps * 32) {
     const int i = e / D, d = e - i * D;
     float mm = -INFINITY;
 #pragma unroll
-    for (int w = 0; w < kWarps; ++w) mm = fmaxf(mm, sm_ml[w][i][0]);
+    for (int w = 0; w < kWarps; ++w) mm = fmaxf(mm, sm_ml[(w * G + i) * 2]);
     float ll = 0.0f, oo = 0.0f;
 #pragma unroll
     for (int w = 0; w < kWarps; ++w) {
-      const float mw = sm_ml[w][i][0];
+      const float mw = sm_ml[(w * G + i) * 2];
       const float f = mw == -INFINITY ? 0.0f : ex2(mw - mm);
-      ll = fmaf(sm_ml[w][i][1], f, ll);
-      oo = fmaf(sm_o[w][i][d], f, oo);
+      ll = fmaf(sm_ml[(w * G + i) * 2 + 1], f, ll);
+      oo = fmaf(sm_o[(w * G + i) * D + d], f, oo);
     }
     float* dst = partial + (((int64_t)b * H + g * G + i) * kMaxSplits + s) * (2 + D);
     if (d == 0) {
@@ -165,14 +206,30 @@ __global__ void decode_combine_kernel(const float* __restrict__ partial, uint16_
   const int bh = blockIdx.x;
   const int d = threadIdx.x;
   const float* p = partial + (int64_t)bh * kMaxSplits * (2 + D);
+  // every split's (m, l, o[d]) read up front: independent loads, one round trip
+  float ms[kMaxSplits], ls[kMaxSplits], os[kMaxSplits];
+#pragma unroll
+  for (int s = 0; s < kMaxSplits; ++s) {
+    if (s < splits) {
+      const float* q = p + s * (2 + D);
+      ms[s] = q[0];
+      ls[s] = q[1];
+      os[s] = q[2 + d];
+    } else {
+      ms[s] = -INFINITY;
+      ls[s] = 0.0f;
+      os[s] = 0.0f;
+    }
+  }
   float mm = -INFINITY;
-  for (int s = 0; s < splits; ++s) mm = fmaxf(mm, p[s * (2 + D)]);
+#pragma unroll
+  for (int s = 0; s < kMaxSplits; ++s) mm = fmaxf(mm, ms[s]);
   float ll = 0.0f, oo = 0.0f;
-  for (int s = 0; s < splits; ++s) {
-    const float* q = p + s * (2 + D);
-    const float f = q[0] == -INFINITY ? 0.0f : ex2(q[0] - mm);
-    ll = fmaf(q[1], f, ll);
-    oo = fmaf(q[2 + d], f, oo);
+#pragma unroll
+  for (int s = 0; s < kMaxSplits; ++s) {
+    const float f = ms[s] == -INFINITY ? 0.0f : ex2(ms[s] - mm);
+    ll = fmaf(ls[s], f, ll);
+    oo = fmaf(os[s], f, oo);
   }
   const float v = ll > 0.0f ? oo / ll : 0.0f;
   const float v1 = __shfl_down_sync(0xffffffffu, v, 1);  // blockDim = D, a multiple of 32
@@ -254,21 +311,42 @@ nc_status decode_dispatch(const uint16_t* q, int64_t ldq, const uint16_t* cache,
                           int Hkv, int T_max, int lo, int hi, int splits, int chunk, float scale_log2,
                           cudaStream_t stream) {
   const dim3 grid(splits, Hkv, B);
+  constexpr int D = DW * 32;
+  // staging of the chunk's K/V rows, reused for the warps' merge
+  const int G = H / Hkv;
+  const size_t stage = (size_t)chunk * 2 * D * 2, merge = (size_t)kWarps * G * (2 + D) * 4;
+  const size_t smem = stage > merge ? stage : merge;
   switch (H / Hkv) {
     case 1:
-      decode_attn_kernel<DW, 1, F16><<<grid, kWarps * 32, 0, stream>>>(q, ldq, cache, partial, H, Hkv, T_max, lo,
+      if (smem > 48 * 1024 &&
+          cudaFuncSetAttribute(decode_attn_kernel<DW, 1, F16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)smem) != cudaSuccess)
+        return NC_ERR_CUDA;
+      decode_attn_kernel<DW, 1, F16><<<grid, kWarps * 32, smem, stream>>>(q, ldq, cache, partial, H, Hkv, T_max, lo,
                                                                        hi, chunk, scale_log2);
       break;
     case 2:
-      decode_attn_kernel<DW, 2, F16><<<grid, kWarps * 32, 0, stream>>>(q, ldq, cache, partial, H, Hkv, T_max, lo,
+      if (smem > 48 * 1024 &&
+          cudaFuncSetAttribute(decode_attn_kernel<DW, 2, F16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)smem) != cudaSuccess)
+        return NC_ERR_CUDA;
+      decode_attn_kernel<DW, 2, F16><<<grid, kWarps * 32, smem, stream>>>(q, ldq, cache, partial, H, Hkv, T_max, lo,
                                                                        hi, chunk, scale_log2);
       break;
     case 4:
-      decode_attn_kernel<DW, 4, F16><<<grid, kWarps * 32, 0, stream>>>(q, ldq, cache, partial, H, Hkv, T_max, lo,
+      if (smem > 48 * 1024 &&
+          cudaFuncSetAttribute(decode_attn_kernel<DW, 4, F16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)smem) != cudaSuccess)
+        return NC_ERR_CUDA;
+      decode_attn_kernel<DW, 4, F16><<<grid, kWarps * 32, smem, stream>>>(q, ldq, cache, partial, H, Hkv, T_max, lo,
                                                                        hi, chunk, scale_log2);
       break;
     case 8:
-      decode_attn_kernel<DW, 8, F16><<<grid, kWarps * 32, 0, stream>>>(q, ldq, cache, partial, H, Hkv, T_max, lo,
+      if (smem > 48 * 1024 &&
+          cudaFuncSetAttribute(decode_attn_kernel<DW, 8, F16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)smem) != cudaSuccess)
+        return NC_ERR_CUDA;
+      decode_attn_kernel<DW, 8, F16><<<grid, kWarps * 32, smem, stream>>>(q, ldq, cache, partial, H, Hkv, T_max, lo,
                                                                        hi, chunk, scale_log2);
       break;
     default:
@@ -332,12 +410,12 @@ nc_status decode_attention_launch(const uint16_t* q, int64_t ldq, const uint16_t
   if ((D != 64 && D != 128) || H % Hkv != 0) return NC_ERR_SHAPE;
   const int lo = pos - W + 1 > 0 ? pos - W + 1 : 0;
   const int n_keys = pos - lo + 1;
-  // enough CTAs to keep every SM streaming K/V: about 16 per SM
-  int splits = (16 * device_sm_count() + B * Hkv - 1) / (B * Hkv);
-  splits = splits < 1 ? 1 : (splits > kMaxSplits ? kMaxSplits : splits);
-  int chunk = (n_keys + splits - 1) / splits;
-  chunk = chunk < 16 ? 16 : chunk;
-  splits = (n_keys + chunk - 1) / chunk;
+  // chunks of 64 keys (32 KB of K/V staging at D = 128), more when the window
+  // needs more than kMaxSplits of them
+  int chunk = (n_keys + kMaxSplits - 1) / kMaxSplits;
+  chunk = chunk < 64 ? 64 : (chunk + 15) / 16 * 16;
+  const int splits = (n_keys + chunk - 1) / chunk;
+  if ((size_t)chunk * 2 * D * 2 > 200 * 1024) return NC_ERR_SHAPE;  // T_max beyond the staging
   const float scale_log2 = 1.4426950408889634f / sqrtf((float)D);
   nc_status s;
   if (D == 128)
