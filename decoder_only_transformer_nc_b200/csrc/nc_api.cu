@@ -493,22 +493,12 @@ static nc_status forward_impl(const nc_config* cfg, const nc_weights* w, const i
   if (!config_ok(cfg)) return NC_ERR_CONFIG;
   if (B < 1 || T < 1 || T > cfg->seq_len) return NC_ERR_SHAPE;
   if ((token_loss || loss) && !targets) return NC_ERR_INVALID_ARG;
-  if (!w->wte || !w->lm_head || !w->c_q || !w->c_k || !w->c_v || !w->attn_proj || !w->c_fc ||
-      !w->mlp_proj)
-    return NC_ERR_INVALID_ARG;
   if ((int64_t)B * T > (int64_t)1 << 30) return NC_ERR_SHAPE;
   const WsLayout L = ws_layout(cfg, B, T, sess == nullptr);
   if (ws_bytes < L.total) return NC_ERR_WORKSPACE;
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return NC_ERR_ALIGNMENT;
-  if (!aligned16(w->wte) || !aligned16(w->lm_head) || (logits && !aligned16(logits)))
-    return NC_ERR_ALIGNMENT;
-  for (int l = 0; l < cfg->n_layer; ++l) {
-    const float* ps[6] = {w->c_q[l], w->c_k[l], w->c_v[l], w->attn_proj[l], w->c_fc[l], w->mlp_proj[l]};
-    for (const float* p : ps) {
-      if (!p) return NC_ERR_INVALID_ARG;
-      if (!aligned16(p)) return NC_ERR_ALIGNMENT;
-    }
-  }
+  if (logits && !aligned16(logits)) return NC_ERR_ALIGNMENT;
+  if (nc_status s = check_weights(cfg, w)) return s;
   const uint32_t ex = cfg->extras;
   if (ex & NC_EXTRA_SMEAR) {
     if (!w->smear_gate) return NC_ERR_INVALID_ARG;
