@@ -60,6 +60,14 @@ one-line descriptions there:
 
 Those pins live in ``tests/test_oracle_extras.py``.
 
+FP8 ("Nanochat与nanoGPT对比" §1 table, FP8-training row: dynamic tensor-level
+e4m3/e5m2): ``forward(..., fp8="block" | "all")`` runs the block projections
+(and with "all" the LM head) through dynamic tensorwise e4m3; the readings are
+in ``oracle/fp8.py`` and its pins in ``tests/test_oracle_fp8.py``.  With
+tensorwise scales the scale of an activation depends on every row and
+position of the batch, so the fp8 forward is causal and row-independent only
+up to that shared scale.
+
 Parity pins live in ``tests/test_oracle_pins.py``.  Every function below is
 pinned there by closed forms, invariants, brute force or an independent library
 routine.  The composition of the full forward at random weights is pinned only
@@ -88,3 +96,4 @@ from .model import (  # noqa: F401
     value_embed_layers,
     backout_layer,
 )
+from .fp8 import round_e4m3, quantize_e4m3, linear_e4m3, tensor_scale  # noqa: F401,E402

@@ -14,6 +14,8 @@ from dataclasses import dataclass, field
 
 import numpy as np
 
+from .fp8 import linear_e4m3
+
 F64 = np.float64
 
 
@@ -155,11 +157,13 @@ def attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, W: int,
     return out
 
 
-def relu2_mlp(a: np.ndarray, w_fc: np.ndarray, w_proj: np.ndarray) -> np.ndarray:
-    """"从文本到聊天模型" §5.7: c_fc (C -> 4C), relu(x)^2, c_proj (4C -> C)."""
-    h = linear(a, w_fc)
+def relu2_mlp(a: np.ndarray, w_fc: np.ndarray, w_proj: np.ndarray, lin=None) -> np.ndarray:
+    """"从文本到聊天模型" §5.7: c_fc (C -> 4C), relu(x)^2, c_proj (4C -> C).
+    ``lin`` is the linear map to use (``linear`` unless given)."""
+    lin = lin or linear
+    h = lin(a, w_fc)
     h = np.maximum(h, 0.0) ** 2
-    return linear(h, w_proj)
+    return lin(h, w_proj)
 
 
 def softcap(z: np.ndarray, cap: float) -> np.ndarray:
@@ -248,7 +252,7 @@ def smear(x: np.ndarray, gate_w: np.ndarray) -> np.ndarray:
 
 
 def forward(cfg: OracleConfig, weights: dict, idx: np.ndarray, targets=None,
-            want_logits: bool = True, extras: dict = None):
+            want_logits: bool = True, extras: dict = None, fp8: str = None):
     """The whole forward for the rows of ``idx`` ([B, T] int).
 
     Steps in the order of "从文本到聊天模型" §5 (embedding, blocks of
@@ -270,10 +274,18 @@ def forward(cfg: OracleConfig, weights: dict, idx: np.ndarray, targets=None,
     * ``backout_lambda`` (scalar): x_mid = the stream after the first
       ``backout_layer`` blocks; before the final norm x = x - lambda * x_mid.
 
+    ``fp8`` (optional, "Nanochat与nanoGPT对比" §1, FP8-training row): "block"
+    sends the six block projections through ``fp8.linear_e4m3`` (dynamic
+    tensorwise e4m3 of both operands), "all" the LM head as well.
+
     Returns a dict with ``logits`` ([B,T,V] capped, fp64, if ``want_logits``),
     ``token_loss`` ([B,T]) and ``loss`` (scalar) when targets are given.
     """
     ex = extras or {}
+    if fp8 not in (None, "block", "all"):
+        raise ValueError(f"fp8 must be None, 'block' or 'all', not {fp8!r}")
+    blin = linear_e4m3 if fp8 else linear
+    hlin = linear_e4m3 if fp8 == "all" else linear
     idx = np.asarray(idx)
     B, T = idx.shape
     C, H, Hkv, D = cfg.d_model, cfg.n_head, cfg.n_kv_head, cfg.head_dim
@@ -292,22 +304,22 @@ def forward(cfg: OracleConfig, weights: dict, idx: np.ndarray, targets=None,
         if "resid_lambdas" in ex:
             x = F64(ex["resid_lambdas"][l]) * x + F64(ex["x0_lambdas"][l]) * x0
         a = rms_norm(x, eps)
-        q = linear(a, lw["c_q"]).reshape(B, T, H, D)
-        k = linear(a, lw["c_k"]).reshape(B, T, Hkv, D)
-        v = linear(a, lw["c_v"]).reshape(B, T, Hkv, D)
+        q = blin(a, lw["c_q"]).reshape(B, T, H, D)
+        k = blin(a, lw["c_k"]).reshape(B, T, Hkv, D)
+        v = blin(a, lw["c_v"]).reshape(B, T, Hkv, D)
         if "value_embeds" in ex and value_embed_layers(L)[l]:
             ve = embed(ex["value_embeds"][l], idx).reshape(B, T, Hkv, D)
             v = v + np.asarray(ex["ve_gates"][l], dtype=F64)[None, None, :, None] * ve
         q = rms_norm(rope(q, cos, sin), eps)
         k = rms_norm(rope(k, cos, sin), eps)
         o = attention(q, k, v, windows[l])
-        x = x + linear(o.reshape(B, T, H * D), lw["attn_proj"])
+        x = x + blin(o.reshape(B, T, H * D), lw["attn_proj"])
         a = rms_norm(x, eps)
-        x = x + relu2_mlp(a, lw["c_fc"], lw["mlp_proj"])
+        x = x + relu2_mlp(a, lw["c_fc"], lw["mlp_proj"], lin=blin)
     if x_mid is not None:
         x = x - F64(ex["backout_lambda"]) * x_mid
     a = rms_norm(x, eps)
-    logits = softcap(linear(a, weights["lm_head"]), cfg.softcap)  # [B,T,V]
+    logits = softcap(hlin(a, weights["lm_head"]), cfg.softcap)  # [B,T,V]
     res = {}
     if want_logits:
         res["logits"] = logits
