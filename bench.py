@@ -42,6 +42,9 @@ UNIT = "tokens/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 DTYPE_NOTE = ("f16 tensor-core operands (weights rounded fp32->bf16 as the method casts them, "
               "held exactly in f16; activations f16), fp32 accumulation, fp32 residual/softmax/loss")
+DTYPE_NOTE_FP8 = ("e4m3 tensor-core operands with dynamic tensorwise scales for the {what} "
+                  "(activations quantised from f16, weights from fp32), fp32 accumulation; other products "
+                  "f16; fp32 residual/softmax/loss")
 GEMM_KINDS = ("gemm_qkv", "gemm_attn_proj", "gemm_fc", "gemm_mlp_proj", "gemm_lm_head")
 ROOFLINE_KIND = "gemm_fc"  # the kind with the largest share of the step
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one c_fc launch of
@@ -83,7 +86,32 @@ def kernel_work(s, kind):
         L = s.n_layer
         n = L * (C * (H + 2 * Hkv) * D + C * H * D + 8 * C * C) + V * C
         return n * 6.0
+    if kind == "fp8_quant":  # 16-bit read + e4m3 write (amax folded into the producer), mean of a layer's 4
+        return 3.0 * M * (6 * C + H * D) / 4
     return 0.0
+
+
+def kernels_per_step(n_entries, L, fp8_bits, extras_bits):
+    """CUDA kernels one forward launches.  The trace has one entry per step of
+    the path.  An activation quantisation is one kernel when its producer
+    folded the amax in (norms, attention, the relu^2 epilogue), two when a norm
+    that mixes in the residual-stream terms produced it.  The weight pass is
+    one cast launch, or two launches per batch of up to 112 e4m3 weight tensors
+    plus a cast launch for what stays 16-bit."""
+    n = n_entries
+    if fp8_bits:
+        unfused = 0
+        if fp8_bits & 1:
+            if extras_bits & 4:
+                unfused += L  # every first norm mixes in x0
+            elif extras_bits & 8:
+                unfused += 1  # the norm that keeps x_mid
+        if (fp8_bits & 2) and (extras_bits & 8):
+            unfused += 1  # the final norm subtracts x_mid
+        nq = (6 * L if fp8_bits & 1 else 0) + (1 if fp8_bits & 2 else 0)
+        cast_kernels = 2 * ((nq + 111) // 112) + (0 if (fp8_bits & 1 and fp8_bits & 2) else 1)
+        n += unfused + cast_kernels - 1
+    return n
 
 
 class ClockSampler:
@@ -155,7 +183,7 @@ def blas_threads():
     return len(os.sched_getaffinity(0))
 
 
-def oracle_sample(s, prefix, seed=TOKEN_SEED, weights=None, extras=None):
+def oracle_sample(s, prefix, seed=TOKEN_SEED, weights=None, extras=None, fp8=None):
     """Runs the fp64 oracle on batch row 0, first `prefix` positions (with the
     full-nanochat terms when `extras` is given); returns (tokens processed,
     seconds)."""
@@ -165,7 +193,7 @@ def oracle_sample(s, prefix, seed=TOKEN_SEED, weights=None, extras=None):
     cfg = oracle.OracleConfig(s.n_layer, s.d_model, s.n_head, s.n_kv_head, s.head_dim, s.seq_len,
                               s.vocab, short_window=s.short_window)
     t0 = time.perf_counter()
-    oracle.forward(cfg, w, x[:1, :prefix], y[:1, :prefix], want_logits=False, extras=extras)
+    oracle.forward(cfg, w, x[:1, :prefix], y[:1, :prefix], want_logits=False, extras=extras, fp8=fp8)
     return prefix, time.perf_counter() - t0
 
 
@@ -186,9 +214,10 @@ def run_reference(args, s):
     prefix = args.ref_prefix
     w = make_weights(s)
     ex = _extras_for(s) if args.extras == "all" else None
+    f8 = None if args.fp8 == "none" else args.fp8
     for _ in range(args.warmup):
-        oracle_sample(s, prefix, weights=w, extras=ex)
-    times = [oracle_sample(s, prefix, weights=w, extras=ex)[1] for _ in range(args.steps)]
+        oracle_sample(s, prefix, weights=w, extras=ex, fp8=f8)
+    times = [oracle_sample(s, prefix, weights=w, extras=ex, fp8=f8)[1] for _ in range(args.steps)]
     sec = sum(times) / len(times)
     value = prefix / sec
     sample = f"{s.name} batch row 0, first {prefix} positions, forward+loss per step"
@@ -196,7 +225,9 @@ def run_reference(args, s):
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": s.name + ("+extras" if ex else ""), "global_batch": 1, "seq_len": prefix,
+        "config": {"workload": s.name + ("+extras" if ex else "") + ({None: "", "block": "+fp8block",
+                                                                       "all": "+fp8"}[f8]),
+                   "global_batch": 1, "seq_len": prefix,
                    "parallelism": "none"},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
                          "sample": sample},
@@ -224,8 +255,9 @@ def run_ours(args, s):
         dist.init_process_group("nccl", device_id=dev, timeout=timedelta(seconds=120))
 
     bits = nc.EXTRA_ALL if args.extras == "all" else 0
+    fp8_bits = {"none": 0, "block": nc.FP8_BLOCK, "all": nc.FP8_ALL}[args.fp8]
     cfg = nc.make_config(s.n_layer, s.d_model, s.n_head, s.n_kv_head, s.head_dim, s.seq_len, s.vocab,
-                         s.short_window, extras=bits)
+                         s.short_window, extras=bits, fp8=fp8_bits)
     weights = make_weights(s)
     extras = _extras_for(s, nc) if bits else None
     model = nc.Model.from_numpy(cfg, weights, device=dev, extras=extras)
@@ -332,6 +364,9 @@ def run_ours(args, s):
     gemm_flops = sum(kernel_work(s, k) * per_kind[k][1] for k in GEMM_KINDS if k in per_kind)
     achieved = gemm_flops / (gemm_ms / 1e3) / 1e12 if gemm_ms > 0 else 0.0
     peak = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+    peak16 = peak
+    if fp8_bits:  # e4m3 products: the measured bf16 peak x the nominal e4m3/bf16 ratio 4.5 / 2.25
+        peak = 2.0 * peak
     total_traced = sum(v[0] for v in per_kind.values())
     attn_flops_step = flops - sum(kernel_work(s, g) * per_kind[g][1] / args.steps
                                   for g in GEMM_KINDS if g in per_kind)
@@ -340,6 +375,8 @@ def run_ours(args, s):
         ent = {"launches": n, "ms_total": round(kms, 3), "share": round(kms / total_traced, 4)}
         if k.startswith("gemm"):
             ent["tflops"] = round(kernel_work(s, k) * n / (kms / 1e3) / 1e12, 1)
+            if fp8_bits and (k != "gemm_lm_head" or fp8_bits & 2):
+                ent["precision"] = "e4m3"
         elif k == "attention":
             ent["tflops"] = round(attn_flops_step * args.steps / (kms / 1e3) / 1e12, 1)
         elif kernel_work(s, k) > 0:
@@ -353,31 +390,39 @@ def run_ours(args, s):
         result = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": DTYPE_NOTE, "data": "synthetic",
-            "config": {"workload": s.name + ("+extras" if bits else ""), "global_batch": world * B, "seq_len": T,
+            "vs_baseline": None,
+            "dtype": DTYPE_NOTE if not fp8_bits else DTYPE_NOTE_FP8.format(
+                what="six block projections" + (" and the LM head" if fp8_bits & 2 else "")),
+            "data": "synthetic",
+            "config": {"workload": s.name + ("+extras" if bits else "") + ({0: "", 1: "+fp8block", 3: "+fp8"}[fp8_bits]),
+                       "global_batch": world * B, "seq_len": T,
                        "parallelism": f"dp{world}" if world > 1 else "none",
                        "layers": s.n_layer, "d_model": s.d_model,
                        "l2": "inputs larger than L2 (fp32 weights %.2f GB, residual stream %.2f GB per step)"
                              % (4 * sum(a.size for a in _flat(weights)) / 1e9, 4 * B * T * s.d_model / 1e9)},
             "tflops": round(tflops, 1),
             "pct_of_bf16_peak": {"measured_burst": round(100 * tflops / world / burst, 2),
-                                 "measured_sustained": round(100 * tflops / world / peak, 2),
+                                 "measured_sustained": round(100 * tflops / world / peak16, 2),
                                  "datasheet_dense_2250": round(100 * tflops / world / 2250.0, 2),
                                  "source": peak_src},
             "roofline": {"kernel": "gemm_kernel<EPI_RELU2_16> (c_fc + ReLU^2: M=B*T, N=4C, K=C)",
                          "bound": "tensor", "achieved": round(rk_achieved, 1),
                          "peak": peak,
-                         "peak_kind": f"bf16_tflops_sustained ({peak_src}); f16 operands, same nominal rate",
+                         "peak_kind": (f"bf16_tflops_sustained ({peak_src}); f16 operands, same nominal rate"
+                                       if not fp8_bits else
+                                       f"2 x bf16_tflops_sustained ({peak_src}): e4m3 operands, nominal "
+                                       "e4m3/bf16 dense ratio 4.5/2.25"),
                          "unit": "TFLOP/s", "frac": round(rk_achieved / peak, 4),
-                         "traffic": FC_TRAFFIC.get((s.name, B, T)),
-                         "algorithmic_bytes": 2 * (B * T * s.d_model + 4 * s.d_model * s.d_model
-                                                   + 4 * B * T * s.d_model),
+                         "traffic": None if fp8_bits else FC_TRAFFIC.get((s.name, B, T)),
+                         "algorithmic_bytes": (1 if fp8_bits else 2) * (B * T * s.d_model
+                                                                         + 4 * s.d_model * s.d_model)
+                                              + 2 * 4 * B * T * s.d_model,
                          "launches": rk_n, "avg_launch_ms": round(rk_ms / max(1, rk_n), 4)},
             "gemm_family": {"kernel": "gemm_kernel, all projections (qkv, attn c_proj, c_fc, mlp c_proj, lm_head)",
                             "achieved": round(achieved, 1), "frac": round(achieved / peak, 4),
                             "launches": gemm_launches},
             "kernels": kernels,
-            "gpu_launches": n_launch * args.steps,
+            "gpu_launches": kernels_per_step(n_launch, s.n_layer, fp8_bits, bits) * args.steps,
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": int(x.nbytes + y.nbytes),
                     "d2h_bytes_per_step": 4},
             "clocks": clk,
@@ -390,7 +435,8 @@ def run_ours(args, s):
         if world == 1 and not args.no_cpu_baseline:
             del model, ws
             torch.cuda.empty_cache()
-            n_tok, sec = oracle_sample(s, args.cpu_prefix, weights=weights, extras=extras)
+            fp8_mode = {0: None, 1: "block", 3: "all"}[fp8_bits]
+            n_tok, sec = oracle_sample(s, args.cpu_prefix, weights=weights, extras=extras, fp8=fp8_mode)
             result["cpu_baseline"] = {
                 "value": n_tok / sec, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
                 "sample": f"{s.name} batch row 0, first {args.cpu_prefix} positions, fp64 forward+loss "
@@ -534,6 +580,9 @@ def main():
     ap.add_argument("--mode", default="forward", choices=["forward", "decode"],
                     help="decode: KV-cache decode steps after a prefill of --prompt tokens")
     ap.add_argument("--prompt", type=int, default=1024, help="decode mode: prompt length")
+    ap.add_argument("--fp8", default="none", choices=["none", "block", "all"],
+                    help="forward mode: dynamic tensorwise e4m3 for the block projections "
+                         "('block') or for them and the LM head ('all')")
     ap.add_argument("--extras", default="none", choices=["none", "all"],
                     help="all: also run the full nanochat terms (smear, value embeddings, "
                          "residual lambdas + x0, backout)")

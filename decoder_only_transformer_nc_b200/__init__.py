@@ -18,7 +18,8 @@ __all__ = [
     "NcError", "NcConfig", "lib", "init_config", "make_config", "check_config", "layer_window",
     "workspace_bytes", "forward_flops", "Model", "forward", "LaunchTrace", "KERNEL_KINDS", "get_status", "cast_bf16", "embedding",
     "rmsnorm", "rope_table", "rope_qknorm", "attention", "linear", "qkv_rope", "softcap_ce",
-    "loss_mean", "cast_weights", "selftest_bounded_wait", "BF16", "F16",
+    "loss_mean", "cast_weights", "selftest_bounded_wait", "BF16", "F16", "F32",
+    "fp8_quantize", "linear_fp8", "FP8_BLOCK", "FP8_LM_HEAD", "FP8_ALL",
     "EPI_STORE_16", "EPI_RELU2_16", "EPI_RESID_F32", "EPI_STORE_F32", "EPI_SOFTCAP_F32",
 ]
 
@@ -26,7 +27,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libnc.so")
 
 EPI_STORE_16, EPI_RELU2_16, EPI_RESID_F32, EPI_STORE_F32, EPI_SOFTCAP_F32 = range(5)
-BF16, F16 = 0, 1  # nc_dtype
+BF16, F16, F32 = 0, 1, 2  # nc_dtype (F32: fp8_quantize sources only)
 DEV_TOKEN_RANGE, DEV_TARGET_RANGE, DEV_TIMEOUT = 0x1, 0x2, 0x4
 
 STATUS_NAMES = {0: "NC_OK", 1: "NC_ERR_INVALID_ARG", 2: "NC_ERR_CONFIG", 3: "NC_ERR_SHAPE",
@@ -46,7 +47,7 @@ class NcConfig(ctypes.Structure):
                 ("seq_len", ctypes.c_int32), ("short_window", ctypes.c_int32),
                 ("window_pattern", ctypes.c_char * 8), ("softcap", ctypes.c_float),
                 ("norm_eps", ctypes.c_float), ("rope_base", ctypes.c_float), ("act_dtype", ctypes.c_int32),
-                ("extras", ctypes.c_uint32)]
+                ("extras", ctypes.c_uint32), ("fp8", ctypes.c_uint32)]
 
     def __repr__(self):
         return ("NcConfig(n_layer=%d, d_model=%d, n_head=%d, n_kv_head=%d, head_dim=%d, vocab=%d, "
@@ -70,6 +71,10 @@ class NcWeights(ctypes.Structure):
 EXTRA_SMEAR, EXTRA_VALUE_EMBED, EXTRA_RESID_LAMBDAS, EXTRA_BACKOUT = 1, 2, 4, 8
 EXTRA_ALL = 15
 
+# Dynamic tensorwise e4m3 products (bits of NcConfig.fp8): the six block
+# projections, the LM head.
+FP8_BLOCK, FP8_LM_HEAD, FP8_ALL = 1, 2, 3
+
 
 class NcTrace(ctypes.Structure):
     _fields_ = [("events", ctypes.POINTER(ctypes.c_void_p)), ("capacity", ctypes.c_int32),
@@ -77,7 +82,8 @@ class NcTrace(ctypes.Structure):
 
 
 KERNEL_KINDS = ("rope_table", "cast", "embedding", "rmsnorm", "gemm_qkv", "rope_qknorm", "attention",
-                "gemm_attn_proj", "gemm_fc", "gemm_mlp_proj", "gemm_lm_head", "ce_finalize", "loss_mean")
+                "gemm_attn_proj", "gemm_fc", "gemm_mlp_proj", "gemm_lm_head", "ce_finalize", "loss_mean",
+                "fp8_quant")
 
 _lib = None
 
@@ -116,6 +122,8 @@ def lib():
             "nc_attention": (i32, [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, vp]),
             "nc_attention_strided": (i32, [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i64, i64, i32, vp]),
             "nc_linear": (i32, [vp, vp, vp, i32, i32, i32, i64, i32, f32, i32, vp, vp]),
+            "nc_fp8_quantize": (i32, [vp, i32, i64, vp, vp, vp]),
+            "nc_linear_fp8": (i32, [vp, vp, vp, vp, vp, i32, i32, i32, i64, i32, f32, i32, vp, vp]),
             "nc_qkv_rope": (i32, [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, f32, i32, vp, vp]),
             "nc_softcap_ce": (i32, [vp, vp, vp, vp, i32, i32, f32, vp, vp]),
             "nc_loss_mean": (i32, [vp, vp, i32, i32, vp, vp]),
@@ -160,10 +168,10 @@ def init_config(depth: int, aspect_ratio: int = 64, head_dim: int = 128, n_kv_he
 
 def make_config(n_layer, d_model, n_head, n_kv_head, head_dim, seq_len, vocab, short_window=0,
                 window_pattern="SSSL", softcap=15.0, norm_eps=1e-6, rope_base=10000.0,
-                act_dtype=F16, extras=0) -> NcConfig:
+                act_dtype=F16, extras=0, fp8=0) -> NcConfig:
     c = NcConfig(n_layer, d_model, n_head, n_kv_head, head_dim, vocab, seq_len,
                  short_window if short_window > 0 else seq_len // 4, window_pattern.encode(),
-                 softcap, norm_eps, rope_base, act_dtype, extras)
+                 softcap, norm_eps, rope_base, act_dtype, extras, fp8)
     _check(lib().nc_check_config(ctypes.byref(c)), "nc_check_config")
     return c
 
@@ -437,6 +445,24 @@ def linear(a, w, out, epilogue, cap=15.0, status=None, stream=None):
     N = w.shape[0]
     _check(lib().nc_linear(_ptr(a), _ptr(w), _ptr(out), M, N, K, out.stride(0), epilogue, cap, _dt(a),
                            _ptr(status), _stream(stream)), "nc_linear")
+
+
+def fp8_quantize(x, codes, amax, stream=None):
+    """Dynamic tensorwise e4m3 codes of x (fp32, bf16 or fp16 device tensor)
+    into codes (uint8, same element count); amax: one-element fp32 tensor."""
+    import torch
+    dt = {torch.float32: F32, torch.bfloat16: BF16, torch.float16: F16}[x.dtype]
+    _check(lib().nc_fp8_quantize(_ptr(x), dt, x.numel(), _ptr(codes), _ptr(amax), _stream(stream)),
+           "nc_fp8_quantize")
+
+
+def linear_fp8(a8, amax_a, w8, amax_w, out, epilogue, cap=15.0, dtype=F16, status=None, stream=None):
+    """out = epilogue((a8 @ w8^T) / (s_a s_w)) on e4m3 codes (uint8 tensors)."""
+    M, K = a8.shape
+    N = w8.shape[0]
+    _check(lib().nc_linear_fp8(_ptr(a8), _ptr(amax_a), _ptr(w8), _ptr(amax_w), _ptr(out), M, N, K,
+                               out.stride(0), epilogue, cap, dtype, _ptr(status), _stream(stream)),
+           "nc_linear_fp8")
 
 
 def qkv_rope(a, w, out, table, T, H, Hkv, D, eps=1e-6, status=None, stream=None):

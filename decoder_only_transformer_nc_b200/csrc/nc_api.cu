@@ -18,6 +18,7 @@
 // accumulation.
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -82,6 +83,7 @@ bool config_ok(const nc_config* c) {
   if (!(c->softcap > 0.0f) || !(c->norm_eps >= 0.0f) || !(c->rope_base > 1.0f)) return false;
   if (c->act_dtype != NC_F16 && c->act_dtype != NC_BF16) return false;
   if ((c->extras & ~NC_EXTRA_ALL) != 0) return false;
+  if ((c->fp8 & ~NC_FP8_ALL) != 0) return false;
   const size_t plen = strnlen(c->window_pattern, sizeof(c->window_pattern));
   if (plen == 0 || plen >= sizeof(c->window_pattern)) return false;
   for (size_t i = 0; i < plen; ++i)
@@ -91,9 +93,19 @@ bool config_ok(const nc_config* c) {
 
 // Workspace layout of nc_forward.  Offsets are 256-byte aligned.
 struct WsLayout {
-  size_t status, rope, wqkv, wo, wfc, wmp, wlm, x, a, qkv, o, h, part, tgt, tl, x0, xmid, total;
+  size_t status, rope, wqkv, wo, wfc, wmp, wlm, x, a, qkv, o, h, part, tgt, tl, x0, xmid, a8, amax, total;
   size_t wqkv_elems, wo_elems, wfc_elems, wmp_elems;  // per layer
 };
+
+// FP8 amax slots of a forward: per layer the weights c_q, c_k, c_v (adjacent:
+// the QKV product reads three), attention c_proj, c_fc, MLP c_proj, then the
+// LM head; after them per layer the activations entering the QKV, attention
+// c_proj, c_fc and MLP c_proj products, then the one entering the LM head.
+inline int amax_w_slot(int l, int which) { return 6 * l + which; }
+inline int amax_wlm_slot(int L) { return 6 * L; }
+inline int amax_a_slot(int L, int l, int which) { return 6 * L + 1 + 4 * l + which; }
+inline int amax_alm_slot(int L) { return 10 * L + 1; }
+inline int amax_slots(int L) { return 10 * L + 2; }
 
 WsLayout ws_layout(const nc_config* c, int B, int T, bool own_weights = true) {
   WsLayout L;
@@ -111,13 +123,15 @@ WsLayout ws_layout(const nc_config* c, int B, int T, bool own_weights = true) {
     return o;
   };
   L.status = take(256);
+  const size_t wb = (c->fp8 & NC_FP8_BLOCK) ? 1 : 2;    // bytes per block weight element
+  const size_t lb = (c->fp8 & NC_FP8_LM_HEAD) ? 1 : 2;  // ... per LM-head element
   if (own_weights) {  // else the 16-bit weights and the RoPE table live in a session
     L.rope = take((size_t)T * D * sizeof(float));
-    L.wqkv = take(c->n_layer * L.wqkv_elems * 2);
-    L.wo = take(c->n_layer * L.wo_elems * 2);
-    L.wfc = take(c->n_layer * L.wfc_elems * 2);
-    L.wmp = take(c->n_layer * L.wmp_elems * 2);
-    L.wlm = take(V * C * 2);
+    L.wqkv = take(c->n_layer * L.wqkv_elems * wb);
+    L.wo = take(c->n_layer * L.wo_elems * wb);
+    L.wfc = take(c->n_layer * L.wfc_elems * wb);
+    L.wmp = take(c->n_layer * L.wmp_elems * wb);
+    L.wlm = take(V * C * lb);
   } else {
     L.rope = L.wqkv = L.wo = L.wfc = L.wmp = L.wlm = 0;
   }
@@ -131,6 +145,11 @@ WsLayout ws_layout(const nc_config* c, int B, int T, bool own_weights = true) {
   L.tl = take(M * 4);
   L.x0 = (c->extras & NC_EXTRA_RESID_LAMBDAS) ? take(M * C * 4) : 0;
   L.xmid = (c->extras & NC_EXTRA_BACKOUT) ? take(M * C * 4) : 0;
+  // e4m3 codes of the activation entering the current product (the widest is
+  // the MLP c_proj input, 4C), and the amax slots
+  const size_t widest = std::max(4 * C, H * D);
+  L.a8 = c->fp8 ? take(M * widest) : 0;
+  L.amax = c->fp8 ? take((size_t)amax_slots(c->n_layer) * 4) : 0;
   L.total = off;
   return L;
 }
@@ -212,8 +231,10 @@ struct Tracer {
 // Number of kernel launches of one forward.
 int forward_launch_count(const nc_config* c, bool targets, bool loss, bool logits) {
   int n = 3 + c->n_layer * 7 + 1;  // rope table, cast, embedding; layers; final norm
+  if (c->fp8 & NC_FP8_BLOCK) n += 4 * c->n_layer;  // activation quantisations
   if (targets) n += 2 + (loss ? 1 : 0);
   else if (logits) n += 1;
+  if ((c->fp8 & NC_FP8_LM_HEAD) && (targets || logits)) n += 1;
   return n;
 }
 
@@ -406,6 +427,40 @@ nc_status nc_linear(const uint16_t* a, const uint16_t* w, void* out, int M, int 
   return gemm_launch(a, K, w, K, M, N, K, (int)epilogue, dtype == NC_F16, ep, dev_status, S(stream));
 }
 
+nc_status nc_fp8_quantize(const void* x, nc_dtype src_dtype, int64_t n, uint8_t* codes, float* amax,
+                          void* stream) {
+  if (!x || !codes || !amax || n < 0) return NC_ERR_INVALID_ARG;
+  if (src_dtype != NC_F32 && src_dtype != NC_BF16 && src_dtype != NC_F16) return NC_ERR_INVALID_ARG;
+  if (n % 16 != 0) return NC_ERR_SHAPE;
+  if (!aligned16(x) || !aligned16(codes)) return NC_ERR_ALIGNMENT;
+  if (nc_status s = device_ok()) return s;
+  cudaStream_t st = S(stream);
+  if (cudaMemsetAsync(amax, 0, sizeof(float), st) != cudaSuccess) return NC_ERR_CUDA;
+  const Fp8Seg seg{x, codes, n, 0};
+  const int kind = src_dtype == NC_F32 ? FP8_SRC_F32 : src_dtype == NC_F16 ? FP8_SRC_F16 : FP8_SRC_BF16;
+  return fp8_quantize_launch(&seg, 1, kind, amax, true, st);
+}
+
+nc_status nc_linear_fp8(const uint8_t* a, const float* amax_a, const uint8_t* w, const float* amax_w,
+                        void* out, int M, int N, int K, int64_t ldo, nc_epilogue epilogue, float cap,
+                        nc_dtype dtype, uint32_t* dev_status, void* stream) {
+  if (!a || !w || !amax_a || !amax_w || !out || M < 0 || N < 32 || K < 16 || !dtype_ok(dtype))
+    return NC_ERR_INVALID_ARG;
+  if ((int)epilogue < 0 || (int)epilogue > (int)NC_EPI_SOFTCAP_F32) return NC_ERR_INVALID_ARG;
+  if (N % 32 != 0 || K % 16 != 0 || ldo < N || ldo % 8 != 0) return NC_ERR_SHAPE;
+  if (epilogue == NC_EPI_SOFTCAP_F32 && !(cap > 0.0f)) return NC_ERR_INVALID_ARG;
+  if (!aligned16(a) || !aligned16(w) || !aligned16(out)) return NC_ERR_ALIGNMENT;
+  if (nc_status s = device_ok()) return s;
+  if (M == 0) return NC_OK;
+  EpiParams ep{};
+  ep.out = out;
+  ep.ldo = ldo;
+  ep.cap = cap;
+  ep.amax_a = amax_a;
+  ep.amax_b = amax_w;
+  return gemm_launch_e4m3(a, K, w, K, M, N, K, (int)epilogue, dtype == NC_F16, ep, dev_status, S(stream));
+}
+
 nc_status nc_qkv_rope(const uint16_t* a, const uint16_t* w, uint16_t* out, const float* table,
                       int M, int T, int C, int H, int Hkv, int D, float eps, nc_dtype dtype,
                       uint32_t* dev_status, void* stream) {
@@ -450,14 +505,38 @@ nc_status nc_loss_mean(const float* token_loss, const int32_t* targets, int M, i
 // The one weight-cast launch: every fp32 matmul weight -> its bf16 value (held
 // in fp16 when f16); c_q, c_k, c_v of a layer packed into one matrix, with the
 // rows of c_q and c_k reordered so each RoPE pair is adjacent.
+//
+// With cfg->fp8 the weights of the chosen products are quantised to e4m3
+// instead (same packing and row order, one byte per element): one amax launch
+// and one quantise launch over all of them, each weight tensor with its own
+// slot in `amax` (zeroed by the caller).
 static nc_status launch_weight_cast(const nc_config* cfg, const nc_weights* w, uint16_t* wqkv, uint16_t* wo,
                                     uint16_t* wfc, uint16_t* wmp, uint16_t* wlm, size_t e_qkv, size_t e_wo,
-                                    size_t e_fc, size_t e_mp, bool f16, cudaStream_t st) {
+                                    size_t e_fc, size_t e_mp, bool f16, cudaStream_t st, float* amax = nullptr) {
   const int C = cfg->d_model, D = cfg->head_dim, H = cfg->n_head, Hkv = cfg->n_kv_head, V = cfg->vocab;
+  const size_t nq = (size_t)H * D * C, nk = (size_t)Hkv * D * C;
+  const bool q_block = (cfg->fp8 & NC_FP8_BLOCK) != 0, q_head = (cfg->fp8 & NC_FP8_LM_HEAD) != 0;
+  if (q_block || q_head) {
+    std::vector<Fp8Seg> qs;
+    qs.reserve(cfg->n_layer * 6 + 1);
+    if (q_block) {
+      for (int l = 0; l < cfg->n_layer; ++l) {
+        uint8_t* dq = reinterpret_cast<uint8_t*>(wqkv) + l * e_qkv;
+        qs.push_back({w->c_q[l], dq, (int64_t)nq, amax_w_slot(l, 0), true});
+        qs.push_back({w->c_k[l], dq + nq, (int64_t)nk, amax_w_slot(l, 1), true});
+        qs.push_back({w->c_v[l], dq + nq + nk, (int64_t)nk, amax_w_slot(l, 2)});
+        qs.push_back({w->attn_proj[l], reinterpret_cast<uint8_t*>(wo) + l * e_wo, (int64_t)e_wo, amax_w_slot(l, 3)});
+        qs.push_back({w->c_fc[l], reinterpret_cast<uint8_t*>(wfc) + l * e_fc, (int64_t)e_fc, amax_w_slot(l, 4)});
+        qs.push_back({w->mlp_proj[l], reinterpret_cast<uint8_t*>(wmp) + l * e_mp, (int64_t)e_mp, amax_w_slot(l, 5)});
+      }
+    }
+    if (q_head)
+      qs.push_back({w->lm_head, reinterpret_cast<uint8_t*>(wlm), (int64_t)V * C, amax_wlm_slot(cfg->n_layer)});
+    if (nc_status s = fp8_quantize_launch(qs.data(), (int)qs.size(), FP8_SRC_F32, amax, true, st, C, D)) return s;
+  }
   std::vector<CastSeg> segs;
   segs.reserve(cfg->n_layer * 6 + 1);
-  const size_t nq = (size_t)H * D * C, nk = (size_t)Hkv * D * C;
-  for (int l = 0; l < cfg->n_layer; ++l) {
+  for (int l = 0; l < cfg->n_layer && !q_block; ++l) {
     uint16_t* dq = wqkv + l * e_qkv;
     segs.push_back({w->c_q[l], dq, (int64_t)nq, true});  // RoPE pairs made adjacent
     segs.push_back({w->c_k[l], dq + nq, (int64_t)nk, true});
@@ -466,7 +545,8 @@ static nc_status launch_weight_cast(const nc_config* cfg, const nc_weights* w, u
     segs.push_back({w->c_fc[l], wfc + l * e_fc, (int64_t)e_fc});
     segs.push_back({w->mlp_proj[l], wmp + l * e_mp, (int64_t)e_mp});
   }
-  segs.push_back({w->lm_head, wlm, (int64_t)V * C});
+  if (!q_head) segs.push_back({w->lm_head, wlm, (int64_t)V * C});
+  if (segs.empty()) return NC_OK;
   return cast_launch(segs.data(), (int)segs.size(), f16, st, C, D);
 }
 
@@ -568,6 +648,9 @@ static nc_status forward_impl(const nc_config* cfg, const nc_weights* w, const i
   float* tl = token_loss ? token_loss : reinterpret_cast<float*>(ws + L.tl);
   float* x0 = (ex & NC_EXTRA_RESID_LAMBDAS) ? reinterpret_cast<float*>(ws + L.x0) : nullptr;
   float* xmid = (ex & NC_EXTRA_BACKOUT) ? reinterpret_cast<float*>(ws + L.xmid) : nullptr;
+  const bool q_block = (cfg->fp8 & NC_FP8_BLOCK) != 0, q_head = (cfg->fp8 & NC_FP8_LM_HEAD) != 0;
+  uint8_t* a8 = cfg->fp8 ? ws + L.a8 : nullptr;
+  float* amax = cfg->fp8 ? reinterpret_cast<float*>(ws + L.amax) : nullptr;
   const int mid = cfg->n_layer / 2;  // backout: the stream after the first n_layer / 2 blocks
 
   const int M = B * T;
@@ -577,11 +660,22 @@ static nc_status forward_impl(const nc_config* cfg, const nc_weights* w, const i
   const bool f16 = cfg->act_dtype == NC_F16;
 
   if (cudaMemsetAsync(status, 0, 256, st) != cudaSuccess) return NC_ERR_CUDA;
+  if (amax && cudaMemsetAsync(amax, 0, (size_t)amax_slots(cfg->n_layer) * 4, st) != cudaSuccess)
+    return NC_ERR_CUDA;
   NC_RUN(NC_K_ROPE_TABLE, rope_table_launch(rope, T_rope, D, cfg->rope_base, st));
 
-  // fp32 -> bf16 weight cast; c_q|c_k|c_v rows packed into one matrix per layer.
+  // fp32 -> bf16 weight cast (e4m3 for the fp8 products); c_q|c_k|c_v rows
+  // packed into one matrix per layer.
   NC_RUN(NC_K_CAST, launch_weight_cast(cfg, w, wqkv, wo, wfc, wmp, wlm, L.wqkv_elems, L.wo_elems, L.wfc_elems,
-                                       L.wmp_elems, f16, st));
+                                       L.wmp_elems, f16, st, amax));
+  const int src16 = f16 ? FP8_SRC_F16 : FP8_SRC_BF16;
+  // e4m3 codes of the activation `src` ([M, K] 16-bit) into a8, amax into its slot
+  // (the producers of the plain path fold the amax in themselves: fused = true)
+  auto quant_act = [&](const uint16_t* src, int K, int slot, bool fused) -> nc_status {
+    const Fp8Seg seg{src, a8, (int64_t)M * K, slot};
+    return fp8_quantize_launch(&seg, 1, src16, amax, !fused, st);
+  };
+  auto slot_ptr = [&](int slot) { return amax ? amax + slot : nullptr; };
 
   if (ex & (NC_EXTRA_SMEAR | NC_EXTRA_RESID_LAMBDAS))
     NC_RUN(NC_K_EMBEDDING, embedding_extra_launch(tokens, w->wte, (ex & NC_EXTRA_SMEAR) ? w->smear_gate : nullptr,
@@ -592,12 +686,14 @@ static nc_status forward_impl(const nc_config* cfg, const nc_weights* w, const i
   for (int l = 0; l < cfg->n_layer; ++l) {
     const int W = nc_layer_window(cfg, l);
     float* keep = (xmid && l == mid) ? xmid : nullptr;
-    if (x0 || keep)  // x_mid = the stream entering block `mid`; then x = a_l x + b_l x0
+    const bool mixed = x0 || keep;
+    if (mixed)  // x_mid = the stream entering block `mid`; then x = a_l x + b_l x0
       NC_RUN(NC_K_RMSNORM, rmsnorm_mix_launch(x, x0, x0 ? w->resid_lambdas + l : nullptr,
                                               x0 ? w->x0_lambdas + l : nullptr, keep, nullptr, nullptr,
                                               x0 != nullptr, a, M, C, cfg->norm_eps, f16, st));
     else
-      NC_RUN(NC_K_RMSNORM, rmsnorm_launch(x, a, M, C, cfg->norm_eps, f16, st));
+      NC_RUN(NC_K_RMSNORM, rmsnorm_launch(x, a, M, C, cfg->norm_eps, f16, st,
+                                          q_block ? slot_ptr(amax_a_slot(cfg->n_layer, l, 0)) : nullptr));
     EpiParams eq{};  // QKV projection with RoPE + QK-norm in the epilogue
     eq.out = qkv;
     eq.ldo = NQKV;
@@ -614,18 +710,55 @@ static nc_status forward_impl(const nc_config* cfg, const nc_weights* w, const i
       eq.ve_gate = w->ve_gates[l];
       eq.V = V;
     }
-    NC_RUN(NC_K_GEMM_QKV, gemm_launch(a, C, wqkv + l * L.wqkv_elems, C, M, NQKV, C, EPI_QKV_ROPE_IL, f16,
-                                      eq, status, st));
+    if (q_block) {
+      NC_RUN(NC_K_FP8_QUANT, quant_act(a, C, amax_a_slot(cfg->n_layer, l, 0), !mixed));
+      eq.amax_a = amax + amax_a_slot(cfg->n_layer, l, 0);
+      eq.amax_b = amax + amax_w_slot(l, 0);  // q, k, v
+      NC_RUN(NC_K_GEMM_QKV, gemm_launch_e4m3(a8, C, reinterpret_cast<uint8_t*>(wqkv) + l * L.wqkv_elems, C, M,
+                                             NQKV, C, EPI_QKV_ROPE_IL, f16, eq, status, st));
+    } else {
+      NC_RUN(NC_K_GEMM_QKV, gemm_launch(a, C, wqkv + l * L.wqkv_elems, C, M, NQKV, C, EPI_QKV_ROPE_IL, f16,
+                                        eq, status, st));
+    }
     if (sess) {  // keep this layer's k and v for decoding
       uint16_t* cache = reinterpret_cast<uint16_t*>(sess->base + SL.cache) + l * SL.cache_layer_elems;
       nc_status s_ = kv_append_launch(qkv, NQKV, H * D, 2 * Hkv * D, cache, M, T, sess->T_max, 0, st);
       if (s_ != NC_OK) return s_;
     }
     NC_RUN(NC_K_ATTENTION, attention_launch(qkv, qkv + H * D, qkv + (H + Hkv) * D, o, B, T, H, Hkv,
-                                            D, W, NQKV, NQKV, f16, status, st));
+                                            D, W, NQKV, NQKV, f16, status, st,
+                                            q_block ? slot_ptr(amax_a_slot(cfg->n_layer, l, 1)) : nullptr));
     EpiParams ep{};
     ep.out = x;
     ep.ldo = C;
+    if (q_block) {  // the three remaining products in e4m3, each input quantised first
+      const int Lc = cfg->n_layer;
+      uint8_t* w8o = reinterpret_cast<uint8_t*>(wo) + l * L.wo_elems;
+      uint8_t* w8fc = reinterpret_cast<uint8_t*>(wfc) + l * L.wfc_elems;
+      uint8_t* w8mp = reinterpret_cast<uint8_t*>(wmp) + l * L.wmp_elems;
+      NC_RUN(NC_K_FP8_QUANT, quant_act(o, H * D, amax_a_slot(Lc, l, 1), true));
+      ep.amax_a = amax + amax_a_slot(Lc, l, 1);
+      ep.amax_b = amax + amax_w_slot(l, 3);
+      NC_RUN(NC_K_GEMM_ATTN_PROJ,
+             gemm_launch_e4m3(a8, H * D, w8o, H * D, M, C, H * D, EPI_RESID_F32, f16, ep, status, st));
+      NC_RUN(NC_K_RMSNORM, rmsnorm_launch(x, a, M, C, cfg->norm_eps, f16, st, amax + amax_a_slot(Lc, l, 2)));
+      NC_RUN(NC_K_FP8_QUANT, quant_act(a, C, amax_a_slot(Lc, l, 2), true));
+      ep.out = h;
+      ep.ldo = 4 * C;
+      ep.amax_a = amax + amax_a_slot(Lc, l, 2);
+      ep.amax_b = amax + amax_w_slot(l, 4);
+      ep.amax_out = amax + amax_a_slot(Lc, l, 3);
+      NC_RUN(NC_K_GEMM_FC, gemm_launch_e4m3(a8, C, w8fc, C, M, 4 * C, C, EPI_RELU2_16, f16, ep, status, st));
+      NC_RUN(NC_K_FP8_QUANT, quant_act(h, 4 * C, amax_a_slot(Lc, l, 3), true));
+      ep.amax_out = nullptr;
+      ep.out = x;
+      ep.ldo = C;
+      ep.amax_a = amax + amax_a_slot(Lc, l, 3);
+      ep.amax_b = amax + amax_w_slot(l, 5);
+      NC_RUN(NC_K_GEMM_MLP_PROJ,
+             gemm_launch_e4m3(a8, 4 * C, w8mp, 4 * C, M, C, 4 * C, EPI_RESID_F32, f16, ep, status, st));
+      continue;
+    }
     NC_RUN(NC_K_GEMM_ATTN_PROJ, gemm_launch(o, H * D, wo + l * L.wo_elems, H * D, M, C, H * D,
                                             EPI_RESID_F32, f16, ep, status, st));
     NC_RUN(NC_K_RMSNORM, rmsnorm_launch(x, a, M, C, cfg->norm_eps, f16, st));
@@ -643,7 +776,18 @@ static nc_status forward_impl(const nc_config* cfg, const nc_weights* w, const i
     NC_RUN(NC_K_RMSNORM, rmsnorm_mix_launch(x, nullptr, nullptr, nullptr, nullptr, xmid, w->backout_lambda, false,
                                             a, M, C, cfg->norm_eps, f16, st));
   else
-    NC_RUN(NC_K_RMSNORM, rmsnorm_launch(x, a, M, C, cfg->norm_eps, f16, st));
+    NC_RUN(NC_K_RMSNORM, rmsnorm_launch(x, a, M, C, cfg->norm_eps, f16, st,
+                                        q_head ? slot_ptr(amax_alm_slot(cfg->n_layer)) : nullptr));
+  // LM head: 16-bit, or e4m3 codes of the final normalised stream
+  const int alm = amax_alm_slot(cfg->n_layer);
+  if (q_head && (targets || logits)) NC_RUN(NC_K_FP8_QUANT, quant_act(a, C, alm, xmid == nullptr));
+  auto lm_head = [&](int epi, const EpiParams& ep0) -> nc_status {
+    if (!q_head) return gemm_launch(a, C, wlm, C, M, V, C, epi, f16, ep0, status, st);
+    EpiParams e8 = ep0;
+    e8.amax_a = amax + alm;
+    e8.amax_b = amax + amax_wlm_slot(cfg->n_layer);
+    return gemm_launch_e4m3(a8, C, reinterpret_cast<uint8_t*>(wlm), C, M, V, C, epi, f16, e8, status, st);
+  };
   if (targets) {
     EpiParams ep{};
     ep.out = logits;
@@ -653,7 +797,7 @@ static nc_status forward_impl(const nc_config* cfg, const nc_weights* w, const i
     ep.ce_partial = part;
     ep.ce_target = tgt;
     ep.targets = targets;
-    NC_RUN(NC_K_GEMM_LM_HEAD, gemm_launch(a, C, wlm, C, M, V, C, EPI_CE_PARTIAL, f16, ep, status, st));
+    NC_RUN(NC_K_GEMM_LM_HEAD, lm_head(EPI_CE_PARTIAL, ep));
     NC_RUN(NC_K_CE_FINALIZE, ce_finalize_launch(part, gemm_ce_partials_per_row(V), tgt, targets, tl, M, V,
                                                 cfg->softcap, status, st));
     if (loss) NC_RUN(NC_K_LOSS_MEAN, loss_mean_launch(tl, targets, M, V, loss, st));
@@ -662,7 +806,7 @@ static nc_status forward_impl(const nc_config* cfg, const nc_weights* w, const i
     ep.out = logits;
     ep.ldo = V;
     ep.cap = cfg->softcap;
-    NC_RUN(NC_K_GEMM_LM_HEAD, gemm_launch(a, C, wlm, C, M, V, C, EPI_SOFTCAP_F32, f16, ep, status, st));
+    NC_RUN(NC_K_GEMM_LM_HEAD, lm_head(EPI_SOFTCAP_F32, ep));
   }
 #undef NC_RUN
   return NC_OK;
@@ -697,7 +841,7 @@ nc_status nc_prefill(const nc_config* cfg, const nc_weights* w, const int32_t* t
                      float* logits, void* session, size_t session_bytes, int T_max, void* workspace,
                      size_t ws_bytes, void* stream) {
   if (!cfg || !w || !session) return NC_ERR_INVALID_ARG;
-  if (!config_ok(cfg) || cfg->extras != 0) return NC_ERR_CONFIG;
+  if (!config_ok(cfg) || cfg->extras != 0 || cfg->fp8 != 0) return NC_ERR_CONFIG;
   if (T_max < 1 || T_max > cfg->seq_len || T < 0 || T > T_max || B < 1) return NC_ERR_SHAPE;
   const SessionLayout SL = session_layout(cfg, B, T_max);
   if (session_bytes < SL.total) return NC_ERR_WORKSPACE;
@@ -732,7 +876,7 @@ static int resid_ksplit(int M, int N, int K) {
 nc_status nc_decode_step(const nc_config* cfg, const nc_weights* w, const int32_t* tokens, int B, int pos,
                          float* logits, void* session, size_t session_bytes, int T_max, void* stream) {
   if (!cfg || !w || !w->wte || !tokens || !logits || !session) return NC_ERR_INVALID_ARG;
-  if (!config_ok(cfg) || cfg->extras != 0) return NC_ERR_CONFIG;
+  if (!config_ok(cfg) || cfg->extras != 0 || cfg->fp8 != 0) return NC_ERR_CONFIG;
   if (T_max < 1 || T_max > cfg->seq_len || B < 1 || pos < 0 || pos >= T_max) return NC_ERR_SHAPE;
   const SessionLayout SL = session_layout(cfg, B, T_max);
   if (session_bytes < SL.total) return NC_ERR_WORKSPACE;

@@ -152,7 +152,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                    const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
                    uint16_t* __restrict__ out, int B,
                    int T, int H, int Hkv, int W, float scale_log2, uint32_t* dev_status,
-                   uint64_t limit_ns) {
+                   uint64_t limit_ns, float* __restrict__ amax) {
   using G = Geo<D>;
   constexpr uint32_t IDESC_S = idesc_f32acc(BQ, BKV, F16);
   constexpr uint32_t IDESC_PV = idesc_f32acc_bmn(BQ, D, F16);
@@ -406,6 +406,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     Pending pend{};
     bool has_pend = false;
     uint32_t store_busy = 0;  // P buffers a TMA store of this warp may still be reading
+    uint32_t om = 0;          // max |output| of this thread's rows (bits), for *amax
+    auto track = [&](float a) { om = max(om, __float_as_uint(a) & 0x7FFFFFFFu); };
     auto finish = [&](const Pending& pd, bool& ok_) {
       const float lsum = pd.l + exchange(pd.l, ok_);  // full row sum
       if (!ok_) return;
@@ -430,6 +432,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         // TMA write them to out.
         uint8_t* sbase = sm + G::OFF_P + (pd.gl & 1) * G::P_BYTES + half * ATOM;
         uint8_t* srow = sbase + r * 128;
+        if (amax && pd.q0 + r < T) {
+#pragma unroll
+          for (int c = 0; c < DC / 32; ++c)
+#pragma unroll
+            for (int e = 0; e < 32; ++e) track(__uint_as_float(rr[c][e]) * inv);
+        }
 #pragma unroll
         for (int q = 0; q < 8; ++q) {
           uint4 pk;
@@ -451,6 +459,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       } else {
         const int i = pd.q0 + r;
         if (i < T) {
+          if (amax) {
+#pragma unroll
+            for (int c = 0; c < DC / 32; ++c)
+#pragma unroll
+              for (int e = 0; e < 32; ++e) track(__uint_as_float(rr[c][e]) * inv);
+          }
           uint16_t* orow = out + (((int64_t)pd.b * T + i) * H + pd.h) * D + half * DC;
 #pragma unroll
           for (int q = 0; q < DC / 8; ++q) {
@@ -602,6 +616,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       if (lane == 0) mbar_arrive(smem_u32(&bar->next_empty[ns]));
     }
     if (ok && has_pend) finish(pend, ok);
+    if (amax) {
+      om = __reduce_max_sync(0xFFFFFFFFu, om);
+      if (lane == 0) fold_amax(amax, stored_abs_bits<F16>(om));
+    }
     if (lane == 0) bulk_wait0();
     __syncwarp();
   }
@@ -626,7 +644,7 @@ static bool make_map4(CUtensorMap* map, const void* base, int B, int T, int head
 template <int D, bool F16>
 static nc_status launch_t(const uint16_t* q, const uint16_t* k, const uint16_t* v, uint16_t* out,
                           int B, int T, int H, int Hkv, int W, int64_t q_stride, int64_t kv_stride,
-                          uint32_t* dev_status, cudaStream_t stream) {
+                          uint32_t* dev_status, cudaStream_t stream, float* amax) {
   using G = Geo<D>;
   static bool attr_done[64] = {};
   int dev = 0;
@@ -653,7 +671,7 @@ static nc_status launch_t(const uint16_t* q, const uint16_t* k, const uint16_t* 
   const int grid = B * H * ((T + BQ - 1) / BQ);
   const float scale_log2 = 1.4426950408889634f / sqrtf((float)D);
   attn_tc_kernel<D, F16><<<grid, NUM_THREADS, G::SMEM_BYTES, stream>>>(
-      mq, mk, mv, mo, out, B, T, H, Hkv, W, scale_log2, dev_status, kWaitLimitNs);
+      mq, mk, mv, mo, out, B, T, H, Hkv, W, scale_log2, dev_status, kWaitLimitNs, amax);
   return cudaGetLastError() == cudaSuccess ? NC_OK : NC_ERR_CUDA;
 }
 
@@ -661,15 +679,20 @@ static nc_status launch_t(const uint16_t* q, const uint16_t* k, const uint16_t* 
 
 nc_status attention_launch(const uint16_t* q, const uint16_t* k, const uint16_t* v, uint16_t* out,
                            int B, int T, int H, int Hkv, int D, int window, int64_t q_stride,
-                           int64_t kv_stride, bool f16, uint32_t* dev_status, cudaStream_t stream) {
+                           int64_t kv_stride, bool f16, uint32_t* dev_status, cudaStream_t stream,
+                           float* amax) {
   if (D != 64 && D != 128) return NC_ERR_SHAPE;
   if (B == 0 || T == 0) return NC_OK;
   const int W = (window <= 0 || window > T) ? T : window;
   if (D == 128)
-    return f16 ? attn::launch_t<128, true>(q, k, v, out, B, T, H, Hkv, W, q_stride, kv_stride, dev_status, stream)
-               : attn::launch_t<128, false>(q, k, v, out, B, T, H, Hkv, W, q_stride, kv_stride, dev_status, stream);
-  return f16 ? attn::launch_t<64, true>(q, k, v, out, B, T, H, Hkv, W, q_stride, kv_stride, dev_status, stream)
-             : attn::launch_t<64, false>(q, k, v, out, B, T, H, Hkv, W, q_stride, kv_stride, dev_status, stream);
+    return f16 ? attn::launch_t<128, true>(q, k, v, out, B, T, H, Hkv, W, q_stride, kv_stride, dev_status, stream,
+                                           amax)
+               : attn::launch_t<128, false>(q, k, v, out, B, T, H, Hkv, W, q_stride, kv_stride, dev_status,
+                                            stream, amax);
+  return f16 ? attn::launch_t<64, true>(q, k, v, out, B, T, H, Hkv, W, q_stride, kv_stride, dev_status, stream,
+                                        amax)
+             : attn::launch_t<64, false>(q, k, v, out, B, T, H, Hkv, W, q_stride, kv_stride, dev_status, stream,
+                                         amax);
 }
 
 }  // namespace nc

@@ -17,6 +17,11 @@
 //               two warps share each lane quarter and split the 256 columns),
 //               fused epilogue op, direct global stores; then hand the
 //               accumulator back.
+// e4m3 operands (dynamic tensorwise FP8, "Nanochat与nanoGPT对比" §1 table, FP8
+// row): the same pipeline with tcgen05.mma kind::f8f6f4.  A 128-byte swizzle
+// row then holds 128 elements instead of 64, so a stage covers K = 128 with the
+// same byte layout, descriptors and four MMAs (K = 32 each); the epilogue
+// scales the fp32 accumulator by 1 / (s_a s_w) before its fused op.
 // Tiles are visited with the N index fastest so consecutive CTAs share one A
 // row-block and the weight matrix stays resident in L2.
 // Every mbarrier wait is bounded; on timeout the CTA records NC_DEV_TIMEOUT,
@@ -53,6 +58,18 @@ constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + EPI_WARPS * STG_BYTES + 1024 /
                            256 /*barriers*/;
 constexpr uint32_t IDESC_BF16 = idesc_f32acc(BM, BN, false);
 constexpr uint32_t IDESC_F16 = idesc_f32acc(BM, BN, true);
+constexpr uint32_t IDESC_E4M3 = idesc_e4m3_f32acc(BM, BN);
+
+// Dequantisation factors of an e4m3 product, 1 / (s_a s_w), for the q, k and v
+// column ranges of the QKV projection (all three equal elsewhere).
+struct Dq {
+  float q, k, v;
+};
+
+__device__ __forceinline__ void scale32(uint32_t (&r)[32], float f) {
+#pragma unroll
+  for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * f);
+}
 
 struct Smem {  // barrier block placed after the tile ring and the staging tiles
   uint64_t full[STAGES];
@@ -177,10 +194,10 @@ __device__ __forceinline__ void epilogue_ce_chunk(const uint32_t (&r)[32], int r
 
 // fp32 epilogues (residual add, plain store, soft-cap): 32-column chunks.  The
 // TMEM load of chunk c+1 overlaps the TMA read of chunk c.
-template <int EPI>
+template <int EPI, bool SC>
 __device__ __forceinline__ void epilogue_f32_half(uint32_t taddr, const CUtensorMap* tmC, uint8_t* stg,
                                                   int n0, int row0, int N, const EpiParams& ep,
-                                                  uint32_t lane) {
+                                                  uint32_t lane, float dq) {
   uint32_t r[32];
   if (n0 < N) {
     tmem_ld_32x32b_x32(taddr, r);
@@ -190,6 +207,7 @@ __device__ __forceinline__ void epilogue_f32_half(uint32_t taddr, const CUtensor
   for (int c = 0; c < EPI_COLS / 32; ++c) {
     const int col0 = n0 + c * 32;
     if (col0 >= N) break;  // warp-uniform
+    if constexpr (SC) scale32(r, dq);
     if constexpr (EPI == EPI_SOFTCAP_F32) {
       const SoftCap sc(ep.cap);
 #pragma unroll
@@ -208,9 +226,12 @@ __device__ __forceinline__ void epilogue_f32_half(uint32_t taddr, const CUtensor
 
 // 16-bit epilogues (plain store, relu^2): 64-column chunks (128 B per row).
 // The TMEM loads of chunk c+1 overlap the TMA read of chunk c.
-template <int EPI, bool F16>
+// With SC (e4m3 operands) the relu^2 epilogue also keeps the running maximum
+// of its outputs in *om (bits; fp32 before the 16-bit rounding).
+template <int EPI, bool F16, bool SC = false>
 __device__ __forceinline__ void epilogue_16_half(uint32_t taddr, const CUtensorMap* tmC, uint8_t* stg,
-                                                 int n0, int row0, int N, uint32_t lane) {
+                                                 int n0, int row0, int N, uint32_t lane, float dq = 1.0f,
+                                                 uint32_t* om = nullptr) {
   uint32_t r[2][32];
   if (n0 < N) {
     tmem_ld_32x32b_x32(taddr, r[0]);
@@ -227,11 +248,16 @@ __device__ __forceinline__ void epilogue_16_half(uint32_t taddr, const CUtensorM
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
         float a = __uint_as_float(r[h][2 * i]), b = __uint_as_float(r[h][2 * i + 1]);
+        if constexpr (SC) {
+          a *= dq;
+          b *= dq;
+        }
         if constexpr (EPI == EPI_RELU2_16) {
           a = fmaxf(a, 0.0f);
           b = fmaxf(b, 0.0f);
           a *= a;
           b *= b;
+          if constexpr (SC) *om = max(*om, max(__float_as_uint(a), __float_as_uint(b)));  // a, b >= 0
         }
         w[16 * h + i] = Half<F16>::pack2(a, b);
       }
@@ -254,16 +280,17 @@ __device__ __forceinline__ void epilogue_16_half(uint32_t taddr, const CUtensorM
 // the fp32 accumulator.  Pass 2 rotates 32-pair groups; the first halves of the
 // pairs fill the staging tile (columns [0, HD/2) of the head) while the second
 // halves wait in registers, then take its place for columns [HD/2, HD).
-template <bool F16, int HD>
+template <bool F16, int HD, bool SC>
 __device__ __forceinline__ void epilogue_qkv_head(uint32_t taddr, const CUtensorMap* tmC, uint8_t* stg,
                                                   int row, int col0, int row0, int M,
-                                                  const EpiParams& ep, uint32_t lane) {
+                                                  const EpiParams& ep, uint32_t lane, const Dq& dqs) {
   constexpr int G = HD / 64;  // 32-pair groups per head (1 or 2)
   const int head = col0 / HD;
   if (head >= ep.H + ep.Hkv) {  // v head (warp-uniform): plain 16-bit store
-    epilogue_16_half<EPI_STORE_16, F16>(taddr, tmC, stg, col0, row0, col0 + HD, lane);
+    epilogue_16_half<EPI_STORE_16, F16, SC>(taddr, tmC, stg, col0, row0, col0 + HD, lane, dqs.v);
     return;
   }
+  const float dq = head < ep.H ? dqs.q : dqs.k;
   float ss = 0.0f;
 #pragma unroll
   for (int c = 0; c < HD / 64; ++c) {  // two 32-column loads per wait
@@ -279,7 +306,8 @@ __device__ __forceinline__ void epilogue_qkv_head(uint32_t taddr, const CUtensor
     }
     ss += (s4[0] + s4[1]) + (s4[2] + s4[3]);
   }
-  const float rs = rsqrtf(ss * (1.0f / HD) + ep.eps);
+  // e4m3: the head's values are dq * acc, so its mean square is dq^2 ss / HD
+  const float rs = SC ? rsqrtf(ss * (dq * dq) * (1.0f / HD) + ep.eps) * dq : rsqrtf(ss * (1.0f / HD) + ep.eps);
   const int t = ep.pos0 + (row < M ? row : 0) % ep.T;
   const float* cs = ep.rope + (int64_t)t * (HD / 2);
   const float* sn = ep.rope + ((int64_t)(ep.rope_T > 0 ? ep.rope_T : ep.T) + t) * (HD / 2);
@@ -328,10 +356,10 @@ __device__ __forceinline__ void epilogue_qkv_head(uint32_t taddr, const CUtensor
 // v head of the QKV projection with a value embedding (full nanochat forward,
 // "Nanochat与nanoGPT对比" §1, value-residual note): v + gate[g] * table[token]
 // for kv head g, the table row read in fp32 and added to the fp32 accumulator.
-template <bool F16, int HD>
+template <bool F16, int HD, bool SC>
 __device__ __forceinline__ void epilogue_v_embed(uint32_t taddr, const CUtensorMap* tmC, uint8_t* stg,
                                                  int row, int col0, int row0, int M, const EpiParams& ep,
-                                                 uint32_t lane) {
+                                                 uint32_t lane, float dq) {
   const int g = col0 / HD - ep.H - ep.Hkv;  // kv head
   int tok = row < M ? ep.tokens[row] : 0;
   if (tok < 0 || tok >= ep.V) tok = 0;  // flagged by the embedding kernel
@@ -343,6 +371,10 @@ __device__ __forceinline__ void epilogue_v_embed(uint32_t taddr, const CUtensorM
     tmem_ld_32x32b_x32(taddr + c * 64, r0);
     tmem_ld_32x32b_x32(taddr + c * 64 + 32, r1);
     tmem_wait_ld();
+    if constexpr (SC) {
+      scale32(r0, dq);
+      scale32(r1, dq);
+    }
     uint32_t w[32];
 #pragma unroll
     for (int j = 0; j < 16; ++j) {  // columns 4j .. 4j+3 of this 64-column chunk
@@ -361,18 +393,19 @@ __device__ __forceinline__ void epilogue_v_embed(uint32_t taddr, const CUtensorM
   flush_wait(lane);
 }
 
-template <bool F16, int HD>
+template <bool F16, int HD, bool SC>
 __device__ __forceinline__ void epilogue_qkv_head_il(uint32_t taddr, const CUtensorMap* tmC,
                                                      uint8_t* stg, int row, int col0, int row0, int M,
-                                                     const EpiParams& ep, uint32_t lane) {
+                                                     const EpiParams& ep, uint32_t lane, const Dq& dqs) {
   const int head = col0 / HD;
   if (head >= ep.H + ep.Hkv) {  // v head (warp-uniform)
     if (ep.ve)
-      epilogue_v_embed<F16, HD>(taddr, tmC, stg, row, col0, row0, M, ep, lane);
+      epilogue_v_embed<F16, HD, SC>(taddr, tmC, stg, row, col0, row0, M, ep, lane, dqs.v);
     else  // plain 16-bit store
-      epilogue_16_half<EPI_STORE_16, F16>(taddr, tmC, stg, col0, row0, col0 + HD, lane);
+      epilogue_16_half<EPI_STORE_16, F16, SC>(taddr, tmC, stg, col0, row0, col0 + HD, lane, dqs.v);
     return;
   }
+  const float dq = head < ep.H ? dqs.q : dqs.k;
   float ss = 0.0f;
 #pragma unroll
   for (int c = 0; c < HD / 64; ++c) {
@@ -388,7 +421,8 @@ __device__ __forceinline__ void epilogue_qkv_head_il(uint32_t taddr, const CUten
     }
     ss += (s4[0] + s4[1]) + (s4[2] + s4[3]);
   }
-  const float rs = rsqrtf(ss * (1.0f / HD) + ep.eps);
+  // e4m3: the head's values are dq * acc, so its mean square is dq^2 ss / HD
+  const float rs = SC ? rsqrtf(ss * (dq * dq) * (1.0f / HD) + ep.eps) * dq : rsqrtf(ss * (1.0f / HD) + ep.eps);
   const int t = ep.pos0 + (row < M ? row : 0) % ep.T;
   const float* cs = ep.rope + (int64_t)t * (HD / 2);
   const float* sn = ep.rope + ((int64_t)(ep.rope_T > 0 ? ep.rope_T : ep.T) + t) * (HD / 2);
@@ -421,14 +455,16 @@ __device__ __forceinline__ void epilogue_qkv_head_il(uint32_t taddr, const CUten
   flush_wait(lane);
 }
 
-// EPI: epilogue selector; F16: operands (and 16-bit outputs) fp16 instead of
-// bf16; HD: head size of the QKV epilogues (0 otherwise).
-template <int EPI, bool F16, int HD>
+// EPI: epilogue selector; F16: 16-bit operands (and 16-bit outputs) fp16
+// instead of bf16; HD: head size of the QKV epilogues (0 otherwise); FP8:
+// e4m3 operands (16-bit outputs still in the F16 format).
+template <int EPI, bool F16, int HD, bool FP8>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const __grid_constant__ CUtensorMap tmC, int M, int N, int K, EpiParams ep,
                 uint32_t* dev_status, uint64_t limit_ns) {
-  constexpr uint32_t IDESC = F16 ? IDESC_F16 : IDESC_BF16;
+  constexpr uint32_t IDESC = FP8 ? IDESC_E4M3 : (F16 ? IDESC_F16 : IDESC_BF16);
+  constexpr int KE = FP8 ? 2 * BK : BK;  // elements per 128-byte swizzle row
   extern __shared__ uint8_t smem_raw[];
   uint8_t* tiles = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~static_cast<uintptr_t>(1023));
@@ -443,7 +479,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const int ksplit = (EPI == EPI_RESID_F32 && ep.ksplit > 1) ? ep.ksplit : 1;
   const int num_mn = num_m * num_n;
   const int num_tiles = num_mn * ksplit;
-  const int num_kb = (K + BK - 1) / BK;
+  const int num_kb = (K + KE - 1) / KE;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -493,8 +529,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           const uint32_t fb = smem_u32(&sm->full[stage]);
           mbar_arrive_expect_tx(fb, STAGE_BYTES);
           uint8_t* a_dst = tiles + stage * STAGE_BYTES;
-          tma_load_2d(smem_u32(a_dst), &tmA, kb * BK, m0, fb);
-          tma_load_2d(smem_u32(a_dst + A_BYTES), &tmB, kb * BK, n0, fb);
+          tma_load_2d(smem_u32(a_dst), &tmA, kb * KE, m0, fb);
+          tma_load_2d(smem_u32(a_dst + A_BYTES), &tmB, kb * KE, n0, fb);
           outstanding |= 1u << stage;
           out_phase = (out_phase & ~(1u << stage)) | (phase << stage);
           if (++stage == STAGES) {
@@ -535,10 +571,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           const uint32_t a_addr = smem_u32(tiles + stage * STAGE_BYTES);
           const uint32_t b_addr = a_addr + A_BYTES;
 #pragma unroll
-          for (int k = 0; k < BK / 16; ++k) {
+          for (int k = 0; k < BK / 16; ++k) {  // 32 bytes of each row per MMA
             const uint64_t adesc = sw128_kmajor_desc(a_addr + k * 32);
             const uint64_t bdesc = sw128_kmajor_desc(b_addr + k * 32);
-            umma_f16(d_tmem, adesc, bdesc, IDESC, (kb != kb_begin || k != 0) ? 1u : 0u);
+            if constexpr (FP8)
+              umma_f8(d_tmem, adesc, bdesc, IDESC, (kb != kb_begin || k != 0) ? 1u : 0u);
+            else
+              umma_f16(d_tmem, adesc, bdesc, IDESC, (kb != kb_begin || k != 0) ? 1u : 0u);
           }
           umma_commit(smem_u32(&sm->empty[stage]));
           if (++stage == STAGES) {
@@ -565,6 +604,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const int half = (int)(warp - 2) / 4;  // which half of the tile's columns
     const int row_in_tile = quarter * 32 + lane;
     uint8_t* stg = staging + (warp - 2) * STG_BYTES;  // this warp's staging tile
+    Dq dqs{1.0f, 1.0f, 1.0f};
+    uint32_t om = 0;  // relu^2 with e4m3 operands: max output (bits) for ep.amax_out
+    if constexpr (FP8) {  // 1 / (s_a s_w) from the tensors' amax values
+      const float sa = e4m3_scale(__ldg(ep.amax_a));
+      dqs.q = 1.0f / (sa * e4m3_scale(__ldg(ep.amax_b)));
+      if constexpr (EPI == EPI_QKV_ROPE || EPI == EPI_QKV_ROPE_IL) {
+        dqs.k = 1.0f / (sa * e4m3_scale(__ldg(ep.amax_b + 1)));
+        dqs.v = 1.0f / (sa * e4m3_scale(__ldg(ep.amax_b + 2)));
+      } else {
+        dqs.k = dqs.v = dqs.q;
+      }
+    }
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
@@ -600,12 +651,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           const int col0 = n0 + hh * HD;
           if (col0 >= N) break;  // warp-uniform
           if constexpr (EPI == EPI_QKV_ROPE)
-            epilogue_qkv_head<F16, HD>(taddr + hh * HD, &tmC, stg, row, col0, row0, M, ep, lane);
+            epilogue_qkv_head<F16, HD, FP8>(taddr + hh * HD, &tmC, stg, row, col0, row0, M, ep, lane, dqs);
           else
-            epilogue_qkv_head_il<F16, HD>(taddr + hh * HD, &tmC, stg, row, col0, row0, M, ep, lane);
+            epilogue_qkv_head_il<F16, HD, FP8>(taddr + hh * HD, &tmC, stg, row, col0, row0, M, ep, lane, dqs);
         }
       } else if constexpr (EPI == EPI_STORE_16 || EPI == EPI_RELU2_16) {
-        epilogue_16_half<EPI, F16>(taddr, &tmC, stg, n0, row0, N, lane);
+        epilogue_16_half<EPI, F16, FP8>(taddr, &tmC, stg, n0, row0, N, lane, dqs.q, &om);
       } else if constexpr (EPI == EPI_CE_PARTIAL) {
         if (row < M) target = ep.targets ? ep.targets[row] : -1;
 #pragma unroll 1
@@ -615,10 +666,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           uint32_t r[32];
           tmem_ld_32x32b_x32(taddr + c * 32, r);
           tmem_wait_ld();
+          if constexpr (FP8) scale32(r, dqs.q);
           if (row < M) epilogue_ce_chunk(r, row, col0, ep, ce_sum, ce_tl, target);
         }
       } else {
-        epilogue_f32_half<EPI>(taddr, &tmC, stg, n0, row0, N, ep, lane);
+        epilogue_f32_half<EPI, FP8>(taddr, &tmC, stg, n0, row0, N, ep, lane, dqs.q);
       }
       if constexpr (EPI == EPI_CE_PARTIAL) {
         if (row < M) {
@@ -632,6 +684,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       if (++acc == NUM_ACC) {
         acc = 0;
         acc_phase ^= 1u;
+      }
+    }
+    if constexpr (FP8 && EPI == EPI_RELU2_16) {
+      if (ep.amax_out) {
+        om = __reduce_max_sync(0xFFFFFFFFu, om);
+        if (lane == 0) fold_amax(ep.amax_out, stored_abs_bits<F16>(om));
       }
     }
     if (lane == 0) bulk_wait0();  // every TMA store / reduce of this warp has landed
@@ -673,7 +731,16 @@ static bool make_map(CUtensorMap* map, const void* ptr, int64_t rows, int64_t co
   return encode_tensor_map(map, f16, 2, ptr, dims, strides, box);
 }
 
-template <int EPI, bool F16, int HD>
+// 8-bit row-major [rows, cols] with row stride `ld` bytes; box = 128 x box_rows.
+static bool make_map_u8(CUtensorMap* map, const void* ptr, int64_t rows, int64_t cols, int64_t ld,
+                        int box_rows) {
+  const uint64_t dims[2] = {(uint64_t)cols, (uint64_t)rows};
+  const uint64_t strides[1] = {(uint64_t)ld};
+  const uint32_t box[2] = {(uint32_t)(2 * BK), (uint32_t)box_rows};
+  return encode_tensor_map_u8(map, 2, ptr, dims, strides, box);
+}
+
+template <int EPI, bool F16, int HD, bool FP8>
 static cudaError_t launch_t(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& mc, int M,
                             int N, int K, const EpiParams& ep, uint32_t* dev_status, uint64_t limit_ns,
                             cudaStream_t stream) {
@@ -681,7 +748,7 @@ static cudaError_t launch_t(const CUtensorMap& ma, const CUtensorMap& mb, const 
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 64 && !attr_done[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_kernel<EPI, F16, HD>,
+    cudaError_t e = cudaFuncSetAttribute(gemm_kernel<EPI, F16, HD, FP8>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
     if (e != cudaSuccess) return e;
     attr_done[dev] = true;
@@ -689,28 +756,30 @@ static cudaError_t launch_t(const CUtensorMap& ma, const CUtensorMap& mb, const 
   const int tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN) * (EPI == EPI_RESID_F32 && ep.ksplit > 1 ? ep.ksplit : 1);
   const int sms = device_sm_count();
   const int grid = tiles < sms ? tiles : sms;
-  gemm_kernel<EPI, F16, HD><<<grid, NUM_THREADS, SMEM_BYTES, stream>>>(ma, mb, mc, M, N, K, ep,
-                                                                       dev_status, limit_ns);
+  gemm_kernel<EPI, F16, HD, FP8><<<grid, NUM_THREADS, SMEM_BYTES, stream>>>(ma, mb, mc, M, N, K, ep,
+                                                                            dev_status, limit_ns);
   return cudaGetLastError();
 }
 
-template <bool F16>
+template <bool F16, bool FP8>
 static cudaError_t dispatch(int epi, const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& mc,
                             int M, int N, int K, const EpiParams& ep, uint32_t* st, uint64_t lim,
                             cudaStream_t s) {
   switch (epi) {
-    case EPI_STORE_16: return launch_t<EPI_STORE_16, F16, 0>(ma, mb, mc, M, N, K, ep, st, lim, s);
-    case EPI_RELU2_16: return launch_t<EPI_RELU2_16, F16, 0>(ma, mb, mc, M, N, K, ep, st, lim, s);
-    case EPI_RESID_F32: return launch_t<EPI_RESID_F32, F16, 0>(ma, mb, mc, M, N, K, ep, st, lim, s);
-    case EPI_STORE_F32: return launch_t<EPI_STORE_F32, F16, 0>(ma, mb, mc, M, N, K, ep, st, lim, s);
-    case EPI_SOFTCAP_F32: return launch_t<EPI_SOFTCAP_F32, F16, 0>(ma, mb, mc, M, N, K, ep, st, lim, s);
-    case EPI_CE_PARTIAL: return launch_t<EPI_CE_PARTIAL, F16, 0>(ma, mb, mc, M, N, K, ep, st, lim, s);
+    case EPI_STORE_16: return launch_t<EPI_STORE_16, F16, 0, FP8>(ma, mb, mc, M, N, K, ep, st, lim, s);
+    case EPI_RELU2_16: return launch_t<EPI_RELU2_16, F16, 0, FP8>(ma, mb, mc, M, N, K, ep, st, lim, s);
+    case EPI_RESID_F32: return launch_t<EPI_RESID_F32, F16, 0, FP8>(ma, mb, mc, M, N, K, ep, st, lim, s);
+    case EPI_STORE_F32: return launch_t<EPI_STORE_F32, F16, 0, FP8>(ma, mb, mc, M, N, K, ep, st, lim, s);
+    case EPI_SOFTCAP_F32: return launch_t<EPI_SOFTCAP_F32, F16, 0, FP8>(ma, mb, mc, M, N, K, ep, st, lim, s);
+    case EPI_CE_PARTIAL: return launch_t<EPI_CE_PARTIAL, F16, 0, FP8>(ma, mb, mc, M, N, K, ep, st, lim, s);
     case EPI_QKV_ROPE:
-      return ep.D == 128 ? launch_t<EPI_QKV_ROPE, F16, 128>(ma, mb, mc, M, N, K, ep, st, lim, s)
-                         : launch_t<EPI_QKV_ROPE, F16, 64>(ma, mb, mc, M, N, K, ep, st, lim, s);
+      if constexpr (FP8) return cudaErrorInvalidValue;  // the interleaved form only
+      else
+        return ep.D == 128 ? launch_t<EPI_QKV_ROPE, F16, 128, false>(ma, mb, mc, M, N, K, ep, st, lim, s)
+                           : launch_t<EPI_QKV_ROPE, F16, 64, false>(ma, mb, mc, M, N, K, ep, st, lim, s);
     case EPI_QKV_ROPE_IL:
-      return ep.D == 128 ? launch_t<EPI_QKV_ROPE_IL, F16, 128>(ma, mb, mc, M, N, K, ep, st, lim, s)
-                         : launch_t<EPI_QKV_ROPE_IL, F16, 64>(ma, mb, mc, M, N, K, ep, st, lim, s);
+      return ep.D == 128 ? launch_t<EPI_QKV_ROPE_IL, F16, 128, FP8>(ma, mb, mc, M, N, K, ep, st, lim, s)
+                         : launch_t<EPI_QKV_ROPE_IL, F16, 64, FP8>(ma, mb, mc, M, N, K, ep, st, lim, s);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -744,6 +813,11 @@ bool encode_tensor_map(CUtensorMap* map, bool f16, int rank, const void* base, c
                     base, dims, strides, box);
 }
 
+bool encode_tensor_map_u8(CUtensorMap* map, int rank, const void* base, const uint64_t* dims,
+                          const uint64_t* strides, const uint32_t* box) {
+  return encode_any(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, rank, base, dims, strides, box);
+}
+
 bool encode_tensor_map_f32(CUtensorMap* map, int rank, const void* base, const uint64_t* dims,
                            const uint64_t* strides, const uint32_t* box) {
   return encode_any(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, rank, base, dims, strides, box);
@@ -774,31 +848,54 @@ nc_status selftest_wait_launch(uint32_t* dev_status, uint64_t limit_ns, cudaStre
 
 int gemm_ce_partials_per_row(int N) { return 2 * ((N + gemm::BN - 1) / gemm::BN); }
 
+// Output tile map for the TMA stores of the epilogue: 32 rows x 128 bytes
+// (64 16-bit or 32 fp32 columns), the box one epilogue warp stages.
+static bool make_out_map(CUtensorMap* mc, int epi, int M, int N, bool f16, const EpiParams& ep) {
+  memset(mc, 0, sizeof(*mc));
+  if (epi == EPI_CE_PARTIAL) return true;
+  const uint64_t dims[2] = {(uint64_t)N, (uint64_t)M};
+  const bool out16 = (epi == EPI_STORE_16 || epi == EPI_RELU2_16 || epi == EPI_QKV_ROPE ||
+                      epi == EPI_QKV_ROPE_IL);
+  const uint64_t strides[1] = {(uint64_t)ep.ldo * (out16 ? 2 : 4)};
+  const uint32_t box[2] = {out16 ? 64u : 32u, 32u};
+  return out16 ? encode_tensor_map(mc, f16, 2, ep.out, dims, strides, box)
+               : encode_tensor_map_f32(mc, 2, ep.out, dims, strides, box);
+}
+
+static nc_status check_epi(int epi, int K, int ke, const EpiParams& ep) {
+  if (epi < EPI_STORE_16 || epi > EPI_QKV_ROPE_IL) return NC_ERR_INVALID_ARG;
+  if ((epi == EPI_QKV_ROPE || epi == EPI_QKV_ROPE_IL) && (ep.D != 64 && ep.D != 128)) return NC_ERR_SHAPE;
+  if (ep.ksplit > 1 && (epi != EPI_RESID_F32 || ep.ksplit > (K + ke - 1) / ke)) return NC_ERR_INVALID_ARG;
+  return NC_OK;
+}
+
 nc_status gemm_launch(const uint16_t* a, int64_t lda, const uint16_t* w, int64_t ldw, int M, int N,
                       int K, int epi, bool f16, const EpiParams& ep, uint32_t* dev_status,
                       cudaStream_t stream, uint64_t limit_ns) {
   using namespace gemm;
-  if (epi < EPI_STORE_16 || epi > EPI_QKV_ROPE_IL) return NC_ERR_INVALID_ARG;
-  if ((epi == EPI_QKV_ROPE || epi == EPI_QKV_ROPE_IL) && (ep.D != 64 && ep.D != 128)) return NC_ERR_SHAPE;
-  if (ep.ksplit > 1 && (epi != EPI_RESID_F32 || ep.ksplit > (K + BK - 1) / BK)) return NC_ERR_INVALID_ARG;
+  if (nc_status s = check_epi(epi, K, BK, ep)) return s;
   CUtensorMap ma, mb, mc;
   if (!make_map(&ma, a, M, K, lda, BM, f16)) return NC_ERR_CUDA;
   if (!make_map(&mb, w, N, K, ldw, BN, f16)) return NC_ERR_CUDA;
-  // Output tile map for the TMA stores of the epilogue: 32 rows x 128 bytes
-  // (64 16-bit or 32 fp32 columns), the box one epilogue warp stages.
-  memset(&mc, 0, sizeof(mc));
-  if (epi != EPI_CE_PARTIAL) {
-    const uint64_t dims[2] = {(uint64_t)N, (uint64_t)M};
-    const bool out16 = (epi == EPI_STORE_16 || epi == EPI_RELU2_16 || epi == EPI_QKV_ROPE ||
-                        epi == EPI_QKV_ROPE_IL);
-    const uint64_t strides[1] = {(uint64_t)ep.ldo * (out16 ? 2 : 4)};
-    const uint32_t box[2] = {out16 ? 64u : 32u, 32u};
-    const bool ok = out16 ? encode_tensor_map(&mc, f16, 2, ep.out, dims, strides, box)
-                          : encode_tensor_map_f32(&mc, 2, ep.out, dims, strides, box);
-    if (!ok) return NC_ERR_CUDA;
-  }
-  const cudaError_t e = f16 ? dispatch<true>(epi, ma, mb, mc, M, N, K, ep, dev_status, limit_ns, stream)
-                            : dispatch<false>(epi, ma, mb, mc, M, N, K, ep, dev_status, limit_ns, stream);
+  if (!make_out_map(&mc, epi, M, N, f16, ep)) return NC_ERR_CUDA;
+  const cudaError_t e = f16 ? dispatch<true, false>(epi, ma, mb, mc, M, N, K, ep, dev_status, limit_ns, stream)
+                            : dispatch<false, false>(epi, ma, mb, mc, M, N, K, ep, dev_status, limit_ns, stream);
+  return e == cudaSuccess ? NC_OK : NC_ERR_CUDA;
+}
+
+nc_status gemm_launch_e4m3(const uint8_t* a, int64_t lda, const uint8_t* w, int64_t ldw, int M, int N, int K,
+                           int epi, bool f16, const EpiParams& ep, uint32_t* dev_status, cudaStream_t stream,
+                           uint64_t limit_ns) {
+  using namespace gemm;
+  if (nc_status s = check_epi(epi, K, 2 * BK, ep)) return s;
+  if (epi == EPI_QKV_ROPE || !ep.amax_a || !ep.amax_b || K % 16 || lda % 16 || ldw % 16)
+    return NC_ERR_INVALID_ARG;
+  CUtensorMap ma, mb, mc;
+  if (!make_map_u8(&ma, a, M, K, lda, BM)) return NC_ERR_CUDA;
+  if (!make_map_u8(&mb, w, N, K, ldw, BN)) return NC_ERR_CUDA;
+  if (!make_out_map(&mc, epi, M, N, f16, ep)) return NC_ERR_CUDA;
+  const cudaError_t e = f16 ? dispatch<true, true>(epi, ma, mb, mc, M, N, K, ep, dev_status, limit_ns, stream)
+                            : dispatch<false, true>(epi, ma, mb, mc, M, N, K, ep, dev_status, limit_ns, stream);
   return e == cudaSuccess ? NC_OK : NC_ERR_CUDA;
 }
 

@@ -46,6 +46,12 @@ struct EpiParams {
   const float* ve;          //   [V, Hkv*D] table of this layer (NULL: none)
   const float* ve_gate;     //   [Hkv] gates
   int V;                    //   vocabulary size (ids outside [0, V) read row 0)
+  const float* amax_a;      // e4m3 operands: [1] amax of A, and
+  const float* amax_b;      //   [1] amax of W ([3]: q, k, v parts for EPI_QKV_ROPE*); the
+                            //   epilogue scales the product by 1 / (s_a s_w),
+                            //   s = 448 / max(amax, 1e-12)
+  float* amax_out;          // EPI_RELU2_16 with e4m3 operands: fold max |stored output| into
+                            //   this slot (the quantisation of the output that follows)
 };
 
 // ---- device / argument helpers (nc_api.cu)
@@ -62,20 +68,44 @@ nc_status gemm_launch(const uint16_t* a, int64_t lda, const uint16_t* w, int64_t
                       int K, int epi, bool f16, const EpiParams& ep, uint32_t* dev_status,
                       cudaStream_t stream, uint64_t limit_ns = kWaitLimitNs);
 
+// The same with e4m3 operands a [M, K] (row stride lda bytes) and w [N, K]
+// (row stride ldw bytes), tcgen05 kind::f8f6f4; ep.amax_a / ep.amax_b give the
+// tensorwise scales.  16-bit outputs are in format `f16`.  K % 16 == 0.
+nc_status gemm_launch_e4m3(const uint8_t* a, int64_t lda, const uint8_t* w, int64_t ldw, int M, int N, int K,
+                           int epi, bool f16, const EpiParams& ep, uint32_t* dev_status, cudaStream_t stream,
+                           uint64_t limit_ns = kWaitLimitNs);
+
 nc_status selftest_wait_launch(uint32_t* dev_status, uint64_t limit_ns, cudaStream_t stream);
+
+// ---- dynamic tensorwise e4m3 quantisation (nc_fp8.cu)
+enum { FP8_SRC_F32 = 0, FP8_SRC_BF16 = 1, FP8_SRC_F16 = 2 };
+struct Fp8Seg {
+  const void* src;         // source tensor (element type: the launch's src_kind)
+  uint8_t* dst;            // e4m3 codes, n bytes
+  int64_t n;               // elements, multiple of 16
+  int slot;                // amax slot (index into the launch's amax array)
+  bool pair_rows = false;  // destination rows in the QKV RoPE-pair order (perm_cols, perm_d)
+};
+// amax pass (when do_amax; slots must hold 0) then quantise pass over every
+// segment.  Source pointers 16-byte aligned.
+nc_status fp8_quantize_launch(const Fp8Seg* segs, int nseg, int src_kind, float* amax, bool do_amax,
+                              cudaStream_t stream, int perm_cols = 0, int perm_d = 0);
 
 // TMA tensor map with 128-byte swizzling: dims innermost first, strides in
 // bytes for dims 1..rank-1.  Element type: fp16 if f16, else bf16; the _f32
 // variant maps fp32 data.
 bool encode_tensor_map(CUtensorMap* map, bool f16, int rank, const void* base, const uint64_t* dims,
                        const uint64_t* strides, const uint32_t* box);
+bool encode_tensor_map_u8(CUtensorMap* map, int rank, const void* base, const uint64_t* dims,
+                          const uint64_t* strides, const uint32_t* box);
 bool encode_tensor_map_f32(CUtensorMap* map, int rank, const void* base, const uint64_t* dims,
                            const uint64_t* strides, const uint32_t* box);
 
 // ---- attention (nc_attention.cu)
 nc_status attention_launch(const uint16_t* q, const uint16_t* k, const uint16_t* v, uint16_t* out,
                            int B, int T, int H, int Hkv, int D, int window, int64_t q_stride,
-                           int64_t kv_stride, bool f16, uint32_t* dev_status, cudaStream_t stream);
+                           int64_t kv_stride, bool f16, uint32_t* dev_status, cudaStream_t stream,
+                           float* amax = nullptr);
 
 // ---- elementwise / row kernels (nc_rowops.cu)
 struct CastSeg {
@@ -127,7 +157,8 @@ nc_status qkv_finish_launch(const float* acc, uint16_t* qkv, uint16_t* cache, co
 nc_status relu2_finish_launch(const float* acc, uint16_t* out, int64_t n, bool f16, cudaStream_t stream);
 
 nc_status rmsnorm_launch(const float* x, uint16_t* out, int M, int C, float eps, bool f16,
-                         cudaStream_t stream);
+                         cudaStream_t stream,
+                         float* amax = nullptr);
 nc_status rope_table_launch(float* table, int T, int D, float base, cudaStream_t stream);
 nc_status rope_qknorm_launch(uint16_t* q, uint16_t* k, const float* table, int B, int T, int H,
                              int Hkv, int D, int64_t q_stride, int64_t k_stride, float eps, bool f16,

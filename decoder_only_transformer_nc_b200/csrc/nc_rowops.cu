@@ -160,11 +160,13 @@ __global__ void __launch_bounds__(256) embedding_extra_kernel(const int32_t* __r
 
 // ---------------------------------------------------------------- RMSNorm
 
-// One warp per row; the row is held in registers (C <= 32 * 4 * NV).
+// One warp per row; the row is held in registers (C <= 32 * 4 * NV).  With
+// amax != NULL the largest |stored value| is folded into *amax (the e4m3
+// quantisation of the output that follows).
 template <int NV, bool F16>
 __global__ void __launch_bounds__(256) rmsnorm_kernel(const float* __restrict__ x,
                                                       uint16_t* __restrict__ out, int M, int C,
-                                                      float eps) {
+                                                      float eps, float* __restrict__ amax) {
   const int row = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (row >= M) return;
@@ -181,11 +183,21 @@ __global__ void __launch_bounds__(256) rmsnorm_kernel(const float* __restrict__ 
   ss = warp_sum(ss);
   const float r = rsqrtf(ss / (float)C + eps);
   uint2* o = reinterpret_cast<uint2*>(out + (int64_t)row * C);
+  uint32_t om = 0;
 #pragma unroll
   for (int j = 0; j < NV; ++j) {
     const int i = j * 32 + lane;
-    if (i < n4)
-      o[i] = make_uint2(Half<F16>::pack2(v[j].x * r, v[j].y * r), Half<F16>::pack2(v[j].z * r, v[j].w * r));
+    if (i < n4) {
+      const float a = v[j].x * r, b = v[j].y * r, c = v[j].z * r, d = v[j].w * r;
+      o[i] = make_uint2(Half<F16>::pack2(a, b), Half<F16>::pack2(c, d));
+      if (amax)
+        om = max(max(om, max(__float_as_uint(a) & 0x7FFFFFFFu, __float_as_uint(b) & 0x7FFFFFFFu)),
+                 max(__float_as_uint(c) & 0x7FFFFFFFu, __float_as_uint(d) & 0x7FFFFFFFu));
+    }
+  }
+  if (amax) {
+    om = __reduce_max_sync(0xFFFFFFFFu, om);
+    if (lane == 0) fold_amax(amax, stored_abs_bits<F16>(om));
   }
 }
 
@@ -193,7 +205,7 @@ __global__ void __launch_bounds__(256) rmsnorm_kernel(const float* __restrict__ 
 template <bool F16>
 __global__ void __launch_bounds__(256) rmsnorm_wide_kernel(const float* __restrict__ x,
                                                            uint16_t* __restrict__ out, int M, int C,
-                                                           float eps) {
+                                                           float eps, float* __restrict__ amax) {
   const int row = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (row >= M) return;
@@ -207,9 +219,17 @@ __global__ void __launch_bounds__(256) rmsnorm_wide_kernel(const float* __restri
   ss = warp_sum(ss);
   const float r = rsqrtf(ss / (float)C + eps);
   uint2* o = reinterpret_cast<uint2*>(out + (int64_t)row * C);
+  uint32_t om = 0;
   for (int i = lane; i < n4; i += 32) {
     const float4 a = xr[i];
-    o[i] = make_uint2(Half<F16>::pack2(a.x * r, a.y * r), Half<F16>::pack2(a.z * r, a.w * r));
+    const float p = a.x * r, q = a.y * r, u = a.z * r, w = a.w * r;
+    o[i] = make_uint2(Half<F16>::pack2(p, q), Half<F16>::pack2(u, w));
+    om = max(max(om, max(__float_as_uint(p) & 0x7FFFFFFFu, __float_as_uint(q) & 0x7FFFFFFFu)),
+             max(__float_as_uint(u) & 0x7FFFFFFFu, __float_as_uint(w) & 0x7FFFFFFFu));
+  }
+  if (amax) {
+    om = __reduce_max_sync(0xFFFFFFFFu, om);
+    if (lane == 0) fold_amax(amax, stored_abs_bits<F16>(om));
   }
 }
 
@@ -621,26 +641,26 @@ nc_status rmsnorm_mix_launch(float* x, const float* x0, const float* lam_r, cons
 }
 
 template <bool F16>
-static void rmsnorm_dispatch(const float* x, uint16_t* out, int M, int C, float eps,
+static void rmsnorm_dispatch(const float* x, uint16_t* out, int M, int C, float eps, float* amax,
                              cudaStream_t stream) {
   const int grid = (M + 7) / 8;
   if (C <= 32 * 4 * 4)
-    rmsnorm_kernel<4, F16><<<grid, 256, 0, stream>>>(x, out, M, C, eps);
+    rmsnorm_kernel<4, F16><<<grid, 256, 0, stream>>>(x, out, M, C, eps, amax);
   else if (C <= 32 * 4 * 8)
-    rmsnorm_kernel<8, F16><<<grid, 256, 0, stream>>>(x, out, M, C, eps);
+    rmsnorm_kernel<8, F16><<<grid, 256, 0, stream>>>(x, out, M, C, eps, amax);
   else if (C <= 32 * 4 * 16)
-    rmsnorm_kernel<16, F16><<<grid, 256, 0, stream>>>(x, out, M, C, eps);
+    rmsnorm_kernel<16, F16><<<grid, 256, 0, stream>>>(x, out, M, C, eps, amax);
   else
-    rmsnorm_wide_kernel<F16><<<grid, 256, 0, stream>>>(x, out, M, C, eps);
+    rmsnorm_wide_kernel<F16><<<grid, 256, 0, stream>>>(x, out, M, C, eps, amax);
 }
 
 nc_status rmsnorm_launch(const float* x, uint16_t* out, int M, int C, float eps, bool f16,
-                         cudaStream_t stream) {
+                         cudaStream_t stream, float* amax) {
   if (M == 0) return NC_OK;
   if (f16)
-    rmsnorm_dispatch<true>(x, out, M, C, eps, stream);
+    rmsnorm_dispatch<true>(x, out, M, C, eps, amax, stream);
   else
-    rmsnorm_dispatch<false>(x, out, M, C, eps, stream);
+    rmsnorm_dispatch<false>(x, out, M, C, eps, amax, stream);
   return last_error();
 }
 

@@ -62,7 +62,8 @@ typedef enum {
 /* 16-bit storage formats. */
 typedef enum {
   NC_BF16 = 0, /* bfloat16: 8 significant bits, fp32 range                     */
-  NC_F16 = 1   /* IEEE binary16: 11 significant bits, |x| <= 65504 (saturating) */
+  NC_F16 = 1,  /* IEEE binary16: 11 significant bits, |x| <= 65504 (saturating) */
+  NC_F32 = 2   /* fp32: accepted only as the source of nc_fp8_quantize          */
 } nc_dtype;
 
 /* Bits of the device status word. */
@@ -90,6 +91,17 @@ typedef enum {
                                        n_layer / 2 mixes in x0)                                   */
 #define NC_EXTRA_ALL 0xFu
 
+/* nc_config.fp8: dynamic tensorwise FP8 ("Nanochat与nanoGPT对比：关键升级" §1,
+ * architecture table, FP8-training row).  Each operand of a chosen matrix
+ * product -- the activation entering it and the fp32 master weight -- is
+ * quantised as a whole tensor: amax = max |x|, s = 448 / max(amax, 1e-12) in
+ * fp32, codes = e4m3(x * s) rounded to nearest even and saturated at +-448; the
+ * fp32 product of the codes is multiplied by 1 / (s_a s_w). */
+#define NC_FP8_BLOCK 0x1u   /* the six block projections c_q, c_k, c_v, attention
+                               c_proj, c_fc, MLP c_proj                          */
+#define NC_FP8_LM_HEAD 0x2u /* the LM head                                       */
+#define NC_FP8_ALL 0x3u
+
 /* Model configuration.  "从文本到聊天模型" §5.1: d_model = depth * aspect_ratio,
  * n_head = d_model / head_dim.  window_pattern: one char per layer, cycled;
  * 'S' = short window (short_window keys), 'L' = full context; the last layer is
@@ -114,6 +126,7 @@ typedef struct {
                                 are held in fp16 (exact for |w| >= 2^-14) so
                                 both tensor-core operands share one format. */
   uint32_t extras;           /* NC_EXTRA_* bits (0: the plain block stack)    */
+  uint32_t fp8;              /* NC_FP8_* bits (0: every product in 16-bit)    */
 } nc_config;
 
 /* fp32 master weights (device pointers; the per-layer members are HOST arrays
@@ -143,7 +156,7 @@ typedef struct {
 /* Fills *out from the depth knob ("从文本到聊天模型" §5.1): d_model =
  * depth*aspect_ratio, n_head = d_model/head_dim, n_kv_head = n_kv_head or
  * n_head when 0, pattern "SSSL", short_window = seq_len/4, softcap 15,
- * norm_eps 1e-6, rope_base 10000, act_dtype NC_F16, extras 0.  Host only; touches no
+ * norm_eps 1e-6, rope_base 10000, act_dtype NC_F16, extras 0, fp8 0.  Host only; touches no
  * device. */
 nc_status nc_init_config(nc_config* out, int depth, int aspect_ratio, int head_dim,
                          int n_kv_head, int seq_len, int vocab);
@@ -206,8 +219,8 @@ nc_status nc_forward(const nc_config* cfg, const nc_weights* w, const int32_t* t
  *     head-dimension order) then the v heads,
  *   the scratch of one decode step, and the device status word (first 4
  *     bytes, cleared by every call).
- * The KV-cache path covers the plain block stack: cfg->extras must be 0
- * (NC_ERR_CONFIG otherwise).  Decode attention needs n_head / n_kv_head in
+ * The KV-cache path covers the plain block stack in 16-bit: cfg->extras and
+ * cfg->fp8 must be 0 (NC_ERR_CONFIG otherwise).  Decode attention needs n_head / n_kv_head in
  * {1, 2, 4, 8} (NC_ERR_SHAPE otherwise).  T_max <= cfg->seq_len. */
 
 /* Session bytes for B rows of up to T_max positions (0 on bad input).  Host only. */
@@ -253,7 +266,8 @@ typedef enum {
   NC_K_GEMM_LM_HEAD = 10,
   NC_K_CE_FINALIZE = 11,
   NC_K_LOSS_MEAN = 12,
-  NC_K_COUNT = 13
+  NC_K_FP8_QUANT = 13,  /* amax + e4m3 quantisation of one activation (2 launches) */
+  NC_K_COUNT = 14
 } nc_kernel_kind;
 
 /* Per-launch timing hook.  `events` holds 2*capacity cudaEvent_t handles
@@ -354,6 +368,24 @@ typedef enum {
 nc_status nc_linear(const uint16_t* a, const uint16_t* w, void* out, int M, int N, int K,
                     int64_t ldo, nc_epilogue epilogue, float cap, nc_dtype dtype,
                     uint32_t* dev_status, void* stream);
+
+/* Dynamic tensorwise e4m3 quantisation of one tensor (the NC_FP8_* rule
+ * above): x [n] in src_dtype (NC_F32, NC_BF16 or NC_F16; device, 16-byte
+ * aligned), n % 16 == 0.  Writes *amax (one device float; the call zeroes it
+ * first) and then codes [n] (device, 16-byte aligned), in stream order.  Two
+ * launches. */
+nc_status nc_fp8_quantize(const void* x, nc_dtype src_dtype, int64_t n, uint8_t* codes, float* amax,
+                          void* stream);
+
+/* out = epilogue((a @ w^T) / (s_a s_w)) with e4m3 codes a [M, K] and w [N, K]
+ * (row-major, device, 16-byte aligned) and their tensors' amax values amax_a,
+ * amax_w (one device float each, as nc_fp8_quantize writes them; s = 448 /
+ * max(amax, 1e-12)).  tcgen05.mma kind::f8f6f4, fp32 accumulation in tensor
+ * memory.  16-bit outputs are in format dtype (NC_BF16 or NC_F16).  K % 16 ==
+ * 0, N % 32 == 0, ldo as for nc_linear. */
+nc_status nc_linear_fp8(const uint8_t* a, const float* amax_a, const uint8_t* w, const float* amax_w,
+                        void* out, int M, int N, int K, int64_t ldo, nc_epilogue epilogue, float cap,
+                        nc_dtype dtype, uint32_t* dev_status, void* stream);
 
 /* Fused Q/K/V projection ("从文本到聊天模型" §5.4) + RoPE + QK-norm
  * ("Nanochat与nanoGPT对比" §1) in one GEMM: qkv = a @ w^T with w the

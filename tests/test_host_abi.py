@@ -233,3 +233,51 @@ def test_kv_cache_host_rules(nclib):
     if not torch.cuda.is_available():
         assert dec(cfg, 5) == 8          # valid arguments, no sm_100 device
         assert pre(100) == 8
+
+
+def test_fp8_host_rules(nclib):
+    """nc_config.fp8: accepted bits, workspace sizing, and the host-side
+    refusals of the standalone e4m3 entry points and of the KV-cache path."""
+    L = nclib.lib()
+    cfg = nclib.init_config(2, 64, 64, 0, 256, 512)
+    assert cfg.fp8 == 0
+    base = nclib.workspace_bytes(cfg, 2, 100)
+    for bits in (nclib.FP8_BLOCK, nclib.FP8_LM_HEAD, nclib.FP8_ALL):
+        c = nclib.NcConfig.from_buffer_copy(cfg)
+        c.fp8 = bits
+        assert nclib.check_config(c) == 0
+        assert nclib.workspace_bytes(c, 2, 100) > 0
+    c = nclib.NcConfig.from_buffer_copy(cfg)
+    c.fp8 = 4
+    assert nclib.check_config(c) == 2
+    assert nclib.workspace_bytes(c, 2, 100) == 0
+    # e4m3 block weights take one byte instead of two; the a8 / amax scratch is M x 4C bytes + slots
+    c.fp8 = nclib.FP8_BLOCK
+    C, L_ = cfg.d_model, cfg.n_layer
+    wblock = L_ * ((cfg.n_head + 2 * cfg.n_kv_head) * cfg.head_dim * C + C * cfg.n_head * cfg.head_dim + 8 * C * C)
+    M = 200
+    assert nclib.workspace_bytes(c, 2, 100) - base >= M * 4 * C - wblock - 4096
+    # the KV-cache path is 16-bit only
+    n = L.nc_session_bytes(ctypes.byref(cfg), 2, 256)
+    fw = _FakeWeights(nclib, 2)
+    assert L.nc_decode_step(ctypes.byref(c), ctypes.byref(fw.w), 1 << 41, 2, 5, 1 << 44, 1 << 43, n, 256, None) == 2
+    assert L.nc_prefill(ctypes.byref(c), ctypes.byref(fw.w), 1 << 41, 2, 10, None, 1 << 43, n, 256,
+                        1 << 42, 1 << 30, None) == 2
+    # standalone entry points: argument checks before any device work
+    q = lambda x, dt, n, codes, amax: L.nc_fp8_quantize(x, dt, n, codes, amax, None)
+    assert q(None, nclib.F32, 16, 1 << 40, 1 << 41) == 1
+    assert q(1 << 40, 7, 16, 1 << 40, 1 << 41) == 1      # bad source dtype
+    assert q(1 << 40, nclib.F32, 24, 1 << 40, 1 << 41) == 3  # n % 16
+    assert q((1 << 40) + 8, nclib.BF16, 16, 1 << 40, 1 << 41) == 4
+    lin = lambda M, N, K, ldo, epi=0, dt=nclib.F16: L.nc_linear_fp8(1 << 40, 1 << 41, 1 << 42, 1 << 43, 1 << 44,
+                                                                   M, N, K, ldo, epi, 15.0, dt, None, None)
+    assert lin(128, 64, 8, 64) == 1      # K < 16
+    assert lin(128, 64, 40, 64) == 3     # K % 16
+    assert lin(128, 48, 64, 64) == 3     # N % 32
+    assert lin(128, 64, 64, 32) == 3     # ldo < N
+    assert lin(128, 64, 64, 64, epi=9) == 1
+    assert lin(128, 64, 64, 64, dt=nclib.F32) == 1  # 16-bit outputs only
+    import torch
+    if not torch.cuda.is_available():
+        assert lin(128, 64, 64, 64) == 8
+        assert q(1 << 40, nclib.F32, 16, 1 << 40, 1 << 41) == 8
