@@ -60,6 +60,12 @@ one-line descriptions there:
 
 Those pins live in ``tests/test_oracle_extras.py``.
 
+Backward ("从文本到聊天模型" §6.5: the training step's loss.backward()):
+``oracle.grad.forward_backward`` gives the mean loss of the plain stack and its
+gradient with respect to every fp32 master weight, the bf16 cast taken as
+straight-through; pinned in ``tests/test_oracle_grad.py`` by finite
+differences and torch float64 autograd.
+
 FP8 ("Nanochat与nanoGPT对比" §1 table, FP8-training row: dynamic tensor-level
 e4m3/e5m2): ``forward(..., fp8="block" | "all")`` runs the block projections
 (and with "all" the LM head) through dynamic tensorwise e4m3; the readings are

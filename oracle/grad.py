@@ -1,0 +1,183 @@
+"""fp64 backward of the nanochat block stack: the training micro-step's
+``loss.backward()``.
+
+TEST INFRASTRUCTURE ONLY (see the package docstring for who may import it).
+
+"从文本到聊天模型" §6.5 (training loop: forward, loss, backward, optimizer
+step) puts the backward right after the loss the forward computes.  This
+module gives, for the plain block stack of ``model.forward`` (no extras, no
+fp8), the mean loss and its gradient with respect to every fp32 master weight:
+wte, lm_head and, per layer, c_q, c_k, c_v, attn_proj, c_fc, mlp_proj.
+
+Readings where the pages are silent:
+
+* The fp32 -> bf16 cast of a weight at matmul time passes the gradient
+  through unchanged to the fp32 master weight (a straight-through cast, as
+  autocast does): dW = dY^T X, and the backward products use the same bf16
+  weight values as the forward.
+* The loss is the mean over targets != -1; ignored positions get no gradient.
+* Embedding rows collect the gradient of every position holding their token.
+
+The backward is derived step by step from the forward's definitions, in the
+forward's notation, the steps in reverse order.  ``cast`` lets a test swap the
+bf16 cast for the identity (finite differences need a loss that is smooth in
+the weights).  The pins are in ``tests/test_oracle_grad.py``.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+from .model import F64, OracleConfig, embed, layer_windows, rope_tables, to_bf16
+
+
+def _rms_rstd(u, eps):
+    return 1.0 / np.sqrt(np.mean(u * u, axis=-1, keepdims=True) + eps)
+
+
+def rmsnorm_backward(y, r, dy):
+    """y = u r with r = (mean(u^2) + eps)^(-1/2) per row: du = r (dy - y mean(dy y))."""
+    return r * (dy - y * np.mean(dy * y, axis=-1, keepdims=True))
+
+
+def _rope_apply(u, cos, sin, sign):
+    """Rotate pairs (u_i, u_{i+D/2}) by sign * t * theta_i (u: [B, T, heads, D])."""
+    D = u.shape[-1]
+    h = D // 2
+    c = cos[None, :, None, :]
+    s = sign * sin[None, :, None, :]
+    a, b = u[..., :h], u[..., h:]
+    return np.concatenate([a * c - b * s, a * s + b * c], axis=-1)
+
+
+def _mask(T, W):
+    i = np.arange(T)[:, None]
+    j = np.arange(T)[None, :]
+    return (j <= i) & ((i - j) < W)
+
+
+def _forward(cfg: OracleConfig, weights: dict, idx: np.ndarray, targets: np.ndarray, cast):
+    """The forward of ``model.forward`` (plain stack) keeping what the backward reads."""
+    idx = np.asarray(idx)
+    targets = np.asarray(targets)
+    B, T = idx.shape
+    C, H, Hkv, D = cfg.d_model, cfg.n_head, cfg.n_kv_head, cfg.head_dim
+    G = H // Hkv
+    eps, cap = cfg.norm_eps, cfg.softcap
+    windows = layer_windows(cfg)
+    cos, sin = rope_tables(T, D, cfg.rope_base)
+    scale = 1.0 / np.sqrt(D)
+    Wb = [{k: cast(v) for k, v in lw.items()} for lw in weights["layers"]]
+    Wlm = cast(weights["lm_head"])
+
+    # ---------------- forward, keeping what the backward reads
+    x = embed(weights["wte"], idx)
+    saved = []
+    for l, lw in enumerate(Wb):
+        s = {"x_in": x}
+        r1 = _rms_rstd(x, eps)
+        a = x * r1
+        uq = (a @ lw["c_q"].T).reshape(B, T, H, D)
+        uk = (a @ lw["c_k"].T).reshape(B, T, Hkv, D)
+        v = (a @ lw["c_v"].T).reshape(B, T, Hkv, D)
+        pq = _rope_apply(uq, cos, sin, 1.0)
+        pk = _rope_apply(uk, cos, sin, 1.0)
+        rq, rk = _rms_rstd(pq, eps), _rms_rstd(pk, eps)
+        q, k = pq * rq, pk * rk
+        m = _mask(T, windows[l])
+        P = np.empty((B, H, T, T))
+        o = np.empty((B, T, H, D))
+        for h in range(H):
+            g = h // G
+            sc = np.einsum("bid,bjd->bij", q[:, :, h], k[:, :, g]) * scale
+            sc = np.where(m[None], sc, -np.inf)
+            sc = sc - sc.max(axis=-1, keepdims=True)
+            e = np.exp(sc)
+            P[:, h] = e / e.sum(axis=-1, keepdims=True)
+            o[:, :, h] = np.einsum("bij,bjd->bid", P[:, h], v[:, :, g])
+        of = o.reshape(B, T, H * D)
+        x_mid = x + of @ lw["attn_proj"].T
+        r2 = _rms_rstd(x_mid, eps)
+        a2 = x_mid * r2
+        u = a2 @ lw["c_fc"].T
+        hh = np.maximum(u, 0.0) ** 2
+        x = x_mid + hh @ lw["mlp_proj"].T
+        s.update(r1=r1, a=a, q=q, k=k, v=v, rq=rq, rk=rk, P=P, of=of, x_mid=x_mid, r2=r2, a2=a2, u=u, h=hh)
+        saved.append(s)
+    rf = _rms_rstd(x, eps)
+    af = x * rf
+    z = af @ Wlm.T
+    lg = cap * np.tanh(z / cap)
+    mx = lg.max(axis=-1, keepdims=True)
+    lse = mx[..., 0] + np.log(np.exp(lg - mx).sum(axis=-1))
+    valid = targets != -1
+    n = int(valid.sum())
+    tl = np.where(valid, lse - np.take_along_axis(lg, np.where(valid, targets, 0)[..., None], -1)[..., 0], 0.0)
+    loss = float(tl.sum() / n) if n else float("nan")
+    return loss, dict(saved=saved, Wb=Wb, Wlm=Wlm, lg=lg, lse=lse, valid=valid, n=n, af=af, rf=rf, cos=cos,
+                      sin=sin, idx=idx, targets=targets)
+
+
+def forward_backward(cfg: OracleConfig, weights: dict, idx: np.ndarray, targets: np.ndarray, cast=to_bf16):
+    """Returns (loss, grads) with grads = {"wte", "lm_head", "layers": [{...}]},
+    each the same shape as its weight, float64."""
+    loss, c = _forward(cfg, weights, idx, targets, cast)
+    saved, Wb, Wlm, lg, lse, valid, n = c["saved"], c["Wb"], c["Wlm"], c["lg"], c["lse"], c["valid"], c["n"]
+    af, rf, cos, sin, idx, targets = c["af"], c["rf"], c["cos"], c["sin"], c["idx"], c["targets"]
+    B, T = idx.shape
+    C, H, Hkv, D = cfg.d_model, cfg.n_head, cfg.n_kv_head, cfg.head_dim
+    G = H // Hkv
+    cap = cfg.softcap
+    scale = 1.0 / np.sqrt(D)
+
+    # ---------------- backward
+    grads = {"layers": [dict() for _ in Wb]}
+    p = np.exp(lg - lse[..., None])
+    onehot = np.zeros_like(lg)
+    bi, ti = np.nonzero(valid)
+    onehot[bi, ti, targets[bi, ti]] = 1.0
+    dlg = np.where(valid[..., None], (p - onehot) / max(n, 1), 0.0)
+    dz = dlg * (1.0 - (lg / cap) ** 2)  # d/dz cap tanh(z / cap)
+    grads["lm_head"] = np.einsum("btv,btc->vc", dz, af)
+    daf = dz @ Wlm
+    dx = rmsnorm_backward(af, rf, daf)
+    for l in range(len(Wb) - 1, -1, -1):
+        lw, s, gl = Wb[l], saved[l], grads["layers"][l]
+        # MLP: x = x_mid + relu(u)^2 W_mp^T with u = norm(x_mid) W_fc^T
+        gl["mlp_proj"] = np.einsum("btc,btf->cf", dx, s["h"])
+        dh = dx @ lw["mlp_proj"]
+        du = dh * 2.0 * np.maximum(s["u"], 0.0)
+        gl["c_fc"] = np.einsum("btf,btc->fc", du, s["a2"])
+        da2 = du @ lw["c_fc"]
+        dx_mid = dx + rmsnorm_backward(s["a2"], s["r2"], da2)
+        # attention block: x_mid = x_in + o W_p^T
+        gl["attn_proj"] = np.einsum("btc,bte->ce", dx_mid, s["of"])
+        do = (dx_mid @ lw["attn_proj"]).reshape(B, T, H, D)
+        dq = np.zeros((B, T, H, D))
+        dk = np.zeros((B, T, Hkv, D))
+        dv = np.zeros((B, T, Hkv, D))
+        for h in range(H):
+            g = h // G
+            Ph = s["P"][:, h]
+            dv[:, :, g] += np.einsum("bij,bid->bjd", Ph, do[:, :, h])
+            dP = np.einsum("bid,bjd->bij", do[:, :, h], s["v"][:, :, g])
+            dS = Ph * (dP - np.sum(dP * Ph, axis=-1, keepdims=True)) * scale
+            dq[:, :, h] = np.einsum("bij,bjd->bid", dS, s["k"][:, :, g])
+            dk[:, :, g] += np.einsum("bij,bid->bjd", dS, s["q"][:, :, h])
+        # QK-norm after RoPE, then the inverse rotation
+        duq = _rope_apply(rmsnorm_backward(s["q"], s["rq"], dq), cos, sin, -1.0).reshape(B, T, H * D)
+        duk = _rope_apply(rmsnorm_backward(s["k"], s["rk"], dk), cos, sin, -1.0).reshape(B, T, Hkv * D)
+        dvf = dv.reshape(B, T, Hkv * D)
+        gl["c_q"] = np.einsum("bte,btc->ec", duq, s["a"])
+        gl["c_k"] = np.einsum("bte,btc->ec", duk, s["a"])
+        gl["c_v"] = np.einsum("bte,btc->ec", dvf, s["a"])
+        da = duq @ lw["c_q"] + duk @ lw["c_k"] + dvf @ lw["c_v"]
+        dx = dx_mid + rmsnorm_backward(s["a"], s["r1"], da)
+    dwte = np.zeros(np.asarray(weights["wte"]).shape, dtype=F64)
+    np.add.at(dwte, idx.reshape(-1), dx.reshape(-1, C))
+    grads["wte"] = dwte
+    return loss, grads
+
+
+def loss_only(cfg: OracleConfig, weights: dict, idx, targets, cast=to_bf16) -> float:
+    """The same loss without the backward (for finite differences)."""
+    return _forward(cfg, weights, idx, targets, cast)[0]
