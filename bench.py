@@ -558,6 +558,133 @@ def run_decode(args, s):
         torch.distributed.destroy_process_group()
 
 
+def run_train(args, s):
+    """Training micro-step: forward + loss + backward (gradients of every weight)
+    on the workload's [B, T] batch; the optimizer step is out of scope."""
+    import torch
+
+    import decoder_only_transformer_nc_b200 as nc
+    from decoder_only_transformer_nc_b200 import dp
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import torch.distributed as dist
+        from datetime import timedelta
+        dist.init_process_group("nccl", device_id=dev, timeout=timedelta(seconds=120))
+    cfg = nc.make_config(s.n_layer, s.d_model, s.n_head, s.n_kv_head, s.head_dim, s.seq_len, s.vocab,
+                         s.short_window)
+    weights = make_weights(s)
+    model = nc.Model.from_numpy(cfg, weights, device=dev)
+    B, T = s.batch, s.seq_len
+    x, y = make_tokens(s, seed=dp.shard_seed(TOKEN_SEED, rank))
+    tx, ty = torch.from_numpy(x).to(dev), torch.from_numpy(y).to(dev)
+    ws = torch.empty(nc.train_workspace_bytes(cfg, B, T), dtype=torch.uint8, device=dev)
+    loss = torch.empty((), dtype=torch.float32, device=dev)
+    _, grads, _ = nc.forward_backward(model, tx, ty, workspace=ws, loss=loss)
+    for _ in range(args.warmup - 1):
+        nc.forward_backward(model, tx, ty, grads=grads, workspace=ws, loss=loss)
+    torch.cuda.synchronize()
+    if nc.get_status(ws) != 0:
+        raise SystemExit(f"device status after warm-up: {nc.get_status(ws)}")
+    n_entries = 12 + 24 * s.n_layer
+    traces = [nc.LaunchTrace(n_entries) for _ in range(args.steps)]
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier(device_ids=[local])
+
+    stream = torch.cuda.current_stream()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clocks:
+        t0.record(stream)
+        for k in range(args.steps):
+            nc.forward_backward(model, tx, ty, grads=grads, workspace=ws, loss=loss, trace=traces[k])
+        t1.record(stream)
+        torch.cuda.synchronize()
+    barrier()
+    ms = t0.elapsed_time(t1) / args.steps
+    per_kind = {}
+    for tr in traces:
+        for kind, kms in tr.launches():
+            d = per_kind.setdefault(kind, [0.0, 0])
+            d[0] += kms
+            d[1] += 1
+        tr.close()
+    # e2e: tokens and targets from pinned host memory in, the loss out, every step
+    hx, hy = torch.from_numpy(x).pin_memory(), torch.from_numpy(y).pin_memory()
+    dx, dy = torch.empty_like(tx), torch.empty_like(ty)
+    hloss = torch.empty((), dtype=torch.float32).pin_memory()
+    barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        dx.copy_(hx, non_blocking=True)
+        dy.copy_(hy, non_blocking=True)
+        nc.forward_backward(model, dx, dy, grads=grads, workspace=ws, loss=loss)
+        hloss.copy_(loss, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = e0.elapsed_time(e1) / args.steps
+    if world > 1:
+        tt = torch.tensor([ms, e2e_ms], dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
+        ms, e2e_ms = float(tt[0]), float(tt[1])
+    status = nc.get_status(ws)
+    fwd_flops = nc.forward_flops(cfg, B, T)
+    M = B * T
+    C, H, Hkv, D, V = s.d_model, s.n_head, s.n_kv_head, s.head_dim, s.vocab
+    proj = 2.0 * M * s.n_layer * (C * (H + 2 * Hkv) * D + H * D * C + 8 * C * C)  # block projections
+    head = 2.0 * M * C * V
+    attn_fwd = fwd_flops - proj - head
+    # algorithmic FLOPs of one launch of each backward kind
+    work = {"gemm_dgrad": (proj + head) / (4 * s.n_layer + 1), "gemm_wgrad": (proj + head) / (4 * s.n_layer + 1),
+            "ce_bwd": head, "attn_bwd": 2.5 * attn_fwd / s.n_layer}
+    peaks, peak_src = load_peaks()
+    peak = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+    total = sum(v[0] for v in per_kind.values())
+    kernels = {}
+    for k, (kms, n) in sorted(per_kind.items(), key=lambda kv: -kv[1][0]):
+        ent = {"launches": n, "ms_total": round(kms, 3), "share": round(kms / total, 4)}
+        if k in work:
+            ent["tflops"] = round(work[k] * n / (kms / 1e3) / 1e12, 1)
+        kernels[k] = ent
+    top = max((k for k in work if k in per_kind), key=lambda k: per_kind[k][0])
+    top_ach = work[top] * per_kind[top][1] / (per_kind[top][0] / 1e3) / 1e12
+    if rank == 0:
+        train_flops = 3.0 * fwd_flops
+        print(json.dumps({
+            "metric": "forward+backward tokens/sec at d20 (1xB200), training micro-step without the optimizer",
+            "value": world * M / (ms / 1e3), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": DTYPE_NOTE, "data": "synthetic",
+            "config": {"workload": f"{s.name} train", "global_batch": world * B, "seq_len": T,
+                       "parallelism": f"dp{world}" if world > 1 else "none",
+                       "l2": "inputs larger than L2 (saved activations ~40 GB per step)"},
+            "tflops_3x_forward": round(train_flops * world / (ms / 1e3) / 1e12, 1),
+            "roofline": {"kernel": top, "bound": "tensor", "achieved": round(top_ach, 1), "peak": peak,
+                         "peak_kind": f"bf16_tflops_sustained ({peak_src})", "unit": "TFLOP/s",
+                         "frac": round(top_ach / peak, 4), "traffic": None,
+                         "launches": per_kind[top][1], "avg_launch_ms": round(per_kind[top][0] / per_kind[top][1], 4)},
+            "kernels": kernels,
+            "gpu_launches": n_entries * args.steps,  # 2 L copies launch no kernel; attention bwd is 3 per layer
+            "e2e": {"value": world * M / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": int(x.nbytes + y.nbytes),
+                    "d2h_bytes_per_step": 4},
+            "clocks": clocks.summary(),
+            "device_status": nc.STATUS_NAMES.get(status, status),
+        }), flush=True)
+    if world > 1:
+        torch.distributed.barrier(device_ids=[local])
+        torch.distributed.destroy_process_group()
+
+
 def _flat(w):
     yield w["wte"]
     yield w["lm_head"]
@@ -577,7 +704,7 @@ def main():
     ap.add_argument("--ref-prefix", type=int, default=256,
                     help="positions of batch row 0 per step of the reference (oracle) arm")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--mode", default="forward", choices=["forward", "decode"],
+    ap.add_argument("--mode", default="forward", choices=["forward", "decode", "train"],
                     help="decode: KV-cache decode steps after a prefill of --prompt tokens")
     ap.add_argument("--prompt", type=int, default=1024, help="decode mode: prompt length")
     ap.add_argument("--fp8", default="none", choices=["none", "block", "all"],
@@ -600,6 +727,8 @@ def main():
         run_reference(args, s)
     elif args.mode == "decode":
         run_decode(args, s)
+    elif args.mode == "train":
+        run_train(args, s)
     else:
         run_ours(args, s)
 

@@ -20,6 +20,8 @@ __all__ = [
     "rmsnorm", "rope_table", "rope_qknorm", "attention", "linear", "qkv_rope", "softcap_ce",
     "loss_mean", "cast_weights", "selftest_bounded_wait", "BF16", "F16", "F32",
     "fp8_quantize", "linear_fp8", "FP8_BLOCK", "FP8_LM_HEAD", "FP8_ALL",
+    "train_workspace_bytes", "forward_backward", "linear_dgrad", "linear_wgrad", "attention_lse",
+    "attention_backward",
     "EPI_STORE_16", "EPI_RELU2_16", "EPI_RESID_F32", "EPI_STORE_F32", "EPI_SOFTCAP_F32",
 ]
 
@@ -67,6 +69,11 @@ class NcWeights(ctypes.Structure):
                 ("backout_lambda", ctypes.c_void_p)]
 
 
+class NcGrads(ctypes.Structure):
+    _fields_ = [("wte", ctypes.c_void_p), ("c_q", _FPP), ("c_k", _FPP), ("c_v", _FPP),
+                ("attn_proj", _FPP), ("c_fc", _FPP), ("mlp_proj", _FPP), ("lm_head", ctypes.c_void_p)]
+
+
 # Further terms of the full nanochat forward (bits of NcConfig.extras).
 EXTRA_SMEAR, EXTRA_VALUE_EMBED, EXTRA_RESID_LAMBDAS, EXTRA_BACKOUT = 1, 2, 4, 8
 EXTRA_ALL = 15
@@ -83,7 +90,8 @@ class NcTrace(ctypes.Structure):
 
 KERNEL_KINDS = ("rope_table", "cast", "embedding", "rmsnorm", "gemm_qkv", "rope_qknorm", "attention",
                 "gemm_attn_proj", "gemm_fc", "gemm_mlp_proj", "gemm_lm_head", "ce_finalize", "loss_mean",
-                "fp8_quant")
+                "fp8_quant", "copy", "ce_bwd", "gemm_dgrad", "gemm_wgrad", "norm_bwd", "attn_bwd", "qk_bwd",
+                "emb_bwd")
 
 _lib = None
 
@@ -123,6 +131,15 @@ def lib():
             "nc_attention_strided": (i32, [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i64, i64, i32, vp]),
             "nc_linear": (i32, [vp, vp, vp, i32, i32, i32, i64, i32, f32, i32, vp, vp]),
             "nc_fp8_quantize": (i32, [vp, i32, i64, vp, vp, vp]),
+            "nc_train_workspace_bytes": (sz, [cfgp, i32, i32]),
+            "nc_forward_backward": (i32, [cfgp, ctypes.POINTER(NcWeights), vp, vp, i32, i32, vp,
+                                          ctypes.POINTER(NcGrads), vp, sz, vp]),
+            "nc_forward_backward_traced": (i32, [cfgp, ctypes.POINTER(NcWeights), vp, vp, i32, i32, vp,
+                                                 ctypes.POINTER(NcGrads), vp, sz, vp, ctypes.POINTER(NcTrace)]),
+            "nc_attention_lse": (i32, [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i64, i64, i32, vp]),
+            "nc_attention_backward": (i32, [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, vp]),
+            "nc_linear_dgrad": (i32, [vp, vp, vp, i32, i32, i32, i32, i32, vp, vp]),
+            "nc_linear_wgrad": (i32, [vp, vp, vp, i32, i32, i32, f32, i32, vp, vp]),
             "nc_linear_fp8": (i32, [vp, vp, vp, vp, vp, i32, i32, i32, i64, i32, f32, i32, vp, vp]),
             "nc_qkv_rope": (i32, [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, f32, i32, vp, vp]),
             "nc_softcap_ce": (i32, [vp, vp, vp, vp, i32, i32, f32, vp, vp]),
@@ -463,6 +480,87 @@ def linear_fp8(a8, amax_a, w8, amax_w, out, epilogue, cap=15.0, dtype=F16, statu
     _check(lib().nc_linear_fp8(_ptr(a8), _ptr(amax_a), _ptr(w8), _ptr(amax_w), _ptr(out), M, N, K,
                                out.stride(0), epilogue, cap, dtype, _ptr(status), _stream(stream)),
            "nc_linear_fp8")
+
+
+def train_workspace_bytes(c: NcConfig, B: int, T: int) -> int:
+    return lib().nc_train_workspace_bytes(ctypes.byref(c), B, T)
+
+
+def forward_backward(model: Model, tokens, targets, grads: dict | None = None, workspace=None, stream=None,
+                     loss=None, trace: "LaunchTrace | None" = None):
+    """The training micro-step's forward + loss.backward() (nc_forward_backward).
+
+    tokens/targets: int32 CUDA tensors [B, T].  ``grads`` (optional) holds fp32
+    CUDA tensors in the layout of ``Model.tensors`` ("wte", "lm_head",
+    "layers": [{c_q, ...}]); the gradients are ADDED to them.  Without it,
+    zeroed tensors are made.  Returns (loss: scalar CUDA tensor, grads,
+    workspace).
+    """
+    import torch
+    cfg = model.cfg
+    B, T = tokens.shape
+    need = train_workspace_bytes(cfg, B, T)
+    if need == 0:
+        raise NcError(2, "nc_train_workspace_bytes")
+    dev = tokens.device
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    t = model.tensors
+    if grads is None:
+        z = lambda x: torch.zeros_like(x)
+        grads = {"wte": z(t["wte"]), "lm_head": z(t["lm_head"]),
+                 "layers": [{k: z(lw[k]) for k in ("c_q", "c_k", "c_v", "attn_proj", "c_fc", "mlp_proj")}
+                            for lw in t["layers"]]}
+    L = cfg.n_layer
+    arrs = [(ctypes.c_void_p * L)(*[grads["layers"][l][n].data_ptr() for l in range(L)])
+            for n in ("c_q", "c_k", "c_v", "attn_proj", "c_fc", "mlp_proj")]
+    g = NcGrads(grads["wte"].data_ptr(), *[ctypes.cast(a, _FPP) for a in arrs], grads["lm_head"].data_ptr())
+    if loss is None:
+        loss = torch.empty((), dtype=torch.float32, device=dev)
+    _check(lib().nc_forward_backward_traced(ctypes.byref(cfg), ctypes.byref(model.weights), _ptr(tokens),
+                                            _ptr(targets), B, T, _ptr(loss), ctypes.byref(g), _ptr(workspace),
+                                            workspace.numel(), _stream(stream),
+                                            None if trace is None else ctypes.byref(trace.struct)),
+           "nc_forward_backward")
+    return loss, grads, workspace
+
+
+def attention_lse(qkv, out, lse, H, Hkv, D, window, stream=None):
+    """Forward attention on a packed qkv [B, T, (H + 2 Hkv) D] tensor; out [B, T, H*D], lse [B, T, H] fp32."""
+    B, T, W = qkv.shape
+    q = qkv.view(B * T, W)
+    _check(lib().nc_attention_lse(_ptr(q), ctypes.c_void_p(q.data_ptr() + H * D * q.element_size()),
+                                  ctypes.c_void_p(q.data_ptr() + (H + Hkv) * D * q.element_size()), _ptr(out),
+                                  _ptr(lse), B, T, H, Hkv, D, window, W, W, _dt(qkv), _stream(stream)),
+           "nc_attention_lse")
+
+
+def attention_backward(qkv, o, dO, lse, dqkv, H, Hkv, D, window, delta=None, stream=None):
+    """dq | dk | dv into dqkv (qkv's packed layout) from o, dO and lse."""
+    import torch
+    B, T, _ = qkv.shape
+    if delta is None:
+        delta = torch.empty((B, T, H), dtype=torch.float32, device=qkv.device)
+    _check(lib().nc_attention_backward(_ptr(qkv), _ptr(o), _ptr(dO), _ptr(lse), _ptr(delta), _ptr(dqkv), B, T, H,
+                                       Hkv, D, window, _dt(qkv), _stream(stream)), "nc_attention_backward")
+
+
+def linear_dgrad(dy, w, dx, status=None, stream=None):
+    """dx [M, K] = dy [M, N] . w [N, K]; dx fp32 or 16-bit (same format as dy)."""
+    import torch
+    M, N = dy.shape
+    K = w.shape[1]
+    epi = EPI_STORE_F32 if dx.dtype == torch.float32 else EPI_STORE_16
+    _check(lib().nc_linear_dgrad(_ptr(dy), _ptr(w), _ptr(dx), M, N, K, epi, _dt(dy), _ptr(status),
+                                 _stream(stream)), "nc_linear_dgrad")
+
+
+def linear_wgrad(dy, x, dw, alpha=1.0, status=None, stream=None):
+    """dw [N, K] += alpha dy [M, N]^T . x [M, K] (fp32)."""
+    M, N = dy.shape
+    K = x.shape[1]
+    _check(lib().nc_linear_wgrad(_ptr(dy), _ptr(x), _ptr(dw), M, N, K, alpha, _dt(dy), _ptr(status),
+                                 _stream(stream)), "nc_linear_wgrad")
 
 
 def qkv_rope(a, w, out, table, T, H, Hkv, D, eps=1e-6, status=None, stream=None):

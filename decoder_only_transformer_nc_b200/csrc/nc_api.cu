@@ -404,6 +404,33 @@ nc_status nc_attention_strided(const uint16_t* q, const uint16_t* k, const uint1
                           dtype == NC_F16, nullptr, S(stream));
 }
 
+nc_status nc_attention_lse(const uint16_t* q, const uint16_t* k, const uint16_t* v, uint16_t* out, float* lse,
+                           int B, int T, int H, int Hkv, int D, int window, int64_t q_row_stride,
+                           int64_t kv_row_stride, nc_dtype dtype, void* stream) {
+  if (!q || !k || !v || !out || !lse || B < 0 || T < 0 || H < 1 || Hkv < 1 || H % Hkv != 0 || !dtype_ok(dtype))
+    return NC_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return NC_ERR_SHAPE;
+  if (q_row_stride < (int64_t)H * D || kv_row_stride < (int64_t)Hkv * D || q_row_stride % 8 || kv_row_stride % 8)
+    return NC_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return NC_ERR_ALIGNMENT;
+  if (nc_status s = device_ok()) return s;
+  return attention_launch(q, k, v, out, B, T, H, Hkv, D, window, q_row_stride, kv_row_stride, dtype == NC_F16,
+                          nullptr, S(stream), nullptr, lse);
+}
+
+nc_status nc_attention_backward(const uint16_t* qkv, const uint16_t* o, const uint16_t* dO, const float* lse,
+                                float* delta, uint16_t* dqkv, int B, int T, int H, int Hkv, int D, int window,
+                                nc_dtype dtype, void* stream) {
+  if (!qkv || !o || !dO || !lse || !delta || !dqkv || B < 0 || T < 0 || H < 1 || Hkv < 1 || H % Hkv != 0 ||
+      !dtype_ok(dtype))
+    return NC_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return NC_ERR_SHAPE;
+  if (!aligned16(qkv) || !aligned16(o) || !aligned16(dO) || !aligned16(dqkv)) return NC_ERR_ALIGNMENT;
+  if (nc_status s = device_ok()) return s;
+  return attn_bwd_launch(qkv, (int64_t)(H + 2 * Hkv) * D, o, dO, lse, delta, dqkv, B, T, H, Hkv, D, window,
+                         dtype == NC_F16, S(stream));
+}
+
 nc_status nc_attention(const uint16_t* q, const uint16_t* k, const uint16_t* v, uint16_t* out, int B,
                        int T, int H, int Hkv, int D, int window, nc_dtype dtype, void* stream) {
   return nc_attention_strided(q, k, v, out, B, T, H, Hkv, D, window, (int64_t)H * D,
@@ -425,6 +452,40 @@ nc_status nc_linear(const uint16_t* a, const uint16_t* w, void* out, int M, int 
   ep.ldo = ldo;
   ep.cap = cap;
   return gemm_launch(a, K, w, K, M, N, K, (int)epilogue, dtype == NC_F16, ep, dev_status, S(stream));
+}
+
+nc_status nc_linear_dgrad(const uint16_t* dy, const uint16_t* w, void* dx, int M, int N, int K,
+                          nc_epilogue epilogue, nc_dtype dtype, uint32_t* dev_status, void* stream) {
+  if (!dy || !w || !dx || M < 0 || N < 8 || K < 8 || !dtype_ok(dtype)) return NC_ERR_INVALID_ARG;
+  if (epilogue != NC_EPI_STORE_16 && epilogue != NC_EPI_STORE_F32) return NC_ERR_INVALID_ARG;
+  if (N % 8 != 0 || K % 8 != 0) return NC_ERR_SHAPE;
+  if (!aligned16(dy) || !aligned16(w) || !aligned16(dx)) return NC_ERR_ALIGNMENT;
+  if (nc_status s = device_ok()) return s;
+  if (M == 0) return NC_OK;
+  EpiParams ep{};
+  ep.out = dx;
+  ep.ldo = K;
+  // dx = dy . w: contraction over N, output columns K; w [N, K] is the MN-major operand
+  return gemm_launch_layout(dy, N, w, K, M, K, N, (int)epilogue, dtype == NC_F16, GEMM_NN, ep, dev_status, S(stream));
+}
+
+nc_status nc_linear_wgrad(const uint16_t* dy, const uint16_t* x, float* dw, int M, int N, int K, float alpha,
+                          nc_dtype dtype, uint32_t* dev_status, void* stream) {
+  if (!dy || !x || !dw || M < 1 || N < 8 || K < 8 || !dtype_ok(dtype)) return NC_ERR_INVALID_ARG;
+  if (N % 8 != 0 || K % 8 != 0) return NC_ERR_SHAPE;
+  if (!aligned16(dy) || !aligned16(x) || !aligned16(dw)) return NC_ERR_ALIGNMENT;
+  if (nc_status s = device_ok()) return s;
+  if (alpha == 0.0f) return NC_OK;  // nothing to add
+  EpiParams ep{};
+  ep.out = dw;
+  ep.ldo = K;
+  ep.alpha = alpha;
+  const int tiles = ((N + 127) / 128) * ((K + 255) / 256);
+  const int nkb = (M + 63) / 64;
+  int ks = (8 * device_sm_count() + tiles - 1) / tiles;
+  ks = std::min(ks, std::max(1, nkb / 16));
+  ep.ksplit = std::max(ks, 1);
+  return gemm_launch_layout(dy, N, x, K, N, K, M, EPI_RESID_F32, dtype == NC_F16, GEMM_TN, ep, dev_status, S(stream));
 }
 
 nc_status nc_fp8_quantize(const void* x, nc_dtype src_dtype, int64_t n, uint8_t* codes, float* amax,
@@ -956,6 +1017,280 @@ nc_status nc_decode_step(const nc_config* cfg, const nc_weights* w, const int32_
   ep.cap = cfg->softcap;
   NC_TRY(gemm_launch(a, C, wlm, C, B, V, C, EPI_SOFTCAP_F32, f16, ep, status, st));
 #undef NC_TRY
+  return NC_OK;
+}
+
+}  // extern "C"
+
+namespace {
+
+// Workspace of nc_forward_backward.  Per layer l: the residual stream entering
+// the block (xs[2l]) and after attention (xs[2l+1]); xs[2L] is the final
+// stream.  Offsets are 256-byte aligned.
+struct TrainLayout {
+  size_t status, rope, wqkv, wo, wfc, wmp, wlm, xs, qkv, rstd, o, lse, h, af, a, part, tgt, tl, scal, dz, dx, dx16,
+      dy, du, dO, dqkv, delta, dwqkv, total;
+  size_t wqkv_elems, wo_elems, wfc_elems, wmp_elems;
+};
+
+TrainLayout train_layout(const nc_config* c, int B, int T) {
+  TrainLayout L;
+  const size_t M = (size_t)B * T, C = c->d_model, D = c->head_dim, H = c->n_head, Hkv = c->n_kv_head,
+               V = c->vocab, NL = c->n_layer;
+  const size_t nqkv = (H + 2 * Hkv) * D, HD = H * D;
+  L.wqkv_elems = nqkv * C;
+  L.wo_elems = C * HD;
+  L.wfc_elems = 4 * C * C;
+  L.wmp_elems = C * 4 * C;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    size_t o = off;
+    off = align_up(off + bytes, 256);
+    return o;
+  };
+  L.status = take(256);
+  L.rope = take((size_t)T * D * 4);
+  L.wqkv = take(NL * L.wqkv_elems * 2);
+  L.wo = take(NL * L.wo_elems * 2);
+  L.wfc = take(NL * L.wfc_elems * 2);
+  L.wmp = take(NL * L.wmp_elems * 2);
+  L.wlm = take(V * C * 2);
+  L.xs = take((2 * NL + 1) * M * C * 4);
+  L.qkv = take(NL * M * nqkv * 2);
+  L.rstd = take(NL * M * (H + Hkv) * 4);
+  L.o = take(NL * M * HD * 2);
+  L.lse = take(NL * M * H * 4);
+  L.h = take(NL * M * 4 * C * 2);
+  L.af = take(M * C * 2);
+  L.a = take(M * C * 2);
+  L.part = take(M * (size_t)gemm_ce_partials_per_row((int)V) * 4);
+  L.tgt = take(M * 4);
+  L.tl = take(M * 4);
+  L.scal = take(256);  // 1 / (counted targets)
+  L.dz = take(M * V * 2);
+  L.dx = take(M * C * 4);
+  L.dx16 = take(M * C * 2);
+  L.dy = take(M * C * 4);
+  L.du = take(M * 4 * C * 2);
+  L.dO = take(M * HD * 2);
+  L.dqkv = take(M * nqkv * 2);
+  L.delta = take(M * H * 4);
+  L.dwqkv = take(nqkv * C * 4);
+  L.total = off;
+  return L;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t nc_train_workspace_bytes(const nc_config* cfg, int B, int T) {
+  if (!config_ok(cfg) || cfg->extras != 0 || cfg->fp8 != 0 || B < 1 || T < 1 || T > cfg->seq_len) return 0;
+  return train_layout(cfg, B, T).total;
+}
+
+nc_status nc_forward_backward(const nc_config* cfg, const nc_weights* w, const int32_t* tokens,
+                              const int32_t* targets, int B, int T, float* loss, const nc_grads* g,
+                              void* workspace, size_t ws_bytes, void* stream) {
+  return nc_forward_backward_traced(cfg, w, tokens, targets, B, T, loss, g, workspace, ws_bytes, stream, nullptr);
+}
+
+nc_status nc_forward_backward_traced(const nc_config* cfg, const nc_weights* w, const int32_t* tokens,
+                                     const int32_t* targets, int B, int T, float* loss, const nc_grads* g,
+                                     void* workspace, size_t ws_bytes, void* stream, nc_trace* trace) {
+  if (!cfg || !w || !tokens || !targets || !loss || !g || !workspace) return NC_ERR_INVALID_ARG;
+  if (!config_ok(cfg) || cfg->extras != 0 || cfg->fp8 != 0) return NC_ERR_CONFIG;
+  if (B < 1 || T < 1 || T > cfg->seq_len || (int64_t)B * T > ((int64_t)1 << 30)) return NC_ERR_SHAPE;
+  const TrainLayout L = train_layout(cfg, B, T);
+  if (ws_bytes < L.total) return NC_ERR_WORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return NC_ERR_ALIGNMENT;
+  if (nc_status s = check_weights(cfg, w)) return s;
+  if (!g->wte || !g->lm_head || !g->c_q || !g->c_k || !g->c_v || !g->attn_proj || !g->c_fc || !g->mlp_proj)
+    return NC_ERR_INVALID_ARG;
+  if (!aligned16(g->wte) || !aligned16(g->lm_head) || !aligned16(loss)) return NC_ERR_ALIGNMENT;
+  for (int l = 0; l < cfg->n_layer; ++l) {
+    const float* ps[6] = {g->c_q[l], g->c_k[l], g->c_v[l], g->attn_proj[l], g->c_fc[l], g->mlp_proj[l]};
+    for (const float* p : ps) {
+      if (!p) return NC_ERR_INVALID_ARG;
+      if (!aligned16(p)) return NC_ERR_ALIGNMENT;
+    }
+  }
+  if (trace) {
+    const int need = 12 + 24 * cfg->n_layer;
+    trace->count = need;
+    if (!trace->events || trace->capacity < need) return NC_ERR_INVALID_ARG;
+    for (int i = 0; i < 2 * need; ++i)
+      if (!trace->events[i]) return NC_ERR_INVALID_ARG;
+  }
+  if (nc_status s = device_ok()) return s;
+
+  cudaStream_t st = S(stream);
+  Tracer tr{trace, st, 0, false};
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const int M = B * T, NL = cfg->n_layer;
+  const int C = cfg->d_model, D = cfg->head_dim, H = cfg->n_head, Hkv = cfg->n_kv_head, V = cfg->vocab;
+  const int NQKV = (H + 2 * Hkv) * D, HD = H * D;
+  const bool f16 = cfg->act_dtype == NC_F16;
+  const float eps = cfg->norm_eps;
+  const size_t MC = (size_t)M * C;
+  uint32_t* status = reinterpret_cast<uint32_t*>(ws + L.status);
+  float* rope = reinterpret_cast<float*>(ws + L.rope);
+  uint16_t* wqkv = reinterpret_cast<uint16_t*>(ws + L.wqkv);
+  uint16_t* wo = reinterpret_cast<uint16_t*>(ws + L.wo);
+  uint16_t* wfc = reinterpret_cast<uint16_t*>(ws + L.wfc);
+  uint16_t* wmp = reinterpret_cast<uint16_t*>(ws + L.wmp);
+  uint16_t* wlm = reinterpret_cast<uint16_t*>(ws + L.wlm);
+  float* xs = reinterpret_cast<float*>(ws + L.xs);
+  auto qkv_l = [&](int l) { return reinterpret_cast<uint16_t*>(ws + L.qkv) + (size_t)l * M * NQKV; };
+  auto rstd_l = [&](int l) { return reinterpret_cast<float*>(ws + L.rstd) + (size_t)l * M * (H + Hkv); };
+  auto o_l = [&](int l) { return reinterpret_cast<uint16_t*>(ws + L.o) + (size_t)l * M * HD; };
+  auto lse_l = [&](int l) { return reinterpret_cast<float*>(ws + L.lse) + (size_t)l * M * H; };
+  auto h_l = [&](int l) { return reinterpret_cast<uint16_t*>(ws + L.h) + (size_t)l * M * 4 * C; };
+  uint16_t* af = reinterpret_cast<uint16_t*>(ws + L.af);
+  uint16_t* a = reinterpret_cast<uint16_t*>(ws + L.a);
+  float* part = reinterpret_cast<float*>(ws + L.part);
+  float* tgt = reinterpret_cast<float*>(ws + L.tgt);
+  float* tl = reinterpret_cast<float*>(ws + L.tl);
+  float* inv = reinterpret_cast<float*>(ws + L.scal);
+  uint16_t* dz = reinterpret_cast<uint16_t*>(ws + L.dz);
+  float* dx = reinterpret_cast<float*>(ws + L.dx);
+  uint16_t* dx16 = reinterpret_cast<uint16_t*>(ws + L.dx16);
+  float* dy = reinterpret_cast<float*>(ws + L.dy);
+  uint16_t* du = reinterpret_cast<uint16_t*>(ws + L.du);
+  uint16_t* dO = reinterpret_cast<uint16_t*>(ws + L.dO);
+  uint16_t* dqkv = reinterpret_cast<uint16_t*>(ws + L.dqkv);
+  float* delta = reinterpret_cast<float*>(ws + L.delta);
+  float* dwqkv = reinterpret_cast<float*>(ws + L.dwqkv);
+
+  nc_status s = NC_OK;
+#define NC_RUN(kind, call)                   \
+  do {                                       \
+    if (!tr.begin(kind)) return NC_ERR_CUDA; \
+    s = (call);                              \
+    if (s != NC_OK) return s;                \
+    if (!tr.end()) return NC_ERR_CUDA;       \
+  } while (0)
+  auto copy = [&](float* dst, const float* src) -> nc_status {
+    return cudaMemcpyAsync(dst, src, MC * 4, cudaMemcpyDeviceToDevice, st) == cudaSuccess ? NC_OK : NC_ERR_CUDA;
+  };
+  // ---------------- forward, keeping what the backward reads
+  if (cudaMemsetAsync(status, 0, 256, st) != cudaSuccess) return NC_ERR_CUDA;
+  NC_RUN(NC_K_ROPE_TABLE, rope_table_launch(rope, T, D, cfg->rope_base, st));
+  NC_RUN(NC_K_CAST, launch_weight_cast(cfg, w, wqkv, wo, wfc, wmp, wlm, L.wqkv_elems, L.wo_elems, L.wfc_elems, L.wmp_elems,
+                            f16, st));
+  NC_RUN(NC_K_EMBEDDING, embedding_launch(tokens, w->wte, xs, M, C, V, status, st));
+  for (int l = 0; l < NL; ++l) {
+    float* xin = xs + (size_t)(2 * l) * MC;
+    float* xmid = xin + MC;
+    float* xnext = xmid + MC;
+    NC_RUN(NC_K_RMSNORM, rmsnorm_launch(xin, a, M, C, eps, f16, st));
+    EpiParams eq{};
+    eq.out = qkv_l(l);
+    eq.ldo = NQKV;
+    eq.rope = rope;
+    eq.T = T;
+    eq.H = H;
+    eq.Hkv = Hkv;
+    eq.D = D;
+    eq.eps = eps;
+    eq.rope_T = T;
+    eq.rstd_out = rstd_l(l);
+    NC_RUN(NC_K_GEMM_QKV, gemm_launch(a, C, wqkv + l * L.wqkv_elems, C, M, NQKV, C, EPI_QKV_ROPE_IL, f16, eq, status, st));
+    uint16_t* q = qkv_l(l);
+    NC_RUN(NC_K_ATTENTION, attention_launch(q, q + HD, q + (H + Hkv) * D, o_l(l), B, T, H, Hkv, D, nc_layer_window(cfg, l), NQKV,
+                            NQKV, f16, status, st, nullptr, lse_l(l)));
+    NC_RUN(NC_K_COPY, copy(xmid, xin));
+    EpiParams ep{};
+    ep.out = xmid;
+    ep.ldo = C;
+    NC_RUN(NC_K_GEMM_ATTN_PROJ, gemm_launch(o_l(l), HD, wo + l * L.wo_elems, HD, M, C, HD, EPI_RESID_F32, f16, ep, status, st));
+    NC_RUN(NC_K_RMSNORM, rmsnorm_launch(xmid, a, M, C, eps, f16, st));
+    ep.out = h_l(l);
+    ep.ldo = 4 * C;
+    NC_RUN(NC_K_GEMM_FC, gemm_launch(a, C, wfc + l * L.wfc_elems, C, M, 4 * C, C, EPI_RELU2_16, f16, ep, status, st));
+    NC_RUN(NC_K_COPY, copy(xnext, xmid));
+    ep.out = xnext;
+    ep.ldo = C;
+    NC_RUN(NC_K_GEMM_MLP_PROJ, gemm_launch(h_l(l), 4 * C, wmp + l * L.wmp_elems, 4 * C, M, C, 4 * C, EPI_RESID_F32, f16, ep, status,
+                       st));
+  }
+  float* xf = xs + (size_t)(2 * NL) * MC;
+  NC_RUN(NC_K_RMSNORM, rmsnorm_launch(xf, af, M, C, eps, f16, st));
+  {
+    EpiParams ep{};
+    ep.ldo = V;
+    ep.cap = cfg->softcap;
+    ep.ce_partial = part;
+    ep.ce_target = tgt;
+    ep.targets = targets;
+    NC_RUN(NC_K_GEMM_LM_HEAD, gemm_launch(af, C, wlm, C, M, V, C, EPI_CE_PARTIAL, f16, ep, status, st));
+    NC_RUN(NC_K_CE_FINALIZE, ce_finalize_launch(part, gemm_ce_partials_per_row(V), tgt, targets, tl, M, V, cfg->softcap, status, st));
+    NC_RUN(NC_K_LOSS_MEAN, loss_mean_launch(tl, targets, M, V, loss, st, inv));
+  }
+
+  // ---------------- backward (gradients of the summed token loss; weight
+  // gradients take the factor 1 / count from `inv`)
+  auto wgrad = [&](const uint16_t* dyt, int64_t ld_dy, const uint16_t* xt, int64_t ld_x, int No, int Ko, float* out,
+                   int64_t ldo) -> nc_status {  // out [No, Ko] += inv * dyt^T xt, over the M tokens
+    EpiParams e{};
+    e.out = out;
+    e.ldo = ldo;
+    e.alpha_ptr = inv;
+    const int tiles = ((No + 127) / 128) * ((Ko + 255) / 256);
+    const int nkb = (M + 63) / 64;
+    int ks = (8 * device_sm_count() + tiles - 1) / tiles;
+    ks = std::min(ks, std::max(1, nkb / 16));
+    e.ksplit = std::max(ks, 1);
+    return gemm_launch_layout(dyt, ld_dy, xt, ld_x, No, Ko, M, EPI_RESID_F32, f16, GEMM_TN, e, status, st);
+  };
+  auto dgrad = [&](const uint16_t* dyt, int K, const uint16_t* wt, int N, int epi, void* out,
+                   const uint16_t* aux = nullptr) -> nc_status {  // out [M, N] = dyt [M, K] . wt [K, N]
+    EpiParams e{};
+    e.out = out;
+    e.ldo = N;
+    e.aux = aux;
+    e.ld_aux = N;
+    return gemm_launch_layout(dyt, K, wt, N, M, N, K, epi, f16, GEMM_NN, e, status, st);
+  };
+  {
+    EpiParams ep{};
+    ep.out = dz;
+    ep.ldo = V;
+    ep.cap = cfg->softcap;
+    ep.targets = targets;
+    ep.row_lse = tl;
+    ep.ce_target = tgt;
+    NC_RUN(NC_K_CE_BWD, gemm_launch(af, C, wlm, C, M, V, C, EPI_CE_BWD_16, f16, ep, status, st));
+  }
+  NC_RUN(NC_K_GEMM_WGRAD, wgrad(dz, V, af, C, V, C, g->lm_head, C));
+  NC_RUN(NC_K_GEMM_DGRAD, dgrad(dz, V, wlm, C, EPI_STORE_F32, dy));
+  NC_RUN(NC_K_NORM_BWD, rmsnorm_bwd_launch(xf, dy, dx, dx16, M, C, eps, false, f16, st));
+  for (int l = NL - 1; l >= 0; --l) {
+    float* xin = xs + (size_t)(2 * l) * MC;
+    float* xmid = xin + MC;
+    // MLP
+    NC_RUN(NC_K_GEMM_WGRAD, wgrad(dx16, C, h_l(l), 4 * C, C, 4 * C, g->mlp_proj[l], 4 * C));
+    NC_RUN(NC_K_GEMM_DGRAD, dgrad(dx16, C, wmp + l * L.wmp_elems, 4 * C, EPI_RELU2_BWD_16, du, h_l(l)));
+    NC_RUN(NC_K_RMSNORM, rmsnorm_launch(xmid, a, M, C, eps, f16, st));
+    NC_RUN(NC_K_GEMM_WGRAD, wgrad(du, 4 * C, a, C, 4 * C, C, g->c_fc[l], C));
+    NC_RUN(NC_K_GEMM_DGRAD, dgrad(du, 4 * C, wfc + l * L.wfc_elems, C, EPI_STORE_F32, dy));
+    NC_RUN(NC_K_NORM_BWD, rmsnorm_bwd_launch(xmid, dy, dx, dx16, M, C, eps, true, f16, st));
+    // attention block
+    NC_RUN(NC_K_GEMM_WGRAD, wgrad(dx16, C, o_l(l), HD, C, HD, g->attn_proj[l], HD));
+    NC_RUN(NC_K_GEMM_DGRAD, dgrad(dx16, C, wo + l * L.wo_elems, HD, EPI_STORE_16, dO));
+    NC_RUN(NC_K_ATTN_BWD, attn_bwd_launch(qkv_l(l), NQKV, o_l(l), dO, lse_l(l), delta, dqkv, B, T, H, Hkv, D,
+                           nc_layer_window(cfg, l), f16, st));
+    NC_RUN(NC_K_QK_BWD, qk_bwd_launch(dqkv, qkv_l(l), NQKV, rstd_l(l), rope, T, M, T, H, Hkv, D, f16, st));
+    NC_RUN(NC_K_RMSNORM, rmsnorm_launch(xin, a, M, C, eps, f16, st));
+    NC_RUN(NC_K_GEMM_WGRAD, cudaMemsetAsync(dwqkv, 0, (size_t)NQKV * C * 4, st) == cudaSuccess
+                                ? wgrad(dqkv, NQKV, a, C, NQKV, C, dwqkv, C)
+                                : NC_ERR_CUDA);
+    NC_RUN(NC_K_EMB_BWD, qkv_grad_scatter_launch(dwqkv, g->c_q[l], g->c_k[l], g->c_v[l], H, Hkv, D, C, 1.0f, st));
+    NC_RUN(NC_K_GEMM_DGRAD, dgrad(dqkv, NQKV, wqkv + l * L.wqkv_elems, C, EPI_STORE_F32, dy));
+    NC_RUN(NC_K_NORM_BWD, rmsnorm_bwd_launch(xin, dy, dx, dx16, M, C, eps, true, f16, st));
+  }
+  NC_RUN(NC_K_EMB_BWD, embedding_bwd_launch(tokens, dx, g->wte, M, C, V, inv, st));
+#undef NC_RUN
   return NC_OK;
 }
 

@@ -152,7 +152,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                    const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
                    uint16_t* __restrict__ out, int B,
                    int T, int H, int Hkv, int W, float scale_log2, uint32_t* dev_status,
-                   uint64_t limit_ns, float* __restrict__ amax) {
+                   uint64_t limit_ns, float* __restrict__ amax, float* __restrict__ lse_out) {
   using G = Geo<D>;
   constexpr uint32_t IDESC_S = idesc_f32acc(BQ, BKV, F16);
   constexpr uint32_t IDESC_PV = idesc_f32acc_bmn(BQ, D, F16);
@@ -401,7 +401,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     // n + 1 does not use.
     struct Pending {
       int b, h, q0, gl, ob;
-      float l;
+      float l, m;
     };
     Pending pend{};
     bool has_pend = false;
@@ -418,6 +418,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
       tc_fence_after();
       const float inv = lsum > 0.0f ? 1.0f / lsum : 0.0f;
+      // natural log-sum-exp of the row's scaled scores (kept for the backward)
+      if (lse_out && half == 0 && pd.q0 + r < T)
+        lse_out[((int64_t)pd.b * T + pd.q0 + r) * H + pd.h] = pd.m * (scale_log2 * 0.6931471805599453f) + logf(lsum);
       const uint32_t ocol = O_COL + pd.ob * D + half * DC;
       uint32_t rr[DC / 32][32];
 #pragma unroll
@@ -602,7 +605,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
       }
       if (!ok) break;
-      pend = Pending{it.b, it.h, it.q0, g + it.n_tiles - 1, n & 1, l};
+      pend = Pending{it.b, it.h, it.q0, g + it.n_tiles - 1, n & 1, l, m_used};
       has_pend = true;
       g += it.n_tiles;
       const int ns = n & 1;
@@ -644,7 +647,7 @@ static bool make_map4(CUtensorMap* map, const void* base, int B, int T, int head
 template <int D, bool F16>
 static nc_status launch_t(const uint16_t* q, const uint16_t* k, const uint16_t* v, uint16_t* out,
                           int B, int T, int H, int Hkv, int W, int64_t q_stride, int64_t kv_stride,
-                          uint32_t* dev_status, cudaStream_t stream, float* amax) {
+                          uint32_t* dev_status, cudaStream_t stream, float* amax, float* lse) {
   using G = Geo<D>;
   static bool attr_done[64] = {};
   int dev = 0;
@@ -671,7 +674,7 @@ static nc_status launch_t(const uint16_t* q, const uint16_t* k, const uint16_t* 
   const int grid = B * H * ((T + BQ - 1) / BQ);
   const float scale_log2 = 1.4426950408889634f / sqrtf((float)D);
   attn_tc_kernel<D, F16><<<grid, NUM_THREADS, G::SMEM_BYTES, stream>>>(
-      mq, mk, mv, mo, out, B, T, H, Hkv, W, scale_log2, dev_status, kWaitLimitNs, amax);
+      mq, mk, mv, mo, out, B, T, H, Hkv, W, scale_log2, dev_status, kWaitLimitNs, amax, lse);
   return cudaGetLastError() == cudaSuccess ? NC_OK : NC_ERR_CUDA;
 }
 
@@ -680,19 +683,19 @@ static nc_status launch_t(const uint16_t* q, const uint16_t* k, const uint16_t* 
 nc_status attention_launch(const uint16_t* q, const uint16_t* k, const uint16_t* v, uint16_t* out,
                            int B, int T, int H, int Hkv, int D, int window, int64_t q_stride,
                            int64_t kv_stride, bool f16, uint32_t* dev_status, cudaStream_t stream,
-                           float* amax) {
+                           float* amax, float* lse) {
   if (D != 64 && D != 128) return NC_ERR_SHAPE;
   if (B == 0 || T == 0) return NC_OK;
   const int W = (window <= 0 || window > T) ? T : window;
   if (D == 128)
     return f16 ? attn::launch_t<128, true>(q, k, v, out, B, T, H, Hkv, W, q_stride, kv_stride, dev_status, stream,
-                                           amax)
+                                           amax, lse)
                : attn::launch_t<128, false>(q, k, v, out, B, T, H, Hkv, W, q_stride, kv_stride, dev_status,
-                                            stream, amax);
+                                            stream, amax, lse);
   return f16 ? attn::launch_t<64, true>(q, k, v, out, B, T, H, Hkv, W, q_stride, kv_stride, dev_status, stream,
-                                        amax)
+                                        amax, lse)
              : attn::launch_t<64, false>(q, k, v, out, B, T, H, Hkv, W, q_stride, kv_stride, dev_status, stream,
-                                         amax);
+                                         amax, lse);
 }
 
 }  // namespace nc

@@ -208,6 +208,8 @@ __device__ __forceinline__ void epilogue_f32_half(uint32_t taddr, const CUtensor
     const int col0 = n0 + c * 32;
     if (col0 >= N) break;  // warp-uniform
     if constexpr (SC) scale32(r, dq);
+    if (ep.alpha_ptr) scale32(r, *ep.alpha_ptr);
+    else if (ep.alpha != 0.0f) scale32(r, ep.alpha);
     if constexpr (EPI == EPI_SOFTCAP_F32) {
       const SoftCap sc(ep.cap);
 #pragma unroll
@@ -269,6 +271,86 @@ __device__ __forceinline__ void epilogue_16_half(uint32_t taddr, const CUtensorM
     stage_row(stg, (int)lane, w);
     flush_issue<false>(tmC, stg, col0, row0, lane);
     tmem_wait_ld();
+  }
+  flush_wait(lane);
+}
+
+// Backward epilogues with a 16-bit output that depend on the row (and column):
+//   EPI_CE_BWD_16     the accumulator is the recomputed logit z; with l the
+//                     soft-capped logit, p = exp(l - lse_row) its probability:
+//                     out = (p - [col == target]) (1 - (l / cap)^2), 0 for rows
+//                     whose target is -1 (the gradient of the summed
+//                     cross-entropy with respect to z);
+//   EPI_RELU2_BWD_16  the accumulator is dL/dh for h = relu(u)^2 (saved, 16-bit,
+//                     in ep.aux): out = dL/du = acc * 2 sqrt(h).
+// 64-column chunks, staged and stored by TMA like epilogue_16_half.
+template <int EPI, bool F16>
+__device__ __forceinline__ void epilogue_16_rowdep(uint32_t taddr, const CUtensorMap* tmC, uint8_t* stg, int n0,
+                                                   int row0, int row, int M, int N, const EpiParams& ep,
+                                                   uint32_t lane) {
+  const bool live = row < M;
+  int target = -1;
+  float f = 0.0f;  // exp(cap - lse_row): p = exp(l - cap) f
+  const SoftCap sc(ep.cap);
+  if constexpr (EPI == EPI_CE_BWD_16) {
+    if (live) {
+      target = ep.targets[row];
+      const float lse = ep.row_lse[row] + (ep.ce_target ? ep.ce_target[row] : 0.0f);
+      f = ex2_approx((ep.cap - lse) * 1.4426950408889634f);
+    }
+  }
+  const float inv_cap2 = 1.0f / (ep.cap * ep.cap);
+#pragma unroll 1
+  for (int c = 0; c < EPI_COLS / 64; ++c) {
+    const int col0 = n0 + c * 64;
+    if (col0 >= N) break;  // warp-uniform
+    uint32_t r[2][32];
+    tmem_ld_32x32b_x32(taddr + c * 64, r[0]);
+    tmem_ld_32x32b_x32(taddr + c * 64 + 32, r[1]);
+    tmem_wait_ld();
+    uint32_t hv[32];  // RELU2_BWD: the saved h of these 64 columns
+    if constexpr (EPI == EPI_RELU2_BWD_16) {
+      if (live) {
+        const uint4* hp = reinterpret_cast<const uint4*>(ep.aux + (int64_t)row * ep.ld_aux + col0);
+        const int nv = N - col0;  // columns of this chunk inside the row (a multiple of 8)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const uint4 u = 8 * j < nv ? __ldg(hp + j) : make_uint4(0u, 0u, 0u, 0u);
+          hv[4 * j] = u.x;
+          hv[4 * j + 1] = u.y;
+          hv[4 * j + 2] = u.z;
+          hv[4 * j + 3] = u.w;
+        }
+      } else {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) hv[j] = 0u;
+      }
+    }
+    uint32_t w[32];
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        float g[2];
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const float acc = __uint_as_float(r[h][2 * i + e]);
+          if constexpr (EPI == EPI_CE_BWD_16) {
+            float pc;
+            const float l = sc.apply(acc, pc);
+            const int col = col0 + 32 * h + 2 * i + e;
+            const float p = pc * f - (col == target ? 1.0f : 0.0f);
+            g[e] = target >= 0 ? p * (1.0f - l * l * inv_cap2) : 0.0f;
+          } else {
+            const float2 hh = Half<F16>::unpack2(hv[16 * h + i]);
+            g[e] = acc * 2.0f * sqrtf(e == 0 ? hh.x : hh.y);
+          }
+        }
+        w[16 * h + i] = Half<F16>::pack2(g[0], g[1]);
+      }
+    if (c > 0) flush_wait(lane);
+    stage_row(stg, (int)lane, w);
+    flush_issue<false>(tmC, stg, col0, row0, lane);
   }
   flush_wait(lane);
 }
@@ -423,6 +505,7 @@ __device__ __forceinline__ void epilogue_qkv_head_il(uint32_t taddr, const CUten
   }
   // e4m3: the head's values are dq * acc, so its mean square is dq^2 ss / HD
   const float rs = SC ? rsqrtf(ss * (dq * dq) * (1.0f / HD) + ep.eps) * dq : rsqrtf(ss * (1.0f / HD) + ep.eps);
+  if (ep.rstd_out && row < M) ep.rstd_out[(int64_t)row * (ep.H + ep.Hkv) + head] = rs;
   const int t = ep.pos0 + (row < M ? row : 0) % ep.T;
   const float* cs = ep.rope + (int64_t)t * (HD / 2);
   const float* sn = ep.rope + ((int64_t)(ep.rope_T > 0 ? ep.rope_T : ep.T) + t) * (HD / 2);
@@ -458,12 +541,20 @@ __device__ __forceinline__ void epilogue_qkv_head_il(uint32_t taddr, const CUten
 // EPI: epilogue selector; F16: 16-bit operands (and 16-bit outputs) fp16
 // instead of bf16; HD: head size of the QKV epilogues (0 otherwise); FP8:
 // e4m3 operands (16-bit outputs still in the F16 format).
-template <int EPI, bool F16, int HD, bool FP8>
+// LAY: operand layout (GEMM_NT, GEMM_NN, GEMM_TN).  An MN-major operand is
+// loaded as boxes of 64 K rows x 64 MN elements (128 bytes, swizzled); the
+// descriptor then steps 64-element MN blocks by the box size and 8-row K
+// groups by 1024 bytes, and each MMA of K = 16 advances 16 rows (2048 bytes).
+template <int EPI, bool F16, int HD, bool FP8, int LAY = GEMM_NT>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const __grid_constant__ CUtensorMap tmC, int M, int N, int K, EpiParams ep,
                 uint32_t* dev_status, uint64_t limit_ns) {
-  constexpr uint32_t IDESC = FP8 ? IDESC_E4M3 : (F16 ? IDESC_F16 : IDESC_BF16);
+  constexpr bool A_MN = LAY == GEMM_TN, B_MN = LAY != GEMM_NT;
+  static_assert(!(FP8 && LAY != GEMM_NT), "e4m3 operands are K-major");
+  constexpr uint32_t IDESC = (FP8 ? IDESC_E4M3 : (F16 ? IDESC_F16 : IDESC_BF16)) | (A_MN ? (1u << 15) : 0u) |
+                             (B_MN ? (1u << 16) : 0u);
+  constexpr int MN_BOX = 64 * BK * 2;  // bytes of one MN-major box
   constexpr int KE = FP8 ? 2 * BK : BK;  // elements per 128-byte swizzle row
   extern __shared__ uint8_t smem_raw[];
   uint8_t* tiles = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -529,8 +620,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           const uint32_t fb = smem_u32(&sm->full[stage]);
           mbar_arrive_expect_tx(fb, STAGE_BYTES);
           uint8_t* a_dst = tiles + stage * STAGE_BYTES;
-          tma_load_2d(smem_u32(a_dst), &tmA, kb * KE, m0, fb);
-          tma_load_2d(smem_u32(a_dst + A_BYTES), &tmB, kb * KE, n0, fb);
+          if constexpr (A_MN) {
+#pragma unroll
+            for (int i = 0; i < BM / 64; ++i) tma_load_2d(smem_u32(a_dst + i * MN_BOX), &tmA, m0 + 64 * i, kb * BK, fb);
+          } else {
+            tma_load_2d(smem_u32(a_dst), &tmA, kb * KE, m0, fb);
+          }
+          if constexpr (B_MN) {
+#pragma unroll
+            for (int i = 0; i < BN / 64; ++i)
+              tma_load_2d(smem_u32(a_dst + A_BYTES + i * MN_BOX), &tmB, n0 + 64 * i, kb * BK, fb);
+          } else {
+            tma_load_2d(smem_u32(a_dst + A_BYTES), &tmB, kb * KE, n0, fb);
+          }
           outstanding |= 1u << stage;
           out_phase = (out_phase & ~(1u << stage)) | (phase << stage);
           if (++stage == STAGES) {
@@ -571,9 +673,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           const uint32_t a_addr = smem_u32(tiles + stage * STAGE_BYTES);
           const uint32_t b_addr = a_addr + A_BYTES;
 #pragma unroll
-          for (int k = 0; k < BK / 16; ++k) {  // 32 bytes of each row per MMA
-            const uint64_t adesc = sw128_kmajor_desc(a_addr + k * 32);
-            const uint64_t bdesc = sw128_kmajor_desc(b_addr + k * 32);
+          for (int k = 0; k < BK / 16; ++k) {  // 32 bytes of each row (K-major) or 16 rows (MN-major) per MMA
+            const uint64_t adesc = A_MN ? sw128_desc(a_addr + k * 2048, MN_BOX, 1024) : sw128_kmajor_desc(a_addr + k * 32);
+            const uint64_t bdesc = B_MN ? sw128_desc(b_addr + k * 2048, MN_BOX, 1024) : sw128_kmajor_desc(b_addr + k * 32);
             if constexpr (FP8)
               umma_f8(d_tmem, adesc, bdesc, IDESC, (kb != kb_begin || k != 0) ? 1u : 0u);
             else
@@ -657,6 +759,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
       } else if constexpr (EPI == EPI_STORE_16 || EPI == EPI_RELU2_16) {
         epilogue_16_half<EPI, F16, FP8>(taddr, &tmC, stg, n0, row0, N, lane, dqs.q, &om);
+      } else if constexpr (EPI == EPI_CE_BWD_16 || EPI == EPI_RELU2_BWD_16) {
+        epilogue_16_rowdep<EPI, F16>(taddr, &tmC, stg, n0, row0, row, M, N, ep, lane);
       } else if constexpr (EPI == EPI_CE_PARTIAL) {
         if (row < M) target = ep.targets ? ep.targets[row] : -1;
 #pragma unroll 1
@@ -740,7 +844,7 @@ static bool make_map_u8(CUtensorMap* map, const void* ptr, int64_t rows, int64_t
   return encode_tensor_map_u8(map, 2, ptr, dims, strides, box);
 }
 
-template <int EPI, bool F16, int HD, bool FP8>
+template <int EPI, bool F16, int HD, bool FP8, int LAY = GEMM_NT>
 static cudaError_t launch_t(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& mc, int M,
                             int N, int K, const EpiParams& ep, uint32_t* dev_status, uint64_t limit_ns,
                             cudaStream_t stream) {
@@ -748,7 +852,7 @@ static cudaError_t launch_t(const CUtensorMap& ma, const CUtensorMap& mb, const 
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 64 && !attr_done[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_kernel<EPI, F16, HD, FP8>,
+    cudaError_t e = cudaFuncSetAttribute(gemm_kernel<EPI, F16, HD, FP8, LAY>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
     if (e != cudaSuccess) return e;
     attr_done[dev] = true;
@@ -756,8 +860,8 @@ static cudaError_t launch_t(const CUtensorMap& ma, const CUtensorMap& mb, const 
   const int tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN) * (EPI == EPI_RESID_F32 && ep.ksplit > 1 ? ep.ksplit : 1);
   const int sms = device_sm_count();
   const int grid = tiles < sms ? tiles : sms;
-  gemm_kernel<EPI, F16, HD, FP8><<<grid, NUM_THREADS, SMEM_BYTES, stream>>>(ma, mb, mc, M, N, K, ep,
-                                                                            dev_status, limit_ns);
+  gemm_kernel<EPI, F16, HD, FP8, LAY><<<grid, NUM_THREADS, SMEM_BYTES, stream>>>(ma, mb, mc, M, N, K, ep,
+                                                                                 dev_status, limit_ns);
   return cudaGetLastError();
 }
 
@@ -772,6 +876,9 @@ static cudaError_t dispatch(int epi, const CUtensorMap& ma, const CUtensorMap& m
     case EPI_STORE_F32: return launch_t<EPI_STORE_F32, F16, 0, FP8>(ma, mb, mc, M, N, K, ep, st, lim, s);
     case EPI_SOFTCAP_F32: return launch_t<EPI_SOFTCAP_F32, F16, 0, FP8>(ma, mb, mc, M, N, K, ep, st, lim, s);
     case EPI_CE_PARTIAL: return launch_t<EPI_CE_PARTIAL, F16, 0, FP8>(ma, mb, mc, M, N, K, ep, st, lim, s);
+    case EPI_CE_BWD_16:
+      if constexpr (FP8) return cudaErrorInvalidValue;
+      else return launch_t<EPI_CE_BWD_16, F16, 0, false>(ma, mb, mc, M, N, K, ep, st, lim, s);
     case EPI_QKV_ROPE:
       if constexpr (FP8) return cudaErrorInvalidValue;  // the interleaved form only
       else
@@ -780,6 +887,20 @@ static cudaError_t dispatch(int epi, const CUtensorMap& ma, const CUtensorMap& m
     case EPI_QKV_ROPE_IL:
       return ep.D == 128 ? launch_t<EPI_QKV_ROPE_IL, F16, 128, FP8>(ma, mb, mc, M, N, K, ep, st, lim, s)
                          : launch_t<EPI_QKV_ROPE_IL, F16, 64, FP8>(ma, mb, mc, M, N, K, ep, st, lim, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+template <bool F16, int LAY>
+static cudaError_t dispatch_layout(int epi, const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& mc,
+                                   int M, int N, int K, const EpiParams& ep, uint32_t* st, uint64_t lim,
+                                   cudaStream_t s) {
+  switch (epi) {
+    case EPI_STORE_16: return launch_t<EPI_STORE_16, F16, 0, false, LAY>(ma, mb, mc, M, N, K, ep, st, lim, s);
+    case EPI_STORE_F32: return launch_t<EPI_STORE_F32, F16, 0, false, LAY>(ma, mb, mc, M, N, K, ep, st, lim, s);
+    case EPI_RESID_F32: return launch_t<EPI_RESID_F32, F16, 0, false, LAY>(ma, mb, mc, M, N, K, ep, st, lim, s);
+    case EPI_RELU2_BWD_16:
+      return launch_t<EPI_RELU2_BWD_16, F16, 0, false, LAY>(ma, mb, mc, M, N, K, ep, st, lim, s);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -855,7 +976,7 @@ static bool make_out_map(CUtensorMap* mc, int epi, int M, int N, bool f16, const
   if (epi == EPI_CE_PARTIAL) return true;
   const uint64_t dims[2] = {(uint64_t)N, (uint64_t)M};
   const bool out16 = (epi == EPI_STORE_16 || epi == EPI_RELU2_16 || epi == EPI_QKV_ROPE ||
-                      epi == EPI_QKV_ROPE_IL);
+                      epi == EPI_QKV_ROPE_IL || epi == EPI_CE_BWD_16 || epi == EPI_RELU2_BWD_16);
   const uint64_t strides[1] = {(uint64_t)ep.ldo * (out16 ? 2 : 4)};
   const uint32_t box[2] = {out16 ? 64u : 32u, 32u};
   return out16 ? encode_tensor_map(mc, f16, 2, ep.out, dims, strides, box)
@@ -863,7 +984,9 @@ static bool make_out_map(CUtensorMap* mc, int epi, int M, int N, bool f16, const
 }
 
 static nc_status check_epi(int epi, int K, int ke, const EpiParams& ep) {
-  if (epi < EPI_STORE_16 || epi > EPI_QKV_ROPE_IL) return NC_ERR_INVALID_ARG;
+  if (epi < EPI_STORE_16 || epi > EPI_RELU2_BWD_16) return NC_ERR_INVALID_ARG;
+  if (epi == EPI_CE_BWD_16 && (!ep.targets || !ep.row_lse)) return NC_ERR_INVALID_ARG;
+  if (epi == EPI_RELU2_BWD_16 && (!ep.aux || ep.ld_aux % 8)) return NC_ERR_INVALID_ARG;
   if ((epi == EPI_QKV_ROPE || epi == EPI_QKV_ROPE_IL) && (ep.D != 64 && ep.D != 128)) return NC_ERR_SHAPE;
   if (ep.ksplit > 1 && (epi != EPI_RESID_F32 || ep.ksplit > (K + ke - 1) / ke)) return NC_ERR_INVALID_ARG;
   return NC_OK;
@@ -880,6 +1003,38 @@ nc_status gemm_launch(const uint16_t* a, int64_t lda, const uint16_t* w, int64_t
   if (!make_out_map(&mc, epi, M, N, f16, ep)) return NC_ERR_CUDA;
   const cudaError_t e = f16 ? dispatch<true, false>(epi, ma, mb, mc, M, N, K, ep, dev_status, limit_ns, stream)
                             : dispatch<false, false>(epi, ma, mb, mc, M, N, K, ep, dev_status, limit_ns, stream);
+  return e == cudaSuccess ? NC_OK : NC_ERR_CUDA;
+}
+
+// MN-major operand given as [K rows, MN cols] with row stride `ld` elements;
+// box = 64 MN elements x 64 K rows.
+static bool make_map_mn(CUtensorMap* map, const void* ptr, int64_t k_rows, int64_t mn_cols, int64_t ld, bool f16) {
+  const uint64_t dims[2] = {(uint64_t)mn_cols, (uint64_t)k_rows};
+  const uint64_t strides[1] = {(uint64_t)(ld * 2)};
+  const uint32_t box[2] = {64u, (uint32_t)gemm::BK};
+  return encode_tensor_map(map, f16, 2, ptr, dims, strides, box);
+}
+
+nc_status gemm_launch_layout(const uint16_t* a, int64_t lda, const uint16_t* w, int64_t ldw, int M, int N, int K,
+                             int epi, bool f16, int layout, const EpiParams& ep, uint32_t* dev_status,
+                             cudaStream_t stream, uint64_t limit_ns) {
+  using namespace gemm;
+  if (layout == GEMM_NT) return gemm_launch(a, lda, w, ldw, M, N, K, epi, f16, ep, dev_status, stream, limit_ns);
+  if (layout != GEMM_NN && layout != GEMM_TN) return NC_ERR_INVALID_ARG;
+  if (epi != EPI_STORE_16 && epi != EPI_STORE_F32 && epi != EPI_RESID_F32 && epi != EPI_RELU2_BWD_16)
+    return NC_ERR_INVALID_ARG;
+  if (nc_status s = check_epi(epi, K, BK, ep)) return s;
+  CUtensorMap ma, mb, mc;
+  const bool ok_a = layout == GEMM_TN ? make_map_mn(&ma, a, K, M, lda, f16) : make_map(&ma, a, M, K, lda, BM, f16);
+  if (!ok_a || !make_map_mn(&mb, w, K, N, ldw, f16)) return NC_ERR_CUDA;
+  if (!make_out_map(&mc, epi, M, N, f16, ep)) return NC_ERR_CUDA;
+  cudaError_t e;
+  if (layout == GEMM_NN)
+    e = f16 ? dispatch_layout<true, GEMM_NN>(epi, ma, mb, mc, M, N, K, ep, dev_status, limit_ns, stream)
+            : dispatch_layout<false, GEMM_NN>(epi, ma, mb, mc, M, N, K, ep, dev_status, limit_ns, stream);
+  else
+    e = f16 ? dispatch_layout<true, GEMM_TN>(epi, ma, mb, mc, M, N, K, ep, dev_status, limit_ns, stream)
+            : dispatch_layout<false, GEMM_TN>(epi, ma, mb, mc, M, N, K, ep, dev_status, limit_ns, stream);
   return e == cudaSuccess ? NC_OK : NC_ERR_CUDA;
 }
 

@@ -23,7 +23,15 @@ enum : int {
   EPI_CE_PARTIAL = 5,   // soft-cap, per-tile sum of exp(l - cap), target logit
   EPI_QKV_ROPE = 6,     // q/k heads: RoPE + per-head RMSNorm; v heads: plain store
   EPI_QKV_ROPE_IL = 7,  // as EPI_QKV_ROPE with q/k head dims pair-interleaved (see nc_forward)
+  EPI_CE_BWD_16 = 8,    // backward of soft-cap + cross-entropy from the recomputed logits:
+                        //   out16 = (exp(l - lse_row) - [col == target]) (1 - (l / cap)^2)
+  EPI_RELU2_BWD_16 = 9, // out16 = acc * 2 sqrt(h) with h = relu(u)^2 the saved 16-bit output
 };
+
+// Operand layouts of the GEMM.  NT: a [M, K], w [N, K] (both K contiguous);
+// NN: a [M, K], w given as [K, N] (dgrad: dX = dY W with W stored [N_out, K_in]);
+// TN: a given as [K, M], w given as [K, N] (wgrad: dW = dY^T X over the tokens).
+enum : int { GEMM_NT = 0, GEMM_NN = 1, GEMM_TN = 2 };
 
 struct EpiParams {
   void* out;                // 16-bit or fp32 output (or logits for EPI_CE_PARTIAL)
@@ -52,6 +60,14 @@ struct EpiParams {
                             //   s = 448 / max(amax, 1e-12)
   float* amax_out;          // EPI_RELU2_16 with e4m3 operands: fold max |stored output| into
                             //   this slot (the quantisation of the output that follows)
+  float alpha;              // fp32 epilogues: acc is multiplied by alpha first (0: by 1)
+  const float* alpha_ptr;   //   or by *alpha_ptr (device), when given
+  const float* row_lse;     // EPI_CE_BWD_16: [M] log-sum-exp of each row's capped logits (plus
+                            //   ce_target[row] when ce_target is given: the forward's token
+                            //   loss plus target logit)
+  const uint16_t* aux;      // EPI_RELU2_BWD_16: h [M, ld_aux] (16-bit)
+  int64_t ld_aux;
+  float* rstd_out;          // EPI_QKV_ROPE_IL: [M, H + Hkv] the QK-norm factor of each q/k head
 };
 
 // ---- device / argument helpers (nc_api.cu)
@@ -75,7 +91,32 @@ nc_status gemm_launch_e4m3(const uint8_t* a, int64_t lda, const uint8_t* w, int6
                            int epi, bool f16, const EpiParams& ep, uint32_t* dev_status, cudaStream_t stream,
                            uint64_t limit_ns = kWaitLimitNs);
 
+// 16-bit GEMM in one of the GEMM_* layouts (see above); lda / ldw are the row
+// strides of a and w as given.  GEMM_NN and GEMM_TN take EPI_STORE_16,
+// EPI_STORE_F32, EPI_RESID_F32 and EPI_RELU2_BWD_16.
+nc_status gemm_launch_layout(const uint16_t* a, int64_t lda, const uint16_t* w, int64_t ldw, int M, int N, int K,
+                             int epi, bool f16, int layout, const EpiParams& ep, uint32_t* dev_status,
+                             cudaStream_t stream, uint64_t limit_ns = kWaitLimitNs);
+
 nc_status selftest_wait_launch(uint32_t* dev_status, uint64_t limit_ns, cudaStream_t stream);
+
+// ---- backward (nc_backward.cu); gradients of the summed token losses
+// dx_acc (+)= RMSNorm backward of x with upstream dy; dx16 = dx_acc in 16-bit.
+nc_status rmsnorm_bwd_launch(const float* x, const float* dy, float* dx_acc, uint16_t* dx16, int M, int C, float eps,
+                             bool accumulate, bool f16, cudaStream_t stream);
+// In place on the q and k columns of dqkv: QK-norm backward, then inverse RoPE
+// (pair-interleaved columns), from the saved normalised qkv and QK-norm factors.
+nc_status qk_bwd_launch(uint16_t* dqkv, const uint16_t* qkv, int64_t ld, const float* rstd, const float* rope,
+                        int rope_T, int M, int T, int H, int Hkv, int D, bool f16, cudaStream_t stream);
+// dq, dk, dv (into the q / k / v columns of dqkv) from qkv, o, dO [M, H*D], the
+// forward's lse [M, H]; delta [M, H] is scratch.
+nc_status attn_bwd_launch(const uint16_t* qkv, int64_t ldqkv, const uint16_t* o, const uint16_t* dO,
+                          const float* lse, float* delta, uint16_t* dqkv, int B, int T, int H, int Hkv, int D,
+                          int window, bool f16, cudaStream_t stream);
+nc_status embedding_bwd_launch(const int32_t* tokens, const float* dx, float* dwte, int M, int C, int V,
+                               const float* alpha, cudaStream_t stream);
+nc_status qkv_grad_scatter_launch(const float* packed, float* gq, float* gk, float* gv, int H, int Hkv, int D, int C,
+                                  float alpha, cudaStream_t stream);
 
 // ---- dynamic tensorwise e4m3 quantisation (nc_fp8.cu)
 enum { FP8_SRC_F32 = 0, FP8_SRC_BF16 = 1, FP8_SRC_F16 = 2 };
@@ -105,7 +146,7 @@ bool encode_tensor_map_f32(CUtensorMap* map, int rank, const void* base, const u
 nc_status attention_launch(const uint16_t* q, const uint16_t* k, const uint16_t* v, uint16_t* out,
                            int B, int T, int H, int Hkv, int D, int window, int64_t q_stride,
                            int64_t kv_stride, bool f16, uint32_t* dev_status, cudaStream_t stream,
-                           float* amax = nullptr);
+                           float* amax = nullptr, float* lse = nullptr);
 
 // ---- elementwise / row kernels (nc_rowops.cu)
 struct CastSeg {
@@ -169,7 +210,8 @@ nc_status softcap_ce_launch(const float* z, const int32_t* targets, float* cappe
 nc_status ce_finalize_launch(const float* partial, int n_tiles, const float* target_logit,
                              const int32_t* targets, float* token_loss, int M, int V, float cap,
                              uint32_t* dev_status, cudaStream_t stream);
+// loss = mean token loss over targets in [0, V); inv_count (optional) = 1 / that count (0 if none).
 nc_status loss_mean_launch(const float* token_loss, const int32_t* targets, int M, int V,
-                           float* loss, cudaStream_t stream);
+                           float* loss, cudaStream_t stream, float* inv_count = nullptr);
 
 }  // namespace nc

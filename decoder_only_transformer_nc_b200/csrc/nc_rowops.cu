@@ -524,7 +524,7 @@ __global__ void __launch_bounds__(256) ce_finalize_kernel(const float* __restric
 // Single CTA, fixed-order reduction in fp64: mean over valid targets.
 __global__ void __launch_bounds__(1024) loss_mean_kernel(const float* __restrict__ token_loss,
                                                          const int32_t* __restrict__ targets, int M,
-                                                         int V, float* loss) {
+                                                         int V, float* loss, float* inv_count) {
   __shared__ double rs[32];
   __shared__ int rc[32];
   double s = 0.0;
@@ -556,7 +556,10 @@ __global__ void __launch_bounds__(1024) loss_mean_kernel(const float* __restrict
       s += __shfl_xor_sync(0xffffffffu, s, o);
       c += __shfl_xor_sync(0xffffffffu, c, o);
     }
-    if (lane == 0) loss[0] = c > 0 ? (float)(s / (double)c) : __int_as_float(0x7fc00000);
+    if (lane == 0) {
+      loss[0] = c > 0 ? (float)(s / (double)c) : __int_as_float(0x7fc00000);
+      if (inv_count) inv_count[0] = c > 0 ? (float)(1.0 / (double)c) : 0.0f;
+    }
   }
 }
 
@@ -709,8 +712,8 @@ nc_status ce_finalize_launch(const float* partial, int n_tiles, const float* tar
 }
 
 nc_status loss_mean_launch(const float* token_loss, const int32_t* targets, int M, int V,
-                           float* loss, cudaStream_t stream) {
-  loss_mean_kernel<<<1, 1024, 0, stream>>>(token_loss, targets, M, V, loss);
+                           float* loss, cudaStream_t stream, float* inv_count) {
+  loss_mean_kernel<<<1, 1024, 0, stream>>>(token_loss, targets, M, V, loss, inv_count);
   return last_error();
 }
 

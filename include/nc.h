@@ -266,8 +266,16 @@ typedef enum {
   NC_K_GEMM_LM_HEAD = 10,
   NC_K_CE_FINALIZE = 11,
   NC_K_LOSS_MEAN = 12,
-  NC_K_FP8_QUANT = 13,  /* amax + e4m3 quantisation of one activation (2 launches) */
-  NC_K_COUNT = 14
+  NC_K_FP8_QUANT = 13,  /* e4m3 quantisation of one activation (+ its amax when no producer folded it) */
+  NC_K_COPY = 14,       /* residual-stream snapshot of the training forward (device copy) */
+  NC_K_CE_BWD = 15,     /* logit gradient: lm_head recomputed, soft-cap + CE backward epilogue */
+  NC_K_GEMM_DGRAD = 16, /* dX = dY W (tcgen05, W as the MN-major operand) */
+  NC_K_GEMM_WGRAD = 17, /* dW += dY^T X over the tokens (tcgen05, both operands MN-major) */
+  NC_K_NORM_BWD = 18,   /* RMSNorm backward into the residual gradient */
+  NC_K_ATTN_BWD = 19,   /* attention backward: Delta, dQ, dK/dV (3 launches) */
+  NC_K_QK_BWD = 20,     /* QK-norm + RoPE backward */
+  NC_K_EMB_BWD = 21,    /* embedding backward, and the QKV weight-gradient scatter */
+  NC_K_COUNT = 22
 } nc_kernel_kind;
 
 /* Per-launch timing hook.  `events` holds 2*capacity cudaEvent_t handles
@@ -368,6 +376,80 @@ typedef enum {
 nc_status nc_linear(const uint16_t* a, const uint16_t* w, void* out, int M, int N, int K,
                     int64_t ldo, nc_epilogue epilogue, float cap, nc_dtype dtype,
                     uint32_t* dev_status, void* stream);
+
+/* ---------------------------------------------------------------- backward
+ * The training micro-step's loss.backward() ("从文本到聊天模型" §6.5): the
+ * mean loss of the plain block stack and its gradient with respect to every
+ * fp32 master weight.  The fp32 -> 16-bit cast of a weight is taken as
+ * straight-through (dW = dY^T X).  Targets of -1 contribute nothing; the mean
+ * is over the others.  */
+
+/* fp32 gradients, device pointers; the per-layer members are HOST arrays of
+ * n_layer device pointers, each the shape of its weight in nc_weights.  The
+ * backward ADDS into them (zero them for a fresh step, keep them to accumulate
+ * micro-steps).  16-byte aligned. */
+typedef struct {
+  float* wte;                 /* [V, C]        */
+  float* const* c_q;          /* n_layer x [H*D, C]   */
+  float* const* c_k;          /* n_layer x [Hkv*D, C] */
+  float* const* c_v;          /* n_layer x [Hkv*D, C] */
+  float* const* attn_proj;    /* n_layer x [C, H*D]   */
+  float* const* c_fc;         /* n_layer x [4C, C]    */
+  float* const* mlp_proj;     /* n_layer x [C, 4C]    */
+  float* lm_head;             /* [V, C]        */
+} nc_grads;
+
+/* Workspace bytes of nc_forward_backward for a [B, T] batch (0 on bad input):
+ * the 16-bit weights, per layer the activations the backward reads (residual
+ * stream at the block's input and after attention, q|k|v, the QK-norm factors,
+ * the attention output and its log-sum-exp, the MLP hidden activations), the
+ * 16-bit gradient of the logits [B*T, V] and the backward's scratch.  Host only. */
+size_t nc_train_workspace_bytes(const nc_config* cfg, int B, int T);
+
+/* Forward with the activations kept, then the backward: writes *loss (device
+ * float, the mean over counted targets) and adds the gradients into *g.
+ * cfg->extras and cfg->fp8 must be 0 (NC_ERR_CONFIG).  tokens, targets [B, T]
+ * int32 device.  The attention backward runs on the warp-level mma.sync path;
+ * the projections' products on the tcgen05 GEMM.  Split-K weight gradients
+ * are summed in no fixed order (not bitwise reproducible run to run).
+ * Asynchronous on `stream`. */
+nc_status nc_forward_backward(const nc_config* cfg, const nc_weights* w, const int32_t* tokens,
+                              const int32_t* targets, int B, int T, float* loss, const nc_grads* g,
+                              void* workspace, size_t ws_bytes, void* stream);
+
+/* The same, recording each step's pair of events into *trace (as
+ * nc_forward_traced: trace->count = the number of steps, 12 + 24 n_layer). */
+nc_status nc_forward_backward_traced(const nc_config* cfg, const nc_weights* w, const int32_t* tokens,
+                                     const int32_t* targets, int B, int T, float* loss, const nc_grads* g,
+                                     void* workspace, size_t ws_bytes, void* stream, nc_trace* trace);
+
+/* nc_attention_strided that also writes lse [B*T, H] (fp32, device): the
+ * natural log-sum-exp of each query row's scaled, visible scores, which the
+ * backward uses to recompute the attention weights. */
+nc_status nc_attention_lse(const uint16_t* q, const uint16_t* k, const uint16_t* v, uint16_t* out, float* lse,
+                           int B, int T, int H, int Hkv, int D, int window, int64_t q_row_stride,
+                           int64_t kv_row_stride, nc_dtype dtype, void* stream);
+
+/* Attention backward: qkv [B*T, (H + 2 Hkv) D] packed q | k | v heads (the
+ * fused projection's layout), o and dO [B*T, H*D], lse as nc_attention_lse
+ * writes it; dqkv gets dq | dk | dv in qkv's layout (dk, dv summed over the
+ * query heads of each kv group).  delta [B*T, H] fp32 is scratch.  Warp-level
+ * mma.sync tensor cores, fp32 accumulation; no atomics. */
+nc_status nc_attention_backward(const uint16_t* qkv, const uint16_t* o, const uint16_t* dO, const float* lse,
+                                float* delta, uint16_t* dqkv, int B, int T, int H, int Hkv, int D, int window,
+                                nc_dtype dtype, void* stream);
+
+/* The two products of a linear layer's backward, on the tcgen05 GEMM with
+ * 16-bit operands in format dtype (device, 16-byte aligned, row-major):
+ * dgrad  dx [M, K] = dy [M, N] . w [N, K]  (w as stored for the forward);
+ *        epilogue NC_EPI_STORE_16 (dx in dtype) or NC_EPI_STORE_F32 (fp32);
+ * wgrad  dw [N, K] += alpha dy[M, N]^T . x [M, K]  (fp32, summed over the M
+ *        rows; split over M in no fixed order).
+ * N % 8 == 0 and K % 8 == 0; M >= 1. */
+nc_status nc_linear_dgrad(const uint16_t* dy, const uint16_t* w, void* dx, int M, int N, int K,
+                          nc_epilogue epilogue, nc_dtype dtype, uint32_t* dev_status, void* stream);
+nc_status nc_linear_wgrad(const uint16_t* dy, const uint16_t* x, float* dw, int M, int N, int K, float alpha,
+                          nc_dtype dtype, uint32_t* dev_status, void* stream);
 
 /* Dynamic tensorwise e4m3 quantisation of one tensor (the NC_FP8_* rule
  * above): x [n] in src_dtype (NC_F32, NC_BF16 or NC_F16; device, 16-byte

@@ -55,6 +55,40 @@ def _mask(T, W):
     return (j <= i) & ((i - j) < W)
 
 
+def attention_backward(q, k, v, do, W):
+    """Gradients of o = softmax(q k^T / sqrt(D), window W, causal) v for one
+    layer, with query head h reading kv head h // (H / Hkv).
+
+    q [B, T, H, D], k and v [B, T, Hkv, D], do = dL/do [B, T, H, D].  With
+    P the attention weights: dV = P^T dO, dP = dO V^T, dS = P o (dP - rowsum(dP o P)),
+    dQ = dS K / sqrt(D), dK = dS^T Q / sqrt(D) (summed over the heads of a group).
+    Returns (dq, dk, dv) and P [B, H, T, T].
+    """
+    B, T, H, D = q.shape
+    Hkv = k.shape[2]
+    G = H // Hkv
+    scale = 1.0 / np.sqrt(D)
+    m = _mask(T, W)
+    dq = np.zeros((B, T, H, D))
+    dk = np.zeros((B, T, Hkv, D))
+    dv = np.zeros((B, T, Hkv, D))
+    P = np.empty((B, H, T, T))
+    for h in range(H):
+        g = h // G
+        sc = np.einsum("bid,bjd->bij", q[:, :, h], k[:, :, g]) * scale
+        sc = np.where(m[None], sc, -np.inf)
+        sc = sc - sc.max(axis=-1, keepdims=True)
+        e = np.exp(sc)
+        Ph = e / e.sum(axis=-1, keepdims=True)
+        P[:, h] = Ph
+        dv[:, :, g] += np.einsum("bij,bid->bjd", Ph, do[:, :, h])
+        dP = np.einsum("bid,bjd->bij", do[:, :, h], v[:, :, g])
+        dS = Ph * (dP - np.sum(dP * Ph, axis=-1, keepdims=True)) * scale
+        dq[:, :, h] = np.einsum("bij,bjd->bid", dS, k[:, :, g])
+        dk[:, :, g] += np.einsum("bij,bid->bjd", dS, q[:, :, h])
+    return dq, dk, dv, P
+
+
 def _forward(cfg: OracleConfig, weights: dict, idx: np.ndarray, targets: np.ndarray, cast):
     """The forward of ``model.forward`` (plain stack) keeping what the backward reads."""
     idx = np.asarray(idx)
@@ -101,7 +135,8 @@ def _forward(cfg: OracleConfig, weights: dict, idx: np.ndarray, targets: np.ndar
         u = a2 @ lw["c_fc"].T
         hh = np.maximum(u, 0.0) ** 2
         x = x_mid + hh @ lw["mlp_proj"].T
-        s.update(r1=r1, a=a, q=q, k=k, v=v, rq=rq, rk=rk, P=P, of=of, x_mid=x_mid, r2=r2, a2=a2, u=u, h=hh)
+        s.update(r1=r1, a=a, q=q, k=k, v=v, rq=rq, rk=rk, P=P, of=of, x_mid=x_mid, r2=r2, a2=a2, u=u, h=hh,
+                 W=windows[l])
         saved.append(s)
     rf = _rms_rstd(x, eps)
     af = x * rf
@@ -152,17 +187,7 @@ def forward_backward(cfg: OracleConfig, weights: dict, idx: np.ndarray, targets:
         # attention block: x_mid = x_in + o W_p^T
         gl["attn_proj"] = np.einsum("btc,bte->ce", dx_mid, s["of"])
         do = (dx_mid @ lw["attn_proj"]).reshape(B, T, H, D)
-        dq = np.zeros((B, T, H, D))
-        dk = np.zeros((B, T, Hkv, D))
-        dv = np.zeros((B, T, Hkv, D))
-        for h in range(H):
-            g = h // G
-            Ph = s["P"][:, h]
-            dv[:, :, g] += np.einsum("bij,bid->bjd", Ph, do[:, :, h])
-            dP = np.einsum("bid,bjd->bij", do[:, :, h], s["v"][:, :, g])
-            dS = Ph * (dP - np.sum(dP * Ph, axis=-1, keepdims=True)) * scale
-            dq[:, :, h] = np.einsum("bij,bjd->bid", dS, s["k"][:, :, g])
-            dk[:, :, g] += np.einsum("bij,bid->bjd", dS, s["q"][:, :, h])
+        dq, dk, dv, _ = attention_backward(s["q"], s["k"], s["v"], do, s["W"])
         # QK-norm after RoPE, then the inverse rotation
         duq = _rope_apply(rmsnorm_backward(s["q"], s["rq"], dq), cos, sin, -1.0).reshape(B, T, H * D)
         duk = _rope_apply(rmsnorm_backward(s["k"], s["rk"], dk), cos, sin, -1.0).reshape(B, T, Hkv * D)

@@ -281,3 +281,42 @@ def test_fp8_host_rules(nclib):
     if not torch.cuda.is_available():
         assert lin(128, 64, 64, 64) == 8
         assert q(1 << 40, nclib.F32, 16, 1 << 40, 1 << 41) == 8
+
+
+def test_backward_host_rules(nclib):
+    """Sizing and host-side refusals of nc_forward_backward and the backward products."""
+    L = nclib.lib()
+    cfg = nclib.init_config(2, 64, 64, 0, 256, 512)
+    n = nclib.train_workspace_bytes(cfg, 2, 100)
+    M, C, V = 200, cfg.d_model, cfg.vocab
+    # at least the saved residual streams (2L + 1 fp32 [M, C]) and the logit gradient [M, V] (16-bit)
+    assert n >= (2 * cfg.n_layer + 1) * M * C * 4 + M * V * 2
+    assert nclib.train_workspace_bytes(cfg, 2, 300) == 0  # T > seq_len
+    for field, val in (("extras", nclib.EXTRA_SMEAR), ("fp8", nclib.FP8_BLOCK)):
+        c = nclib.NcConfig.from_buffer_copy(cfg)
+        setattr(c, field, val)
+        assert nclib.train_workspace_bytes(c, 2, 100) == 0
+    fw = _FakeWeights(nclib, 2)
+    arr = (ctypes.c_void_p * 2)(1 << 40, (1 << 40) + 4096)
+    FPP = ctypes.POINTER(ctypes.c_void_p)
+    g = nclib.NcGrads(1 << 41, *[ctypes.cast(arr, FPP)] * 6, 1 << 42)
+    fb = lambda c, T=100, ws_bytes=n, loss=1 << 43, grads=g: L.nc_forward_backward(
+        ctypes.byref(c), ctypes.byref(fw.w), 1 << 41, 1 << 41, 2, T, loss, ctypes.byref(grads), 1 << 44, ws_bytes,
+        None)
+    assert fb(cfg, T=300) == 3
+    assert fb(cfg, ws_bytes=n - 1) == 5
+    assert fb(cfg, loss=None) == 1
+    c = nclib.NcConfig.from_buffer_copy(cfg)
+    c.fp8 = nclib.FP8_BLOCK
+    assert fb(c) == 2
+    g_bad = nclib.NcGrads(1 << 41, *[ctypes.cast(arr, FPP)] * 6, (1 << 42) + 4)
+    assert fb(cfg, grads=g_bad) == 4
+    A = 1 << 40
+    assert L.nc_linear_dgrad(A, A, A, 128, 60, 64, 3, 1, None, None) == 3     # N % 8
+    assert L.nc_linear_dgrad(A, A, A, 128, 64, 64, 4, 1, None, None) == 1     # epilogue
+    assert L.nc_linear_wgrad(A, A, A, 0, 64, 64, 1.0, 1, None, None) == 1     # M < 1
+    assert L.nc_linear_wgrad(A + 2, A, A, 8, 64, 64, 1.0, 1, None, None) == 4
+    import torch
+    if not torch.cuda.is_available():
+        assert fb(cfg) == 8
+        assert L.nc_linear_dgrad(A, A, A, 128, 64, 64, 3, 1, None, None) == 8
