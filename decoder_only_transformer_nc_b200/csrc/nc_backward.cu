@@ -272,6 +272,33 @@ __device__ __forceinline__ void stage_tile(uint16_t* dst, const uint16_t* src, i
   }
 }
 
+// The same with 16-byte cp.async copies (rows >= T zero-filled), so the load
+// of the next tile overlaps the products of the current one.
+__device__ __forceinline__ void cp_async16(uint16_t* dst, const uint16_t* src, bool valid) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src),
+               "r"(valid ? 16 : 0)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async4(float* dst, const float* src, bool valid) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(smem_u32(dst)), "l"(src), "r"(valid ? 4 : 0)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+template <int D, int LD>
+__device__ __forceinline__ void stage_tile_async(uint16_t* dst, const uint16_t* src, int64_t ld, int64_t row_base,
+                                                 int row0, int T) {
+  constexpr int CH = D / 8;
+  for (int i = threadIdx.x; i < BLK * CH; i += NTH) {
+    const int r = i / CH, c = i % CH;
+    const bool valid = row0 + r < T;
+    const uint16_t* g = src + (row_base + (valid ? row0 + r : 0)) * ld + c * 8;
+    cp_async16(dst + r * LD + c * 8, g, valid);
+  }
+}
+
 // S (16 x 64 per warp) = A_tile[rows w*16..] . B_tile^T over D, both [row][D] tiles.
 template <int D, int LD, bool F16>
 __device__ __forceinline__ void tile_dots(float (&acc)[8][4], uint32_t a_base, uint32_t b_base, int wrow, int lane) {
@@ -339,8 +366,7 @@ __global__ void __launch_bounds__(NTH, 1)
   extern __shared__ __align__(16) uint8_t smem_raw[];
   uint16_t* sQ = reinterpret_cast<uint16_t*>(smem_raw);
   uint16_t* sdO = sQ + BLK * LD;
-  uint16_t* sK = sdO + BLK * LD;
-  uint16_t* sV = sK + BLK * LD;
+  uint16_t* sKV = sdO + BLK * LD;  // two buffers of (K tile, V tile)
   const int q0 = blockIdx.x * BLK, h = blockIdx.y, b = blockIdx.z;
   const int g = h / (H / Hkv);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -359,13 +385,24 @@ __global__ void __launch_bounds__(NTH, 1)
     for (int e = 0; e < 4; ++e) dq[i][e] = 0.0f;
   const int q_last = min(T - 1, q0 + BLK - 1);
   const int kt_lo = max(0, q0 - W + 1) / BLK, kt_hi = q_last / BLK;
-  const uint32_t bq = smem_u32(sQ), bdo = smem_u32(sdO), bk = smem_u32(sK), bv = smem_u32(sV);
+  const uint32_t bq = smem_u32(sQ), bdo = smem_u32(sdO);
+  auto issue = [&](int kt) {  // K and V tiles of key tile kt into buffer kt & 1
+    uint16_t* dst = sKV + (kt & 1) * 2 * BLK * LD;
+    stage_tile_async<D, LD>(dst, qkv + (int64_t)(H + g) * D, ldqkv, rb, kt * BLK, T);
+    stage_tile_async<D, LD>(dst + BLK * LD, qkv + (int64_t)(H + Hkv + g) * D, ldqkv, rb, kt * BLK, T);
+    cp_async_commit();
+  };
+  issue(kt_lo);
   for (int kt = kt_lo; kt <= kt_hi; ++kt) {
     const int k0 = kt * BLK;
+    if (kt < kt_hi) {
+      issue(kt + 1);
+      cp_async_wait<1>();  // this tile's group has landed; the next one may still be in flight
+    } else {
+      cp_async_wait<0>();
+    }
     __syncthreads();
-    stage_tile<D, LD>(sK, qkv + (int64_t)(H + g) * D, ldqkv, rb, k0, T);
-    stage_tile<D, LD>(sV, qkv + (int64_t)(H + Hkv + g) * D, ldqkv, rb, k0, T);
-    __syncthreads();
+    const uint32_t bk = smem_u32(sKV + (kt & 1) * 2 * BLK * LD), bv = bk + BLK * LD * 2;
     float s[8][4], dp[8][4];
     tile_dots<D, LD, F16>(s, bq, bk, warp * 16, lane);
     tile_dots<D, LD, F16>(dp, bdo, bv, warp * 16, lane);
@@ -380,6 +417,7 @@ __global__ void __launch_bounds__(NTH, 1)
         s[nt][e] = p * (dp[nt][e] - (e < 2 ? dl_a : dl_b));  // dS / scale
       }
     tile_accum<D, LD, F16>(dq, s, bk, lane);
+    __syncthreads();  // buffer kt & 1 is refilled by the issue of tile kt + 2
   }
   store_rows<D, F16>(dq, dqkv + (int64_t)h * D, ldqkv, rb, q0 + warp * 16, T, lane, scale);
 }
@@ -393,9 +431,8 @@ __global__ void __launch_bounds__(NTH, 1)
   extern __shared__ __align__(16) uint8_t smem_raw[];
   uint16_t* sK = reinterpret_cast<uint16_t*>(smem_raw);
   uint16_t* sV = sK + BLK * LD;
-  uint16_t* sQ = sV + BLK * LD;
-  uint16_t* sdO = sQ + BLK * LD;
-  float* sL = reinterpret_cast<float*>(sdO + BLK * LD);  // [BLK] lse, then [BLK] delta
+  uint16_t* sQD = sV + BLK * LD;                            // two buffers of (Q tile, dO tile)
+  float* sLD = reinterpret_cast<float*>(sQD + 4 * BLK * LD);  // two buffers of ([BLK] lse, [BLK] delta)
   const int k0 = blockIdx.x * BLK, g = blockIdx.y, b = blockIdx.z;
   const int G = H / Hkv;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -412,20 +449,35 @@ __global__ void __launch_bounds__(NTH, 1)
     for (int e = 0; e < 4; ++e) dk[i][e] = dv[i][e] = 0.0f;
   const int k_last = min(T - 1, k0 + BLK - 1);
   const int qt_lo = k0 / BLK, qt_hi = min(T - 1, k_last + W - 1) / BLK;
-  const uint32_t bq = smem_u32(sQ), bdo = smem_u32(sdO), bk = smem_u32(sK), bv = smem_u32(sV);
-  for (int hi = 0; hi < G; ++hi) {
-    const int h = g * G + hi;
-    for (int qt = qt_lo; qt <= qt_hi; ++qt) {
-      const int q0 = qt * BLK;
-      __syncthreads();
-      stage_tile<D, LD>(sQ, qkv + (int64_t)h * D, ldqkv, rb, q0, T);
-      stage_tile<D, LD>(sdO, dO + (int64_t)h * D, HD, rb, q0, T);
-      for (int i = threadIdx.x; i < BLK; i += NTH) {
-        const bool in = q0 + i < T;
-        sL[i] = in ? lse[(rb + q0 + i) * H + h] : 0.0f;
-        sL[BLK + i] = in ? delta[(rb + q0 + i) * H + h] : 0.0f;
+  const uint32_t bk = smem_u32(sK), bv = smem_u32(sV);
+  const int nq = qt_hi - qt_lo + 1, n_it = G * nq;  // iterations: (head of the group, query tile)
+  auto issue = [&](int it) {  // Q, dO tiles and lse, delta of iteration it into buffer it & 1
+    const int h = g * G + it / nq, q0 = (qt_lo + it % nq) * BLK;
+    uint16_t* dst = sQD + (it & 1) * 2 * BLK * LD;
+    stage_tile_async<D, LD>(dst, qkv + (int64_t)h * D, ldqkv, rb, q0, T);
+    stage_tile_async<D, LD>(dst + BLK * LD, dO + (int64_t)h * D, HD, rb, q0, T);
+    float* l = sLD + (it & 1) * 2 * BLK;
+    for (int i = threadIdx.x; i < BLK; i += NTH) {
+      const bool in = q0 + i < T;
+      const int64_t r = (rb + (in ? q0 + i : 0)) * H + h;
+      cp_async4(l + i, lse + r, in);
+      cp_async4(l + BLK + i, delta + r, in);
+    }
+    cp_async_commit();
+  };
+  if (n_it > 0) issue(0);
+  for (int it = 0; it < n_it; ++it) {
+    {
+      const int q0 = (qt_lo + it % nq) * BLK;
+      if (it + 1 < n_it) {
+        issue(it + 1);
+        cp_async_wait<1>();
+      } else {
+        cp_async_wait<0>();
       }
       __syncthreads();
+      const uint32_t bq = smem_u32(sQD + (it & 1) * 2 * BLK * LD), bdo = bq + BLK * LD * 2;
+      const float* sL = sLD + (it & 1) * 2 * BLK;
       float s[8][4], dp[8][4];
       tile_dots<D, LD, F16>(s, bk, bq, warp * 16, lane);   // S^T: keys x queries
       tile_dots<D, LD, F16>(dp, bv, bdo, warp * 16, lane); // dP^T
@@ -443,6 +495,7 @@ __global__ void __launch_bounds__(NTH, 1)
         }
       tile_accum<D, LD, F16>(dv, s, bdo, lane);
       tile_accum<D, LD, F16>(dk, dp, bq, lane);
+      __syncthreads();  // buffer it & 1 is refilled by the issue of iteration it + 2
     }
   }
   store_rows<D, F16>(dk, dqkv + (int64_t)(H + g) * D, ldqkv, rb, k0 + warp * 16, T, lane, scale);
@@ -454,8 +507,8 @@ static nc_status attn_bwd_t(const uint16_t* qkv, int64_t ldqkv, const uint16_t* 
                             const float* delta, uint16_t* dqkv, int B, int T, int H, int Hkv, int W,
                             cudaStream_t stream) {
   constexpr int LD = D + 8;
-  const int smem_q = 4 * BLK * LD * 2;
-  const int smem_k = smem_q + 2 * BLK * 4;
+  const int smem_q = 6 * BLK * LD * 2;                  // Q, dO, and two (K, V) buffers
+  const int smem_k = 6 * BLK * LD * 2 + 4 * BLK * 4;    // K, V, two (Q, dO) and two (lse, delta) buffers
   static bool attr_done[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
