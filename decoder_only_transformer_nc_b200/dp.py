@@ -1,10 +1,17 @@
-"""Data-parallel plumbing of the forward (one process per GPU).
+"""Data-parallel plumbing (one process per GPU).
 
-The forward shards by batch row ("从文本到聊天模型" §4.5: each rank reads its own
-rows): every rank holds the whole model and runs ``nc_forward`` on its own
-[B, T] shard.  The only exchange is the global mean loss: each rank
-contributes (local mean * local count, local count) and one all-reduce of that
-2-vector (fp64) gives sum / count over all ranks' non-ignored targets.
+The batch shards by row ("从文本到聊天模型" §4.5: each rank reads its own rows):
+every rank holds the whole model and runs the library on its own [B, T] shard.
+
+* Forward: the only exchange is the global mean loss.  Each rank contributes
+  (local mean * local count, local count); one all-reduce of that 2-vector
+  (fp64) gives sum / count over all ranks' non-ignored targets.
+* Training micro-step (``nc_forward_backward``): each rank's gradients are of
+  its local mean loss.  The gradient of the global mean is
+  sum_r count_r g_r / sum_r count_r.  All weight gradients live in one flat
+  fp32 bucket (``grad_bucket``) whose last slot carries the count, so one
+  all-reduce of count * g, followed by a device-side division, averages them
+  with no host synchronisation (``average_grads_``).
 """
 from __future__ import annotations
 
@@ -33,3 +40,48 @@ def reduce_loss_into(buf: torch.Tensor, local_mean: torch.Tensor, local_count: f
 def global_mean_loss(local_mean: torch.Tensor, local_count: float, group=None) -> torch.Tensor:
     buf = torch.zeros(2, dtype=torch.float64, device=local_mean.device)
     return reduce_loss_into(buf, local_mean, local_count, group)
+
+
+NAMES = ("c_q", "c_k", "c_v", "attn_proj", "c_fc", "mlp_proj")
+
+
+def grad_bucket(tensors: dict, device=None):
+    """One flat fp32 buffer holding a gradient for every weight of ``tensors``
+    (the layout of ``Model.tensors``), each view starting on a 16-byte boundary,
+    plus a last slot for the local target count.  Returns (flat, grads) with
+    ``grads`` in the layout ``forward_backward`` takes; the buffer is zeroed."""
+    shapes = [("wte", tensors["wte"].shape), ("lm_head", tensors["lm_head"].shape)]
+    for l, lw in enumerate(tensors["layers"]):
+        shapes += [((l, n), lw[n].shape) for n in NAMES]
+    offs, off = [], 0
+    for _, shp in shapes:
+        offs.append(off)
+        n = 1
+        for d in shp:
+            n *= d
+        off += (n + 3) // 4 * 4
+    dev = device if device is not None else tensors["wte"].device
+    flat = torch.zeros(off + 4, dtype=torch.float32, device=dev)
+    grads = {"layers": [dict() for _ in tensors["layers"]]}
+    for (key, shp), o in zip(shapes, offs):
+        n = 1
+        for d in shp:
+            n *= d
+        view = flat[o:o + n].view(shp)
+        if isinstance(key, tuple):
+            grads["layers"][key[0]][key[1]] = view
+        else:
+            grads[key] = view
+    return flat, grads
+
+
+def average_grads_(flat: torch.Tensor, local_count: float, group=None) -> torch.Tensor:
+    """In place: the bucket's gradients (of each rank's local mean loss) become
+    the gradient of the global mean loss over every rank's counted targets."""
+    body = flat[:-4]
+    body.mul_(float(local_count))
+    flat[-4:].zero_()
+    flat[-4] = float(local_count)
+    dist.all_reduce(flat, op=dist.ReduceOp.SUM, group=group)
+    body.div_(flat[-4].clamp_min(1.0))
+    return flat

@@ -53,3 +53,72 @@ def test_global_loss_over_two_gloo_ranks(tmp_path):
     for i in range(world):
         assert abs(r[i][0] - want) <= 1e-12 * abs(want)
     assert r[0][2] != r[1][2]
+
+
+def _grad_rank_main(rank, world, port, out_dir):
+    import torch.distributed as dist
+
+    import oracle
+    from oracle.grad import forward_backward
+    from decoder_only_transformer_nc_b200 import dp
+    from workloads import SHAPES, TOKEN_SEED, make_tokens, make_weights
+
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    s = SHAPES["tiny"]
+    w = make_weights(s)
+    x, y = make_tokens(s, seed=dp.shard_seed(TOKEN_SEED, rank), batch=1, seq_len=48)
+    y = y.copy()
+    if rank == 1:
+        y[0, ::4] = -1  # unequal counts
+    cfg = oracle.OracleConfig(s.n_layer, s.d_model, s.n_head, s.n_kv_head, s.head_dim, s.seq_len, s.vocab,
+                              short_window=s.short_window)
+    _, g = forward_backward(cfg, w, x, y)
+    t = {"wte": torch.from_numpy(w["wte"]), "lm_head": torch.from_numpy(w["lm_head"]),
+         "layers": [{k: torch.from_numpy(v) for k, v in lw.items()} for lw in w["layers"]]}
+    flat, grads = dp.grad_bucket(t, device="cpu")
+    grads["wte"].copy_(torch.from_numpy(g["wte"]))
+    grads["lm_head"].copy_(torch.from_numpy(g["lm_head"]))
+    for l, lw in enumerate(g["layers"]):
+        for k, v in lw.items():
+            grads["layers"][l][k].copy_(torch.from_numpy(v))
+    dp.average_grads_(flat, int((y != -1).sum()))
+    np.save(os.path.join(out_dir, f"g{rank}.npy"), flat.numpy())
+    dist.destroy_process_group()
+
+
+def test_gradient_average_matches_the_whole_batch(tmp_path):
+    """Two gloo ranks, each with the oracle's gradient of its own shard's mean
+    loss, average through the bucket; both must hold the gradient of the mean
+    over the concatenated batch (oracle, fp64), to fp32 rounding."""
+    import oracle
+    from oracle.grad import forward_backward
+    from decoder_only_transformer_nc_b200 import dp
+    from workloads import SHAPES, TOKEN_SEED, make_tokens, make_weights
+
+    world, port = 2, _free_port()
+    mp.spawn(_grad_rank_main, args=(world, port, str(tmp_path)), nprocs=world, join=True)
+    s = SHAPES["tiny"]
+    w = make_weights(s)
+    xs, ys = [], []
+    for r in range(world):
+        x, y = make_tokens(s, seed=dp.shard_seed(TOKEN_SEED, r), batch=1, seq_len=48)
+        y = y.copy()
+        if r == 1:
+            y[0, ::4] = -1
+        xs.append(x)
+        ys.append(y)
+    cfg = oracle.OracleConfig(s.n_layer, s.d_model, s.n_head, s.n_kv_head, s.head_dim, s.seq_len, s.vocab,
+                              short_window=s.short_window)
+    _, want = forward_backward(cfg, w, np.concatenate(xs), np.concatenate(ys))
+    t = {"wte": torch.from_numpy(w["wte"]), "lm_head": torch.from_numpy(w["lm_head"]),
+         "layers": [{k: torch.from_numpy(v) for k, v in lw.items()} for lw in w["layers"]]}
+    flat, grads = dp.grad_bucket(t, device="cpu")
+    for r in range(world):
+        flat.copy_(torch.from_numpy(np.load(tmp_path / f"g{r}.npy")))
+        np.testing.assert_allclose(grads["wte"].numpy(), want["wte"], rtol=1e-5, atol=1e-9)
+        np.testing.assert_allclose(grads["lm_head"].numpy(), want["lm_head"], rtol=1e-5, atol=1e-9)
+        for l, lw in enumerate(want["layers"]):
+            for k, v in lw.items():
+                np.testing.assert_allclose(grads["layers"][l][k].numpy(), v, rtol=1e-4, atol=1e-9)
