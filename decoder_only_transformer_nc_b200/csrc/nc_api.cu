@@ -976,46 +976,49 @@ nc_status nc_decode_step(const nc_config* cfg, const nc_weights* w, const int32_
   } while (0)
   if (cudaMemsetAsync(status, 0, 256, st) != cudaSuccess) return NC_ERR_CUDA;
   NC_TRY(embedding_launch(tokens, w->wte, x, B, C, V, status, st));
-  // Few rows (B): every projection splits K over about one tile per SM.  The
-  // residual adds land in x directly; QKV and c_fc sum into an fp32 scratch that
-  // a small kernel finishes (RoPE + QK-norm + cache write, or ReLU^2).
+  // Few rows (B): every projection splits K.  The residual adds land in x
+  // directly; QKV and c_fc sum into an fp32 scratch that a small kernel finishes
+  // (RoPE + QK-norm + cache write, or ReLU^2).  Up to 32 rows the projections
+  // run on the skinny GEMM (all rows per CTA, weights streamed once); beyond,
+  // on the tcgen05 GEMM with split K.
+  const bool skinny = B <= 32;
   const int ks_qkv = resid_ksplit(B, NQKV, C), ks_fc = resid_ksplit(B, 4 * C, C);
+  // out (+)= in . w^T over the step's B rows
+  auto proj = [&](const uint16_t* in, int K, const uint16_t* wt, int N, float* out, int ks) -> nc_status {
+    if (skinny) return skinny_gemm_launch(in, K, wt, K, out, N, B, N, K, 0, 0.0f, f16, st);
+    EpiParams e{};
+    e.out = out;
+    e.ldo = N;
+    e.ksplit = ks;
+    return gemm_launch(in, K, wt, K, B, N, K, EPI_RESID_F32, f16, e, status, st);
+  };
   for (int l = 0; l < cfg->n_layer; ++l) {
     NC_TRY(rmsnorm_launch(x, a, B, C, eps, f16, st));
     uint16_t* cl = cache + l * SL.cache_layer_elems;
-    EpiParams eq{};
-    eq.out = acc;
-    eq.ldo = NQKV;
-    eq.ksplit = ks_qkv;
     if (cudaMemsetAsync(acc, 0, (size_t)B * NQKV * 4, st) != cudaSuccess) return NC_ERR_CUDA;
-    NC_TRY(gemm_launch(a, C, wqkv + l * SL.wqkv_elems, C, B, NQKV, C, EPI_RESID_F32, f16, eq, status, st));
+    NC_TRY(proj(a, C, wqkv + l * SL.wqkv_elems, NQKV, acc, ks_qkv));
     NC_TRY(qkv_finish_launch(acc, qkv, cl, rope, T_max, pos, B, H, Hkv, D, T_max, eps, f16, st));
     NC_TRY(decode_attention_launch(qkv, NQKV, cl, part, o, B, H, Hkv, D, T_max, pos, nc_layer_window(cfg, l),
                                    f16, st));
-    // Few rows: the residual adds split K over about one tile per SM (the
-    // partial products land in x by TMA reduce-add, in no fixed order).
-    EpiParams ep{};
-    ep.out = x;
-    ep.ldo = C;
-    ep.ksplit = resid_ksplit(B, C, H * D);
-    NC_TRY(gemm_launch(o, H * D, wo + l * SL.wo_elems, H * D, B, C, H * D, EPI_RESID_F32, f16, ep, status, st));
+    // the residual adds: partial products over K land in x (atomic or TMA
+    // reduce-add, in no fixed order)
+    NC_TRY(proj(o, H * D, wo + l * SL.wo_elems, C, x, resid_ksplit(B, C, H * D)));
     NC_TRY(rmsnorm_launch(x, a, B, C, eps, f16, st));
-    EpiParams ef{};
-    ef.out = acc;
-    ef.ldo = 4 * C;
-    ef.ksplit = ks_fc;
     if (cudaMemsetAsync(acc, 0, (size_t)B * 4 * C * 4, st) != cudaSuccess) return NC_ERR_CUDA;
-    NC_TRY(gemm_launch(a, C, wfc + l * SL.wfc_elems, C, B, 4 * C, C, EPI_RESID_F32, f16, ef, status, st));
+    NC_TRY(proj(a, C, wfc + l * SL.wfc_elems, 4 * C, acc, ks_fc));
     NC_TRY(relu2_finish_launch(acc, h, (int64_t)B * 4 * C, f16, st));
-    ep.ksplit = resid_ksplit(B, C, 4 * C);
-    NC_TRY(gemm_launch(h, 4 * C, wmp + l * SL.wmp_elems, 4 * C, B, C, 4 * C, EPI_RESID_F32, f16, ep, status, st));
+    NC_TRY(proj(h, 4 * C, wmp + l * SL.wmp_elems, C, x, resid_ksplit(B, C, 4 * C)));
   }
   NC_TRY(rmsnorm_launch(x, a, B, C, eps, f16, st));
-  EpiParams ep{};
-  ep.out = logits;
-  ep.ldo = V;
-  ep.cap = cfg->softcap;
-  NC_TRY(gemm_launch(a, C, wlm, C, B, V, C, EPI_SOFTCAP_F32, f16, ep, status, st));
+  if (skinny) {
+    NC_TRY(skinny_gemm_launch(a, C, wlm, C, logits, V, B, V, C, 2, cfg->softcap, f16, st));
+  } else {
+    EpiParams ep{};
+    ep.out = logits;
+    ep.ldo = V;
+    ep.cap = cfg->softcap;
+    NC_TRY(gemm_launch(a, C, wlm, C, B, V, C, EPI_SOFTCAP_F32, f16, ep, status, st));
+  }
 #undef NC_TRY
   return NC_OK;
 }

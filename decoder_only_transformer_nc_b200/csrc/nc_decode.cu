@@ -22,6 +22,7 @@
 
 #include "nc_half.cuh"
 #include "nc_internal.h"
+#include "nc_mma.cuh"
 
 namespace nc {
 namespace {
@@ -355,6 +356,102 @@ nc_status decode_dispatch(const uint16_t* q, int64_t ldq, const uint16_t* cache,
   return cudaGetLastError() == cudaSuccess ? NC_OK : NC_ERR_CUDA;
 }
 
+
+// ---------------------------------------------------------------- skinny GEMM
+// The projections of a decode step: out (+)= A W^T with A [M <= 32, K] (the
+// step's rows) and W [N, K] streamed once.  Each CTA (4 warps) owns 64 output
+// features and one slice of K; each warp multiplies all 32 rows by its 16
+// features with mma.sync m16n8k16 (fp32 accumulation), over 128-wide K chunks
+// that cp.async double-buffers in shared memory (rows >= M and columns >= K
+// zero-filled).  Slices of K are summed by fp32 atomic adds into `out` (which
+// holds the residual stream, or zeros), so their order is not fixed; with a
+// single slice the CTA stores (optionally soft-capped) values instead.
+constexpr int SK_M = 32, SK_N = 64, SK_KC = 128, SK_LD = SK_KC + 8, SK_THREADS = 128;
+constexpr int SK_BUF = (SK_M + SK_N) * SK_LD;  // 16-bit elements per buffer
+
+template <bool F16, int MODE>  // MODE 0: atomic add, 1: store, 2: soft-capped store
+__global__ void __launch_bounds__(SK_THREADS) skinny_gemm_kernel(const uint16_t* __restrict__ A, int64_t lda,
+                                                                 const uint16_t* __restrict__ W, int64_t ldw,
+                                                                 float* __restrict__ out, int64_t ldo, int M, int N,
+                                                                 int K, int kslice, float cap) {
+  using namespace wmma16;
+  extern __shared__ __align__(16) uint16_t sk_smem[];
+  const int n0 = blockIdx.x * SK_N;
+  const int k_begin = blockIdx.y * kslice, k_end = min(K, k_begin + kslice);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nchunks = (k_end - k_begin + SK_KC - 1) / SK_KC;
+  auto issue = [&](int c) {
+    uint16_t* sa = sk_smem + (c & 1) * SK_BUF;
+    uint16_t* sw = sa + SK_M * SK_LD;
+    const int k0 = k_begin + c * SK_KC;
+    for (int i = threadIdx.x; i < (SK_M + SK_N) * (SK_KC / 8); i += SK_THREADS) {
+      const int r = i / (SK_KC / 8), ch = i % (SK_KC / 8);
+      const int k = k0 + ch * 8;
+      if (r < SK_M) {
+        const bool v = r < M && k < k_end;
+        cp_async16(sa + r * SK_LD + ch * 8, A + (int64_t)(v ? r : 0) * lda + (v ? k : 0), v);
+      } else {
+        const int n = n0 + r - SK_M;
+        const bool v = n < N && k < k_end;
+        cp_async16(sw + (r - SK_M) * SK_LD + ch * 8, W + (int64_t)(v ? n : 0) * ldw + (v ? k : 0), v);
+      }
+    }
+    cp_async_commit();
+  };
+  float acc[2][2][4];
+#pragma unroll
+  for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[mt][nt][e] = 0.0f;
+  if (nchunks > 0) issue(0);
+  for (int c = 0; c < nchunks; ++c) {
+    if (c + 1 < nchunks) {
+      issue(c + 1);
+      cp_async_wait<1>();
+    } else {
+      cp_async_wait<0>();
+    }
+    __syncthreads();
+    const uint32_t sa = smem_u32(sk_smem + (c & 1) * SK_BUF), sw = sa + SK_M * SK_LD * 2;
+#pragma unroll
+    for (int kk = 0; kk < SK_KC / 16; ++kk) {
+      uint32_t a0[4], a1[4], b[4];
+      load_a<SK_LD>(a0, sa, 0, kk * 16, lane);
+      load_a<SK_LD>(a1, sa, 16, kk * 16, lane);
+      load_b_nk<SK_LD>(b, sw, warp * 16, kk * 16, lane);
+      mma16816<F16>(acc[0][0], a0, b[0], b[1]);
+      mma16816<F16>(acc[0][1], a0, b[2], b[3]);
+      mma16816<F16>(acc[1][0], a1, b[0], b[1]);
+      mma16816<F16>(acc[1][1], a1, b[2], b[3]);
+    }
+    __syncthreads();  // buffer c & 1 is refilled by the issue of chunk c + 2
+  }
+  const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+  for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+      for (int hr = 0; hr < 2; ++hr) {
+        const int r = mt * 16 + g + 8 * hr;
+        const int col = n0 + warp * 16 + nt * 8 + 2 * t;
+        if (r >= M || col >= N) continue;
+        float* p = out + (int64_t)r * ldo + col;
+        const float v0 = acc[mt][nt][2 * hr], v1 = acc[mt][nt][2 * hr + 1];
+        if constexpr (MODE == 0) {
+          atomicAdd(p, v0);
+          if (col + 1 < N) atomicAdd(p + 1, v1);
+        } else {
+          const float o0 = MODE == 2 ? cap * tanhf(v0 / cap) : v0;
+          const float o1 = MODE == 2 ? cap * tanhf(v1 / cap) : v1;
+          p[0] = o0;
+          if (col + 1 < N) p[1] = o1;
+        }
+      }
+}
+
 }  // namespace
 
 int decode_attention_max_splits() { return kMaxSplits; }
@@ -375,6 +472,47 @@ nc_status qkv_finish_launch(const float* acc, uint16_t* qkv, uint16_t* cache, co
                                                                 eps);
   else
     return NC_ERR_SHAPE;
+  return cudaGetLastError() == cudaSuccess ? NC_OK : NC_ERR_CUDA;
+}
+
+nc_status skinny_gemm_launch(const uint16_t* a, int64_t lda, const uint16_t* w, int64_t ldw, float* out,
+                             int64_t ldo, int M, int N, int K, int mode, float cap, bool f16, cudaStream_t stream) {
+  if (M < 1 || M > SK_M || N < 1 || K < 8 || K % 8 || lda % 8 || ldw % 8) return NC_ERR_SHAPE;
+  const int ntiles = (N + SK_N - 1) / SK_N;
+  const int max_slices = (K + SK_KC - 1) / SK_KC;
+  int slices = 1;
+  if (mode == 0) {  // about four CTAs per SM
+    slices = (4 * device_sm_count() + ntiles - 1) / ntiles;
+    slices = slices < 1 ? 1 : (slices > max_slices ? max_slices : slices);
+  }
+  const int kslice = ((K + slices - 1) / slices + SK_KC - 1) / SK_KC * SK_KC;
+  slices = (K + kslice - 1) / kslice;
+  const dim3 grid(ntiles, slices);
+  const int smem = 2 * SK_BUF * 2;
+  static bool attr_done[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !attr_done[dev]) {
+    if (cudaFuncSetAttribute(skinny_gemm_kernel<true, 0>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) ||
+        cudaFuncSetAttribute(skinny_gemm_kernel<true, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) ||
+        cudaFuncSetAttribute(skinny_gemm_kernel<false, 0>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) ||
+        cudaFuncSetAttribute(skinny_gemm_kernel<false, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem))
+      return NC_ERR_CUDA;
+    attr_done[dev] = true;
+  }
+  if (mode == 0) {
+    if (f16)
+      skinny_gemm_kernel<true, 0><<<grid, SK_THREADS, smem, stream>>>(a, lda, w, ldw, out, ldo, M, N, K, kslice, cap);
+    else
+      skinny_gemm_kernel<false, 0><<<grid, SK_THREADS, smem, stream>>>(a, lda, w, ldw, out, ldo, M, N, K, kslice, cap);
+  } else if (mode == 2) {
+    if (f16)
+      skinny_gemm_kernel<true, 2><<<grid, SK_THREADS, smem, stream>>>(a, lda, w, ldw, out, ldo, M, N, K, kslice, cap);
+    else
+      skinny_gemm_kernel<false, 2><<<grid, SK_THREADS, smem, stream>>>(a, lda, w, ldw, out, ldo, M, N, K, kslice, cap);
+  } else {
+    return NC_ERR_INVALID_ARG;
+  }
   return cudaGetLastError() == cudaSuccess ? NC_OK : NC_ERR_CUDA;
 }
 

@@ -186,6 +186,11 @@ nc_status kv_append_launch(const uint16_t* qkv, int64_t ldq, int col0, int width
 nc_status decode_attention_launch(const uint16_t* q, int64_t ldq, const uint16_t* cache, float* partial,
                                   uint16_t* out, int B, int H, int Hkv, int D, int T_max, int pos, int W,
                                   bool f16, cudaStream_t stream);
+// Decode projections (M <= 32 rows): mode 0 adds A W^T into out (fp32 atomic
+// adds of K-slice partial sums; out holds the residual stream or zeros), mode 2
+// stores cap * tanh(A W^T / cap) (one slice).
+nc_status skinny_gemm_launch(const uint16_t* a, int64_t lda, const uint16_t* w, int64_t ldw, float* out,
+                             int64_t ldo, int M, int N, int K, int mode, float cap, bool f16, cudaStream_t stream);
 // Upper bound of the per-(b, h) splits decode_attention_launch uses.
 int decode_attention_max_splits();
 // From the fp32 split-K sum of a decode step's QKV projection: RoPE at `pos` and

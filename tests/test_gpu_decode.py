@@ -93,3 +93,17 @@ def test_decode_full_size_model(gpu, name, T0):
     want = oracle.forward(_oracle_cfg(s), w, x[1:2, :T0 + steps])["logits"][0, T0:]
     err = np.abs(dec[:, 1].cpu().numpy() - want).max()
     assert err <= 3e-2, f"{name} decode logits max-abs {err:.3e}"
+
+
+@pytest.mark.parametrize("B", [32, 40])
+def test_decode_batch_sizes_around_the_skinny_limit(gpu, B):
+    """Up to 32 rows the decode projections run on the skinny mma.sync GEMM,
+    beyond on the tcgen05 GEMM with split K: both against the oracle."""
+    s = SHAPES["tiny"]
+    w, model = _model(gpu, s)
+    x, _ = make_tokens(s, seed=B, batch=B)
+    T0, steps = 70, 3
+    _, dec = _run(gpu, model, x, T0, steps, 96)
+    want = oracle.forward(_oracle_cfg(s), w, x[:, :T0 + steps])["logits"]
+    err = np.abs(dec.cpu().numpy() - np.transpose(want[:, T0:T0 + steps], (1, 0, 2))).max()
+    assert err <= 3e-2, f"B={B} decode logits max-abs {err:.3e}"
