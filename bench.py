@@ -489,8 +489,10 @@ def run_decode(args, s):
     sess.prefill(tx[:, :T0].contiguous())
     logits = torch.empty((B, s.vocab), dtype=torch.float32, device=dev)
     steps_tok = [tx[:, T0 + k].contiguous() for k in range(Wm + 2 * K)]
+    # the step captured once in a CUDA graph (position in device memory), or eager launches
+    step = (lambda tok: sess.decode_graph(tok)) if args.graph else (lambda tok: sess.decode(tok, logits=logits))
     for k in range(Wm):
-        sess.decode(steps_tok[k], logits=logits)
+        step(steps_tok[k])
     torch.cuda.synchronize()
     if sess.status() != 0:
         raise SystemExit(f"device status after warm-up: {sess.status()}")
@@ -507,7 +509,7 @@ def run_decode(args, s):
     with ClockSampler(local) as clocks:
         t0.record(stream)
         for k in range(K):
-            sess.decode(steps_tok[Wm + k], logits=logits)
+            step(steps_tok[Wm + k])
         t1.record(stream)
         torch.cuda.synchronize()
     barrier()
@@ -522,8 +524,8 @@ def run_decode(args, s):
     e0.record(stream)
     for k in range(K):
         dtok.copy_(hx[:, sess.pos], non_blocking=True)
-        sess.decode(dtok, logits=logits)
-        hlog.copy_(logits, non_blocking=True)
+        out = step(dtok)
+        hlog.copy_(out, non_blocking=True)
     e1.record(stream)
     torch.cuda.synchronize()
     barrier()
@@ -542,6 +544,7 @@ def run_decode(args, s):
             "unit": UNIT, "n_gpus": world, "steps": K, "warmup": Wm, "ms_per_step": ms, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": DTYPE_NOTE, "data": "synthetic",
             "config": {"workload": f"{s.name} decode", "global_batch": world * B, "prompt": T0,
+                       "launch": "one CUDA graph per step" if args.graph else "eager launches",
                        "positions": [pos0, pos0 + K - 1], "parallelism": f"dp{world}" if world > 1 else "none",
                        "l2": "weights (0.87 GB 16-bit) and KV cache larger than L2"},
             "roofline": {"kernel": "whole decode step (weights + cached K/V streamed once)", "bound": "hbm",
@@ -718,6 +721,8 @@ def main():
     ap.add_argument("--mode", default="forward", choices=["forward", "decode", "train"],
                     help="decode: KV-cache decode steps after a prefill of --prompt tokens")
     ap.add_argument("--prompt", type=int, default=1024, help="decode mode: prompt length")
+    ap.add_argument("--graph", action=argparse.BooleanOptionalAction, default=True,
+                    help="decode mode: replay one captured CUDA graph per step (--no-graph: eager launches)")
     ap.add_argument("--fp8", default="none", choices=["none", "block", "all"],
                     help="forward mode: dynamic tensorwise e4m3 for the block projections "
                          "('block') or for them and the LM head ('all')")

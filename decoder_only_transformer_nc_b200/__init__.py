@@ -149,6 +149,7 @@ def lib():
             "nc_prefill_workspace_bytes": (sz, [cfgp, i32, i32]),
             "nc_prefill": (i32, [cfgp, ctypes.POINTER(NcWeights), vp, i32, i32, vp, vp, sz, i32, vp, sz, vp]),
             "nc_decode_step": (i32, [cfgp, ctypes.POINTER(NcWeights), vp, i32, i32, vp, vp, sz, i32, vp]),
+            "nc_decode_step_dev": (i32, [cfgp, ctypes.POINTER(NcWeights), vp, i32, vp, vp, vp, sz, i32, vp]),
         }
         for name, (res, args) in sigs.items():
             fn = getattr(L, name)
@@ -332,6 +333,7 @@ class Session:
         self.model, self.B, self.T_max = model, B, T_max
         self.buffer = torch.empty(n, dtype=torch.uint8, device=device)
         self.pos = 0
+        self._graph = None
 
     def prefill(self, tokens, want_logits=False, stream=None):
         """Runs the prompt tokens [B, T]; returns the logits [B, T, V] if asked."""
@@ -358,6 +360,37 @@ class Session:
                                     _stream(stream)), "nc_decode_step")
         self.pos += 1
         return logits
+
+    def _step_dev(self, stream=None):
+        cfg = self.model.cfg
+        _check(lib().nc_decode_step_dev(ctypes.byref(cfg), ctypes.byref(self.model.weights), _ptr(self._g_tokens),
+                                        self.B, _ptr(self._g_pos), _ptr(self._g_logits), _ptr(self.buffer),
+                                        self.buffer.numel(), self.T_max, _stream(stream)), "nc_decode_step_dev")
+
+    def decode_graph(self, tokens):
+        """As ``decode``, through one CUDA graph of the step replayed for every
+        further position (the position lives in device memory,
+        nc_decode_step_dev).  tokens [B] int32 are copied into the graph's input;
+        the returned logits [B, V] are the graph's buffer, overwritten by the
+        next step.  The first call runs the step eagerly, then captures it."""
+        import torch
+        if self._graph is None:
+            cfg = self.model.cfg
+            dev = tokens.device
+            self._g_tokens = tokens.clone()
+            self._g_logits = torch.empty((self.B, cfg.vocab), dtype=torch.float32, device=dev)
+            self._g_pos = torch.full((4,), self.pos, dtype=torch.int32, device=dev)
+            self._step_dev()
+            torch.cuda.synchronize()
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                self._step_dev()
+            self._graph = g
+        else:
+            self._g_tokens.copy_(tokens)
+            self._graph.replay()
+        self.pos += 1
+        return self._g_logits
 
     def status(self):
         return get_status(self.buffer)

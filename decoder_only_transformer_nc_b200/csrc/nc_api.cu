@@ -934,11 +934,17 @@ static int resid_ksplit(int M, int N, int K) {
   return s < 1 ? 1 : (s > kb ? kb : s);
 }
 
-nc_status nc_decode_step(const nc_config* cfg, const nc_weights* w, const int32_t* tokens, int B, int pos,
-                         float* logits, void* session, size_t session_bytes, int T_max, void* stream) {
+}  // extern "C"
+
+// One decode step at host position `pos`, or at the position *pos_dev holds on
+// the device (then advanced by one at the end of the step).
+static nc_status decode_impl(const nc_config* cfg, const nc_weights* w, const int32_t* tokens, int B, int pos,
+                             int32_t* pos_dev, float* logits, void* session, size_t session_bytes, int T_max,
+                             void* stream) {
   if (!cfg || !w || !w->wte || !tokens || !logits || !session) return NC_ERR_INVALID_ARG;
   if (!config_ok(cfg) || cfg->extras != 0 || cfg->fp8 != 0) return NC_ERR_CONFIG;
-  if (T_max < 1 || T_max > cfg->seq_len || B < 1 || pos < 0 || pos >= T_max) return NC_ERR_SHAPE;
+  if (T_max < 1 || T_max > cfg->seq_len || B < 1 || (!pos_dev && (pos < 0 || pos >= T_max))) return NC_ERR_SHAPE;
+  if (pos_dev && (T_max > decode_attention_max_splits() * 64 || !aligned16(pos_dev))) return NC_ERR_SHAPE;
   const SessionLayout SL = session_layout(cfg, B, T_max);
   if (session_bytes < SL.total) return NC_ERR_WORKSPACE;
   if ((reinterpret_cast<uintptr_t>(session) & 255u) != 0) return NC_ERR_ALIGNMENT;
@@ -997,9 +1003,9 @@ nc_status nc_decode_step(const nc_config* cfg, const nc_weights* w, const int32_
     uint16_t* cl = cache + l * SL.cache_layer_elems;
     if (cudaMemsetAsync(acc, 0, (size_t)B * NQKV * 4, st) != cudaSuccess) return NC_ERR_CUDA;
     NC_TRY(proj(a, C, wqkv + l * SL.wqkv_elems, NQKV, acc, ks_qkv));
-    NC_TRY(qkv_finish_launch(acc, qkv, cl, rope, T_max, pos, B, H, Hkv, D, T_max, eps, f16, st));
+    NC_TRY(qkv_finish_launch(acc, qkv, cl, rope, T_max, pos, B, H, Hkv, D, T_max, eps, f16, st, pos_dev));
     NC_TRY(decode_attention_launch(qkv, NQKV, cl, part, o, B, H, Hkv, D, T_max, pos, nc_layer_window(cfg, l),
-                                   f16, st));
+                                   f16, st, pos_dev));
     // the residual adds: partial products over K land in x (atomic or TMA
     // reduce-add, in no fixed order)
     NC_TRY(proj(o, H * D, wo + l * SL.wo_elems, C, x, resid_ksplit(B, C, H * D)));
@@ -1019,8 +1025,23 @@ nc_status nc_decode_step(const nc_config* cfg, const nc_weights* w, const int32_
     ep.cap = cfg->softcap;
     NC_TRY(gemm_launch(a, C, wlm, C, B, V, C, EPI_SOFTCAP_F32, f16, ep, status, st));
   }
+  if (pos_dev) NC_TRY(pos_advance_launch(pos_dev, st));
 #undef NC_TRY
   return NC_OK;
+}
+
+extern "C" {
+
+nc_status nc_decode_step(const nc_config* cfg, const nc_weights* w, const int32_t* tokens, int B, int pos,
+                         float* logits, void* session, size_t session_bytes, int T_max, void* stream) {
+  return decode_impl(cfg, w, tokens, B, pos, nullptr, logits, session, session_bytes, T_max, stream);
+}
+
+nc_status nc_decode_step_dev(const nc_config* cfg, const nc_weights* w, const int32_t* tokens, int B,
+                             int32_t* pos_dev, float* logits, void* session, size_t session_bytes, int T_max,
+                             void* stream) {
+  if (!pos_dev) return NC_ERR_INVALID_ARG;
+  return decode_impl(cfg, w, tokens, B, 0, pos_dev, logits, session, session_bytes, T_max, stream);
 }
 
 }  // extern "C"

@@ -62,12 +62,18 @@ __global__ void __launch_bounds__(kWarps * 32) decode_attn_kernel(const uint16_t
                                                                   const uint16_t* __restrict__ cache,
                                                                   float* __restrict__ partial, int H, int Hkv,
                                                                   int T_max, int lo, int hi, int chunk,
-                                                                  float scale_log2) {
+                                                                  float scale_log2, const int* __restrict__ pos_dev,
+                                                                  int W) {
   constexpr int D = DW * 32;
   const int s = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (pos_dev) {  // position from device memory (a graph replays the step): clamp to the cache
+    hi = min(max(*pos_dev, 0), T_max - 1);
+    lo = max(hi - W + 1, 0);
+  }
   const int k_begin = lo + s * chunk;
   const int n = min(k_begin + chunk, hi + 1) - k_begin;  // keys of this CTA (<= kChunk)
+  if (n <= 0) return;  // a split past the context (fixed-size grid only)
 
   extern __shared__ __align__(16) uint16_t kv_s[];  // [n][2][D]: k then v of each key
   {
@@ -203,9 +209,13 @@ __global__ void __launch_bounds__(kWarps * 32) decode_attn_kernel(const uint16_t
 // One block per (row, head); thread d merges dimension d over the splits.
 template <bool F16>
 __global__ void decode_combine_kernel(const float* __restrict__ partial, uint16_t* __restrict__ out, int H, int D,
-                                      int splits) {
+                                      int splits, const int* __restrict__ pos_dev, int T_max, int W, int chunk) {
   const int bh = blockIdx.x;
   const int d = threadIdx.x;
+  if (pos_dev) {  // the same split count the attention kernel used
+    const int hi = min(max(*pos_dev, 0), T_max - 1), lo = max(hi - W + 1, 0);
+    splits = (hi - lo + 1 + chunk - 1) / chunk;
+  }
   const float* p = partial + (int64_t)bh * kMaxSplits * (2 + D);
   // every split's (m, l, o[d]) read up front: independent loads, one round trip
   float ms[kMaxSplits], ls[kMaxSplits], os[kMaxSplits];
@@ -249,8 +259,9 @@ template <int DW, bool F16>
 __global__ void __launch_bounds__(256) qkv_finish_kernel(const float* __restrict__ acc, uint16_t* __restrict__ qkv,
                                                          uint16_t* __restrict__ cache, const float* __restrict__ rope,
                                                          int rope_T, int pos, int B, int H, int Hkv, int T_max,
-                                                         float eps) {
+                                                         float eps, const int* __restrict__ pos_dev) {
   constexpr int D = DW * 32;
+  if (pos_dev) pos = min(max(*pos_dev, 0), T_max - 1);
   const int heads = H + 2 * Hkv;
   const int wid = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
@@ -310,7 +321,7 @@ __global__ void relu2_finish_kernel(const float4* __restrict__ acc, uint2* __res
 template <int DW, bool F16>
 nc_status decode_dispatch(const uint16_t* q, int64_t ldq, const uint16_t* cache, float* partial, int B, int H,
                           int Hkv, int T_max, int lo, int hi, int splits, int chunk, float scale_log2,
-                          cudaStream_t stream) {
+                          cudaStream_t stream, const int* pos_dev, int W) {
   const dim3 grid(splits, Hkv, B);
   constexpr int D = DW * 32;
   // staging of the chunk's K/V rows, reused for the warps' merge
@@ -324,7 +335,7 @@ nc_status decode_dispatch(const uint16_t* q, int64_t ldq, const uint16_t* cache,
                                (int)smem) != cudaSuccess)
         return NC_ERR_CUDA;
       decode_attn_kernel<DW, 1, F16><<<grid, kWarps * 32, smem, stream>>>(q, ldq, cache, partial, H, Hkv, T_max, lo,
-                                                                       hi, chunk, scale_log2);
+                                                                       hi, chunk, scale_log2, pos_dev, W);
       break;
     case 2:
       if (smem > 48 * 1024 &&
@@ -332,7 +343,7 @@ nc_status decode_dispatch(const uint16_t* q, int64_t ldq, const uint16_t* cache,
                                (int)smem) != cudaSuccess)
         return NC_ERR_CUDA;
       decode_attn_kernel<DW, 2, F16><<<grid, kWarps * 32, smem, stream>>>(q, ldq, cache, partial, H, Hkv, T_max, lo,
-                                                                       hi, chunk, scale_log2);
+                                                                       hi, chunk, scale_log2, pos_dev, W);
       break;
     case 4:
       if (smem > 48 * 1024 &&
@@ -340,7 +351,7 @@ nc_status decode_dispatch(const uint16_t* q, int64_t ldq, const uint16_t* cache,
                                (int)smem) != cudaSuccess)
         return NC_ERR_CUDA;
       decode_attn_kernel<DW, 4, F16><<<grid, kWarps * 32, smem, stream>>>(q, ldq, cache, partial, H, Hkv, T_max, lo,
-                                                                       hi, chunk, scale_log2);
+                                                                       hi, chunk, scale_log2, pos_dev, W);
       break;
     case 8:
       if (smem > 48 * 1024 &&
@@ -348,7 +359,7 @@ nc_status decode_dispatch(const uint16_t* q, int64_t ldq, const uint16_t* cache,
                                (int)smem) != cudaSuccess)
         return NC_ERR_CUDA;
       decode_attn_kernel<DW, 8, F16><<<grid, kWarps * 32, smem, stream>>>(q, ldq, cache, partial, H, Hkv, T_max, lo,
-                                                                       hi, chunk, scale_log2);
+                                                                       hi, chunk, scale_log2, pos_dev, W);
       break;
     default:
       return NC_ERR_SHAPE;
@@ -458,20 +469,32 @@ int decode_attention_max_splits() { return kMaxSplits; }
 
 nc_status qkv_finish_launch(const float* acc, uint16_t* qkv, uint16_t* cache, const float* rope, int rope_T,
                             int pos, int B, int H, int Hkv, int D, int T_max, float eps, bool f16,
-                            cudaStream_t stream) {
+                            cudaStream_t stream, const int* pos_dev) {
   const int warps = B * (H + 2 * Hkv);
   if (warps == 0) return NC_OK;
   const unsigned grid = (unsigned)((warps + 7) / 8);
   if (D == 128)
-    f16 ? qkv_finish_kernel<4, true><<<grid, 256, 0, stream>>>(acc, qkv, cache, rope, rope_T, pos, B, H, Hkv, T_max, eps)
+    f16 ? qkv_finish_kernel<4, true><<<grid, 256, 0, stream>>>(acc, qkv, cache, rope, rope_T, pos, B, H, Hkv, T_max, eps,
+                                                               pos_dev)
         : qkv_finish_kernel<4, false><<<grid, 256, 0, stream>>>(acc, qkv, cache, rope, rope_T, pos, B, H, Hkv, T_max,
-                                                                eps);
+                                                                eps, pos_dev);
   else if (D == 64)
-    f16 ? qkv_finish_kernel<2, true><<<grid, 256, 0, stream>>>(acc, qkv, cache, rope, rope_T, pos, B, H, Hkv, T_max, eps)
+    f16 ? qkv_finish_kernel<2, true><<<grid, 256, 0, stream>>>(acc, qkv, cache, rope, rope_T, pos, B, H, Hkv, T_max, eps,
+                                                               pos_dev)
         : qkv_finish_kernel<2, false><<<grid, 256, 0, stream>>>(acc, qkv, cache, rope, rope_T, pos, B, H, Hkv, T_max,
-                                                                eps);
+                                                                eps, pos_dev);
   else
     return NC_ERR_SHAPE;
+  return cudaGetLastError() == cudaSuccess ? NC_OK : NC_ERR_CUDA;
+}
+
+// *pos += 1: the end of a decode step whose position lives in device memory.
+__global__ void pos_advance_kernel(int* pos) {
+  if (threadIdx.x == 0) *pos += 1;
+}
+
+nc_status pos_advance_launch(int* pos, cudaStream_t stream) {
+  pos_advance_kernel<<<1, 32, 0, stream>>>(pos);
   return cudaGetLastError() == cudaSuccess ? NC_OK : NC_ERR_CUDA;
 }
 
@@ -543,34 +566,42 @@ nc_status kv_append_launch(const uint16_t* qkv, int64_t ldq, int col0, int width
 
 nc_status decode_attention_launch(const uint16_t* q, int64_t ldq, const uint16_t* cache, float* partial,
                                   uint16_t* out, int B, int H, int Hkv, int D, int T_max, int pos, int W, bool f16,
-                                  cudaStream_t stream) {
+                                  cudaStream_t stream, const int* pos_dev) {
   if (B == 0) return NC_OK;
   if ((D != 64 && D != 128) || H % Hkv != 0) return NC_ERR_SHAPE;
-  const int lo = pos - W + 1 > 0 ? pos - W + 1 : 0;
-  const int n_keys = pos - lo + 1;
+  const int Wc = W <= 0 || W > T_max ? T_max : W;
+  int lo = pos - W + 1 > 0 ? pos - W + 1 : 0;
+  int n_keys = pos - lo + 1;
   // chunks of 64 keys (32 KB of K/V staging at D = 128), more when the window
   // needs more than kMaxSplits of them
   int chunk = (n_keys + kMaxSplits - 1) / kMaxSplits;
   chunk = chunk < 64 ? 64 : (chunk + 15) / 16 * 16;
-  const int splits = (n_keys + chunk - 1) / chunk;
+  int splits = (n_keys + chunk - 1) / chunk;
+  if (pos_dev) {  // position known on the device only: the fixed grid of kMaxSplits chunks of 64
+    if (T_max > kMaxSplits * 64) return NC_ERR_SHAPE;
+    chunk = 64;
+    splits = kMaxSplits;
+    lo = 0;
+    pos = 0;
+  }
   if ((size_t)chunk * 2 * D * 2 > 200 * 1024) return NC_ERR_SHAPE;  // T_max beyond the staging
   const float scale_log2 = 1.4426950408889634f / sqrtf((float)D);
   nc_status s;
   if (D == 128)
     s = f16 ? decode_dispatch<4, true>(q, ldq, cache, partial, B, H, Hkv, T_max, lo, pos, splits, chunk, scale_log2,
-                                       stream)
+                                       stream, pos_dev, Wc)
             : decode_dispatch<4, false>(q, ldq, cache, partial, B, H, Hkv, T_max, lo, pos, splits, chunk,
-                                        scale_log2, stream);
+                                        scale_log2, stream, pos_dev, Wc);
   else
     s = f16 ? decode_dispatch<2, true>(q, ldq, cache, partial, B, H, Hkv, T_max, lo, pos, splits, chunk, scale_log2,
-                                       stream)
+                                       stream, pos_dev, Wc)
             : decode_dispatch<2, false>(q, ldq, cache, partial, B, H, Hkv, T_max, lo, pos, splits, chunk,
-                                        scale_log2, stream);
+                                        scale_log2, stream, pos_dev, Wc);
   if (s != NC_OK) return s;
   if (f16)
-    decode_combine_kernel<true><<<B * H, D, 0, stream>>>(partial, out, H, D, splits);
+    decode_combine_kernel<true><<<B * H, D, 0, stream>>>(partial, out, H, D, splits, pos_dev, T_max, Wc, chunk);
   else
-    decode_combine_kernel<false><<<B * H, D, 0, stream>>>(partial, out, H, D, splits);
+    decode_combine_kernel<false><<<B * H, D, 0, stream>>>(partial, out, H, D, splits, pos_dev, T_max, Wc, chunk);
   return cudaGetLastError() == cudaSuccess ? NC_OK : NC_ERR_CUDA;
 }
 

@@ -185,12 +185,17 @@ nc_status kv_append_launch(const uint16_t* qkv, int64_t ldq, int col0, int width
 // -> out [B, H*D] (16-bit).  `partial` holds splits x (2 + D) fp32 per (b, h).
 nc_status decode_attention_launch(const uint16_t* q, int64_t ldq, const uint16_t* cache, float* partial,
                                   uint16_t* out, int B, int H, int Hkv, int D, int T_max, int pos, int W,
-                                  bool f16, cudaStream_t stream);
+                                  bool f16, cudaStream_t stream,
+                                  const int* pos_dev = nullptr);
 // Decode projections (M <= 32 rows): mode 0 adds A W^T into out (fp32 atomic
 // adds of K-slice partial sums; out holds the residual stream or zeros), mode 2
 // stores cap * tanh(A W^T / cap) (one slice).
 nc_status skinny_gemm_launch(const uint16_t* a, int64_t lda, const uint16_t* w, int64_t ldw, float* out,
                              int64_t ldo, int M, int N, int K, int mode, float cap, bool f16, cudaStream_t stream);
+// With pos_dev, the kernels of a decode step read the position from device
+// memory (clamped to the cache) and the attention runs on a fixed grid, so a
+// captured graph of the step can be replayed; pos_advance_launch adds one to it.
+nc_status pos_advance_launch(int* pos, cudaStream_t stream);
 // Upper bound of the per-(b, h) splits decode_attention_launch uses.
 int decode_attention_max_splits();
 // From the fp32 split-K sum of a decode step's QKV projection: RoPE at `pos` and
@@ -198,7 +203,7 @@ int decode_attention_max_splits();
 // into the layer's cache at `pos`.
 nc_status qkv_finish_launch(const float* acc, uint16_t* qkv, uint16_t* cache, const float* rope, int rope_T,
                             int pos, int B, int H, int Hkv, int D, int T_max, float eps, bool f16,
-                            cudaStream_t stream);
+                            cudaStream_t stream, const int* pos_dev = nullptr);
 // out = relu(acc)^2 as 16-bit (n elements, n % 4 == 0).
 nc_status relu2_finish_launch(const float* acc, uint16_t* out, int64_t n, bool f16, cudaStream_t stream);
 
