@@ -944,7 +944,8 @@ static nc_status decode_impl(const nc_config* cfg, const nc_weights* w, const in
   if (!cfg || !w || !w->wte || !tokens || !logits || !session) return NC_ERR_INVALID_ARG;
   if (!config_ok(cfg) || cfg->extras != 0 || cfg->fp8 != 0) return NC_ERR_CONFIG;
   if (T_max < 1 || T_max > cfg->seq_len || B < 1 || (!pos_dev && (pos < 0 || pos >= T_max))) return NC_ERR_SHAPE;
-  if (pos_dev && (T_max > decode_attention_max_splits() * 64 || !aligned16(pos_dev))) return NC_ERR_SHAPE;
+  if (pos_dev && T_max > decode_attention_max_splits() * 64) return NC_ERR_SHAPE;
+  if (pos_dev && !aligned16(pos_dev)) return NC_ERR_ALIGNMENT;
   const SessionLayout SL = session_layout(cfg, B, T_max);
   if (session_bytes < SL.total) return NC_ERR_WORKSPACE;
   if ((reinterpret_cast<uintptr_t>(session) & 255u) != 0) return NC_ERR_ALIGNMENT;

@@ -256,7 +256,8 @@ nc_status nc_decode_step(const nc_config* cfg, const nc_weights* w, const int32_
  * advanced by one at the end of the step, so the whole step can be captured
  * once in a CUDA graph and replayed for every further position.  The
  * attention then runs on a fixed grid of 32 chunks of 64 keys, which needs
- * T_max <= 2048 (NC_ERR_SHAPE otherwise).  The other rules are nc_decode_step's. */
+ * T_max <= 2048 (NC_ERR_SHAPE otherwise); pos_dev misaligned: NC_ERR_ALIGNMENT.
+ * The other rules are nc_decode_step's. */
 nc_status nc_decode_step_dev(const nc_config* cfg, const nc_weights* w, const int32_t* tokens, int B,
                              int32_t* pos_dev, float* logits, void* session, size_t session_bytes, int T_max,
                              void* stream);

@@ -320,3 +320,37 @@ def test_backward_host_rules(nclib):
     if not torch.cuda.is_available():
         assert fb(cfg) == 8
         assert L.nc_linear_dgrad(A, A, A, 128, 64, 64, 3, 1, None, None) == 8
+
+
+def test_device_position_and_attention_backward_host_rules(nclib):
+    """Host-side refusals of nc_decode_step_dev, nc_attention_lse and
+    nc_attention_backward (before any device work)."""
+    L = nclib.lib()
+    cfg = nclib.init_config(2, 64, 64, 0, 4096, 512)
+    fw = _FakeWeights(nclib, 2)
+    n = L.nc_session_bytes(ctypes.byref(cfg), 2, 4096)
+    dev = lambda pos_dev, T_max=4096, nbytes=n: L.nc_decode_step_dev(
+        ctypes.byref(cfg), ctypes.byref(fw.w), 1 << 41, 2, pos_dev, 1 << 44, 1 << 43, nbytes, T_max, None)
+    assert dev(None) == 1                       # no device position
+    assert dev(1 << 42) == 3                    # the fixed attention grid covers T_max <= 2048
+    assert dev((1 << 42) + 4, T_max=2048, nbytes=L.nc_session_bytes(ctypes.byref(cfg), 2, 2048)) == 4  # alignment
+    c = nclib.NcConfig.from_buffer_copy(cfg)
+    c.fp8 = nclib.FP8_BLOCK
+    assert L.nc_decode_step_dev(ctypes.byref(c), ctypes.byref(fw.w), 1 << 41, 2, 1 << 42, 1 << 44, 1 << 43, n,
+                                4096, None) == 2
+    A = 1 << 40
+    lse = lambda **kw: L.nc_attention_lse(kw.get("q", A), A, A, A, kw.get("lse", A), 1, 16, kw.get("H", 4),
+                                          kw.get("Hkv", 2), kw.get("D", 128), 0, kw.get("qs", 512), 256, 1, None)
+    assert lse(lse=None) == 1
+    assert lse(H=3) == 1                         # H % Hkv
+    assert lse(D=96) == 3
+    assert lse(qs=100) == 1                      # row stride below H * D
+    bwd = lambda **kw: L.nc_attention_backward(kw.get("qkv", A), A, A, A, kw.get("delta", A), A, 1, 16, 4, 2,
+                                               kw.get("D", 128), 0, kw.get("dt", 1), None)
+    assert bwd(delta=None) == 1
+    assert bwd(D=80) == 3
+    assert bwd(dt=5) == 1
+    assert bwd(qkv=A + 8) == 4
+    import torch
+    if not torch.cuda.is_available():
+        assert lse() == 8 and bwd() == 8
