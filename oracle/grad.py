@@ -94,7 +94,7 @@ def _forward(cfg: OracleConfig, weights: dict, idx: np.ndarray, targets: np.ndar
     idx = np.asarray(idx)
     targets = np.asarray(targets)
     B, T = idx.shape
-    C, H, Hkv, D = cfg.d_model, cfg.n_head, cfg.n_kv_head, cfg.head_dim
+    H, Hkv, D = cfg.n_head, cfg.n_kv_head, cfg.head_dim
     G = H // Hkv
     eps, cap = cfg.norm_eps, cfg.softcap
     windows = layer_windows(cfg)
@@ -160,9 +160,7 @@ def forward_backward(cfg: OracleConfig, weights: dict, idx: np.ndarray, targets:
     af, rf, cos, sin, idx, targets = c["af"], c["rf"], c["cos"], c["sin"], c["idx"], c["targets"]
     B, T = idx.shape
     C, H, Hkv, D = cfg.d_model, cfg.n_head, cfg.n_kv_head, cfg.head_dim
-    G = H // Hkv
     cap = cfg.softcap
-    scale = 1.0 / np.sqrt(D)
 
     # ---------------- backward
     grads = {"layers": [dict() for _ in Wb]}
