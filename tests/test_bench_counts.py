@@ -1,0 +1,26 @@
+"""The bench's kernel-launch claims (`gpu_launches`) against the launch lists
+ncu recorded for the same workloads (summaries under profiles/): one d20
+forward is 147 kernels, 231 with every product in e4m3."""
+import bench
+
+
+def test_forward_kernel_counts_match_the_launch_lists():
+    L = 20
+    # trace entries of one forward with targets and loss (nc_forward_traced)
+    plain = 3 + 7 * L + 1 + 3
+    assert bench.kernels_per_step(plain, L, 0, 0) == 147
+    fp8_all = plain + 4 * L + 1  # four activation quantisations per layer, one before the LM head
+    assert bench.kernels_per_step(fp8_all, L, 3, 0) == 231
+    fp8_block = plain + 4 * L
+    # block only: 120 e4m3 weights (two amax + quantise batches) and the 16-bit lm_head cast
+    assert bench.kernels_per_step(fp8_block, L, 1, 0) == fp8_block + 4
+
+
+def test_unfused_activation_quantisations_add_an_amax_launch():
+    L = 4
+    base = 3 + 7 * L + 1 + 3 + 4 * L + 1
+    fused = bench.kernels_per_step(base, L, 3, 0)
+    assert bench.kernels_per_step(base, L, 3, 4) == fused + L      # x0 mixing in every first norm
+    assert bench.kernels_per_step(base, L, 3, 8) == fused + 2      # backout: one first norm + the final norm
+    assert bench.kernels_per_step(base, L, 1, 8) == bench.kernels_per_step(base, L, 1, 0) + 1
+
