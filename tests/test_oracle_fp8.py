@@ -206,3 +206,24 @@ def test_forward_fp8_close_to_the_plain_forward():
     d = np.abs(p["logits"] - f["logits"]).max()
     assert 1e-3 < d < 0.5
     assert abs(p["loss"] - f["loss"]) < 0.05 * p["loss"]
+
+
+def test_forward_fp8_with_neutral_extras_is_the_plain_fp8_forward():
+    # residual lambdas 1, x0 lambdas 0, value-embedding gates 0, backout 0:
+    # every extra term adds exact zeros, so the e4m3 decisions are the same
+    c = _cfg(n_layer=3)
+    w = _weights(c)
+    rng = np.random.default_rng(12)
+    idx = rng.integers(0, c.vocab, (2, c.seq_len))
+    L, kvw = c.n_layer, c.n_kv_head * c.head_dim
+    ex = {"resid_lambdas": np.ones(L, np.float32), "x0_lambdas": np.zeros(L, np.float32),
+          "value_embeds": [rng.standard_normal((c.vocab, kvw)).astype(np.float32) for _ in range(L)],
+          "ve_gates": [np.zeros(c.n_kv_head, np.float32) for _ in range(L)],
+          "backout_lambda": np.float32(0.0)}
+    for mode in ("block", "all"):
+        a = oracle.forward(c, w, idx, fp8=mode)["logits"]
+        b = oracle.forward(c, w, idx, fp8=mode, extras=ex)["logits"]
+        assert np.array_equal(a, b), mode
+    ex["backout_lambda"] = np.float32(0.25)
+    assert not np.array_equal(oracle.forward(c, w, idx, fp8="all", extras=ex)["logits"],
+                              oracle.forward(c, w, idx, fp8="all")["logits"])
