@@ -122,3 +122,44 @@ def test_gradient_average_matches_the_whole_batch(tmp_path):
         for l, lw in enumerate(want["layers"]):
             for k, v in lw.items():
                 np.testing.assert_allclose(grads["layers"][l][k].numpy(), v, rtol=1e-4, atol=1e-9)
+
+
+def test_grad_bucket_layout():
+    """Every view 16-byte aligned (the library's rule for gradient pointers),
+    shaped like its weight, disjoint, and the whole bucket zeroed."""
+    from decoder_only_transformer_nc_b200 import dp
+    from workloads import SHAPES, make_weights
+
+    s = SHAPES["tiny"]
+    w = make_weights(s)
+    t = {"wte": torch.from_numpy(w["wte"]), "lm_head": torch.from_numpy(w["lm_head"]),
+         "layers": [{k: torch.from_numpy(v) for k, v in lw.items()} for lw in w["layers"]]}
+    flat, grads = dp.grad_bucket(t, device="cpu")
+    views = [("wte", grads["wte"], t["wte"]), ("lm_head", grads["lm_head"], t["lm_head"])]
+    views += [(f"{l}.{k}", grads["layers"][l][k], t["layers"][l][k]) for l in range(s.n_layer) for k in dp.NAMES]
+    spans = []
+    for name, g, ref in views:
+        assert g.shape == ref.shape and g.dtype == torch.float32, name
+        assert g.data_ptr() % 16 == 0, name
+        off = (g.data_ptr() - flat.data_ptr()) // 4
+        spans.append((off, off + g.numel()))
+    spans.sort()
+    assert all(a[1] <= b[0] for a, b in zip(spans, spans[1:]))
+    assert spans[-1][1] <= flat.numel() - 4 and not flat.any()
+
+
+def test_average_with_no_counted_targets_anywhere(tmp_path):
+    """A world whose ranks count no targets keeps zero gradients (no division by zero)."""
+    world, port = 1, _free_port()
+    import torch.distributed as dist
+    from decoder_only_transformer_nc_b200 import dp
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=0, world_size=world)
+    try:
+        flat = torch.zeros(16 + 4)
+        flat[:16] = 3.0
+        dp.average_grads_(flat, 0)
+        assert torch.isfinite(flat).all() and not flat[:16].any()
+    finally:
+        dist.destroy_process_group()
