@@ -30,11 +30,11 @@ LIB_PATH = os.path.join(_HERE, "libnc.so")
 
 EPI_STORE_16, EPI_RELU2_16, EPI_RESID_F32, EPI_STORE_F32, EPI_SOFTCAP_F32 = range(5)
 BF16, F16, F32 = 0, 1, 2  # nc_dtype (F32: fp8_quantize sources only)
-DEV_TOKEN_RANGE, DEV_TARGET_RANGE, DEV_TIMEOUT = 0x1, 0x2, 0x4
+DEV_TOKEN_RANGE, DEV_TARGET_RANGE, DEV_TIMEOUT, DEV_SMEM_ALIGN, DEV_POSITION = 0x1, 0x2, 0x4, 0x8, 0x10
 
 STATUS_NAMES = {0: "NC_OK", 1: "NC_ERR_INVALID_ARG", 2: "NC_ERR_CONFIG", 3: "NC_ERR_SHAPE",
                 4: "NC_ERR_ALIGNMENT", 5: "NC_ERR_WORKSPACE", 6: "NC_ERR_TOKEN_RANGE",
-                7: "NC_ERR_TIMEOUT", 8: "NC_ERR_UNSUPPORTED_DEVICE", 9: "NC_ERR_CUDA"}
+                7: "NC_ERR_TIMEOUT", 8: "NC_ERR_UNSUPPORTED_DEVICE", 9: "NC_ERR_CUDA", 10: "NC_ERR_F16_RANGE"}
 
 
 class NcError(RuntimeError):
@@ -372,8 +372,11 @@ class Session:
         further position (the position lives in device memory,
         nc_decode_step_dev).  tokens [B] int32 are copied into the graph's input;
         the returned logits [B, V] are the graph's buffer, overwritten by the
-        next step.  The first call runs the step eagerly, then captures it."""
+        next step.  The first call runs the step eagerly, then captures it.
+        Raises NcError(NC_ERR_SHAPE) once every cache position is used."""
         import torch
+        if self.pos >= self.T_max:
+            raise NcError(3, f"Session.decode_graph: position {self.pos} is past the cache (T_max {self.T_max})")
         if self._graph is None:
             cfg = self.model.cfg
             dev = tokens.device

@@ -260,6 +260,7 @@ const char* nc_status_string(nc_status s) {
     case NC_ERR_TIMEOUT: return "bounded device wait ran out";
     case NC_ERR_UNSUPPORTED_DEVICE: return "device is not sm_100";
     case NC_ERR_CUDA: return "CUDA runtime error";
+    case NC_ERR_F16_RANGE: return "an fp16 activation saturated at +-65504";
   }
   return "unknown status";
 }
@@ -334,6 +335,8 @@ nc_status nc_get_status(const void* dev_status, void* stream) {
     return NC_ERR_CUDA;
   if (st & NC_DEV_TIMEOUT) return NC_ERR_TIMEOUT;
   if (st & NC_DEV_SMEM_ALIGN) return NC_ERR_CUDA;
+  if (st & NC_DEV_POSITION) return NC_ERR_SHAPE;
+  if (st & NC_DEV_F16_RANGE) return NC_ERR_F16_RANGE;
   if (st & (NC_DEV_TOKEN_RANGE | NC_DEV_TARGET_RANGE)) return NC_ERR_TOKEN_RANGE;
   return NC_OK;
 }
@@ -1004,7 +1007,7 @@ static nc_status decode_impl(const nc_config* cfg, const nc_weights* w, const in
     uint16_t* cl = cache + l * SL.cache_layer_elems;
     if (cudaMemsetAsync(acc, 0, (size_t)B * NQKV * 4, st) != cudaSuccess) return NC_ERR_CUDA;
     NC_TRY(proj(a, C, wqkv + l * SL.wqkv_elems, NQKV, acc, ks_qkv));
-    NC_TRY(qkv_finish_launch(acc, qkv, cl, rope, T_max, pos, B, H, Hkv, D, T_max, eps, f16, st, pos_dev));
+    NC_TRY(qkv_finish_launch(acc, qkv, cl, rope, T_max, pos, B, H, Hkv, D, T_max, eps, f16, st, pos_dev, status));
     NC_TRY(decode_attention_launch(qkv, NQKV, cl, part, o, B, H, Hkv, D, T_max, pos, nc_layer_window(cfg, l),
                                    f16, st, pos_dev));
     // the residual adds: partial products over K land in x (atomic or TMA
@@ -1013,7 +1016,7 @@ static nc_status decode_impl(const nc_config* cfg, const nc_weights* w, const in
     NC_TRY(rmsnorm_launch(x, a, B, C, eps, f16, st));
     if (cudaMemsetAsync(acc, 0, (size_t)B * 4 * C * 4, st) != cudaSuccess) return NC_ERR_CUDA;
     NC_TRY(proj(a, C, wfc + l * SL.wfc_elems, 4 * C, acc, ks_fc));
-    NC_TRY(relu2_finish_launch(acc, h, (int64_t)B * 4 * C, f16, st));
+    NC_TRY(relu2_finish_launch(acc, h, (int64_t)B * 4 * C, f16, st, status));
     NC_TRY(proj(h, 4 * C, wmp + l * SL.wmp_elems, C, x, resid_ksplit(B, C, 4 * C)));
   }
   NC_TRY(rmsnorm_launch(x, a, B, C, eps, f16, st));

@@ -259,9 +259,16 @@ template <int DW, bool F16>
 __global__ void __launch_bounds__(256) qkv_finish_kernel(const float* __restrict__ acc, uint16_t* __restrict__ qkv,
                                                          uint16_t* __restrict__ cache, const float* __restrict__ rope,
                                                          int rope_T, int pos, int B, int H, int Hkv, int T_max,
-                                                         float eps, const int* __restrict__ pos_dev) {
+                                                         float eps, const int* __restrict__ pos_dev,
+                                                         uint32_t* __restrict__ dev_status) {
   constexpr int D = DW * 32;
-  if (pos_dev) pos = min(max(*pos_dev, 0), T_max - 1);
+  bool store_cache = true;
+  if (pos_dev) {  // a replayed graph step: refuse a position past the cache
+    const int p = *pos_dev;
+    store_cache = p >= 0 && p < T_max;
+    if (!store_cache && blockIdx.x == 0 && threadIdx.x == 0 && dev_status) atomicOr(dev_status, NC_DEV_POSITION);
+    pos = min(max(p, 0), T_max - 1);
+  }
   const int heads = H + 2 * Hkv;
   const int wid = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
@@ -290,10 +297,15 @@ __global__ void __launch_bounds__(256) qkv_finish_kernel(const float* __restrict
     for (int d = 0; d < DW; ++d) v[d] *= r;
   }
   uint32_t pk[DW / 2];
+  float vmax = 0.0f;
 #pragma unroll
-  for (int p = 0; p < DW / 2; ++p) pk[p] = Half<F16>::pack2(v[2 * p], v[2 * p + 1]);
+  for (int p = 0; p < DW / 2; ++p) {
+    pk[p] = Half<F16>::pack2(v[2 * p], v[2 * p + 1]);
+    vmax = fmaxf(vmax, fmaxf(fabsf(v[2 * p]), fabsf(v[2 * p + 1])));
+  }
+  if (F16 && dev_status && vmax > 65504.0f) atomicOr(dev_status, NC_DEV_F16_RANGE);
   uint16_t* dst = qkv + ((int64_t)b * heads + hd) * D + lane * DW;
-  uint16_t* cdst = hd >= H ? cache + ((int64_t)b * T_max + pos) * 2 * Hkv * D + (int64_t)(hd - H) * D + lane * DW
+  uint16_t* cdst = (hd >= H && store_cache) ? cache + ((int64_t)b * T_max + pos) * 2 * Hkv * D + (int64_t)(hd - H) * D + lane * DW
                            : nullptr;
   if constexpr (DW == 4) {
     const uint2 w2 = make_uint2(pk[0], pk[1]);
@@ -307,7 +319,8 @@ __global__ void __launch_bounds__(256) qkv_finish_kernel(const float* __restrict
 
 // relu(acc)^2 -> 16-bit ("从文本到聊天模型" §5.7), for the split-K c_fc of a decode step.
 template <bool F16>
-__global__ void relu2_finish_kernel(const float4* __restrict__ acc, uint2* __restrict__ out, int64_t n4) {
+__global__ void relu2_finish_kernel(const float4* __restrict__ acc, uint2* __restrict__ out, int64_t n4,
+                                    uint32_t* __restrict__ dev_status) {
   const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= n4) return;
   float4 a = acc[i];
@@ -315,7 +328,12 @@ __global__ void relu2_finish_kernel(const float4* __restrict__ acc, uint2* __res
   a.y = fmaxf(a.y, 0.f);
   a.z = fmaxf(a.z, 0.f);
   a.w = fmaxf(a.w, 0.f);
-  out[i] = make_uint2(Half<F16>::pack2(a.x * a.x, a.y * a.y), Half<F16>::pack2(a.z * a.z, a.w * a.w));
+  a.x *= a.x;
+  a.y *= a.y;
+  a.z *= a.z;
+  a.w *= a.w;
+  if (F16 && dev_status && fmaxf(fmaxf(a.x, a.y), fmaxf(a.z, a.w)) > 65504.0f) atomicOr(dev_status, NC_DEV_F16_RANGE);
+  out[i] = make_uint2(Half<F16>::pack2(a.x, a.y), Half<F16>::pack2(a.z, a.w));
 }
 
 template <int DW, bool F16>
@@ -469,20 +487,20 @@ int decode_attention_max_splits() { return kMaxSplits; }
 
 nc_status qkv_finish_launch(const float* acc, uint16_t* qkv, uint16_t* cache, const float* rope, int rope_T,
                             int pos, int B, int H, int Hkv, int D, int T_max, float eps, bool f16,
-                            cudaStream_t stream, const int* pos_dev) {
+                            cudaStream_t stream, const int* pos_dev, uint32_t* dev_status) {
   const int warps = B * (H + 2 * Hkv);
   if (warps == 0) return NC_OK;
   const unsigned grid = (unsigned)((warps + 7) / 8);
   if (D == 128)
     f16 ? qkv_finish_kernel<4, true><<<grid, 256, 0, stream>>>(acc, qkv, cache, rope, rope_T, pos, B, H, Hkv, T_max, eps,
-                                                               pos_dev)
+                                                               pos_dev, dev_status)
         : qkv_finish_kernel<4, false><<<grid, 256, 0, stream>>>(acc, qkv, cache, rope, rope_T, pos, B, H, Hkv, T_max,
-                                                                eps, pos_dev);
+                                                                eps, pos_dev, dev_status);
   else if (D == 64)
     f16 ? qkv_finish_kernel<2, true><<<grid, 256, 0, stream>>>(acc, qkv, cache, rope, rope_T, pos, B, H, Hkv, T_max, eps,
-                                                               pos_dev)
+                                                               pos_dev, dev_status)
         : qkv_finish_kernel<2, false><<<grid, 256, 0, stream>>>(acc, qkv, cache, rope, rope_T, pos, B, H, Hkv, T_max,
-                                                                eps, pos_dev);
+                                                                eps, pos_dev, dev_status);
   else
     return NC_ERR_SHAPE;
   return cudaGetLastError() == cudaSuccess ? NC_OK : NC_ERR_CUDA;
@@ -539,17 +557,18 @@ nc_status skinny_gemm_launch(const uint16_t* a, int64_t lda, const uint16_t* w, 
   return cudaGetLastError() == cudaSuccess ? NC_OK : NC_ERR_CUDA;
 }
 
-nc_status relu2_finish_launch(const float* acc, uint16_t* out, int64_t n, bool f16, cudaStream_t stream) {
+nc_status relu2_finish_launch(const float* acc, uint16_t* out, int64_t n, bool f16, cudaStream_t stream,
+                              uint32_t* dev_status) {
   if (n == 0) return NC_OK;
   if (n % 4) return NC_ERR_SHAPE;
   const int64_t n4 = n / 4;
   const unsigned grid = (unsigned)((n4 + 255) / 256);
   if (f16)
     relu2_finish_kernel<true><<<grid, 256, 0, stream>>>(reinterpret_cast<const float4*>(acc),
-                                                        reinterpret_cast<uint2*>(out), n4);
+                                                        reinterpret_cast<uint2*>(out), n4, dev_status);
   else
     relu2_finish_kernel<false><<<grid, 256, 0, stream>>>(reinterpret_cast<const float4*>(acc),
-                                                         reinterpret_cast<uint2*>(out), n4);
+                                                         reinterpret_cast<uint2*>(out), n4, dev_status);
   return cudaGetLastError() == cudaSuccess ? NC_OK : NC_ERR_CUDA;
 }
 

@@ -15,7 +15,9 @@
 //   warps 2..9  epilogue: tcgen05.ld of the accumulator (a warp may only read
 //               the 32 TMEM lanes = tile rows its warp index mod 4 selects, so
 //               two warps share each lane quarter and split the 256 columns),
-//               fused epilogue op, direct global stores; then hand the
+//               fused epilogue op; results are staged per warp in a 4 KB
+//               swizzled shared-memory tile and written by a TMA tensor store
+//               (a TMA reduce-add for the fp32 residual); then hand the
 //               accumulator back.
 // e4m3 operands (dynamic tensorwise FP8, "Nanochat与nanoGPT对比" §1 table, FP8
 // row): the same pipeline with tcgen05.mma kind::f8f6f4.  A 128-byte swizzle
@@ -259,8 +261,8 @@ __device__ __forceinline__ void epilogue_16_half(uint32_t taddr, const CUtensorM
           b = fmaxf(b, 0.0f);
           a *= a;
           b *= b;
-          if constexpr (SC) *om = max(*om, max(__float_as_uint(a), __float_as_uint(b)));  // a, b >= 0
         }
+        if (om) *om = max(*om, max(__float_as_uint(a) & 0x7FFFFFFFu, __float_as_uint(b) & 0x7FFFFFFFu));
         w[16 * h + i] = Half<F16>::pack2(a, b);
       }
     if (c + 1 < EPI_COLS / 64 && col0 + 64 < N) {
@@ -365,11 +367,12 @@ __device__ __forceinline__ void epilogue_16_rowdep(uint32_t taddr, const CUtenso
 template <bool F16, int HD, bool SC>
 __device__ __forceinline__ void epilogue_qkv_head(uint32_t taddr, const CUtensorMap* tmC, uint8_t* stg,
                                                   int row, int col0, int row0, int M,
-                                                  const EpiParams& ep, uint32_t lane, const Dq& dqs) {
+                                                  const EpiParams& ep, uint32_t lane, const Dq& dqs,
+                                                  uint32_t* om) {
   constexpr int G = HD / 64;  // 32-pair groups per head (1 or 2)
   const int head = col0 / HD;
   if (head >= ep.H + ep.Hkv) {  // v head (warp-uniform): plain 16-bit store
-    epilogue_16_half<EPI_STORE_16, F16, SC>(taddr, tmC, stg, col0, row0, col0 + HD, lane, dqs.v);
+    epilogue_16_half<EPI_STORE_16, F16, SC>(taddr, tmC, stg, col0, row0, col0 + HD, lane, dqs.v, om);
     return;
   }
   const float dq = head < ep.H ? dqs.q : dqs.k;
@@ -441,7 +444,7 @@ __device__ __forceinline__ void epilogue_qkv_head(uint32_t taddr, const CUtensor
 template <bool F16, int HD, bool SC>
 __device__ __forceinline__ void epilogue_v_embed(uint32_t taddr, const CUtensorMap* tmC, uint8_t* stg,
                                                  int row, int col0, int row0, int M, const EpiParams& ep,
-                                                 uint32_t lane, float dq) {
+                                                 uint32_t lane, float dq, uint32_t* om) {
   const int g = col0 / HD - ep.H - ep.Hkv;  // kv head
   int tok = row < M ? ep.tokens[row] : 0;
   if (tok < 0 || tok >= ep.V) tok = 0;  // flagged by the embedding kernel
@@ -463,10 +466,12 @@ __device__ __forceinline__ void epilogue_v_embed(uint32_t taddr, const CUtensorM
       const float4 e = __ldg(ve + c * 16 + j);
       const uint32_t* src = j < 8 ? r0 : r1;
       const int k = (j & 7) * 4;
-      w[2 * j] = Half<F16>::pack2(fmaf(gate, e.x, __uint_as_float(src[k])),
-                                  fmaf(gate, e.y, __uint_as_float(src[k + 1])));
-      w[2 * j + 1] = Half<F16>::pack2(fmaf(gate, e.z, __uint_as_float(src[k + 2])),
-                                      fmaf(gate, e.w, __uint_as_float(src[k + 3])));
+      const float v0 = fmaf(gate, e.x, __uint_as_float(src[k])), v1 = fmaf(gate, e.y, __uint_as_float(src[k + 1]));
+      const float v2 = fmaf(gate, e.z, __uint_as_float(src[k + 2])), v3 = fmaf(gate, e.w, __uint_as_float(src[k + 3]));
+      *om = max(*om, max(max(__float_as_uint(v0) & 0x7FFFFFFFu, __float_as_uint(v1) & 0x7FFFFFFFu),
+                         max(__float_as_uint(v2) & 0x7FFFFFFFu, __float_as_uint(v3) & 0x7FFFFFFFu)));
+      w[2 * j] = Half<F16>::pack2(v0, v1);
+      w[2 * j + 1] = Half<F16>::pack2(v2, v3);
     }
     if (c > 0) flush_wait(lane);
     stage_row(stg, (int)lane, w);
@@ -478,13 +483,14 @@ __device__ __forceinline__ void epilogue_v_embed(uint32_t taddr, const CUtensorM
 template <bool F16, int HD, bool SC>
 __device__ __forceinline__ void epilogue_qkv_head_il(uint32_t taddr, const CUtensorMap* tmC,
                                                      uint8_t* stg, int row, int col0, int row0, int M,
-                                                     const EpiParams& ep, uint32_t lane, const Dq& dqs) {
+                                                     const EpiParams& ep, uint32_t lane, const Dq& dqs,
+                                                     uint32_t* om) {
   const int head = col0 / HD;
   if (head >= ep.H + ep.Hkv) {  // v head (warp-uniform)
     if (ep.ve)
-      epilogue_v_embed<F16, HD, SC>(taddr, tmC, stg, row, col0, row0, M, ep, lane, dqs.v);
+      epilogue_v_embed<F16, HD, SC>(taddr, tmC, stg, row, col0, row0, M, ep, lane, dqs.v, om);
     else  // plain 16-bit store
-      epilogue_16_half<EPI_STORE_16, F16, SC>(taddr, tmC, stg, col0, row0, col0 + HD, lane, dqs.v);
+      epilogue_16_half<EPI_STORE_16, F16, SC>(taddr, tmC, stg, col0, row0, col0 + HD, lane, dqs.v, om);
     return;
   }
   const float dq = head < ep.H ? dqs.q : dqs.k;
@@ -707,7 +713,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const int row_in_tile = quarter * 32 + lane;
     uint8_t* stg = staging + (warp - 2) * STG_BYTES;  // this warp's staging tile
     Dq dqs{1.0f, 1.0f, 1.0f};
-    uint32_t om = 0;  // relu^2 with e4m3 operands: max output (bits) for ep.amax_out
+    // max |16-bit output| (bits): the fp16 range check, and with e4m3 operands
+    // the relu^2 output's amax for ep.amax_out
+    uint32_t om = 0;
     if constexpr (FP8) {  // 1 / (s_a s_w) from the tensors' amax values
       const float sa = e4m3_scale(__ldg(ep.amax_a));
       dqs.q = 1.0f / (sa * e4m3_scale(__ldg(ep.amax_b)));
@@ -753,9 +761,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           const int col0 = n0 + hh * HD;
           if (col0 >= N) break;  // warp-uniform
           if constexpr (EPI == EPI_QKV_ROPE)
-            epilogue_qkv_head<F16, HD, FP8>(taddr + hh * HD, &tmC, stg, row, col0, row0, M, ep, lane, dqs);
+            epilogue_qkv_head<F16, HD, FP8>(taddr + hh * HD, &tmC, stg, row, col0, row0, M, ep, lane, dqs, &om);
           else
-            epilogue_qkv_head_il<F16, HD, FP8>(taddr + hh * HD, &tmC, stg, row, col0, row0, M, ep, lane, dqs);
+            epilogue_qkv_head_il<F16, HD, FP8>(taddr + hh * HD, &tmC, stg, row, col0, row0, M, ep, lane, dqs,
+                                               &om);
         }
       } else if constexpr (EPI == EPI_STORE_16 || EPI == EPI_RELU2_16) {
         epilogue_16_half<EPI, F16, FP8>(taddr, &tmC, stg, n0, row0, N, lane, dqs.q, &om);
@@ -790,11 +799,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         acc_phase ^= 1u;
       }
     }
-    if constexpr (FP8 && EPI == EPI_RELU2_16) {
-      if (ep.amax_out) {
-        om = __reduce_max_sync(0xFFFFFFFFu, om);
-        if (lane == 0) fold_amax(ep.amax_out, stored_abs_bits<F16>(om));
-      }
+    if constexpr (EPI == EPI_STORE_16 || EPI == EPI_RELU2_16 || EPI == EPI_QKV_ROPE || EPI == EPI_QKV_ROPE_IL) {
+      om = __reduce_max_sync(0xFFFFFFFFu, om);
+      // fp16 saturates above 65504 (0x477FE000 as fp32 bits): flag it
+      if constexpr (F16)
+        if (lane == 0 && om > 0x477FE000u && dev_status) atomicOr(dev_status, NC_DEV_F16_RANGE);
+      if constexpr (FP8 && EPI == EPI_RELU2_16)
+        if (ep.amax_out && lane == 0) fold_amax(ep.amax_out, stored_abs_bits<F16>(om));
     }
     if (lane == 0) bulk_wait0();  // every TMA store / reduce of this warp has landed
     __syncwarp();

@@ -193,19 +193,23 @@ nc_status decode_attention_launch(const uint16_t* q, int64_t ldq, const uint16_t
 nc_status skinny_gemm_launch(const uint16_t* a, int64_t lda, const uint16_t* w, int64_t ldw, float* out,
                              int64_t ldo, int M, int N, int K, int mode, float cap, bool f16, cudaStream_t stream);
 // With pos_dev, the kernels of a decode step read the position from device
-// memory (clamped to the cache) and the attention runs on a fixed grid, so a
+// memory (clamped to the cache for their reads; the cache write refuses a
+// position past it) and the attention runs on a fixed grid, so a
 // captured graph of the step can be replayed; pos_advance_launch adds one to it.
 nc_status pos_advance_launch(int* pos, cudaStream_t stream);
 // Upper bound of the per-(b, h) splits decode_attention_launch uses.
 int decode_attention_max_splits();
 // From the fp32 split-K sum of a decode step's QKV projection: RoPE at `pos` and
 // QK-norm of q and k heads (pair-interleaved columns), 16-bit qkv, and k|v heads
-// into the layer's cache at `pos`.
+// into the layer's cache at `pos`.  A device position outside [0, T_max) writes
+// no cache entry and sets NC_DEV_POSITION in dev_status.
 nc_status qkv_finish_launch(const float* acc, uint16_t* qkv, uint16_t* cache, const float* rope, int rope_T,
                             int pos, int B, int H, int Hkv, int D, int T_max, float eps, bool f16,
-                            cudaStream_t stream, const int* pos_dev = nullptr);
-// out = relu(acc)^2 as 16-bit (n elements, n % 4 == 0).
-nc_status relu2_finish_launch(const float* acc, uint16_t* out, int64_t n, bool f16, cudaStream_t stream);
+                            cudaStream_t stream, const int* pos_dev = nullptr, uint32_t* dev_status = nullptr);
+// out = relu(acc)^2 as 16-bit (n elements, n % 4 == 0); an fp16 value past
+// 65504 sets NC_DEV_F16_RANGE in dev_status.
+nc_status relu2_finish_launch(const float* acc, uint16_t* out, int64_t n, bool f16, cudaStream_t stream,
+                              uint32_t* dev_status = nullptr);
 
 nc_status rmsnorm_launch(const float* x, uint16_t* out, int M, int C, float eps, bool f16,
                          cudaStream_t stream,

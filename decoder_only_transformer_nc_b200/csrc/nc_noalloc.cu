@@ -13,7 +13,9 @@
 // pass the array's name to a kernel -- on the host that name is only a
 // stand-in symbol, not a device address -- so the device address is looked
 // up with cudaGetSymbolAddress once per device (with that device current) and
-// cached.
+// cached.  The cached address belongs to the device's primary context: after
+// cudaDeviceReset destroys that context the address is stale, so a process
+// that resets a device must not call this entry point on it again.
 #include <cuda_runtime.h>
 
 #include <cstdint>

@@ -62,6 +62,20 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Non-blocking test of the phase with the given parity (never suspends the
+// thread, so a caller can poll several barriers in turn).
+__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 // Shared abort state of one CTA: once any role gives up, every other role's
 // waits return false at their next check, so the whole CTA winds down.
 struct WaitCtl {
@@ -87,6 +101,25 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const W
       }
     }
   }
+}
+
+// One step of a bounded polling loop over several barriers (each tested with
+// mbar_test_wait).  Returns false once another role of the CTA has aborted or
+// `limit_ns` has passed since the loop's first step, recording NC_DEV_TIMEOUT
+// in the latter case.
+__device__ __forceinline__ bool poll_step(uint32_t& spins, uint64_t& t0, const WaitCtl& ctl) {
+  if (spins++ == 0u) {
+    t0 = global_timer_ns();
+    return true;
+  }
+  if ((spins & 255u) != 0u) return true;
+  if (*ctl.abort_flag) return false;
+  if (global_timer_ns() - t0 > ctl.limit_ns) {
+    *ctl.abort_flag = 1;
+    if (ctl.dev_status) atomicOr(ctl.dev_status, NC_DEV_TIMEOUT);
+    return false;
+  }
+  return true;
 }
 
 // ---------------------------------------------------------------- TMA

@@ -56,7 +56,9 @@ typedef enum {
   NC_ERR_TOKEN_RANGE = 6,        /* device: token or target id out of range  */
   NC_ERR_TIMEOUT = 7,            /* device: a bounded wait in a kernel ran out */
   NC_ERR_UNSUPPORTED_DEVICE = 8, /* current device is not sm_100             */
-  NC_ERR_CUDA = 9                /* a CUDA runtime call failed               */
+  NC_ERR_CUDA = 9,               /* a CUDA runtime call failed               */
+  NC_ERR_F16_RANGE = 10          /* device: a value stored as fp16 exceeded
+                                    +-65504 and was saturated               */
 } nc_status;
 
 /* 16-bit storage formats. */
@@ -72,6 +74,13 @@ typedef enum {
 #define NC_DEV_TIMEOUT 0x4u      /* a pipeline wait gave up; outputs invalid   */
 #define NC_DEV_SMEM_ALIGN 0x8u   /* a kernel's shared-memory window was not 1024-byte
                                     aligned; it did nothing (reported as NC_ERR_CUDA) */
+#define NC_DEV_F16_RANGE 0x20u   /* a projection output stored in fp16 (act_dtype
+                                    NC_F16) exceeded +-65504 and was saturated to it
+                                    (reported as NC_ERR_F16_RANGE) */
+#define NC_DEV_POSITION 0x10u    /* nc_decode_step_dev read a position outside
+                                    [0, T_max): nothing was written to the cache and
+                                    the step's logits are invalid (reported as
+                                    NC_ERR_SHAPE) */
 
 /* Further terms of the full nanochat forward ("Nanochat与nanoGPT对比" §1,
  * architecture table and notes); bits of nc_config.extras.  Each reads its
@@ -252,11 +261,15 @@ nc_status nc_decode_step(const nc_config* cfg, const nc_weights* w, const int32_
                          float* logits, void* session, size_t session_bytes, int T_max, void* stream);
 
 /* nc_decode_step with the position in device memory: *pos_dev (one int32,
- * 16-byte aligned) is read by the step's kernels -- clamped to [0, T_max) -- and
- * advanced by one at the end of the step, so the whole step can be captured
+ * 16-byte aligned) is read by the step's kernels and advanced by one at the
+ * end of the step, so the whole step can be captured
  * once in a CUDA graph and replayed for every further position.  The
  * attention then runs on a fixed grid of 32 chunks of 64 keys, which needs
  * T_max <= 2048 (NC_ERR_SHAPE otherwise); pos_dev misaligned: NC_ERR_ALIGNMENT.
+ * A position outside [0, T_max) (the cache is full) is caught on the device:
+ * the step writes nothing to the cache, its logits are invalid, and the
+ * session's status word gets NC_DEV_POSITION (nc_get_status on the session
+ * then returns NC_ERR_SHAPE).
  * The other rules are nc_decode_step's. */
 nc_status nc_decode_step_dev(const nc_config* cfg, const nc_weights* w, const int32_t* tokens, int B,
                              int32_t* pos_dev, float* logits, void* session, size_t session_bytes, int T_max,
@@ -524,7 +537,10 @@ nc_status nc_loss_mean(const float* token_loss, const int32_t* targets, int M, i
  * exits), so it allocates nothing and calls no allocating routine.  Limits:
  * M <= 8192 rows and V <= 32768 (NC_ERR_SHAPE beyond them).  The first call
  * on a device looks up the array's device address (cudaGetSymbolAddress, with
- * that device current); make that first call before any stream capture.  All
+ * that device current) and keeps it for the life of the process; make that
+ * first call before any stream capture, and do not call this entry point on a
+ * device after cudaDeviceReset (the kept address belonged to the destroyed
+ * context).  All
  * calls share the array and it keeps the previous call's contents (nothing in
  * it needs clearing), so calls whose work overlaps on the GPU race with each
  * other: order them on one stream. */

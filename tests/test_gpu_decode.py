@@ -140,3 +140,32 @@ def test_decode_graph_matches_eager(gpu, name, B):
     torch.cuda.empty_cache()
     want = oracle.forward(_oracle_cfg(s), w, x[rows, :T0 + steps])["logits"][:, T0:]
     assert np.abs(g[:, rows].cpu().numpy() - np.transpose(want, (1, 0, 2))).max() <= 3e-2
+
+
+def test_decode_graph_past_the_cache_is_refused(gpu):
+    """A full cache: the graph session refuses the next step on the host, and the
+    device-position step run past T_max reports NC_DEV_POSITION (NC_ERR_SHAPE
+    from the session's status) instead of overwriting the last cache slot."""
+    s = SHAPES["tiny"]
+    w, model = _model(gpu, s)
+    x, _ = make_tokens(s, seed=5, batch=2)
+    tx = torch.from_numpy(x).to(DEV)
+    T_max = 8
+    sess = gpu.Session(model, 2, T_max)
+    sess.prefill(tx[:, :T_max - 1].contiguous())
+    last = sess.decode_graph(tx[:, T_max - 1].contiguous()).clone()  # the last free position
+    torch.cuda.synchronize()
+    assert sess.status() == 0 and sess.pos == T_max
+    want = oracle.forward(_oracle_cfg(s), w, x[:, :T_max])["logits"][:, T_max - 1]
+    assert np.abs(last.cpu().numpy() - want).max() <= 3e-2
+    with pytest.raises(gpu.NcError):
+        sess.decode_graph(tx[:, T_max].contiguous())
+    assert sess.pos == T_max
+    sess._step_dev()  # the device position now reads T_max
+    torch.cuda.synchronize()
+    assert sess.status() == 3  # NC_ERR_SHAPE
+    # a later in-range step clears the per-step status
+    sess._g_pos.fill_(T_max - 1)
+    sess._step_dev()
+    torch.cuda.synchronize()
+    assert sess.status() == 0

@@ -233,6 +233,45 @@ def test_linear_parity(gpu, M, N, K, epi, dt):
         np.testing.assert_allclose(got, want, rtol=1e-5, atol=2e-6 * math.sqrt(K), err_msg=f"linear {epi}")
 
 
+@pytest.mark.parametrize("epi", ["store_16", "relu2_16"])
+def test_linear_f16_saturation_flagged(gpu, epi):
+    """fp16 activations saturate at +-65504: a ReLU^2 pre-activation above 256
+    (or a stored product above 65504) sets NC_DEV_F16_RANGE, reported as
+    NC_ERR_F16_RANGE; the same product just inside the range, and in bf16, does
+    not.  Host-made inputs, no fault."""
+    M, N, K = 300, 256, 64
+    code = gpu.EPI_STORE_16 if epi == "store_16" else gpu.EPI_RELU2_16
+    limit = 65504.0 if epi == "store_16" else 256.0  # largest pre-activation that fits
+    for scale, dt, flagged in ((1.05, "f16", True), (0.95, "f16", False), (1.05, "bf16", False)):
+        a = np.zeros((M, K), dtype=np.float32)
+        a[:, :2] = 1.0
+        w = np.zeros((N, K), dtype=np.float32)
+        w[7, :2] = limit * scale / 2  # column 7 of every row: a pre-activation of limit * scale
+        w[9, 0] = 1.0
+        st = status_word()
+        out = torch.empty((M, N), dtype=TDT[dt], device=DEV)
+        gpu.linear(dev16(a, dt), dev16(w, dt), out, code, status=st)
+        assert gpu.get_status(st) == (10 if flagged else 0), (epi, scale, dt)
+        if flagged:
+            assert host(out)[:, 7].max() == 65504.0  # saturated, not inf
+
+
+def test_forward_f16_saturation_flagged(gpu):
+    """The tiny forward with c_fc weights scaled so its pre-activations pass 256:
+    the fp16 forward reports NC_ERR_F16_RANGE, the bf16 forward does not."""
+    s = SHAPES["tiny"]
+    w = make_weights(s)
+    w = {**w, "layers": [dict(L) for L in w["layers"]]}
+    w["layers"][0]["c_fc"] = w["layers"][0]["c_fc"] * 4000.0
+    x, y = make_tokens(s)
+    for act, want in ((gpu.F16, 10), (gpu.BF16, 0)):
+        cfg = gpu.make_config(s.n_layer, s.d_model, s.n_head, s.n_kv_head, s.head_dim, s.seq_len, s.vocab,
+                              s.short_window, act_dtype=act)
+        model = gpu.Model.from_numpy(cfg, w)
+        res = gpu.forward(model, torch.from_numpy(x).to(DEV), torch.from_numpy(y).to(DEV))
+        assert gpu.get_status(res["workspace"]) == want
+
+
 @pytest.mark.parametrize("dt", DTYPES)
 @pytest.mark.parametrize("M,C,H,Hkv,D,T", [(2 * 300, 256, 2, 1, 64, 300), (1024, 768, 6, 6, 128, 512),
                                           (384, 512, 4, 2, 128, 128), (4096, 1280, 10, 10, 128, 2048)])
@@ -410,17 +449,21 @@ PREFIX = 640  # > the 512-key short window, so windowed rows are compared too
 @pytest.mark.parametrize("name", ["d12", "d20", "d26", "d26_gqa"])
 def test_forward_full_size_sampled_rows(gpu, name):
     """Full-size batch in the bench's launch configuration; the oracle recomputes
-    rows 0 and B-1 over their first PREFIX positions (causality makes those
-    outputs depend on nothing later)."""
+    the whole of row B-1 (all T positions: the full-context layers' attention
+    over every prefix length, the short-window layers at every window offset)
+    and row 0 over its first PREFIX positions (causality makes those outputs
+    depend on nothing later).  Bars: logits max-abs <= 3e-2, per-token and
+    mean loss relative <= 5e-3."""
     s = SHAPES[name]
     w, model = _model(gpu, name)
     x, y = make_tokens(s)
     tx, ty = torch.from_numpy(x).to(DEV), torch.from_numpy(y).to(DEV)
     res = gpu.forward(model, tx, ty, want_logits=True, want_token_loss=True)
     assert gpu.get_status(res["workspace"]) == 0
-    rows = [0, s.batch - 1]
-    got_logits = res["logits"][rows, :PREFIX].cpu().numpy()
-    got_tl = res["token_loss"][rows, :PREFIX].cpu().numpy()
+    full_row, pre_row = s.batch - 1, 0
+    got = {"full": (res["logits"][full_row].cpu().numpy(), res["token_loss"][full_row].cpu().numpy()),
+           "prefix": (res["logits"][pre_row, :PREFIX].cpu().numpy(),
+                      res["token_loss"][pre_row, :PREFIX].cpu().numpy())}
     # the timed configuration (no logits requested) gives bit-identical losses
     res_fast = gpu.forward(model, tx, ty, want_token_loss=True)
     torch.cuda.synchronize()
@@ -428,14 +471,17 @@ def test_forward_full_size_sampled_rows(gpu, name):
     assert res_fast["loss"].item() == res["loss"].item()
     tl_all = res["token_loss"].double()
     assert abs(tl_all.mean().item() - res["loss"].item()) <= 1e-5 * abs(res["loss"].item())
-    del res
-    want = oracle.forward(_oracle_cfg(s), w, x[rows, :PREFIX], y[rows, :PREFIX])
-    err = np.abs(got_logits - want["logits"]).max()
-    assert err <= 3e-2, f"{name} logits max-abs {err:.3e}"
-    rel_rows = np.abs(got_tl - want["token_loss"]) / np.abs(want["token_loss"])
-    assert rel_rows.max() <= 5e-3, f"{name} per-token loss rel {rel_rows.max():.3e}"
-    rel = abs(got_tl.mean() - want["loss"]) / abs(want["loss"])
-    assert rel <= 5e-3, f"{name} sampled loss rel {rel:.3e}"
+    del res, res_fast
+    inputs = {"full": (x[[full_row]], y[[full_row]]), "prefix": (x[[pre_row], :PREFIX], y[[pre_row], :PREFIX])}
+    for part, (xi, yi) in inputs.items():
+        want = oracle.forward(_oracle_cfg(s), w, xi, yi)
+        got_logits, got_tl = got[part]
+        err = np.abs(got_logits - want["logits"][0]).max()
+        assert err <= 3e-2, f"{name} {part} row logits max-abs {err:.3e}"
+        rel_rows = np.abs(got_tl - want["token_loss"][0]) / np.abs(want["token_loss"][0])
+        assert rel_rows.max() <= 5e-3, f"{name} {part} row per-token loss rel {rel_rows.max():.3e}"
+        rel = abs(got_tl.mean() - want["loss"]) / abs(want["loss"])
+        assert rel <= 5e-3, f"{name} {part} row loss rel {rel:.3e}"
 
 
 def test_forward_deterministic_and_causal(gpu):
