@@ -42,6 +42,8 @@ UNIT = "tokens/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 DTYPE_NOTE = ("f16 tensor-core operands (weights rounded fp32->bf16 as the method casts them, "
               "held exactly in f16; activations f16), fp32 accumulation, fp32 residual/softmax/loss")
+DTYPE_NOTE_BF16 = ("bf16 tensor-core operands (weights rounded fp32->bf16 as the method casts them; "
+                   "activations bf16, the pages' compute dtype), fp32 accumulation, fp32 residual/softmax/loss")
 DTYPE_NOTE_FP8 = ("e4m3 tensor-core operands with dynamic tensorwise scales for the {what} "
                   "(activations quantised from f16, weights from fp32), fp32 accumulation; other products "
                   "f16; fp32 residual/softmax/loss")
@@ -256,8 +258,9 @@ def run_ours(args, s):
 
     bits = nc.EXTRA_ALL if args.extras == "all" else 0
     fp8_bits = {"none": 0, "block": nc.FP8_BLOCK, "all": nc.FP8_ALL}[args.fp8]
+    act = nc.BF16 if args.act_dtype == "bf16" else nc.F16
     cfg = nc.make_config(s.n_layer, s.d_model, s.n_head, s.n_kv_head, s.head_dim, s.seq_len, s.vocab,
-                         s.short_window, extras=bits, fp8=fp8_bits)
+                         s.short_window, extras=bits, fp8=fp8_bits, act_dtype=act)
     weights = make_weights(s)
     extras = _extras_for(s, nc) if bits else None
     model = nc.Model.from_numpy(cfg, weights, device=dev, extras=extras)
@@ -391,10 +394,11 @@ def run_ours(args, s):
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None,
-            "dtype": DTYPE_NOTE if not fp8_bits else DTYPE_NOTE_FP8.format(
+            "dtype": (DTYPE_NOTE if act == nc.F16 else DTYPE_NOTE_BF16) if not fp8_bits else DTYPE_NOTE_FP8.format(
                 what="six block projections" + (" and the LM head" if fp8_bits & 2 else "")),
             "data": "synthetic",
-            "config": {"workload": s.name + ("+extras" if bits else "") + ({0: "", 1: "+fp8block", 3: "+fp8"}[fp8_bits]),
+            "config": {"workload": s.name + ("+extras" if bits else "") + ({0: "", 1: "+fp8block", 3: "+fp8"}[fp8_bits])
+                                   + ("+bf16act" if act == nc.BF16 else ""),
                        "global_batch": world * B, "seq_len": T,
                        "parallelism": f"dp{world}" if world > 1 else "none",
                        "layers": s.n_layer, "d_model": s.d_model,
@@ -729,6 +733,8 @@ def main():
     ap.add_argument("--prompt", type=int, default=1024, help="decode mode: prompt length")
     ap.add_argument("--graph", action=argparse.BooleanOptionalAction, default=True,
                     help="decode mode: replay one captured CUDA graph per step (--no-graph: eager launches)")
+    ap.add_argument("--act-dtype", default="f16", choices=["f16", "bf16"],
+                    help="forward mode: 16-bit activation format (bf16 = the pages' compute dtype)")
     ap.add_argument("--fp8", default="none", choices=["none", "block", "all"],
                     help="forward mode: dynamic tensorwise e4m3 for the block projections "
                          "('block') or for them and the LM head ('all')")
