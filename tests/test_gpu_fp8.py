@@ -204,6 +204,22 @@ def test_forward_fp8_full_width_two_layers(gpu, name, B, T):
     _check_forward(got, want, plain, f"{name} 2 layers fp8=all")
 
 
+@pytest.mark.parametrize("bits", ["block", "all"])
+def test_forward_fp8_d20_full_depth_whole_row(gpu, bits):
+    """d20 at full depth and width (20 layers, C = 1280, V = 32768) over one
+    whole 2048-token row: every short-window and full-context layer of the
+    bench's model, in e4m3, against the oracle's e4m3 forward of the same row.
+    One row, because the tensorwise scales tie every row to the whole batch
+    and the oracle must run the whole batch; the bars are those of the other
+    forward cases."""
+    f = SHAPES["d20"]
+    s = ModelShape("d20_row", n_layer=f.n_layer, d_model=f.d_model, n_head=f.n_head, n_kv_head=f.n_kv_head,
+                   head_dim=f.head_dim, vocab=f.vocab, seq_len=f.seq_len, batch=1, short_window=f.short_window)
+    x, y = make_tokens(s, seed=21)
+    got, want, plain = _forward_case(gpu, s, gpu.FP8_ALL if bits == "all" else gpu.FP8_BLOCK, x, y)
+    _check_forward(got, want, plain, f"d20 whole row fp8={bits}")
+
+
 @pytest.mark.parametrize("T", [128, 77])
 def test_forward_fp8_head_decisions_exact(gpu, T):
     """One layer whose attention and MLP output projections are zero and whose
