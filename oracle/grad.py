@@ -152,9 +152,19 @@ def _forward(cfg: OracleConfig, weights: dict, idx: np.ndarray, targets: np.ndar
                       sin=sin, idx=idx, targets=targets)
 
 
-def forward_backward(cfg: OracleConfig, weights: dict, idx: np.ndarray, targets: np.ndarray, cast=to_bf16):
+def _term_magnitude(dy, x):
+    """sum over tokens of |dy_m|^T |x_m|: the size of the terms whose sum is the
+    weight gradient dy^T x (a scale for comparing a rounded computation of it)."""
+    return np.abs(dy.reshape(-1, dy.shape[-1])).T @ np.abs(x.reshape(-1, x.shape[-1]))
+
+
+def forward_backward(cfg: OracleConfig, weights: dict, idx: np.ndarray, targets: np.ndarray, cast=to_bf16,
+                     magnitudes: bool = False):
     """Returns (loss, grads) with grads = {"wte", "lm_head", "layers": [{...}]},
-    each the same shape as its weight, float64."""
+    each the same shape as its weight, float64.  With magnitudes=True, returns
+    (loss, grads, mags): mags has the same structure and holds, per gradient
+    element, the sum of the absolute values of the per-token terms it adds up
+    (for wte, of the rows it gathers)."""
     loss, c = _forward(cfg, weights, idx, targets, cast)
     saved, Wb, Wlm, lg, lse, valid, n = c["saved"], c["Wb"], c["Wlm"], c["lg"], c["lse"], c["valid"], c["n"]
     af, rf, cos, sin, idx, targets = c["af"], c["rf"], c["cos"], c["sin"], c["idx"], c["targets"]
@@ -171,6 +181,9 @@ def forward_backward(cfg: OracleConfig, weights: dict, idx: np.ndarray, targets:
     dlg = np.where(valid[..., None], (p - onehot) / max(n, 1), 0.0)
     dz = dlg * (1.0 - (lg / cap) ** 2)  # d/dz cap tanh(z / cap)
     grads["lm_head"] = np.einsum("btv,btc->vc", dz, af)
+    mags = {"layers": [dict() for _ in Wb]}
+    if magnitudes:
+        mags["lm_head"] = _term_magnitude(dz, af)
     daf = dz @ Wlm
     dx = rmsnorm_backward(af, rf, daf)
     for l in range(len(Wb) - 1, -1, -1):
@@ -193,12 +206,25 @@ def forward_backward(cfg: OracleConfig, weights: dict, idx: np.ndarray, targets:
         gl["c_q"] = np.einsum("bte,btc->ec", duq, s["a"])
         gl["c_k"] = np.einsum("bte,btc->ec", duk, s["a"])
         gl["c_v"] = np.einsum("bte,btc->ec", dvf, s["a"])
+        if magnitudes:
+            ml = mags["layers"][l]
+            ml["mlp_proj"] = _term_magnitude(dx, s["h"])
+            ml["c_fc"] = _term_magnitude(du, s["a2"])
+            ml["attn_proj"] = _term_magnitude(dx_mid, s["of"])
+            ml["c_q"] = _term_magnitude(duq, s["a"])
+            ml["c_k"] = _term_magnitude(duk, s["a"])
+            ml["c_v"] = _term_magnitude(dvf, s["a"])
         da = duq @ lw["c_q"] + duk @ lw["c_k"] + dvf @ lw["c_v"]
         dx = dx_mid + rmsnorm_backward(s["a"], s["r1"], da)
     dwte = np.zeros(np.asarray(weights["wte"]).shape, dtype=F64)
     np.add.at(dwte, idx.reshape(-1), dx.reshape(-1, C))
     grads["wte"] = dwte
-    return loss, grads
+    if not magnitudes:
+        return loss, grads
+    mwte = np.zeros_like(dwte)
+    np.add.at(mwte, idx.reshape(-1), np.abs(dx.reshape(-1, C)))
+    mags["wte"] = mwte
+    return loss, grads, mags
 
 
 def loss_only(cfg: OracleConfig, weights: dict, idx, targets, cast=to_bf16) -> float:

@@ -170,3 +170,28 @@ def test_ignored_positions_get_no_gradient():
     for tok in later:  # tokens seen only after the counted position
         assert not g["wte"][tok].any()
     assert g["lm_head"].any()
+
+
+def test_term_magnitudes_bound_the_gradient_and_are_exact_for_one_term():
+    """The per-element term magnitudes (the scale the GPU gradients are compared
+    against): by the triangle inequality they bound |gradient| element by
+    element; with one token and one target every gradient element is a single
+    term, so they equal |gradient| (wte: a single gathered row); the gradient
+    values themselves do not change when magnitudes are asked for."""
+    c = _cfg()
+    w = _weights(c)
+    rng = np.random.default_rng(8)
+    idx = rng.integers(0, c.vocab, (2, c.seq_len))
+    tgt = rng.integers(0, c.vocab, (2, c.seq_len))
+    loss0, g0 = forward_backward(c, w, idx, tgt)
+    loss, g, m = forward_backward(c, w, idx, tgt, magnitudes=True)
+    assert loss == loss0
+    leaves = [("wte",), ("lm_head",)] + [(l, n) for l in range(c.n_layer) for n in NAMES]
+    for path in leaves:
+        assert np.array_equal(_get(g, path), _get(g0, path))
+        assert np.all(_get(m, path) >= np.abs(_get(g, path)) * (1 - 1e-12)), path
+    c1 = _cfg(seq_len=1)
+    _, g1, m1 = forward_backward(c1, w, idx[:1, :1], tgt[:1, :1], magnitudes=True)
+    for path in leaves:
+        np.testing.assert_allclose(_get(m1, path), np.abs(_get(g1, path)), rtol=1e-12, atol=1e-300,
+                                   err_msg=str(path))
