@@ -684,6 +684,9 @@ nc_status attention_launch(const uint16_t* q, const uint16_t* k, const uint16_t*
                            int B, int T, int H, int Hkv, int D, int window, int64_t q_stride,
                            int64_t kv_stride, bool f16, uint32_t* dev_status, cudaStream_t stream,
                            float* amax, float* lse) {
+  if (lse)  // the backward's log-sum-exp: the run-to-run reproducible kernel
+    return attention_lse_launch(q, k, v, out, B, T, H, Hkv, D, window, q_stride, kv_stride, f16, dev_status,
+                                stream, amax, lse);
   if (D != 64 && D != 128) return NC_ERR_SHAPE;
   if (B == 0 || T == 0) return NC_OK;
   const int W = (window <= 0 || window > T) ? T : window;

@@ -142,11 +142,17 @@ bool encode_tensor_map_u8(CUtensorMap* map, int rank, const void* base, const ui
 bool encode_tensor_map_f32(CUtensorMap* map, int rank, const void* base, const uint64_t* dims,
                            const uint64_t* strides, const uint32_t* box);
 
-// ---- attention (nc_attention.cu)
+// ---- attention (nc_attention.cu; with lse, nc_attention_lse.cu)
+// When `lse` is given ([B, T, H] fp32 row log-sum-exp, for the backward) the
+// launch goes to the kernel whose outputs are bit-reproducible run to run.
 nc_status attention_launch(const uint16_t* q, const uint16_t* k, const uint16_t* v, uint16_t* out,
                            int B, int T, int H, int Hkv, int D, int window, int64_t q_stride,
                            int64_t kv_stride, bool f16, uint32_t* dev_status, cudaStream_t stream,
                            float* amax = nullptr, float* lse = nullptr);
+nc_status attention_lse_launch(const uint16_t* q, const uint16_t* k, const uint16_t* v, uint16_t* out,
+                               int B, int T, int H, int Hkv, int D, int window, int64_t q_stride,
+                               int64_t kv_stride, bool f16, uint32_t* dev_status, cudaStream_t stream,
+                               float* amax, float* lse);
 
 // ---- elementwise / row kernels (nc_rowops.cu)
 struct CastSeg {

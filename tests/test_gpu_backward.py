@@ -166,8 +166,10 @@ def test_forward_backward_d20_width_full_context(gpu):
 def test_forward_backward_full_size_properties(gpu):
     """d20, B = 32, T = 2048: clean status, the forward's loss, finite
     gradients, run-to-run agreement and accumulation (a second call adds the
-    same gradients again), both up to the summation order of the atomics and
-    split-K partial sums (bar 1e-3 relative)."""
+    same gradients again), both up to the summation order of the embedding
+    atomics and the split-K partial sums of the weight gradients (bar 1e-5
+    relative): everything else, the attention's log-sum-exp included, is
+    bit-reproducible."""
     s = SHAPES["d20"]
     w = make_weights(s)
     x, y = make_tokens(s)
@@ -196,7 +198,7 @@ def test_forward_backward_full_size_properties(gpu):
         info.append((name, rel, rr))
     print("accumulated vs 2x first, fresh vs first:", info)
     # summation order only: atomics (embedding rows) and split-K partial sums
-    assert all(rel < 1e-3 and rr < 1e-3 for _, rel, rr in info), info
+    assert all(rel < 1e-5 and rr < 1e-5 for _, rel, rr in info), info
 
 
 @pytest.mark.parametrize("B,T,H,Hkv,D,W", [(2, 300, 4, 2, 128, 100), (1, 256, 2, 2, 64, 256), (1, 1, 2, 1, 128, 1),

@@ -200,6 +200,30 @@ def test_attention_sweep_parity(gpu, T, Hkv, full, dt):
     assert err <= 2e-2, f"attention sweep T={T} Hkv={Hkv} W={W}: max-abs {err:.3e}"
 
 
+@pytest.mark.parametrize("W", [1024, 0])
+def test_attention_lse_run_to_run_identical(gpu, W):
+    """The forward attention with its log-sum-exp output (the backward reads it),
+    twice on the same inputs with many work items per CTA (B=4, H=16, T=4096,
+    four query heads per kv head; a 1024-key window and full causal): output
+    and log-sum-exp are bit-identical -- no state crosses work items and every
+    sum runs in a fixed order."""
+    B, T, H, Hkv, D = 4, 4096, 16, 4, 128
+    g = torch.Generator().manual_seed(5)
+    qkv = torch.randn((B, T, H + 2 * Hkv, D), generator=g)
+    qk = qkv[:, :, :H + Hkv]
+    qkv[:, :, :H + Hkv] = qk / qk.pow(2).mean(-1, keepdim=True).sqrt()
+    qkv = qkv.to(torch.float16).reshape(B, T, -1).contiguous().to(DEV)
+    runs = []
+    for _ in range(2):
+        out = torch.full((B, T, H * D), float("nan"), dtype=torch.float16, device=DEV)
+        lse = torch.full((B, T, H), float("nan"), dtype=torch.float32, device=DEV)
+        gpu.attention_lse(qkv, out, lse, H, Hkv, D, W)
+        runs.append((out, lse))
+    torch.cuda.synchronize()
+    assert torch.isfinite(runs[0][1]).all() and not torch.isnan(runs[0][0]).any()
+    assert torch.equal(runs[0][0], runs[1][0]) and torch.equal(runs[0][1], runs[1][1])
+
+
 GEMM_SHAPES = [(128, 256, 64), (1, 256, 128), (300, 352, 200), (1000, 800, 520), (64, 32, 8),
                (2048, 3840, 1280), (520, 5120, 1280), (256, 1280, 5120)]
 
