@@ -50,10 +50,12 @@ DTYPE_NOTE_FP8 = ("e4m3 tensor-core operands with dynamic tensorwise scales for 
 GEMM_KINDS = ("gemm_qkv", "gemm_attn_proj", "gemm_fc", "gemm_mlp_proj", "gemm_lm_head")
 ROOFLINE_KIND = "gemm_fc"  # the kind with the largest share of the step
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one c_fc launch of
-# the d20 workload at B=32, T=2048, from a one-pass ncu capture of this kernel:
-# 181.33 MB read (A + W once) + 618.75 MB written (the rest of the 671 MB output
-# is still in L2 when the kernel ends).  Valid for that workload and kernel only.
-FC_TRAFFIC = {("d20", 32, 2048): 181.33e6 + 618.75e6}
+# the d20 workload at B=32, T=2048, from an ncu capture of the current kernel at
+# B=8 scaled to B=32 by the tokens processed: reads 55.09 MB = A (42.0 MB, x4)
+# + W (13.1 MB, once); writes 116.29 MB of the 167.8 MB output, the other
+# 51.5 MB still dirty in L2 when the kernel ends (671.1 - 51.5 MB at B=32).
+# Valid for that workload and kernel only.
+FC_TRAFFIC = {("d20", 32, 2048): (4 * 41.94e6 + 13.11e6) + (4 * 167.77e6 - 51.48e6)}
 
 
 def load_peaks():
@@ -417,13 +419,11 @@ def run_ours(args, s):
                                        f"2 x bf16_tflops_sustained ({peak_src}): e4m3 operands, nominal "
                                        "e4m3/bf16 dense ratio 4.5/2.25"),
                          "unit": "TFLOP/s", "frac": round(rk_achieved / peak, 4),
-                         # the counters predate the e4m3 / operand-layout template parameters of
-                         # gemm_kernel (compiled out of this instantiation, but the source changed)
-                         "traffic": None,
-                         "traffic_note": (None if fp8_bits or (s.name, B, T) not in FC_TRAFFIC else
-                                          "%.0f MB per launch in an ncu capture of this instantiation taken "
-                                          "before gemm_kernel gained its e4m3 and operand-layout template "
-                                          "parameters" % (FC_TRAFFIC[(s.name, B, T)] / 1e6)),
+                         "traffic": (None if fp8_bits or act == nc.BF16 or (s.name, B, T) not in FC_TRAFFIC
+                                     else round(FC_TRAFFIC[(s.name, B, T)])),
+                         "traffic_note": (None if fp8_bits or act == nc.BF16 or (s.name, B, T) not in FC_TRAFFIC
+                                          else "DRAM bytes of one launch: ncu capture of this kernel at B=8, "
+                                               "scaled to B=32 by the tokens processed"),
                          "algorithmic_bytes": (1 if fp8_bits else 2) * (B * T * s.d_model
                                                                          + 4 * s.d_model * s.d_model)
                                               + 2 * 4 * B * T * s.d_model,
