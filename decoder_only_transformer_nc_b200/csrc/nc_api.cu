@@ -126,7 +126,7 @@ WsLayout ws_layout(const nc_config* c, int B, int T, bool own_weights = true) {
   const size_t wb = (c->fp8 & NC_FP8_BLOCK) ? 1 : 2;    // bytes per block weight element
   const size_t lb = (c->fp8 & NC_FP8_LM_HEAD) ? 1 : 2;  // ... per LM-head element
   if (own_weights) {  // else the 16-bit weights and the RoPE table live in a session
-    L.rope = take((size_t)T * D * sizeof(float));
+    L.rope = take((size_t)T * D * sizeof(float) * 2);  // [2][T][D/2] and the pair-major copy
     L.wqkv = take(c->n_layer * L.wqkv_elems * wb);
     L.wo = take(c->n_layer * L.wo_elems * wb);
     L.wfc = take(c->n_layer * L.wfc_elems * wb);
@@ -178,7 +178,7 @@ SessionLayout session_layout(const nc_config* c, int B, int T_max) {
     return o;
   };
   L.status = take(256);
-  L.rope = take((size_t)T_max * D * sizeof(float));
+  L.rope = take((size_t)T_max * D * sizeof(float) * 2);  // [2][T_max][D/2] and the pair-major copy
   L.wqkv = take(c->n_layer * L.wqkv_elems * 2);
   L.wo = take(c->n_layer * L.wo_elems * 2);
   L.wfc = take(c->n_layer * L.wfc_elems * 2);
@@ -726,7 +726,7 @@ static nc_status forward_impl(const nc_config* cfg, const nc_weights* w, const i
   if (cudaMemsetAsync(status, 0, 256, st) != cudaSuccess) return NC_ERR_CUDA;
   if (amax && cudaMemsetAsync(amax, 0, (size_t)amax_slots(cfg->n_layer) * 4, st) != cudaSuccess)
     return NC_ERR_CUDA;
-  NC_RUN(NC_K_ROPE_TABLE, rope_table_launch(rope, T_rope, D, cfg->rope_base, st));
+  NC_RUN(NC_K_ROPE_TABLE, rope_table_launch(rope, T_rope, D, cfg->rope_base, st, rope_pairs_of(rope, T_rope, D)));
 
   // fp32 -> bf16 weight cast (e4m3 for the fp8 products); c_q|c_k|c_v rows
   // packed into one matrix per layer.
@@ -768,6 +768,7 @@ static nc_status forward_impl(const nc_config* cfg, const nc_weights* w, const i
     eq.D = D;
     eq.eps = cfg->norm_eps;
     eq.rope_T = T_rope;
+    eq.rope_pairs = rope_pairs_of(rope, T_rope, D);
     if ((ex & NC_EXTRA_VALUE_EMBED) && nc_layer_value_embed(cfg, l) == 1) {
       eq.tokens = tokens;
       eq.ve = w->value_embeds[l];
@@ -916,8 +917,9 @@ nc_status nc_prefill(const nc_config* cfg, const nc_weights* w, const int32_t* t
     uint8_t* base = static_cast<uint8_t*>(session);
     cudaStream_t st = S(stream);
     if (cudaMemsetAsync(base + SL.status, 0, 256, st) != cudaSuccess) return NC_ERR_CUDA;
-    if (nc_status s = rope_table_launch(reinterpret_cast<float*>(base + SL.rope), T_max, cfg->head_dim,
-                                        cfg->rope_base, st))
+    float* rope = reinterpret_cast<float*>(base + SL.rope);
+    if (nc_status s = rope_table_launch(rope, T_max, cfg->head_dim, cfg->rope_base, st,
+                                        rope_pairs_of(rope, T_max, cfg->head_dim)))
       return s;
     return launch_weight_cast(cfg, w, reinterpret_cast<uint16_t*>(base + SL.wqkv),
                               reinterpret_cast<uint16_t*>(base + SL.wo), reinterpret_cast<uint16_t*>(base + SL.wfc),
@@ -1077,7 +1079,7 @@ TrainLayout train_layout(const nc_config* c, int B, int T) {
     return o;
   };
   L.status = take(256);
-  L.rope = take((size_t)T * D * 4);
+  L.rope = take((size_t)T * D * 4 * 2);  // [2][T][D/2] and the pair-major copy
   L.wqkv = take(NL * L.wqkv_elems * 2);
   L.wo = take(NL * L.wo_elems * 2);
   L.wfc = take(NL * L.wfc_elems * 2);
@@ -1203,7 +1205,7 @@ nc_status nc_forward_backward_traced(const nc_config* cfg, const nc_weights* w, 
   };
   // ---------------- forward, keeping what the backward reads
   if (cudaMemsetAsync(status, 0, 256, st) != cudaSuccess) return NC_ERR_CUDA;
-  NC_RUN(NC_K_ROPE_TABLE, rope_table_launch(rope, T, D, cfg->rope_base, st));
+  NC_RUN(NC_K_ROPE_TABLE, rope_table_launch(rope, T, D, cfg->rope_base, st, rope_pairs_of(rope, T, D)));
   NC_RUN(NC_K_CAST, launch_weight_cast(cfg, w, wqkv, wo, wfc, wmp, wlm, L.wqkv_elems, L.wo_elems, L.wfc_elems, L.wmp_elems,
                             f16, st));
   NC_RUN(NC_K_EMBEDDING, embedding_launch(tokens, w->wte, xs, M, C, V, status, st));
@@ -1222,6 +1224,7 @@ nc_status nc_forward_backward_traced(const nc_config* cfg, const nc_weights* w, 
     eq.D = D;
     eq.eps = eps;
     eq.rope_T = T;
+    eq.rope_pairs = rope_pairs_of(rope, T, D);
     eq.rstd_out = rstd_l(l);
     NC_RUN(NC_K_GEMM_QKV, gemm_launch(a, C, wqkv + l * L.wqkv_elems, C, M, NQKV, C, EPI_QKV_ROPE_IL, f16, eq, status, st));
     uint16_t* q = qkv_l(l);

@@ -12,6 +12,15 @@
 //   warp 1      allocates 512 TMEM columns; one thread issues
 //               tcgen05.mma.cta_group::1.kind::f16 (M=128, N=256, K=16) into one of
 //               two 256-column fp32 accumulators and commits stage releases;
+//   CTA pairs   (16-bit K-major operands, M > 128): a cluster of two CTAs
+//               computes 256x256 tiles with tcgen05.mma.cta_group::2 (M=256).
+//               Each CTA loads its own 128 rows of A and 128 of the 256 W rows
+//               (6 stages of 32 KB), both halves signalling rank 0's barrier;
+//               rank 0 issues the MMAs and commits to the barriers of both
+//               CTAs; each CTA's tensor memory receives its 128 rows x 256
+//               columns, and its epilogue warps hand the accumulator back to
+//               rank 0.  Every W byte loaded into shared memory then serves
+//               256 rows instead of 128.
 //   warps 2..9  epilogue: tcgen05.ld of the accumulator (a warp may only read
 //               the 32 TMEM lanes = tile rows its warp index mod 4 selects, so
 //               two warps share each lane quarter and split the 256 columns),
@@ -60,6 +69,17 @@ constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + EPI_WARPS * STG_BYTES + 1024 /
                            256 /*barriers*/;
 constexpr uint32_t IDESC_BF16 = idesc_f32acc(BM, BN, false);
 constexpr uint32_t IDESC_F16 = idesc_f32acc(BM, BN, true);
+// CTA pairs (16-bit K-major operands): one MMA of M = 256 rows over two SMs.
+// Each CTA loads its 128 rows of A and 128 of the tile's 256 rows of W, so a
+// stage is 32 KB and the same ring space holds six of them; each CTA's tensor
+// memory receives the full 256 columns of its own 128 rows.
+constexpr int PAIR_STAGES = 6;
+constexpr int PAIR_B_BYTES = (BN / 2) * BK * 2;
+constexpr int PAIR_STAGE_BYTES = A_BYTES + PAIR_B_BYTES;
+static_assert(PAIR_STAGES * PAIR_STAGE_BYTES <= STAGES * STAGE_BYTES, "pair ring fits the tile ring");
+constexpr int MAX_STAGES = PAIR_STAGES > STAGES ? PAIR_STAGES : STAGES;
+constexpr uint32_t IDESC_PAIR_BF16 = idesc_f32acc(2 * BM, BN, false);
+constexpr uint32_t IDESC_PAIR_F16 = idesc_f32acc(2 * BM, BN, true);
 constexpr uint32_t IDESC_E4M3 = idesc_e4m3_f32acc(BM, BN);
 
 // Dequantisation factors of an e4m3 product, 1 / (s_a s_w), for the q, k and v
@@ -74,8 +94,8 @@ __device__ __forceinline__ void scale32(uint32_t (&r)[32], float f) {
 }
 
 struct Smem {  // barrier block placed after the tile ring and the staging tiles
-  uint64_t full[STAGES];
-  uint64_t empty[STAGES];
+  uint64_t full[MAX_STAGES];
+  uint64_t empty[MAX_STAGES];
   uint64_t tmem_full[NUM_ACC];
   uint64_t tmem_empty[NUM_ACC];
   uint64_t drain;
@@ -513,8 +533,12 @@ __device__ __forceinline__ void epilogue_qkv_head_il(uint32_t taddr, const CUten
   const float rs = SC ? rsqrtf(ss * (dq * dq) * (1.0f / HD) + ep.eps) * dq : rsqrtf(ss * (1.0f / HD) + ep.eps);
   if (ep.rstd_out && row < M) ep.rstd_out[(int64_t)row * (ep.H + ep.Hkv) + head] = rs;
   const int t = ep.pos0 + (row < M ? row : 0) % ep.T;
+  const int rt = ep.rope_T > 0 ? ep.rope_T : ep.T;
   const float* cs = ep.rope + (int64_t)t * (HD / 2);
-  const float* sn = ep.rope + ((int64_t)(ep.rope_T > 0 ? ep.rope_T : ep.T) + t) * (HD / 2);
+  const float* sn = ep.rope + ((int64_t)rt + t) * (HD / 2);
+  // pair-major copy: the warp's 32 rows are consecutive positions, so each
+  // load of one pair's (cos, sin) reads one contiguous run of the table
+  const float2* cp = ep.rope_pairs ? ep.rope_pairs + t : nullptr;
 #pragma unroll 1
   for (int c = 0; c < HD / 64; ++c) {  // pairs 32c .. 32c+31
     uint32_t r0[32], r1[32];
@@ -524,10 +548,20 @@ __device__ __forceinline__ void epilogue_qkv_head_il(uint32_t taddr, const CUten
     uint32_t w[32];
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
-      const float4 c4 = __ldg(reinterpret_cast<const float4*>(cs + c * 32) + j);
-      const float4 s4 = __ldg(reinterpret_cast<const float4*>(sn + c * 32) + j);
-      const float cc[4] = {c4.x, c4.y, c4.z, c4.w};
-      const float sv[4] = {s4.x, s4.y, s4.z, s4.w};
+      float cc[4], sv[4];
+      if (cp) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 v = __ldg(cp + (int64_t)(c * 32 + 4 * j + e) * rt);
+          cc[e] = v.x;
+          sv[e] = v.y;
+        }
+      } else {
+        const float4 c4 = __ldg(reinterpret_cast<const float4*>(cs + c * 32) + j);
+        const float4 s4 = __ldg(reinterpret_cast<const float4*>(sn + c * 32) + j);
+        cc[0] = c4.x, cc[1] = c4.y, cc[2] = c4.z, cc[3] = c4.w;
+        sv[0] = s4.x, sv[1] = s4.y, sv[2] = s4.z, sv[3] = s4.w;
+      }
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const int pp = 4 * j + e;  // pair within the chunk
@@ -551,15 +585,20 @@ __device__ __forceinline__ void epilogue_qkv_head_il(uint32_t taddr, const CUten
 // loaded as boxes of 64 K rows x 64 MN elements (128 bytes, swizzled); the
 // descriptor then steps 64-element MN blocks by the box size and 8-row K
 // groups by 1024 bytes, and each MMA of K = 16 advances 16 rows (2048 bytes).
-template <int EPI, bool F16, int HD, bool FP8, int LAY = GEMM_NT>
+template <int EPI, bool F16, int HD, bool FP8, int LAY = GEMM_NT, bool PAIR = false>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const __grid_constant__ CUtensorMap tmC, int M, int N, int K, EpiParams ep,
                 uint32_t* dev_status, uint64_t limit_ns) {
   constexpr bool A_MN = LAY == GEMM_TN, B_MN = LAY != GEMM_NT;
   static_assert(!(FP8 && LAY != GEMM_NT), "e4m3 operands are K-major");
-  constexpr uint32_t IDESC = (FP8 ? IDESC_E4M3 : (F16 ? IDESC_F16 : IDESC_BF16)) | (A_MN ? (1u << 15) : 0u) |
-                             (B_MN ? (1u << 16) : 0u);
+  static_assert(!PAIR || (!FP8 && LAY == GEMM_NT), "CTA pairs: 16-bit K-major operands");
+  constexpr uint32_t IDESC = PAIR ? (F16 ? IDESC_PAIR_F16 : IDESC_PAIR_BF16)
+                                  : (FP8 ? IDESC_E4M3 : (F16 ? IDESC_F16 : IDESC_BF16)) | (A_MN ? (1u << 15) : 0u) |
+                                        (B_MN ? (1u << 16) : 0u);
+  constexpr int NST = PAIR ? PAIR_STAGES : STAGES;            // ring stages
+  constexpr int SBYTES = PAIR ? PAIR_STAGE_BYTES : STAGE_BYTES;  // bytes of one stage in this CTA
+  constexpr int TM = PAIR ? 2 * BM : BM;                      // rows of one output tile
   constexpr int MN_BOX = 64 * BK * 2;  // bytes of one MN-major box
   constexpr int KE = FP8 ? 2 * BK : BK;  // elements per 128-byte swizzle row
   extern __shared__ uint8_t smem_raw[];
@@ -570,7 +609,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
   const uint32_t warp = warp_id_sync();
   const uint32_t lane = lane_id();
-  const int num_m = (M + BM - 1) / BM;
+  // With CTA pairs both CTAs of cluster c walk the same tiles; rank 0 issues
+  // the MMAs, and each rank owns rows [rank * BM, rank * BM + BM) of a tile.
+  const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
+  const int tile0 = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
+  const int tstride = PAIR ? (int)(gridDim.x >> 1) : (int)gridDim.x;
+  const int num_m = (M + TM - 1) / TM;
   const int num_n = (N + BN - 1) / BN;
   // Split-K (residual-add epilogue only): tile t covers K slice t / (num_m * num_n).
   const int ksplit = (EPI == EPI_RESID_F32 && ep.ksplit > 1) ? ep.ksplit : 1;
@@ -579,13 +623,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const int num_kb = (K + KE - 1) / KE;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < STAGES; ++s) {
+    for (int s = 0; s < NST; ++s) {
       mbar_init(smem_u32(&sm->full[s]), 1);
       mbar_init(smem_u32(&sm->empty[s]), 1);
     }
     for (int a = 0; a < NUM_ACC; ++a) {
       mbar_init(smem_u32(&sm->tmem_full[a]), 1);
-      mbar_init(smem_u32(&sm->tmem_empty[a]), EPI_WARPS);
+      mbar_init(smem_u32(&sm->tmem_empty[a]), PAIR ? 2 * EPI_WARPS : EPI_WARPS);
     }
     mbar_init(smem_u32(&sm->drain), 1);
     sm->abort_flag = 0;
@@ -596,11 +640,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     prefetch_tmap(&tmB);
   }
   if (warp == 1) {
-    tmem_alloc(smem_u32(&sm->tmem_base), TMEM_COLS);
-    tmem_relinquish();
+    if constexpr (PAIR) {
+      tmem_alloc_pair(smem_u32(&sm->tmem_base), TMEM_COLS);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(smem_u32(&sm->tmem_base), TMEM_COLS);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
   __syncthreads();
+  if constexpr (PAIR) cluster_sync();  // both CTAs' barriers are initialised
   tc_fence_after();
   const uint32_t tmem_base = sm->tmem_base;
   const WaitCtl ctl{&sm->abort_flag, dev_status, limit_ns};
@@ -613,19 +663,28 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       uint32_t outstanding = 0;  // bit s: stage s has a load this thread issued
       uint32_t out_phase = 0;    // bit s: phase of that load
       bool ok = true;
-      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+      for (int tile = tile0; tile < num_tiles && ok; tile += tstride) {
         const int mn = tile % num_mn, ks = tile / num_mn;
-        const int m0 = (mn / num_n) * BM;
+        const int m0 = (mn / num_n) * TM;
         const int n0 = (mn % num_n) * BN;
         const int kb_end = (ks + 1) * num_kb / ksplit;
         for (int kb = ks * num_kb / ksplit; kb < kb_end; ++kb) {
-          if (!mbar_wait(smem_u32(&sm->empty[stage]), phase ^ 1u, ctl)) {
+          const uint32_t eb = smem_u32(&sm->empty[stage]);
+          if (!(PAIR ? mbar_wait_cluster(eb, phase ^ 1u, ctl) : mbar_wait(eb, phase ^ 1u, ctl))) {
             ok = false;
             break;
           }
           const uint32_t fb = smem_u32(&sm->full[stage]);
+          uint8_t* a_dst = tiles + stage * SBYTES;
+          if constexpr (PAIR) {
+            // Both halves complete on rank 0's barrier, which expects the bytes
+            // of both CTAs.
+            const uint32_t fb0 = mapa_shared(fb, 0);
+            if (rank == 0) mbar_arrive_expect_tx(fb, 2 * SBYTES);
+            tma_load_2d_pair(smem_u32(a_dst), &tmA, kb * KE, m0 + (int)rank * BM, fb0);
+            tma_load_2d_pair(smem_u32(a_dst + A_BYTES), &tmB, kb * KE, n0 + (int)rank * (BN / 2), fb0);
+          } else {
           mbar_arrive_expect_tx(fb, STAGE_BYTES);
-          uint8_t* a_dst = tiles + stage * STAGE_BYTES;
           if constexpr (A_MN) {
 #pragma unroll
             for (int i = 0; i < BM / 64; ++i) tma_load_2d(smem_u32(a_dst + i * MN_BOX), &tmA, m0 + 64 * i, kb * BK, fb);
@@ -639,33 +698,47 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           } else {
             tma_load_2d(smem_u32(a_dst + A_BYTES), &tmB, kb * KE, n0, fb);
           }
+          }
           outstanding |= 1u << stage;
           out_phase = (out_phase & ~(1u << stage)) | (phase << stage);
-          if (++stage == STAGES) {
+          if (++stage == NST) {
             stage = 0;
             phase ^= 1u;
           }
         }
       }
-      if (!ok || sm->abort_flag) {
-        // Let every copy this thread started land before the CTA exits.
+      if ((!ok || sm->abort_flag) && rank == 0) {
+        // Let every copy this thread started land before the CTA exits (with
+        // CTA pairs, rank 0's barriers also count the peer's copies, and the
+        // closing cluster barrier keeps both CTAs resident until then).
         int zero = 0;
         const WaitCtl drain_ctl{&zero, nullptr, limit_ns};
-        for (int s = 0; s < STAGES; ++s)
+        for (int s = 0; s < NST; ++s)
           if (outstanding & (1u << s))
             mbar_wait(smem_u32(&sm->full[s]), (out_phase >> s) & 1u, drain_ctl);
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
-      // ---------------- UMMA issuer
+    if (lane == 0 && rank == 0) {
+      // ---------------- UMMA issuer (rank 0 of a pair issues for both CTAs)
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
       uint32_t acc_phase = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-        if (!mbar_wait(smem_u32(&sm->tmem_empty[acc]), acc_phase ^ 1u, ctl)) break;
+      // Arrive on a barrier of this CTA and, with CTA pairs, on the same
+      // barrier of the peer once the MMAs issued so far are done.
+      auto commit = [&](uint64_t* bar) {
+        if constexpr (PAIR) {
+          umma_commit_pair(smem_u32(bar));
+          umma_commit_pair(mapa_shared(smem_u32(bar), 1));
+        } else {
+          umma_commit(smem_u32(bar));
+        }
+      };
+      for (int tile = tile0; tile < num_tiles && ok; tile += tstride) {
+        const uint32_t teb = smem_u32(&sm->tmem_empty[acc]);
+        if (!(PAIR ? mbar_wait_cluster(teb, acc_phase ^ 1u, ctl) : mbar_wait(teb, acc_phase ^ 1u, ctl))) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * BN;
         const int ks = tile / num_mn;
@@ -676,32 +749,38 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             break;
           }
           tc_fence_after();
-          const uint32_t a_addr = smem_u32(tiles + stage * STAGE_BYTES);
+          const uint32_t a_addr = smem_u32(tiles + stage * SBYTES);
           const uint32_t b_addr = a_addr + A_BYTES;
 #pragma unroll
           for (int k = 0; k < BK / 16; ++k) {  // 32 bytes of each row (K-major) or 16 rows (MN-major) per MMA
             const uint64_t adesc = A_MN ? sw128_desc(a_addr + k * 2048, MN_BOX, 1024) : sw128_kmajor_desc(a_addr + k * 32);
             const uint64_t bdesc = B_MN ? sw128_desc(b_addr + k * 2048, MN_BOX, 1024) : sw128_kmajor_desc(b_addr + k * 32);
-            if constexpr (FP8)
-              umma_f8(d_tmem, adesc, bdesc, IDESC, (kb != kb_begin || k != 0) ? 1u : 0u);
+            const uint32_t accum = (kb != kb_begin || k != 0) ? 1u : 0u;
+            if constexpr (PAIR)
+              umma_f16_pair(d_tmem, adesc, bdesc, IDESC, accum);
+            else if constexpr (FP8)
+              umma_f8(d_tmem, adesc, bdesc, IDESC, accum);
             else
-              umma_f16(d_tmem, adesc, bdesc, IDESC, (kb != kb_begin || k != 0) ? 1u : 0u);
+              umma_f16(d_tmem, adesc, bdesc, IDESC, accum);
           }
-          umma_commit(smem_u32(&sm->empty[stage]));
-          if (++stage == STAGES) {
+          commit(&sm->empty[stage]);
+          if (++stage == NST) {
             stage = 0;
             phase ^= 1u;
           }
         }
         if (!ok) break;
-        umma_commit(smem_u32(&sm->tmem_full[acc]));
+        commit(&sm->tmem_full[acc]);
         if (++acc == NUM_ACC) {
           acc = 0;
           acc_phase ^= 1u;
         }
       }
       // Wait until every MMA this thread issued has completed.
-      umma_commit(smem_u32(&sm->drain));
+      if constexpr (PAIR)
+        umma_commit_pair(smem_u32(&sm->drain));
+      else
+        umma_commit(smem_u32(&sm->drain));
       int zero = 0;
       WaitCtl drain_ctl{&zero, nullptr, limit_ns};
       mbar_wait(smem_u32(&sm->drain), 0, drain_ctl);
@@ -728,16 +807,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+    for (int tile = tile0; tile < num_tiles; tile += tstride) {
       const int m_blk = (tile % num_mn) / num_n;
       const int n_blk = (tile % num_mn) % num_n;
-      const int m0 = m_blk * BM;
+      const int m0 = m_blk * TM + (int)rank * BM;  // this CTA's first row
       const int n0 = n_blk * BN + half * EPI_COLS;  // this warp's first column
       const int row = m0 + row_in_tile;
       if constexpr (EPI == EPI_QKV_ROPE || EPI == EPI_QKV_ROPE_IL) {
         // This row's cos/sin lines are known before the accumulator is ready:
         // pull them into L1 while the MMAs run (q and k heads only).
-        if (row < M && n0 < N && n0 / HD < ep.H + ep.Hkv) {
+        if (row < M && n0 < N && n0 / HD < ep.H + ep.Hkv && !(EPI == EPI_QKV_ROPE_IL && ep.rope_pairs)) {
           const int t = ep.pos0 + row % ep.T;
           const int rt = ep.rope_T > 0 ? ep.rope_T : ep.T;
           const char* cl = reinterpret_cast<const char*>(ep.rope + (int64_t)t * (HD / 2));
@@ -749,7 +828,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
         }
       }
-      if (!mbar_wait(smem_u32(&sm->tmem_full[acc]), acc_phase, ctl)) break;
+      const uint32_t tfb = smem_u32(&sm->tmem_full[acc]);
+      if (!(PAIR ? mbar_wait_cluster(tfb, acc_phase, ctl) : mbar_wait(tfb, acc_phase, ctl))) break;
       tc_fence_after();
       const uint32_t taddr = tmem_base + ((quarter * 32u) << 16) + acc * BN + half * EPI_COLS;
       const int row0 = m0 + (int)quarter * 32;  // first tile row of this warp
@@ -793,7 +873,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&sm->tmem_empty[acc]));
+      if (lane == 0) {  // the accumulator is free again (rank 0 of a pair counts both CTAs)
+        if constexpr (PAIR)
+          mbar_arrive_cluster(mapa_shared(smem_u32(&sm->tmem_empty[acc]), 0));
+        else
+          mbar_arrive(smem_u32(&sm->tmem_empty[acc]));
+      }
       if (++acc == NUM_ACC) {
         acc = 0;
         acc_phase ^= 1u;
@@ -813,8 +898,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
   tc_fence_before();
   __syncthreads();
+  // With CTA pairs neither CTA may leave while the other can still reach its
+  // shared memory, barriers or tensor memory.
+  if constexpr (PAIR) cluster_sync();
   tc_fence_after();
-  if (warp == 1) tmem_dealloc(tmem_base, TMEM_COLS);
+  if (warp == 1) {
+    if constexpr (PAIR)
+      tmem_dealloc_pair(tmem_base, TMEM_COLS);
+    else
+      tmem_dealloc(tmem_base, TMEM_COLS);
+  }
 }
 
 // ---------------------------------------------------------------- host side
@@ -855,49 +948,89 @@ static bool make_map_u8(CUtensorMap* map, const void* ptr, int64_t rows, int64_t
   return encode_tensor_map_u8(map, 2, ptr, dims, strides, box);
 }
 
-template <int EPI, bool F16, int HD, bool FP8, int LAY = GEMM_NT>
+// Persistent grid: one CTA (or CTA pair) per SM that can hold one.  With CTA
+// pairs the grid is the number of two-CTA clusters the device can keep
+// resident at once (queried once per device), times two.
+template <int EPI, bool F16, int HD, bool FP8, int LAY = GEMM_NT, bool PAIR = false>
 static cudaError_t launch_t(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& mc, int M,
                             int N, int K, const EpiParams& ep, uint32_t* dev_status, uint64_t limit_ns,
                             cudaStream_t stream) {
+  auto kern = gemm_kernel<EPI, F16, HD, FP8, LAY, PAIR>;
   static bool attr_done[64] = {};
+  static int pair_slots[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
-  if (dev < 64 && !attr_done[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_kernel<EPI, F16, HD, FP8, LAY>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (!attr_done[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
     if (e != cudaSuccess) return e;
+    if constexpr (PAIR) {
+      cudaLaunchConfig_t q = {};
+      cudaLaunchAttribute qa[1];
+      qa[0].id = cudaLaunchAttributeClusterDimension;
+      qa[0].val.clusterDim.x = 2;
+      qa[0].val.clusterDim.y = 1;
+      qa[0].val.clusterDim.z = 1;
+      q.gridDim = dim3(2 * 148);
+      q.blockDim = dim3(NUM_THREADS);
+      q.dynamicSmemBytes = SMEM_BYTES;
+      q.attrs = qa;
+      q.numAttrs = 1;
+      int clusters = 0;
+      e = cudaOccupancyMaxActiveClusters(&clusters, kern, &q);
+      if (e != cudaSuccess) return e;
+      if (clusters < 1) return cudaErrorInvalidConfiguration;
+      pair_slots[dev] = clusters;
+    }
     attr_done[dev] = true;
   }
-  const int tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN) * (EPI == EPI_RESID_F32 && ep.ksplit > 1 ? ep.ksplit : 1);
-  const int sms = device_sm_count();
-  const int grid = tiles < sms ? tiles : sms;
-  gemm_kernel<EPI, F16, HD, FP8, LAY><<<grid, NUM_THREADS, SMEM_BYTES, stream>>>(ma, mb, mc, M, N, K, ep,
-                                                                                 dev_status, limit_ns);
-  return cudaGetLastError();
+  const int tm = PAIR ? 2 * BM : BM;
+  const int tiles = ((M + tm - 1) / tm) * ((N + BN - 1) / BN) * (EPI == EPI_RESID_F32 && ep.ksplit > 1 ? ep.ksplit : 1);
+  if constexpr (PAIR) {
+    const int clusters = tiles < pair_slots[dev] ? tiles : pair_slots[dev];
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = 2;
+    at[0].val.clusterDim.y = 1;
+    at[0].val.clusterDim.z = 1;
+    cfg.gridDim = dim3(2 * clusters);
+    cfg.blockDim = dim3(NUM_THREADS);
+    cfg.dynamicSmemBytes = SMEM_BYTES;
+    cfg.stream = stream;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, ma, mb, mc, M, N, K, ep, dev_status, limit_ns);
+  } else {
+    const int sms = device_sm_count();
+    const int grid = tiles < sms ? tiles : sms;
+    kern<<<grid, NUM_THREADS, SMEM_BYTES, stream>>>(ma, mb, mc, M, N, K, ep, dev_status, limit_ns);
+    return cudaGetLastError();
+  }
 }
 
-template <bool F16, bool FP8>
+template <bool F16, bool FP8, bool PAIR = false>
 static cudaError_t dispatch(int epi, const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& mc,
                             int M, int N, int K, const EpiParams& ep, uint32_t* st, uint64_t lim,
                             cudaStream_t s) {
   switch (epi) {
-    case EPI_STORE_16: return launch_t<EPI_STORE_16, F16, 0, FP8>(ma, mb, mc, M, N, K, ep, st, lim, s);
-    case EPI_RELU2_16: return launch_t<EPI_RELU2_16, F16, 0, FP8>(ma, mb, mc, M, N, K, ep, st, lim, s);
-    case EPI_RESID_F32: return launch_t<EPI_RESID_F32, F16, 0, FP8>(ma, mb, mc, M, N, K, ep, st, lim, s);
-    case EPI_STORE_F32: return launch_t<EPI_STORE_F32, F16, 0, FP8>(ma, mb, mc, M, N, K, ep, st, lim, s);
-    case EPI_SOFTCAP_F32: return launch_t<EPI_SOFTCAP_F32, F16, 0, FP8>(ma, mb, mc, M, N, K, ep, st, lim, s);
-    case EPI_CE_PARTIAL: return launch_t<EPI_CE_PARTIAL, F16, 0, FP8>(ma, mb, mc, M, N, K, ep, st, lim, s);
+    case EPI_STORE_16: return launch_t<EPI_STORE_16, F16, 0, FP8, GEMM_NT, PAIR>(ma, mb, mc, M, N, K, ep, st, lim, s);
+    case EPI_RELU2_16: return launch_t<EPI_RELU2_16, F16, 0, FP8, GEMM_NT, PAIR>(ma, mb, mc, M, N, K, ep, st, lim, s);
+    case EPI_RESID_F32: return launch_t<EPI_RESID_F32, F16, 0, FP8, GEMM_NT, PAIR>(ma, mb, mc, M, N, K, ep, st, lim, s);
+    case EPI_STORE_F32: return launch_t<EPI_STORE_F32, F16, 0, FP8, GEMM_NT, PAIR>(ma, mb, mc, M, N, K, ep, st, lim, s);
+    case EPI_SOFTCAP_F32: return launch_t<EPI_SOFTCAP_F32, F16, 0, FP8, GEMM_NT, PAIR>(ma, mb, mc, M, N, K, ep, st, lim, s);
+    case EPI_CE_PARTIAL: return launch_t<EPI_CE_PARTIAL, F16, 0, FP8, GEMM_NT, PAIR>(ma, mb, mc, M, N, K, ep, st, lim, s);
     case EPI_CE_BWD_16:
       if constexpr (FP8) return cudaErrorInvalidValue;
-      else return launch_t<EPI_CE_BWD_16, F16, 0, false>(ma, mb, mc, M, N, K, ep, st, lim, s);
+      else return launch_t<EPI_CE_BWD_16, F16, 0, false, GEMM_NT, PAIR>(ma, mb, mc, M, N, K, ep, st, lim, s);
     case EPI_QKV_ROPE:
       if constexpr (FP8) return cudaErrorInvalidValue;  // the interleaved form only
       else
-        return ep.D == 128 ? launch_t<EPI_QKV_ROPE, F16, 128, false>(ma, mb, mc, M, N, K, ep, st, lim, s)
-                           : launch_t<EPI_QKV_ROPE, F16, 64, false>(ma, mb, mc, M, N, K, ep, st, lim, s);
+        return ep.D == 128 ? launch_t<EPI_QKV_ROPE, F16, 128, false, GEMM_NT, PAIR>(ma, mb, mc, M, N, K, ep, st, lim, s)
+                           : launch_t<EPI_QKV_ROPE, F16, 64, false, GEMM_NT, PAIR>(ma, mb, mc, M, N, K, ep, st, lim, s);
     case EPI_QKV_ROPE_IL:
-      return ep.D == 128 ? launch_t<EPI_QKV_ROPE_IL, F16, 128, FP8>(ma, mb, mc, M, N, K, ep, st, lim, s)
-                         : launch_t<EPI_QKV_ROPE_IL, F16, 64, FP8>(ma, mb, mc, M, N, K, ep, st, lim, s);
+      return ep.D == 128 ? launch_t<EPI_QKV_ROPE_IL, F16, 128, FP8, GEMM_NT, PAIR>(ma, mb, mc, M, N, K, ep, st, lim, s)
+                         : launch_t<EPI_QKV_ROPE_IL, F16, 64, FP8, GEMM_NT, PAIR>(ma, mb, mc, M, N, K, ep, st, lim, s);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -1010,10 +1143,17 @@ nc_status gemm_launch(const uint16_t* a, int64_t lda, const uint16_t* w, int64_t
   if (nc_status s = check_epi(epi, K, BK, ep)) return s;
   CUtensorMap ma, mb, mc;
   if (!make_map(&ma, a, M, K, lda, BM, f16)) return NC_ERR_CUDA;
-  if (!make_map(&mb, w, N, K, ldw, BN, f16)) return NC_ERR_CUDA;
+  // CTA pairs for every product with more than one 128-row block (no split K).
+  const bool pair = M > BM && ep.ksplit <= 1;
+  if (!make_map(&mb, w, N, K, ldw, pair ? BN / 2 : BN, f16)) return NC_ERR_CUDA;
   if (!make_out_map(&mc, epi, M, N, f16, ep)) return NC_ERR_CUDA;
-  const cudaError_t e = f16 ? dispatch<true, false>(epi, ma, mb, mc, M, N, K, ep, dev_status, limit_ns, stream)
-                            : dispatch<false, false>(epi, ma, mb, mc, M, N, K, ep, dev_status, limit_ns, stream);
+  cudaError_t e;
+  if (pair)
+    e = f16 ? dispatch<true, false, true>(epi, ma, mb, mc, M, N, K, ep, dev_status, limit_ns, stream)
+            : dispatch<false, false, true>(epi, ma, mb, mc, M, N, K, ep, dev_status, limit_ns, stream);
+  else
+    e = f16 ? dispatch<true, false>(epi, ma, mb, mc, M, N, K, ep, dev_status, limit_ns, stream)
+            : dispatch<false, false>(epi, ma, mb, mc, M, N, K, ep, dev_status, limit_ns, stream);
   return e == cudaSuccess ? NC_OK : NC_ERR_CUDA;
 }
 

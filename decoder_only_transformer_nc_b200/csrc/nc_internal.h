@@ -45,6 +45,9 @@ struct EpiParams {
   int T;                    // EPI_QKV_ROPE: positions per sequence (row m is at pos0 + m % T)
   int pos0;                 // EPI_QKV_ROPE: position of the first row of each sequence
   int rope_T;               // EPI_QKV_ROPE: positions in the rope table (0: T)
+  const float2* rope_pairs;  // EPI_QKV_ROPE_IL: the same angles as [D/2][rope_T] (cos, sin)
+                            //   pairs, so a warp's 32 consecutive positions read one line
+                            //   per pair; null: read `rope`
   int ksplit;               // EPI_RESID_F32: K is split into this many slices, each tile of a
                             //   slice adding its partial product into out (0 or 1: no split;
                             //   the fp32 sums then depend on the order the slices land)
@@ -220,7 +223,12 @@ nc_status relu2_finish_launch(const float* acc, uint16_t* out, int64_t n, bool f
 nc_status rmsnorm_launch(const float* x, uint16_t* out, int M, int C, float eps, bool f16,
                          cudaStream_t stream,
                          float* amax = nullptr);
-nc_status rope_table_launch(float* table, int T, int D, float base, cudaStream_t stream);
+// table [2][T][D/2] (cos, sin); pairs, when given, the same values as [D/2][T] float2.
+nc_status rope_table_launch(float* table, int T, int D, float base, cudaStream_t stream, float2* pairs = nullptr);
+// The pair-major copy kept right after a [2][T][D/2] table in the library's own buffers.
+inline float2* rope_pairs_of(float* table, int T, int D) {
+  return reinterpret_cast<float2*>(table + (size_t)T * D);
+}
 nc_status rope_qknorm_launch(uint16_t* q, uint16_t* k, const float* table, int B, int T, int H,
                              int Hkv, int D, int64_t q_stride, int64_t k_stride, float eps, bool f16,
                              cudaStream_t stream);

@@ -363,7 +363,8 @@ __global__ void __launch_bounds__(256) rmsnorm_mix_kernel(float* __restrict__ x,
 
 // ---------------------------------------------------------------- RoPE
 
-__global__ void rope_table_kernel(float* __restrict__ table, int T, int D, double base) {
+__global__ void rope_table_kernel(float* __restrict__ table, int T, int D, double base,
+                                  float2* __restrict__ pairs) {
   const int half = D / 2;
   const int idx = blockIdx.x * blockDim.x + threadIdx.x;
   if (idx >= T * half) return;
@@ -371,8 +372,10 @@ __global__ void rope_table_kernel(float* __restrict__ table, int T, int D, doubl
   const int i = idx - t * half;
   const double theta = pow(base, -2.0 * (double)i / (double)D);
   const double ang = (double)t * theta;
-  table[idx] = (float)cos(ang);
-  table[(int64_t)T * half + idx] = (float)sin(ang);
+  const float c = (float)cos(ang), s = (float)sin(ang);
+  table[idx] = c;
+  table[(int64_t)T * half + idx] = s;
+  if (pairs) pairs[(int64_t)i * T + t] = make_float2(c, s);
 }
 
 // One group of D/4 lanes per (token, head).  Lane l of the group holds the
@@ -667,10 +670,10 @@ nc_status rmsnorm_launch(const float* x, uint16_t* out, int M, int C, float eps,
   return last_error();
 }
 
-nc_status rope_table_launch(float* table, int T, int D, float base, cudaStream_t stream) {
+nc_status rope_table_launch(float* table, int T, int D, float base, cudaStream_t stream, float2* pairs) {
   const int n = T * (D / 2);
   if (n == 0) return NC_OK;
-  rope_table_kernel<<<(n + 255) / 256, 256, 0, stream>>>(table, T, D, (double)base);
+  rope_table_kernel<<<(n + 255) / 256, 256, 0, stream>>>(table, T, D, (double)base, pairs);
   return last_error();
 }
 
