@@ -50,12 +50,12 @@ DTYPE_NOTE_FP8 = ("e4m3 tensor-core operands with dynamic tensorwise scales for 
 GEMM_KINDS = ("gemm_qkv", "gemm_attn_proj", "gemm_fc", "gemm_mlp_proj", "gemm_lm_head")
 ROOFLINE_KIND = "gemm_fc"  # the kind with the largest share of the step
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one c_fc launch of
-# the d20 workload at B=32, T=2048, from an ncu capture of the current kernel at
-# B=8 scaled to B=32 by the tokens processed: reads 55.09 MB = A (42.0 MB, x4)
-# + W (13.1 MB, once); writes 116.29 MB of the 167.8 MB output, the other
-# 51.5 MB still dirty in L2 when the kernel ends (671.1 - 51.5 MB at B=32).
-# Valid for that workload and kernel only.
-FC_TRAFFIC = {("d20", 32, 2048): (4 * 41.94e6 + 13.11e6) + (4 * 167.77e6 - 51.48e6)}
+# the d20 workload at B=32, T=2048, from an ncu capture of the current kernel
+# (CTA pairs, 256x256 tiles) at B=8 scaled to B=32 by the tokens processed:
+# reads 55.11 MB = A (41.9 MB, x4) + W (13.1 MB, once); writes 119.29 MB of the
+# 167.8 MB output, the other 48.5 MB still dirty in L2 when the kernel ends
+# (671.1 - 48.5 MB at B=32).  Valid for that workload and kernel only.
+FC_TRAFFIC = {("d20", 32, 2048): (4 * 41.94e6 + 13.11e6) + (4 * 167.77e6 - 48.48e6)}
 
 
 def load_peaks():

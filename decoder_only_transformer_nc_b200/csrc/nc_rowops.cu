@@ -363,19 +363,28 @@ __global__ void __launch_bounds__(256) rmsnorm_mix_kernel(float* __restrict__ x,
 
 // ---------------------------------------------------------------- RoPE
 
+// Threads [0, T D/2) write the [2][T][D/2] table in its order; with `pairs`,
+// threads [T D/2, T D) write the [D/2][T] (cos, sin) copy in its own order, so
+// both stores are coalesced.  Both compute the same fp64 angle.
 __global__ void rope_table_kernel(float* __restrict__ table, int T, int D, double base,
                                   float2* __restrict__ pairs) {
   const int half = D / 2;
-  const int idx = blockIdx.x * blockDim.x + threadIdx.x;
-  if (idx >= T * half) return;
-  const int t = idx / half;
-  const int i = idx - t * half;
+  const int n = T * half;
+  int idx = blockIdx.x * blockDim.x + threadIdx.x;
+  const bool pair_major = idx >= n;
+  if (pair_major) idx -= n;
+  if (idx >= n || (pair_major && !pairs)) return;
+  const int t = pair_major ? idx % T : idx / half;
+  const int i = pair_major ? idx / T : idx % half;
   const double theta = pow(base, -2.0 * (double)i / (double)D);
   const double ang = (double)t * theta;
   const float c = (float)cos(ang), s = (float)sin(ang);
-  table[idx] = c;
-  table[(int64_t)T * half + idx] = s;
-  if (pairs) pairs[(int64_t)i * T + t] = make_float2(c, s);
+  if (pair_major) {
+    pairs[idx] = make_float2(c, s);
+  } else {
+    table[idx] = c;
+    table[(int64_t)n + idx] = s;
+  }
 }
 
 // One group of D/4 lanes per (token, head).  Lane l of the group holds the
@@ -671,7 +680,7 @@ nc_status rmsnorm_launch(const float* x, uint16_t* out, int M, int C, float eps,
 }
 
 nc_status rope_table_launch(float* table, int T, int D, float base, cudaStream_t stream, float2* pairs) {
-  const int n = T * (D / 2);
+  const int n = T * (D / 2) * (pairs ? 2 : 1);
   if (n == 0) return NC_OK;
   rope_table_kernel<<<(n + 255) / 256, 256, 0, stream>>>(table, T, D, (double)base, pairs);
   return last_error();
