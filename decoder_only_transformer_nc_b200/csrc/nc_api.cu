@@ -1310,7 +1310,7 @@ nc_status nc_forward_backward_traced(const nc_config* cfg, const nc_weights* w, 
     NC_RUN(NC_K_GEMM_WGRAD, wgrad(dx16, C, o_l(l), HD, C, HD, g->attn_proj[l], HD));
     NC_RUN(NC_K_GEMM_DGRAD, dgrad(dx16, C, wo + l * L.wo_elems, HD, EPI_STORE_16, dO));
     NC_RUN(NC_K_ATTN_BWD, attn_bwd_launch(qkv_l(l), NQKV, o_l(l), dO, lse_l(l), delta, dqkv, B, T, H, Hkv, D,
-                           nc_layer_window(cfg, l), f16, st));
+                           nc_layer_window(cfg, l), f16, st, status));
     NC_RUN(NC_K_QK_BWD, qk_bwd_launch(dqkv, qkv_l(l), NQKV, rstd_l(l), rope, T, M, T, H, Hkv, D, f16, st));
     NC_RUN(NC_K_RMSNORM, rmsnorm_launch(xin, a, M, C, eps, f16, st));
     NC_RUN(NC_K_GEMM_WGRAD, cudaMemsetAsync(dwqkv, 0, (size_t)NQKV * C * 4, st) == cudaSuccess

@@ -1,6 +1,5 @@
 // Backward of the block stack ("从文本到聊天模型" §6.5: the training step's
-// loss.backward() after the forward's loss): the row kernels and the attention
-// backward.  The projections' dgrad / wgrad products run on the tcgen05 GEMM
+// loss.backward() after the forward's loss): the row kernels.  The projections' dgrad / wgrad products run on the tcgen05 GEMM
 // (nc_gemm.cu, GEMM_NN / GEMM_TN layouts; soft-cap + cross-entropy and relu^2
 // backward in its epilogues).
 //
@@ -8,31 +7,17 @@
 // 1 / (number of counted targets) of the mean into the weight gradients, so the
 // 16-bit intermediate gradients stay O(1) per token.
 //
-// Attention backward (per head, window W, scale 1/sqrt(D), P recomputed from
-// the forward's log-sum-exp):  dV = P^T dO,  dP = dO V^T,
-// dS = P o (dP - Delta) with Delta_i = sum_d dO_i O_i,  dQ = scale dS K,
-// dK = scale dS^T Q.  Two kernels, so that no sum needs atomics:
-//   attn_bwd_dq_kernel    one CTA per (64 queries, head, row): loops over the
-//                         key tiles inside the window;
-//   attn_bwd_dkdv_kernel  one CTA per (64 keys, kv head, row): loops over the
-//                         query heads of its group and the query tiles that see
-//                         these keys.
-// Both use the warp-level mma.sync.m16n8k16 tensor-core path (fp32
-// accumulation) with 16-bit tiles staged in padded shared memory and read by
-// ldmatrix; each warp owns 16 rows of the CTA's tile.
+// The attention backward runs on tcgen05 in nc_attention_bwd.cu.
 #include <cuda_runtime.h>
 
 #include <cstdint>
 
 #include "nc_half.cuh"
 #include "nc_internal.h"
-#include "nc_mma.cuh"
 #include "nc_ptx.cuh"
 
 namespace nc {
 namespace bwd {
-
-using namespace wmma16;
 
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
@@ -129,24 +114,6 @@ __global__ void __launch_bounds__(256) qk_bwd_kernel(uint16_t* __restrict__ dqkv
 }
 
 // ---------------------------------------------------------------- small kernels
-// Delta[m, h] = sum_d dO[m, h, d] O[m, h, d]
-template <bool F16>
-__global__ void __launch_bounds__(256) attn_delta_kernel(const uint16_t* __restrict__ dO, const uint16_t* __restrict__ O,
-                                                         float* __restrict__ delta, int M, int H, int D) {
-  const int64_t wid = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int lane = threadIdx.x & 31;
-  if (wid >= (int64_t)M * H) return;
-  const int64_t base = wid * D;
-  float s = 0.0f;
-  for (int d = lane * 2; d < D; d += 64) {
-    const float2 a = Half<F16>::unpack2(*reinterpret_cast<const uint32_t*>(dO + base + d));
-    const float2 b = Half<F16>::unpack2(*reinterpret_cast<const uint32_t*>(O + base + d));
-    s += a.x * b.x + a.y * b.y;
-  }
-  s = warp_sum(s);
-  if (lane == 0) delta[wid] = s;
-}
-
 // dwte[token[m]] += alpha dx[m] (alpha read from device memory); one warp per row.
 __global__ void __launch_bounds__(256) embedding_bwd_kernel(const int32_t* __restrict__ tokens,
                                                             const float* __restrict__ dx, float* __restrict__ dwte,
@@ -199,274 +166,6 @@ __global__ void __launch_bounds__(256) qkv_grad_scatter_kernel(const float* __re
   }
 }
 
-// ---------------------------------------------------------------- attention backward
-constexpr int BLK = 64;        // rows of a tile (queries or keys)
-constexpr int NTH = 128;       // 4 warps x 16 rows
-constexpr float kLog2e = 1.4426950408889634f;
-
-__device__ __forceinline__ float ex2f(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
-
-// rows [row0, row0 + 64) of a 16-bit [rows, D] view (row stride ld elements,
-// head column offset col) into a padded shared tile; rows >= T are zeros.
-template <int D, int LD>
-__device__ __forceinline__ void stage_tile(uint16_t* dst, const uint16_t* src, int64_t ld, int64_t row_base,
-                                           int row0, int T) {
-  constexpr int CH = D / 8;  // 16-byte chunks per row
-  for (int i = threadIdx.x; i < BLK * CH; i += NTH) {
-    const int r = i / CH, c = i % CH;
-    uint4 v = make_uint4(0u, 0u, 0u, 0u);
-    if (row0 + r < T) v = *reinterpret_cast<const uint4*>(src + (row_base + row0 + r) * ld + c * 8);
-    *reinterpret_cast<uint4*>(dst + r * LD + c * 8) = v;
-  }
-}
-
-// The same with 16-byte cp.async copies (rows >= T zero-filled), so the load
-// of the next tile overlaps the products of the current one.
-template <int D, int LD>
-__device__ __forceinline__ void stage_tile_async(uint16_t* dst, const uint16_t* src, int64_t ld, int64_t row_base,
-                                                 int row0, int T) {
-  constexpr int CH = D / 8;
-  for (int i = threadIdx.x; i < BLK * CH; i += NTH) {
-    const int r = i / CH, c = i % CH;
-    const bool valid = row0 + r < T;
-    const uint16_t* g = src + (row_base + (valid ? row0 + r : 0)) * ld + c * 8;
-    cp_async16(dst + r * LD + c * 8, g, valid);
-  }
-}
-
-// S (16 x 64 per warp) = A_tile[rows w*16..] . B_tile^T over D, both [row][D] tiles.
-template <int D, int LD, bool F16>
-__device__ __forceinline__ void tile_dots(float (&acc)[8][4], uint32_t a_base, uint32_t b_base, int wrow, int lane) {
-#pragma unroll
-  for (int nt = 0; nt < 8; ++nt)
-#pragma unroll
-    for (int e = 0; e < 4; ++e) acc[nt][e] = 0.0f;
-#pragma unroll
-  for (int kk = 0; kk < D / 16; ++kk) {
-    uint32_t a[4];
-    load_a<LD>(a, a_base, wrow, kk * 16, lane);
-#pragma unroll
-    for (int np = 0; np < 4; ++np) {
-      uint32_t b[4];
-      load_b_nk<LD>(b, b_base, np * 16, kk * 16, lane);
-      mma16816<F16>(acc[2 * np], a, b[0], b[1]);
-      mma16816<F16>(acc[2 * np + 1], a, b[2], b[3]);
-    }
-  }
-}
-
-// out (16 x D per warp) += X (16 x 64, C-fragments) . Y_tile (64 x D, stored [k][d]).
-template <int D, int LD, bool F16>
-__device__ __forceinline__ void tile_accum(float (&out)[D / 8][4], const float (&x)[8][4], uint32_t y_base, int lane) {
-#pragma unroll
-  for (int kc = 0; kc < 4; ++kc) {  // 16 of the 64 contraction rows
-    uint32_t a[4];
-    a[0] = Half<F16>::pack2(x[2 * kc][0], x[2 * kc][1]);
-    a[1] = Half<F16>::pack2(x[2 * kc][2], x[2 * kc][3]);
-    a[2] = Half<F16>::pack2(x[2 * kc + 1][0], x[2 * kc + 1][1]);
-    a[3] = Half<F16>::pack2(x[2 * kc + 1][2], x[2 * kc + 1][3]);
-#pragma unroll
-    for (int dp = 0; dp < D / 16; ++dp) {
-      uint32_t b[4];
-      load_b_kn<LD>(b, y_base, kc * 16, dp * 16, lane);
-      mma16816<F16>(out[2 * dp], a, b[0], b[1]);
-      mma16816<F16>(out[2 * dp + 1], a, b[2], b[3]);
-    }
-  }
-}
-
-// Write a warp's 16 x D fp32 fragment rows (row0 + g, row0 + g + 8) as 16-bit.
-template <int D, bool F16>
-__device__ __forceinline__ void store_rows(const float (&acc)[D / 8][4], uint16_t* dst, int64_t ld, int64_t row_base,
-                                           int row0, int T, int lane, float f) {
-  const int g = lane >> 2, t = lane & 3;
-#pragma unroll
-  for (int half = 0; half < 2; ++half) {
-    const int r = row0 + g + 8 * half;
-    if (r >= T) continue;
-    uint16_t* p = dst + (row_base + r) * ld;
-#pragma unroll
-    for (int nt = 0; nt < D / 8; ++nt)
-      *reinterpret_cast<uint32_t*>(p + nt * 8 + 2 * t) =
-          Half<F16>::pack2(acc[nt][2 * half] * f, acc[nt][2 * half + 1] * f);
-  }
-}
-
-template <int D, bool F16>
-__global__ void __launch_bounds__(NTH, 1)
-    attn_bwd_dq_kernel(const uint16_t* __restrict__ qkv, int64_t ldqkv, const uint16_t* __restrict__ dO,
-                       const float* __restrict__ lse, const float* __restrict__ delta, uint16_t* __restrict__ dqkv,
-                       int T, int H, int Hkv, int W, float scale) {
-  constexpr int LD = D + 8;
-  extern __shared__ __align__(16) uint8_t smem_raw[];
-  uint16_t* sQ = reinterpret_cast<uint16_t*>(smem_raw);
-  uint16_t* sdO = sQ + BLK * LD;
-  uint16_t* sKV = sdO + BLK * LD;  // two buffers of (K tile, V tile)
-  const int q0 = blockIdx.x * BLK, h = blockIdx.y, b = blockIdx.z;
-  const int g = h / (H / Hkv);
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t rb = (int64_t)b * T;
-  const int64_t HD = (int64_t)H * D;
-  stage_tile<D, LD>(sQ, qkv + (int64_t)h * D, ldqkv, rb, q0, T);
-  stage_tile<D, LD>(sdO, dO + (int64_t)h * D, HD, rb, q0, T);
-  const int ra = q0 + warp * 16 + (lane >> 2), rbw = ra + 8;  // this thread's two query rows
-  const float lse_a = ra < T ? lse[(rb + ra) * H + h] : 0.0f, lse_b = rbw < T ? lse[(rb + rbw) * H + h] : 0.0f;
-  const float dl_a = ra < T ? delta[(rb + ra) * H + h] : 0.0f, dl_b = rbw < T ? delta[(rb + rbw) * H + h] : 0.0f;
-  const float c1 = scale * kLog2e;
-  float dq[D / 8][4];
-#pragma unroll
-  for (int i = 0; i < D / 8; ++i)
-#pragma unroll
-    for (int e = 0; e < 4; ++e) dq[i][e] = 0.0f;
-  const int q_last = min(T - 1, q0 + BLK - 1);
-  const int kt_lo = max(0, q0 - W + 1) / BLK, kt_hi = q_last / BLK;
-  const uint32_t bq = smem_u32(sQ), bdo = smem_u32(sdO);
-  auto issue = [&](int kt) {  // K and V tiles of key tile kt into buffer kt & 1
-    uint16_t* dst = sKV + (kt & 1) * 2 * BLK * LD;
-    stage_tile_async<D, LD>(dst, qkv + (int64_t)(H + g) * D, ldqkv, rb, kt * BLK, T);
-    stage_tile_async<D, LD>(dst + BLK * LD, qkv + (int64_t)(H + Hkv + g) * D, ldqkv, rb, kt * BLK, T);
-    cp_async_commit();
-  };
-  issue(kt_lo);
-  for (int kt = kt_lo; kt <= kt_hi; ++kt) {
-    const int k0 = kt * BLK;
-    if (kt < kt_hi) {
-      issue(kt + 1);
-      cp_async_wait<1>();  // this tile's group has landed; the next one may still be in flight
-    } else {
-      cp_async_wait<0>();
-    }
-    __syncthreads();
-    const uint32_t bk = smem_u32(sKV + (kt & 1) * 2 * BLK * LD), bv = bk + BLK * LD * 2;
-    float s[8][4], dp[8][4];
-    tile_dots<D, LD, F16>(s, bq, bk, warp * 16, lane);
-    tile_dots<D, LD, F16>(dp, bdo, bv, warp * 16, lane);
-#pragma unroll
-    for (int nt = 0; nt < 8; ++nt)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int i = e < 2 ? ra : rbw;
-        const int j = k0 + nt * 8 + 2 * (lane & 3) + (e & 1);
-        const bool vis = i < T && j <= i && i - j < W;
-        const float p = vis ? ex2f(fmaf(s[nt][e], c1, -(e < 2 ? lse_a : lse_b) * kLog2e)) : 0.0f;
-        s[nt][e] = p * (dp[nt][e] - (e < 2 ? dl_a : dl_b));  // dS / scale
-      }
-    tile_accum<D, LD, F16>(dq, s, bk, lane);
-    __syncthreads();  // buffer kt & 1 is refilled by the issue of tile kt + 2
-  }
-  store_rows<D, F16>(dq, dqkv + (int64_t)h * D, ldqkv, rb, q0 + warp * 16, T, lane, scale);
-}
-
-template <int D, bool F16>
-__global__ void __launch_bounds__(NTH, 1)
-    attn_bwd_dkdv_kernel(const uint16_t* __restrict__ qkv, int64_t ldqkv, const uint16_t* __restrict__ dO,
-                         const float* __restrict__ lse, const float* __restrict__ delta, uint16_t* __restrict__ dqkv,
-                         int T, int H, int Hkv, int W, float scale) {
-  constexpr int LD = D + 8;
-  extern __shared__ __align__(16) uint8_t smem_raw[];
-  uint16_t* sK = reinterpret_cast<uint16_t*>(smem_raw);
-  uint16_t* sV = sK + BLK * LD;
-  uint16_t* sQD = sV + BLK * LD;                            // two buffers of (Q tile, dO tile)
-  float* sLD = reinterpret_cast<float*>(sQD + 4 * BLK * LD);  // two buffers of ([BLK] lse, [BLK] delta)
-  const int k0 = blockIdx.x * BLK, g = blockIdx.y, b = blockIdx.z;
-  const int G = H / Hkv;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t rb = (int64_t)b * T;
-  const int64_t HD = (int64_t)H * D;
-  stage_tile<D, LD>(sK, qkv + (int64_t)(H + g) * D, ldqkv, rb, k0, T);
-  stage_tile<D, LD>(sV, qkv + (int64_t)(H + Hkv + g) * D, ldqkv, rb, k0, T);
-  const int ja = k0 + warp * 16 + (lane >> 2), jb = ja + 8;  // this thread's two key rows
-  const float c1 = scale * kLog2e;
-  float dk[D / 8][4], dv[D / 8][4];
-#pragma unroll
-  for (int i = 0; i < D / 8; ++i)
-#pragma unroll
-    for (int e = 0; e < 4; ++e) dk[i][e] = dv[i][e] = 0.0f;
-  const int k_last = min(T - 1, k0 + BLK - 1);
-  const int qt_lo = k0 / BLK, qt_hi = min(T - 1, k_last + W - 1) / BLK;
-  const uint32_t bk = smem_u32(sK), bv = smem_u32(sV);
-  const int nq = qt_hi - qt_lo + 1, n_it = G * nq;  // iterations: (head of the group, query tile)
-  auto issue = [&](int it) {  // Q, dO tiles and lse, delta of iteration it into buffer it & 1
-    const int h = g * G + it / nq, q0 = (qt_lo + it % nq) * BLK;
-    uint16_t* dst = sQD + (it & 1) * 2 * BLK * LD;
-    stage_tile_async<D, LD>(dst, qkv + (int64_t)h * D, ldqkv, rb, q0, T);
-    stage_tile_async<D, LD>(dst + BLK * LD, dO + (int64_t)h * D, HD, rb, q0, T);
-    float* l = sLD + (it & 1) * 2 * BLK;
-    for (int i = threadIdx.x; i < BLK; i += NTH) {
-      const bool in = q0 + i < T;
-      const int64_t r = (rb + (in ? q0 + i : 0)) * H + h;
-      cp_async4(l + i, lse + r, in);
-      cp_async4(l + BLK + i, delta + r, in);
-    }
-    cp_async_commit();
-  };
-  if (n_it > 0) issue(0);
-  for (int it = 0; it < n_it; ++it) {
-    {
-      const int q0 = (qt_lo + it % nq) * BLK;
-      if (it + 1 < n_it) {
-        issue(it + 1);
-        cp_async_wait<1>();
-      } else {
-        cp_async_wait<0>();
-      }
-      __syncthreads();
-      const uint32_t bq = smem_u32(sQD + (it & 1) * 2 * BLK * LD), bdo = bq + BLK * LD * 2;
-      const float* sL = sLD + (it & 1) * 2 * BLK;
-      float s[8][4], dp[8][4];
-      tile_dots<D, LD, F16>(s, bk, bq, warp * 16, lane);   // S^T: keys x queries
-      tile_dots<D, LD, F16>(dp, bv, bdo, warp * 16, lane); // dP^T
-#pragma unroll
-      for (int nt = 0; nt < 8; ++nt)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int jq = nt * 8 + 2 * (lane & 3) + (e & 1);  // query within the tile
-          const int i = q0 + jq;
-          const int j = e < 2 ? ja : jb;
-          const bool vis = i < T && j < T && j <= i && i - j < W;
-          const float p = vis ? ex2f(fmaf(s[nt][e], c1, -sL[jq] * kLog2e)) : 0.0f;
-          s[nt][e] = p;                              // P^T
-          dp[nt][e] = p * (dp[nt][e] - sL[BLK + jq]);  // dS^T / scale
-        }
-      tile_accum<D, LD, F16>(dv, s, bdo, lane);
-      tile_accum<D, LD, F16>(dk, dp, bq, lane);
-      __syncthreads();  // buffer it & 1 is refilled by the issue of iteration it + 2
-    }
-  }
-  store_rows<D, F16>(dk, dqkv + (int64_t)(H + g) * D, ldqkv, rb, k0 + warp * 16, T, lane, scale);
-  store_rows<D, F16>(dv, dqkv + (int64_t)(H + Hkv + g) * D, ldqkv, rb, k0 + warp * 16, T, lane, 1.0f);
-}
-
-template <int D, bool F16>
-static nc_status attn_bwd_t(const uint16_t* qkv, int64_t ldqkv, const uint16_t* dO, const float* lse,
-                            const float* delta, uint16_t* dqkv, int B, int T, int H, int Hkv, int W,
-                            cudaStream_t stream) {
-  constexpr int LD = D + 8;
-  const int smem_q = 6 * BLK * LD * 2;                  // Q, dO, and two (K, V) buffers
-  const int smem_k = 6 * BLK * LD * 2 + 4 * BLK * 4;    // K, V, two (Q, dO) and two (lse, delta) buffers
-  static bool attr_done[64] = {};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 64 && !attr_done[dev]) {
-    if (cudaFuncSetAttribute(attn_bwd_dq_kernel<D, F16>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_q) !=
-            cudaSuccess ||
-        cudaFuncSetAttribute(attn_bwd_dkdv_kernel<D, F16>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_k) !=
-            cudaSuccess)
-      return NC_ERR_CUDA;
-    attr_done[dev] = true;
-  }
-  const float scale = 1.0f / sqrtf((float)D);
-  const dim3 gq((T + BLK - 1) / BLK, H, B), gk((T + BLK - 1) / BLK, Hkv, B);
-  attn_bwd_dq_kernel<D, F16><<<gq, NTH, smem_q, stream>>>(qkv, ldqkv, dO, lse, delta, dqkv, T, H, Hkv, W, scale);
-  if (cudaGetLastError() != cudaSuccess) return NC_ERR_CUDA;
-  attn_bwd_dkdv_kernel<D, F16><<<gk, NTH, smem_k, stream>>>(qkv, ldqkv, dO, lse, delta, dqkv, T, H, Hkv, W, scale);
-  return cudaGetLastError() == cudaSuccess ? NC_OK : NC_ERR_CUDA;
-}
-
 }  // namespace bwd
 
 nc_status rmsnorm_bwd_launch(const float* x, const float* dy, float* dx_acc, uint16_t* dx16, int M, int C, float eps,
@@ -492,26 +191,6 @@ nc_status qk_bwd_launch(uint16_t* dqkv, const uint16_t* qkv, int64_t ld, const f
   else
     bwd::qk_bwd_kernel<false><<<grid, 256, 0, stream>>>(dqkv, qkv, ld, rstd, rope, rope_T, M, T, H + Hkv, D);
   return cudaGetLastError() == cudaSuccess ? NC_OK : NC_ERR_CUDA;
-}
-
-nc_status attn_bwd_launch(const uint16_t* qkv, int64_t ldqkv, const uint16_t* o, const uint16_t* dO,
-                          const float* lse, float* delta, uint16_t* dqkv, int B, int T, int H, int Hkv, int D,
-                          int window, bool f16, cudaStream_t stream) {
-  if (B == 0 || T == 0) return NC_OK;
-  if (D != 64 && D != 128) return NC_ERR_SHAPE;
-  const int M = B * T;
-  const int64_t warps = (int64_t)M * H;
-  if (f16)
-    bwd::attn_delta_kernel<true><<<(unsigned)((warps + 7) / 8), 256, 0, stream>>>(dO, o, delta, M, H, D);
-  else
-    bwd::attn_delta_kernel<false><<<(unsigned)((warps + 7) / 8), 256, 0, stream>>>(dO, o, delta, M, H, D);
-  if (cudaGetLastError() != cudaSuccess) return NC_ERR_CUDA;
-  const int W = (window <= 0 || window > T) ? T : window;
-  if (D == 128)
-    return f16 ? bwd::attn_bwd_t<128, true>(qkv, ldqkv, dO, lse, delta, dqkv, B, T, H, Hkv, W, stream)
-               : bwd::attn_bwd_t<128, false>(qkv, ldqkv, dO, lse, delta, dqkv, B, T, H, Hkv, W, stream);
-  return f16 ? bwd::attn_bwd_t<64, true>(qkv, ldqkv, dO, lse, delta, dqkv, B, T, H, Hkv, W, stream)
-             : bwd::attn_bwd_t<64, false>(qkv, ldqkv, dO, lse, delta, dqkv, B, T, H, Hkv, W, stream);
 }
 
 nc_status embedding_bwd_launch(const int32_t* tokens, const float* dx, float* dwte, int M, int C, int V,

@@ -113,9 +113,12 @@ nc_status qk_bwd_launch(uint16_t* dqkv, const uint16_t* qkv, int64_t ld, const f
                         int rope_T, int M, int T, int H, int Hkv, int D, bool f16, cudaStream_t stream);
 // dq, dk, dv (into the q / k / v columns of dqkv) from qkv, o, dO [M, H*D], the
 // forward's lse [M, H]; delta [M, H] is scratch.
+// Attention backward (nc_attention_bwd.cu): delta is scratch of B*T*H floats
+// (Delta_i per head, [B][H][T]); dq | dk | dv written in qkv's layout.
 nc_status attn_bwd_launch(const uint16_t* qkv, int64_t ldqkv, const uint16_t* o, const uint16_t* dO,
                           const float* lse, float* delta, uint16_t* dqkv, int B, int T, int H, int Hkv, int D,
-                          int window, bool f16, cudaStream_t stream);
+                          int window, bool f16, cudaStream_t stream, uint32_t* dev_status = nullptr,
+                          uint64_t limit_ns = kWaitLimitNs);
 nc_status embedding_bwd_launch(const int32_t* tokens, const float* dx, float* dwte, int M, int C, int V,
                                const float* alpha, cudaStream_t stream);
 nc_status qkv_grad_scatter_launch(const float* packed, float* gq, float* gk, float* gv, int H, int Hkv, int D, int C,

@@ -457,8 +457,10 @@ nc_status nc_attention_lse(const uint16_t* q, const uint16_t* k, const uint16_t*
 /* Attention backward: qkv [B*T, (H + 2 Hkv) D] packed q | k | v heads (the
  * fused projection's layout), o and dO [B*T, H*D], lse as nc_attention_lse
  * writes it; dqkv gets dq | dk | dv in qkv's layout (dk, dv summed over the
- * query heads of each kv group).  delta [B*T, H] fp32 is scratch.  Warp-level
- * mma.sync tensor cores, fp32 accumulation; no atomics. */
+ * query heads of each kv group).  delta (B*T*H fp32) is scratch.  tcgen05
+ * tensor cores with the scores in tensor memory (one kernel per 128 keys for
+ * dK, dV; one per 128 queries for dQ), fp32 accumulation; no atomics, so the
+ * result is the same run to run. */
 nc_status nc_attention_backward(const uint16_t* qkv, const uint16_t* o, const uint16_t* dO, const float* lse,
                                 float* delta, uint16_t* dqkv, int B, int T, int H, int Hkv, int D, int window,
                                 nc_dtype dtype, void* stream);
