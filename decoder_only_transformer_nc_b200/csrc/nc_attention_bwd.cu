@@ -34,9 +34,6 @@
 #include "nc_internal.h"
 #include "nc_ptx.cuh"
 
-#ifndef ATT_VARIANT
-#define ATT_VARIANT 0
-#endif
 
 namespace nc {
 namespace attn_bwd {
@@ -74,6 +71,23 @@ __device__ __forceinline__ void tmem_st_x16(uint32_t taddr, const uint32_t (&r)[
       "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
       "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
       : "memory");
+}
+
+// 32 lanes x 16 consecutive 32-bit columns into registers.
+__device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32"
+      " {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
+
+// 32 lanes x 8 consecutive 32-bit columns from registers.
+__device__ __forceinline__ void tmem_st_x8(uint32_t taddr, const uint32_t (&r)[8]) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr), "r"(r[0]),
+               "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+               : "memory");
 }
 
 template <int D>
@@ -297,26 +311,22 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         tc_fence_after();
         auto scores = [&](int i, int h) {
           const int st = i % NST;
-#if ATT_VARIANT != 33
 #pragma unroll
           for (int k = 0; k < D / 16; ++k)
             umma_f16(tS + 64 * h, kmajor(sK, 0, k), kmajor(sQt(st), 64 * h, k), IS, k > 0 ? 1u : 0u);
 #pragma unroll
           for (int k = 0; k < D / 16; ++k)
             umma_f16(tP + 64 * h, kmajor(sV, 0, k), kmajor(sDOt(st), 64 * h, k), IS, k > 0 ? 1u : 0u);
-#endif
         };
         // dV += P^T dO and dK += dS^T Q over the 64 queries of half h of tile i
         auto grads = [&](int i, int h) {
           const int st = i % NST;
-#if ATT_VARIANT != 32
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
             const uint32_t acc = (i > 0 || h > 0 || kk > 0) ? 1u : 0u;
             umma_ts(tdV, tS + 64 * h + 8 * kk, mnmajor(sDOt(st), 64 * h + 16 * kk), IG, acc);
             umma_ts(tdK, tP + 64 * h + 8 * kk, mnmajor(sQt(st), 64 * h + 16 * kk), IG, acc);
           }
-#endif
         };
         mma_schedule(bar, n, ctl, scores, grads);
       }
@@ -345,42 +355,40 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tc_fence_after();
       const float* l = sLD + st * 2 * BT;
 #pragma unroll 1
-      for (int c = 0; c < 2; ++c) {
-        uint32_t rs[32], rp[32];
-#if ATT_VARIANT != 34
-        tmem_ld_32x32b_x32(tS + lane_off + 64 * h + 32 * c, rs);
-        tmem_ld_32x32b_x32(tP + lane_off + 64 * h + 32 * c, rp);
+      for (int c = 0; c < 4; ++c) {  // 16 queries at a time
+        const int qb = 64 * h + 16 * c;  // first query of this chunk within the tile
+        uint32_t rs[16], rp[16];
+        tmem_ld_32x32b_x16(tS + lane_off + qb, rs);
+        tmem_ld_32x32b_x16(tP + lane_off + qb, rp);
+        // the chunk's lse and delta, the same for every lane (broadcast reads)
+        float lv[16], dl[16];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float4 a = reinterpret_cast<const float4*>(l + qb)[q];
+          const float4 b = reinterpret_cast<const float4*>(l + BT + qb)[q];
+          lv[4 * q] = a.x, lv[4 * q + 1] = a.y, lv[4 * q + 2] = a.z, lv[4 * q + 3] = a.w;
+          dl[4 * q] = b.x, dl[4 * q + 1] = b.y, dl[4 * q + 2] = b.z, dl[4 * q + 3] = b.w;
+        }
+        const int lo = j - q0 - qb, hi = jhi - q0 - qb;  // visible e: lo <= e <= hi
         tmem_wait_ld();
-#else
+        uint32_t wp[8], wd[8];
 #pragma unroll
-        for (int e = 0; e < 32; ++e) rs[e] = rp[e] = 0u;
-#endif
-        const int qb = 64 * h + 32 * c;              // first query of this chunk within the tile
-        uint32_t wp[16], wd[16];
-#pragma unroll
-        for (int e = 0; e < 32; e += 2) {
+        for (int e = 0; e < 16; e += 2) {
           float p[2], d[2];
 #pragma unroll
           for (int v = 0; v < 2; ++v) {
-            const int qq = qb + e + v, iq = q0 + qq;
-            const bool vis = iq >= j && iq <= jhi;
-#if ATT_VARIANT == 31 || ATT_VARIANT == 34
-            const float pv = vis ? __uint_as_float(rs[e + v]) : 0.0f;
-            p[v] = pv;
-            d[v] = pv;
-#else
+            const bool vis = e + v >= lo && e + v <= hi;
             // exp(s x - lse) in base 2
-            const float pv = vis ? ex2(fmaf(__uint_as_float(rs[e + v]), scale, -l[qq]) * kLog2e) : 0.0f;
+            const float pv = vis ? ex2(fmaf(__uint_as_float(rs[e + v]), scale, -lv[e + v]) * kLog2e) : 0.0f;
             p[v] = pv;
-            d[v] = pv * (__uint_as_float(rp[e + v]) - l[BT + qq]);
-#endif
+            d[v] = pv * (__uint_as_float(rp[e + v]) - dl[e + v]);
           }
           wp[e / 2] = Half<F16>::pack2(p[0], p[1]);
           wd[e / 2] = Half<F16>::pack2(d[0], d[1]);
         }
         // 16-bit P^T and dS^T over the columns this chunk's scores came from
-        tmem_st_x16(tS + lane_off + 64 * h + 16 * c, wp);
-        tmem_st_x16(tP + lane_off + 64 * h + 16 * c, wd);
+        tmem_st_x8(tS + lane_off + 64 * h + 8 * c, wp);
+        tmem_st_x8(tP + lane_off + 64 * h + 8 * c, wd);
       }
       tmem_wait_st();
       tc_fence_before();
