@@ -592,10 +592,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 uint32_t* dev_status, uint64_t limit_ns) {
   constexpr bool A_MN = LAY == GEMM_TN, B_MN = LAY != GEMM_NT;
   static_assert(!(FP8 && LAY != GEMM_NT), "e4m3 operands are K-major");
-  static_assert(!PAIR || (!FP8 && LAY == GEMM_NT), "CTA pairs: 16-bit K-major operands");
-  constexpr uint32_t IDESC = PAIR ? (F16 ? IDESC_PAIR_F16 : IDESC_PAIR_BF16)
-                                  : (FP8 ? IDESC_E4M3 : (F16 ? IDESC_F16 : IDESC_BF16)) | (A_MN ? (1u << 15) : 0u) |
-                                        (B_MN ? (1u << 16) : 0u);
+  static_assert(!PAIR || !FP8, "CTA pairs: 16-bit operands");
+  constexpr uint32_t IDESC = (PAIR ? (F16 ? IDESC_PAIR_F16 : IDESC_PAIR_BF16)
+                                   : (FP8 ? IDESC_E4M3 : (F16 ? IDESC_F16 : IDESC_BF16))) |
+                             (A_MN ? (1u << 15) : 0u) | (B_MN ? (1u << 16) : 0u);
   constexpr int NST = PAIR ? PAIR_STAGES : STAGES;            // ring stages
   constexpr int SBYTES = PAIR ? PAIR_STAGE_BYTES : STAGE_BYTES;  // bytes of one stage in this CTA
   constexpr int TM = PAIR ? 2 * BM : BM;                      // rows of one output tile
@@ -681,8 +681,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             // of both CTAs.
             const uint32_t fb0 = mapa_shared(fb, 0);
             if (rank == 0) mbar_arrive_expect_tx(fb, 2 * SBYTES);
-            tma_load_2d_pair(smem_u32(a_dst), &tmA, kb * KE, m0 + (int)rank * BM, fb0);
-            tma_load_2d_pair(smem_u32(a_dst + A_BYTES), &tmB, kb * KE, n0 + (int)rank * (BN / 2), fb0);
+            const int ma = m0 + (int)rank * BM, nb = n0 + (int)rank * (BN / 2);  // this CTA's rows of A and W
+            if constexpr (A_MN) {
+#pragma unroll
+              for (int i = 0; i < BM / 64; ++i)
+                tma_load_2d_pair(smem_u32(a_dst + i * MN_BOX), &tmA, ma + 64 * i, kb * BK, fb0);
+            } else {
+              tma_load_2d_pair(smem_u32(a_dst), &tmA, kb * KE, ma, fb0);
+            }
+            if constexpr (B_MN) {
+#pragma unroll
+              for (int i = 0; i < BN / 2 / 64; ++i)
+                tma_load_2d_pair(smem_u32(a_dst + A_BYTES + i * MN_BOX), &tmB, nb + 64 * i, kb * BK, fb0);
+            } else {
+              tma_load_2d_pair(smem_u32(a_dst + A_BYTES), &tmB, kb * KE, nb, fb0);
+            }
           } else {
           mbar_arrive_expect_tx(fb, STAGE_BYTES);
           if constexpr (A_MN) {
@@ -1035,16 +1048,16 @@ static cudaError_t dispatch(int epi, const CUtensorMap& ma, const CUtensorMap& m
   }
 }
 
-template <bool F16, int LAY>
+template <bool F16, int LAY, bool PAIR>
 static cudaError_t dispatch_layout(int epi, const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& mc,
                                    int M, int N, int K, const EpiParams& ep, uint32_t* st, uint64_t lim,
                                    cudaStream_t s) {
   switch (epi) {
-    case EPI_STORE_16: return launch_t<EPI_STORE_16, F16, 0, false, LAY>(ma, mb, mc, M, N, K, ep, st, lim, s);
-    case EPI_STORE_F32: return launch_t<EPI_STORE_F32, F16, 0, false, LAY>(ma, mb, mc, M, N, K, ep, st, lim, s);
-    case EPI_RESID_F32: return launch_t<EPI_RESID_F32, F16, 0, false, LAY>(ma, mb, mc, M, N, K, ep, st, lim, s);
+    case EPI_STORE_16: return launch_t<EPI_STORE_16, F16, 0, false, LAY, PAIR>(ma, mb, mc, M, N, K, ep, st, lim, s);
+    case EPI_STORE_F32: return launch_t<EPI_STORE_F32, F16, 0, false, LAY, PAIR>(ma, mb, mc, M, N, K, ep, st, lim, s);
+    case EPI_RESID_F32: return launch_t<EPI_RESID_F32, F16, 0, false, LAY, PAIR>(ma, mb, mc, M, N, K, ep, st, lim, s);
     case EPI_RELU2_BWD_16:
-      return launch_t<EPI_RELU2_BWD_16, F16, 0, false, LAY>(ma, mb, mc, M, N, K, ep, st, lim, s);
+      return launch_t<EPI_RELU2_BWD_16, F16, 0, false, LAY, PAIR>(ma, mb, mc, M, N, K, ep, st, lim, s);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -1176,16 +1189,21 @@ nc_status gemm_launch_layout(const uint16_t* a, int64_t lda, const uint16_t* w, 
     return NC_ERR_INVALID_ARG;
   if (nc_status s = check_epi(epi, K, BK, ep)) return s;
   CUtensorMap ma, mb, mc;
+  // CTA pairs for the weight gradients (GEMM_TN) with more than one 128-row
+  // block; the GEMM_NN products measured 6 % slower per clock on pairs
+  const bool pair = layout == GEMM_TN && M > BM;
   const bool ok_a = layout == GEMM_TN ? make_map_mn(&ma, a, K, M, lda, f16) : make_map(&ma, a, M, K, lda, BM, f16);
   if (!ok_a || !make_map_mn(&mb, w, K, N, ldw, f16)) return NC_ERR_CUDA;
   if (!make_out_map(&mc, epi, M, N, f16, ep)) return NC_ERR_CUDA;
   cudaError_t e;
+#define NC_LAYOUT_CASE(L, P)                                                                           \
+  (f16 ? dispatch_layout<true, L, P>(epi, ma, mb, mc, M, N, K, ep, dev_status, limit_ns, stream)        \
+       : dispatch_layout<false, L, P>(epi, ma, mb, mc, M, N, K, ep, dev_status, limit_ns, stream))
   if (layout == GEMM_NN)
-    e = f16 ? dispatch_layout<true, GEMM_NN>(epi, ma, mb, mc, M, N, K, ep, dev_status, limit_ns, stream)
-            : dispatch_layout<false, GEMM_NN>(epi, ma, mb, mc, M, N, K, ep, dev_status, limit_ns, stream);
+    e = pair ? NC_LAYOUT_CASE(GEMM_NN, true) : NC_LAYOUT_CASE(GEMM_NN, false);
   else
-    e = f16 ? dispatch_layout<true, GEMM_TN>(epi, ma, mb, mc, M, N, K, ep, dev_status, limit_ns, stream)
-            : dispatch_layout<false, GEMM_TN>(epi, ma, mb, mc, M, N, K, ep, dev_status, limit_ns, stream);
+    e = pair ? NC_LAYOUT_CASE(GEMM_TN, true) : NC_LAYOUT_CASE(GEMM_TN, false);
+#undef NC_LAYOUT_CASE
   return e == cudaSuccess ? NC_OK : NC_ERR_CUDA;
 }
 
