@@ -16,21 +16,23 @@
 //              V slot after its P V, so the next K tile loads while the softmax
 //              of the current one runs;
 //   warp 1     owns 512 TMEM columns; one thread issues S = Q K^T (M=128,
-//              N=128 keys) into one of two S buffers, then O += P V (A = P from
-//              shared memory, B = V read MN-major) into one of two O
-//              accumulators (item n uses accumulator n & 1);
+//              N=128 keys) into one of two S buffers, then O += P V (A = P read
+//              from tensor memory, B = V read MN-major from shared memory) into
+//              one of two O accumulators (item n uses accumulator n & 1);
 //   warps 2-9  softmax: each TMEM lane quarter (32 query rows, one per thread)
 //              is served by two warps that own 64 of the tile's 128 keys; they
 //              swap partial row maxima (and, at the end, row sums) through
 //              shared memory.  Mask the window/causal edge only on tiles that
 //              straddle it (one visible-column interval per row), online
-//              softmax in fp32 with exp2, write P (16-bit) to a swizzled
-//              shared-memory tile for the next MMA; O is rescaled in TMEM only
+//              softmax in fp32 with exp2, write P (16-bit, two keys per
+//              column) back over the first half of its own S columns, where
+//              the P V product reads it (the S that next overwrites the buffer
+//              is issued after that product); O is rescaled in TMEM only
 //              when the running row maximum grows by more than 2^8 in the
 //              exponent (P stays <= 256, exact in fp16).  The output O / l of
 //              an item is written after the first tile of the next item has
 //              gone to the MMA warp, so neither the last P V nor the store
-//              stalls the softmax: staged in the freed P tile, TMA-stored.
+//              stalls the softmax: staged in shared memory, TMA-stored.
 // Only key tiles intersecting [q0 - W + 1, q0 + 127] are visited.
 // Every wait is bounded; on timeout the CTA records NC_DEV_TIMEOUT, drains
 // its copies and MMAs, frees its tensor memory and exits.
@@ -345,13 +347,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               break;
             }
             tc_fence_after();
-            const uint32_t pbase = s_p + pb * G::P_BYTES;
             const uint32_t vbase = s_kv + pb * G::KV_STAGE + G::KA * ATOM;
+            // P (16-bit, two keys per column) sits over the first 32 columns of
+            // each key half of S buffer pb
 #pragma unroll
             for (int k = 0; k < BKV / 16; ++k) {
-              const uint64_t adesc = sw128_kmajor_desc(pbase + (k >> 2) * ATOM + (k & 3) * 32);
               const uint64_t bdesc = sw128_desc(vbase + k * 2048, ATOM, 1024);
-              umma_f16(tmem + O_COL + (n & 1) * D, adesc, bdesc, IDESC_PV, (j > 1 || k > 0) ? 1u : 0u);
+              umma_f16_ts(tmem + O_COL + (n & 1) * D, tmem + pb * BKV + 64 * (k >> 2) + 8 * (k & 3), bdesc, IDESC_PV,
+                      (j > 1 || k > 0) ? 1u : 0u);
             }
             umma_commit(smem_u32(&bar->p_free[pb]));
             umma_commit(smem_u32(&bar->v_empty[pb]));
@@ -435,6 +438,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         // TMA write them to out.
         uint8_t* sbase = sm + G::OFF_P + (pd.gl & 1) * G::P_BYTES + half * ATOM;
         uint8_t* srow = sbase + r * 128;
+        if (store_busy & (1u << (pd.gl & 1))) {  // an earlier output store still reads this buffer
+          if (lane == 0) bulk_wait_read0();
+          __syncwarp();
+          store_busy = 0;
+        }
         if (amax && pd.q0 + r < T) {
 #pragma unroll
           for (int c = 0; c < DC / 32; ++c)
@@ -566,18 +574,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
         }
         const float ms = (m_used == -INFINITY) ? 0.0f : m_used * scale_log2;
-        // P buffer sb is free once the P V two tiles back has completed.
-        if (__any_sync(0xffffffffu, !mbar_wait(smem_u32(&bar->p_free[sb]), (use & 1) ^ 1, ctl))) {
-          ok = false;
-          break;
-        }
-        if (store_busy & (1u << sb)) {  // an output store still reads this buffer
-          if (lane == 0) bulk_wait_read0();
-          __syncwarp();
-          store_busy = 0;
-        }
-        uint8_t* prow = sm + G::OFF_P + sb * G::P_BYTES + half * ATOM + r * 128;
+        // P goes back over the first 32 columns of this warp's half of S
+        // buffer sb (two 16-bit values per column), already read into s[]; the
+        // MMA warp issues the S that next overwrites the buffer only after the
+        // P V that reads it.
         float ls8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};  // 8 independent sums
+        uint32_t pk[KC / 2];
 #pragma unroll
         for (int c = 0; c < KC / 8; ++c) {
           float p[8];
@@ -586,15 +588,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             p[e] = ex2f(fmaf(s[c * 8 + e], scale_log2, -ms));
             ls8[e] += p[e];
           }
-          uint4 pk;
-          pk.x = Half<F16>::pack2(p[0], p[1]);
-          pk.y = Half<F16>::pack2(p[2], p[3]);
-          pk.z = Half<F16>::pack2(p[4], p[5]);
-          pk.w = Half<F16>::pack2(p[6], p[7]);
-          *reinterpret_cast<uint4*>(prow + ((c ^ (r & 7)) << 4)) = pk;
+#pragma unroll
+          for (int e = 0; e < 4; ++e) pk[4 * c + e] = Half<F16>::pack2(p[2 * e], p[2 * e + 1]);
         }
         l += ((ls8[0] + ls8[1]) + (ls8[2] + ls8[3])) + ((ls8[4] + ls8[5]) + (ls8[6] + ls8[7]));
-        fence_proxy_async_smem();
+        tmem_st_32x32b_x32(tmem + lane_off + sb * BKV + half * KC, pk);
+        tmem_wait_st();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(&bar->p_full[sb]));

@@ -50,18 +50,6 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
-// D[tmem] (+)= A[tmem] * B[smem desc]^T: the A operand (16-bit, two per column)
-// read from tensor memory.
-__device__ __forceinline__ void umma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
-                                        uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
 // 32 lanes x 16 consecutive 32-bit columns from registers (thread i -> lane
 // base + i).
 __device__ __forceinline__ void tmem_st_x16(uint32_t taddr, const uint32_t (&r)[16]) {
@@ -324,8 +312,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
             const uint32_t acc = (i > 0 || h > 0 || kk > 0) ? 1u : 0u;
-            umma_ts(tdV, tS + 64 * h + 8 * kk, mnmajor(sDOt(st), 64 * h + 16 * kk), IG, acc);
-            umma_ts(tdK, tP + 64 * h + 8 * kk, mnmajor(sQt(st), 64 * h + 16 * kk), IG, acc);
+            umma_f16_ts(tdV, tS + 64 * h + 8 * kk, mnmajor(sDOt(st), 64 * h + 16 * kk), IG, acc);
+            umma_f16_ts(tdK, tP + 64 * h + 8 * kk, mnmajor(sQt(st), 64 * h + 16 * kk), IG, acc);
           }
         };
         mma_schedule(bar, n, ctl, scores, grads);
@@ -520,7 +508,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           const int st = i % NST;
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
-            umma_ts(tdQ, tP + 64 * h + 8 * kk, mnmajor(sKt(st), 64 * h + 16 * kk), IG,
+            umma_f16_ts(tdQ, tP + 64 * h + 8 * kk, mnmajor(sKt(st), 64 * h + 16 * kk), IG,
                     (i > 0 || h > 0 || kk > 0) ? 1u : 0u);
         };
         mma_schedule(bar, n, ctl, scores, grads);
