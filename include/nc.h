@@ -433,9 +433,9 @@ size_t nc_train_workspace_bytes(const nc_config* cfg, int B, int T);
 /* Forward with the activations kept, then the backward: writes *loss (device
  * float, the mean over counted targets) and adds the gradients into *g.
  * cfg->extras and cfg->fp8 must be 0 (NC_ERR_CONFIG).  tokens, targets [B, T]
- * int32 device.  The attention backward runs on the warp-level mma.sync path;
- * the projections' products on the tcgen05 GEMM.  Split-K weight gradients
- * are summed in no fixed order (not bitwise reproducible run to run).
+ * int32 device.  The attention backward and the projections' products run on
+ * tcgen05 tensor cores.  Split-K weight gradients are summed in no fixed order
+ * (not bitwise reproducible run to run).
  * Asynchronous on `stream`. */
 nc_status nc_forward_backward(const nc_config* cfg, const nc_weights* w, const int32_t* tokens,
                               const int32_t* targets, int B, int T, float* loss, const nc_grads* g,
