@@ -71,7 +71,10 @@ class NcWeights(ctypes.Structure):
 
 class NcGrads(ctypes.Structure):
     _fields_ = [("wte", ctypes.c_void_p), ("c_q", _FPP), ("c_k", _FPP), ("c_v", _FPP),
-                ("attn_proj", _FPP), ("c_fc", _FPP), ("mlp_proj", _FPP), ("lm_head", ctypes.c_void_p)]
+                ("attn_proj", _FPP), ("c_fc", _FPP), ("mlp_proj", _FPP), ("lm_head", ctypes.c_void_p),
+                ("smear_gate", ctypes.c_void_p), ("value_embeds", _FPP), ("ve_gates", _FPP),
+                ("resid_lambdas", ctypes.c_void_p), ("x0_lambdas", ctypes.c_void_p),
+                ("backout_lambda", ctypes.c_void_p)]
 
 
 # Further terms of the full nanochat forward (bits of NcConfig.extras).
@@ -528,8 +531,9 @@ def forward_backward(model: Model, tokens, targets, grads: dict | None = None, w
 
     tokens/targets: int32 CUDA tensors [B, T].  ``grads`` (optional) holds fp32
     CUDA tensors in the layout of ``Model.tensors`` ("wte", "lm_head",
-    "layers": [{c_q, ...}]); the gradients are ADDED to them.  Without it,
-    zeroed tensors are made.  Returns (loss: scalar CUDA tensor, grads,
+    "layers": [{c_q, ...}], and "extras" with the same keys as the model's for
+    the terms enabled in cfg.extras); the gradients are ADDED to them.  Without
+    it, zeroed tensors are made.  Returns (loss: scalar CUDA tensor, grads,
     workspace).
     """
     import torch
@@ -543,14 +547,26 @@ def forward_backward(model: Model, tokens, targets, grads: dict | None = None, w
         workspace = torch.empty(need, dtype=torch.uint8, device=dev)
     t = model.tensors
     if grads is None:
-        z = lambda x: torch.zeros_like(x)
+        z = lambda x: None if x is None else torch.zeros_like(x)
         grads = {"wte": z(t["wte"]), "lm_head": z(t["lm_head"]),
                  "layers": [{k: z(lw[k]) for k in ("c_q", "c_k", "c_v", "attn_proj", "c_fc", "mlp_proj")}
                             for lw in t["layers"]]}
+        tex = t.get("extras") or {}
+        if tex:
+            grads["extras"] = {k: ([z(x) for x in v] if isinstance(v, list) else z(v)) for k, v in tex.items()}
     L = cfg.n_layer
     arrs = [(ctypes.c_void_p * L)(*[grads["layers"][l][n].data_ptr() for l in range(L)])
             for n in ("c_q", "c_k", "c_v", "attn_proj", "c_fc", "mlp_proj")]
-    g = NcGrads(grads["wte"].data_ptr(), *[ctypes.cast(a, _FPP) for a in arrs], grads["lm_head"].data_ptr())
+    gex = grads.get("extras") or {}
+    p = lambda x: None if x is None else x.data_ptr()
+    per_layer = {}
+    for name in ("value_embeds", "ve_gates"):
+        lst = gex.get(name)
+        per_layer[name] = None if lst is None else (ctypes.c_void_p * L)(*[p(x) for x in lst])
+    fpp = lambda a: None if a is None else ctypes.cast(a, _FPP)
+    g = NcGrads(grads["wte"].data_ptr(), *[ctypes.cast(a, _FPP) for a in arrs], grads["lm_head"].data_ptr(),
+                p(gex.get("smear_gate")), fpp(per_layer["value_embeds"]), fpp(per_layer["ve_gates"]),
+                p(gex.get("resid_lambdas")), p(gex.get("x0_lambdas")), p(gex.get("backout_lambda")))
     if loss is None:
         loss = torch.empty((), dtype=torch.float32, device=dev)
     _check(lib().nc_forward_backward_traced(ctypes.byref(cfg), ctypes.byref(model.weights), _ptr(tokens),

@@ -629,20 +629,8 @@ static nc_status check_weights(const nc_config* cfg, const nc_weights* w) {
   return NC_OK;
 }
 
-static nc_status forward_impl(const nc_config* cfg, const nc_weights* w, const int32_t* tokens,
-                              const int32_t* targets, int B, int T, float* logits, float* token_loss,
-                              float* loss, void* workspace, size_t ws_bytes, void* stream, nc_trace* trace,
-                              const SessionRef* sess) {
-  if (!cfg || !w || !tokens || !workspace) return NC_ERR_INVALID_ARG;
-  if (!config_ok(cfg)) return NC_ERR_CONFIG;
-  if (B < 1 || T < 1 || T > cfg->seq_len) return NC_ERR_SHAPE;
-  if ((token_loss || loss) && !targets) return NC_ERR_INVALID_ARG;
-  if ((int64_t)B * T > (int64_t)1 << 30) return NC_ERR_SHAPE;
-  const WsLayout L = ws_layout(cfg, B, T, sess == nullptr);
-  if (ws_bytes < L.total) return NC_ERR_WORKSPACE;
-  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return NC_ERR_ALIGNMENT;
-  if (logits && !aligned16(logits)) return NC_ERR_ALIGNMENT;
-  if (nc_status s = check_weights(cfg, w)) return s;
+// The parameters of the further forward terms that cfg->extras switches on.
+static nc_status check_extras(const nc_config* cfg, const nc_weights* w) {
   const uint32_t ex = cfg->extras;
   if (ex & NC_EXTRA_SMEAR) {
     if (!w->smear_gate) return NC_ERR_INVALID_ARG;
@@ -658,6 +646,25 @@ static nc_status forward_impl(const nc_config* cfg, const nc_weights* w, const i
   }
   if ((ex & NC_EXTRA_RESID_LAMBDAS) && (!w->resid_lambdas || !w->x0_lambdas)) return NC_ERR_INVALID_ARG;
   if ((ex & NC_EXTRA_BACKOUT) && !w->backout_lambda) return NC_ERR_INVALID_ARG;
+  return NC_OK;
+}
+
+static nc_status forward_impl(const nc_config* cfg, const nc_weights* w, const int32_t* tokens,
+                              const int32_t* targets, int B, int T, float* logits, float* token_loss,
+                              float* loss, void* workspace, size_t ws_bytes, void* stream, nc_trace* trace,
+                              const SessionRef* sess) {
+  if (!cfg || !w || !tokens || !workspace) return NC_ERR_INVALID_ARG;
+  if (!config_ok(cfg)) return NC_ERR_CONFIG;
+  if (B < 1 || T < 1 || T > cfg->seq_len) return NC_ERR_SHAPE;
+  if ((token_loss || loss) && !targets) return NC_ERR_INVALID_ARG;
+  if ((int64_t)B * T > (int64_t)1 << 30) return NC_ERR_SHAPE;
+  const WsLayout L = ws_layout(cfg, B, T, sess == nullptr);
+  if (ws_bytes < L.total) return NC_ERR_WORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return NC_ERR_ALIGNMENT;
+  if (logits && !aligned16(logits)) return NC_ERR_ALIGNMENT;
+  if (nc_status s = check_weights(cfg, w)) return s;
+  if (nc_status s = check_extras(cfg, w)) return s;
+  const uint32_t ex = cfg->extras;
   if (trace) {
     const int need = forward_launch_count(cfg, targets != nullptr, loss != nullptr, logits != nullptr);
     trace->count = need;
@@ -1059,7 +1066,7 @@ namespace {
 // stream.  Offsets are 256-byte aligned.
 struct TrainLayout {
   size_t status, rope, wqkv, wo, wfc, wmp, wlm, xs, qkv, rstd, o, lse, h, af, a, part, tgt, tl, scal, dz, dx, dx16,
-      dy, du, dO, dqkv, delta, dwqkv, total;
+      dy, du, dO, dqkv, delta, dwqkv, x0, xpre, dx0, dxf, sdz, total;
   size_t wqkv_elems, wo_elems, wfc_elems, wmp_elems;
 };
 
@@ -1106,6 +1113,15 @@ TrainLayout train_layout(const nc_config* c, int B, int T) {
   L.dqkv = take(M * nqkv * 2);
   L.delta = take(M * H * 4);
   L.dwqkv = take(nqkv * C * 4);
+  // further forward terms: x0, each block's stream before the lambda mix and
+  // the gradient collected for x0 (resid lambdas); the final-norm gradient
+  // (backout); the smear gates' gradient per token
+  const bool lam = c->extras & NC_EXTRA_RESID_LAMBDAS;
+  L.x0 = lam ? take(M * C * 4) : 0;
+  L.xpre = lam ? take(NL * M * C * 4) : 0;
+  L.dx0 = lam ? take(M * C * 4) : 0;
+  L.dxf = (c->extras & NC_EXTRA_BACKOUT) ? take(M * C * 4) : 0;
+  L.sdz = (c->extras & NC_EXTRA_SMEAR) ? take(M * 4) : 0;
   L.total = off;
   return L;
 }
@@ -1115,7 +1131,7 @@ TrainLayout train_layout(const nc_config* c, int B, int T) {
 extern "C" {
 
 size_t nc_train_workspace_bytes(const nc_config* cfg, int B, int T) {
-  if (!config_ok(cfg) || cfg->extras != 0 || cfg->fp8 != 0 || B < 1 || T < 1 || T > cfg->seq_len) return 0;
+  if (!config_ok(cfg) || cfg->fp8 != 0 || B < 1 || T < 1 || T > cfg->seq_len) return 0;
   return train_layout(cfg, B, T).total;
 }
 
@@ -1129,14 +1145,26 @@ nc_status nc_forward_backward_traced(const nc_config* cfg, const nc_weights* w, 
                                      const int32_t* targets, int B, int T, float* loss, const nc_grads* g,
                                      void* workspace, size_t ws_bytes, void* stream, nc_trace* trace) {
   if (!cfg || !w || !tokens || !targets || !loss || !g || !workspace) return NC_ERR_INVALID_ARG;
-  if (!config_ok(cfg) || cfg->extras != 0 || cfg->fp8 != 0) return NC_ERR_CONFIG;
+  if (!config_ok(cfg) || cfg->fp8 != 0) return NC_ERR_CONFIG;
   if (B < 1 || T < 1 || T > cfg->seq_len || (int64_t)B * T > ((int64_t)1 << 30)) return NC_ERR_SHAPE;
   const TrainLayout L = train_layout(cfg, B, T);
   if (ws_bytes < L.total) return NC_ERR_WORKSPACE;
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return NC_ERR_ALIGNMENT;
   if (nc_status s = check_weights(cfg, w)) return s;
+  if (nc_status s = check_extras(cfg, w)) return s;
   if (!g->wte || !g->lm_head || !g->c_q || !g->c_k || !g->c_v || !g->attn_proj || !g->c_fc || !g->mlp_proj)
     return NC_ERR_INVALID_ARG;
+  {  // gradients of the further terms
+    const uint32_t ex = cfg->extras;
+    if ((ex & NC_EXTRA_SMEAR) && !g->smear_gate) return NC_ERR_INVALID_ARG;
+    if ((ex & NC_EXTRA_RESID_LAMBDAS) && (!g->resid_lambdas || !g->x0_lambdas)) return NC_ERR_INVALID_ARG;
+    if ((ex & NC_EXTRA_BACKOUT) && !g->backout_lambda) return NC_ERR_INVALID_ARG;
+    if (ex & NC_EXTRA_VALUE_EMBED) {
+      if (!g->value_embeds || !g->ve_gates) return NC_ERR_INVALID_ARG;
+      for (int l = 0; l < cfg->n_layer; ++l)
+        if (nc_layer_value_embed(cfg, l) == 1 && (!g->value_embeds[l] || !g->ve_gates[l])) return NC_ERR_INVALID_ARG;
+    }
+  }
   if (!aligned16(g->wte) || !aligned16(g->lm_head) || !aligned16(loss)) return NC_ERR_ALIGNMENT;
   for (int l = 0; l < cfg->n_layer; ++l) {
     const float* ps[6] = {g->c_q[l], g->c_k[l], g->c_v[l], g->attn_proj[l], g->c_fc[l], g->mlp_proj[l]};
@@ -1191,6 +1219,13 @@ nc_status nc_forward_backward_traced(const nc_config* cfg, const nc_weights* w, 
   uint16_t* dqkv = reinterpret_cast<uint16_t*>(ws + L.dqkv);
   float* delta = reinterpret_cast<float*>(ws + L.delta);
   float* dwqkv = reinterpret_cast<float*>(ws + L.dwqkv);
+  const uint32_t ex = cfg->extras;
+  float* x0 = (ex & NC_EXTRA_RESID_LAMBDAS) ? reinterpret_cast<float*>(ws + L.x0) : nullptr;
+  auto xpre_l = [&](int l) { return reinterpret_cast<float*>(ws + L.xpre) + (size_t)l * MC; };
+  float* dx0 = x0 ? reinterpret_cast<float*>(ws + L.dx0) : nullptr;
+  float* dxf = (ex & NC_EXTRA_BACKOUT) ? reinterpret_cast<float*>(ws + L.dxf) : nullptr;
+  const int mid = NL / 2;  // backout: the stream entering block `mid`, before its lambda mix
+  const float* x_back = dxf ? (x0 ? xpre_l(mid) : xs + (size_t)(2 * mid) * MC) : nullptr;
 
   nc_status s = NC_OK;
 #define NC_RUN(kind, call)                   \
@@ -1208,12 +1243,20 @@ nc_status nc_forward_backward_traced(const nc_config* cfg, const nc_weights* w, 
   NC_RUN(NC_K_ROPE_TABLE, rope_table_launch(rope, T, D, cfg->rope_base, st, rope_pairs_of(rope, T, D)));
   NC_RUN(NC_K_CAST, launch_weight_cast(cfg, w, wqkv, wo, wfc, wmp, wlm, L.wqkv_elems, L.wo_elems, L.wfc_elems, L.wmp_elems,
                             f16, st));
-  NC_RUN(NC_K_EMBEDDING, embedding_launch(tokens, w->wte, xs, M, C, V, status, st));
+  if (ex & (NC_EXTRA_SMEAR | NC_EXTRA_RESID_LAMBDAS))
+    NC_RUN(NC_K_EMBEDDING, embedding_extra_launch(tokens, w->wte, (ex & NC_EXTRA_SMEAR) ? w->smear_gate : nullptr,
+                                                  xs, x0, M, C, V, T, status, st));
+  else
+    NC_RUN(NC_K_EMBEDDING, embedding_launch(tokens, w->wte, xs, M, C, V, status, st));
   for (int l = 0; l < NL; ++l) {
     float* xin = xs + (size_t)(2 * l) * MC;
     float* xmid = xin + MC;
     float* xnext = xmid + MC;
-    NC_RUN(NC_K_RMSNORM, rmsnorm_launch(xin, a, M, C, eps, f16, st));
+    if (x0)  // x = resid_lambda x + x0_lambda x0 in place, the stream before it kept
+      NC_RUN(NC_K_RMSNORM, rmsnorm_mix_launch(xin, x0, w->resid_lambdas + l, w->x0_lambdas + l, xpre_l(l), nullptr,
+                                              nullptr, true, a, M, C, eps, f16, st));
+    else
+      NC_RUN(NC_K_RMSNORM, rmsnorm_launch(xin, a, M, C, eps, f16, st));
     EpiParams eq{};
     eq.out = qkv_l(l);
     eq.ldo = NQKV;
@@ -1226,6 +1269,13 @@ nc_status nc_forward_backward_traced(const nc_config* cfg, const nc_weights* w, 
     eq.rope_T = T;
     eq.rope_pairs = rope_pairs_of(rope, T, D);
     eq.rstd_out = rstd_l(l);
+    const bool ve_on = (ex & NC_EXTRA_VALUE_EMBED) && nc_layer_value_embed(cfg, l) == 1;
+    if (ve_on) {  // v + gate * ve[token] in the epilogue
+      eq.tokens = tokens;
+      eq.ve = w->value_embeds[l];
+      eq.ve_gate = w->ve_gates[l];
+      eq.V = V;
+    }
     NC_RUN(NC_K_GEMM_QKV, gemm_launch(a, C, wqkv + l * L.wqkv_elems, C, M, NQKV, C, EPI_QKV_ROPE_IL, f16, eq, status, st));
     uint16_t* q = qkv_l(l);
     NC_RUN(NC_K_ATTENTION, attention_launch(q, q + HD, q + (H + Hkv) * D, o_l(l), B, T, H, Hkv, D, nc_layer_window(cfg, l), NQKV,
@@ -1246,7 +1296,11 @@ nc_status nc_forward_backward_traced(const nc_config* cfg, const nc_weights* w, 
                        st));
   }
   float* xf = xs + (size_t)(2 * NL) * MC;
-  NC_RUN(NC_K_RMSNORM, rmsnorm_launch(xf, af, M, C, eps, f16, st));
+  if (x_back)  // x -= backout_lambda x_back in place
+    NC_RUN(NC_K_RMSNORM, rmsnorm_mix_launch(xf, nullptr, nullptr, nullptr, nullptr, x_back, w->backout_lambda, true,
+                                            af, M, C, eps, f16, st));
+  else
+    NC_RUN(NC_K_RMSNORM, rmsnorm_launch(xf, af, M, C, eps, f16, st));
   {
     EpiParams ep{};
     ep.ldo = V;
@@ -1296,6 +1350,17 @@ nc_status nc_forward_backward_traced(const nc_config* cfg, const nc_weights* w, 
   NC_RUN(NC_K_GEMM_WGRAD, wgrad(dz, V, af, C, V, C, g->lm_head, C));
   NC_RUN(NC_K_GEMM_DGRAD, dgrad(dz, V, wlm, C, EPI_STORE_F32, dy));
   NC_RUN(NC_K_NORM_BWD, rmsnorm_bwd_launch(xf, dy, dx, dx16, M, C, eps, false, f16, st));
+  // The further terms' backward launches are not recorded in the trace.
+#define NC_TRY_EX(call)                     \
+  do {                                      \
+    s = (call);                             \
+    if (s != NC_OK) return s;               \
+  } while (0)
+  if (x_back) {  // x_final = x_L - lambda x_back: dlambda = -sum dx . x_back; keep dx_final
+    NC_TRY_EX(dots_launch(dx, x_back, nullptr, (int64_t)MC, inv, -1.0f, g->backout_lambda, nullptr, st));
+    NC_TRY_EX(cudaMemcpyAsync(dxf, dx, MC * 4, cudaMemcpyDeviceToDevice, st) == cudaSuccess ? NC_OK : NC_ERR_CUDA);
+  }
+  if (dx0) NC_TRY_EX(cudaMemsetAsync(dx0, 0, MC * 4, st) == cudaSuccess ? NC_OK : NC_ERR_CUDA);
   for (int l = NL - 1; l >= 0; --l) {
     float* xin = xs + (size_t)(2 * l) * MC;
     float* xmid = xin + MC;
@@ -1312,6 +1377,9 @@ nc_status nc_forward_backward_traced(const nc_config* cfg, const nc_weights* w, 
     NC_RUN(NC_K_ATTN_BWD, attn_bwd_launch(qkv_l(l), NQKV, o_l(l), dO, lse_l(l), delta, dqkv, B, T, H, Hkv, D,
                            nc_layer_window(cfg, l), f16, st, status));
     NC_RUN(NC_K_QK_BWD, qk_bwd_launch(dqkv, qkv_l(l), NQKV, rstd_l(l), rope, T, M, T, H, Hkv, D, f16, st));
+    if ((ex & NC_EXTRA_VALUE_EMBED) && nc_layer_value_embed(cfg, l) == 1)  // v + gate ve[token]
+      NC_TRY_EX(ve_bwd_launch(dqkv, NQKV, tokens, w->value_embeds[l], w->ve_gates[l], g->value_embeds[l],
+                              g->ve_gates[l], M, H, Hkv, D, V, inv, f16, st));
     NC_RUN(NC_K_RMSNORM, rmsnorm_launch(xin, a, M, C, eps, f16, st));
     NC_RUN(NC_K_GEMM_WGRAD, cudaMemsetAsync(dwqkv, 0, (size_t)NQKV * C * 4, st) == cudaSuccess
                                 ? wgrad(dqkv, NQKV, a, C, NQKV, C, dwqkv, C)
@@ -1319,8 +1387,24 @@ nc_status nc_forward_backward_traced(const nc_config* cfg, const nc_weights* w, 
     NC_RUN(NC_K_EMB_BWD, qkv_grad_scatter_launch(dwqkv, g->c_q[l], g->c_k[l], g->c_v[l], H, Hkv, D, C, 1.0f, st));
     NC_RUN(NC_K_GEMM_DGRAD, dgrad(dqkv, NQKV, wqkv + l * L.wqkv_elems, C, EPI_STORE_F32, dy));
     NC_RUN(NC_K_NORM_BWD, rmsnorm_bwd_launch(xin, dy, dx, dx16, M, C, eps, true, f16, st));
+    // dx: of the block's (mixed) input
+    if (x0)  // x_in = resid_lambda x_pre + x0_lambda x0
+      NC_TRY_EX(dots_launch(dx, xpre_l(l), x0, (int64_t)MC, inv, 1.0f, g->resid_lambdas + l, g->x0_lambdas + l, st));
+    const bool back_here = x_back && l == mid;  // x_pre of block `mid` also enters the final norm
+    if (x0 || back_here)
+      NC_TRY_EX(mix_bwd_launch(dx, dx0, back_here ? dxf : nullptr, nullptr, x0 ? w->resid_lambdas + l : nullptr,
+                               x0 ? w->x0_lambdas + l : nullptr, back_here ? w->backout_lambda : nullptr, dx16,
+                               (int64_t)MC, f16, st));
   }
-  NC_RUN(NC_K_EMB_BWD, embedding_bwd_launch(tokens, dx, g->wte, M, C, V, inv, st));
+  if (dx0) NC_TRY_EX(mix_bwd_launch(dx, nullptr, nullptr, dx0, nullptr, nullptr, nullptr, nullptr, (int64_t)MC, f16, st));
+  const float* demb = dx;
+  if (ex & NC_EXTRA_SMEAR) {  // x_t = e_t + sigmoid(e_t . w) e_{t-1}
+    NC_TRY_EX(smear_bwd_launch(tokens, w->wte, w->smear_gate, dx, dy, reinterpret_cast<float*>(ws + L.sdz),
+                               g->smear_gate, M, T, C, V, inv, st));
+    demb = dy;
+  }
+  NC_RUN(NC_K_EMB_BWD, embedding_bwd_launch(tokens, demb, g->wte, M, C, V, inv, st));
+#undef NC_TRY_EX
 #undef NC_RUN
   return NC_OK;
 }

@@ -119,6 +119,17 @@ nc_status attn_bwd_launch(const uint16_t* qkv, int64_t ldqkv, const uint16_t* o,
                           const float* lse, float* delta, uint16_t* dqkv, int B, int T, int H, int Hkv, int D,
                           int window, bool f16, cudaStream_t stream, uint32_t* dev_status = nullptr,
                           uint64_t limit_ns = kWaitLimitNs);
+// Backward of the further forward terms (nc_backward.cu).
+nc_status dots_launch(const float* a, const float* b0, const float* b1, int64_t n, const float* inv, float sign,
+                      float* out0, float* out1, cudaStream_t stream);
+nc_status mix_bwd_launch(float* dx, float* acc0, const float* sub, const float* add, const float* lam_r,
+                         const float* lam_0, const float* lam_sub, uint16_t* dx16, int64_t n, bool f16,
+                         cudaStream_t stream);
+nc_status ve_bwd_launch(const uint16_t* dqkv, int64_t ld, const int32_t* tokens, const float* table, const float* gate,
+                        float* dtable, float* dgate, int M, int H, int Hkv, int D, int V, const float* inv, bool f16,
+                        cudaStream_t stream);
+nc_status smear_bwd_launch(const int32_t* tokens, const float* wte, const float* w, const float* dx, float* de,
+                           float* dz, float* dw, int M, int T, int C, int V, const float* inv, cudaStream_t stream);
 nc_status embedding_bwd_launch(const int32_t* tokens, const float* dx, float* dwte, int M, int C, int V,
                                const float* alpha, cudaStream_t stream);
 nc_status qkv_grad_scatter_launch(const float* packed, float* gq, float* gk, float* gv, int H, int Hkv, int D, int C,

@@ -421,18 +421,33 @@ typedef struct {
   float* const* c_fc;         /* n_layer x [4C, C]    */
   float* const* mlp_proj;     /* n_layer x [C, 4C]    */
   float* lm_head;             /* [V, C]        */
+  /* Written only for the terms enabled in nc_config.extras (may be NULL
+   * otherwise), shapes as in nc_weights; summed over tokens with atomics (not
+   * bitwise reproducible run to run). */
+  float* smear_gate;          /* [C]                NC_EXTRA_SMEAR         */
+  float* const* value_embeds; /* n_layer x [V, Hkv*D] NC_EXTRA_VALUE_EMBED;  */
+  float* const* ve_gates;     /* n_layer x [Hkv]: entries of layers without a
+                                 value embedding are not written (may be NULL) */
+  float* resid_lambdas;       /* [n_layer]          NC_EXTRA_RESID_LAMBDAS */
+  float* x0_lambdas;          /* [n_layer]          NC_EXTRA_RESID_LAMBDAS */
+  float* backout_lambda;      /* [1]                NC_EXTRA_BACKOUT       */
 } nc_grads;
 
 /* Workspace bytes of nc_forward_backward for a [B, T] batch (0 on bad input):
  * the 16-bit weights, per layer the activations the backward reads (residual
  * stream at the block's input and after attention, q|k|v, the QK-norm factors,
  * the attention output and its log-sum-exp, the MLP hidden activations), the
- * 16-bit gradient of the logits [B*T, V] and the backward's scratch.  Host only. */
+ * 16-bit gradient of the logits [B*T, V] and the backward's scratch; with
+ * NC_EXTRA_RESID_LAMBDAS also x0, each block's stream before the mix and a
+ * gradient accumulator for x0 (n_layer + 2 fp32 [B*T, C] arrays), with
+ * NC_EXTRA_BACKOUT one more such array.  Host only. */
 size_t nc_train_workspace_bytes(const nc_config* cfg, int B, int T);
 
 /* Forward with the activations kept, then the backward: writes *loss (device
  * float, the mean over counted targets) and adds the gradients into *g.
- * cfg->extras and cfg->fp8 must be 0 (NC_ERR_CONFIG).  tokens, targets [B, T]
+ * cfg->fp8 must be 0 (NC_ERR_CONFIG); the further terms of cfg->extras are
+ * supported, their parameters' gradients going to the matching members of *g
+ * ("Nanochat与nanoGPT对比" §1).  tokens, targets [B, T]
  * int32 device.  The attention backward and the projections' products run on
  * tcgen05 tensor cores.  Split-K weight gradients are summed in no fixed order
  * (not bitwise reproducible run to run).

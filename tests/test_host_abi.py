@@ -292,10 +292,19 @@ def test_backward_host_rules(nclib):
     # at least the saved residual streams (2L + 1 fp32 [M, C]) and the logit gradient [M, V] (16-bit)
     assert n >= (2 * cfg.n_layer + 1) * M * C * 4 + M * V * 2
     assert nclib.train_workspace_bytes(cfg, 2, 300) == 0  # T > seq_len
-    for field, val in (("extras", nclib.EXTRA_SMEAR), ("fp8", nclib.FP8_BLOCK)):
+    c = nclib.NcConfig.from_buffer_copy(cfg)
+    c.fp8 = nclib.FP8_BLOCK
+    assert nclib.train_workspace_bytes(c, 2, 100) == 0  # e4m3 training is not supported
+    # the further terms add x0, the pre-mix streams and the x0 gradient
+    # (lambdas: n_layer + 2 fp32 [M, C]), the final-norm gradient (backout) and
+    # the smear gates' per-token gradient
+    for bits, extra in ((nclib.EXTRA_SMEAR, M * 4), (nclib.EXTRA_VALUE_EMBED, 0),
+                        (nclib.EXTRA_RESID_LAMBDAS, (cfg.n_layer + 2) * M * C * 4),
+                        (nclib.EXTRA_BACKOUT, M * C * 4)):
         c = nclib.NcConfig.from_buffer_copy(cfg)
-        setattr(c, field, val)
-        assert nclib.train_workspace_bytes(c, 2, 100) == 0
+        c.extras = bits
+        got = nclib.train_workspace_bytes(c, 2, 100)
+        assert extra <= got - n <= extra + 3 * 256, (bits, got - n, extra)
     fw = _FakeWeights(nclib, 2)
     arr = (ctypes.c_void_p * 2)(1 << 40, (1 << 40) + 4096)
     FPP = ctypes.POINTER(ctypes.c_void_p)
