@@ -155,10 +155,11 @@ WsLayout ws_layout(const nc_config* c, int B, int T, bool own_weights = true) {
 }
 
 // KV-cache session: the 16-bit weights and the RoPE table (cast and built once
-// by nc_prefill), the cache of every layer, and the scratch of one decode step
-// (B rows).  Offsets are 256-byte aligned.
+// by nc_prefill), the cache of every layer, the token of every position (smear
+// reads the previous one), and the scratch of one decode step (B rows; x0 and
+// x_mid for the residual lambdas and backout).  Offsets are 256-byte aligned.
 struct SessionLayout {
-  size_t status, rope, wqkv, wo, wfc, wmp, wlm, cache, x, a, qkv, o, h, part, acc, total;
+  size_t status, rope, wqkv, wo, wfc, wmp, wlm, cache, hist, x, a, qkv, o, h, part, acc, x0, xmid, total;
   size_t wqkv_elems, wo_elems, wfc_elems, wmp_elems, cache_layer_elems;
 };
 
@@ -185,6 +186,7 @@ SessionLayout session_layout(const nc_config* c, int B, int T_max) {
   L.wmp = take(c->n_layer * L.wmp_elems * 2);
   L.wlm = take(V * C * 2);
   L.cache = take(c->n_layer * L.cache_layer_elems * 2);
+  L.hist = (c->extras & NC_EXTRA_SMEAR) ? take(Bs * T_max * 4) : 0;
   L.x = take(Bs * C * 4);
   L.a = take(Bs * C * 2);
   L.qkv = take(Bs * nqkv * 2);
@@ -192,6 +194,8 @@ SessionLayout session_layout(const nc_config* c, int B, int T_max) {
   L.h = take(Bs * 4 * C * 2);
   L.part = take(Bs * H * (size_t)decode_attention_max_splits() * (2 + D) * 4);
   L.acc = take(Bs * (nqkv > 4 * C ? nqkv : 4 * C) * 4);  // fp32 split-K sums of QKV, then c_fc
+  L.x0 = (c->extras & NC_EXTRA_RESID_LAMBDAS) ? take(Bs * C * 4) : 0;
+  L.xmid = (c->extras & NC_EXTRA_BACKOUT) ? take(Bs * C * 4) : 0;
   L.total = off;
   return L;
 }
@@ -913,7 +917,7 @@ nc_status nc_prefill(const nc_config* cfg, const nc_weights* w, const int32_t* t
                      float* logits, void* session, size_t session_bytes, int T_max, void* workspace,
                      size_t ws_bytes, void* stream) {
   if (!cfg || !w || !session) return NC_ERR_INVALID_ARG;
-  if (!config_ok(cfg) || cfg->extras != 0 || cfg->fp8 != 0) return NC_ERR_CONFIG;
+  if (!config_ok(cfg) || cfg->fp8 != 0) return NC_ERR_CONFIG;
   if (T_max < 1 || T_max > cfg->seq_len || T < 0 || T > T_max || B < 1) return NC_ERR_SHAPE;
   const SessionLayout SL = session_layout(cfg, B, T_max);
   if (session_bytes < SL.total) return NC_ERR_WORKSPACE;
@@ -934,8 +938,14 @@ nc_status nc_prefill(const nc_config* cfg, const nc_weights* w, const int32_t* t
                               SL.wqkv_elems, SL.wo_elems, SL.wfc_elems, SL.wmp_elems, cfg->act_dtype == NC_F16, st);
   }
   const SessionRef sess{static_cast<uint8_t*>(session), T_max};
-  return forward_impl(cfg, w, tokens, nullptr, B, T, logits, nullptr, nullptr, workspace, ws_bytes, stream,
-                      nullptr, &sess);
+  if (nc_status s = forward_impl(cfg, w, tokens, nullptr, B, T, logits, nullptr, nullptr, workspace, ws_bytes,
+                                 stream, nullptr, &sess))
+    return s;
+  if (cfg->extras & NC_EXTRA_SMEAR)  // the prompt's tokens, for the smear of the first decode step
+    if (cudaMemcpy2DAsync(static_cast<uint8_t*>(session) + SL.hist, (size_t)T_max * 4, tokens, (size_t)T * 4,
+                          (size_t)T * 4, B, cudaMemcpyDeviceToDevice, S(stream)) != cudaSuccess)
+      return NC_ERR_CUDA;
+  return NC_OK;
 }
 
 // K slices for a residual-add GEMM with few output tiles: about one tile per SM.
@@ -954,7 +964,7 @@ static nc_status decode_impl(const nc_config* cfg, const nc_weights* w, const in
                              int32_t* pos_dev, float* logits, void* session, size_t session_bytes, int T_max,
                              void* stream) {
   if (!cfg || !w || !w->wte || !tokens || !logits || !session) return NC_ERR_INVALID_ARG;
-  if (!config_ok(cfg) || cfg->extras != 0 || cfg->fp8 != 0) return NC_ERR_CONFIG;
+  if (!config_ok(cfg) || cfg->fp8 != 0) return NC_ERR_CONFIG;
   if (T_max < 1 || T_max > cfg->seq_len || B < 1 || (!pos_dev && (pos < 0 || pos >= T_max))) return NC_ERR_SHAPE;
   if (pos_dev && T_max > decode_attention_max_splits() * 64) return NC_ERR_SHAPE;
   if (pos_dev && !aligned16(pos_dev)) return NC_ERR_ALIGNMENT;
@@ -964,6 +974,7 @@ static nc_status decode_impl(const nc_config* cfg, const nc_weights* w, const in
   if (!aligned16(w->wte) || !aligned16(logits)) return NC_ERR_ALIGNMENT;
   if (cfg->n_head / cfg->n_kv_head > 8 || (cfg->n_head / cfg->n_kv_head) & (cfg->n_head / cfg->n_kv_head - 1))
     return NC_ERR_SHAPE;  // decode attention groups of 1, 2, 4 or 8 query heads
+  if (nc_status s = check_extras(cfg, w)) return s;
   if (nc_status s = device_ok()) return s;
 
   cudaStream_t st = S(stream);
@@ -983,6 +994,11 @@ static nc_status decode_impl(const nc_config* cfg, const nc_weights* w, const in
   uint16_t* h = reinterpret_cast<uint16_t*>(base + SL.h);
   float* part = reinterpret_cast<float*>(base + SL.part);
   float* acc = reinterpret_cast<float*>(base + SL.acc);
+  const uint32_t ex = cfg->extras;
+  int32_t* hist = (ex & NC_EXTRA_SMEAR) ? reinterpret_cast<int32_t*>(base + SL.hist) : nullptr;
+  float* x0 = (ex & NC_EXTRA_RESID_LAMBDAS) ? reinterpret_cast<float*>(base + SL.x0) : nullptr;
+  float* xmid = (ex & NC_EXTRA_BACKOUT) ? reinterpret_cast<float*>(base + SL.xmid) : nullptr;
+  const int mid = cfg->n_layer / 2;  // backout: the stream after the first n_layer / 2 blocks
   const int C = cfg->d_model, D = cfg->head_dim, H = cfg->n_head, Hkv = cfg->n_kv_head, V = cfg->vocab;
   const int NQKV = (H + 2 * Hkv) * D;
   const bool f16 = cfg->act_dtype == NC_F16;
@@ -994,7 +1010,11 @@ static nc_status decode_impl(const nc_config* cfg, const nc_weights* w, const in
     if (s != NC_OK) return s; \
   } while (0)
   if (cudaMemsetAsync(status, 0, 256, st) != cudaSuccess) return NC_ERR_CUDA;
-  NC_TRY(embedding_launch(tokens, w->wte, x, B, C, V, status, st));
+  if (ex & (NC_EXTRA_SMEAR | NC_EXTRA_RESID_LAMBDAS))
+    NC_TRY(decode_embedding_launch(tokens, hist, w->wte, hist ? w->smear_gate : nullptr, x, x0, B, C, V, T_max, pos,
+                                   pos_dev, status, st));
+  else
+    NC_TRY(embedding_launch(tokens, w->wte, x, B, C, V, status, st));
   // Few rows (B): every projection splits K.  The residual adds land in x
   // directly; QKV and c_fc sum into an fp32 scratch that a small kernel finishes
   // (RoPE + QK-norm + cache write, or ReLU^2).  Up to 32 rows the projections
@@ -1012,11 +1032,20 @@ static nc_status decode_impl(const nc_config* cfg, const nc_weights* w, const in
     return gemm_launch(in, K, wt, K, B, N, K, EPI_RESID_F32, f16, e, status, st);
   };
   for (int l = 0; l < cfg->n_layer; ++l) {
-    NC_TRY(rmsnorm_launch(x, a, B, C, eps, f16, st));
+    float* keep = (xmid && l == mid) ? xmid : nullptr;
+    if (x0 || keep)  // x_mid = the stream entering block `mid`; then x = a_l x + b_l x0
+      NC_TRY(rmsnorm_mix_launch(x, x0, x0 ? w->resid_lambdas + l : nullptr, x0 ? w->x0_lambdas + l : nullptr, keep,
+                                nullptr, nullptr, x0 != nullptr, a, B, C, eps, f16, st));
+    else
+      NC_TRY(rmsnorm_launch(x, a, B, C, eps, f16, st));
     uint16_t* cl = cache + l * SL.cache_layer_elems;
     if (cudaMemsetAsync(acc, 0, (size_t)B * NQKV * 4, st) != cudaSuccess) return NC_ERR_CUDA;
     NC_TRY(proj(a, C, wqkv + l * SL.wqkv_elems, NQKV, acc, ks_qkv));
-    NC_TRY(qkv_finish_launch(acc, qkv, cl, rope, T_max, pos, B, H, Hkv, D, T_max, eps, f16, st, pos_dev, status));
+    DecodeVe ve{};
+    if ((ex & NC_EXTRA_VALUE_EMBED) && nc_layer_value_embed(cfg, l) == 1)
+      ve = DecodeVe{tokens, w->value_embeds[l], w->ve_gates[l], V};
+    NC_TRY(qkv_finish_launch(acc, qkv, cl, rope, T_max, pos, B, H, Hkv, D, T_max, eps, f16, st, pos_dev, status,
+                             ve));
     NC_TRY(decode_attention_launch(qkv, NQKV, cl, part, o, B, H, Hkv, D, T_max, pos, nc_layer_window(cfg, l),
                                    f16, st, pos_dev));
     // the residual adds: partial products over K land in x (atomic or TMA
@@ -1028,7 +1057,11 @@ static nc_status decode_impl(const nc_config* cfg, const nc_weights* w, const in
     NC_TRY(relu2_finish_launch(acc, h, (int64_t)B * 4 * C, f16, st, status));
     NC_TRY(proj(h, 4 * C, wmp + l * SL.wmp_elems, C, x, resid_ksplit(B, C, 4 * C)));
   }
-  NC_TRY(rmsnorm_launch(x, a, B, C, eps, f16, st));
+  if (xmid)  // backout: x - lambda * x_mid, then the final norm
+    NC_TRY(rmsnorm_mix_launch(x, nullptr, nullptr, nullptr, nullptr, xmid, w->backout_lambda, false, a, B, C, eps, f16,
+                              st));
+  else
+    NC_TRY(rmsnorm_launch(x, a, B, C, eps, f16, st));
   if (skinny) {
     NC_TRY(skinny_gemm_launch(a, C, wlm, C, logits, V, B, V, C, 2, cfg->softcap, f16, st));
   } else {

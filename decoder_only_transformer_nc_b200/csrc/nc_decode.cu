@@ -260,7 +260,7 @@ __global__ void __launch_bounds__(256) qkv_finish_kernel(const float* __restrict
                                                          uint16_t* __restrict__ cache, const float* __restrict__ rope,
                                                          int rope_T, int pos, int B, int H, int Hkv, int T_max,
                                                          float eps, const int* __restrict__ pos_dev,
-                                                         uint32_t* __restrict__ dev_status) {
+                                                         uint32_t* __restrict__ dev_status, DecodeVe ve) {
   constexpr int D = DW * 32;
   bool store_cache = true;
   if (pos_dev) {  // a replayed graph step: refuse a position past the cache
@@ -295,6 +295,14 @@ __global__ void __launch_bounds__(256) qkv_finish_kernel(const float* __restrict
     const float r = rsqrtf(warp_allsum(ss) * (1.0f / D) + eps);
 #pragma unroll
     for (int d = 0; d < DW; ++d) v[d] *= r;
+  } else if (ve.table) {  // v head with a value embedding: v + gate[g] * table[token], kv head g
+    const int g = hd - H - Hkv;
+    int tok = ve.tokens[b];
+    if (tok < 0 || tok >= ve.V) tok = 0;  // flagged by the embedding kernel
+    const float* e = ve.table + ((int64_t)tok * Hkv + g) * D + lane * DW;
+    const float gt = ve.gate[g];
+#pragma unroll
+    for (int d = 0; d < DW; ++d) v[d] = fmaf(gt, e[d], v[d]);
   }
   uint32_t pk[DW / 2];
   float vmax = 0.0f;
@@ -487,20 +495,20 @@ int decode_attention_max_splits() { return kMaxSplits; }
 
 nc_status qkv_finish_launch(const float* acc, uint16_t* qkv, uint16_t* cache, const float* rope, int rope_T,
                             int pos, int B, int H, int Hkv, int D, int T_max, float eps, bool f16,
-                            cudaStream_t stream, const int* pos_dev, uint32_t* dev_status) {
+                            cudaStream_t stream, const int* pos_dev, uint32_t* dev_status, DecodeVe ve) {
   const int warps = B * (H + 2 * Hkv);
   if (warps == 0) return NC_OK;
   const unsigned grid = (unsigned)((warps + 7) / 8);
   if (D == 128)
     f16 ? qkv_finish_kernel<4, true><<<grid, 256, 0, stream>>>(acc, qkv, cache, rope, rope_T, pos, B, H, Hkv, T_max, eps,
-                                                               pos_dev, dev_status)
+                                                               pos_dev, dev_status, ve)
         : qkv_finish_kernel<4, false><<<grid, 256, 0, stream>>>(acc, qkv, cache, rope, rope_T, pos, B, H, Hkv, T_max,
-                                                                eps, pos_dev, dev_status);
+                                                                eps, pos_dev, dev_status, ve);
   else if (D == 64)
     f16 ? qkv_finish_kernel<2, true><<<grid, 256, 0, stream>>>(acc, qkv, cache, rope, rope_T, pos, B, H, Hkv, T_max, eps,
-                                                               pos_dev, dev_status)
+                                                               pos_dev, dev_status, ve)
         : qkv_finish_kernel<2, false><<<grid, 256, 0, stream>>>(acc, qkv, cache, rope, rope_T, pos, B, H, Hkv, T_max,
-                                                                eps, pos_dev, dev_status);
+                                                                eps, pos_dev, dev_status, ve);
   else
     return NC_ERR_SHAPE;
   return cudaGetLastError() == cudaSuccess ? NC_OK : NC_ERR_CUDA;
@@ -513,6 +521,82 @@ __global__ void pos_advance_kernel(int* pos) {
 
 nc_status pos_advance_launch(int* pos, cudaStream_t stream) {
   pos_advance_kernel<<<1, 32, 0, stream>>>(pos);
+  return cudaGetLastError() == cudaSuccess ? NC_OK : NC_ERR_CUDA;
+}
+
+// The embedding of a decode step's tokens with the further terms of the full
+// nanochat forward ("Nanochat与nanoGPT对比" §1): smear (gate != NULL) mixes in
+// the embedding of the token at the row's previous position, read from the
+// per-position token record hist [B][T_max], where this step also writes its
+// own token; x0 (!= NULL) keeps a copy of the result for the residual lambdas.
+// One warp per row; the gate's weight enters as bf16, as in the whole forward.
+__global__ void __launch_bounds__(256) decode_embedding_kernel(const int32_t* __restrict__ tokens,
+                                                               int32_t* __restrict__ hist,
+                                                               const float* __restrict__ wte,
+                                                               const float* __restrict__ gate, float* __restrict__ x,
+                                                               float* __restrict__ x0, int B, int C, int V, int T_max,
+                                                               int pos, const int* __restrict__ pos_dev,
+                                                               uint32_t* __restrict__ dev_status) {
+  const int b = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (b >= B) return;
+  bool in_cache = true;
+  if (pos_dev) {  // flagged (NC_DEV_POSITION) by the QKV finish of the same step
+    const int p = *pos_dev;
+    in_cache = p >= 0 && p < T_max;
+    pos = min(max(p, 0), T_max - 1);
+  }
+  int tok = tokens[b];
+  if (tok < 0 || tok >= V) {
+    if (lane == 0 && dev_status) atomicOr(dev_status, NC_DEV_TOKEN_RANGE);
+    tok = 0;
+  }
+  const float4* e = reinterpret_cast<const float4*>(wte + (int64_t)tok * C);
+  float4* dst = reinterpret_cast<float4*>(x + (int64_t)b * C);
+  float4* dst0 = x0 ? reinterpret_cast<float4*>(x0 + (int64_t)b * C) : nullptr;
+  const int n4 = C / 4;
+  const bool has_prev = gate && pos > 0;
+  float sg = 0.0f;
+  const float4* ep = e;
+  if (gate) {
+    if (lane == 0 && in_cache) hist[(int64_t)b * T_max + pos] = tok;
+    int ptok = has_prev ? hist[(int64_t)b * T_max + pos - 1] : 0;
+    if (ptok < 0 || ptok >= V) ptok = 0;
+    ep = reinterpret_cast<const float4*>(wte + (int64_t)ptok * C);
+    const float4* g4 = reinterpret_cast<const float4*>(gate);
+    float dot = 0.0f;
+    for (int i = lane; i < n4; i += 32) {
+      const float4 a = e[i], g = g4[i];
+      dot = fmaf(a.x, __bfloat162float(__float2bfloat16_rn(g.x)), dot);
+      dot = fmaf(a.y, __bfloat162float(__float2bfloat16_rn(g.y)), dot);
+      dot = fmaf(a.z, __bfloat162float(__float2bfloat16_rn(g.z)), dot);
+      dot = fmaf(a.w, __bfloat162float(__float2bfloat16_rn(g.w)), dot);
+    }
+    dot = warp_allsum(dot);
+    sg = has_prev ? 1.0f / (1.0f + expf(-dot)) : 0.0f;
+  }
+  for (int i = lane; i < n4; i += 32) {
+    float4 a = e[i];
+    if (has_prev) {
+      const float4 p = ep[i];
+      a.x = fmaf(sg, p.x, a.x);
+      a.y = fmaf(sg, p.y, a.y);
+      a.z = fmaf(sg, p.z, a.z);
+      a.w = fmaf(sg, p.w, a.w);
+    }
+    dst[i] = a;
+    if (dst0) dst0[i] = a;
+  }
+}
+
+nc_status decode_embedding_launch(const int32_t* tokens, int32_t* hist, const float* wte, const float* smear_gate,
+                                  float* x, float* x0, int B, int C, int V, int T_max, int pos, const int* pos_dev,
+                                  uint32_t* dev_status, cudaStream_t stream) {
+  if (B == 0) return NC_OK;
+  if (C % 4 || (smear_gate && !hist)) return NC_ERR_SHAPE;
+  const unsigned grid = (unsigned)((B + 7) / 8);
+  decode_embedding_kernel<<<grid, 256, 0, stream>>>(tokens, hist, wte, smear_gate, x, x0, B, C, V, T_max, pos,
+                                                    pos_dev, dev_status);
   return cudaGetLastError() == cudaSuccess ? NC_OK : NC_ERR_CUDA;
 }
 

@@ -226,9 +226,24 @@ int decode_attention_max_splits();
 // QK-norm of q and k heads (pair-interleaved columns), 16-bit qkv, and k|v heads
 // into the layer's cache at `pos`.  A device position outside [0, T_max) writes
 // no cache entry and sets NC_DEV_POSITION in dev_status.
+// With ve.table set, each v head g also gets ve.gate[g] * ve.table[token][g]
+// (the value embedding of the full nanochat forward; table [V][Hkv][D] fp32).
+struct DecodeVe {
+  const int32_t* tokens;
+  const float* table;
+  const float* gate;
+  int V;
+};
 nc_status qkv_finish_launch(const float* acc, uint16_t* qkv, uint16_t* cache, const float* rope, int rope_T,
                             int pos, int B, int H, int Hkv, int D, int T_max, float eps, bool f16,
-                            cudaStream_t stream, const int* pos_dev = nullptr, uint32_t* dev_status = nullptr);
+                            cudaStream_t stream, const int* pos_dev = nullptr, uint32_t* dev_status = nullptr,
+                            DecodeVe ve = DecodeVe{});
+// The token embedding of a decode step at `pos` (or *pos_dev) with smear
+// (smear_gate != NULL: reads the previous position's token from hist [B][T_max]
+// and records this step's token there) and an optional copy into x0 [B, C].
+nc_status decode_embedding_launch(const int32_t* tokens, int32_t* hist, const float* wte, const float* smear_gate,
+                                  float* x, float* x0, int B, int C, int V, int T_max, int pos, const int* pos_dev,
+                                  uint32_t* dev_status, cudaStream_t stream);
 // out = relu(acc)^2 as 16-bit (n elements, n % 4 == 0); an fp16 value past
 // 65504 sets NC_DEV_F16_RANGE in dev_status.
 nc_status relu2_finish_launch(const float* acc, uint16_t* out, int64_t n, bool f16, cudaStream_t stream,

@@ -226,11 +226,16 @@ nc_status nc_forward(const nc_config* cfg, const nc_weights* w, const int32_t* t
  *   the cache of every layer, [B][T_max][2][Hkv][D] 16-bit -- per row and
  *     position the k heads after RoPE and QK-norm (in the library's internal
  *     head-dimension order) then the v heads,
- *   the scratch of one decode step, and the device status word (first 4
- *     bytes, cleared by every call).
- * The KV-cache path covers the plain block stack in 16-bit: cfg->extras and
- * cfg->fp8 must be 0 (NC_ERR_CONFIG otherwise).  Decode attention needs n_head / n_kv_head in
- * {1, 2, 4, 8} (NC_ERR_SHAPE otherwise).  T_max <= cfg->seq_len. */
+ *   with NC_EXTRA_SMEAR, the token id of every position [B][T_max] int32 (a
+ *     step's smear mixes in the embedding of the previous position's token),
+ *   the scratch of one decode step (with NC_EXTRA_RESID_LAMBDAS / _BACKOUT
+ *     also the step's x0 and x_mid rows), and the device status word (first
+ *     4 bytes, cleared by every call).
+ * The KV-cache path computes in 16-bit: cfg->fp8 must be 0 (NC_ERR_CONFIG
+ * otherwise).  Every term of cfg->extras is supported; its parameters in `w`
+ * follow nc_forward's rules (NC_ERR_INVALID_ARG / NC_ERR_ALIGNMENT).  Decode
+ * attention needs n_head / n_kv_head in {1, 2, 4, 8} (NC_ERR_SHAPE otherwise).
+ * T_max <= cfg->seq_len. */
 
 /* Session bytes for B rows of up to T_max positions (0 on bad input).  Host only. */
 size_t nc_session_bytes(const nc_config* cfg, int B, int T_max);

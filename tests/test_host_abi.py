@@ -223,9 +223,17 @@ def test_kv_cache_host_rules(nclib):
     assert dec(cfg, 256) == 3           # pos >= T_max
     assert dec(cfg, -1) == 3
     assert dec(cfg, 5, nbytes=n - 1) == 5  # session too small
+    # the further terms: the session grows by the token record (smear) and the
+    # x0 / x_mid rows; their parameters are checked as nc_forward checks them
     cx = nclib.NcConfig.from_buffer_copy(cfg)
     cx.extras = nclib.EXTRA_SMEAR
-    assert dec(cx, 5) == 2               # the KV-cache path is the plain stack
+    nx = L.nc_session_bytes(ctypes.byref(cx), 2, 256)
+    assert nx >= n + 2 * 256 * 4
+    assert dec(cx, 5) == 5               # the plain stack's session is too small
+    assert dec(cx, 5, nbytes=nx) == 1    # no smear gate
+    call = nclib.NcConfig.from_buffer_copy(cfg)
+    call.extras = nclib.EXTRA_ALL
+    assert L.nc_session_bytes(ctypes.byref(call), 2, 256) >= nx + 2 * 2 * cfg.d_model * 4
     pre = lambda T, T_max=256: L.nc_prefill(ctypes.byref(cfg), ctypes.byref(fw.w), tok, 2, T, None, sess, n, T_max,
                                              1 << 42, 1 << 30, None)
     assert pre(300) == 3                 # T > T_max
@@ -233,6 +241,10 @@ def test_kv_cache_host_rules(nclib):
     if not torch.cuda.is_available():
         assert dec(cfg, 5) == 8          # valid arguments, no sm_100 device
         assert pre(100) == 8
+        fw.w.smear_gate = (1 << 44) + 256
+        assert dec(cx, 5, nbytes=nx) == 8
+        fw.w.smear_gate = (1 << 44) + 8  # misaligned
+        assert dec(cx, 5, nbytes=nx) == 4
 
 
 def test_fp8_host_rules(nclib):
