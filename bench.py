@@ -118,6 +118,27 @@ def kernels_per_step(n_entries, L, fp8_bits, extras_bits):
     return n
 
 
+def train_extra_kernels(L, n_ve, extras_bits):
+    """Kernels the further terms add to one training micro-step (the trace
+    does not record them): the backout product dlambda = -sum dx . x_mid, one
+    value-embedding backward per layer that has a table, per layer the
+    lambda products and the mix that carries dx to the block's input (and to
+    x0, added back once at the end), and the smear backward (token and gate
+    passes).  The forward's terms ride in kernels it launches anyway."""
+    n = 0
+    if extras_bits & 8:
+        n += 1
+    if extras_bits & 2:
+        n += n_ve
+    if extras_bits & 4:
+        n += 2 * L + 1
+    elif extras_bits & 8:
+        n += 1  # the mix at the middle block
+    if extras_bits & 1:
+        n += 2
+    return n
+
+
 class ClockSampler:
     """nvidia-smi clocks/throttle reasons sampled every 200 ms while running."""
 
@@ -588,10 +609,12 @@ def run_train(args, s):
         import torch.distributed as dist
         from datetime import timedelta
         dist.init_process_group("nccl", device_id=dev, timeout=timedelta(seconds=120))
+    bits = nc.EXTRA_ALL if args.extras == "all" else 0
     cfg = nc.make_config(s.n_layer, s.d_model, s.n_head, s.n_kv_head, s.head_dim, s.seq_len, s.vocab,
-                         s.short_window)
+                         s.short_window, extras=bits)
     weights = make_weights(s)
-    model = nc.Model.from_numpy(cfg, weights, device=dev)
+    model = nc.Model.from_numpy(cfg, weights, device=dev, extras=_extras_for(s, nc) if bits else None)
+    n_ve = sum(nc.layer_value_embed(cfg, l) == 1 for l in range(s.n_layer)) if bits & nc.EXTRA_VALUE_EMBED else 0
     B, T = s.batch, s.seq_len
     x, y = make_tokens(s, seed=dp.shard_seed(TOKEN_SEED, rank))
     tx, ty = torch.from_numpy(x).to(dev), torch.from_numpy(y).to(dev)
@@ -688,7 +711,8 @@ def run_train(args, s):
             "value": world * M / (ms / 1e3), "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": DTYPE_NOTE, "data": "synthetic",
-            "config": {"workload": f"{s.name} train", "global_batch": world * B, "seq_len": T,
+            "config": {"workload": f"{s.name}{'+extras' if bits else ''} train", "global_batch": world * B,
+                       "seq_len": T,
                        "parallelism": (f"dp{world}, one NCCL all-reduce of the fp32 gradient bucket per step"
                                        if world > 1 else "none"),
                        "l2": "inputs larger than L2 (saved activations ~40 GB per step)"},
@@ -698,7 +722,8 @@ def run_train(args, s):
                          "frac": round(top_ach / peak, 4), "traffic": None,
                          "launches": per_kind[top][1], "avg_launch_ms": round(per_kind[top][0] / per_kind[top][1], 4)},
             "kernels": kernels,
-            "gpu_launches": n_entries * args.steps,  # 2 L copies launch no kernel; attention bwd is 3 per layer
+            # 2 L copies launch no kernel; attention bwd is 3 per layer; the further terms' kernels are untraced
+            "gpu_launches": (n_entries + train_extra_kernels(s.n_layer, n_ve, bits)) * args.steps,
             "e2e": {"value": world * M / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": int(x.nbytes + y.nbytes),
                     "d2h_bytes_per_step": 4},
             "clocks": clocks.summary(),
@@ -751,6 +776,8 @@ def main():
         if args.batch < 1:
             raise SystemExit("--batch must be >= 1")
         s = dataclasses.replace(s, batch=args.batch)
+    if args.mode == "train" and args.fp8 != "none":
+        raise SystemExit("--mode train: the training step runs on 16-bit operands (no --fp8)")
     if args.impl == "reference":
         run_reference(args, s)
     elif args.mode == "decode":

@@ -47,12 +47,19 @@ NAMES = ("c_q", "c_k", "c_v", "attn_proj", "c_fc", "mlp_proj")
 
 def grad_bucket(tensors: dict, device=None):
     """One flat fp32 buffer holding a gradient for every weight of ``tensors``
-    (the layout of ``Model.tensors``), each view starting on a 16-byte boundary,
-    plus a last slot for the local target count.  Returns (flat, grads) with
-    ``grads`` in the layout ``forward_backward`` takes; the buffer is zeroed."""
+    (the layout of ``Model.tensors``, the further terms' "extras" included),
+    each view starting on a 16-byte boundary, plus a last slot for the local
+    target count.  Returns (flat, grads) with ``grads`` in the layout
+    ``forward_backward`` takes; the buffer is zeroed."""
     shapes = [("wte", tensors["wte"].shape), ("lm_head", tensors["lm_head"].shape)]
     for l, lw in enumerate(tensors["layers"]):
         shapes += [((l, n), lw[n].shape) for n in NAMES]
+    ex = tensors.get("extras") or {}
+    for k, v in ex.items():  # per-layer lists keep their None entries
+        if isinstance(v, list):
+            shapes += [(("extras", k, l), x.shape) for l, x in enumerate(v) if x is not None]
+        elif v is not None:
+            shapes.append((("extras", k), v.shape))
     offs, off = [], 0
     for _, shp in shapes:
         offs.append(off)
@@ -63,12 +70,19 @@ def grad_bucket(tensors: dict, device=None):
     dev = device if device is not None else tensors["wte"].device
     flat = torch.zeros(off + 4, dtype=torch.float32, device=dev)
     grads = {"layers": [dict() for _ in tensors["layers"]]}
+    if ex:
+        grads["extras"] = {k: ([None] * len(v) if isinstance(v, list) else None) for k, v in ex.items()}
     for (key, shp), o in zip(shapes, offs):
         n = 1
         for d in shp:
             n *= d
         view = flat[o:o + n].view(shp)
-        if isinstance(key, tuple):
+        if isinstance(key, tuple) and key[0] == "extras":
+            if len(key) == 3:
+                grads["extras"][key[1]][key[2]] = view
+            else:
+                grads["extras"][key[1]] = view
+        elif isinstance(key, tuple):
             grads["layers"][key[0]][key[1]] = view
         else:
             grads[key] = view

@@ -24,3 +24,18 @@ def test_unfused_activation_quantisations_add_an_amax_launch():
     assert bench.kernels_per_step(base, L, 3, 8) == fused + 2      # backout: one first norm + the final norm
     assert bench.kernels_per_step(base, L, 1, 8) == bench.kernels_per_step(base, L, 1, 0) + 1
 
+
+
+def test_training_extras_kernel_counts():
+    """The further terms' backward kernels of one training micro-step, item by
+    item for four layers with tables on layers 1 and 3 (the trace records none
+    of them)."""
+    L, n_ve = 4, 2
+    backout_dot = 1
+    ve_bwd = n_ve
+    lambda_dots, mixes, final_mix = L, L, 1  # the middle block's mix also carries the backout term
+    smear = 2  # per-token pass, then the gate's weight gradient
+    assert bench.train_extra_kernels(L, n_ve, 15) == backout_dot + ve_bwd + lambda_dots + mixes + final_mix + smear
+    assert bench.train_extra_kernels(L, n_ve, 0) == 0
+    assert bench.train_extra_kernels(L, n_ve, 8) == 2  # backout alone: its dot and one mix
+    assert bench.train_extra_kernels(L, n_ve, 2) == n_ve

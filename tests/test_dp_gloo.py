@@ -135,8 +135,38 @@ def test_grad_bucket_layout():
     t = {"wte": torch.from_numpy(w["wte"]), "lm_head": torch.from_numpy(w["lm_head"]),
          "layers": [{k: torch.from_numpy(v) for k, v in lw.items()} for lw in w["layers"]]}
     flat, grads = dp.grad_bucket(t, device="cpu")
+    assert "extras" not in grads
     views = [("wte", grads["wte"], t["wte"]), ("lm_head", grads["lm_head"], t["lm_head"])]
     views += [(f"{l}.{k}", grads["layers"][l][k], t["layers"][l][k]) for l in range(s.n_layer) for k in dp.NAMES]
+    _check_views(flat, views)
+
+
+def test_grad_bucket_layout_with_extras():
+    """The further terms' gradients join the bucket; a per-layer list keeps its
+    None entries (layers without a value embedding)."""
+    from decoder_only_transformer_nc_b200 import dp
+    from workloads import SHAPES, make_extras, make_weights
+
+    s = SHAPES["tiny"]
+    w = make_weights(s)
+    ex = make_extras(s, layers=[1])
+    T = lambda a: torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32))
+    t = {"wte": T(w["wte"]), "lm_head": T(w["lm_head"]),
+         "layers": [{k: T(v) for k, v in lw.items()} for lw in w["layers"]],
+         "extras": {"smear_gate": T(ex["smear_gate"]), "resid_lambdas": T(ex["resid_lambdas"]),
+                    "x0_lambdas": T(ex["x0_lambdas"]), "backout_lambda": T(np.reshape(ex["backout_lambda"], 1)),
+                    "value_embeds": [None, T(ex["value_embeds"][1])], "ve_gates": [None, T(ex["ve_gates"][1])]}}
+    flat, grads = dp.grad_bucket(t, device="cpu")
+    ge, te = grads["extras"], t["extras"]
+    assert ge["value_embeds"][0] is None and ge["ve_gates"][0] is None
+    views = [("wte", grads["wte"], t["wte"]), ("lm_head", grads["lm_head"], t["lm_head"])]
+    views += [(f"{l}.{k}", grads["layers"][l][k], t["layers"][l][k]) for l in range(s.n_layer) for k in dp.NAMES]
+    views += [(k, ge[k], te[k]) for k in ("smear_gate", "resid_lambdas", "x0_lambdas", "backout_lambda")]
+    views += [(f"{k}[1]", ge[k][1], te[k][1]) for k in ("value_embeds", "ve_gates")]
+    _check_views(flat, views)
+
+
+def _check_views(flat, views):
     spans = []
     for name, g, ref in views:
         assert g.shape == ref.shape and g.dtype == torch.float32, name
