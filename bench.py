@@ -428,8 +428,10 @@ def run_ours(args, s):
                        "l2": "inputs larger than L2 (fp32 weights %.2f GB, residual stream %.2f GB per step)"
                              % (4 * sum(a.size for a in _flat(weights)) / 1e9, 4 * B * T * s.d_model / 1e9)},
             "tflops": round(tflops, 1),
-            "pct_of_bf16_peak": {"measured_burst": round(100 * tflops / world / burst, 2),
-                                 "measured_sustained": round(100 * tflops / world / peak16, 2),
+            # burst / sustained: MEASURED_PEAKS.json's figures, else the fallback ones ("source")
+            "pct_of_bf16_peak": {"burst": round(100 * tflops / world / burst, 2),
+                                 "sustained": round(100 * tflops / world / peak16, 2),
+                                 "burst_tflops": burst, "sustained_tflops": peak16,
                                  "datasheet_dense_2250": round(100 * tflops / world / 2250.0, 2),
                                  "source": peak_src},
             "roofline": {"kernel": "gemm_kernel<EPI_RELU2_16> (c_fc + ReLU^2: M=B*T, N=4C, K=C)",
