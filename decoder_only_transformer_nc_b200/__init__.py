@@ -124,6 +124,7 @@ def lib():
             "nc_event_create": (i32, [ctypes.POINTER(ctypes.c_void_p)]),
             "nc_event_destroy": (i32, [vp]),
             "nc_event_elapsed_ms": (i32, [vp, vp, ctypes.POINTER(ctypes.c_float)]),
+            "nc_stream_wait_event": (i32, [vp, vp]),
             "nc_get_status": (i32, [vp, vp]),
             "nc_cast_weights": (i32, [vp, vp, i64, i32, vp]),
             "nc_embedding": (i32, [vp, vp, vp, i32, i32, i32, vp, vp]),
@@ -427,6 +428,16 @@ class LaunchTrace:
                    "nc_event_elapsed_ms")
             out.append((KERNEL_KINDS[self._kinds[i]], ms.value))
         return out
+
+    def kinds(self):
+        """Kind names of the last traced call's launches (known once it is enqueued)."""
+        return [KERNEL_KINDS[self._kinds[i]] for i in range(self.struct.count)]
+
+    def end_event(self, i: int):
+        """The event recorded right after launch i (a cudaEvent_t handle)."""
+        if not 0 <= i < self.struct.count:
+            raise IndexError(f"launch {i} of {self.struct.count}")
+        return self._ev[2 * i + 1]
 
     def close(self):
         if self._ev is not None:

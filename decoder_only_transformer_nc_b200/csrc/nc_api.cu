@@ -1461,6 +1461,11 @@ nc_status nc_event_destroy(void* event) {
   return cudaEventDestroy(static_cast<cudaEvent_t>(event)) == cudaSuccess ? NC_OK : NC_ERR_CUDA;
 }
 
+nc_status nc_stream_wait_event(void* stream, void* event) {
+  if (!event) return NC_ERR_INVALID_ARG;
+  return cudaStreamWaitEvent(S(stream), static_cast<cudaEvent_t>(event), 0) == cudaSuccess ? NC_OK : NC_ERR_CUDA;
+}
+
 nc_status nc_event_elapsed_ms(void* start, void* end, float* ms) {
   if (!start || !end || !ms) return NC_ERR_INVALID_ARG;
   if (cudaEventSynchronize(static_cast<cudaEvent_t>(end)) != cudaSuccess) return NC_ERR_CUDA;

@@ -331,6 +331,11 @@ nc_status nc_event_create(void** event);
 nc_status nc_event_destroy(void* event);
 /* Milliseconds between two recorded events (waits for `end`). */
 nc_status nc_event_elapsed_ms(void* start, void* end, float* ms);
+/* Work enqueued on `stream` after this call waits for `event` (one of a
+ * trace's events: e.g. a side stream that starts a collective on a layer's
+ * gradients once the launch that last writes them has finished).  Host only;
+ * NULL stream: the legacy default stream. */
+nc_status nc_stream_wait_event(void* stream, void* event);
 
 /* Synchronises `stream` and returns the status recorded in the device status
  * word at `dev_status` (e.g. the workspace of nc_forward): NC_OK,
