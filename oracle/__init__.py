@@ -64,7 +64,12 @@ Backward ("从文本到聊天模型" §6.5: the training step's loss.backward())
 ``oracle.grad.forward_backward`` gives the mean loss of the plain stack and its
 gradient with respect to every fp32 master weight, the bf16 cast taken as
 straight-through; pinned in ``tests/test_oracle_grad.py`` by finite
-differences and torch float64 autograd.
+differences and torch float64 autograd.  With ``extras`` it also
+differentiates the further terms (smear, residual lambdas with x0, value
+embeddings, backout) and returns their parameters' gradients; pinned in
+``tests/test_oracle_grad_extras.py`` by finite differences, by its loss
+against the separately pinned ``forward(..., extras=...)``, and by neutral
+terms leaving the plain gradients unchanged.
 
 FP8 ("Nanochat与nanoGPT对比" §1 table, FP8-training row: dynamic tensor-level
 e4m3/e5m2): ``forward(..., fp8="block" | "all")`` runs the block projections
