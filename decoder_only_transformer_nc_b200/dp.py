@@ -137,6 +137,8 @@ def average_grads_sliced_(flat: torch.Tensor, slices, local_count: float, group=
     count.  ``before(k)``, when given, runs ahead of slice k (the overlapped
     schedule makes the side stream wait there).  Every rank must pass the same
     slices in the same order."""
+    if not slices or slices[-1][2] != flat.numel():
+        raise ValueError("the last slice must end with the bucket's count slot")
     for k, (_, a, b) in enumerate(slices):
         if before is not None:
             before(k)

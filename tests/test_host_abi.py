@@ -158,6 +158,7 @@ def test_single_step_argument_checks(nclib):
     assert L.nc_cast_weights(A, B_, 16, 5, None) == 1
     assert L.nc_softcap_ce(A, A, None, B_, 4, 512, -1.0, None, None) == 1
     assert L.nc_selftest_bounded_wait(None, 100, None) == 1
+    assert L.nc_stream_wait_event(None, None) == 1  # no event
     assert L.nc_status_string(7) == b"bounded device wait ran out"
     c = nclib.init_config(2, 64, 64, 0, 256, 512)
     assert c.act_dtype == nclib.F16
