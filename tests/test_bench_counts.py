@@ -39,3 +39,14 @@ def test_training_extras_kernel_counts():
     assert bench.train_extra_kernels(L, n_ve, 0) == 0
     assert bench.train_extra_kernels(L, n_ve, 8) == 2  # backout alone: its dot and one mix
     assert bench.train_extra_kernels(L, n_ve, 2) == n_ve
+
+
+def test_training_claim_matches_the_recorded_launch_list():
+    """One d20 training step with every term: 492 trace entries (the 40
+    residual copies launch no kernel, the 20 attention backwards three kernels
+    each) plus the terms' untraced backward kernels are the 546 library kernels
+    ncu recorded for one step (profiles/launches_d20_train_extras_b8.md)."""
+    L, n_ve = 20, 10
+    entries = 12 + 24 * L
+    assert entries - 2 * L + 2 * L == 492
+    assert entries + bench.train_extra_kernels(L, n_ve, 15) == 546
